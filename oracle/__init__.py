@@ -1,0 +1,249 @@
+"""ctypes binding of the fp64 CPU oracle (csa_oracle.cpp).
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, the smoke check and the
+benchmark's CPU-baseline leg, never by the CUDA library. It takes and returns numpy
+arrays; the shared object is built on first use (or by the package build step).
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "csa_oracle.cpp")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with g++ (plain -O2, no fast-math: IEEE fp64 throughout)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".{os.getpid()}.tmp"
+        subprocess.check_call(["g++", "-O2", "-std=c++17", "-shared", "-fPIC", "-pthread",
+                               "-o", tmp, _SRC])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _p(a, ctype):
+    return None if a is None else a.ctypes.data_as(C.POINTER(ctype))
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = C.CDLL(build())
+            d, i, i64 = C.c_double, C.c_int, C.c_int64
+            P = C.POINTER
+            u8, u16, f32, f64, i32 = (P(C.c_uint8), P(C.c_uint16), P(C.c_float),
+                                      P(C.c_double), P(C.c_int32))
+            L.or_bf16_decode.restype = d
+            L.or_bf16_decode.argtypes = [C.c_uint16]
+            L.or_bf16_encode.restype = C.c_uint16
+            L.or_bf16_encode.argtypes = [d]
+            L.or_e4m3_decode.restype = d
+            L.or_e4m3_decode.argtypes = [C.c_uint8]
+            L.or_e4m3_encode.restype = C.c_uint8
+            L.or_e4m3_encode.argtypes = [d]
+            L.or_e2m1_decode.restype = d
+            L.or_e2m1_decode.argtypes = [C.c_uint8]
+            L.or_e8m0_decode.restype = d
+            L.or_e8m0_decode.argtypes = [C.c_uint8]
+            L.or_key_sf_offset.restype = C.c_size_t
+            L.or_key_sf_offset.argtypes = [i64, i]
+            L.or_compress.restype = i
+            L.or_compress.argtypes = [i, i, i, i, i64, d, d, u16, u16, f32, f32, f32, f32,
+                                      u16, f32, f64, f64, u8, f32]
+            L.or_dequant_row.restype = None
+            L.or_dequant_row.argtypes = [u8, C.c_float, f64]
+            L.or_indexer_scores.restype = i
+            L.or_indexer_scores.argtypes = [i, i, i64, i32, u8, u8, f32, u8, u8, f64, i]
+            L.or_topk.restype = i
+            L.or_topk.argtypes = [i64, i, f64, i32]
+            L.or_attention.restype = i
+            L.or_attention.argtypes = [i, i, i, i64, i, u16, i32, i32, i32, u8, f32, u16,
+                                       f32, d, d, i, f64, f64, i]
+            L.or_swa_row.restype = None
+            L.or_swa_row.argtypes = [u16, i64, d, d, f32, u16]
+            L.or_prefill.restype = i
+            L.or_prefill.argtypes = [i64, i, i, i, i, i, d, d, d, i, u16, u16, f32, f32, f32,
+                                     f32, u16, f32, u8, f32, i64, u8, u8, f32, u8, u8, u16,
+                                     f32, u16, i, i32, f64, f64, i32, i]
+            _lib = L
+    return _lib
+
+
+def _c(a, dtype):
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a)
+    assert a.dtype == dtype, (a.dtype, dtype)
+    return a
+
+
+# ------------------------------------------------------------------ formats
+def bf16_decode(h):
+    h = np.asarray(h, dtype=np.uint16)
+    return np.vectorize(lambda x: lib().or_bf16_decode(int(x)), otypes=[np.float64])(h)
+
+
+def bf16_encode(x):
+    return np.vectorize(lambda v: lib().or_bf16_encode(float(v)), otypes=[np.uint16])(x)
+
+
+def e4m3_decode(c):
+    return np.vectorize(lambda x: lib().or_e4m3_decode(int(x)), otypes=[np.float64])(c)
+
+
+def e4m3_encode(x):
+    return np.vectorize(lambda v: lib().or_e4m3_encode(float(v)), otypes=[np.uint8])(x)
+
+
+def e2m1_decode(c):
+    return np.vectorize(lambda x: lib().or_e2m1_decode(int(x)), otypes=[np.float64])(c)
+
+
+def e8m0_decode(c):
+    return np.vectorize(lambda x: lib().or_e8m0_decode(int(x)), otypes=[np.float64])(c)
+
+
+def key_sf_offset(j: int, s: int) -> int:
+    return int(lib().or_key_sf_offset(int(j), int(s)))
+
+
+def dequant_rows(kv_rows: np.ndarray, scale: np.ndarray) -> np.ndarray:
+    """[n][576] stored rows + [n] scales -> [n][512] float64."""
+    kv_rows = _c(kv_rows, np.uint8).reshape(-1, 576)
+    scale = _c(scale, np.float32).reshape(-1)
+    out = np.empty((kv_rows.shape[0], 512), dtype=np.float64)
+    for r in range(kv_rows.shape[0]):
+        lib().or_dequant_row(_p(kv_rows[r], C.c_uint8), float(scale[r]),
+                             _p(out[r], C.c_double))
+    return out
+
+
+# ------------------------------------------------------------------ layer
+def compress(a, za, bias, m: int, overlap: bool, b=None, zb=None, pos0: int = 0,
+             prev_b=None, prev_zb=None, rope_base: float = 10000.0, eps: float = 1e-6,
+             norm_w=None) -> dict:
+    """a, b bf16 bits [B][T][512]; za, zb float32 [B][T][512] -> dict with e, y
+    (float64 [B][N][512]), kv (uint8 [B][N][576]) and kv_scale (float32 [B][N])."""
+    a = _c(a, np.uint16)
+    B, T, _ = a.shape
+    N = T // m
+    e = np.empty((B, N, 512)); y = np.empty((B, N, 512))
+    kv = np.empty((B, N, 576), dtype=np.uint8); sc = np.empty((B, N), dtype=np.float32)
+    args = [_c(b, np.uint16), _c(za, np.float32), _c(zb, np.float32), _c(bias, np.float32),
+            _c(norm_w, np.float32), _c(prev_b, np.uint16), _c(prev_zb, np.float32)]
+    rc = lib().or_compress(B, T, m, int(overlap), pos0, rope_base, eps, _p(a, C.c_uint16),
+                           _p(args[0], C.c_uint16), _p(args[1], C.c_float),
+                           _p(args[2], C.c_float), _p(args[3], C.c_float),
+                           _p(args[4], C.c_float), _p(args[5], C.c_uint16),
+                           _p(args[6], C.c_float), _p(e, C.c_double), _p(y, C.c_double),
+                           _p(kv, C.c_uint8), _p(sc, C.c_float))
+    if rc:
+        raise ValueError("oracle compress rejected its arguments")
+    return {"e": e, "y": y, "kv": kv, "kv_scale": sc}
+
+
+def indexer_scores(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, nthreads: int = 0) -> np.ndarray:
+    """-> float64 [B][Nmax] (NaN past n_entries[b])."""
+    q_fp4 = _c(q_fp4, np.uint8)
+    B, H_I, _ = q_fp4.shape
+    k_fp4 = _c(k_fp4, np.uint8)
+    Nmax = k_fp4.shape[1]
+    n = _c(np.asarray(n_entries, dtype=np.int32), np.int32)
+    out = np.empty((B, Nmax))
+    qs, ww, ks = _c(q_sf, np.uint8), _c(w, np.float32), _c(k_sf, np.uint8)
+    rc = lib().or_indexer_scores(B, H_I, Nmax, _p(n, C.c_int32), _p(q_fp4, C.c_uint8),
+                                 _p(qs, C.c_uint8), _p(ww, C.c_float),
+                                 _p(k_fp4, C.c_uint8), _p(ks, C.c_uint8),
+                                 _p(out, C.c_double), nthreads)
+    if rc:
+        raise ValueError("oracle indexer rejected its arguments")
+    return out
+
+
+def topk(scores: np.ndarray, n: int, k: int) -> np.ndarray:
+    s = _c(np.asarray(scores[:n], dtype=np.float64), np.float64)
+    idx = np.empty(k, dtype=np.int32)
+    if lib().or_topk(n, k, _p(s, C.c_double), _p(idx, C.c_int32)):
+        raise ValueError("oracle topk rejected its arguments")
+    return idx
+
+
+def attention(q, pos, n_entries, kv, kv_scale, swa, sink, idx=None, k: int = 0,
+              tau: float | None = None, rope_base: float = 10000.0, derotate: bool = True,
+              nthreads: int = 0) -> tuple[np.ndarray, np.ndarray]:
+    """q bf16 bits [B][H][512]; kv [B][Nmax][576]; kv_scale [B][Nmax]; swa [B][128][512];
+    idx [B][k] (CSA) or None (HCA: all n_entries) -> (out float64 [B][H][512], lse [B][H])."""
+    q = _c(q, np.uint16)
+    B, H, _ = q.shape
+    kv = _c(kv, np.uint8)
+    Nmax = kv.shape[1]
+    sparse = idx is not None
+    if sparse:
+        idx = _c(np.asarray(idx, dtype=np.int32), np.int32)
+        k = idx.shape[1]
+    tau = 1.0 / np.sqrt(512.0) if tau is None else tau
+    pos = _c(np.asarray(pos, dtype=np.int32), np.int32)
+    n = _c(np.asarray(n_entries, dtype=np.int32), np.int32)
+    sc, sw, sk = _c(kv_scale, np.float32), _c(swa, np.uint16), _c(sink, np.float32)
+    out = np.empty((B, H, 512)); lse = np.empty((B, H))
+    rc = lib().or_attention(B, H, k, Nmax, int(sparse), _p(q, C.c_uint16), _p(pos, C.c_int32),
+                            _p(idx, C.c_int32), _p(n, C.c_int32), _p(kv, C.c_uint8),
+                            _p(sc, C.c_float), _p(sw, C.c_uint16), _p(sk, C.c_float), tau,
+                            rope_base, int(derotate), _p(out, C.c_double),
+                            _p(lse, C.c_double), nthreads)
+    if rc:
+        raise ValueError("oracle attention rejected its arguments")
+    return out, lse
+
+
+def swa_row(a_row, t: int, rope_base: float = 10000.0, eps: float = 1e-6,
+            norm_w=None) -> np.ndarray:
+    a_row = _c(a_row, np.uint16)
+    out = np.empty(512, dtype=np.uint16)
+    nw = _c(norm_w, np.float32)
+    lib().or_swa_row(_p(a_row, C.c_uint16), t, rope_base, eps, _p(nw, C.c_float),
+                     _p(out, C.c_uint16))
+    return out
+
+
+def prefill(inp: dict, k: int, q_rows, tau: float | None = None, rope_base: float = 10000.0,
+            eps: float = 1e-6, derotate: bool = True, nthreads: int = 0) -> dict:
+    """Evaluate the rows `q_rows` of a prefill described by a synth.prefill_inputs dict.
+    Returns out [nq][H][512], lse [nq][H], idx [nq][k] and the cache after compression."""
+    P, T, m, H, H_I, Nmax = (inp[x] for x in ("P", "T", "m", "H", "H_I", "Nmax"))
+    tau = 1.0 / np.sqrt(512.0) if tau is None else tau
+    kv = np.array(inp["kv"], dtype=np.uint8, copy=True)
+    sc = np.array(inp["kv_scale"], dtype=np.float32, copy=True)
+    rows = _c(np.asarray(q_rows, dtype=np.int32), np.int32)
+    nq = rows.shape[0]
+    out = np.empty((nq, H, 512)); lse = np.empty((nq, H)); idx = np.empty((nq, k), np.int32)
+    g = {x: _c(inp.get(x), t) for x, t in (
+        ("a", np.uint16), ("b", np.uint16), ("za", np.float32), ("zb", np.float32),
+        ("bias", np.float32), ("prev_b", np.uint16), ("prev_zb", np.float32),
+        ("q_fp4", np.uint8), ("q_sf", np.uint8), ("w", np.float32), ("k_fp4", np.uint8),
+        ("k_sf", np.uint8), ("q", np.uint16), ("sink", np.float32),
+        ("swa_prefix", np.uint16))}
+    U16, F32, U8 = C.c_uint16, C.c_float, C.c_uint8
+    rc = lib().or_prefill(P, T, m, H, H_I, k, rope_base, eps, tau, int(derotate),
+                          _p(g["a"], U16), _p(g["b"], U16), _p(g["za"], F32),
+                          _p(g["zb"], F32), _p(g["bias"], F32), None,
+                          _p(g["prev_b"], U16), _p(g["prev_zb"], F32), _p(kv, U8),
+                          _p(sc, F32), Nmax, _p(g["q_fp4"], U8), _p(g["q_sf"], U8),
+                          _p(g["w"], F32), _p(g["k_fp4"], U8), _p(g["k_sf"], U8),
+                          _p(g["q"], U16), _p(g["sink"], F32), _p(g["swa_prefix"], U16),
+                          nq, _p(rows, C.c_int32), _p(out, C.c_double), _p(lse, C.c_double),
+                          _p(idx, C.c_int32), nthreads)
+    if rc:
+        raise ValueError("oracle prefill rejected its arguments")
+    return {"out": out, "lse": lse, "idx": idx, "kv": kv, "kv_scale": sc}

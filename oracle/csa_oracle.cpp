@@ -1,0 +1,509 @@
+// CPU oracle for the CSA/HCA compressed attention layer.
+//
+// TEST INFRASTRUCTURE ONLY. This file is the slow, plain, fp64 statement of what the
+// layer computes. Only the test suite, the smoke check and the benchmark's CPU-baseline
+// leg may load it. It shares no code, header, table or constant generator with the
+// CUDA library; the two meet only at the seeded synthetic inputs.
+//
+// Sources (five web pages summarising the DeepSeek-V4 technical report):
+//   [walkthrough]  cyqw.cn/news/842812, the long DeepSeek-V4 walkthrough,
+//                  §2.2 "混合注意力CSA+HCA", §2.3, §3.3, §3.4, §3.5
+//   [digest]       "DeepSeek V4技术报告详解：484天演进路、百万Token架构与国产芯片适配"
+//                  (firecat-web), section "2. 混合注意力机制"
+//   [chooseai]     chooseai.net/news/3476, section "一、CSA + HCA 混合注意力"
+//   [tutorial]     "DeepSeek-V4：百万上下文的工程答案" (mewclaw tutorial),
+//                  sections "Hybrid Attention", "Partial RoPE", "Attention sink", "低精度路径"
+//
+// The pages give prose only: no formula, constant or worked example for the layer.
+// Every precise choice below that the prose leaves open is a numbered reading (R#);
+// the list of readings and their reasons lives with the design notes.
+//
+// Parity status: every function here is pinned by the CPU test suite against format
+// definitions, closed forms, invariants, textbook reductions or brute force; none is
+// "parity unpinned" against its own definition. The readings R1-R17 themselves are
+// not fixed by the pages and are pinned only to this statement.
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <limits>
+#include <thread>
+#include <vector>
+
+namespace {
+
+constexpr int kD = 512;        // head_dim of the shared KV entry [digest, 2.]
+constexpr int kNope = 448;     // dims stored as FP8 E4M3 [chooseai, 一]
+constexpr int kRope = 64;      // last 64 dims carry RoPE [digest, 2.]
+constexpr int kDI = 128;       // indexer head dim (config tables of the workload)
+constexpr int kWin = 128;      // sliding-window tokens [walkthrough §2.2]
+constexpr int kRow = 576;      // 448 E4M3 bytes + 64 bf16 = stored bytes per entry
+
+const double kInf = std::numeric_limits<double>::infinity();
+const double kNaN = std::numeric_limits<double>::quiet_NaN();
+
+// ---------------------------------------------------------------- formats
+// Round x to the nearest value of a binary floating-point format with `p`
+// significand bits (implicit bit included) and minimum normal exponent `emin`;
+// ties go to the even significand. Overflow is the caller's business.
+double round_binary(double x, int p, int emin) {
+  if (x == 0.0 || !std::isfinite(x)) return x;
+  int e;
+  std::frexp(std::fabs(x), &e);  // |x| = f * 2^e, f in [0.5, 1)
+  int lead = e - 1;              // exponent of the leading bit
+  if (lead < emin) lead = emin;  // subnormal range: fixed quantum
+  const double quantum = std::ldexp(1.0, lead - p + 1);
+  const double r = x / quantum;  // exact: scaling by a power of two
+  return std::nearbyint(r) * quantum;  // default mode: nearest, ties to even
+}
+
+}  // namespace
+
+extern "C" {
+
+// bfloat16: the upper half of an IEEE-754 binary32 (8 significand bits, emin -126).
+double or_bf16_decode(uint16_t h) {
+  const int s = h >> 15, e = (h >> 7) & 0xFF, m = h & 0x7F;
+  double v;
+  if (e == 0xFF) v = m ? kNaN : kInf;
+  else if (e == 0) v = std::ldexp((double)m, -126 - 7);
+  else v = std::ldexp(1.0 + m / 128.0, e - 127);
+  return s ? -v : v;
+}
+
+uint16_t or_bf16_encode(double x) {
+  if (std::isnan(x)) return 0x7FC0;
+  const uint16_t s = std::signbit(x) ? 0x8000 : 0;
+  double v = std::fabs(round_binary(x, 8, -126));
+  if (v >= std::ldexp(2.0, 127)) return s | 0x7F80;  // rounds past the largest finite
+  if (v == 0.0) return s;
+  int e;
+  std::frexp(v, &e);
+  const int lead = e - 1;
+  if (lead < -126) {  // subnormal: m * 2^-133
+    return s | (uint16_t)std::lround(std::ldexp(v, 133));
+  }
+  const int m = (int)std::lround((std::ldexp(v, -lead) - 1.0) * 128.0);
+  return s | (uint16_t)((lead + 127) << 7) | (uint16_t)m;
+}
+
+// OCP FP8 E4M3 ("fn"): bias 7, no infinities, S.1111.111 is NaN, max 448,
+// subnormals m * 2^-9.
+double or_e4m3_decode(uint8_t c) {
+  const int s = c >> 7, e = (c >> 3) & 0xF, m = c & 0x7;
+  double v;
+  if (e == 0xF && m == 0x7) v = kNaN;
+  else if (e == 0) v = std::ldexp((double)m, -9);
+  else v = std::ldexp(1.0 + m / 8.0, e - 7);
+  return s ? -v : v;
+}
+
+// Round-to-nearest-even, saturating to +-448 (R7: the cache never stores NaN for
+// finite inputs).
+uint8_t or_e4m3_encode(double x) {
+  if (std::isnan(x)) return 0x7F;
+  const uint8_t s = std::signbit(x) ? 0x80 : 0;
+  double v = std::fabs(round_binary(x, 4, -6));
+  if (v > 448.0) v = 448.0;
+  if (v == 0.0) return s;
+  if (v < std::ldexp(1.0, -6)) return s | (uint8_t)std::lround(std::ldexp(v, 9));
+  int e;
+  std::frexp(v, &e);
+  const int lead = e - 1;
+  const int m = (int)std::lround((std::ldexp(v, -lead) - 1.0) * 8.0);
+  return s | (uint8_t)((lead + 7) << 3) | (uint8_t)m;
+}
+
+// OCP MX E2M1 (a 4-bit code): bias 1, values 0, .5, 1, 1.5, 2, 3, 4, 6 with sign.
+double or_e2m1_decode(uint8_t nib) {
+  const int s = (nib >> 3) & 1, e = (nib >> 1) & 3, m = nib & 1;
+  const double v = (e == 0) ? 0.5 * m : std::ldexp(1.0 + 0.5 * m, e - 1);
+  return s ? -v : v;
+}
+
+// OCP MX E8M0 block scale: 2^(e-127), 0xFF is NaN.
+double or_e8m0_decode(uint8_t e) {
+  if (e == 0xFF) return kNaN;
+  return std::ldexp(1.0, (int)e - 127);
+}
+
+// Byte offset of the E8M0 scale of entry j, 32-element block s, in the indexer-key
+// scale array. Keys are grouped 128 to a 512-byte group; inside a group entry
+// j = r0 + 32*r1 (r0 < 32, r1 < 4) keeps its four block scales at 16*r0 + 4*r1 + s.
+size_t or_key_sf_offset(int64_t j, int s) {
+  const int64_t g = j / 128, r = j % 128;
+  return (size_t)(g * 512 + 16 * (r % 32) + 4 * (r / 32) + s);
+}
+
+// ------------------------------------------------------------ compression
+// One call compresses the T tokens at absolute positions pos0 .. pos0+T-1 of each of
+// B sequences (pos0 a multiple of m) into N = floor(T/m) entries (R3: only complete
+// blocks are emitted), entry i covering tokens pos0+m*i .. pos0+m*i+m-1.
+//
+// Gated merge [walkthrough §2.2: two independent KV sequences merged with
+// softmax-normalised gate weights, adjacent blocks overlap; chooseai 一: softmax with a
+// positional bias]: for every dim d the candidates are the m own-block tokens of `a`
+// with logits za + bias[r] and, when overlap = 1 (CSA), the m previous-block tokens of
+// `b` with logits zb + bias[m + r] (R1). The very first block of a sequence has no
+// previous block (R2); the first block of a later chunk takes it from prev_b/prev_zb.
+// Then RMSNorm (R4) [walkthrough §2.3: RMSNorm on the KV entries], RoPE on the last 64
+// dims at the entry's block-start position (R5, R6) [digest 2.: partial RoPE on the
+// last 64 dims], and the split store (R7): dims 0..447 as E4M3 of y/scale with
+// scale = amax/448, dims 448..511 as bf16 [chooseai 一: RoPE dims BF16, the rest FP8].
+//
+// Outputs (each nullable): e_out [B][N][512] merged entry before the norm,
+// y_out [B][N][512] final pre-quantisation value, kv [B][N][576], kv_scale [B][N].
+// Returns 0, or -1 for bad arguments.
+int or_compress(int B, int T, int m, int overlap, int64_t pos0, double rope_base,
+                double eps, const uint16_t* a, const uint16_t* b, const float* za,
+                const float* zb, const float* bias, const float* norm_w,
+                const uint16_t* prev_b, const float* prev_zb, double* e_out,
+                double* y_out, uint8_t* kv, float* kv_scale) {
+  if (B < 0 || T < 0 || m < 1 || pos0 < 0 || pos0 % m != 0) return -1;
+  if (!a || !za || !bias) return -1;
+  if (overlap && (!b || !zb)) return -1;
+  if (overlap && pos0 > 0 && (!prev_b || !prev_zb)) return -1;
+  const int N = T / m;
+  std::vector<double> xs, zs, e(kD), y(kD);
+  for (int bb = 0; bb < B; ++bb) {
+    for (int i = 0; i < N; ++i) {
+      for (int d = 0; d < kD; ++d) {
+        xs.clear();
+        zs.clear();
+        for (int r = 0; r < m; ++r) {  // own block, slots 0..m-1
+          const int64_t t = (int64_t)m * i + r;
+          const size_t o = ((size_t)bb * T + t) * kD + d;
+          xs.push_back(or_bf16_decode(a[o]));
+          zs.push_back((double)za[o] + (double)bias[r]);
+        }
+        if (overlap) {  // previous block, slots m..2m-1
+          for (int r = 0; r < m; ++r) {
+            if (i > 0) {
+              const size_t o = ((size_t)bb * T + (int64_t)m * (i - 1) + r) * kD + d;
+              xs.push_back(or_bf16_decode(b[o]));
+              zs.push_back((double)zb[o] + (double)bias[m + r]);
+            } else if (pos0 > 0) {
+              const size_t o = ((size_t)bb * m + r) * kD + d;
+              xs.push_back(or_bf16_decode(prev_b[o]));
+              zs.push_back((double)prev_zb[o] + (double)bias[m + r]);
+            }
+          }
+        }
+        double zmax = -kInf;
+        for (double z : zs) zmax = std::max(zmax, z);
+        double den = 0.0, num = 0.0;
+        for (size_t c = 0; c < zs.size(); ++c) {
+          const double g = std::exp(zs[c] - zmax);
+          den += g;
+          num += g * xs[c];
+        }
+        e[d] = num / den;
+      }
+      // RMSNorm
+      double ss = 0.0;
+      for (int d = 0; d < kD; ++d) ss += e[d] * e[d];
+      const double inv = 1.0 / std::sqrt(ss / kD + eps);
+      for (int d = 0; d < kD; ++d) y[d] = e[d] * inv * (norm_w ? (double)norm_w[d] : 1.0);
+      // RoPE on the interleaved pairs of the last 64 dims, position = block start
+      const double p = (double)(pos0 + (int64_t)m * i);
+      for (int j = 0; j < kRope / 2; ++j) {
+        const double theta = std::pow(rope_base, -(double)j / (kRope / 2));
+        const double c = std::cos(p * theta), s = std::sin(p * theta);
+        const double x0 = y[kNope + 2 * j], x1 = y[kNope + 2 * j + 1];
+        y[kNope + 2 * j] = x0 * c - x1 * s;
+        y[kNope + 2 * j + 1] = x0 * s + x1 * c;
+      }
+      const size_t eo = ((size_t)bb * N + i) * kD;
+      if (e_out) std::memcpy(e_out + eo, e.data(), kD * sizeof(double));
+      if (y_out) std::memcpy(y_out + eo, y.data(), kD * sizeof(double));
+      // split quantisation
+      double amax = 0.0;
+      for (int d = 0; d < kNope; ++d) amax = std::max(amax, std::fabs(y[d]));
+      const float sc = amax > 0.0 ? (float)(amax / 448.0) : 1.0f;
+      if (kv_scale) kv_scale[(size_t)bb * N + i] = sc;
+      if (kv) {
+        uint8_t* row = kv + ((size_t)bb * N + i) * kRow;
+        for (int d = 0; d < kNope; ++d) row[d] = or_e4m3_encode(y[d] / (double)sc);
+        for (int d = kNope; d < kD; ++d) {
+          const uint16_t h = or_bf16_encode(y[d]);
+          std::memcpy(row + kNope + 2 * (d - kNope), &h, 2);
+        }
+      }
+    }
+  }
+  return 0;
+}
+
+// Dequantise one stored entry (448 E4M3 codes times the entry scale, then 64 bf16).
+void or_dequant_row(const uint8_t* row, float scale, double* v) {
+  for (int d = 0; d < kNope; ++d) v[d] = or_e4m3_decode(row[d]) * (double)scale;
+  for (int d = kNope; d < kD; ++d) {
+    uint16_t h;
+    std::memcpy(&h, row + kNope + 2 * (d - kNope), 2);
+    v[d] = or_bf16_decode(h);
+  }
+}
+
+// ----------------------------------------------------------------- indexer
+// Lightning-indexer score of entry j for sequence b [walkthrough §2.2: low-rank,
+// low-precision indexer queries score the compressed entries; §3.4: the indexer QK
+// path runs in FP4 (MXFP4)]:
+//   s_j = sum_h w_h * max(0, sum_d q[h][d] * k[j][d])
+// with q and k decoded from E2M1 codes (element d in the low nibble of byte d/2 when d
+// is even) times their E8M0 block scale (one per 32 elements). No further scale (R9).
+// scores [B][Nmax]: entries j >= n_entries[b] are set to NaN.
+int or_indexer_scores(int B, int H_I, int64_t Nmax, const int32_t* n_entries,
+                      const uint8_t* q_fp4, const uint8_t* q_sf, const float* w,
+                      const uint8_t* k_fp4, const uint8_t* k_sf, double* scores,
+                      int nthreads) {
+  if (B < 0 || H_I < 1 || Nmax < 0 || Nmax % 128 != 0) return -1;
+  for (int bb = 0; bb < B; ++bb)
+    if (n_entries[bb] < 0 || n_entries[bb] > Nmax) return -1;
+  if (nthreads <= 0) nthreads = (int)std::max(1u, std::thread::hardware_concurrency());
+  auto work = [&](int tid) {
+    std::vector<double> q((size_t)H_I * kDI), k(kDI);
+    for (int bb = 0; bb < B; ++bb) {
+      for (int h = 0; h < H_I; ++h)
+        for (int d = 0; d < kDI; ++d) {
+          const uint8_t byte = q_fp4[((size_t)bb * H_I + h) * (kDI / 2) + d / 2];
+          const uint8_t nib = (d % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+          q[(size_t)h * kDI + d] =
+              or_e2m1_decode(nib) * or_e8m0_decode(q_sf[((size_t)bb * H_I + h) * 4 + d / 32]);
+        }
+      for (int64_t j = tid; j < Nmax; j += nthreads) {
+        double* out = scores + (size_t)bb * Nmax + j;
+        if (j >= n_entries[bb]) {
+          *out = kNaN;
+          continue;
+        }
+        const uint8_t* kr = k_fp4 + ((size_t)bb * Nmax + j) * (kDI / 2);
+        const uint8_t* ks = k_sf + (size_t)bb * Nmax * 4;
+        for (int d = 0; d < kDI; ++d) {
+          const uint8_t nib = (d % 2 == 0) ? (kr[d / 2] & 0xF) : (kr[d / 2] >> 4);
+          k[d] = or_e2m1_decode(nib) * or_e8m0_decode(ks[or_key_sf_offset(j, d / 32)]);
+        }
+        double s = 0.0;
+        for (int h = 0; h < H_I; ++h) {
+          double dot = 0.0;
+          for (int d = 0; d < kDI; ++d) dot += q[(size_t)h * kDI + d] * k[d];
+          s += (double)w[(size_t)bb * H_I + h] * std::max(0.0, dot);
+        }
+        *out = s;
+      }
+    }
+  };
+  std::vector<std::thread> pool;
+  for (int t = 0; t < nthreads; ++t) pool.emplace_back(work, t);
+  for (auto& th : pool) th.join();
+  return 0;
+}
+
+// Top-k [walkthrough §2.2: each query selects the top-k compressed entries; one index
+// set per query shared by all heads]: order the n scores by (score descending, index
+// ascending), keep the first min(k, n), emit them in ascending index order and pad
+// with -1 up to k.
+int or_topk(int64_t n, int k, const double* scores, int32_t* idx) {
+  if (n < 0 || k < 1) return -1;
+  std::vector<int32_t> order((size_t)n);
+  for (int64_t j = 0; j < n; ++j) order[(size_t)j] = (int32_t)j;
+  std::sort(order.begin(), order.end(), [&](int32_t x, int32_t y) {
+    if (scores[x] != scores[y]) return scores[x] > scores[y];
+    return x < y;
+  });
+  const int64_t keep = std::min<int64_t>(k, n);
+  std::sort(order.begin(), order.begin() + keep);
+  for (int i = 0; i < k; ++i) idx[i] = i < keep ? order[(size_t)i] : -1;
+  return 0;
+}
+
+// --------------------------------------------------------------- attention
+// Shared-KV MQA for one query token per sequence [tutorial, Hybrid Attention: shared
+// key-value MQA, every head reads the same entry as key and value]; the row set is
+// the selected entries (CSA, sparse = 1) or all n_entries[b] entries (HCA, sparse = 0)
+// [chooseai 一: HCA attends densely, no top-k], plus the sliding-window tokens
+// max(0,t-127)..t [walkthrough §2.2: the most recent 128 uncompressed tokens join the
+// core attention] read from the ring swa[b][p % 128] (R8, R13), with the sink logit
+// sigma_h added to the denominator only [digest 2.: learnable sink logit, the scores
+// may sum to less than 1]:
+//   l_j = tau * q_h . v_j,  Z = exp(sigma_h) + sum_j exp(l_j),  o_h = sum_j exp(l_j)/Z v_j
+// (R12: tau given by the caller, sink unscaled). lse = log Z. When derotate = 1 the
+// last 64 output dims are rotated by -t*theta (R15) [tutorial, Partial RoPE: the
+// output is processed so absolute position does not leak into the value output].
+// out [B][H][512], lse [B][H]. Returns 0, or -1 for an out-of-range index.
+int or_attention(int B, int H, int k, int64_t Nmax, int sparse, const uint16_t* q,
+                 const int32_t* pos, const int32_t* idx, const int32_t* n_entries,
+                 const uint8_t* kv, const float* kv_scale, const uint16_t* swa,
+                 const float* sink, double tau, double rope_base, int derotate,
+                 double* out, double* lse, int nthreads) {
+  if (B < 0 || H < 1 || Nmax < 0) return -1;
+  for (int bb = 0; bb < B; ++bb) {
+    if (pos[bb] < 0 || n_entries[bb] < 0 || n_entries[bb] > Nmax) return -1;
+    if (sparse)
+      for (int i = 0; i < k; ++i) {
+        const int32_t j = idx[(size_t)bb * k + i];
+        if (j < -1 || j >= n_entries[bb]) return -1;
+      }
+  }
+  if (nthreads <= 0) nthreads = (int)std::max(1u, std::thread::hardware_concurrency());
+  auto work = [&](int tid) {
+    std::vector<double> rows, v(kD);
+    for (int bb = tid; bb < B; bb += nthreads) {
+      const int64_t t = pos[bb];
+      rows.clear();  // gather every visible row, dequantised
+      if (sparse) {
+        for (int i = 0; i < k; ++i) {
+          const int32_t j = idx[(size_t)bb * k + i];
+          if (j < 0) continue;
+          or_dequant_row(kv + ((size_t)bb * Nmax + j) * kRow, kv_scale[(size_t)bb * Nmax + j],
+                         v.data());
+          rows.insert(rows.end(), v.begin(), v.end());
+        }
+      } else {
+        for (int32_t j = 0; j < n_entries[bb]; ++j) {
+          or_dequant_row(kv + ((size_t)bb * Nmax + j) * kRow, kv_scale[(size_t)bb * Nmax + j],
+                         v.data());
+          rows.insert(rows.end(), v.begin(), v.end());
+        }
+      }
+      for (int64_t p = std::max<int64_t>(0, t - (kWin - 1)); p <= t; ++p) {
+        const uint16_t* sr = swa + ((size_t)bb * kWin + (size_t)(p % kWin)) * kD;
+        for (int d = 0; d < kD; ++d) v[d] = or_bf16_decode(sr[d]);
+        rows.insert(rows.end(), v.begin(), v.end());
+      }
+      const size_t nr = rows.size() / kD;
+      std::vector<double> l(nr);
+      for (int h = 0; h < H; ++h) {
+        const uint16_t* qh = q + ((size_t)bb * H + h) * kD;
+        double* o = out + ((size_t)bb * H + h) * kD;
+        const double sig = (double)sink[h];
+        if (sig == kInf) {  // the sink takes all of the mass
+          for (int d = 0; d < kD; ++d) o[d] = 0.0;
+          if (lse) lse[(size_t)bb * H + h] = kInf;
+          continue;
+        }
+        double lmax = sig;
+        for (size_t r = 0; r < nr; ++r) {
+          double dot = 0.0;
+          for (int d = 0; d < kD; ++d) dot += or_bf16_decode(qh[d]) * rows[r * kD + d];
+          l[r] = tau * dot;
+          lmax = std::max(lmax, l[r]);
+        }
+        double Z = std::exp(sig - lmax);  // 0 when the sink is -inf
+        for (size_t r = 0; r < nr; ++r) Z += std::exp(l[r] - lmax);
+        for (int d = 0; d < kD; ++d) o[d] = 0.0;
+        for (size_t r = 0; r < nr; ++r) {
+          const double pr = std::exp(l[r] - lmax) / Z;
+          for (int d = 0; d < kD; ++d) o[d] += pr * rows[r * kD + d];
+        }
+        if (lse) lse[(size_t)bb * H + h] = lmax + std::log(Z);
+        if (derotate) {
+          for (int j = 0; j < kRope / 2; ++j) {
+            const double theta = std::pow(rope_base, -(double)j / (kRope / 2));
+            const double c = std::cos((double)t * theta), s = std::sin((double)t * theta);
+            const double x0 = o[kNope + 2 * j], x1 = o[kNope + 2 * j + 1];
+            o[kNope + 2 * j] = x0 * c + x1 * s;
+            o[kNope + 2 * j + 1] = -x0 * s + x1 * c;
+          }
+        }
+      }
+    }
+  };
+  std::vector<std::thread> pool;
+  for (int t = 0; t < nthreads; ++t) pool.emplace_back(work, t);
+  for (auto& th : pool) th.join();
+  return 0;
+}
+
+// ------------------------------------------------------------------ prefill
+// Sliding-window row of token t (R8): the raw KV a[t] goes through the same RMSNorm
+// and the RoPE rotation at position t as an entry, and is stored as bf16.
+void or_swa_row(const uint16_t* a_row, int64_t t, double rope_base, double eps,
+                const float* norm_w, uint16_t* out_row) {
+  std::vector<double> y(kD);
+  double ss = 0.0;
+  for (int d = 0; d < kD; ++d) {
+    y[d] = or_bf16_decode(a_row[d]);
+    ss += y[d] * y[d];
+  }
+  const double inv = 1.0 / std::sqrt(ss / kD + eps);
+  for (int d = 0; d < kD; ++d) y[d] = y[d] * inv * (norm_w ? (double)norm_w[d] : 1.0);
+  for (int j = 0; j < kRope / 2; ++j) {
+    const double theta = std::pow(rope_base, -(double)j / (kRope / 2));
+    const double c = std::cos((double)t * theta), s = std::sin((double)t * theta);
+    const double x0 = y[kNope + 2 * j], x1 = y[kNope + 2 * j + 1];
+    y[kNope + 2 * j] = x0 * c - x1 * s;
+    y[kNope + 2 * j + 1] = x0 * s + x1 * c;
+  }
+  for (int d = 0; d < kD; ++d) out_row[d] = or_bf16_encode(y[d]);
+}
+
+// Causal chunked prefill of T new tokens after a P-token prefix (one sequence)
+// [walkthrough §3.5: the state cache holds the 128 window tokens and the tail of the
+// unfinished block; the classical cache holds the compressed entries]. Compression of
+// the new blocks is part of the pass: entries P/m .. (P+T)/m - 1 are written into
+// kv/kv_scale (rows 0 .. P/m - 1 are the cached prefix). Then, for every requested
+// query row r (token t = P + r): n(t) = floor((t+1)/m) eligible entries (R11), indexer
+// scores over them, top-k, and the attention of or_attention over the selected
+// entries plus the window t-127..t, whose rows come from swa_prefix (ring slot p % 128)
+// for p < P and from or_swa_row of the new tokens for p >= P.
+// q_rows [nq] lists the rows to evaluate; out [nq][H][512], lse [nq][H], idx [nq][k].
+int or_prefill(int64_t P, int T, int m, int H, int H_I, int k, double rope_base,
+               double eps, double tau, int derotate, const uint16_t* a, const uint16_t* b,
+               const float* za, const float* zb, const float* bias, const float* norm_w,
+               const uint16_t* prev_b, const float* prev_zb, uint8_t* kv, float* kv_scale,
+               int64_t Nmax, const uint8_t* q_fp4, const uint8_t* q_sf, const float* w,
+               const uint8_t* k_fp4, const uint8_t* k_sf, const uint16_t* q,
+               const float* sink, const uint16_t* swa_prefix, int nq,
+               const int32_t* q_rows, double* out, double* lse, int32_t* idx,
+               int nthreads) {
+  if (P < 0 || T < 0 || m < 1 || P % m != 0 || (P + T) / m > Nmax) return -1;
+  if (P > 0 && !swa_prefix) return -1;
+  const int64_t n0 = P / m;
+  int rc = or_compress(1, T, m, 1, P, rope_base, eps, a, b, za, zb, bias, norm_w, prev_b,
+                       prev_zb, nullptr, nullptr, kv + (size_t)n0 * kRow, kv_scale + n0);
+  if (rc) return rc;
+  for (int i = 0; i < nq; ++i)
+    if (q_rows[i] < 0 || q_rows[i] >= T) return -1;
+  if (nthreads <= 0) nthreads = (int)std::max(1u, std::thread::hardware_concurrency());
+  std::vector<int> status(nthreads, 0);
+  auto work = [&](int tid) {
+    std::vector<double> scores((size_t)Nmax);
+    std::vector<uint16_t> ring((size_t)kWin * kD);
+    for (int i = tid; i < nq; i += nthreads) {
+      const int r = q_rows[i];
+      const int64_t t = P + r;
+      const int32_t n = (int32_t)((t + 1) / m);
+      int32_t* sel = idx + (size_t)i * k;
+      if (or_indexer_scores(1, H_I, Nmax, &n, q_fp4 + (size_t)r * H_I * (kDI / 2),
+                            q_sf + (size_t)r * H_I * 4, w + (size_t)r * H_I, k_fp4, k_sf,
+                            scores.data(), 1) ||
+          or_topk(n, k, scores.data(), sel)) {
+        status[tid] = -1;
+        return;
+      }
+      for (int64_t p = std::max<int64_t>(0, t - (kWin - 1)); p <= t; ++p) {
+        uint16_t* dst = ring.data() + (size_t)(p % kWin) * kD;
+        if (p < P)
+          std::memcpy(dst, swa_prefix + (size_t)(p % kWin) * kD, kD * sizeof(uint16_t));
+        else
+          or_swa_row(a + (size_t)(p - P) * kD, p, rope_base, eps, norm_w, dst);
+      }
+      const int32_t tq = (int32_t)t;
+      if (or_attention(1, H, k, Nmax, 1, q + (size_t)r * H * kD, &tq, sel, &n, kv, kv_scale,
+                       ring.data(), sink, tau, rope_base, derotate,
+                       out + (size_t)i * H * kD, lse ? lse + (size_t)i * H : nullptr, 1)) {
+        status[tid] = -1;
+        return;
+      }
+    }
+  };
+  std::vector<std::thread> pool;
+  for (int t = 0; t < nthreads; ++t) pool.emplace_back(work, t);
+  for (auto& th : pool) th.join();
+  for (int s : status)
+    if (s) return s;
+  return 0;
+}
+
+}  // extern "C"
