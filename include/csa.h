@@ -1,0 +1,199 @@
+/* C ABI of the B200 (sm_100a) CSA/HCA compressed attention layer.
+ *
+ * The layer is the hybrid compressed attention of the DeepSeek-V4 pages:
+ *   CSA (Compressed Sparse Attention): KV compressed by m = 4 with overlapping
+ *       gated-softmax merges, lightning-indexer scoring of the compressed entries in FP4,
+ *       top-k selection, shared-KV MQA over the selected entries;
+ *   HCA (Heavily Compressed Attention): KV compressed by m' = 128 without overlap, dense
+ *       MQA over every compressed entry;
+ *   both with a 128-token uncompressed sliding window and a per-head sink logit in the
+ *   same softmax, head_dim 512 with RoPE on the last 64 dims, and an entry stored as 448
+ *   FP8-E4M3 dims (with one fp32 scale per entry) plus 64 BF16 dims.
+ * Sources: cyqw.cn/news/842812 DeepSeek-V4 walkthrough §2.2 (CSA/HCA, overlap, indexer,
+ * top-k, window, sink), §2.3 (RMSNorm on KV entries), §3.4 (FP4 indexer QK path), §3.5
+ * (state cache); chooseai.net/news/3476 §一 (m = 4 / 128, softmax merge with positional
+ * bias, FP8 + BF16 split, top-k 512/1024); "DeepSeek V4技术报告详解" §2 (head_dim 512,
+ * partial RoPE on the last 64 dims, sink logit); "DeepSeek-V4：百万上下文的工程答案",
+ * Hybrid Attention / Partial RoPE / Attention sink (shared-KV MQA, output de-rotation).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers, caller-owned, 16-byte aligned, dense
+ *    row-major in the shapes given. The library never allocates, frees or synchronises.
+ *    Scratch memory comes from a caller workspace of at least the size reported by the
+ *    matching *_workspace_size function, 256-byte aligned.
+ *  - Work is enqueued on `stream` (a cudaStream_t; 0 = legacy default stream).
+ *  - Arguments are checked on the host before any launch. On a bad argument the call
+ *    returns CSA_ERR_INVALID_ARG / CSA_ERR_UNSUPPORTED / CSA_ERR_WORKSPACE and launches
+ *    nothing. A failed launch returns CSA_ERR_CUDA.
+ *  - Data-dependent problems found by a kernel (an index outside the eligible range, a
+ *    length beyond the capacity) are written to the optional device word *dev_status
+ *    (first error wins, CSA_ERR_DEVICE); the affected rows are skipped. Read it after
+ *    synchronising the stream.
+ *  - Results are deterministic and batch-invariant: a sequence gives the same bits
+ *    whatever the batch around it.
+ */
+#ifndef CSA_B200_H
+#define CSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* csa_stream_t; /* the same type as cudaStream_t */
+
+enum {
+  CSA_OK = 0,
+  CSA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or flag */
+  CSA_ERR_UNSUPPORTED = 2, /* valid but not built (e.g. a head count outside the list) */
+  CSA_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small */
+  CSA_ERR_CUDA = 4,        /* a CUDA launch or driver call failed */
+  CSA_ERR_DEVICE = 5,      /* written to dev_status by a kernel: bad data, rows skipped */
+  CSA_ERR_TIMEOUT = 6      /* written to dev_status: a bounded device wait gave up */
+};
+
+#define CSA_HEAD_DIM 512   /* shared KV entry dims */
+#define CSA_NOPE_DIM 448   /* dims stored as FP8 E4M3 */
+#define CSA_ROPE_DIM 64    /* last dims, RoPE, stored as BF16 */
+#define CSA_ROW_BYTES 576  /* 448 E4M3 bytes then 64 BF16 values */
+#define CSA_INDEX_DIM 128  /* indexer head dim (E2M1, 64 bytes per head) */
+#define CSA_WINDOW 128     /* sliding-window tokens */
+
+/* Short description of a status code (static storage). */
+const char* csa_status_string(int status);
+
+/* ------------------------------------------------------------------------------------
+ * csa_compress: gated-softmax block compression of the KV stream into stored entries.
+ * (walkthrough §2.2: two independent KV sequences merged with softmax-normalised gate
+ * weights, adjacent blocks overlap; chooseai §一: positional bias; walkthrough §2.3:
+ * RMSNorm on the entries; chooseai §一: RoPE dims BF16, others FP8.)
+ *
+ * The T tokens at absolute positions pos0 .. pos0+T-1 of each sequence (pos0 a multiple
+ * of m) give N = floor(T/m) entries; entry i covers tokens pos0+m*i .. pos0+m*i+m-1 and is
+ * stored at row pos0/m + i. For every dim d the merge is a softmax over the candidates
+ *   own block:  a[m*i + r][d]       with logit za[m*i + r][d] + bias[r],        r < m
+ *   previous:   b[m*(i-1) + r][d]   with logit zb[m*(i-1) + r][d] + bias[m + r]
+ *               (overlap = 1 only; for i = 0 from prev_b / prev_zb when pos0 > 0, absent
+ *               when pos0 == 0)
+ * followed by y = e / sqrt(mean(e^2) + eps) * norm_w, RoPE on the interleaved pairs
+ * (448+2j, 449+2j) by angle (pos0 + m*i) * rope_base^(-j/32), and the split store:
+ * scale = max|y[0..447]| / 448 (1 if zero), bytes 0..447 = E4M3(y[d] / scale) rounded to
+ * nearest even and saturated, bytes 448..575 = BF16(y[448..511]) rounded to nearest even.
+ * Computed in fp32 on the device. Supports 1 <= m <= 128.
+ */
+typedef struct {
+  int32_t B;             /* sequences */
+  int32_t T;             /* tokens per sequence in this call (row pitch of a, b, za, zb) */
+  int32_t m;             /* block size: 4 for CSA, 128 for HCA */
+  int32_t overlap;       /* 1: CSA overlapping merge (needs b, zb); 0: HCA */
+  int64_t pos0;          /* absolute position of token 0, a multiple of m */
+  float rope_base;       /* 10000 */
+  float eps;             /* RMSNorm epsilon, e.g. 1e-6 */
+  const uint16_t* a;     /* bf16 [B][T][512] */
+  const uint16_t* b;     /* bf16 [B][T][512]; NULL when overlap == 0 */
+  const float* za;       /* [B][T][512] gate logits paired with a */
+  const float* zb;       /* [B][T][512] gate logits paired with b; NULL when overlap == 0 */
+  const float* bias;     /* [2m] (overlap) or [m] */
+  const float* norm_w;   /* [512] RMSNorm weight, NULL = ones */
+  const uint16_t* prev_b; /* bf16 [B][m][512]: tokens pos0-m .. pos0-1 of b (overlap, pos0>0) */
+  const float* prev_zb;  /* [B][m][512] */
+  uint8_t* kv;           /* out [B][Nmax][576] */
+  float* kv_scale;       /* out [B][Nmax] */
+  int64_t Nmax;          /* entry capacity per sequence; pos0/m + N <= Nmax */
+  float* dbg;            /* optional out [B][N][512]: fp32 y before quantisation */
+} csa_compress_args;
+
+int csa_compress(const csa_compress_args* args, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa_indexer_topk: lightning-indexer scores of every eligible entry and the top-k set.
+ * (walkthrough §2.2: the indexer scores compressed entries, each query keeps the top-k,
+ * one set shared by all heads; §3.4 and chooseai §二: the indexer QK path is MXFP4.)
+ *
+ *   s_j = sum_h w[h] * max(0, sum_d q[h][d] * k_j[d]),   j < n_entries[b]
+ * where q and k are E2M1 codes times their E8M0 block scale (one per 32 dims). The set
+ * is the first min(k, n) entries by (score descending, index ascending), written in
+ * ascending index order and padded with -1. Scores are formed in fp32 from the FP4
+ * tensor-core products (tcgen05 kind::mxf4).
+ *
+ * Layouts: q_fp4 [B][H_I][64] and k_fp4 [B][Nmax][64] hold two E2M1 codes per byte,
+ * element 2i in the low nibble of byte i. q_sf [B][H_I][4] holds the 4 block scales of
+ * each query head. k_sf is grouped by 128 entries: [B][Nmax/128][512] bytes, and the
+ * scale of entry j (j = 128g + 32r1 + r0), block s, sits at byte 16*r0 + 4*r1 + s of
+ * group g -- the tensor-core scale-factor atom, so a group is copied as is.
+ * Nmax must be a multiple of 128. 1 <= k <= 2048, H_I in {16, 32, 64}.
+ * The workspace must be zero-filled once before its first use; every call leaves it
+ * zeroed again. Calls that share a workspace must not overlap on the device.
+ */
+typedef struct {
+  int32_t B;
+  int32_t H_I;                /* indexer heads: 16, 32 or 64 */
+  int32_t k;                  /* top-k */
+  int64_t Nmax;               /* entry capacity per sequence, multiple of 128 */
+  const int32_t* n_entries;   /* [B] eligible entries per sequence, <= Nmax */
+  const uint8_t* q_fp4;       /* [B][H_I][64] */
+  const uint8_t* q_sf;        /* [B][H_I][4] E8M0 */
+  const float* w;             /* [B][H_I] head weights */
+  const uint8_t* k_fp4;       /* [B][Nmax][64] */
+  const uint8_t* k_sf;        /* [B][Nmax/128][512] grouped E8M0 */
+  int32_t* idx;               /* out [B][k] ascending, -1 padded */
+  float* scores;              /* optional out [B][k]: score of idx[b][i] (NaN for -1) */
+  int32_t* dev_status;        /* optional device word, see conventions */
+} csa_topk_args;
+
+size_t csa_indexer_topk_workspace_size(int32_t B, int64_t Nmax, int32_t k);
+int csa_indexer_topk(const csa_topk_args* args, void* workspace, size_t workspace_bytes,
+                     csa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa_sparse_attn_decode / hca_attn_decode: one query token per sequence.
+ * (tutorial "Hybrid Attention": shared key-value MQA; walkthrough §2.2: the 128 most
+ * recent uncompressed tokens join the core attention, sink added to the denominator;
+ * tutorial "Partial RoPE": the output is de-rotated.)
+ *
+ * For head h of sequence b at position t = pos[b], over the rows
+ *   CSA: the entries idx[b][0..k) (-1 = padding, skipped), every index < n_entries[b];
+ *   HCA: the entries 0 .. n_entries[b]-1;
+ *   both: window tokens p = max(0, t-127) .. t from the ring swa[b][p % 128];
+ *   l_j = tau * q[b][h] . v_j,  Z = exp(sink[h]) + sum_j exp(l_j),
+ *   out[b][h] = sum_j exp(l_j) / Z * v_j,  lse[b][h] = log Z,
+ * with v_j the dequantised entry (E4M3 code * entry scale, then the BF16 dims) or the
+ * BF16 window row; when derotate = 1, output pairs (448+2j, 449+2j) are turned by
+ * -t * rope_base^(-j/32). Products run on tcgen05 BF16 tensor cores (entries are
+ * dequantised to BF16 in shared memory), accumulation and softmax in fp32.
+ * H in {64, 128}. k <= 2048 (CSA); n_entries <= Nmax (HCA, any size).
+ */
+typedef struct {
+  int32_t B;
+  int32_t H;                  /* query heads: 64 or 128 */
+  int32_t k;                  /* CSA: selected entries per sequence; ignored by HCA */
+  int64_t Nmax;               /* entry capacity per sequence */
+  const uint16_t* q;          /* bf16 [B][H][512], already normalised and rotated */
+  const int32_t* pos;         /* [B] query positions t >= 0 */
+  const int32_t* idx;         /* [B][k] (CSA only) */
+  const int32_t* n_entries;   /* [B] eligible entries */
+  const uint8_t* kv;          /* [B][Nmax][576] stored entries */
+  const float* kv_scale;      /* [B][Nmax] */
+  const uint16_t* swa;        /* bf16 [B][128][512] window ring */
+  const float* sink;          /* [H] sink logits (+-inf allowed) */
+  float tau;                  /* softmax scale; 0 selects 1/sqrt(512) */
+  float rope_base;            /* 10000 */
+  int32_t derotate;           /* 1: de-rotate the last 64 output dims by the query position */
+  uint16_t* out;              /* out bf16 [B][H][512] */
+  float* lse;                 /* optional out [B][H] */
+  int32_t* dev_status;        /* optional device word */
+} csa_attn_args;
+
+size_t csa_attn_workspace_size(int32_t B, int32_t H, int32_t rows_max);
+int csa_sparse_attn_decode(const csa_attn_args* args, void* workspace, size_t workspace_bytes,
+                           csa_stream_t stream);
+int hca_attn_decode(const csa_attn_args* args, void* workspace, size_t workspace_bytes,
+                    csa_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_B200_H */

@@ -1,0 +1,206 @@
+"""Python binding of the B200 CSA/HCA compressed attention library (libcsa_b200.so).
+
+Argument marshalling only: every step of the layer runs in the sm_100a kernels behind the
+C ABI declared in include/csa.h. PyTorch supplies device memory and the current stream.
+If the shared library is missing the import of a function raises; there is no fallback.
+
+bf16 inputs may be torch.bfloat16 tensors or 16-bit integer tensors holding bf16 bits.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libcsa_b200.so")
+
+HEAD_DIM, NOPE_DIM, ROPE_DIM, ROW_BYTES, INDEX_DIM, WINDOW = 512, 448, 64, 576, 128, 128
+
+CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE = 0, 1, 2, 3
+CSA_ERR_CUDA, CSA_ERR_DEVICE, CSA_ERR_TIMEOUT = 4, 5, 6
+
+_vp = C.c_void_p
+
+
+class CompressArgs(C.Structure):
+    _fields_ = [("B", C.c_int32), ("T", C.c_int32), ("m", C.c_int32), ("overlap", C.c_int32),
+                ("pos0", C.c_int64), ("rope_base", C.c_float), ("eps", C.c_float),
+                ("a", _vp), ("b", _vp), ("za", _vp), ("zb", _vp), ("bias", _vp),
+                ("norm_w", _vp), ("prev_b", _vp), ("prev_zb", _vp), ("kv", _vp),
+                ("kv_scale", _vp), ("Nmax", C.c_int64), ("dbg", _vp)]
+
+
+class TopkArgs(C.Structure):
+    _fields_ = [("B", C.c_int32), ("H_I", C.c_int32), ("k", C.c_int32), ("Nmax", C.c_int64),
+                ("n_entries", _vp), ("q_fp4", _vp), ("q_sf", _vp), ("w", _vp),
+                ("k_fp4", _vp), ("k_sf", _vp), ("idx", _vp), ("scores", _vp),
+                ("dev_status", _vp)]
+
+
+class AttnArgs(C.Structure):
+    _fields_ = [("B", C.c_int32), ("H", C.c_int32), ("k", C.c_int32), ("Nmax", C.c_int64),
+                ("q", _vp), ("pos", _vp), ("idx", _vp), ("n_entries", _vp), ("kv", _vp),
+                ("kv_scale", _vp), ("swa", _vp), ("sink", _vp), ("tau", C.c_float),
+                ("rope_base", C.c_float), ("derotate", C.c_int32), ("out", _vp), ("lse", _vp),
+                ("dev_status", _vp)]
+
+
+EXPORTS = ["csa_status_string", "csa_compress", "csa_indexer_topk_workspace_size",
+           "csa_indexer_topk", "csa_attn_workspace_size", "csa_sparse_attn_decode",
+           "hca_attn_decode"]
+
+_lib = None
+
+
+def lib() -> C.CDLL:
+    """Load libcsa_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m long_context_compressed_layer_b200.build`")
+        L = C.CDLL(LIB_PATH)
+        L.csa_status_string.restype = C.c_char_p
+        L.csa_status_string.argtypes = [C.c_int]
+        L.csa_compress.restype = C.c_int
+        L.csa_compress.argtypes = [C.POINTER(CompressArgs), _vp]
+        L.csa_indexer_topk_workspace_size.restype = C.c_size_t
+        L.csa_indexer_topk_workspace_size.argtypes = [C.c_int32, C.c_int64, C.c_int32]
+        L.csa_indexer_topk.restype = C.c_int
+        L.csa_indexer_topk.argtypes = [C.POINTER(TopkArgs), _vp, C.c_size_t, _vp]
+        L.csa_attn_workspace_size.restype = C.c_size_t
+        L.csa_attn_workspace_size.argtypes = [C.c_int32, C.c_int32, C.c_int32]
+        for f in ("csa_sparse_attn_decode", "hca_attn_decode"):
+            getattr(L, f).restype = C.c_int
+            getattr(L, f).argtypes = [C.POINTER(AttnArgs), _vp, C.c_size_t, _vp]
+        _lib = L
+    return _lib
+
+
+class CSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {lib().csa_status_string(status).decode()} ({status})")
+        self.status = status
+
+
+def _check(status: int, where: str) -> None:
+    if status != CSA_OK:
+        raise CSAError(status, where)
+
+
+def _ptr(t: torch.Tensor | None, *, elem: int | None = None, name: str = "") -> int | None:
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous CUDA tensor")
+    if elem is not None and t.element_size() != elem:
+        raise ValueError(f"{name}: expected {elem}-byte elements, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+# ------------------------------------------------------------------ compress
+def compress(a, za, bias, m: int, overlap: bool, *, b=None, zb=None, pos0: int = 0,
+             prev_b=None, prev_zb=None, kv=None, kv_scale=None, Nmax: int | None = None,
+             rope_base: float = 10000.0, eps: float = 1e-6, norm_w=None, dbg: bool = False,
+             stream=None):
+    """Compress a [B][T][512] stream into entries pos0/m .. pos0/m + T/m - 1.
+    Returns (kv [B][Nmax][576] uint8, kv_scale [B][Nmax] float32, dbg [B][N][512] or None);
+    kv/kv_scale are written in place when given."""
+    B, T, _ = a.shape
+    N = T // m
+    if Nmax is None:
+        Nmax = kv.shape[1] if kv is not None else pos0 // m + N
+    dev = a.device
+    if kv is None:
+        kv = torch.zeros((B, Nmax, ROW_BYTES), dtype=torch.uint8, device=dev)
+    if kv_scale is None:
+        kv_scale = torch.zeros((B, Nmax), dtype=torch.float32, device=dev)
+    d = torch.empty((B, N, HEAD_DIM), dtype=torch.float32, device=dev) if dbg else None
+    args = CompressArgs(B, T, m, int(overlap), pos0, rope_base, eps,
+                        _ptr(a, elem=2, name="a"), _ptr(b, elem=2, name="b"),
+                        _ptr(za, elem=4, name="za"), _ptr(zb, elem=4, name="zb"),
+                        _ptr(bias, elem=4, name="bias"), _ptr(norm_w, elem=4, name="norm_w"),
+                        _ptr(prev_b, elem=2, name="prev_b"), _ptr(prev_zb, elem=4, name="prev_zb"),
+                        _ptr(kv, elem=1, name="kv"), _ptr(kv_scale, elem=4, name="kv_scale"),
+                        Nmax, _ptr(d, elem=4, name="dbg"))
+    _check(lib().csa_compress(C.byref(args), _stream(stream)), "csa_compress")
+    return kv, kv_scale, d
+
+
+# ------------------------------------------------------------- indexer top-k
+def indexer_topk_workspace(B: int, Nmax: int, k: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace (the library keeps it zeroed between calls)."""
+    n = lib().csa_indexer_topk_workspace_size(B, Nmax, k)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def indexer_topk(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, k: int, *, workspace=None, idx=None,
+                 scores: bool = False, dev_status=None, stream=None):
+    """Top-k entry indices [B][k] (ascending, -1 padded) and optionally their scores."""
+    B, H_I, _ = q_fp4.shape
+    Nmax = k_fp4.shape[1]
+    dev = q_fp4.device
+    if workspace is None:
+        workspace = indexer_topk_workspace(B, Nmax, k, dev)
+    if idx is None:
+        idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+    sc = torch.empty((B, k), dtype=torch.float32, device=dev) if scores else None
+    args = TopkArgs(B, H_I, k, Nmax, _ptr(n_entries, elem=4, name="n_entries"),
+                    _ptr(q_fp4, elem=1, name="q_fp4"), _ptr(q_sf, elem=1, name="q_sf"),
+                    _ptr(w, elem=4, name="w"), _ptr(k_fp4, elem=1, name="k_fp4"),
+                    _ptr(k_sf, elem=1, name="k_sf"), _ptr(idx, elem=4, name="idx"),
+                    _ptr(sc, elem=4, name="scores"), _ptr(dev_status, elem=4, name="dev_status"))
+    _check(lib().csa_indexer_topk(C.byref(args), workspace.data_ptr(), workspace.numel(),
+                                  _stream(stream)), "csa_indexer_topk")
+    return (idx, sc) if scores else idx
+
+
+# ------------------------------------------------------------------ attention
+def attn_workspace(B: int, H: int, rows_max: int, device="cuda") -> torch.Tensor:
+    n = lib().csa_attn_workspace_size(B, H, rows_max)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def _attn(fn: str, sparse: bool, q, pos, n_entries, kv, kv_scale, swa, sink, idx, *,
+          tau: float = 0.0, rope_base: float = 10000.0, derotate: bool = True,
+          workspace=None, out=None, lse: bool = False, dev_status=None, stream=None):
+    B, H, _ = q.shape
+    Nmax = kv.shape[1]
+    k = idx.shape[1] if sparse else 0
+    dev = q.device
+    if workspace is None:
+        workspace = attn_workspace(B, H, (k if sparse else Nmax) + WINDOW, dev)
+    if out is None:
+        out = torch.empty((B, H, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    l = torch.empty((B, H), dtype=torch.float32, device=dev) if lse else None
+    args = AttnArgs(B, H, k, Nmax, _ptr(q, elem=2, name="q"), _ptr(pos, elem=4, name="pos"),
+                    _ptr(idx, elem=4, name="idx") if sparse else None,
+                    _ptr(n_entries, elem=4, name="n_entries"), _ptr(kv, elem=1, name="kv"),
+                    _ptr(kv_scale, elem=4, name="kv_scale"), _ptr(swa, elem=2, name="swa"),
+                    _ptr(sink, elem=4, name="sink"), tau, rope_base, int(derotate),
+                    _ptr(out, elem=2, name="out"), _ptr(l, elem=4, name="lse"),
+                    _ptr(dev_status, elem=4, name="dev_status"))
+    _check(getattr(lib(), fn)(C.byref(args), workspace.data_ptr(), workspace.numel(),
+                              _stream(stream)), fn)
+    return (out, l) if lse else out
+
+
+def sparse_attn_decode(q, pos, n_entries, kv, kv_scale, swa, sink, idx, **kw):
+    """CSA decode: MQA over idx [B][k] + window + sink -> bf16 [B][H][512] (and lse)."""
+    return _attn("csa_sparse_attn_decode", True, q, pos, n_entries, kv, kv_scale, swa, sink,
+                 idx, **kw)
+
+
+def hca_attn_decode(q, pos, n_entries, kv, kv_scale, swa, sink, **kw):
+    """HCA decode: MQA over all n_entries[b] entries + window + sink."""
+    return _attn("hca_attn_decode", False, q, pos, n_entries, kv, kv_scale, swa, sink, None,
+                 **kw)

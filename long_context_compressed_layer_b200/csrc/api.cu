@@ -1,0 +1,179 @@
+// extern "C" entry points of the CSA/HCA layer library: argument checks on the host, TMA
+// tensor maps, workspace carving and kernel launches. Nothing here allocates, frees or
+// synchronises; every failure is a status code.
+#include <cstring>
+
+#include "common.cuh"
+
+namespace csa {
+cudaError_t launch_compress(const csa_compress_args& a, cudaStream_t stream);
+cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
+                                const CUtensorMap& kmap, cudaStream_t stream);
+size_t ix_workspace_size(int B, int64_t Nmax, int k);
+size_t at_workspace_size(int B, int H, int rows_max);
+cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* workspace,
+                        const CUtensorMap& qmap, cudaStream_t stream);
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA; }
+
+}  // namespace
+}  // namespace csa
+
+using namespace csa;
+
+extern "C" {
+
+const char* csa_status_string(int status) {
+  switch (status) {
+    case CSA_OK: return "ok";
+    case CSA_ERR_INVALID_ARG: return "invalid argument";
+    case CSA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case CSA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case CSA_ERR_CUDA: return "CUDA launch or driver error";
+    case CSA_ERR_DEVICE: return "a kernel found invalid data (rows skipped)";
+    case CSA_ERR_TIMEOUT: return "a bounded device wait gave up";
+    default: return "unknown status";
+  }
+}
+
+int csa_compress(const csa_compress_args* a, csa_stream_t stream) {
+  if (!a) return CSA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->T < 0 || a->m < 1 || a->m > 128 || a->pos0 < 0 || a->pos0 % a->m ||
+      a->Nmax < 0 || (a->overlap != 0 && a->overlap != 1) || !(a->eps >= 0.f) ||
+      !(a->rope_base > 0.f))
+    return CSA_ERR_INVALID_ARG;
+  if (a->B > 65535) return CSA_ERR_UNSUPPORTED;
+  const int N = a->T / a->m;
+  if (a->pos0 / a->m + N > a->Nmax) return CSA_ERR_INVALID_ARG;
+  if (a->B == 0 || N == 0) return CSA_OK;
+  if (!ok_ptr(a->a) || !ok_ptr(a->za) || !ok_ptr(a->bias) || !ok_ptr(a->kv) ||
+      !ok_ptr(a->kv_scale) || !ok_opt(a->norm_w) || !ok_opt(a->dbg))
+    return CSA_ERR_INVALID_ARG;
+  if (a->overlap) {
+    if (!ok_ptr(a->b) || !ok_ptr(a->zb)) return CSA_ERR_INVALID_ARG;
+    if (a->pos0 > 0 && (!ok_ptr(a->prev_b) || !ok_ptr(a->prev_zb))) return CSA_ERR_INVALID_ARG;
+  }
+  return cuda_status(launch_compress(*a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t csa_indexer_topk_workspace_size(int32_t B, int64_t Nmax, int32_t k) {
+  if (B < 0 || Nmax < 0 || k < 1) return 0;
+  return ix_workspace_size(B, Nmax, k);
+}
+
+int csa_indexer_topk(const csa_topk_args* a, void* ws, size_t ws_bytes, csa_stream_t stream) {
+  if (!a) return CSA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->k < 1 || a->Nmax < 0 || a->Nmax % 128 != 0) return CSA_ERR_INVALID_ARG;
+  if (a->H_I != 16 && a->H_I != 32 && a->H_I != 64) return CSA_ERR_UNSUPPORTED;
+  if (a->k > 2048 || a->B > 1024 || a->Nmax > ((int64_t)1 << 30)) return CSA_ERR_UNSUPPORTED;
+  if (a->B == 0) return CSA_OK;
+  if (!ok_ptr(a->n_entries) || !ok_ptr(a->q_fp4) || !ok_ptr(a->q_sf) || !ok_ptr(a->w) ||
+      !ok_ptr(a->k_fp4) || !ok_ptr(a->k_sf) || !ok_ptr(a->idx) || !ok_opt(a->scores) ||
+      (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)))
+    return CSA_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255) ||
+      ws_bytes < ix_workspace_size(a->B, a->Nmax, a->k))
+    return CSA_ERR_WORKSPACE;
+  const int sms = num_sms();
+  EncodeTiledFn enc = encode_fn();
+  if (sms <= 0 || !enc) return CSA_ERR_CUDA;
+  if (a->Nmax == 0) {
+    // no entry can be eligible: the select pass alone writes the -1 padding
+  }
+  CUtensorMap kmap;
+  std::memset(&kmap, 0, sizeof(kmap));
+  if (a->Nmax > 0) {
+    const cuuint64_t dims[3] = {64, (cuuint64_t)a->Nmax, (cuuint64_t)a->B};
+    const cuuint64_t strides[2] = {64, (cuuint64_t)a->Nmax * 64};
+    const cuuint32_t box[3] = {64, 128, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(a->k_fp4), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return CSA_ERR_CUDA;
+  }
+  return cuda_status(
+      launch_indexer_topk(*a, ws, sms, kmap, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t csa_attn_workspace_size(int32_t B, int32_t H, int32_t rows_max) {
+  if (B < 0 || H < 1 || rows_max < 0) return 0;
+  return at_workspace_size(B, H, rows_max);
+}
+
+static int attn_common(const csa_attn_args* a, int sparse, void* ws, size_t ws_bytes,
+                       csa_stream_t stream) {
+  if (!a) return CSA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->Nmax < 0 || (sparse && a->k < 1) || !(a->tau >= 0.f) ||
+      !(a->rope_base > 0.f) || (a->derotate != 0 && a->derotate != 1))
+    return CSA_ERR_INVALID_ARG;
+  if (a->H != 64 && a->H != 128) return CSA_ERR_UNSUPPORTED;
+  if ((sparse && a->k > 2048) || a->B > 65535 || a->Nmax > ((int64_t)1 << 30))
+    return CSA_ERR_UNSUPPORTED;
+  if (a->B == 0) return CSA_OK;
+  if (!ok_ptr(a->q) || !ok_ptr(a->pos) || !ok_ptr(a->n_entries) || !ok_ptr(a->kv) ||
+      !ok_ptr(a->kv_scale) || !ok_ptr(a->swa) || !ok_ptr(a->sink) || !ok_ptr(a->out) ||
+      !ok_opt(a->lse) || (sparse && !ok_ptr(a->idx)) ||
+      (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)))
+    return CSA_ERR_INVALID_ARG;
+  const int64_t rows_max64 = (sparse ? (int64_t)a->k : a->Nmax) + CSA_WINDOW;
+  const int rows_max = (int)rows_max64;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255) ||
+      ws_bytes < at_workspace_size(a->B, a->H, rows_max))
+    return CSA_ERR_WORKSPACE;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return CSA_ERR_CUDA;
+  CUtensorMap qmap;
+  const cuuint64_t dims[2] = {CSA_HEAD_DIM, (cuuint64_t)a->B * a->H};
+  const cuuint64_t strides[1] = {CSA_HEAD_DIM * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)a->H};
+  const cuuint32_t estr[2] = {1, 1};
+  if (enc(&qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a->q), dims, strides,
+          box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return CSA_ERR_CUDA;
+  return cuda_status(
+      launch_attn(*a, sparse, rows_max, ws, qmap, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csa_sparse_attn_decode(const csa_attn_args* a, void* ws, size_t ws_bytes,
+                           csa_stream_t stream) {
+  return attn_common(a, 1, ws, ws_bytes, stream);
+}
+
+int hca_attn_decode(const csa_attn_args* a, void* ws, size_t ws_bytes, csa_stream_t stream) {
+  return attn_common(a, 0, ws, ws_bytes, stream);
+}
+
+}  // extern "C"

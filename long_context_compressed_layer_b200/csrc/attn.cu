@@ -1,0 +1,393 @@
+// Shared-KV MQA decode over compressed entries plus the sliding window, with the sink
+// logit in the softmax denominator ("DeepSeek-V4：百万上下文的工程答案", Hybrid Attention:
+// shared key-value MQA, Attention sink; cyqw.cn DeepSeek-V4 walkthrough §2.2: the 128
+// most recent uncompressed tokens join the core attention; Partial RoPE: the output is
+// de-rotated by the query position).
+//
+// The rows a query attends to form one list: the selected entries (CSA) or all eligible
+// entries (HCA), then the 128 window tokens t-127 .. t. The list is cut into chunks of
+// 64 rows. attn_chunk_kernel handles one (sequence, chunk):
+//   - Q [H heads x 512] arrives by TMA (128-byte swizzle, K-major), padded to 128 rows;
+//   - the 64 rows are gathered and dequantised to BF16 in shared memory (E4M3 code x entry
+//     scale, BF16 RoPE dims, BF16 window rows), in the same swizzled layout, which serves
+//     as K-major B for S = Q V^T and as MN-major B for O = P V;
+//   - tcgen05.mma kind::f16 computes S[128 x 64] in TMEM; one thread per head turns its row
+//     into exp(tau*S - m) (fp32), keeps m and l = sum, and writes P as BF16 (K-major A);
+//   - two tcgen05.mma N = 256 halves compute O[128 x 512] in TMEM (S's columns are reused);
+//   - O, m and l go to the workspace.
+// attn_combine_kernel merges the chunks of a sequence in fixed order with the sink,
+// normalises, de-rotates the last 64 dims and stores BF16 (and lse). The chunk count
+// depends only on k (CSA) or n (HCA), never on the batch, so results are batch-invariant.
+#include "common.cuh"
+
+namespace csa {
+
+constexpr int kAtRows = 64;  // rows per chunk = N of the S MMA
+constexpr int kAtThreads = 128;
+
+struct AtSmem {
+  uint8_t q[8][128 * 128];      // 8 K-blocks of [128 heads x 64 dims] bf16, 128-B swizzle
+  uint8_t v[8][kAtRows * 128];  // 8 dim-blocks of [64 rows x 64 dims] bf16, 128-B swizzle
+  uint8_t pm[128 * 128];        // P [128 heads x 64 rows] bf16, 128-B swizzle
+  const uint8_t* src[kAtRows];  // row source
+  float rscale[kAtRows];        // entry scale, 0 for window rows
+  int kind[kAtRows];            // 0 invalid, 1 entry, 2 window row
+  uint64_t q_full, s_done, o_done;
+  uint32_t tmem_base;
+};
+
+struct AtParams {
+  int B, H, k, sparse, C;  // C = chunks per sequence in the workspace
+  int64_t Nmax;
+  const int32_t* pos;
+  const int32_t* idx;
+  const int32_t* n_entries;
+  const uint8_t* kv;
+  const float* kv_scale;
+  const uint16_t* swa;
+  const float* sink;
+  float tau, rope_base;
+  int derotate;
+  uint16_t* out;
+  float* lse;
+  float* part_o;   // [B][C][H][512]
+  float2* part_ml; // [B][C][H]
+  int32_t* dev_status;
+};
+
+__device__ __forceinline__ int at_rows_total(const AtParams& p, int n) {
+  return (p.sparse ? p.k : n) + kWin;
+}
+
+__global__ void __launch_bounds__(kAtThreads, 1)
+    attn_chunk_kernel(const __grid_constant__ CUtensorMap qmap, AtParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  AtSmem& s = *reinterpret_cast<AtSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int c = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  const int warp = tid >> 5;
+  int n = p.n_entries[b];
+  if (n < 0 || n > p.Nmax) {
+    if (tid == 0) report(p.dev_status, CSA_ERR_DEVICE);
+    n = n < 0 ? 0 : (int)p.Nmax;
+  }
+  const int rows_total = at_rows_total(p, n);
+  const int row0 = c * kAtRows;
+  if (row0 >= rows_total) return;  // uniform: this chunk does not exist for this sequence
+  const int t = p.pos[b];
+  if (t < 0 && tid == 0) report(p.dev_status, CSA_ERR_DEVICE);
+  const int nwin_first = p.sparse ? p.k : n;  // list index of the first window row
+
+  if (tid == 0) {
+    mbar_init(&s.q_full, 1);
+    mbar_init(&s.s_done, 1);
+    mbar_init(&s.o_done, 1);
+    mbar_fence_init();
+  }
+  if (warp == 0) tmem_alloc(&s.tmem_base, 512);
+  // Q rows H..127 are zero padding (generic-proxy writes, fenced below)
+  if (p.H < 128) {
+    for (int i = tid; i < 8 * (128 - p.H) * 8; i += kAtThreads) {
+      const int blk = i / ((128 - p.H) * 8), rem = i % ((128 - p.H) * 8);
+      *reinterpret_cast<uint4*>(&s.q[blk][p.H * 128 + rem * 16]) = make_uint4(0, 0, 0, 0);
+    }
+  }
+  // row sources
+  if (tid < kAtRows) {
+    const int r = row0 + tid;
+    int kind = 0;
+    const uint8_t* src = nullptr;
+    float scl = 0.f;
+    if (r < nwin_first) {
+      const int j = p.sparse ? p.idx[(size_t)b * p.k + r] : r;
+      if (j >= 0 && j < n) {
+        kind = 1;
+        src = p.kv + ((size_t)b * p.Nmax + j) * kRow;
+        scl = p.kv_scale[(size_t)b * p.Nmax + j];
+      } else if (j != -1) {
+        report(p.dev_status, CSA_ERR_DEVICE);
+      }
+    } else if (r < rows_total) {
+      const int pp = t - (kWin - 1) + (r - nwin_first);
+      if (pp >= 0) {
+        kind = 2;
+        src = reinterpret_cast<const uint8_t*>(p.swa + ((size_t)b * kWin + (pp % kWin)) * kD);
+      }
+    }
+    s.kind[tid] = kind;
+    s.src[tid] = src;
+    s.rscale[tid] = scl;
+  }
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  if (tid == 0) {
+    prefetch_tensormap(&qmap);
+    mbar_arrive_expect_tx(&s.q_full, (uint32_t)p.H * kD * 2);
+    for (int blk = 0; blk < 8; ++blk) tma_load_2d(s.q[blk], &qmap, &s.q_full, blk * 64, b * p.H);
+  }
+  // gather + dequantise: 64 rows x 64 chunks of 8 dims; chunk ch of row r lands in dim-block
+  // ch/8 at 16-byte slot (ch%8) ^ (r%8) of the row's 128 bytes
+  for (int task = tid; task < kAtRows * 64; task += kAtThreads) {
+    const int r = task >> 6, ch = task & 63;
+    const int d = ch * 8;
+    uint4 o = make_uint4(0, 0, 0, 0);
+    const int kind = s.kind[r];
+    if (kind == 1) {
+      const uint8_t* src = s.src[r];
+      if (d < kNope) {
+        const uint2 raw = *reinterpret_cast<const uint2*>(src + d);
+        const float scl = s.rscale[r];
+        uint32_t w[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t pair = (e < 2 ? raw.x : raw.y) >> (16 * (e & 1));
+          const float lo = e4m3_to_f32((uint8_t)(pair & 0xFF)) * scl;
+          const float hi = e4m3_to_f32((uint8_t)((pair >> 8) & 0xFF)) * scl;
+          w[e] = (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
+        }
+        o = make_uint4(w[0], w[1], w[2], w[3]);
+      } else {
+        o = *reinterpret_cast<const uint4*>(src + kNope + 2 * (d - kNope));
+      }
+    } else if (kind == 2) {
+      o = *reinterpret_cast<const uint4*>(s.src[r] + 2 * d);
+    }
+    *reinterpret_cast<uint4*>(&s.v[ch >> 3][r * 128 + (((ch & 7) ^ (r & 7)) << 4)]) = o;
+  }
+  fence_async_smem();
+  __syncthreads();
+
+  // S = Q V^T : M = 128 heads, N = 64 rows, K = 512 (32 steps of 16)
+  const uint32_t t_o = tmem, t_s = tmem + 256;
+  bool ok = true;
+  if (tid == 0) {
+    ok = mbar_wait(&s.q_full, 0, p.dev_status);
+    if (ok) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, kAtRows, false);
+      for (int kk = 0; kk < 32; ++kk) {
+        const uint32_t off = (kk & 3) * 32;
+        mma_bf16(t_s, smem_desc(smem_u32(s.q[kk >> 2]) + off, 16, 1024, kSwizzle128B),
+                 smem_desc(smem_u32(s.v[kk >> 2]) + off, 16, 1024, kSwizzle128B), id, kk > 0);
+      }
+    }
+    mma_commit(&s.s_done);
+  }
+  {
+    const bool waited = mbar_wait(&s.s_done, 0, p.dev_status);
+    ok = __syncthreads_and(ok && waited) != 0;
+  }
+  tc_fence_after();
+
+  // softmax rows: thread tid owns head tid (TMEM lane tid)
+  const int h = tid;
+  float m_c = -INFINITY, l_c = 0.f;
+  {
+    uint32_t r0[32], r1[32];
+    const uint32_t ta = t_s + ((uint32_t)(warp * 32) << 16);
+    tmem_ld32(ta, r0);
+    tmem_ld32(ta + 32, r1);
+    tmem_ld_wait();
+    float lg[64];
+#pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      lg[r] = s.kind[r] ? __uint_as_float(r0[r]) * p.tau : -INFINITY;
+      lg[32 + r] = s.kind[32 + r] ? __uint_as_float(r1[r]) * p.tau : -INFINITY;
+    }
+#pragma unroll
+    for (int r = 0; r < 64; ++r) m_c = fmaxf(m_c, lg[r]);
+    uint8_t* prow = s.pm + h * 128;
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int r = ch * 8 + 2 * e;
+        const float p0 = m_c == -INFINITY ? 0.f : expf(lg[r] - m_c);
+        const float p1 = m_c == -INFINITY ? 0.f : expf(lg[r + 1] - m_c);
+        l_c += p0;
+        l_c += p1;
+        w[e] = (uint32_t)f32_to_bf16_bits(p0) | ((uint32_t)f32_to_bf16_bits(p1) << 16);
+      }
+      *reinterpret_cast<uint4*>(prow + ((ch ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+
+  // O = P V : M = 128, N = 256 per half, K = 64 rows (4 steps of 16); V read MN-major
+  if (tid == 0) {
+    if (ok) {
+      tc_fence_after();
+      const uint32_t id = idesc_bf16(128, 256, true);
+      for (int half = 0; half < 2; ++half) {
+        for (int kk = 0; kk < 4; ++kk) {
+          mma_bf16(t_o + half * 256, smem_desc(smem_u32(s.pm) + kk * 32, 16, 1024, kSwizzle128B),
+                   smem_desc(smem_u32(s.v[half * 4]) + kk * 2048, kAtRows * 128, 1024, kSwizzle128B),
+                   id, kk > 0);
+        }
+      }
+    }
+    mma_commit(&s.o_done);
+  }
+  ok = mbar_wait(&s.o_done, 0, p.dev_status) && ok;
+  tc_fence_after();
+  if (h < p.H) {
+    const size_t slot = ((size_t)b * p.C + c) * p.H + h;
+    float* dst = p.part_o + slot * kD;
+    for (int cc = 0; cc < 16; ++cc) {
+      uint32_t r[32];
+      tmem_ld32(t_o + ((uint32_t)(warp * 32) << 16) + cc * 32, r);
+      tmem_ld_wait();
+#pragma unroll
+      for (int e = 0; e < 32; e += 4)
+        *reinterpret_cast<float4*>(dst + cc * 32 + e) =
+            make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
+                        __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
+    }
+    p.part_ml[slot] = ok ? make_float2(m_c, l_c) : make_float2(-INFINITY, 0.f);
+  } else {
+    // keep the warp's tcgen05.ld calls uniform
+    for (int cc = 0; cc < 16; ++cc) {
+      uint32_t r[32];
+      tmem_ld32(t_o + ((uint32_t)(warp * 32) << 16) + cc * 32, r);
+      tmem_ld_wait();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// One CTA per (sequence, head): 128 threads x 4 dims.
+__global__ void __launch_bounds__(128) attn_combine_kernel(AtParams p) {
+  const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  __shared__ float rot[32][2];
+  __shared__ float wgt[64];
+  __shared__ float sh_M, sh_Z;
+  int n = p.n_entries[b];
+  n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
+  const int C_b = (at_rows_total(p, n) + kAtRows - 1) / kAtRows;
+  const int t = p.pos[b];
+  if (tid < 32 && p.derotate) {
+    float cs, sn;
+    rope_cos_sin((double)t, tid, (double)p.rope_base, &cs, &sn);
+    rot[tid][0] = cs;
+    rot[tid][1] = sn;
+  }
+  const float sink = p.sink[h];
+  if (tid == 0) {
+    float M = sink;
+    for (int c = 0; c < C_b; ++c) M = fmaxf(M, p.part_ml[((size_t)b * p.C + c) * p.H + h].x);
+    float Z = 0.f;
+    if (M == INFINITY) {
+      Z = INFINITY;
+    } else {
+      Z = sink == -INFINITY ? 0.f : expf(sink - M);
+      for (int c = 0; c < C_b; ++c) {
+        const float2 ml = p.part_ml[((size_t)b * p.C + c) * p.H + h];
+        const float w = ml.x == -INFINITY ? 0.f : expf(ml.x - M);
+        Z += w * ml.y;
+      }
+    }
+    sh_M = M;
+    sh_Z = Z;
+    if (p.lse) p.lse[(size_t)b * p.H + h] = M == INFINITY ? INFINITY : M + logf(Z);
+  }
+  __syncthreads();
+  const float M = sh_M, Z = sh_Z;
+  if (tid < C_b && tid < 64) {
+    const float mx = p.part_ml[((size_t)b * p.C + tid) * p.H + h].x;
+    wgt[tid] = (M == INFINITY || mx == -INFINITY) ? 0.f : expf(mx - M) / Z;
+  }
+  __syncthreads();
+  const int d0 = 4 * tid;
+  float o[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int c = 0; c < C_b; ++c) {
+    float w;
+    if (c < 64) {
+      w = wgt[c];
+    } else {
+      const float mx = p.part_ml[((size_t)b * p.C + c) * p.H + h].x;
+      w = (M == INFINITY || mx == -INFINITY) ? 0.f : expf(mx - M) / Z;
+    }
+    if (w == 0.f) continue;
+    const float4 v = *reinterpret_cast<const float4*>(
+        p.part_o + (((size_t)b * p.C + c) * p.H + h) * kD + d0);
+    o[0] = fmaf(w, v.x, o[0]);
+    o[1] = fmaf(w, v.y, o[1]);
+    o[2] = fmaf(w, v.z, o[2]);
+    o[3] = fmaf(w, v.w, o[3]);
+  }
+  if (p.derotate && d0 >= kNope) {
+#pragma unroll
+    for (int e = 0; e < 4; e += 2) {
+      const int j = (d0 + e - kNope) >> 1;
+      const float cs = rot[j][0], sn = rot[j][1];
+      const float x0 = o[e], x1 = o[e + 1];
+      o[e] = x0 * cs + x1 * sn;
+      o[e + 1] = -x0 * sn + x1 * cs;
+    }
+  }
+  uint2 packed;
+  packed.x = (uint32_t)f32_to_bf16_bits(o[0]) | ((uint32_t)f32_to_bf16_bits(o[1]) << 16);
+  packed.y = (uint32_t)f32_to_bf16_bits(o[2]) | ((uint32_t)f32_to_bf16_bits(o[3]) << 16);
+  *reinterpret_cast<uint2*>(p.out + ((size_t)b * p.H + h) * kD + d0) = packed;
+}
+
+size_t at_smem_bytes() { return sizeof(AtSmem) + 1024; }
+
+size_t at_workspace_size(int B, int H, int rows_max) {
+  const size_t C = (size_t)(rows_max + kAtRows - 1) / kAtRows;
+  const size_t o = (size_t)B * C * H * kD * sizeof(float);
+  return ((o + 255) & ~(size_t)255) + (size_t)B * C * H * sizeof(float2);
+}
+
+cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* workspace,
+                        const CUtensorMap& qmap, cudaStream_t stream) {
+  AtParams p;
+  p.B = a.B;
+  p.H = a.H;
+  p.k = sparse ? a.k : 0;
+  p.sparse = sparse;
+  p.C = (rows_max + kAtRows - 1) / kAtRows;
+  p.Nmax = a.Nmax;
+  p.pos = a.pos;
+  p.idx = a.idx;
+  p.n_entries = a.n_entries;
+  p.kv = a.kv;
+  p.kv_scale = a.kv_scale;
+  p.swa = a.swa;
+  p.sink = a.sink;
+  p.tau = a.tau > 0.f ? a.tau : 0.044194173824159216f;  // 1/sqrt(512)
+  p.rope_base = a.rope_base;
+  p.derotate = a.derotate;
+  p.out = a.out;
+  p.lse = a.lse;
+  const size_t o = (size_t)a.B * p.C * a.H * kD * sizeof(float);
+  p.part_o = reinterpret_cast<float*>(workspace);
+  p.part_ml = reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + ((o + 255) & ~(size_t)255));
+  p.dev_status = a.dev_status;
+  const size_t smem = at_smem_bytes();
+  static int configured = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured != dev) {
+    cudaError_t e = cudaFuncSetAttribute(attn_chunk_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = dev;
+  }
+  attn_chunk_kernel<<<dim3(p.C, a.B), kAtThreads, smem, stream>>>(qmap, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  attn_combine_kernel<<<dim3(a.H, a.B), 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace csa

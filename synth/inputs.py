@@ -76,10 +76,10 @@ _E4M3_EXP_P /= _E4M3_EXP_P.sum()
 
 def e4m3_codes(rng: np.random.Generator, shape) -> np.ndarray:
     n = int(np.prod(shape))
-    e = rng.choice(16, size=n, p=_E4M3_EXP_P).astype(np.uint8)
-    mant = rng.integers(0, 8, size=n, dtype=np.uint8)
+    e = _lut_sample(rng, n, _E4M3_EXP_P)
+    low = rng.integers(0, 16, size=n, dtype=np.uint8)  # 3 mantissa bits + sign bit
+    mant, sign = low & 7, low >> 3
     mant = np.where((e == 15) & (mant == 7), np.uint8(6), mant)
-    sign = rng.integers(0, 2, size=n, dtype=np.uint8)
     return ((sign << 7) | (e << 3) | mant).astype(np.uint8).reshape(shape)
 
 

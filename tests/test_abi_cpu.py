@@ -1,0 +1,131 @@
+"""The C-ABI library: it builds, loads without a GPU, exports every symbol the headers
+declare, and rejects bad arguments on the host before touching the device."""
+
+import ctypes as C
+import glob
+import os
+import re
+
+import pytest
+
+import long_context_compressed_layer_b200 as csa
+from long_context_compressed_layer_b200 import build as csa_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    csa_build.build()
+    return csa.lib()
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(\w+)\s*\([^;{]*\)\s*;",
+                            text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert "csa_indexer_topk" in names and "hca_attn_decode" in names
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(csa.EXPORTS) <= set(names)
+
+
+def test_status_strings(L):
+    for code in range(7):
+        assert L.csa_status_string(code)
+    assert b"unknown" in L.csa_status_string(99)
+
+
+def test_workspace_sizes_are_host_only(L):
+    a = L.csa_indexer_topk_workspace_size(4, 262144, 1024)
+    assert a >= 4 * 262144 * (4 + 8) + 4 * 4096 * 4
+    assert L.csa_indexer_topk_workspace_size(-1, 128, 4) == 0
+    b = L.csa_attn_workspace_size(4, 128, 1024 + 128)
+    assert b >= 4 * 18 * 128 * 512 * 4
+    assert L.csa_attn_workspace_size(1, 0, 10) == 0
+
+
+FAKE = 1 << 20  # a 256-aligned non-null address: never dereferenced on a rejected call
+
+
+def _topk_args(**over):
+    a = csa.TopkArgs(2, 64, 512, 1024, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None)
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_indexer_rejects_on_host(L):
+    ws_ok = L.csa_indexer_topk_workspace_size(2, 1024, 512)
+    call = lambda a, ws=FAKE, n=ws_ok: L.csa_indexer_topk(C.byref(a), ws, n, None)
+    assert L.csa_indexer_topk(None, FAKE, ws_ok, None) == csa.CSA_ERR_INVALID_ARG
+    assert call(_topk_args(Nmax=1000)) == csa.CSA_ERR_INVALID_ARG  # not a multiple of 128
+    assert call(_topk_args(k=0)) == csa.CSA_ERR_INVALID_ARG
+    assert call(_topk_args(H_I=8)) == csa.CSA_ERR_UNSUPPORTED
+    assert call(_topk_args(k=4096)) == csa.CSA_ERR_UNSUPPORTED
+    assert call(_topk_args(q_fp4=FAKE + 8)) == csa.CSA_ERR_INVALID_ARG  # misaligned
+    assert call(_topk_args(w=None)) == csa.CSA_ERR_INVALID_ARG
+    assert call(_topk_args(), ws=None) == csa.CSA_ERR_WORKSPACE
+    assert call(_topk_args(), ws=FAKE + 16) == csa.CSA_ERR_WORKSPACE
+    assert call(_topk_args(), n=ws_ok - 1) == csa.CSA_ERR_WORKSPACE
+    assert call(_topk_args(B=0)) == csa.CSA_OK  # nothing to do
+
+
+def _attn_args(**over):
+    a = csa.AttnArgs(2, 128, 1024, 4096, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 0.0,
+                     10000.0, 1, FAKE, None, None)
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_attention_rejects_on_host(L):
+    ws_ok = L.csa_attn_workspace_size(2, 128, 1024 + 128)
+    f = lambda a, ws=FAKE, n=ws_ok: L.csa_sparse_attn_decode(C.byref(a), ws, n, None)
+    assert f(_attn_args(H=96)) == csa.CSA_ERR_UNSUPPORTED
+    assert f(_attn_args(k=0)) == csa.CSA_ERR_INVALID_ARG
+    assert f(_attn_args(derotate=2)) == csa.CSA_ERR_INVALID_ARG
+    assert f(_attn_args(idx=None)) == csa.CSA_ERR_INVALID_ARG
+    assert f(_attn_args(out=FAKE + 4)) == csa.CSA_ERR_INVALID_ARG
+    assert f(_attn_args(), n=ws_ok - 1) == csa.CSA_ERR_WORKSPACE
+    # HCA sizes its workspace from Nmax, not k
+    hca_ws = L.csa_attn_workspace_size(2, 128, 4096 + 128)
+    assert L.hca_attn_decode(C.byref(_attn_args(idx=None)), FAKE, ws_ok, None) == \
+        csa.CSA_ERR_WORKSPACE
+    assert hca_ws > ws_ok
+
+
+def test_compress_rejects_on_host(L):
+    def args(**over):
+        a = csa.CompressArgs(1, 64, 4, 1, 0, 10000.0, 1e-6, FAKE, FAKE, FAKE, FAKE, FAKE, None,
+                             None, None, FAKE, FAKE, 16, None)
+        for k, v in over.items():
+            setattr(a, k, v)
+        return a
+
+    f = lambda a: L.csa_compress(C.byref(a), None)
+    assert f(args(m=0)) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(m=129)) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(pos0=6)) == csa.CSA_ERR_INVALID_ARG  # not a block boundary
+    assert f(args(pos0=8)) == csa.CSA_ERR_INVALID_ARG  # needs prev_b/prev_zb
+    assert f(args(Nmax=15)) == csa.CSA_ERR_INVALID_ARG  # 16 entries do not fit
+    assert f(args(b=None)) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(overlap=2)) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(T=3)) == csa.CSA_OK  # no complete block: nothing to do
+
+
+def test_cuda_sources_are_sm100a_only():
+    src = open(os.path.join(ROOT, "long_context_compressed_layer_b200", "build.py")).read()
+    assert "arch=compute_100a,code=sm_100a" in src
+    for f in glob.glob(os.path.join(ROOT, "long_context_compressed_layer_b200", "csrc", "*")):
+        text = open(f).read()
+        assert "multicast" not in text  # no TMA multicast anywhere
+        assert "wgmma" not in text and "mma.sync" not in text

@@ -1,0 +1,275 @@
+"""CUDA path vs the fp64 oracle, element by element, on seeded inputs (needs a B200)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import inputs as synth
+from tests import compare
+
+pytestmark = pytest.mark.gpu
+
+csa = pytest.importorskip("long_context_compressed_layer_b200")
+
+
+def dev(x):
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.uint16:
+        x = x.view(np.int16)
+    return torch.from_numpy(x).cuda()
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    csa.lib()
+    torch.cuda.init()
+
+
+# ------------------------------------------------------------------ compress
+def _run_compress(inp, m, overlap, pos0=0, Nmax=None):
+    B, T, _ = inp["a"].shape
+    N = T // m
+    Nmax = Nmax or pos0 // m + N
+    kv, sc, dbg = csa.compress(dev(inp["a"]), dev(inp["za"]), dev(inp["bias"]), m, overlap,
+                               b=dev(inp["b"]) if overlap else None,
+                               zb=dev(inp["zb"]) if overlap else None, pos0=pos0,
+                               prev_b=dev(inp["prev_b"]) if "prev_b" in inp else None,
+                               prev_zb=dev(inp["prev_zb"]) if "prev_zb" in inp else None,
+                               Nmax=Nmax, dbg=True)
+    torch.cuda.synchronize()
+    n0 = pos0 // m
+    return host(kv)[:, n0:n0 + N], host(sc)[:, n0:n0 + N], host(dbg)
+
+
+@pytest.mark.parametrize("B,T,m,overlap,pos0", [
+    (2, 4 * 37 + 3, 4, True, 0),      # CSA, ragged tail (3 tokens stay in state)
+    (1, 4 * 64, 4, True, 4096),       # CSA chunk after a prefix: previous block from state
+    (3, 128 * 3, 128, False, 0),      # HCA
+    (1, 128 * 2, 128, False, 1 << 20),  # HCA at 1M positions (RoPE angle range)
+    (1, 24, 1, True, 0),              # m = 1
+])
+def test_compress_matches_oracle(B, T, m, overlap, pos0):
+    inp = synth.compress_inputs(B, T, m, overlap, seed=100 + m + B, pos0=pos0)
+    kv, sc, dbg = _run_compress(inp, m, overlap, pos0, Nmax=pos0 // m + T // m + 5)
+    ora = oracle.compress(inp["a"], inp["za"], inp["bias"], m, overlap, b=inp.get("b"),
+                          zb=inp.get("zb"), pos0=pos0, prev_b=inp.get("prev_b"),
+                          prev_zb=inp.get("prev_zb"))
+    flips = compare.compare_entries(kv, sc, dbg, ora, what=f"compress m={m}")
+    assert flips <= max(4, kv.size // 5000)
+
+
+def test_compress_workload0_full():
+    # the 8192-token CSA stream of the tiny decode workload -> 2048 entries
+    inp = synth.compress_inputs(1, 8192, 4, True, seed=0)
+    kv, sc, dbg = _run_compress(inp, 4, True)
+    ora = oracle.compress(inp["a"], inp["za"], inp["bias"], 4, True, b=inp["b"], zb=inp["zb"])
+    flips = compare.compare_entries(kv, sc, dbg, ora, what="workload 0 compress")
+    assert flips <= kv.size // 5000
+
+
+# ------------------------------------------------------------- indexer top-k
+def _topk_case(B, H_I, Nmax, n, k, planted=0, seed=0):
+    rng = np.random.default_rng(seed)
+    n = np.asarray(n, dtype=np.int32)
+    ix = synth.indexer_inputs(rng, B, H_I, Nmax, n, planted)
+    idx, sc = csa.indexer_topk(dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]),
+                               dev(ix["k_fp4"]), dev(ix["k_sf"]), k, scores=True)
+    torch.cuda.synchronize()
+    ora = oracle.indexer_scores(n, ix["q_fp4"], ix["q_sf"], ix["w"], ix["k_fp4"], ix["k_sf"])
+    return host(idx), host(sc), ora, n
+
+
+@pytest.mark.parametrize("B,H_I,Nmax,n,k,planted", [
+    (1, 16, 2048, [2048], 512, 0),              # workload 0 shape
+    (3, 64, 4096, [4096, 2999, 130], 512, 0),   # ragged lengths, n < k in one sequence
+    (2, 32, 1024, [1000, 0], 64, 2),            # an empty sequence
+    (2, 64, 16384, [16384, 12345], 1024, 8),    # planted runs, several CTAs per sequence
+    (1, 64, 256, [1], 1, 0),                    # one entry
+])
+def test_indexer_topk_matches_oracle(B, H_I, Nmax, n, k, planted):
+    idx, sc, ora, n = _topk_case(B, H_I, Nmax, n, k, planted, seed=B * 7 + k)
+    total = 0
+    for b in range(B):
+        total += compare.compare_topk(idx[b], ora[b], int(n[b]), k, what=f"seq {b}")
+        sel = idx[b][idx[b] >= 0]
+        np.testing.assert_allclose(sc[b][: len(sel)], ora[b][sel], rtol=2e-5, atol=1e-6)
+    assert total <= 2
+
+
+def test_indexer_scores_exact_on_integer_case():
+    # unit scales, w = 1: every score is a multiple of 1/4 below 2^24, exact in fp32
+    B, H_I, Nmax, k = 1, 64, 1024, 1024
+    rng = np.random.default_rng(3)
+    n = np.array([1000], np.int32)
+    ix = synth.indexer_inputs(rng, B, H_I, Nmax, n)
+    ix["q_sf"][:] = 127
+    ix["k_sf"][:] = 127
+    ix["w"][:] = 1.0
+    idx, sc = csa.indexer_topk(dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]),
+                               dev(ix["k_fp4"]), dev(ix["k_sf"]), k, scores=True)
+    ora = oracle.indexer_scores(n, ix["q_fp4"], ix["q_sf"], ix["w"], ix["k_fp4"], ix["k_sf"])
+    idx, sc = host(idx)[0], host(sc)[0]
+    assert (idx[:1000] == np.arange(1000)).all() and (idx[1000:] == -1).all()
+    np.testing.assert_array_equal(sc[:1000], ora[0, :1000])
+
+
+def test_indexer_workspace_stays_clean_across_calls():
+    B, H_I, Nmax, k = 2, 64, 2048, 256
+    rng = np.random.default_rng(4)
+    n = np.array([2048, 1500], np.int32)
+    ix = synth.indexer_inputs(rng, B, H_I, Nmax, n, 3)
+    args = [dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]), dev(ix["k_fp4"]),
+            dev(ix["k_sf"]), k]
+    ws = csa.indexer_topk_workspace(B, Nmax, k)
+    first = host(csa.indexer_topk(*args, workspace=ws))
+    for _ in range(3):
+        again = host(csa.indexer_topk(*args, workspace=ws))
+        np.testing.assert_array_equal(again, first)
+
+
+# ------------------------------------------------------------------ attention
+def _attn_case(B, H, Nmax, n, pos, k=None, seed=0, sink_override=None):
+    rng = np.random.default_rng(seed)
+    n = np.asarray(n, np.int32)
+    pos = np.asarray(pos, np.int32)
+    kv, sc = synth.kv_cache(rng, B, Nmax)
+    q = synth.bf16_normal(rng, (B, H, 512))
+    swa = synth.bf16_normal(rng, (B, 128, 512))
+    sink = rng.standard_normal(H).astype(np.float32)
+    if sink_override is not None:
+        sink[:] = sink_override
+    idx = None
+    if k is not None:
+        idx = np.full((B, k), -1, np.int32)
+        for b in range(B):
+            c = min(k - 3, int(n[b]))  # leave some padding
+            idx[b, :c] = np.sort(rng.choice(int(n[b]), c, replace=False))
+    return dict(q=q, pos=pos, n=n, kv=kv, sc=sc, swa=swa, sink=sink, idx=idx)
+
+
+def _gpu_attn(d, derotate=True):
+    args = (dev(d["q"]), dev(d["pos"]), dev(d["n"]), dev(d["kv"]), dev(d["sc"]), dev(d["swa"]),
+            dev(d["sink"]))
+    if d["idx"] is not None:
+        out, lse = csa.sparse_attn_decode(*args, dev(d["idx"]), lse=True, derotate=derotate)
+    else:
+        out, lse = csa.hca_attn_decode(*args, lse=True, derotate=derotate)
+    torch.cuda.synchronize()
+    return out.float().cpu().numpy(), host(lse)
+
+
+def _ora_attn(d, derotate=True):
+    return oracle.attention(d["q"], d["pos"], d["n"], d["kv"], d["sc"], d["swa"], d["sink"],
+                            idx=d["idx"], derotate=derotate)
+
+
+@pytest.mark.parametrize("B,H,Nmax,n,pos,k", [
+    (2, 64, 2048, [2048, 1000], [8191, 4003], 512),      # CSA, workload 0/2 heads
+    (2, 128, 4096, [4096, 3000], [16383, 12001], 1024),  # CSA, workload 3 heads
+    (3, 64, 1024, [1024, 7, 0], [131071, 900, 50], None),  # HCA, ragged, early positions
+    (1, 128, 256, [200], [803], 100),                     # CSA, k not a multiple of 64
+])
+def test_attention_matches_oracle(B, H, Nmax, n, pos, k):
+    d = _attn_case(B, H, Nmax, n, pos, k, seed=H + B)
+    out, lse = _gpu_attn(d)
+    want, wlse = _ora_attn(d)
+    compare.close(out, want, what="attention out")
+    np.testing.assert_allclose(lse, wlse, rtol=1e-4, atol=1e-4)
+
+
+def test_attention_sink_limits():
+    d = _attn_case(2, 64, 512, [512, 300], [2047, 1300], 256, seed=5)
+    d["sink"][:5] = -np.inf
+    d["sink"][5:8] = np.inf
+    out, lse = _gpu_attn(d)
+    want, wlse = _ora_attn(d)
+    assert (out[:, 5:8] == 0).all() and np.isinf(lse[:, 5:8]).all()
+    compare.close(out, want, what="sink limits")
+    np.testing.assert_allclose(lse[:, :5], wlse[:, :5], rtol=1e-4)
+
+
+def test_attention_without_derotation():
+    d = _attn_case(1, 128, 1024, [1024], [4095], 512, seed=6)
+    out, _ = _gpu_attn(d, derotate=False)
+    want, _ = _ora_attn(d, derotate=False)
+    compare.close(out, want, what="no derotation")
+
+
+def test_attention_bad_index_is_reported():
+    d = _attn_case(1, 64, 512, [300], [1203], 64, seed=7)
+    d["idx"][0, 5] = 400  # beyond n_entries: skipped and reported
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    csa.sparse_attn_decode(dev(d["q"]), dev(d["pos"]), dev(d["n"]), dev(d["kv"]), dev(d["sc"]),
+                           dev(d["swa"]), dev(d["sink"]), dev(d["idx"]), dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == csa.CSA_ERR_DEVICE
+
+
+# ------------------------------------------------------- invariance, determinism
+def test_batch_invariance_and_determinism():
+    w = synth.WORKLOADS[0]
+    full = synth.decode_inputs(synth.Workload("inv", "csa", B=3, m=4, H=64, H_I=64, k=512,
+                                              L=40000, L_min=9000, seed=11))
+    B = full["B"]
+
+    def step(sl):
+        n = dev(full["n_entries"][sl])
+        idx = csa.indexer_topk(n, dev(full["q_fp4"][sl]), dev(full["q_sf"][sl]),
+                               dev(full["w"][sl]), dev(full["k_fp4"][sl]),
+                               dev(full["k_sf"][sl]), 512)
+        out = csa.sparse_attn_decode(dev(full["q"][sl]), dev(full["pos"][sl]), n,
+                                     dev(full["kv"][sl]), dev(full["kv_scale"][sl]),
+                                     dev(full["swa"][sl]), dev(full["sink"]), idx)
+        torch.cuda.synchronize()
+        return host(idx), out.view(torch.int16).cpu().numpy()
+
+    idx_all, out_all = step(slice(0, B))
+    idx_again, out_again = step(slice(0, B))
+    np.testing.assert_array_equal(idx_all, idx_again)
+    np.testing.assert_array_equal(out_all, out_again)
+    for b in range(B):
+        idx_b, out_b = step(slice(b, b + 1))
+        np.testing.assert_array_equal(idx_b[0], idx_all[b])
+        np.testing.assert_array_equal(out_b[0], out_all[b])
+
+
+# --------------------------------------------------- full decode, small workloads
+def test_workload0_decode_chain():
+    """Compress the 8192-token stream, score/select, attend: each stage vs the oracle fed
+    with the oracle's own upstream result."""
+    w = synth.WORKLOADS[0]
+    inp = synth.compress_inputs(1, w.L, w.m, True, seed=w.seed)
+    d = synth.decode_inputs(w)
+    ora_c = oracle.compress(inp["a"], inp["za"], inp["bias"], 4, True, b=inp["b"], zb=inp["zb"])
+    kv_gpu, sc_gpu, dbg = _run_compress(inp, 4, True)
+    compare.compare_entries(kv_gpu, sc_gpu, dbg, ora_c, what="workload 0")
+    n = d["n_entries"]
+    idx = host(csa.indexer_topk(dev(n), dev(d["q_fp4"]), dev(d["q_sf"]), dev(d["w"]),
+                                dev(d["k_fp4"]), dev(d["k_sf"]), w.k))
+    ora_s = oracle.indexer_scores(n, d["q_fp4"], d["q_sf"], d["w"], d["k_fp4"], d["k_sf"])
+    compare.compare_topk(idx[0], ora_s[0], int(n[0]), w.k, what="workload 0 top-k")
+    ora_idx = oracle.topk(ora_s[0], int(n[0]), w.k)[None]
+    kv, sc = ora_c["kv"], ora_c["kv_scale"]
+    out = csa.sparse_attn_decode(dev(d["q"]), dev(d["pos"]), dev(n), dev(kv), dev(sc),
+                                 dev(d["swa"]), dev(d["sink"]), dev(ora_idx))
+    want, _ = oracle.attention(d["q"], d["pos"], n, kv, sc, d["swa"], d["sink"], idx=ora_idx)
+    compare.close(out.float().cpu().numpy(), want, what="workload 0 attention")
+
+
+def test_workload1_hca_decode():
+    w = synth.WORKLOADS[1]
+    d = synth.decode_inputs(w)
+    out, lse = csa.hca_attn_decode(dev(d["q"]), dev(d["pos"]), dev(d["n_entries"]),
+                                   dev(d["kv"]), dev(d["kv_scale"]), dev(d["swa"]),
+                                   dev(d["sink"]), lse=True)
+    want, wlse = oracle.attention(d["q"], d["pos"], d["n_entries"], d["kv"], d["kv_scale"],
+                                  d["swa"], d["sink"])
+    compare.close(out.float().cpu().numpy(), want, what="workload 1")
+    np.testing.assert_allclose(host(lse), wlse, rtol=1e-4, atol=1e-4)
