@@ -1,0 +1,352 @@
+"""Benchmark of the CSA decode step at 1M context (V4-Pro-shaped layer).
+
+One step = one decode query for each of the B = 4 sequences of the workload
+(context 1,048,576 tokens -> 262,144 compressed entries, 128 heads sharing one KV of
+head_dim 512, indexer 64 heads x 128 FP4 dims, top-k 1024, 128-token window, sink):
+  csa_indexer_topk  (FP4 indexer scores over every entry + top-k selection)
+  csa_sparse_attn_decode  (shared-KV MQA over the selected entries + window + sink)
+Metric: decode queries/s (whole job). Inputs are synthetic and seeded; four device copies
+of the streamed inputs are rotated so that consecutive steps never hit in L2.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun every rank runs its own 4-sequence batch (weak scaling, no collective on
+the data path); rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+WORKLOAD_ID = 3
+METRIC = "CSA decode queries/s at 1M ctx; achieved HBM GB/s as % of B200 peak"
+UNIT = "queries/s"
+COPIES = 4
+
+
+def algorithmic_bytes(d: dict) -> tuple[int, int]:
+    """(indexer_topk bytes per call, whole decode step bytes) by the layer's definition:
+    per query 68 B per eligible entry (64 B E2M1 key + 4 B E8M0 scales), the FP4 query
+    (H_I x 68 B) and weights, the k selected rows of 580 B (576 B + fp32 scale), 128 window
+    rows of 1 KB, Q and O (H x 1 KB each), the indices and positions."""
+    w = d["workload"]
+    n = d["n_entries"].astype(np.int64)
+    idx = int((n * 68).sum() + d["B"] * (w.H_I * 72 + w.k * 4 + 4))
+    attn = d["B"] * (w.k * 580 + 128 * 1024 + 2 * w.H * 1024 + w.k * 4 + 8 + w.H * 4)
+    return idx, idx + attn
+
+
+def peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "src": "measured"}
+    return {"hbm_gbs": 6650.0, "src": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the GPU is busy."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.12)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        mhz, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) != 6:
+                continue
+            try:
+                mhz.append(float(f[0]))
+                mx.append(float(f[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, f[2:]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(mhz) if mhz else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(mhz)}
+
+
+def ncu_traffic() -> dict | None:
+    """DRAM bytes per launch of the indexer call from the committed ncu summary, if it was
+    taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "indexer_topk_csa_decode_pro_1m.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    from long_context_compressed_layer_b200 import build as b
+    if d.get("sources_sha") != b.sources_sha():
+        return None
+    return d
+
+
+def run_reference(args, rank: int) -> None:
+    """The fp64 CPU oracle, as it stands, on the host cores: each step is one decode query
+    (one sequence of the workload: indexer over 262,144 entries, top-k, attention)."""
+    if rank != 0:
+        return
+    import oracle
+    from synth import inputs as synth
+
+    w = synth.WORKLOADS[WORKLOAD_ID]
+    d = synth.decode_inputs(w, B=1)
+    cores = os.cpu_count() or 1
+
+    def step():
+        s = oracle.indexer_scores(d["n_entries"], d["q_fp4"], d["q_sf"], d["w"], d["k_fp4"],
+                                  d["k_sf"])
+        idx = oracle.topk(s[0], int(d["n_entries"][0]), w.k)[None]
+        oracle.attention(d["q"], d["pos"], d["n_entries"], d["kv"], d["kv_scale"], d["swa"],
+                         d["sink"], idx=idx)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    v = args.steps / dt
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "queries_per_step": 1, "context": w.L, "heads": w.H,
+                   "indexer_heads": w.H_I, "top_k": w.k, "l2": "host run"},
+        "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": "one decode query (one sequence of the workload) per step"},
+        "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def cpu_baseline_sample(d_host, w) -> dict:
+    """The oracle timed on a bounded sample: 2 decode queries of the workload."""
+    import oracle
+    cores = os.cpu_count() or 1
+    q = 2
+    t0 = time.perf_counter()
+    for b in range(q):
+        sl = slice(b, b + 1)
+        s = oracle.indexer_scores(d_host["n_entries"][sl], d_host["q_fp4"][sl],
+                                  d_host["q_sf"][sl], d_host["w"][sl], d_host["k_fp4"][sl],
+                                  d_host["k_sf"][sl])
+        idx = oracle.topk(s[0], int(d_host["n_entries"][b]), w.k)[None]
+        oracle.attention(d_host["q"][sl], d_host["pos"][sl], d_host["n_entries"][sl],
+                         d_host["kv"][sl], d_host["kv_scale"][sl], d_host["swa"][sl],
+                         d_host["sink"], idx=idx)
+    dt = time.perf_counter() - t0
+    return {"value": q / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{q} decode queries (sequences 0-1 of the workload), fp64, all host threads"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=500)
+    ap.add_argument("--impl", default="csa", choices=["csa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank)
+        return
+
+    import torch
+    import torch.distributed as dist
+
+    import long_context_compressed_layer_b200 as csa
+    from synth import inputs as synth
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = synth.WORKLOADS[WORKLOAD_ID]
+    d = synth.decode_inputs(w, seed=w.seed + 1000 * rank)
+    B, k, Nmax = d["B"], w.k, d["Nmax"]
+
+    def dev(x):
+        x = np.ascontiguousarray(x)
+        return torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).cuda()
+
+    streamed = ("k_fp4", "k_sf", "kv", "kv_scale", "q_fp4", "q_sf", "w", "q", "swa")
+    base = {key: dev(d[key]) for key in streamed + ("n_entries", "pos", "sink")}
+    copies = [base] + [{key: (base[key].clone() if key in streamed else base[key])
+                        for key in base} for _ in range(COPIES - 1)]
+    ws_idx = csa.indexer_topk_workspace(B, Nmax, k)
+    ws_att = csa.attn_workspace(B, w.H, k + 128)
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    out = torch.empty((B, w.H, 512), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(c, ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        csa.indexer_topk(c["n_entries"], c["q_fp4"], c["q_sf"], c["w"], c["k_fp4"], c["k_sf"],
+                         k, workspace=ws_idx, idx=idx, dev_status=status)
+        if ev is not None:
+            ev[1].record(stream)
+        csa.sparse_attn_decode(c["q"], c["pos"], c["n_entries"], c["kv"], c["kv_scale"],
+                               c["swa"], c["sink"], idx, workspace=ws_att, out=out,
+                               dev_status=status)
+        if ev is not None:
+            ev[2].record(stream)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for i in range(max(args.warmup, 3)):
+        step(copies[i % COPIES])
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for i in range(args.steps):
+        step(copies[i % COPIES])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = t0.elapsed_time(t1)
+
+    # live per-call timing of the dominant call (separate pass, same stream, same rotation)
+    nprobe = min(args.steps, 2000)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nprobe)]
+    for i in range(nprobe):
+        step(copies[i % COPIES], evs[i])
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    t_idx = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    t_att = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during the benchmark")
+
+    # end to end through host buffers: the step's query-side inputs go up, results come down
+    q_inputs = ("q", "q_fp4", "q_sf", "w", "pos", "n_entries")
+    pinned = {key: base[key].cpu().pin_memory() for key in q_inputs}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    idx_h = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
+    dev_in = {key: torch.empty_like(base[key]) for key in q_inputs}
+    h2d = sum(pinned[key].numel() * pinned[key].element_size() for key in q_inputs)
+    d2h = out_h.numel() * 2 + idx_h.numel() * 4
+    e_steps = min(args.steps, 2000)
+
+    def e2e_step(c):
+        for key in q_inputs:
+            dev_in[key].copy_(pinned[key], non_blocking=True)
+        cc = dict(c)
+        cc.update(dev_in)
+        step(cc)
+        out_h.copy_(out, non_blocking=True)
+        idx_h.copy_(idx, non_blocking=True)
+
+    for i in range(3):
+        e2e_step(copies[i % COPIES])
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e_steps):
+        e2e_step(copies[i % COPIES])
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e_steps
+
+    ms_step = ms_total / args.steps
+    if world > 1:
+        t = torch.tensor([ms_step, e2e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_step, e2e_ms = float(t[0]), float(t[1])
+    value = world * B / (ms_step * 1e-3)
+    e2e_value = world * B / (e2e_ms * 1e-3)
+
+    if rank == 0:
+        idx_bytes, step_bytes = algorithmic_bytes(d)
+        pk = peaks()
+        achieved = idx_bytes / (t_idx * 1e-3) / 1e9
+        traffic = ncu_traffic()
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4+fp16",
+            "data": "synthetic",
+            "config": {"workload": w.name, "queries_per_step_per_gpu": B, "context": w.L,
+                       "entries_per_seq": int(d["n_entries"][0]), "heads": w.H,
+                       "indexer_heads": w.H_I, "top_k": w.k, "window": 128,
+                       "l2": f"inputs rotated over {COPIES} device copies "
+                             f"({COPIES * (Nmax * 68 * B) / 1e6:.0f} MB of streamed keys > L2)",
+                       "step_algorithmic_bytes": step_bytes,
+                       "step_achieved_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
+                       "step_frac_of_peak": step_bytes / (ms_step * 1e-3) / 1e9 / pk["hbm_gbs"],
+                       "indexer_topk_ms": t_idx, "sparse_attn_ms": t_att},
+            "roofline": {"bound": "hbm", "kernel": "csa_indexer_topk (score + select)",
+                         "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "peak_src": pk["src"],
+                         "algorithmic_bytes_per_launch": idx_bytes,
+                         "traffic": traffic["dram_bytes_per_launch"] if traffic else None},
+            "clocks": clocks,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 4 * args.steps,
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline_sample(d, w)
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -24,6 +24,17 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
 
 
+def sources_sha() -> str:
+    """Hash of the kernel sources and the ABI header (ties profiles to the code they used)."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(HERE, "csrc", "*"))) + [
+            os.path.join(HERE, "..", "include", "csa.h")]:
+        h.update(open(f, "rb").read())
+    return h.hexdigest()[:16]
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     srcs = sources()
     deps = srcs + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + [

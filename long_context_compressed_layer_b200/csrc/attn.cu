@@ -7,12 +7,14 @@
 // The rows a query attends to form one list: the selected entries (CSA) or all eligible
 // entries (HCA), then the 128 window tokens t-127 .. t. The list is cut into chunks of
 // 64 rows. attn_chunk_kernel handles one (sequence, chunk):
-//   - Q [H heads x 512] arrives by TMA (128-byte swizzle, K-major), padded to 128 rows;
-//   - the 64 rows are gathered and dequantised to BF16 in shared memory (E4M3 code x entry
-//     scale, BF16 RoPE dims, BF16 window rows), in the same swizzled layout, which serves
-//     as K-major B for S = Q V^T and as MN-major B for O = P V;
+//   - Q [H heads x 512] arrives by TMA (128-byte swizzle, K-major), padded to 128 rows,
+//     and is widened in place from BF16 to FP16 (exact for |q| >= 2^-14);
+//   - the 64 rows are gathered and dequantised to FP16 in shared memory (E4M3 code x entry
+//     scale, RoPE dims, window rows), in the same swizzled layout, which serves as K-major
+//     B for S = Q V^T and as MN-major B for O = P V. FP16 (11 significant bits) rather
+//     than BF16 (8) keeps the staging error well inside the output tolerance;
 //   - tcgen05.mma kind::f16 computes S[128 x 64] in TMEM; one thread per head turns its row
-//     into exp(tau*S - m) (fp32), keeps m and l = sum, and writes P as BF16 (K-major A);
+//     into exp(tau*S - m) (fp32), keeps m and l = sum, and writes P as FP16 (K-major A);
 //   - two tcgen05.mma N = 256 halves compute O[128 x 512] in TMEM (S's columns are reused);
 //   - O, m and l go to the workspace.
 // attn_combine_kernel merges the chunks of a sequence in fixed order with the sink,
@@ -26,9 +28,9 @@ constexpr int kAtRows = 64;  // rows per chunk = N of the S MMA
 constexpr int kAtThreads = 128;
 
 struct AtSmem {
-  uint8_t q[8][128 * 128];      // 8 K-blocks of [128 heads x 64 dims] bf16, 128-B swizzle
-  uint8_t v[8][kAtRows * 128];  // 8 dim-blocks of [64 rows x 64 dims] bf16, 128-B swizzle
-  uint8_t pm[128 * 128];        // P [128 heads x 64 rows] bf16, 128-B swizzle
+  uint8_t q[8][128 * 128];      // 8 K-blocks of [128 heads x 64 dims] fp16, 128-B swizzle
+  uint8_t v[8][kAtRows * 128];  // 8 dim-blocks of [64 rows x 64 dims] fp16, 128-B swizzle
+  uint8_t pm[128 * 128];        // P [128 heads x 64 rows] fp16, 128-B swizzle
   const uint8_t* src[kAtRows];  // row source
   float rscale[kAtRows];        // entry scale, 0 for window rows
   int kind[kAtRows];            // 0 invalid, 1 entry, 2 window row
@@ -54,6 +56,14 @@ struct AtParams {
   float2* part_ml; // [B][C][H]
   int32_t* dev_status;
 };
+
+__device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    w[e] = pack_half2(bf16_bits_to_f32(w[e] & 0xFFFF), bf16_bits_to_f32(w[e] >> 16));
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 __device__ __forceinline__ int at_rows_total(const AtParams& p, int n) {
   return (p.sparse ? p.k : n) + kWin;
@@ -142,33 +152,39 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const uint32_t pair = (e < 2 ? raw.x : raw.y) >> (16 * (e & 1));
-          const float lo = e4m3_to_f32((uint8_t)(pair & 0xFF)) * scl;
-          const float hi = e4m3_to_f32((uint8_t)((pair >> 8) & 0xFF)) * scl;
-          w[e] = (uint32_t)f32_to_bf16_bits(lo) | ((uint32_t)f32_to_bf16_bits(hi) << 16);
+          w[e] = pack_half2(e4m3_to_f32((uint8_t)(pair & 0xFF)) * scl,
+                            e4m3_to_f32((uint8_t)((pair >> 8) & 0xFF)) * scl);
         }
         o = make_uint4(w[0], w[1], w[2], w[3]);
       } else {
-        o = *reinterpret_cast<const uint4*>(src + kNope + 2 * (d - kNope));
+        o = bf16x8_to_f16x8(*reinterpret_cast<const uint4*>(src + kNope + 2 * (d - kNope)));
       }
     } else if (kind == 2) {
-      o = *reinterpret_cast<const uint4*>(s.src[r] + 2 * d);
+      o = bf16x8_to_f16x8(*reinterpret_cast<const uint4*>(s.src[r] + 2 * d));
     }
     *reinterpret_cast<uint4*>(&s.v[ch >> 3][r * 128 + (((ch & 7) ^ (r & 7)) << 4)]) = o;
   }
   fence_async_smem();
   __syncthreads();
 
+  // widen Q to FP16 in place once the TMA has landed
+  bool ok = mbar_wait(&s.q_full, 0, p.dev_status);
+  for (int i = tid; i < 8 * p.H * 8; i += kAtThreads) {
+    uint4* c16 = reinterpret_cast<uint4*>(&s.q[i / (p.H * 8)][(i % (p.H * 8)) * 16]);
+    *c16 = bf16x8_to_f16x8(*c16);
+  }
+  fence_async_smem();
+  ok = __syncthreads_and(ok) != 0;
+
   // S = Q V^T : M = 128 heads, N = 64 rows, K = 512 (32 steps of 16)
   const uint32_t t_o = tmem, t_s = tmem + 256;
-  bool ok = true;
   if (tid == 0) {
-    ok = mbar_wait(&s.q_full, 0, p.dev_status);
     if (ok) {
       tc_fence_after();
-      const uint32_t id = idesc_bf16(128, kAtRows, false);
+      const uint32_t id = idesc_f16(128, kAtRows, false);
       for (int kk = 0; kk < 32; ++kk) {
         const uint32_t off = (kk & 3) * 32;
-        mma_bf16(t_s, smem_desc(smem_u32(s.q[kk >> 2]) + off, 16, 1024, kSwizzle128B),
+        mma_f16(t_s, smem_desc(smem_u32(s.q[kk >> 2]) + off, 16, 1024, kSwizzle128B),
                  smem_desc(smem_u32(s.v[kk >> 2]) + off, 16, 1024, kSwizzle128B), id, kk > 0);
       }
     }
@@ -208,7 +224,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
         const float p1 = m_c == -INFINITY ? 0.f : expf(lg[r + 1] - m_c);
         l_c += p0;
         l_c += p1;
-        w[e] = (uint32_t)f32_to_bf16_bits(p0) | ((uint32_t)f32_to_bf16_bits(p1) << 16);
+        w[e] = pack_half2(p0, p1);
       }
       *reinterpret_cast<uint4*>(prow + ((ch ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
@@ -221,10 +237,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   if (tid == 0) {
     if (ok) {
       tc_fence_after();
-      const uint32_t id = idesc_bf16(128, 256, true);
+      const uint32_t id = idesc_f16(128, 256, true);
       for (int half = 0; half < 2; ++half) {
         for (int kk = 0; kk < 4; ++kk) {
-          mma_bf16(t_o + half * 256, smem_desc(smem_u32(s.pm) + kk * 32, 16, 1024, kSwizzle128B),
+          mma_f16(t_o + half * 256, smem_desc(smem_u32(s.pm) + kk * 32, 16, 1024, kSwizzle128B),
                    smem_desc(smem_u32(s.v[half * 4]) + kk * 2048, kAtRows * 128, 1024, kSwizzle128B),
                    id, kk > 0);
         }
