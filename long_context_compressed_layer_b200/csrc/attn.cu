@@ -16,7 +16,8 @@
 //   - tcgen05.mma kind::f16 computes S[128 x 64] in TMEM; one thread per head turns its row
 //     into exp(tau*S - m) (fp32), keeps m and l = sum, and writes P as FP16 (K-major A);
 //   - two tcgen05.mma N = 256 halves compute O[128 x 512] in TMEM (S's columns are reused);
-//   - O, m and l go to the workspace.
+//   - O / l (FP16, [dim-block][head][32] so every warp stores 2 KB contiguous), m and l go
+//     to the workspace.
 // attn_combine_kernel merges the chunks of a sequence in fixed order with the sink,
 // normalises, de-rotates the last 64 dims and stores BF16 (and lse). The chunk count
 // depends only on k (CSA) or n (HCA), never on the batch, so results are batch-invariant.
@@ -25,15 +26,16 @@
 namespace csa {
 
 constexpr int kAtRows = 64;  // rows per chunk = N of the S MMA
-constexpr int kAtThreads = 128;
+constexpr int kAtThreads = 256;
 
 struct AtSmem {
   uint8_t q[8][128 * 128];      // 8 K-blocks of [128 heads x 64 dims] fp16, 128-B swizzle
   uint8_t v[8][kAtRows * 128];  // 8 dim-blocks of [64 rows x 64 dims] fp16, 128-B swizzle
   uint8_t pm[128 * 128];        // P [128 heads x 64 rows] fp16, 128-B swizzle
-  const uint8_t* src[kAtRows];  // row source
-  float rscale[kAtRows];        // entry scale, 0 for window rows
+  const uint8_t* row[kAtRows];  // row source
+  const float* scl[kAtRows];    // entry rows: address of the entry scale
   int kind[kAtRows];            // 0 invalid, 1 entry, 2 window row
+  float inv_l[128];             // 1 / (chunk sum) per head
   uint64_t q_full, s_done, o_done;
   uint32_t tmem_base;
 };
@@ -52,8 +54,8 @@ struct AtParams {
   int derotate;
   uint16_t* out;
   float* lse;
-  float* part_o;   // [B][C][H][512]
-  float2* part_ml; // [B][C][H]
+  __half* part_o;  // [B][C][16][H][32]: chunk output / chunk sum, fp16
+  float2* part_ml; // [B][C][H]: (chunk max logit, chunk sum)
   int32_t* dev_status;
 };
 
@@ -63,6 +65,26 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
   for (int e = 0; e < 4; ++e)
     w[e] = pack_half2(bf16_bits_to_f32(w[e] & 0xFFFF), bf16_bits_to_f32(w[e] >> 16));
   return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// 16 E4M3 codes x scale -> two 16-byte chunks of FP16
+__device__ __forceinline__ void e4m3x16_to_f16(uint4 raw, float scl, uint4* lo, uint4* hi) {
+  const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t x = in[e];
+    o[2 * e] = pack_half2(e4m3_to_f32((uint8_t)(x & 0xFF)) * scl,
+                          e4m3_to_f32((uint8_t)((x >> 8) & 0xFF)) * scl);
+    o[2 * e + 1] = pack_half2(e4m3_to_f32((uint8_t)((x >> 16) & 0xFF)) * scl,
+                              e4m3_to_f32((uint8_t)(x >> 24)) * scl);
+  }
+  *lo = make_uint4(o[0], o[1], o[2], o[3]);
+  *hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+__device__ __forceinline__ void store_v_chunk(AtSmem& s, int r, int ch, uint4 v) {
+  *reinterpret_cast<uint4*>(&s.v[ch >> 3][r * 128 + (((ch & 7) ^ (r & 7)) << 4)]) = v;
 }
 
 __device__ __forceinline__ int at_rows_total(const AtParams& p, int n) {
@@ -76,15 +98,20 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int c = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int row0 = c * kAtRows;
+  pdl_wait();
+  pdl_trigger();
+  // independent loads first: length, position and (CSA) this thread's selected index
   int n = p.n_entries[b];
+  const int t = p.pos[b];
+  int jsel = -1;
+  if (p.sparse && tid < kAtRows && row0 + tid < p.k) jsel = p.idx[(size_t)b * p.k + row0 + tid];
   if (n < 0 || n > p.Nmax) {
     if (tid == 0) report(p.dev_status, CSA_ERR_DEVICE);
     n = n < 0 ? 0 : (int)p.Nmax;
   }
   const int rows_total = at_rows_total(p, n);
-  const int row0 = c * kAtRows;
   if (row0 >= rows_total) return;  // uniform: this chunk does not exist for this sequence
-  const int t = p.pos[b];
   if (t < 0 && tid == 0) report(p.dev_status, CSA_ERR_DEVICE);
   const int nwin_first = p.sparse ? p.k : n;  // list index of the first window row
 
@@ -93,6 +120,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     mbar_init(&s.s_done, 1);
     mbar_init(&s.o_done, 1);
     mbar_fence_init();
+    prefetch_tensormap(&qmap);
+    mbar_arrive_expect_tx(&s.q_full, (uint32_t)p.H * kD * 2);
+    for (int blk = 0; blk < 8; ++blk) tma_load_2d(s.q[blk], &qmap, &s.q_full, blk * 64, b * p.H);
   }
   if (warp == 0) tmem_alloc(&s.tmem_base, 512);
   // Q rows H..127 are zero padding (generic-proxy writes, fenced below)
@@ -102,18 +132,17 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       *reinterpret_cast<uint4*>(&s.q[blk][p.H * 128 + rem * 16]) = make_uint4(0, 0, 0, 0);
     }
   }
-  // row sources
+  // row sources (the entry scale is fetched with the row data below)
   if (tid < kAtRows) {
     const int r = row0 + tid;
     int kind = 0;
     const uint8_t* src = nullptr;
-    float scl = 0.f;
     if (r < nwin_first) {
-      const int j = p.sparse ? p.idx[(size_t)b * p.k + r] : r;
+      const int j = p.sparse ? jsel : r;
       if (j >= 0 && j < n) {
         kind = 1;
         src = p.kv + ((size_t)b * p.Nmax + j) * kRow;
-        scl = p.kv_scale[(size_t)b * p.Nmax + j];
+        s.scl[tid] = p.kv_scale + (size_t)b * p.Nmax + j;
       } else if (j != -1) {
         report(p.dev_status, CSA_ERR_DEVICE);
       }
@@ -125,48 +154,47 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       }
     }
     s.kind[tid] = kind;
-    s.src[tid] = src;
-    s.rscale[tid] = scl;
+    s.row[tid] = src;
   }
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  if (tid == 0) {
-    prefetch_tensormap(&qmap);
-    mbar_arrive_expect_tx(&s.q_full, (uint32_t)p.H * kD * 2);
-    for (int blk = 0; blk < 8; ++blk) tma_load_2d(s.q[blk], &qmap, &s.q_full, blk * 64, b * p.H);
-  }
-  // gather + dequantise: 64 rows x 64 chunks of 8 dims; chunk ch of row r lands in dim-block
-  // ch/8 at 16-byte slot (ch%8) ^ (r%8) of the row's 128 bytes
-  for (int task = tid; task < kAtRows * 64; task += kAtThreads) {
-    const int r = task >> 6, ch = task & 63;
-    const int d = ch * 8;
-    uint4 o = make_uint4(0, 0, 0, 0);
+  // gather: four threads per row; every thread issues all of its 16-byte pieces (and the
+  // row's scale) before converting any, so ~40-64 KB are in flight per CTA
+  {
+    const int r = tid >> 2, qd = tid & 3;
     const int kind = s.kind[r];
-    if (kind == 1) {
-      const uint8_t* src = s.src[r];
-      if (d < kNope) {
-        const uint2 raw = *reinterpret_cast<const uint2*>(src + d);
-        const float scl = s.rscale[r];
-        uint32_t w[4];
+    const uint8_t* src = s.row[r];
+    const int units = kind == 1 ? 36 : (kind == 2 ? 64 : 0);  // 16-byte pieces of the row
+    const float scl = kind == 1 ? __ldg(s.scl[r]) : 0.f;
+    uint4 buf[16];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t pair = (e < 2 ? raw.x : raw.y) >> (16 * (e & 1));
-          w[e] = pack_half2(e4m3_to_f32((uint8_t)(pair & 0xFF)) * scl,
-                            e4m3_to_f32((uint8_t)((pair >> 8) & 0xFF)) * scl);
+    for (int i = 0; i < 16; ++i) {
+      const int u = qd + 4 * i;
+      buf[i] = u < units ? __ldg(reinterpret_cast<const uint4*>(src + 16 * u))
+                         : make_uint4(0, 0, 0, 0);
+    }
+    if (kind == 1) {
+#pragma unroll
+      for (int i = 0; i < 9; ++i) {
+        const int u = qd + 4 * i;
+        if (u < 28) {  // 16 E4M3 dims -> output chunks 2u, 2u+1
+          uint4 lo, hi;
+          e4m3x16_to_f16(buf[i], scl, &lo, &hi);
+          store_v_chunk(s, r, 2 * u, lo);
+          store_v_chunk(s, r, 2 * u + 1, hi);
+        } else {  // 8 BF16 RoPE dims -> chunk 56 + (u - 28)
+          store_v_chunk(s, r, 28 + u, bf16x8_to_f16x8(buf[i]));
         }
-        o = make_uint4(w[0], w[1], w[2], w[3]);
-      } else {
-        o = bf16x8_to_f16x8(*reinterpret_cast<const uint4*>(src + kNope + 2 * (d - kNope)));
       }
     } else if (kind == 2) {
-      o = bf16x8_to_f16x8(*reinterpret_cast<const uint4*>(s.src[r] + 2 * d));
+#pragma unroll
+      for (int i = 0; i < 16; ++i) store_v_chunk(s, r, qd + 4 * i, bf16x8_to_f16x8(buf[i]));
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) store_v_chunk(s, r, qd + 4 * i, make_uint4(0, 0, 0, 0));
     }
-    *reinterpret_cast<uint4*>(&s.v[ch >> 3][r * 128 + (((ch & 7) ^ (r & 7)) << 4)]) = o;
   }
-  fence_async_smem();
-  __syncthreads();
-
   // widen Q to FP16 in place once the TMA has landed
   bool ok = mbar_wait(&s.q_full, 0, p.dev_status);
   for (int i = tid; i < 8 * p.H * 8; i += kAtThreads) {
@@ -185,7 +213,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       for (int kk = 0; kk < 32; ++kk) {
         const uint32_t off = (kk & 3) * 32;
         mma_f16(t_s, smem_desc(smem_u32(s.q[kk >> 2]) + off, 16, 1024, kSwizzle128B),
-                 smem_desc(smem_u32(s.v[kk >> 2]) + off, 16, 1024, kSwizzle128B), id, kk > 0);
+                smem_desc(smem_u32(s.v[kk >> 2]) + off, 16, 1024, kSwizzle128B), id, kk > 0);
       }
     }
     mma_commit(&s.s_done);
@@ -196,10 +224,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   }
   tc_fence_after();
 
-  // softmax rows: thread tid owns head tid (TMEM lane tid)
+  // softmax rows: thread h < 128 owns head h (TMEM lane h)
   const int h = tid;
   float m_c = -INFINITY, l_c = 0.f;
-  {
+  if (tid < 128) {
     uint32_t r0[32], r1[32];
     const uint32_t ta = t_s + ((uint32_t)(warp * 32) << 16);
     tmem_ld32(ta, r0);
@@ -228,6 +256,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       }
       *reinterpret_cast<uint4*>(prow + ((ch ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
+    s.inv_l[h] = l_c > 0.f ? 1.f / l_c : 0.f;
+    if (h < p.H) {
+      const size_t slot = ((size_t)b * p.C + c) * p.H + h;
+      p.part_ml[slot] = ok ? make_float2(m_c, l_c) : make_float2(-INFINITY, 0.f);
+    }
   }
   fence_async_smem();
   tc_fence_before();
@@ -241,35 +274,37 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       for (int half = 0; half < 2; ++half) {
         for (int kk = 0; kk < 4; ++kk) {
           mma_f16(t_o + half * 256, smem_desc(smem_u32(s.pm) + kk * 32, 16, 1024, kSwizzle128B),
-                   smem_desc(smem_u32(s.v[half * 4]) + kk * 2048, kAtRows * 128, 1024, kSwizzle128B),
-                   id, kk > 0);
+                  smem_desc(smem_u32(s.v[half * 4]) + kk * 2048, kAtRows * 128, 1024, kSwizzle128B),
+                  id, kk > 0);
         }
       }
     }
     mma_commit(&s.o_done);
   }
-  ok = mbar_wait(&s.o_done, 0, p.dev_status) && ok;
+  mbar_wait(&s.o_done, 0, p.dev_status);
   tc_fence_after();
-  if (h < p.H) {
-    const size_t slot = ((size_t)b * p.C + c) * p.H + h;
-    float* dst = p.part_o + slot * kD;
-    for (int cc = 0; cc < 16; ++cc) {
+  {
+    // warp w reads lanes of quadrant w % 4, columns [256 * (w / 4), +256): 8 loads of 32
+    const int quad = warp & 3, colh = warp >> 2;
+    const int hh = quad * 32 + (tid & 31);
+    const float inv = s.inv_l[hh];
+    for (int i = 0; i < 8; ++i) {
+      const int cc = colh * 8 + i;  // 32-dim block
       uint32_t r[32];
-      tmem_ld32(t_o + ((uint32_t)(warp * 32) << 16) + cc * 32, r);
+      tmem_ld32(t_o + ((uint32_t)(quad * 32) << 16) + cc * 32, r);
       tmem_ld_wait();
+      if (hh < p.H) {
+        __half* dst = p.part_o + ((((size_t)b * p.C + c) * 16 + cc) * p.H + hh) * 32;
 #pragma unroll
-      for (int e = 0; e < 32; e += 4)
-        *reinterpret_cast<float4*>(dst + cc * 32 + e) =
-            make_float4(__uint_as_float(r[e]), __uint_as_float(r[e + 1]),
-                        __uint_as_float(r[e + 2]), __uint_as_float(r[e + 3]));
-    }
-    p.part_ml[slot] = ok ? make_float2(m_c, l_c) : make_float2(-INFINITY, 0.f);
-  } else {
-    // keep the warp's tcgen05.ld calls uniform
-    for (int cc = 0; cc < 16; ++cc) {
-      uint32_t r[32];
-      tmem_ld32(t_o + ((uint32_t)(warp * 32) << 16) + cc * 32, r);
-      tmem_ld_wait();
+        for (int e = 0; e < 32; e += 8) {
+          uint4 v;
+          v.x = pack_half2(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv);
+          v.y = pack_half2(__uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
+          v.z = pack_half2(__uint_as_float(r[e + 4]) * inv, __uint_as_float(r[e + 5]) * inv);
+          v.w = pack_half2(__uint_as_float(r[e + 6]) * inv, __uint_as_float(r[e + 7]) * inv);
+          *reinterpret_cast<uint4*>(dst + e) = v;
+        }
+      }
     }
   }
   tc_fence_before();
@@ -280,10 +315,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   }
 }
 
-// One CTA per (sequence, head): 128 threads x 4 dims.
+// One CTA per (sequence, head): 128 threads x 4 dims. The chunks are merged in their fixed
+// order: o = sum_c exp(m_c - M) l_c o_c / Z,  Z = exp(sink - M) + sum_c exp(m_c - M) l_c.
 __global__ void __launch_bounds__(128) attn_combine_kernel(AtParams p) {
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   __shared__ float rot[32][2];
+  pdl_wait();
+  pdl_trigger();
   __shared__ float wgt[64];
   __shared__ float sh_M, sh_Z;
   int n = p.n_entries[b];
@@ -297,48 +335,70 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AtParams p) {
     rot[tid][1] = sn;
   }
   const float sink = p.sink[h];
-  if (tid == 0) {
+  if (tid < 32) {  // one warp reduces the chunk statistics
     float M = sink;
-    for (int c = 0; c < C_b; ++c) M = fmaxf(M, p.part_ml[((size_t)b * p.C + c) * p.H + h].x);
+    for (int c = tid; c < C_b; c += 32) M = fmaxf(M, p.part_ml[((size_t)b * p.C + c) * p.H + h].x);
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Z = 0.f;
-    if (M == INFINITY) {
-      Z = INFINITY;
-    } else {
-      Z = sink == -INFINITY ? 0.f : expf(sink - M);
-      for (int c = 0; c < C_b; ++c) {
+    if (M != INFINITY) {
+      for (int c = tid; c < C_b; c += 32) {  // fixed assignment and tree: deterministic
         const float2 ml = p.part_ml[((size_t)b * p.C + c) * p.H + h];
-        const float w = ml.x == -INFINITY ? 0.f : expf(ml.x - M);
-        Z += w * ml.y;
+        Z += ml.x == -INFINITY ? 0.f : expf(ml.x - M) * ml.y;
       }
+      for (int o = 16; o > 0; o >>= 1) Z += __shfl_xor_sync(0xffffffffu, Z, o);
+      if (tid == 0) Z += sink == -INFINITY ? 0.f : expf(sink - M);
+      Z = __shfl_sync(0xffffffffu, Z, 0);
+    } else {
+      Z = INFINITY;
     }
-    sh_M = M;
-    sh_Z = Z;
-    if (p.lse) p.lse[(size_t)b * p.H + h] = M == INFINITY ? INFINITY : M + logf(Z);
+    if (tid == 0) {
+      sh_M = M;
+      sh_Z = Z;
+      if (p.lse) p.lse[(size_t)b * p.H + h] = M == INFINITY ? INFINITY : M + logf(Z);
+    }
   }
   __syncthreads();
   const float M = sh_M, Z = sh_Z;
-  if (tid < C_b && tid < 64) {
-    const float mx = p.part_ml[((size_t)b * p.C + tid) * p.H + h].x;
-    wgt[tid] = (M == INFINITY || mx == -INFINITY) ? 0.f : expf(mx - M) / Z;
+  for (int c = tid; c < C_b && c < 64; c += 128) {
+    const float2 ml = p.part_ml[((size_t)b * p.C + c) * p.H + h];
+    wgt[c] = (M == INFINITY || ml.x == -INFINITY) ? 0.f : expf(ml.x - M) * ml.y / Z;
   }
   __syncthreads();
-  const int d0 = 4 * tid;
+  const int d0 = 4 * tid, cc = d0 >> 5, e0 = d0 & 31;
+  const __half* base = p.part_o + ((size_t)b * p.C * 16 + cc) * p.H * 32 + (size_t)h * 32 + e0;
+  const size_t cstride = (size_t)16 * p.H * 32;
   float o[4] = {0.f, 0.f, 0.f, 0.f};
-  for (int c = 0; c < C_b; ++c) {
+  int c = 0;
+  for (; c + 4 <= C_b && c + 4 <= 64; c += 4) {  // four loads in flight
+    uint2 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const uint2*>(base + (c + u) * cstride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const float w = wgt[c + u];
+      const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&v[u].x));
+      const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&v[u].y));
+      o[0] = fmaf(w, a.x, o[0]);
+      o[1] = fmaf(w, a.y, o[1]);
+      o[2] = fmaf(w, bb.x, o[2]);
+      o[3] = fmaf(w, bb.y, o[3]);
+    }
+  }
+  for (; c < C_b; ++c) {
     float w;
     if (c < 64) {
       w = wgt[c];
     } else {
-      const float mx = p.part_ml[((size_t)b * p.C + c) * p.H + h].x;
-      w = (M == INFINITY || mx == -INFINITY) ? 0.f : expf(mx - M) / Z;
+      const float2 ml = p.part_ml[((size_t)b * p.C + c) * p.H + h];
+      w = (M == INFINITY || ml.x == -INFINITY) ? 0.f : expf(ml.x - M) * ml.y / Z;
     }
-    if (w == 0.f) continue;
-    const float4 v = *reinterpret_cast<const float4*>(
-        p.part_o + (((size_t)b * p.C + c) * p.H + h) * kD + d0);
-    o[0] = fmaf(w, v.x, o[0]);
-    o[1] = fmaf(w, v.y, o[1]);
-    o[2] = fmaf(w, v.z, o[2]);
-    o[3] = fmaf(w, v.w, o[3]);
+    const uint2 v = *reinterpret_cast<const uint2*>(base + c * cstride);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
+    const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
+    o[0] = fmaf(w, a.x, o[0]);
+    o[1] = fmaf(w, a.y, o[1]);
+    o[2] = fmaf(w, bb.x, o[2]);
+    o[3] = fmaf(w, bb.y, o[3]);
   }
   if (p.derotate && d0 >= kNope) {
 #pragma unroll
@@ -360,7 +420,7 @@ size_t at_smem_bytes() { return sizeof(AtSmem) + 1024; }
 
 size_t at_workspace_size(int B, int H, int rows_max) {
   const size_t C = (size_t)(rows_max + kAtRows - 1) / kAtRows;
-  const size_t o = (size_t)B * C * H * kD * sizeof(float);
+  const size_t o = (size_t)B * C * H * kD * sizeof(__half);
   return ((o + 255) & ~(size_t)255) + (size_t)B * C * H * sizeof(float2);
 }
 
@@ -385,8 +445,8 @@ cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* 
   p.derotate = a.derotate;
   p.out = a.out;
   p.lse = a.lse;
-  const size_t o = (size_t)a.B * p.C * a.H * kD * sizeof(float);
-  p.part_o = reinterpret_cast<float*>(workspace);
+  const size_t o = (size_t)a.B * p.C * a.H * kD * sizeof(__half);
+  p.part_o = reinterpret_cast<__half*>(workspace);
   p.part_ml = reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + ((o + 255) & ~(size_t)255));
   p.dev_status = a.dev_status;
   const size_t smem = at_smem_bytes();
@@ -399,11 +459,10 @@ cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* 
     if (e != cudaSuccess) return e;
     configured = dev;
   }
-  attn_chunk_kernel<<<dim3(p.C, a.B), kAtThreads, smem, stream>>>(qmap, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(attn_chunk_kernel, dim3(p.C, a.B), dim3(kAtThreads), smem, stream,
+                             qmap, p);
   if (e != cudaSuccess) return e;
-  attn_combine_kernel<<<dim3(a.H, a.B), 128, 0, stream>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(attn_combine_kernel, dim3(a.H, a.B), dim3(128), 0, stream, p);
 }
 
 }  // namespace csa

@@ -64,6 +64,8 @@ __global__ void __launch_bounds__(128) compress_kernel(csa_compress_args a, int 
   __shared__ float rot[32][2];
   const int i = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   const int m = a.m;
+  pdl_wait();
+  pdl_trigger();
   const size_t tok0 = (size_t)b * a.T + (size_t)m * i;
   const int d0 = 4 * tid;
 
@@ -153,8 +155,7 @@ cudaError_t launch_compress(const csa_compress_args& a, cudaStream_t stream) {
   const int N = a.T / a.m;
   if (N == 0 || a.B == 0) return cudaSuccess;
   dim3 grid(N, a.B);
-  compress_kernel<<<grid, 128, 0, stream>>>(a, N);
-  return cudaGetLastError();
+  return launch_pdl(compress_kernel, grid, dim3(128), 0, stream, a, N);
 }
 
 }  // namespace csa

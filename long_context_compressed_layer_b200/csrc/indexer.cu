@@ -2,27 +2,39 @@
 // indexer queries score the compressed entries and each query keeps the top-k, one set
 // for all heads; §3.4 and chooseai.net §二: the indexer QK path runs in MXFP4).
 //
-// Kernel 1, indexer_score_kernel: a persistent, warp-specialised stream over the FP4 keys.
+// Kernel 1, indexer_score_kernel: a persistent (one CTA per SM), warp-specialised stream
+// over the FP4 keys.
 //   warp 0      TMA producer: 128-entry key tiles (128 x 64 B, 64-byte swizzle) and the
-//               tile's 512-byte scale group, into an 8-stage shared-memory ring;
+//               tile's 512-byte scale group, into a 12-stage shared-memory ring;
 //   warp 1      tcgen05 issuer: copies the key scales into TMEM (tcgen05.cp), then two
 //               kind::mxf4 block-scaled MMAs (K = 64 each) give D[128 entries x 64 heads]
-//               in fp32 TMEM, double-buffered; it also stages each sequence's FP4 queries
-//               (B operand) and their scales;
-//   warps 2..5  epilogue: one thread per entry reads its 64 head sums from TMEM and forms
-//               s = sum_h w_h * max(0, acc_h) in fp32, writes it to the score workspace
-//               and counts it into a 4096-bin histogram of its order-preserving key.
-// Kernel 2, topk_select_kernel: per sequence, the histogram fixes the bin that holds the
-//   k-th score; CTAs compact the entries above that bin and the candidates inside it; the
-//   last CTA of the sequence (atomic ticket, no spinning) radix-selects the rest by
-//   (score desc, index asc), sorts the set by index and clears the workspace it used.
+//               in fp32 TMEM, four accumulators deep; it also stages each sequence's FP4
+//               queries (B operand) and their scales;
+//   warps 2..9  epilogue, two groups of four (one warp per TMEM lane quadrant) taking
+//               alternate tiles: one thread per entry reads its 64 head sums from TMEM and
+//               forms s = sum_h w_h * max(0, acc_h) in fp32 (w held in registers), writes it
+//               to the score workspace and counts its order-preserving key into the warp's
+//               own 4096-bin histogram (16-bit counters), flushed to the sequence's global
+//               histogram when the warp moves to another sequence.
+// Kernels 2-3, the selection (no sorting anywhere):
+//   topk_threshold_kernel: per sequence and 8192-entry slice, the histogram fixes the bin
+//     that holds the k-th score (a parallel suffix scan); each CTA counts its entries above
+//     that bin and appends the in-bin candidates. The last CTA of a sequence (atomic ticket,
+//     no spinning) resolves the exact cut inside the bin by a radix select on the remaining
+//     20 key bits (ties broken by the smaller index), then turns the per-slice counts into
+//     output offsets and clears the histogram and counters for the next call;
+//   topk_write_kernel: every slice writes its selected entries in index order at its offset,
+//     so the output comes out ascending without a sort.
 #include "common.cuh"
 
 namespace csa {
 
 constexpr int kIxTile = 128;        // entries per tile = MMA M
 constexpr int kIxN = 64;            // MMA N: indexer heads padded to 64
-constexpr int kIxStages = 8;
+constexpr int kIxStages = 12;
+constexpr int kIxAcc = 4;           // TMEM accumulators
+constexpr int kIxEpiWarps = 8;      // two groups of four
+constexpr int kIxThreads = 64 + 32 * kIxEpiWarps;
 constexpr int kIxKeyBytes = kIxTile * 64;
 constexpr int kIxSfBytes = 512;
 constexpr int kHistBits = 12;
@@ -34,30 +46,38 @@ constexpr int kSelThreads = 512;
 struct IxSmem {
   uint8_t keys[kIxStages][kIxKeyBytes];  // 1024-byte aligned tiles
   uint8_t q[2][kIxN * 64];               // queries, 64-byte swizzle, two sequence slots
+  uint32_t hist[kIxEpiWarps][kHist / 2]; // per-warp histograms, two 16-bit bins per word
   uint8_t ksf[kIxStages][kIxSfBytes];
   uint8_t qsf[2][512];
-  float w[kIxN];
-  uint32_t hist[kHist];
   int32_t prefix[kIxMaxB + 1];
   uint64_t full[kIxStages], empty[kIxStages];
-  uint64_t acc_full[2], acc_empty[2], q_free[2], done;
+  uint64_t acc_full[kIxAcc], acc_empty[kIxAcc], q_free[2], done;
   uint32_t tmem_base;
   volatile int abort;
 };
 
 // Workspace layout of csa_indexer_topk (all regions 256-byte aligned).
 struct IxWs {
-  float* scores;       // [B][Nmax]
-  uint32_t* hist;      // [B][kHist]
-  uint32_t* counters;  // [B][4]: selected-above count, candidate count, ticket, spare
-  int32_t* sel;        // [B][k]
-  uint64_t* cand;      // [B][Nmax]
+  float* scores;        // [B][Nmax]
+  uint32_t* hist;       // [B][kHist]
+  uint32_t* counters;   // [B][4]: candidate count, ticket
+  uint32_t* slice_cnt;  // [B][S]: above-bin count per slice, then the slice's output offset
+  uint32_t* rule;       // [B][4]: cut key, cut index, selected count
+  uint64_t* cand;       // [B][Nmax]: (key << 32) | index of the in-bin candidates
+  int S;                // slices per sequence
 };
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
+__host__ __device__ inline int ix_slices(int64_t Nmax) {
+  const int64_t s = (Nmax + kSelChunk - 1) / kSelChunk;
+  return s > 0 ? (int)s : 1;
+}
+
 __host__ __device__ inline size_t ix_ws_layout(int B, int64_t Nmax, int k, char* base,
                                                IxWs* ws) {
+  (void)k;
+  const int S = ix_slices(Nmax);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     char* p = base ? base + off : nullptr;
@@ -67,14 +87,17 @@ __host__ __device__ inline size_t ix_ws_layout(int B, int64_t Nmax, int k, char*
   char* p0 = take((size_t)B * Nmax * 4);
   char* p1 = take((size_t)B * kHist * 4);
   char* p2 = take((size_t)B * 16);
-  char* p3 = take((size_t)B * k * 4);
-  char* p4 = take((size_t)B * Nmax * 8);
+  char* p3 = take((size_t)B * S * 4);
+  char* p4 = take((size_t)B * 16);
+  char* p5 = take((size_t)B * Nmax * 8);
   if (ws) {
     ws->scores = (float*)p0;
     ws->hist = (uint32_t*)p1;
     ws->counters = (uint32_t*)p2;
-    ws->sel = (int32_t*)p3;
-    ws->cand = (uint64_t*)p4;
+    ws->slice_cnt = (uint32_t*)p3;
+    ws->rule = (uint32_t*)p4;
+    ws->cand = (uint64_t*)p5;
+    ws->S = S;
   }
   return off;
 }
@@ -103,12 +126,14 @@ __device__ __forceinline__ int clamp_n(int n, int64_t Nmax, int32_t* st) {
   return n;
 }
 
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kIxThreads, 1)
     indexer_score_kernel(const __grid_constant__ CUtensorMap kmap, IxParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   IxSmem& s = *reinterpret_cast<IxSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  pdl_trigger();
 
   // Tile schedule: sequence b owns ceil(n_b / 128) tiles; CTA c takes a contiguous range.
   if (warp == 0) {
@@ -132,27 +157,30 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&s.full[i], 1);
       mbar_init(&s.empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kIxAcc; ++i) {
       mbar_init(&s.acc_full[i], 1);
       mbar_init(&s.acc_empty[i], 4);
-      mbar_init(&s.q_free[i], 1);
     }
+    for (int i = 0; i < 2; ++i) mbar_init(&s.q_free[i], 1);
     mbar_init(&s.done, 1);
     s.abort = 0;
     mbar_fence_init();
   }
-  for (int i = threadIdx.x; i < kHist; i += blockDim.x) s.hist[i] = 0;
+  {
+    uint32_t* hz = &s.hist[0][0];
+    for (int i = threadIdx.x; i < kIxEpiWarps * kHist / 2; i += blockDim.x) hz[i] = 0;
+  }
   __syncthreads();
   const int total = s.prefix[p.B];
   const int g0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
   const int g1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
   if (g0 >= g1) return;  // uniform across the CTA
-  if (warp == 1) tmem_alloc(&s.tmem_base, 256);
+  if (warp == 1) tmem_alloc(&s.tmem_base, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
-  const uint32_t t_sfa = tmem + 128, t_sfb = tmem + 136;
+  const uint32_t t_sfa = tmem + kIxAcc * kIxN, t_sfb = t_sfa + 8;
 
   // first sequence of this CTA
   int b0 = 0;
@@ -224,8 +252,9 @@ __global__ void __launch_bounds__(192, 1)
         }
       }
       if (lane == 0) {
-        const int st = it % kIxStages, a = it & 1;
-        bool ok = !s.abort && mbar_wait(&s.acc_empty[a], ((it >> 1) & 1) ^ 1, p.dev_status) &&
+        const int st = it % kIxStages, a = it % kIxAcc;
+        bool ok = !s.abort &&
+                  mbar_wait(&s.acc_empty[a], ((it / kIxAcc) & 1) ^ 1, p.dev_status) &&
                   mbar_wait(&s.full[st], (it / kIxStages) & 1, p.dev_status);
         if (!ok) {
           s.abort = 1;
@@ -252,40 +281,41 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int quad = warp & 3;
-    const int row = quad * 32 + lane;
-    int b = -1, n_b = 0, it = 0;
-    auto flush = [&](int bb) {
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+    const int ew = warp - 2;            // 0..7
+    const int grp = ew >> 2;            // tiles with it % 2 == grp
+    const int quad = warp & 3;          // TMEM lane quadrant
+    const int row = quad * 32 + lane;   // entry within the tile
+    uint32_t* hist = s.hist[ew];
+    int b = -1, n_b = 0;
+    float w[kIxN];
+    auto flush = [&](int bb) {  // warp-local: add the warp's counts to the global histogram
+      __syncwarp();
       uint32_t* gh = p.ws.hist + (size_t)bb * kHist;
-      for (int i = threadIdx.x - 64; i < kHist; i += 128) {
-        const uint32_t v = s.hist[i];
+      for (int i = lane; i < kHist / 2; i += 32) {
+        const uint32_t v = hist[i];
         if (v) {
-          atomicAdd(gh + i, v);
-          s.hist[i] = 0;
+          if (v & 0xFFFFu) atomicAdd(gh + 2 * i, v & 0xFFFFu);
+          if (v >> 16) atomicAdd(gh + 2 * i + 1, v >> 16);
+          hist[i] = 0;
         }
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      __syncwarp();
     };
+    int it = 0, bseq = b0;
     for (int g = g0; g < g1; ++g, ++it) {
-      int nb = b < 0 ? b0 : b;
-      while (s.prefix[nb + 1] <= g) ++nb;
-      if (nb != b) {
+      while (s.prefix[bseq + 1] <= g) ++bseq;
+      if ((it & 1) != grp) continue;
+      if (bseq != b) {
         if (b >= 0) flush(b);
-        b = nb;
+        b = bseq;
         n_b = clamp_n(p.n_entries[b], p.Nmax, nullptr);
-        if (threadIdx.x - 64 < kIxN) {
-          const int h = threadIdx.x - 64;
-          s.w[h] = h < p.H_I ? p.w[(size_t)b * p.H_I + h] : 0.f;
-        }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+#pragma unroll
+        for (int h = 0; h < kIxN; ++h) w[h] = h < p.H_I ? __ldg(p.w + (size_t)b * p.H_I + h) : 0.f;
       }
-      const int t = g - s.prefix[b], a = it & 1;
-      // one thread waits for the accumulator; the named barrier hands the outcome to the
-      // other 127, so every epilogue thread takes the same path (no divergent barriers)
-      bool fail = false;
-      if (threadIdx.x == 64) fail = s.abort || !mbar_wait(&s.acc_full[a], (it >> 1) & 1, p.dev_status);
-      if (named_bar_or(1, 128, fail)) {
+      const int t = g - s.prefix[b], a = it % kIxAcc;
+      bool ok = true;
+      if (lane == 0) ok = !s.abort && mbar_wait(&s.acc_full[a], (it / kIxAcc) & 1, p.dev_status);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
         s.abort = 1;
         break;
       }
@@ -300,13 +330,14 @@ __global__ void __launch_bounds__(192, 1)
       if (lane == 0) mbar_arrive(&s.acc_empty[a]);
       float sc = 0.f;
 #pragma unroll
-      for (int h = 0; h < 32; ++h) sc = fmaf(s.w[h], fmaxf(__uint_as_float(r0[h]), 0.f), sc);
+      for (int h = 0; h < 32; ++h) sc = fmaf(w[h], fmaxf(__uint_as_float(r0[h]), 0.f), sc);
 #pragma unroll
-      for (int h = 0; h < 32; ++h) sc = fmaf(s.w[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), sc);
+      for (int h = 0; h < 32; ++h) sc = fmaf(w[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), sc);
       const int j = t * kIxTile + row;
       if (j < n_b) {
         p.ws.scores[(size_t)b * p.Nmax + j] = sc;
-        atomicAdd(&s.hist[float_key(sc) >> (32 - kHistBits)], 1u);
+        const uint32_t bin = float_key(sc) >> (32 - kHistBits);
+        atomicAdd(&hist[bin >> 1], 1u << (16 * (bin & 1)));
       }
     }
     if (b >= 0) flush(b);
@@ -315,7 +346,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 
@@ -330,6 +361,42 @@ struct SelParams {
   int32_t* dev_status;
 };
 
+// Inclusive scan over the 512 threads of a CTA (16 warps); `tmp` holds 16 words.
+__device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  __syncthreads();
+  if (lane == 31) tmp[warp] = v;
+  __syncthreads();
+  uint32_t before = 0, all = 0;
+  for (int w = 0; w < kSelThreads / 32; ++w) {
+    const uint32_t t = tmp[w];
+    if (w < warp) before += t;
+    all += t;
+  }
+  if (total) *total = all;
+  return v + before;
+}
+
+constexpr int kSelPer = kSelChunk / kSelThreads;  // 16 entries per thread
+
+// scores[j .. j+15] (entries at or past `end` read as 0, never touched in memory)
+__device__ __forceinline__ void load_scores16(const float* sc, int j, int end, float (&v)[kSelPer]) {
+  if (j + kSelPer <= end) {
+#pragma unroll
+    for (int q = 0; q < kSelPer / 4; ++q) {
+      const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + j) + q);
+      v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < kSelPer; ++e) v[e] = j + e < end ? __ldcg(sc + j + e) : 0.f;
+  }
+}
+
 __device__ __forceinline__ void warp_append(bool pred, uint32_t* counter, uint32_t* slot_out) {
   const uint32_t m = __ballot_sync(0xffffffffu, pred);
   uint32_t base = 0;
@@ -342,167 +409,269 @@ __device__ __forceinline__ void warp_append(bool pred, uint32_t* counter, uint32
   *slot_out = base + __popc(m & ((1u << lane) - 1));
 }
 
-__global__ void __launch_bounds__(kSelThreads) topk_select_kernel(SelParams p) {
-  __shared__ uint32_t sh_hist[kHist];
-  __shared__ uint32_t part[kSelThreads];
+// Radix-select step over the candidates: among those whose field matches `prefix` under
+// `mask`, histogram the digit (field >> shift) & (2^bits - 1) and find the digit where the
+// running count (from the top when `descending`, else from the bottom) reaches *remaining.
+// Updates *prefix / *remaining (shared). Field: key = cand >> 32 (hi) or index (lo).
+__device__ void radix_step(const uint64_t* cand, uint32_t n_cand, bool hi, uint32_t key_eq,
+                           bool need_key_eq, uint32_t mask, int shift, int bits,
+                           bool descending, uint32_t* prefix, uint32_t* remaining,
+                           uint32_t* h, uint32_t* digit_pop = nullptr) {
+  const int tid = threadIdx.x;
+  const uint32_t nd = 1u << bits;
+  for (uint32_t i = tid; i < 256; i += kSelThreads) h[i] = 0;
+  __syncthreads();
+  const uint32_t pre = *prefix;
+  for (uint32_t i = tid; i < n_cand; i += kSelThreads) {
+    const uint64_t c = __ldcg(cand + i);
+    const uint32_t key = (uint32_t)(c >> 32), ix = (uint32_t)c;
+    if (need_key_eq && key != key_eq) continue;
+    const uint32_t f = hi ? key : ix;
+    if ((f & mask) == pre) atomicAdd(&h[(f >> shift) & (nd - 1)], 1u);
+  }
+  __syncthreads();
+  if (threadIdx.x < 32) {  // one warp: 8 digits per lane, walked in the chosen direction
+    const int lane = threadIdx.x;
+    const int per = (int)(nd + 31) / 32;
+    uint32_t mine = 0;
+    for (int i = 0; i < per; ++i) {
+      const int r = lane * per + i;
+      if (r < (int)nd) mine += h[descending ? nd - 1 - r : r];
+    }
+    uint32_t incl = mine;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t rem = *remaining;
+    const bool cross = incl >= rem && incl - mine < rem;
+    if (cross) {
+      uint32_t cum = incl - mine;
+      for (int i = 0; i < per; ++i) {
+        const int r = lane * per + i;
+        const uint32_t d = descending ? nd - 1 - r : r;
+        if (cum + h[d] >= rem) {
+          *prefix = pre | (d << shift);
+          *remaining = rem - cum;
+          if (digit_pop) *digit_pop = h[d];
+          break;
+        }
+        cum += h[d];
+      }
+    }
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p) {
+  __shared__ uint32_t h[kHist];
+  __shared__ uint32_t tmp[kSelThreads / 32];
   __shared__ int sh_tbin, sh_last;
-  __shared__ uint64_t sh_prefix;
-  __shared__ uint32_t sh_remaining;
-  __shared__ int32_t list[2048];
-  __shared__ uint32_t list_n;
+  __shared__ uint32_t sh_above, sh_prefix, sh_rem, sh_sum, sh_pop;
   const int b = blockIdx.y, sblk = blockIdx.x, tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
   const int n = clamp_n(p.n_entries[b], p.Nmax, p.dev_status);
   const int k_eff = n < p.k ? n : p.k;
   const int S_b = n == 0 ? 1 : (n + kSelChunk - 1) / kSelChunk;
   if (sblk >= S_b) return;
   uint32_t* cnt = p.ws.counters + (size_t)b * 4;
+  uint32_t* scnt = p.ws.slice_cnt + (size_t)b * p.ws.S;
   const float* sc = p.ws.scores + (size_t)b * p.Nmax;
 
-  // 1. threshold bin: the highest bin whose suffix count reaches k
+  // 1. threshold bin: highest bin whose suffix count reaches k (parallel suffix scan)
+  if (tid == 0) { sh_tbin = -1; sh_above = 0; }
   if (n > p.k) {
     const uint32_t* gh = p.ws.hist + (size_t)b * kHist;
-    for (int i = tid; i < kHist; i += kSelThreads) sh_hist[i] = __ldcg(gh + i);
+    for (int i = tid; i < kHist; i += kSelThreads) h[i] = __ldcg(gh + i);
     __syncthreads();
-    constexpr int per = kHist / kSelThreads;  // 8 bins per thread, thread 0 = top bins
+    constexpr int per = kHist / kSelThreads;  // thread 0 holds the top bins
     uint32_t mine = 0;
-    for (int i = 0; i < per; ++i) mine += sh_hist[kHist - 1 - (tid * per + i)];
-    part[tid] = mine;
-    __syncthreads();
-    if (tid == 0) {
-      uint32_t cum = 0;
-      int tb = 0;
-      for (int t = 0; t < kSelThreads; ++t) {
-        if (cum + part[t] >= (uint32_t)p.k) {
-          for (int i = 0; i < per; ++i) {
-            const int bin = kHist - 1 - (t * per + i);
-            if (cum + sh_hist[bin] >= (uint32_t)p.k) { tb = bin; break; }
-            cum += sh_hist[bin];
-          }
-          break;
-        }
-        cum += part[t];
+    for (int i = 0; i < per; ++i) mine += h[kHist - 1 - (tid * per + i)];
+    const uint32_t incl = block_incl_scan(mine, tmp, nullptr);
+    if (incl >= (uint32_t)p.k && incl - mine < (uint32_t)p.k) {
+      uint32_t cum = incl - mine;
+      for (int i = 0; i < per; ++i) {
+        const int bin = kHist - 1 - (tid * per + i);
+        if (cum + h[bin] >= (uint32_t)p.k) { sh_tbin = bin; break; }
+        cum += h[bin];
       }
-      sh_tbin = tb;
     }
-  } else if (tid == 0) {
-    sh_tbin = -1;  // everything is selected
   }
   __syncthreads();
   const int tbin = sh_tbin;
 
-  // 2. compaction of this CTA's slice
+  // 2. this slice: count entries above the bin, append the in-bin candidates. Each thread
+  // owns 16 consecutive entries, loaded as four float4 before any is used.
   const int j0 = sblk * kSelChunk, j1 = min(n, j0 + kSelChunk);
-  for (int base = j0; base < j1; base += kSelThreads) {
-    const int j = base + tid;
+  const int jt = j0 + tid * kSelPer;
+  float v[kSelPer];
+  load_scores16(sc, jt, j1, v);
+  uint32_t above = 0;
+#pragma unroll
+  for (int e = 0; e < kSelPer; ++e) {
+    const int j = jt + e;
     const bool in = j < j1;
-    uint32_t key = 0;
-    int bin = -2;
-    if (in) {
-      key = float_key(__ldcg(sc + j));
-      bin = (int)(key >> (32 - kHistBits));
-    }
-    uint32_t slot;
-    const bool above = in && bin > tbin;
-    warp_append(above, &cnt[0], &slot);
-    if (above) {
-      if (slot < (uint32_t)p.k) p.ws.sel[(size_t)b * p.k + slot] = j;
-      else report(p.dev_status, CSA_ERR_DEVICE);  // histogram and scores disagree
-    }
+    const uint32_t key = float_key(v[e]);
+    const int bin = in ? (int)(key >> (32 - kHistBits)) : -2;
+    above += (in && bin > tbin) ? 1u : 0u;
     const bool eq = in && bin == tbin;
-    warp_append(eq, &cnt[1], &slot);
+    uint32_t slot;
+    warp_append(eq, &cnt[0], &slot);
     if (eq) {
-      if (slot < (uint32_t)p.Nmax)
-        p.ws.cand[(size_t)b * p.Nmax + slot] = ((uint64_t)key << 32) | (0xFFFFFFFFu - (uint32_t)j);
+      if (slot < (uint32_t)p.Nmax) p.ws.cand[(size_t)b * p.Nmax + slot] = ((uint64_t)key << 32) | (uint32_t)j;
       else report(p.dev_status, CSA_ERR_DEVICE);
     }
   }
+  for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+  if ((tid & 31) == 0 && above) atomicAdd(&sh_above, above);
   __syncthreads();
   if (tid == 0) {
+    scnt[sblk] = sh_above;
     __threadfence();
-    sh_last = atomicAdd(&cnt[2], 1u) == (uint32_t)(S_b - 1);
+    sh_last = atomicAdd(&cnt[1], 1u) == (uint32_t)(S_b - 1);
   }
   __syncthreads();
   if (!sh_last) return;
   __threadfence();
 
-  // 3. the last CTA of the sequence finishes the selection
-  uint32_t n_sel = __ldcg(&cnt[0]), n_cand = __ldcg(&cnt[1]);
-  if (n_sel > (uint32_t)p.k) n_sel = (uint32_t)p.k;
+  // 3. the last CTA of the sequence: exact cut inside the bin
+  uint32_t part = 0;
+  for (int s2 = tid; s2 < S_b; s2 += kSelThreads) part += __ldcg(scnt + s2);
+  for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+  if (tid == 0) sh_sum = 0;
+  __syncthreads();
+  if ((tid & 31) == 0 && part) atomicAdd(&sh_sum, part);
+  __syncthreads();
+  const uint32_t above_total = sh_sum;
+  uint32_t n_cand = __ldcg(&cnt[0]);
   if (n_cand > (uint32_t)p.Nmax) n_cand = (uint32_t)p.Nmax;
-  const uint32_t need = (uint32_t)k_eff > n_sel ? (uint32_t)k_eff - n_sel : 0u;
   const uint64_t* cand = p.ws.cand + (size_t)b * p.Nmax;
-  if (n_sel > (uint32_t)k_eff || need > n_cand) report(p.dev_status, CSA_ERR_DEVICE);
-  uint64_t thr = 0;  // composites >= thr are kept
-  if (need > 0 && need < n_cand) {
-    if (tid == 0) { sh_prefix = 0; sh_remaining = need; }
-    uint64_t mask = 0;
-    for (int pass = 7; pass >= 0; --pass) {
-      for (int i = tid; i < 256; i += kSelThreads) sh_hist[i] = 0;
+  // rule: entry j with key is selected iff key > cut_key, or key == cut_key and
+  // j <= cut_idx (a signed index; -1 takes none of the entries at the cut key)
+  uint32_t cut_key;
+  int32_t cut_idx;
+  if (tbin < 0) {  // every entry is selected
+    cut_key = 0u;
+    cut_idx = 0x7FFFFFFF;
+  } else {
+    const uint32_t need = (uint32_t)k_eff > above_total ? (uint32_t)k_eff - above_total : 0u;
+    if (need == 0) {  // the bin contributes nothing
+      cut_key = ((uint32_t)(tbin + 1) << (32 - kHistBits)) - 1u;
+      cut_idx = -1;
+    } else if (need >= n_cand) {  // the whole bin (need > n_cand means inconsistent data)
+      if (need > n_cand) report(p.dev_status, CSA_ERR_DEVICE);
+      cut_key = (uint32_t)tbin << (32 - kHistBits);
+      cut_idx = 0x7FFFFFFF;
+    } else {
+      // key: the need-th largest among the candidates (20 bits below the bin)
+      if (tid == 0) { sh_prefix = (uint32_t)tbin << (32 - kHistBits); sh_rem = need; }
       __syncthreads();
-      const uint64_t pre = sh_prefix;
-      for (uint32_t i = tid; i < n_cand; i += kSelThreads) {
-        const uint64_t c = __ldcg(cand + i);
-        if ((c & mask) == pre) atomicAdd(&sh_hist[(c >> (8 * pass)) & 255], 1u);
+      const uint32_t top = ~0u << (32 - kHistBits);
+      radix_step(cand, n_cand, true, 0, false, top, 12, 8, true, &sh_prefix, &sh_rem, h);
+      radix_step(cand, n_cand, true, 0, false, top | (0xFFu << 12), 4, 8, true, &sh_prefix,
+                 &sh_rem, h);
+      radix_step(cand, n_cand, true, 0, false, top | (0xFFFu << 8) | 0xF0u, 0, 4, true,
+                 &sh_prefix, &sh_rem, h, &sh_pop);
+      cut_key = sh_prefix;
+      // sh_rem entries with key == cut_key are taken, sh_pop exist
+      if (sh_pop == sh_rem) {
+        cut_idx = 0x7FFFFFFF;
+      } else {  // a tie at the cut: the sh_rem smallest indices (4 ascending 8-bit passes)
+        __syncthreads();
+        if (tid == 0) sh_prefix = 0;
+        __syncthreads();
+        radix_step(cand, n_cand, false, cut_key, true, 0u, 24, 8, false, &sh_prefix, &sh_rem, h);
+        radix_step(cand, n_cand, false, cut_key, true, 0xFF000000u, 16, 8, false, &sh_prefix,
+                   &sh_rem, h);
+        radix_step(cand, n_cand, false, cut_key, true, 0xFFFF0000u, 8, 8, false, &sh_prefix,
+                   &sh_rem, h);
+        radix_step(cand, n_cand, false, cut_key, true, 0xFFFFFF00u, 0, 8, false, &sh_prefix,
+                   &sh_rem, h);
+        cut_idx = (int32_t)sh_prefix;
       }
-      __syncthreads();
-      if (tid == 0) {
-        uint32_t cum = 0, rem = sh_remaining;
-        int d = 255;
-        for (; d > 0; --d) {
-          if (cum + sh_hist[d] >= rem) break;
-          cum += sh_hist[d];
-        }
-        sh_prefix = pre | ((uint64_t)d << (8 * pass));
-        sh_remaining = rem - cum;
-      }
-      mask |= (uint64_t)255 << (8 * pass);
-      __syncthreads();
-    }
-    thr = sh_prefix;
-  }
-  if (tid == 0) list_n = 0;
-  __syncthreads();
-  for (uint32_t i = tid; i < n_sel && i < (uint32_t)k_eff; i += kSelThreads)
-    list[i] = __ldcg(p.ws.sel + (size_t)b * p.k + i);
-  if (tid == 0) list_n = n_sel < (uint32_t)k_eff ? n_sel : (uint32_t)k_eff;
-  __syncthreads();
-  if (need > 0) {
-    for (uint32_t i = tid; i < n_cand; i += kSelThreads) {
-      const uint64_t c = __ldcg(cand + i);
-      if (c >= thr) {
-        const uint32_t slot = atomicAdd(&list_n, 1u);
-        if (slot < 2048) list[slot] = (int32_t)(0xFFFFFFFFu - (uint32_t)(c & 0xFFFFFFFFu));
-      }
-    }
-  }
-  __syncthreads();
-  const int cnt_sel = list_n < 2048u ? (int)list_n : 2048;
-  int P2 = 1;
-  while (P2 < p.k) P2 <<= 1;
-  for (int i = cnt_sel + tid; i < P2; i += kSelThreads) list[i] = 0x7FFFFFFF;
-  __syncthreads();
-  for (int size = 2; size <= P2; size <<= 1) {  // bitonic sort, ascending
-    for (int stride = size >> 1; stride > 0; stride >>= 1) {
-      for (int i = tid; i < P2; i += kSelThreads) {
-        const int jx = i ^ stride;
-        if (jx > i) {
-          const bool up = (i & size) == 0;
-          const int x = list[i], y = list[jx];
-          if ((x > y) == up) { list[i] = y; list[jx] = x; }
-        }
-      }
-      __syncthreads();
     }
   }
-  for (int i = tid; i < p.k; i += kSelThreads) {
-    const int v = i < cnt_sel ? list[i] : -1;
-    p.idx[(size_t)b * p.k + i] = v;
-    if (p.scores_out) p.scores_out[(size_t)b * p.k + i] = v >= 0 ? __ldcg(sc + v) : __int_as_float(0x7fc00000);
+  // selected count per slice: above-bin entries plus the candidates that pass the cut
+  for (uint32_t i = tid; i < n_cand; i += kSelThreads) {
+    const uint64_t c = __ldcg(cand + i);
+    const uint32_t key = (uint32_t)(c >> 32), j = (uint32_t)c;
+    if (tbin >= 0 && (key > cut_key || (key == cut_key && (int32_t)j <= cut_idx)))
+      atomicAdd(scnt + j / kSelChunk, 1u);
   }
-  // 4. leave the workspace zeroed for the next call
+  __threadfence();
+  __syncthreads();
+  // exclusive scan of the slice counts -> output offsets
+  uint32_t carry = 0;
+  for (int base = 0; base < S_b; base += kSelThreads) {
+    const int s2 = base + tid;
+    const uint32_t v = s2 < S_b ? __ldcg(scnt + s2) : 0u;
+    uint32_t tot;
+    const uint32_t incl = block_incl_scan(v, tmp, &tot);
+    if (s2 < S_b) scnt[s2] = carry + incl - v;
+    carry += tot;
+    __syncthreads();
+  }
+  if (tid == 0) {
+    uint32_t* r = p.ws.rule + (size_t)b * 4;
+    r[0] = cut_key;
+    r[1] = (uint32_t)cut_idx;
+    r[2] = (uint32_t)k_eff;
+    if (carry != (uint32_t)k_eff) report(p.dev_status, CSA_ERR_DEVICE);
+    cnt[0] = 0;
+    cnt[1] = 0;
+  }
   uint32_t* gh = p.ws.hist + (size_t)b * kHist;
   for (int i = tid; i < kHist; i += kSelThreads) gh[i] = 0;
-  if (tid < 4) cnt[tid] = 0;
+}
+
+__global__ void __launch_bounds__(kSelThreads) topk_write_kernel(SelParams p) {
+  __shared__ uint32_t tmp[kSelThreads / 32];
+  const int b = blockIdx.y, sblk = blockIdx.x, tid = threadIdx.x;
+  pdl_wait();
+  pdl_trigger();
+  int n = p.n_entries[b];
+  n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
+  const int S_b = n == 0 ? 1 : (n + kSelChunk - 1) / kSelChunk;
+  if (sblk >= S_b) return;
+  const uint32_t* r = p.ws.rule + (size_t)b * 4;
+  const uint32_t cut_key = __ldcg(r), k_eff = __ldcg(r + 2);
+  const int32_t cut_idx = (int32_t)__ldcg(r + 1);
+  const uint32_t off = __ldcg(p.ws.slice_cnt + (size_t)b * p.ws.S + sblk);
+  const float* sc = p.ws.scores + (size_t)b * p.Nmax;
+  int32_t* out = p.idx + (size_t)b * p.k;
+  const int j0 = sblk * kSelChunk, j1 = min(n, j0 + kSelChunk);
+  const int jt = j0 + tid * kSelPer;  // 16 consecutive entries per thread
+  float v[kSelPer];
+  load_scores16(sc, jt, j1, v);
+  uint32_t mask = 0;
+#pragma unroll
+  for (int e = 0; e < kSelPer; ++e) {
+    const int j = jt + e;
+    const uint32_t key = float_key(v[e]);
+    if (j < j1 && (key > cut_key || (key == cut_key && j <= cut_idx))) mask |= 1u << e;
+  }
+  const uint32_t mine = __popc(mask);
+  const uint32_t incl = block_incl_scan(mine, tmp, nullptr);
+  uint32_t slot = off + incl - mine;
+#pragma unroll
+  for (int e = 0; e < kSelPer; ++e) {
+    if (mask & (1u << e)) {
+      if (slot < (uint32_t)p.k) {
+        out[slot] = jt + e;
+        if (p.scores_out) p.scores_out[(size_t)b * p.k + slot] = v[e];
+      } else {
+        report(p.dev_status, CSA_ERR_DEVICE);
+      }
+      ++slot;
+    }
+  }
+  if (sblk == 0) {
+    for (int i = (int)k_eff + tid; i < p.k; i += kSelThreads) {
+      out[i] = -1;
+      if (p.scores_out) p.scores_out[(size_t)b * p.k + i] = __int_as_float(0x7fc00000);
+    }
+  }
 }
 
 // ------------------------------------------------------------------- launch
@@ -522,16 +691,16 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
     configured = dev;
   }
   const int64_t tiles_max = (int64_t)a.B * (a.Nmax / kIxTile);
-  int grid = 2 * num_sms;
+  int grid = num_sms;
   if (tiles_max < grid) grid = (int)(tiles_max > 0 ? tiles_max : 1);
-  indexer_score_kernel<<<grid, 192, smem, stream>>>(kmap, p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(indexer_score_kernel, dim3(grid), dim3(kIxThreads), smem, stream,
+                             kmap, p);
   if (e != cudaSuccess) return e;
   SelParams sp{a.B, a.k, a.Nmax, a.n_entries, ws, a.idx, a.scores, a.dev_status};
-  const int64_t chunks = (a.Nmax + kSelChunk - 1) / kSelChunk;
-  dim3 g2((unsigned)(chunks > 0 ? chunks : 1), a.B);
-  topk_select_kernel<<<g2, kSelThreads, 0, stream>>>(sp);
-  return cudaGetLastError();
+  dim3 g2((unsigned)ws.S, a.B);
+  e = launch_pdl(topk_threshold_kernel, g2, dim3(kSelThreads), 0, stream, sp);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(topk_write_kernel, g2, dim3(kSelThreads), 0, stream, sp);
 }
 
 size_t ix_smem_bytes() { return sizeof(IxSmem) + 1024; }

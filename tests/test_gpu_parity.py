@@ -120,6 +120,29 @@ def test_indexer_scores_exact_on_integer_case():
     np.testing.assert_array_equal(sc[:1000], ora[0, :1000])
 
 
+@pytest.mark.parametrize("k", [1, 100, 777, 2048])
+def test_indexer_exact_ties_keep_smaller_indices(k):
+    # unit scales, w = 1, every query element 1.0 and key elements 0 or 1: each score is
+    # 16 x (an integer dot <= 128), so the cut falls inside a group of exactly equal scores
+    # and must keep the smaller indices (no tolerance here)
+    B, H_I, Nmax = 1, 16, 5120
+    rng = np.random.default_rng(k)
+    n = np.array([5000], np.int32)
+    ix = synth.indexer_inputs(rng, B, H_I, Nmax, n)
+    ix["q_sf"][:] = 127
+    ix["k_sf"][:] = 127
+    ix["w"][:] = 1.0
+    ix["q_fp4"][:] = 0x22
+    ix["k_fp4"][:] = rng.choice(np.array([0x00, 0x02, 0x20, 0x22], np.uint8), size=ix["k_fp4"].shape)
+    ora = oracle.indexer_scores(n, ix["q_fp4"], ix["q_sf"], ix["w"], ix["k_fp4"], ix["k_sf"])
+    s = ora[0, :5000]
+    assert len(np.unique(s)) <= 129  # the case really is tie-heavy
+    want = oracle.topk(ora[0], 5000, k)
+    idx = csa.indexer_topk(dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]),
+                           dev(ix["k_fp4"]), dev(ix["k_sf"]), k)
+    np.testing.assert_array_equal(host(idx)[0], want)
+
+
 def test_indexer_workspace_stays_clean_across_calls():
     B, H_I, Nmax, k = 2, 64, 2048, 256
     rng = np.random.default_rng(4)
