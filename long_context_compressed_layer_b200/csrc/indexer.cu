@@ -31,10 +31,21 @@ namespace csa {
 
 constexpr int kIxTile = 128;        // entries per tile = MMA M
 constexpr int kIxN = 64;            // MMA N: indexer heads padded to 64
-constexpr int kIxStages = 12;
-constexpr int kIxAcc = 4;           // TMEM accumulators
-constexpr int kIxEpiWarps = 8;      // two groups of four
+#ifndef CSA_IX_CTAS_PER_SM
+#define CSA_IX_CTAS_PER_SM 2
+#endif
+constexpr int kIxCtasPerSm = CSA_IX_CTAS_PER_SM;
+// Two CTAs per SM give every SM two independent TMA producers and tcgen05 issuers; each
+// CTA then owns half of TMEM (256 columns) and about half of shared memory.
+constexpr int kIxStages = kIxCtasPerSm == 2 ? 7 : 12;
+constexpr int kIxBatch = kIxCtasPerSm == 2 ? 1 : 3;  // tiles per accumulator handshake
+constexpr int kIxNbuf = kIxCtasPerSm == 2 ? 3 : 2;   // accumulator batches in flight
+constexpr int kIxAcc = kIxNbuf * kIxBatch;           // TMEM accumulators of 64 columns
+constexpr int kIxEpiWarps = kIxCtasPerSm == 2 ? 4 : 8;  // groups of four (one per quadrant)
+constexpr int kIxGroups = kIxEpiWarps / 4;
+constexpr int kIxTmemCols = kIxCtasPerSm == 2 ? 256 : 512;
 constexpr int kIxThreads = 64 + 32 * kIxEpiWarps;
+static_assert(kIxAcc * 64 + 16 <= kIxTmemCols, "accumulators and scale factors fit TMEM");
 constexpr int kIxKeyBytes = kIxTile * 64;
 constexpr int kIxSfBytes = 512;
 constexpr int kHistBits = 12;
@@ -51,7 +62,7 @@ struct IxSmem {
   uint8_t qsf[2][512];
   int32_t prefix[kIxMaxB + 1];
   uint64_t full[kIxStages], empty[kIxStages];
-  uint64_t acc_full[kIxAcc], acc_empty[kIxAcc], q_free[2], done;
+  uint64_t acc_full[kIxNbuf], acc_empty[kIxNbuf], q_free[2], done;
   uint32_t tmem_base;
   volatile int abort;
 };
@@ -126,12 +137,33 @@ __device__ __forceinline__ int clamp_n(int n, int64_t Nmax, int32_t* st) {
   return n;
 }
 
-__global__ void __launch_bounds__(kIxThreads, 1)
+__global__ void __launch_bounds__(kIxThreads, kIxCtasPerSm)
     indexer_score_kernel(const __grid_constant__ CUtensorMap kmap, IxParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   IxSmem& s = *reinterpret_cast<IxSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // set-up that touches no global memory overlaps the previous kernel's tail
+  if (threadIdx.x == 32) {
+    for (int i = 0; i < kIxStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < kIxNbuf; ++i) {
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_empty[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) mbar_init(&s.q_free[i], 1);
+    mbar_init(&s.done, 1);
+    s.abort = 0;
+    mbar_fence_init();
+  }
+  if (threadIdx.x == 0) prefetch_tensormap(&kmap);
+  {
+    uint32_t* hz = &s.hist[0][0];
+    for (int i = threadIdx.x; i < kIxEpiWarps * kHist / 2; i += blockDim.x) hz[i] = 0;
+  }
+  if (warp == 1) tmem_alloc(&s.tmem_base, kIxTmemCols);
   pdl_wait();
   pdl_trigger();
 
@@ -152,34 +184,17 @@ __global__ void __launch_bounds__(kIxThreads, 1)
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
-  if (threadIdx.x == 32) {
-    for (int i = 0; i < kIxStages; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], 1);
-    }
-    for (int i = 0; i < kIxAcc; ++i) {
-      mbar_init(&s.acc_full[i], 1);
-      mbar_init(&s.acc_empty[i], 4);
-    }
-    for (int i = 0; i < 2; ++i) mbar_init(&s.q_free[i], 1);
-    mbar_init(&s.done, 1);
-    s.abort = 0;
-    mbar_fence_init();
-  }
-  {
-    uint32_t* hz = &s.hist[0][0];
-    for (int i = threadIdx.x; i < kIxEpiWarps * kHist / 2; i += blockDim.x) hz[i] = 0;
-  }
-  __syncthreads();
-  const int total = s.prefix[p.B];
-  const int g0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
-  const int g1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
-  if (g0 >= g1) return;  // uniform across the CTA
-  if (warp == 1) tmem_alloc(&s.tmem_base, 512);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  const int total = s.prefix[p.B];
+  const int g0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
+  const int g1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
   const uint32_t tmem = s.tmem_base;
+  if (g0 >= g1) {  // uniform across the CTA: nothing to score
+    if (warp == 1) tmem_dealloc(tmem, kIxTmemCols);
+    return;
+  }
   const uint32_t t_sfa = tmem + kIxAcc * kIxN, t_sfb = t_sfa + 8;
 
   // first sequence of this CTA
@@ -189,7 +204,6 @@ __global__ void __launch_bounds__(kIxThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      prefetch_tensormap(&kmap);
       int b = b0, it = 0;
       for (int g = g0; g < g1; ++g, ++it) {
         while (s.prefix[b + 1] <= g) ++b;
@@ -252,14 +266,20 @@ __global__ void __launch_bounds__(kIxThreads, 1)
         }
       }
       if (lane == 0) {
-        const int st = it % kIxStages, a = it % kIxAcc;
-        bool ok = !s.abort &&
-                  mbar_wait(&s.acc_empty[a], ((it / kIxAcc) & 1) ^ 1, p.dev_status) &&
-                  mbar_wait(&s.full[st], (it / kIxStages) & 1, p.dev_status);
+        // tile it goes to accumulator a of batch bt = it / kIxBatch, buffer bb
+        const int st = it % kIxStages, bt = it / kIxBatch, bb = bt % kIxNbuf;
+        const int a = bb * kIxBatch + it % kIxBatch;
+        bool ok = !s.abort;
+        if (ok && it % kIxBatch == 0) {  // first tile of a batch: its buffer must be free
+          ok = mbar_wait(&s.acc_empty[bb], ((bt / kIxNbuf) & 1) ^ 1, p.dev_status);
+          // the epilogue's TMEM reads of this buffer happen before our MMAs overwrite it
+          tc_fence_after();
+        }
+        // (the key tile arrives through the async proxy: the barrier alone orders it)
+        ok = ok && mbar_wait(&s.full[st], (it / kIxStages) & 1, p.dev_status);
         if (!ok) {
           s.abort = 1;
         } else {
-          tc_fence_after();
           tmem_cp_32x128b_x4(t_sfa, smem_desc(smem_u32(s.ksf[st]), 0, 128, kSwizzleNone));
           const uint32_t ka = smem_u32(s.keys[st]), qa = smem_u32(s.q[qslot]);
 #pragma unroll
@@ -269,7 +289,8 @@ __global__ void __launch_bounds__(kIxThreads, 1)
                      idesc_mxf4(kIxTile, kIxN, 2 * kh), t_sfa, t_sfb, kh);
           }
           mma_commit(&s.empty[st]);
-          mma_commit(&s.acc_full[a]);
+          // last tile of the batch (or of this CTA): hand the batch to the epilogue
+          if (it % kIxBatch == kIxBatch - 1 || g + 1 == g1) mma_commit(&s.acc_full[bb]);
         }
       }
       if (__shfl_sync(0xffffffffu, s.abort, 0)) break;
@@ -282,11 +303,11 @@ __global__ void __launch_bounds__(kIxThreads, 1)
   } else {
     // ---------------------------------------------------------------- epilogue
     const int ew = warp - 2;            // 0..7
-    const int grp = ew >> 2;            // tiles with it % 2 == grp
+    const int grp = ew >> 2;            // takes the batches bt with bt % kIxGroups == grp
     const int quad = warp & 3;          // TMEM lane quadrant
     const int row = quad * 32 + lane;   // entry within the tile
     uint32_t* hist = s.hist[ew];
-    int b = -1, n_b = 0;
+    int b = -1, n_b = 0, since_flush = 0;
     float w[kIxN];
     auto flush = [&](int bb) {  // warp-local: add the warp's counts to the global histogram
       __syncwarp();
@@ -301,44 +322,59 @@ __global__ void __launch_bounds__(kIxThreads, 1)
       }
       __syncwarp();
     };
-    int it = 0, bseq = b0;
-    for (int g = g0; g < g1; ++g, ++it) {
-      while (s.prefix[bseq + 1] <= g) ++bseq;
-      if ((it & 1) != grp) continue;
-      if (bseq != b) {
-        if (b >= 0) flush(b);
-        b = bseq;
-        n_b = clamp_n(p.n_entries[b], p.Nmax, nullptr);
-#pragma unroll
-        for (int h = 0; h < kIxN; ++h) w[h] = h < p.H_I ? __ldg(p.w + (size_t)b * p.H_I + h) : 0.f;
-      }
-      const int t = g - s.prefix[b], a = it % kIxAcc;
+    // batch bt holds tiles kIxBatch*bt .. of this CTA; group grp takes bt % kIxGroups == grp
+    const int ntiles = g1 - g0;
+    int bseq = b0;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    for (int bt = grp; bt * kIxBatch < ntiles; bt += kIxGroups) {
+      const int bb = bt % kIxNbuf;
       bool ok = true;
-      if (lane == 0) ok = !s.abort && mbar_wait(&s.acc_full[a], (it / kIxAcc) & 1, p.dev_status);
+      if (lane == 0) ok = !s.abort && mbar_wait(&s.acc_full[bb], (bt / kIxNbuf) & 1, p.dev_status);
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         s.abort = 1;
         break;
       }
       tc_fence_after();
-      uint32_t r0[32], r1[32];
-      const uint32_t taddr = tmem + ((uint32_t)(quad * 32) << 16) + a * kIxN;
-      tmem_ld32(taddr, r0);
-      tmem_ld32(taddr + 32, r1);
-      tmem_ld_wait();
+      const int it0 = bt * kIxBatch, it_end = min(ntiles, it0 + kIxBatch);
+      for (int it = it0; it < it_end; ++it) {
+        const int g = g0 + it;
+        while (s.prefix[bseq + 1] <= g) ++bseq;
+        // 16-bit counters: a warp adds at most 32 counts per tile, so flush every 2000
+        // tiles (< 65536 counts) as well as whenever the sequence changes
+        if (bseq != b || since_flush == 2000) {
+          if (b >= 0) flush(b);
+          since_flush = 0;
+          b = bseq;
+          n_b = clamp_n(p.n_entries[b], p.Nmax, nullptr);
+#pragma unroll
+          for (int h = 0; h < kIxN; ++h) w[h] = h < p.H_I ? __ldg(p.w + (size_t)b * p.H_I + h) : 0.f;
+        }
+        ++since_flush;
+        uint32_t r[2][32];
+        const uint32_t ta = lane_base + (bb * kIxBatch + (it - it0)) * kIxN;
+        tmem_ld32(ta, r[0]);
+        tmem_ld32(ta + 32, r[1]);
+        tmem_ld_wait();
+        // s = sum_h w_h * max(0, acc_h): eight independent partial sums (heads h = k mod 8)
+        // combined in a fixed tree, so the FMA latency chain is 8 deep instead of 64
+        float part[8];
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) part[k8] = 0.f;
+#pragma unroll
+        for (int h = 0; h < kIxN; ++h)
+          part[h & 7] = fmaf(w[h], fmaxf(__uint_as_float(r[h >> 5][h & 31]), 0.f), part[h & 7]);
+        const float sc = ((part[0] + part[1]) + (part[2] + part[3])) +
+                         ((part[4] + part[5]) + (part[6] + part[7]));
+        const int j = (g - s.prefix[b]) * kIxTile + row;
+        if (j < n_b) {
+          p.ws.scores[(size_t)b * p.Nmax + j] = sc;
+          const uint32_t bin = float_key(sc) >> (32 - kHistBits);
+          atomicAdd(&hist[bin >> 1], 1u << (16 * (bin & 1)));
+        }
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.acc_empty[a]);
-      float sc = 0.f;
-#pragma unroll
-      for (int h = 0; h < 32; ++h) sc = fmaf(w[h], fmaxf(__uint_as_float(r0[h]), 0.f), sc);
-#pragma unroll
-      for (int h = 0; h < 32; ++h) sc = fmaf(w[32 + h], fmaxf(__uint_as_float(r1[h]), 0.f), sc);
-      const int j = t * kIxTile + row;
-      if (j < n_b) {
-        p.ws.scores[(size_t)b * p.Nmax + j] = sc;
-        const uint32_t bin = float_key(sc) >> (32 - kHistBits);
-        atomicAdd(&hist[bin >> 1], 1u << (16 * (bin & 1)));
-      }
+      if (lane == 0) mbar_arrive(&s.acc_empty[bb]);
     }
     if (b >= 0) flush(b);
   }
@@ -346,7 +382,7 @@ __global__ void __launch_bounds__(kIxThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kIxTmemCols);
   }
 }
 
@@ -413,7 +449,14 @@ __device__ __forceinline__ void warp_append(bool pred, uint32_t* counter, uint32
 // `mask`, histogram the digit (field >> shift) & (2^bits - 1) and find the digit where the
 // running count (from the top when `descending`, else from the bottom) reaches *remaining.
 // Updates *prefix / *remaining (shared). Field: key = cand >> 32 (hi) or index (lo).
-__device__ void radix_step(const uint64_t* cand, uint32_t n_cand, bool hi, uint32_t key_eq,
+// Candidates come from shared memory (staged) or, past its capacity, from global memory.
+__device__ __forceinline__ uint64_t cand_at(const uint64_t* cand, uint32_t i, bool staged) {
+  return staged ? cand[i] : __ldcg(cand + i);
+}
+
+constexpr uint32_t kCandStage = 2048;
+
+__device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, bool hi, uint32_t key_eq,
                            bool need_key_eq, uint32_t mask, int shift, int bits,
                            bool descending, uint32_t* prefix, uint32_t* remaining,
                            uint32_t* h, uint32_t* digit_pop = nullptr) {
@@ -423,7 +466,7 @@ __device__ void radix_step(const uint64_t* cand, uint32_t n_cand, bool hi, uint3
   __syncthreads();
   const uint32_t pre = *prefix;
   for (uint32_t i = tid; i < n_cand; i += kSelThreads) {
-    const uint64_t c = __ldcg(cand + i);
+    const uint64_t c = cand_at(cand, i, staged);
     const uint32_t key = (uint32_t)(c >> 32), ix = (uint32_t)c;
     if (need_key_eq && key != key_eq) continue;
     const uint32_t f = hi ? key : ix;
@@ -468,6 +511,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p
   __shared__ uint32_t tmp[kSelThreads / 32];
   __shared__ int sh_tbin, sh_last;
   __shared__ uint32_t sh_above, sh_prefix, sh_rem, sh_sum, sh_pop;
+  __shared__ uint64_t cand_s[kCandStage];
   const int b = blockIdx.y, sblk = blockIdx.x, tid = threadIdx.x;
   pdl_wait();
   pdl_trigger();
@@ -547,6 +591,12 @@ __global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p
   uint32_t n_cand = __ldcg(&cnt[0]);
   if (n_cand > (uint32_t)p.Nmax) n_cand = (uint32_t)p.Nmax;
   const uint64_t* cand = p.ws.cand + (size_t)b * p.Nmax;
+  const bool staged = n_cand <= kCandStage;
+  if (staged) {
+    for (uint32_t i = tid; i < n_cand; i += kSelThreads) cand_s[i] = __ldcg(cand + i);
+    cand = cand_s;
+    __syncthreads();
+  }
   // rule: entry j with key is selected iff key > cut_key, or key == cut_key and
   // j <= cut_idx (a signed index; -1 takes none of the entries at the cut key)
   uint32_t cut_key;
@@ -568,10 +618,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p
       if (tid == 0) { sh_prefix = (uint32_t)tbin << (32 - kHistBits); sh_rem = need; }
       __syncthreads();
       const uint32_t top = ~0u << (32 - kHistBits);
-      radix_step(cand, n_cand, true, 0, false, top, 12, 8, true, &sh_prefix, &sh_rem, h);
-      radix_step(cand, n_cand, true, 0, false, top | (0xFFu << 12), 4, 8, true, &sh_prefix,
+      radix_step(cand, staged, n_cand, true, 0, false, top, 12, 8, true, &sh_prefix, &sh_rem, h);
+      radix_step(cand, staged, n_cand, true, 0, false, top | (0xFFu << 12), 4, 8, true, &sh_prefix,
                  &sh_rem, h);
-      radix_step(cand, n_cand, true, 0, false, top | (0xFFFu << 8) | 0xF0u, 0, 4, true,
+      radix_step(cand, staged, n_cand, true, 0, false, top | (0xFFFu << 8) | 0xF0u, 0, 4, true,
                  &sh_prefix, &sh_rem, h, &sh_pop);
       cut_key = sh_prefix;
       // sh_rem entries with key == cut_key are taken, sh_pop exist
@@ -581,12 +631,12 @@ __global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p
         __syncthreads();
         if (tid == 0) sh_prefix = 0;
         __syncthreads();
-        radix_step(cand, n_cand, false, cut_key, true, 0u, 24, 8, false, &sh_prefix, &sh_rem, h);
-        radix_step(cand, n_cand, false, cut_key, true, 0xFF000000u, 16, 8, false, &sh_prefix,
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0u, 24, 8, false, &sh_prefix, &sh_rem, h);
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFF000000u, 16, 8, false, &sh_prefix,
                    &sh_rem, h);
-        radix_step(cand, n_cand, false, cut_key, true, 0xFFFF0000u, 8, 8, false, &sh_prefix,
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFFFF0000u, 8, 8, false, &sh_prefix,
                    &sh_rem, h);
-        radix_step(cand, n_cand, false, cut_key, true, 0xFFFFFF00u, 0, 8, false, &sh_prefix,
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFFFFFF00u, 0, 8, false, &sh_prefix,
                    &sh_rem, h);
         cut_idx = (int32_t)sh_prefix;
       }
@@ -594,7 +644,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p
   }
   // selected count per slice: above-bin entries plus the candidates that pass the cut
   for (uint32_t i = tid; i < n_cand; i += kSelThreads) {
-    const uint64_t c = __ldcg(cand + i);
+    const uint64_t c = cand_at(cand, i, staged);
     const uint32_t key = (uint32_t)(c >> 32), j = (uint32_t)c;
     if (tbin >= 0 && (key > cut_key || (key == cut_key && (int32_t)j <= cut_idx)))
       atomicAdd(scnt + j / kSelChunk, 1u);
@@ -691,7 +741,7 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
     configured = dev;
   }
   const int64_t tiles_max = (int64_t)a.B * (a.Nmax / kIxTile);
-  int grid = num_sms;
+  int grid = kIxCtasPerSm * num_sms;
   if (tiles_max < grid) grid = (int)(tiles_max > 0 ? tiles_max : 1);
   cudaError_t e = launch_pdl(indexer_score_kernel, dim3(grid), dim3(kIxThreads), smem, stream,
                              kmap, p);
