@@ -31,40 +31,47 @@ namespace csa {
 
 constexpr int kIxTile = 128;        // entries per tile = MMA M
 constexpr int kIxN = 64;            // MMA N: indexer heads padded to 64
-#ifndef CSA_IX_CTAS_PER_SM
-#define CSA_IX_CTAS_PER_SM 2
-#endif
-constexpr int kIxCtasPerSm = CSA_IX_CTAS_PER_SM;
-// Two CTAs per SM give every SM two independent TMA producers and tcgen05 issuers; each
-// CTA then owns half of TMEM (256 columns) and about half of shared memory.
-constexpr int kIxStages = kIxCtasPerSm == 2 ? 7 : 12;
-constexpr int kIxBatch = kIxCtasPerSm == 2 ? 1 : 3;  // tiles per accumulator handshake
-constexpr int kIxNbuf = kIxCtasPerSm == 2 ? 3 : 2;   // accumulator batches in flight
-constexpr int kIxAcc = kIxNbuf * kIxBatch;           // TMEM accumulators of 64 columns
-constexpr int kIxEpiWarps = kIxCtasPerSm == 2 ? 4 : 8;  // groups of four (one per quadrant)
-constexpr int kIxGroups = kIxEpiWarps / 4;
-constexpr int kIxTmemCols = kIxCtasPerSm == 2 ? 256 : 512;
-constexpr int kIxThreads = 64 + 32 * kIxEpiWarps;
-static_assert(kIxAcc * 64 + 16 <= kIxTmemCols, "accumulators and scale factors fit TMEM");
+// One CTA per SM holding two independent pipelines (each: a TMA producer warp, a tcgen05
+// issuer warp and four epilogue warps, its own shared-memory ring and half of TMEM), so
+// that every SM streams with two producers and two issuers while the whole grid stays
+// resident for the cooperative launch that also runs the selection.
+constexpr int kIxPipes = 2;
+constexpr int kIxStages = 6;        // key tiles in flight per pipeline
+constexpr int kIxBatch = 1;         // tiles per accumulator hand-off
+constexpr int kIxNbuf = 3;          // accumulator buffers per pipeline
+constexpr int kIxAcc = kIxNbuf * kIxBatch;
+constexpr int kIxEpiWarps = 4;      // per pipeline, one per TMEM lane quadrant
+constexpr int kIxGroups = 1;
+constexpr int kIxPipeWarps = 2 + kIxEpiWarps;
+constexpr int kIxPipeCols = 256;    // TMEM columns per pipeline
+constexpr int kIxTmemCols = kIxPipes * kIxPipeCols;
+constexpr int kIxThreads = 32 * kIxPipeWarps * kIxPipes;
+static_assert(kIxAcc * 64 + 16 <= kIxPipeCols, "accumulators and scale factors fit TMEM");
 constexpr int kIxKeyBytes = kIxTile * 64;
 constexpr int kIxSfBytes = 512;
-constexpr int kHistBits = 12;
+constexpr int kHistBits = 11;       // histogram of the top key bits (sign, exponent, 2 mantissa)
+constexpr int kLowBits = 32 - kHistBits;
 constexpr int kHist = 1 << kHistBits;
 constexpr int kIxMaxB = 1024;
-constexpr int kSelChunk = 8192;     // entries per select CTA
-constexpr int kSelThreads = 512;
+constexpr int kSelThreads = kIxThreads;     // the selection runs on the scoring CTAs
+constexpr int kSelPer = 32;                 // consecutive entries per thread
+constexpr int kSelChunk = kSelThreads * kSelPer;  // entries per slice
 
-struct IxSmem {
+struct alignas(1024) PipeSmem {
   uint8_t keys[kIxStages][kIxKeyBytes];  // 1024-byte aligned tiles
   uint8_t q[2][kIxN * 64];               // queries, 64-byte swizzle, two sequence slots
   uint32_t hist[kIxEpiWarps][kHist / 2]; // per-warp histograms, two 16-bit bins per word
   uint8_t ksf[kIxStages][kIxSfBytes];
   uint8_t qsf[2][512];
-  int32_t prefix[kIxMaxB + 1];
   uint64_t full[kIxStages], empty[kIxStages];
   uint64_t acc_full[kIxNbuf], acc_empty[kIxNbuf], q_free[2], done;
-  uint32_t tmem_base;
   volatile int abort;
+};
+
+struct IxSmem {
+  PipeSmem pipe[kIxPipes];
+  int32_t prefix[kIxMaxB + 1];
+  uint32_t tmem_base;
 };
 
 // Workspace layout of csa_indexer_topk (all regions 256-byte aligned).
@@ -72,6 +79,7 @@ struct IxWs {
   float* scores;        // [B][Nmax]
   uint32_t* hist;       // [B][kHist]
   uint32_t* counters;   // [B][4]: candidate count, ticket
+  uint32_t* grid_bar;   // [2]: arrival count, generation (grid-wide barrier)
   uint32_t* slice_cnt;  // [B][S]: above-bin count per slice, then the slice's output offset
   uint32_t* rule;       // [B][4]: cut key, cut index, selected count
   uint64_t* cand;       // [B][Nmax]: (key << 32) | index of the in-bin candidates
@@ -97,7 +105,7 @@ __host__ __device__ inline size_t ix_ws_layout(int B, int64_t Nmax, int k, char*
   };
   char* p0 = take((size_t)B * Nmax * 4);
   char* p1 = take((size_t)B * kHist * 4);
-  char* p2 = take((size_t)B * 16);
+  char* p2 = take((size_t)B * 16 + 8);
   char* p3 = take((size_t)B * S * 4);
   char* p4 = take((size_t)B * 16);
   char* p5 = take((size_t)B * Nmax * 8);
@@ -105,6 +113,7 @@ __host__ __device__ inline size_t ix_ws_layout(int B, int64_t Nmax, int k, char*
     ws->scores = (float*)p0;
     ws->hist = (uint32_t*)p1;
     ws->counters = (uint32_t*)p2;
+    ws->grid_bar = (uint32_t*)(p2 + (size_t)B * 16);
     ws->slice_cnt = (uint32_t*)p3;
     ws->rule = (uint32_t*)p4;
     ws->cand = (uint64_t*)p5;
@@ -118,7 +127,8 @@ size_t ix_workspace_size(int B, int64_t Nmax, int k) {
 }
 
 struct IxParams {
-  int B, H_I;
+  int B, H_I, k;
+  int fused;  // 1: the selection follows in this (cooperative) launch
   int64_t Nmax;
   const int32_t* n_entries;
   const uint8_t* q_fp4;
@@ -126,6 +136,8 @@ struct IxParams {
   const float* w;
   const uint8_t* k_sf;
   IxWs ws;
+  int32_t* idx;
+  float* scores_out;
   int32_t* dev_status;
 };
 
@@ -137,31 +149,41 @@ __device__ __forceinline__ int clamp_n(int n, int64_t Nmax, int32_t* st) {
   return n;
 }
 
-__global__ void __launch_bounds__(kIxThreads, kIxCtasPerSm)
+__device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
+                                            const CUtensorMap& kmap, const IxParams& p,
+                                            const int g0, const int g1, const uint32_t tmem,
+                                            const uint32_t t_sfa, const uint32_t t_sfb,
+                                            const int wp);
+__device__ void select_fused(const IxParams& p, uint8_t* scratch);
+
+__global__ void __launch_bounds__(kIxThreads, 1)
     indexer_score_kernel(const __grid_constant__ CUtensorMap kmap, IxParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   IxSmem& s = *reinterpret_cast<IxSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int pi = warp / kIxPipeWarps, wp = warp % kIxPipeWarps;  // pipeline, warp in it
+  PipeSmem& ps = s.pipe[pi];
   // set-up that touches no global memory overlaps the previous kernel's tail
-  if (threadIdx.x == 32) {
+  if (wp == 1 && lane == 0) {
     for (int i = 0; i < kIxStages; ++i) {
-      mbar_init(&s.full[i], 1);
-      mbar_init(&s.empty[i], 1);
+      mbar_init(&ps.full[i], 1);
+      mbar_init(&ps.empty[i], 1);
     }
     for (int i = 0; i < kIxNbuf; ++i) {
-      mbar_init(&s.acc_full[i], 1);
-      mbar_init(&s.acc_empty[i], 4);
+      mbar_init(&ps.acc_full[i], 1);
+      mbar_init(&ps.acc_empty[i], kIxEpiWarps);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&s.q_free[i], 1);
-    mbar_init(&s.done, 1);
-    s.abort = 0;
+    for (int i = 0; i < 2; ++i) mbar_init(&ps.q_free[i], 1);
+    mbar_init(&ps.done, 1);
+    ps.abort = 0;
     mbar_fence_init();
   }
   if (threadIdx.x == 0) prefetch_tensormap(&kmap);
   {
-    uint32_t* hz = &s.hist[0][0];
-    for (int i = threadIdx.x; i < kIxEpiWarps * kHist / 2; i += blockDim.x) hz[i] = 0;
+    uint32_t* hz = &ps.hist[0][0];
+    for (int i = threadIdx.x % (32 * kIxPipeWarps); i < kIxEpiWarps * kHist / 2; i += 32 * kIxPipeWarps)
+      hz[i] = 0;
   }
   if (warp == 1) tmem_alloc(&s.tmem_base, kIxTmemCols);
   pdl_wait();
@@ -191,23 +213,42 @@ __global__ void __launch_bounds__(kIxThreads, kIxCtasPerSm)
   const int g0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
   const int g1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
   const uint32_t tmem = s.tmem_base;
-  if (g0 >= g1) {  // uniform across the CTA: nothing to score
-    if (warp == 1) tmem_dealloc(tmem, kIxTmemCols);
-    return;
+  {  // the pipelines split the CTA's tiles into two contiguous halves
+    const int gm = g0 + (g1 - g0 + 1) / 2;
+    const int pg0 = pi == 0 ? g0 : gm, pg1 = pi == 0 ? gm : g1;
+    const uint32_t tp = tmem + pi * kIxPipeCols;
+    const uint32_t t_sfa = tp + kIxAcc * kIxN, t_sfb = t_sfa + 8;
+    if (pg0 < pg1) score_roles(ps, s.prefix, kmap, p, pg0, pg1, tp, t_sfa, t_sfb, wp);
   }
-  const uint32_t t_sfa = tmem + kIxAcc * kIxN, t_sfb = t_sfa + 8;
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kIxTmemCols);
+  }
+  if (p.fused) select_fused(p, reinterpret_cast<uint8_t*>(&s.pipe[0].keys[0][0]));
+}
+
+// The three warp roles of one pipeline over its tiles [g0, g1); wp is the warp's index in
+// the pipeline (0 producer, 1 tcgen05 issuer, 2.. epilogue).
+__device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
+                                            const CUtensorMap& kmap, const IxParams& p,
+                                            const int g0, const int g1, const uint32_t tmem,
+                                            const uint32_t t_sfa, const uint32_t t_sfb,
+                                            const int wp) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // first sequence of this CTA
   int b0 = 0;
-  while (s.prefix[b0 + 1] <= g0) ++b0;
+  while (prefix[b0 + 1] <= g0) ++b0;
 
-  if (warp == 0) {
+  if (wp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
       int b = b0, it = 0;
       for (int g = g0; g < g1; ++g, ++it) {
-        while (s.prefix[b + 1] <= g) ++b;
-        const int t = g - s.prefix[b];
+        while (prefix[b + 1] <= g) ++b;
+        const int t = g - prefix[b];
         const int st = it % kIxStages;
         if (s.abort || !mbar_wait(&s.empty[st], ((it / kIxStages) & 1) ^ 1, p.dev_status)) {
           s.abort = 1;
@@ -223,13 +264,13 @@ __global__ void __launch_bounds__(kIxThreads, kIxCtasPerSm)
       for (int i = issued - kIxStages < 0 ? 0 : issued - kIxStages; i < issued; ++i)
         mbar_wait(&s.full[i % kIxStages], (i / kIxStages) & 1, p.dev_status);
     }
-  } else if (warp == 1) {
+  } else if (wp == 1) {
     // ---------------------------------------------------------------- MMA issuer
     int b = -1, nseq = -1, it = 0;
     uint32_t qslot = 0;
     for (int g = g0; g < g1; ++g, ++it) {
       int nb = b < 0 ? b0 : b;
-      while (s.prefix[nb + 1] <= g) ++nb;
+      while (prefix[nb + 1] <= g) ++nb;
       if (nb != b) {  // stage this sequence's queries (B operand) and their scales
         if (b >= 0 && lane == 0) mma_commit(&s.q_free[qslot]);
         b = nb;
@@ -302,7 +343,7 @@ __global__ void __launch_bounds__(kIxThreads, kIxCtasPerSm)
     __syncwarp();
   } else {
     // ---------------------------------------------------------------- epilogue
-    const int ew = warp - 2;            // 0..7
+    const int ew = wp - 2;              // epilogue warp of this pipeline
     const int grp = ew >> 2;            // takes the batches bt with bt % kIxGroups == grp
     const int quad = warp & 3;          // TMEM lane quadrant
     const int row = quad * 32 + lane;   // entry within the tile
@@ -338,7 +379,7 @@ __global__ void __launch_bounds__(kIxThreads, kIxCtasPerSm)
       const int it0 = bt * kIxBatch, it_end = min(ntiles, it0 + kIxBatch);
       for (int it = it0; it < it_end; ++it) {
         const int g = g0 + it;
-        while (s.prefix[bseq + 1] <= g) ++bseq;
+        while (prefix[bseq + 1] <= g) ++bseq;
         // 16-bit counters: a warp adds at most 32 counts per tile, so flush every 2000
         // tiles (< 65536 counts) as well as whenever the sequence changes
         if (bseq != b || since_flush == 2000) {
@@ -365,7 +406,7 @@ __global__ void __launch_bounds__(kIxThreads, kIxCtasPerSm)
           part[h & 7] = fmaf(w[h], fmaxf(__uint_as_float(r[h >> 5][h & 31]), 0.f), part[h & 7]);
         const float sc = ((part[0] + part[1]) + (part[2] + part[3])) +
                          ((part[4] + part[5]) + (part[6] + part[7]));
-        const int j = (g - s.prefix[b]) * kIxTile + row;
+        const int j = (g - prefix[b]) * kIxTile + row;
         if (j < n_b) {
           p.ws.scores[(size_t)b * p.Nmax + j] = sc;
           const uint32_t bin = float_key(sc) >> (32 - kHistBits);
@@ -378,27 +419,23 @@ __global__ void __launch_bounds__(kIxThreads, kIxCtasPerSm)
     }
     if (b >= 0) flush(b);
   }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kIxTmemCols);
-  }
 }
 
 // ------------------------------------------------------------------- select
-struct SelParams {
-  int B, k;
-  int64_t Nmax;
-  const int32_t* n_entries;
-  IxWs ws;
-  int32_t* idx;
-  float* scores_out;
-  int32_t* dev_status;
+// Shared-memory scratch of the selection, carved from the (then idle) key ring.
+struct SelScratch {
+  uint32_t h[kHist];
+  uint64_t cand[2048];
+  uint32_t tmp[32];
+  int tbin, last;
+  uint32_t above, prefix, rem, sum, pop;
 };
+static_assert(sizeof(SelScratch) <= sizeof(uint8_t[kIxStages][kIxKeyBytes]), "scratch fits the ring");
+constexpr uint32_t kCandStage = 2048;
 
-// Inclusive scan over the 512 threads of a CTA (16 warps); `tmp` holds 16 words.
+// Inclusive scan over the CTA (kSelThreads threads); tmp holds one word per warp.
 __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
+  constexpr int nw = kSelThreads / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
@@ -408,7 +445,8 @@ __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* tmp, u
   if (lane == 31) tmp[warp] = v;
   __syncthreads();
   uint32_t before = 0, all = 0;
-  for (int w = 0; w < kSelThreads / 32; ++w) {
+#pragma unroll
+  for (int w = 0; w < nw; ++w) {
     const uint32_t t = tmp[w];
     if (w < warp) before += t;
     all += t;
@@ -417,10 +455,9 @@ __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* tmp, u
   return v + before;
 }
 
-constexpr int kSelPer = kSelChunk / kSelThreads;  // 16 entries per thread
-
-// scores[j .. j+15] (entries at or past `end` read as 0, never touched in memory)
-__device__ __forceinline__ void load_scores16(const float* sc, int j, int end, float (&v)[kSelPer]) {
+// scores[j .. j+31] (entries at or past `end` read as 0 and are never used)
+__device__ __forceinline__ void load_scores(const float* sc, int j, int end,
+                                            float (&v)[kSelPer]) {
   if (j + kSelPer <= end) {
 #pragma unroll
     for (int q = 0; q < kSelPer / 4; ++q) {
@@ -445,20 +482,18 @@ __device__ __forceinline__ void warp_append(bool pred, uint32_t* counter, uint32
   *slot_out = base + __popc(m & ((1u << lane) - 1));
 }
 
-// Radix-select step over the candidates: among those whose field matches `prefix` under
-// `mask`, histogram the digit (field >> shift) & (2^bits - 1) and find the digit where the
-// running count (from the top when `descending`, else from the bottom) reaches *remaining.
-// Updates *prefix / *remaining (shared). Field: key = cand >> 32 (hi) or index (lo).
 // Candidates come from shared memory (staged) or, past its capacity, from global memory.
 __device__ __forceinline__ uint64_t cand_at(const uint64_t* cand, uint32_t i, bool staged) {
   return staged ? cand[i] : __ldcg(cand + i);
 }
 
-constexpr uint32_t kCandStage = 2048;
-
-__device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, bool hi, uint32_t key_eq,
-                           bool need_key_eq, uint32_t mask, int shift, int bits,
-                           bool descending, uint32_t* prefix, uint32_t* remaining,
+// Radix-select step over the candidates: among those whose field matches `prefix` under
+// `mask`, histogram the digit (field >> shift) & (2^bits - 1) and find the digit where the
+// running count (from the top when `descending`, else from the bottom) reaches *remaining.
+// Updates *prefix / *remaining (shared). Field: key = cand >> 32 (hi) or index (lo).
+__device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, bool hi,
+                           uint32_t key_eq, bool need_key_eq, uint32_t mask, int shift,
+                           int bits, bool descending, uint32_t* prefix, uint32_t* remaining,
                            uint32_t* h, uint32_t* digit_pop = nullptr) {
   const int tid = threadIdx.x;
   const uint32_t nd = 1u << bits;
@@ -473,7 +508,7 @@ __device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, b
     if ((f & mask) == pre) atomicAdd(&h[(f >> shift) & (nd - 1)], 1u);
   }
   __syncthreads();
-  if (threadIdx.x < 32) {  // one warp: 8 digits per lane, walked in the chosen direction
+  if (threadIdx.x < 32) {  // one warp: nd/32 digits per lane, walked in the chosen direction
     const int lane = threadIdx.x;
     const int per = (int)(nd + 31) / 32;
     uint32_t mine = 0;
@@ -487,8 +522,7 @@ __device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, b
       if (lane >= o) incl += y;
     }
     const uint32_t rem = *remaining;
-    const bool cross = incl >= rem && incl - mine < rem;
-    if (cross) {
+    if (incl >= rem && incl - mine < rem) {
       uint32_t cum = incl - mine;
       for (int i = 0; i < per; ++i) {
         const int r = lane * per + i;
@@ -506,51 +540,103 @@ __device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, b
   __syncthreads();
 }
 
-__global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p) {
-  __shared__ uint32_t h[kHist];
-  __shared__ uint32_t tmp[kSelThreads / 32];
-  __shared__ int sh_tbin, sh_last;
-  __shared__ uint32_t sh_above, sh_prefix, sh_rem, sh_sum, sh_pop;
-  __shared__ uint64_t cand_s[kCandStage];
-  const int b = blockIdx.y, sblk = blockIdx.x, tid = threadIdx.x;
-  pdl_wait();
-  pdl_trigger();
+__device__ __forceinline__ int slices_of(int n) {
+  return n == 0 ? 1 : (n + kSelChunk - 1) / kSelChunk;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Grid-wide barrier of a cooperative launch (all CTAs resident), bounded in time. The
+// arrival is a release and the wait an acquire, so the writes of every CTA before the
+// barrier are visible to every CTA after it. Returns false after a timeout; *gen_out gets
+// the generation this barrier completed (the same value in every CTA).
+__device__ bool grid_barrier(uint32_t* bar, uint32_t nblocks, int32_t* dev_status,
+                             uint32_t* gen_out) {
+  __shared__ uint32_t sh_gen;
+  __syncthreads();
+  bool ok = true;
+  if (threadIdx.x == 0) {
+    const uint32_t my_gen = ld_acquire(bar + 1);
+    uint32_t old;
+    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(bar) : "memory");
+    if (old == nblocks - 1) {
+      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(bar) : "memory");
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar + 1) : "memory");
+    } else {
+      const uint64_t t0 = globaltimer();
+      while (ld_acquire(bar + 1) == my_gen) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
+          report(dev_status, CSA_ERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+      }
+    }
+    sh_gen = my_gen + 1;
+  }
+  ok = __syncthreads_and(ok) != 0;
+  *gen_out = sh_gen;
+  return ok;
+}
+
+// Phase 1 of the selection for slice sb of sequence b: the threshold bin (highest bin whose
+// suffix count reaches k), the slice's count above it and its in-bin candidates. The last
+// slice of the sequence to finish resolves the exact cut (finalize).
+__device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb,
+                                 uint32_t ready_gen) {
+  const int tid = threadIdx.x;
   const int n = clamp_n(p.n_entries[b], p.Nmax, p.dev_status);
   const int k_eff = n < p.k ? n : p.k;
-  const int S_b = n == 0 ? 1 : (n + kSelChunk - 1) / kSelChunk;
-  if (sblk >= S_b) return;
+  const int S_b = slices_of(n);
   uint32_t* cnt = p.ws.counters + (size_t)b * 4;
   uint32_t* scnt = p.ws.slice_cnt + (size_t)b * p.ws.S;
   const float* sc = p.ws.scores + (size_t)b * p.Nmax;
 
-  // 1. threshold bin: highest bin whose suffix count reaches k (parallel suffix scan)
-  if (tid == 0) { sh_tbin = -1; sh_above = 0; }
+  if (tid == 0) { x.tbin = -1; x.above = 0; }
   if (n > p.k) {
-    const uint32_t* gh = p.ws.hist + (size_t)b * kHist;
-    for (int i = tid; i < kHist; i += kSelThreads) h[i] = __ldcg(gh + i);
+    const uint4* gh = reinterpret_cast<const uint4*>(p.ws.hist + (size_t)b * kHist);
+    constexpr int nv = kHist / 4, vper = (nv + kSelThreads - 1) / kSelThreads;
+    uint4 hv[vper];  // every load in flight before any is stored
+#pragma unroll
+    for (int i = 0; i < vper; ++i) {
+      const int q = tid + i * kSelThreads;
+      hv[i] = q < nv ? __ldcg(gh + q) : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int i = 0; i < vper; ++i) {
+      const int q = tid + i * kSelThreads;
+      if (q < nv) reinterpret_cast<uint4*>(x.h)[q] = hv[i];
+    }
     __syncthreads();
-    constexpr int per = kHist / kSelThreads;  // thread 0 holds the top bins
+    constexpr int per = (kHist + kSelThreads - 1) / kSelThreads;  // thread 0 holds the top
     uint32_t mine = 0;
-    for (int i = 0; i < per; ++i) mine += h[kHist - 1 - (tid * per + i)];
-    const uint32_t incl = block_incl_scan(mine, tmp, nullptr);
+    for (int i = 0; i < per; ++i) {
+      const int r = tid * per + i;
+      if (r < kHist) mine += x.h[kHist - 1 - r];
+    }
+    const uint32_t incl = block_incl_scan(mine, x.tmp, nullptr);
     if (incl >= (uint32_t)p.k && incl - mine < (uint32_t)p.k) {
       uint32_t cum = incl - mine;
       for (int i = 0; i < per; ++i) {
-        const int bin = kHist - 1 - (tid * per + i);
-        if (cum + h[bin] >= (uint32_t)p.k) { sh_tbin = bin; break; }
-        cum += h[bin];
+        const int r = tid * per + i;
+        if (r >= kHist) break;
+        const int bin = kHist - 1 - r;
+        if (cum + x.h[bin] >= (uint32_t)p.k) { x.tbin = bin; break; }
+        cum += x.h[bin];
       }
     }
   }
   __syncthreads();
-  const int tbin = sh_tbin;
+  const int tbin = x.tbin;
 
-  // 2. this slice: count entries above the bin, append the in-bin candidates. Each thread
-  // owns 16 consecutive entries, loaded as four float4 before any is used.
-  const int j0 = sblk * kSelChunk, j1 = min(n, j0 + kSelChunk);
+  const int j0 = sb * kSelChunk, j1 = min(n, j0 + kSelChunk);
   const int jt = j0 + tid * kSelPer;
   float v[kSelPer];
-  load_scores16(sc, jt, j1, v);
+  load_scores(sc, jt, j1, v);
   uint32_t above = 0;
 #pragma unroll
   for (int e = 0; e < kSelPer; ++e) {
@@ -568,33 +654,45 @@ __global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p
     }
   }
   for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
-  if ((tid & 31) == 0 && above) atomicAdd(&sh_above, above);
+  if ((tid & 31) == 0 && above) atomicAdd(&x.above, above);
   __syncthreads();
   if (tid == 0) {
-    scnt[sblk] = sh_above;
+    scnt[sb] = x.above;
     __threadfence();
-    sh_last = atomicAdd(&cnt[1], 1u) == (uint32_t)(S_b - 1);
+    x.last = atomicAdd(&cnt[1], 1u) == (uint32_t)(S_b - 1);
   }
   __syncthreads();
-  if (!sh_last) return;
+  if (!x.last) return;
   __threadfence();
 
-  // 3. the last CTA of the sequence: exact cut inside the bin
+  // ---- finalize: the exact cut inside the bin, per-slice output offsets, workspace reset
   uint32_t part = 0;
   for (int s2 = tid; s2 < S_b; s2 += kSelThreads) part += __ldcg(scnt + s2);
   for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
-  if (tid == 0) sh_sum = 0;
+  if (tid == 0) x.sum = 0;
   __syncthreads();
-  if ((tid & 31) == 0 && part) atomicAdd(&sh_sum, part);
+  if ((tid & 31) == 0 && part) atomicAdd(&x.sum, part);
   __syncthreads();
-  const uint32_t above_total = sh_sum;
+  const uint32_t above_total = x.sum;
   uint32_t n_cand = __ldcg(&cnt[0]);
   if (n_cand > (uint32_t)p.Nmax) n_cand = (uint32_t)p.Nmax;
   const uint64_t* cand = p.ws.cand + (size_t)b * p.Nmax;
   const bool staged = n_cand <= kCandStage;
   if (staged) {
-    for (uint32_t i = tid; i < n_cand; i += kSelThreads) cand_s[i] = __ldcg(cand + i);
-    cand = cand_s;
+    for (uint32_t base = 0; base < n_cand; base += 8 * kSelThreads) {
+      uint64_t cv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t i = base + tid + u * kSelThreads;
+        cv[u] = i < n_cand ? __ldcg(cand + i) : 0ull;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const uint32_t i = base + tid + u * kSelThreads;
+        if (i < n_cand) x.cand[i] = cv[u];
+      }
+    }
+    cand = x.cand;
     __syncthreads();
   }
   // rule: entry j with key is selected iff key > cut_key, or key == cut_key and
@@ -607,38 +705,40 @@ __global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p
   } else {
     const uint32_t need = (uint32_t)k_eff > above_total ? (uint32_t)k_eff - above_total : 0u;
     if (need == 0) {  // the bin contributes nothing
-      cut_key = ((uint32_t)(tbin + 1) << (32 - kHistBits)) - 1u;
+      cut_key = ((uint32_t)(tbin + 1) << kLowBits) - 1u;
       cut_idx = -1;
     } else if (need >= n_cand) {  // the whole bin (need > n_cand means inconsistent data)
       if (need > n_cand) report(p.dev_status, CSA_ERR_DEVICE);
-      cut_key = (uint32_t)tbin << (32 - kHistBits);
+      cut_key = (uint32_t)tbin << kLowBits;
       cut_idx = 0x7FFFFFFF;
     } else {
-      // key: the need-th largest among the candidates (20 bits below the bin)
-      if (tid == 0) { sh_prefix = (uint32_t)tbin << (32 - kHistBits); sh_rem = need; }
+      // key: the need-th largest among the candidates (the kLowBits below the bin), in
+      // digits of 8, 8 and kLowBits - 16 bits
+      if (tid == 0) { x.prefix = (uint32_t)tbin << kLowBits; x.rem = need; }
       __syncthreads();
-      const uint32_t top = ~0u << (32 - kHistBits);
-      radix_step(cand, staged, n_cand, true, 0, false, top, 12, 8, true, &sh_prefix, &sh_rem, h);
-      radix_step(cand, staged, n_cand, true, 0, false, top | (0xFFu << 12), 4, 8, true, &sh_prefix,
-                 &sh_rem, h);
-      radix_step(cand, staged, n_cand, true, 0, false, top | (0xFFFu << 8) | 0xF0u, 0, 4, true,
-                 &sh_prefix, &sh_rem, h, &sh_pop);
-      cut_key = sh_prefix;
-      // sh_rem entries with key == cut_key are taken, sh_pop exist
-      if (sh_pop == sh_rem) {
+      const uint32_t top = ~0u << kLowBits;
+      radix_step(cand, staged, n_cand, true, 0, false, top, kLowBits - 8, 8, true, &x.prefix,
+                 &x.rem, x.h);
+      radix_step(cand, staged, n_cand, true, 0, false, ~0u << (kLowBits - 8), kLowBits - 16, 8,
+                 true, &x.prefix, &x.rem, x.h);
+      radix_step(cand, staged, n_cand, true, 0, false, ~0u << (kLowBits - 16), 0, kLowBits - 16,
+                 true, &x.prefix, &x.rem, x.h, &x.pop);
+      cut_key = x.prefix;
+      if (x.pop == x.rem) {  // x.rem entries with key == cut_key are taken, x.pop exist
         cut_idx = 0x7FFFFFFF;
-      } else {  // a tie at the cut: the sh_rem smallest indices (4 ascending 8-bit passes)
+      } else {  // a tie at the cut: the x.rem smallest indices (4 ascending 8-bit passes)
         __syncthreads();
-        if (tid == 0) sh_prefix = 0;
+        if (tid == 0) x.prefix = 0;
         __syncthreads();
-        radix_step(cand, staged, n_cand, false, cut_key, true, 0u, 24, 8, false, &sh_prefix, &sh_rem, h);
-        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFF000000u, 16, 8, false, &sh_prefix,
-                   &sh_rem, h);
-        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFFFF0000u, 8, 8, false, &sh_prefix,
-                   &sh_rem, h);
-        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFFFFFF00u, 0, 8, false, &sh_prefix,
-                   &sh_rem, h);
-        cut_idx = (int32_t)sh_prefix;
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0u, 24, 8, false, &x.prefix,
+                   &x.rem, x.h);
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFF000000u, 16, 8, false,
+                   &x.prefix, &x.rem, x.h);
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFFFF0000u, 8, 8, false,
+                   &x.prefix, &x.rem, x.h);
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFFFFFF00u, 0, 8, false,
+                   &x.prefix, &x.rem, x.h);
+        cut_idx = (int32_t)x.prefix;
       }
     }
   }
@@ -655,10 +755,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p
   uint32_t carry = 0;
   for (int base = 0; base < S_b; base += kSelThreads) {
     const int s2 = base + tid;
-    const uint32_t v = s2 < S_b ? __ldcg(scnt + s2) : 0u;
+    const uint32_t vv = s2 < S_b ? __ldcg(scnt + s2) : 0u;
     uint32_t tot;
-    const uint32_t incl = block_incl_scan(v, tmp, &tot);
-    if (s2 < S_b) scnt[s2] = carry + incl - v;
+    const uint32_t incl = block_incl_scan(vv, x.tmp, &tot);
+    if (s2 < S_b) scnt[s2] = carry + incl - vv;
     carry += tot;
     __syncthreads();
   }
@@ -673,27 +773,31 @@ __global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(SelParams p
   }
   uint32_t* gh = p.ws.hist + (size_t)b * kHist;
   for (int i = tid; i < kHist; i += kSelThreads) gh[i] = 0;
+  __syncthreads();
+  if (tid == 0 && p.fused) {  // publish the rule and offsets of this sequence
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.ws.rule + (size_t)b * 4 + 3),
+                 "r"(ready_gen)
+                 : "memory");
+  }
+  __threadfence();
+  __syncthreads();
 }
 
-__global__ void __launch_bounds__(kSelThreads) topk_write_kernel(SelParams p) {
-  __shared__ uint32_t tmp[kSelThreads / 32];
-  const int b = blockIdx.y, sblk = blockIdx.x, tid = threadIdx.x;
-  pdl_wait();
-  pdl_trigger();
+// Phase 2: slice sb of sequence b writes its selected entries, in index order, at its offset.
+__device__ void select_write(const IxParams& p, SelScratch& x, int b, int sb) {
+  const int tid = threadIdx.x;
   int n = p.n_entries[b];
   n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
-  const int S_b = n == 0 ? 1 : (n + kSelChunk - 1) / kSelChunk;
-  if (sblk >= S_b) return;
   const uint32_t* r = p.ws.rule + (size_t)b * 4;
   const uint32_t cut_key = __ldcg(r), k_eff = __ldcg(r + 2);
   const int32_t cut_idx = (int32_t)__ldcg(r + 1);
-  const uint32_t off = __ldcg(p.ws.slice_cnt + (size_t)b * p.ws.S + sblk);
+  const uint32_t off = __ldcg(p.ws.slice_cnt + (size_t)b * p.ws.S + sb);
   const float* sc = p.ws.scores + (size_t)b * p.Nmax;
   int32_t* out = p.idx + (size_t)b * p.k;
-  const int j0 = sblk * kSelChunk, j1 = min(n, j0 + kSelChunk);
-  const int jt = j0 + tid * kSelPer;  // 16 consecutive entries per thread
+  const int j0 = sb * kSelChunk, j1 = min(n, j0 + kSelChunk);
+  const int jt = j0 + tid * kSelPer;
   float v[kSelPer];
-  load_scores16(sc, jt, j1, v);
+  load_scores(sc, jt, j1, v);
   uint32_t mask = 0;
 #pragma unroll
   for (int e = 0; e < kSelPer; ++e) {
@@ -702,7 +806,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_write_kernel(SelParams p) {
     if (j < j1 && (key > cut_key || (key == cut_key && j <= cut_idx))) mask |= 1u << e;
   }
   const uint32_t mine = __popc(mask);
-  const uint32_t incl = block_incl_scan(mine, tmp, nullptr);
+  const uint32_t incl = block_incl_scan(mine, x.tmp, nullptr);
   uint32_t slot = off + incl - mine;
 #pragma unroll
   for (int e = 0; e < kSelPer; ++e) {
@@ -716,12 +820,73 @@ __global__ void __launch_bounds__(kSelThreads) topk_write_kernel(SelParams p) {
       ++slot;
     }
   }
-  if (sblk == 0) {
+  if (sb == 0) {
     for (int i = (int)k_eff + tid; i < p.k; i += kSelThreads) {
       out[i] = -1;
       if (p.scores_out) p.scores_out[(size_t)b * p.k + i] = __int_as_float(0x7fc00000);
     }
   }
+  __syncthreads();
+}
+
+// The selection inside the cooperative scoring launch: every CTA takes the slices
+// i = blockIdx.x, + gridDim.x, ... of the (sequence, slice) grid.
+__device__ void select_fused(const IxParams& p, uint8_t* scratch) {
+  SelScratch& x = *reinterpret_cast<SelScratch*>(scratch);
+  uint32_t gen;
+  if (!grid_barrier(p.ws.grid_bar, gridDim.x, p.dev_status, &gen)) return;
+  // the barrier generation is new in every call, so a flag left by an earlier call (or the
+  // zero-filled workspace) never matches it
+  const uint32_t ready_gen = gen;
+  const int items = p.B * p.ws.S;
+  for (int i = blockIdx.x; i < items; i += gridDim.x) {
+    const int b = i / p.ws.S, sb = i % p.ws.S;
+    int n = p.n_entries[b];
+    n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
+    if (sb < slices_of(n)) select_threshold(p, x, b, sb, ready_gen);
+  }
+  // phase 2 needs only its own sequence's rule: wait for its publication, not for the grid
+  for (int i = blockIdx.x; i < items; i += gridDim.x) {
+    const int b = i / p.ws.S, sb = i % p.ws.S;
+    int n = p.n_entries[b];
+    n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
+    if (sb >= slices_of(n)) continue;
+    bool ok = true;
+    if (threadIdx.x == 0) {
+      const uint64_t t0 = globaltimer();
+      while (ld_acquire(p.ws.rule + (size_t)b * 4 + 3) != ready_gen) {
+        if (globaltimer() - t0 > kWaitLimitNs) {
+          report(p.dev_status, CSA_ERR_TIMEOUT);
+          ok = false;
+          break;
+        }
+      }
+    }
+    if (!__syncthreads_and(ok)) return;
+    select_write(p, x, b, sb);
+  }
+}
+
+// Stand-alone selection kernels (when a cooperative launch is not available): one CTA per
+// (slice, sequence).
+__global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(IxParams p) {
+  __shared__ __align__(16) uint8_t raw[sizeof(SelScratch)];
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.y, sb = blockIdx.x;
+  int n = p.n_entries[b];
+  n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
+  if (sb < slices_of(n)) select_threshold(p, *reinterpret_cast<SelScratch*>(raw), b, sb, 0u);
+}
+
+__global__ void __launch_bounds__(kSelThreads) topk_write_kernel(IxParams p) {
+  __shared__ __align__(16) uint8_t raw[sizeof(SelScratch)];
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.y, sb = blockIdx.x;
+  int n = p.n_entries[b];
+  n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
+  if (sb < slices_of(n)) select_write(p, *reinterpret_cast<SelScratch*>(raw), b, sb);
 }
 
 // ------------------------------------------------------------------- launch
@@ -729,7 +894,8 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
                                 const CUtensorMap& kmap, cudaStream_t stream) {
   IxWs ws;
   ix_ws_layout(a.B, a.Nmax, a.k, (char*)workspace, &ws);
-  IxParams p{a.B, a.H_I, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws, a.dev_status};
+  IxParams p{a.B, a.H_I, a.k, 1, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
+             a.idx, a.scores, a.dev_status};
   const size_t smem = sizeof(IxSmem) + 1024;
   static int configured = -1;
   int dev = 0;
@@ -738,19 +904,40 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
     cudaError_t e = cudaFuncSetAttribute(indexer_score_kernel,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    // the whole carveout as shared memory, so two CTAs fit on an SM
+    e = cudaFuncSetAttribute(indexer_score_kernel,
+                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
     configured = dev;
   }
+  // Scoring and selection in one cooperative launch (every CTA resident, so the grid
+  // barrier between the phases always completes); the runtime refuses a grid that cannot
+  // be resident, and the selection then runs as two further kernels.
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(kIxThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  cfg.gridDim = dim3(num_sms);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, indexer_score_kernel, kmap, p);
+  if (e == cudaSuccess) return cudaSuccess;
+  (void)cudaGetLastError();
+  p.fused = 0;
   const int64_t tiles_max = (int64_t)a.B * (a.Nmax / kIxTile);
-  int grid = kIxCtasPerSm * num_sms;
+  int grid = num_sms;
   if (tiles_max < grid) grid = (int)(tiles_max > 0 ? tiles_max : 1);
-  cudaError_t e = launch_pdl(indexer_score_kernel, dim3(grid), dim3(kIxThreads), smem, stream,
-                             kmap, p);
+  e = launch_pdl(indexer_score_kernel, dim3(grid), dim3(kIxThreads), smem, stream, kmap, p);
   if (e != cudaSuccess) return e;
-  SelParams sp{a.B, a.k, a.Nmax, a.n_entries, ws, a.idx, a.scores, a.dev_status};
   dim3 g2((unsigned)ws.S, a.B);
-  e = launch_pdl(topk_threshold_kernel, g2, dim3(kSelThreads), 0, stream, sp);
+  e = launch_pdl(topk_threshold_kernel, g2, dim3(kSelThreads), 0, stream, p);
   if (e != cudaSuccess) return e;
-  return launch_pdl(topk_write_kernel, g2, dim3(kSelThreads), 0, stream, sp);
+  return launch_pdl(topk_write_kernel, g2, dim3(kSelThreads), 0, stream, p);
 }
 
 size_t ix_smem_bytes() { return sizeof(IxSmem) + 1024; }
