@@ -544,45 +544,6 @@ __device__ __forceinline__ int slices_of(int n) {
   return n == 0 ? 1 : (n + kSelChunk - 1) / kSelChunk;
 }
 
-__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
-  uint32_t v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Grid-wide barrier of a cooperative launch (all CTAs resident), bounded in time. The
-// arrival is a release and the wait an acquire, so the writes of every CTA before the
-// barrier are visible to every CTA after it. Returns false after a timeout; *gen_out gets
-// the generation this barrier completed (the same value in every CTA).
-__device__ bool grid_barrier(uint32_t* bar, uint32_t nblocks, int32_t* dev_status,
-                             uint32_t* gen_out) {
-  __shared__ uint32_t sh_gen;
-  __syncthreads();
-  bool ok = true;
-  if (threadIdx.x == 0) {
-    const uint32_t my_gen = ld_acquire(bar + 1);
-    uint32_t old;
-    asm volatile("atom.add.release.gpu.global.u32 %0, [%1], 1;" : "=r"(old) : "l"(bar) : "memory");
-    if (old == nblocks - 1) {
-      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(bar) : "memory");
-      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar + 1) : "memory");
-    } else {
-      const uint64_t t0 = globaltimer();
-      while (ld_acquire(bar + 1) == my_gen) {
-        if (globaltimer() - t0 > kWaitLimitNs) {
-          report(dev_status, CSA_ERR_TIMEOUT);
-          ok = false;
-          break;
-        }
-      }
-    }
-    sh_gen = my_gen + 1;
-  }
-  ok = __syncthreads_and(ok) != 0;
-  *gen_out = sh_gen;
-  return ok;
-}
-
 // Phase 1 of the selection for slice sb of sequence b: the threshold bin (highest bin whose
 // suffix count reaches k), the slice's count above it and its in-bin candidates. The last
 // slice of the sequence to finish resolves the exact cut (finalize).

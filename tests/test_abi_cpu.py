@@ -46,7 +46,7 @@ def test_status_strings(L):
 
 def test_workspace_sizes_are_host_only(L):
     a = L.csa_indexer_topk_workspace_size(4, 262144, 1024)
-    assert a >= 4 * 262144 * (4 + 8) + 4 * 4096 * 4
+    assert a >= 4 * 262144 * (4 + 8) + 4 * 2048 * 4  # scores, candidates, 11-bit histograms
     assert L.csa_indexer_topk_workspace_size(-1, 128, 4) == 0
     b = L.csa_attn_workspace_size(4, 128, 1024 + 128)
     assert b >= 4 * 18 * 128 * 512 * 2  # fp16 partial outputs per 64-row chunk
