@@ -192,6 +192,31 @@ int csa_sparse_attn_decode(const csa_attn_args* args, void* workspace, size_t wo
 int hca_attn_decode(const csa_attn_args* args, void* workspace, size_t workspace_bytes,
                     csa_stream_t stream);
 
+/* ------------------------------------------------------------------------------------
+ * csa_sparse_attn_decode_noalloc: csa_sparse_attn_decode without a workspace argument.
+ * The pages have no counterpart: this is an interface convenience, not part of the method.
+ *
+ * It is for callers that cannot hand over scratch memory: a host that exposes only a
+ * C function taking the layer's inputs and outputs (a plugin slot with no allocator), or
+ * code running while a stream is being captured into a graph, where cudaMalloc/cudaFree
+ * are not allowed and would otherwise synchronise the device.
+ *
+ * Scratch comes from one file-scope device array of CSA_NOALLOC_SCRATCH_BYTES per device
+ * (12 MiB; enough for B = 4, H = 128, k = 1024). Its address is looked up with
+ * cudaGetSymbolAddress on the first call on each device and cached; make that first call
+ * outside stream capture (for instance one ordinary call before capturing). Nothing in
+ * the scratch has to start at zero: every partial result is written before it is read.
+ *
+ * Results are the same as csa_sparse_attn_decode with a caller workspace (the same
+ * kernels run). Arguments are checked as there; a problem whose scratch
+ * (csa_attn_workspace_size(B, H, k + 128)) exceeds the array returns CSA_ERR_UNSUPPORTED
+ * before anything touches the device. Calls that can overlap in time on one device (two
+ * streams, two host threads, or concurrently replayed graphs) share the array and race;
+ * calls on a single stream are ordered and safe.
+ */
+#define CSA_NOALLOC_SCRATCH_BYTES (12u << 20)
+int csa_sparse_attn_decode_noalloc(const csa_attn_args* args, csa_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

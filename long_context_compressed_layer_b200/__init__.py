@@ -50,7 +50,9 @@ class AttnArgs(C.Structure):
 
 EXPORTS = ["csa_status_string", "csa_compress", "csa_indexer_topk_workspace_size",
            "csa_indexer_topk", "csa_attn_workspace_size", "csa_sparse_attn_decode",
-           "hca_attn_decode"]
+           "hca_attn_decode", "csa_sparse_attn_decode_noalloc"]
+
+NOALLOC_SCRATCH_BYTES = 12 << 20
 
 _lib = None
 
@@ -76,6 +78,8 @@ def lib() -> C.CDLL:
         for f in ("csa_sparse_attn_decode", "hca_attn_decode"):
             getattr(L, f).restype = C.c_int
             getattr(L, f).argtypes = [C.POINTER(AttnArgs), _vp, C.c_size_t, _vp]
+        L.csa_sparse_attn_decode_noalloc.restype = C.c_int
+        L.csa_sparse_attn_decode_noalloc.argtypes = [C.POINTER(AttnArgs), _vp]
         _lib = L
     return _lib
 
@@ -177,7 +181,8 @@ def _attn(fn: str, sparse: bool, q, pos, n_entries, kv, kv_scale, swa, sink, idx
     Nmax = kv.shape[1]
     k = idx.shape[1] if sparse else 0
     dev = q.device
-    if workspace is None:
+    noalloc = fn.endswith("_noalloc")
+    if workspace is None and not noalloc:
         workspace = attn_workspace(B, H, (k if sparse else Nmax) + WINDOW, dev)
     if out is None:
         out = torch.empty((B, H, HEAD_DIM), dtype=torch.bfloat16, device=dev)
@@ -189,8 +194,11 @@ def _attn(fn: str, sparse: bool, q, pos, n_entries, kv, kv_scale, swa, sink, idx
                     _ptr(sink, elem=4, name="sink"), tau, rope_base, int(derotate),
                     _ptr(out, elem=2, name="out"), _ptr(l, elem=4, name="lse"),
                     _ptr(dev_status, elem=4, name="dev_status"))
-    _check(getattr(lib(), fn)(C.byref(args), workspace.data_ptr(), workspace.numel(),
-                              _stream(stream)), fn)
+    if noalloc:
+        _check(getattr(lib(), fn)(C.byref(args), _stream(stream)), fn)
+    else:
+        _check(getattr(lib(), fn)(C.byref(args), workspace.data_ptr(), workspace.numel(),
+                                  _stream(stream)), fn)
     return (out, l) if lse else out
 
 
@@ -198,6 +206,15 @@ def sparse_attn_decode(q, pos, n_entries, kv, kv_scale, swa, sink, idx, **kw):
     """CSA decode: MQA over idx [B][k] + window + sink -> bf16 [B][H][512] (and lse)."""
     return _attn("csa_sparse_attn_decode", True, q, pos, n_entries, kv, kv_scale, swa, sink,
                  idx, **kw)
+
+
+def sparse_attn_decode_noalloc(q, pos, n_entries, kv, kv_scale, swa, sink, idx, **kw):
+    """sparse_attn_decode with the library's static per-device scratch instead of a workspace
+    (no scratch allocation; overlapping calls on one device race on the shared scratch)."""
+    if kw.get("workspace") is not None:
+        raise ValueError("sparse_attn_decode_noalloc takes no workspace")
+    return _attn("csa_sparse_attn_decode_noalloc", True, q, pos, n_entries, kv, kv_scale, swa,
+                 sink, idx, **kw)
 
 
 def hca_attn_decode(q, pos, n_entries, kv, kv_scale, swa, sink, **kw):

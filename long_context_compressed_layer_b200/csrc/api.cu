@@ -1,6 +1,7 @@
 // extern "C" entry points of the CSA/HCA layer library: argument checks on the host, TMA
 // tensor maps, workspace carving and kernel launches. Nothing here allocates, frees or
 // synchronises; every failure is a status code.
+#include <atomic>
 #include <cstring>
 
 #include "common.cuh"
@@ -46,6 +47,23 @@ bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA; }
+
+// Scratch of csa_sparse_attn_decode_noalloc: one array per device, zero-initialised when
+// the module loads. Its device address is cached per device after the first lookup.
+__device__ __align__(256) unsigned char g_noalloc_scratch[CSA_NOALLOC_SCRATCH_BYTES];
+constexpr int kMaxDevices = 64;
+
+void* noalloc_scratch() {
+  static std::atomic<void*> cache[kMaxDevices];
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  void* p = cache[dev].load(std::memory_order_acquire);
+  if (!p) {
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    cache[dev].store(p, std::memory_order_release);
+  }
+  return p;
+}
 
 }  // namespace
 }  // namespace csa
@@ -174,6 +192,19 @@ int csa_sparse_attn_decode(const csa_attn_args* a, void* ws, size_t ws_bytes,
 
 int hca_attn_decode(const csa_attn_args* a, void* ws, size_t ws_bytes, csa_stream_t stream) {
   return attn_common(a, 0, ws, ws_bytes, stream);
+}
+
+int csa_sparse_attn_decode_noalloc(const csa_attn_args* a, csa_stream_t stream) {
+  // Out-of-range sizes: let the ordinary checks pick the status (no workspace is passed,
+  // so nothing can launch).
+  if (!a || a->B <= 0 || a->B > 65535 || (a->H != 64 && a->H != 128) || a->k < 1 ||
+      a->k > 2048)
+    return attn_common(a, 1, nullptr, 0, stream);
+  if (at_workspace_size(a->B, a->H, a->k + CSA_WINDOW) > CSA_NOALLOC_SCRATCH_BYTES)
+    return CSA_ERR_UNSUPPORTED;
+  void* ws = noalloc_scratch();
+  if (!ws) return CSA_ERR_CUDA;
+  return attn_common(a, 1, ws, CSA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"
