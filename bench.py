@@ -9,8 +9,13 @@ Metric: decode queries/s (whole job). Inputs are synthetic and seeded; four devi
 of the streamed inputs are rotated so that consecutive steps never hit in L2.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                       [--workload decode|prefill]
 Under torchrun every rank runs its own 4-sequence batch (weak scaling, no collective on
 the data path); rank 0 prints one JSON line.
+
+--workload prefill times csa_prefill instead: 65,536 new tokens after a 196,608-token
+prefix (one sequence, 128 heads, indexer 64 heads, top-k 1024); one step is the whole
+prefill call (compression, indexer top-k and attention for every new token).
 """
 
 from __future__ import annotations
@@ -123,6 +128,109 @@ def ncu_traffic() -> dict | None:
     return d
 
 
+PREFILL_ID = 4
+PREFILL_METRIC = "CSA prefill tokens/s (65,536 new tokens after a 196,608-token prefix)"
+
+
+def prefill_flops(P: int, T: int, m: int, H: int, H_I: int, k: int) -> tuple[int, int]:
+    """(FP4 indexer FLOPs, BF16/FP16 attention FLOPs) of one prefill by the layer's
+    definition: every query scores its n(t) = floor((t+1)/m) eligible entries with H_I heads
+    of 128 dims; attention forms S = Q V^T and O = P V over min(k, n(t)) entries + the
+    window rows (at most 128) for H heads of 512 dims."""
+    t = P + np.arange(T, dtype=np.int64)
+    n = (t + 1) // m
+    rows = np.minimum(k, n) + np.minimum(128, t + 1)
+    return int(2 * H_I * 128 * n.sum()), int(4 * H * 512 * rows.sum())
+
+
+def bench_prefill(args, rank: int, world: int, local: int) -> None:
+    import torch
+
+    import long_context_compressed_layer_b200 as csa
+    from synth import inputs as synth
+
+    torch.cuda.set_device(local)
+    w = synth.WORKLOADS[PREFILL_ID]
+    d = synth.prefill_inputs_device(w.P, w.T, w.m, w.H, w.H_I, seed=w.seed + 1000 * rank)
+    T, k = w.T, w.k
+    kv0 = d["kv"].clone()
+    ws = csa.prefill_workspace(T, d["Nmax"], w.H, k)
+    out = torch.empty((T, w.H, 512), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+    bf = lambda x: x.view(torch.bfloat16) if x.dtype == torch.int16 else x
+
+    def step():
+        csa.prefill(w.P, w.m, k, a=d["a"], b=d["b"], za=d["za"], zb=d["zb"], bias=d["bias"],
+                    kv=d["kv"], kv_scale=d["kv_scale"], q_fp4=d["q_fp4"], q_sf=d["q_sf"],
+                    w=d["w"], k_fp4=d["k_fp4"], k_sf=d["k_sf"], q=d["q"], sink=d["sink"],
+                    prev_b=d["prev_b"], prev_zb=d["prev_zb"], swa_prefix=d["swa_prefix"],
+                    workspace=ws, out=out, dev_status=status)
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during the benchmark")
+
+    # end to end: the new tokens' inputs go up from pinned host memory and the output
+    # comes back, around the same call
+    up = ("a", "b", "za", "zb", "q", "q_fp4", "q_sf", "w")
+    pinned = {x: d[x].cpu().pin_memory() for x in up}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_h.numel() * out_h.element_size()
+    x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    x0.record(stream)
+    for _ in range(args.steps):
+        for x in up:
+            d[x].copy_(pinned[x], non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+    x1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = x0.elapsed_time(x1) / args.steps
+    d["kv"].copy_(kv0)
+    if rank != 0:
+        return
+    f4, f16 = prefill_flops(w.P, T, w.m, w.H, w.H_I, k)
+    pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
+    bf16_peak = pk.get("bf16_tflops_sustained", 1400.0)  # a long step: the sustained figure
+    # FP4 counts at the nominal 4x of dense BF16 (no FP4 peak is measured on this pool)
+    eq_tflops = (f4 / 4 + f16) / (ms * 1e-3) / 1e12
+    line = {
+        "metric": PREFILL_METRIC, "value": T / (ms * 1e-3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp4+fp16", "data": "synthetic",
+        "config": {"workload": w.name, "prefix_tokens": w.P, "new_tokens": T, "heads": w.H,
+                   "indexer_heads": w.H_I, "top_k": k, "window": 128,
+                   "l2": "inputs larger than L2 (8.6 GB of queries)",
+                   "fp4_tflop": f4 / 1e12, "bf16_tflop": f16 / 1e12},
+        "roofline": {"bound": "tensor", "kernel": "csa_prefill (whole call)",
+                     "achieved": eq_tflops, "peak": bf16_peak, "unit": "TFLOP/s",
+                     "frac": eq_tflops / bf16_peak,
+                     "peak_src": ("measured sustained bf16; FP4 FLOPs weighted 1/4 (nominal ratio)"
+                                  if "bf16_tflops_sustained" in pk else "fallback"),
+                     "traffic": None},
+        "clocks": clocks,
+        "e2e": {"value": T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, rank: int) -> None:
     """The fp64 CPU oracle, as it stands, on the host cores: each step is one decode query
     (one sequence of the workload: indexer over 262,144 entries, top-k, attention)."""
@@ -192,6 +300,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--copies", type=int, default=COPIES,
                     help="device copies of the streamed inputs rotated across steps")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -199,6 +308,9 @@ def main():
     local = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, rank)
+        return
+    if args.workload == "prefill":
+        bench_prefill(args, rank, world, local)
         return
 
     import torch
@@ -365,7 +477,9 @@ def main():
             "clocks": clocks,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-            "gpu_launches": 5 * steps_run,
+            # per step: the cooperative indexer launch (scores + selection) and the two
+            # attention kernels
+            "gpu_launches": 3 * steps_run,
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline_sample(d, w)

@@ -125,7 +125,9 @@ int csa_compress(const csa_compress_args* args, csa_stream_t stream);
  * group g -- the tensor-core scale-factor atom, so a group is copied as is.
  * Nmax must be a multiple of 128. 1 <= k <= 2048, H_I in {16, 32, 64}.
  * The workspace must be zero-filled once before its first use; every call leaves it
- * zeroed again. Calls that share a workspace must not overlap on the device.
+ * zeroed again. One workspace serves calls of any B and Nmax up to the sizes it was
+ * created for (the parts kept at zero sit at offsets that do not depend on B). Calls
+ * that share a workspace must not overlap on the device.
  */
 typedef struct {
   int32_t B;
@@ -191,6 +193,73 @@ int csa_sparse_attn_decode(const csa_attn_args* args, void* workspace, size_t wo
                            csa_stream_t stream);
 int hca_attn_decode(const csa_attn_args* args, void* workspace, size_t workspace_bytes,
                     csa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
+ * csa_prefill: causal CSA prefill of T new tokens of one sequence after a P-token prefix.
+ * (walkthrough §2.2 for every step; §3.5: the state cache carries the 128 window tokens
+ * and the previous block across chunks, the classical cache the compressed entries.)
+ *
+ * 1. Compression of the new blocks (as csa_compress with pos0 = P, overlap on): entries
+ *    P/m .. (P+T)/m - 1 are written into kv / kv_scale; rows 0 .. P/m - 1 are the cached
+ *    prefix and are only read. T may leave a tail of T % m tokens: their block is not
+ *    emitted (it stays in the caller's state).
+ * 2. For every new token t = P + r (r = 0 .. T-1), with n(t) = floor((t+1)/m) eligible
+ *    entries: the indexer top-k over entries j < n(t) (as csa_indexer_topk, all queries
+ *    scoring the one key array k_fp4 / k_sf, which must hold the indexer keys of every
+ *    entry up to (P+T)/m), then CSA attention over the selected entries, the window
+ *    t-127 .. t and the sink (as csa_sparse_attn_decode with pos = t). Window rows of
+ *    prefix positions come from the ring swa_prefix[p % 128]; window rows of new tokens
+ *    are RMSNorm (eps, norm_w) then RoPE at position p of a[p - P], rounded to BF16.
+ *
+ * Layouts: a, b bf16 [T][512]; za, zb [T][512]; bias [2m]; prev_b bf16 [m][512] and
+ * prev_zb [m][512] are the m tokens before P (needed when P > 0); kv [Nmax][576];
+ * kv_scale [Nmax]; q_fp4 [T][H_I][64]; q_sf [T][H_I][4]; w [T][H_I]; k_fp4 [Nmax][64];
+ * k_sf [Nmax/128][512] (grouped as in csa_indexer_topk); q bf16 [T][H][512];
+ * swa_prefix bf16 [128][512] (needed when P > 0); out bf16 [T][H][512]; lse [T][H];
+ * idx [T][k]. m in 1..128, P % m == 0, Nmax a multiple of 128 with (P+T)/m <= Nmax,
+ * H in {64, 128}, H_I in {16, 32, 64}, 1 <= k <= 2048.
+ * The workspace (csa_prefill_workspace_size) must be zero-filled once before its first
+ * use; every call leaves the parts that must start at zero zeroed again.
+ */
+typedef struct {
+  int64_t P;                  /* prefix tokens, a multiple of m */
+  int32_t T;                  /* new tokens */
+  int32_t m;                  /* compression ratio (4 for CSA) */
+  int32_t H;                  /* query heads: 64 or 128 */
+  int32_t H_I;                /* indexer heads: 16, 32 or 64 */
+  int32_t k;                  /* top-k */
+  int64_t Nmax;               /* entry capacity, multiple of 128 */
+  float tau;                  /* softmax scale; 0 selects 1/sqrt(512) */
+  float rope_base;            /* 10000 */
+  float eps;                  /* RMSNorm epsilon */
+  int32_t derotate;           /* 1: de-rotate the last 64 output dims by t */
+  const uint16_t* a;          /* new tokens (see Layouts) */
+  const uint16_t* b;
+  const float* za;
+  const float* zb;
+  const float* bias;
+  const float* norm_w;        /* [512] or NULL = ones (entries and window rows) */
+  const uint16_t* prev_b;
+  const float* prev_zb;
+  uint8_t* kv;                /* in: prefix rows; out: the new rows */
+  float* kv_scale;
+  const uint8_t* q_fp4;
+  const uint8_t* q_sf;
+  const float* w;
+  const uint8_t* k_fp4;
+  const uint8_t* k_sf;
+  const uint16_t* q;
+  const float* sink;          /* [H] */
+  const uint16_t* swa_prefix;
+  uint16_t* out;
+  float* lse;                 /* optional */
+  int32_t* idx;               /* optional: the selected sets */
+  int32_t* dev_status;        /* optional device word */
+} csa_prefill_args;
+
+size_t csa_prefill_workspace_size(int32_t T, int64_t Nmax, int32_t H, int32_t k);
+int csa_prefill(const csa_prefill_args* args, void* workspace, size_t workspace_bytes,
+                csa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
  * csa_sparse_attn_decode_noalloc: csa_sparse_attn_decode without a workspace argument.

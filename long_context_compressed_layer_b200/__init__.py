@@ -48,9 +48,21 @@ class AttnArgs(C.Structure):
                 ("dev_status", _vp)]
 
 
+class PrefillArgs(C.Structure):
+    _fields_ = [("P", C.c_int64), ("T", C.c_int32), ("m", C.c_int32), ("H", C.c_int32),
+                ("H_I", C.c_int32), ("k", C.c_int32), ("Nmax", C.c_int64), ("tau", C.c_float),
+                ("rope_base", C.c_float), ("eps", C.c_float), ("derotate", C.c_int32),
+                ("a", _vp), ("b", _vp), ("za", _vp), ("zb", _vp), ("bias", _vp),
+                ("norm_w", _vp), ("prev_b", _vp), ("prev_zb", _vp), ("kv", _vp),
+                ("kv_scale", _vp), ("q_fp4", _vp), ("q_sf", _vp), ("w", _vp), ("k_fp4", _vp),
+                ("k_sf", _vp), ("q", _vp), ("sink", _vp), ("swa_prefix", _vp), ("out", _vp),
+                ("lse", _vp), ("idx", _vp), ("dev_status", _vp)]
+
+
 EXPORTS = ["csa_status_string", "csa_compress", "csa_indexer_topk_workspace_size",
            "csa_indexer_topk", "csa_attn_workspace_size", "csa_sparse_attn_decode",
-           "hca_attn_decode", "csa_sparse_attn_decode_noalloc"]
+           "hca_attn_decode", "csa_sparse_attn_decode_noalloc", "csa_prefill_workspace_size",
+           "csa_prefill"]
 
 NOALLOC_SCRATCH_BYTES = 12 << 20
 
@@ -78,6 +90,10 @@ def lib() -> C.CDLL:
         for f in ("csa_sparse_attn_decode", "hca_attn_decode"):
             getattr(L, f).restype = C.c_int
             getattr(L, f).argtypes = [C.POINTER(AttnArgs), _vp, C.c_size_t, _vp]
+        L.csa_prefill_workspace_size.restype = C.c_size_t
+        L.csa_prefill_workspace_size.argtypes = [C.c_int32, C.c_int64, C.c_int32, C.c_int32]
+        L.csa_prefill.restype = C.c_int
+        L.csa_prefill.argtypes = [C.POINTER(PrefillArgs), _vp, C.c_size_t, _vp]
         L.csa_sparse_attn_decode_noalloc.restype = C.c_int
         L.csa_sparse_attn_decode_noalloc.argtypes = [C.POINTER(AttnArgs), _vp]
         _lib = L
@@ -221,3 +237,53 @@ def hca_attn_decode(q, pos, n_entries, kv, kv_scale, swa, sink, **kw):
     """HCA decode: MQA over all n_entries[b] entries + window + sink."""
     return _attn("hca_attn_decode", False, q, pos, n_entries, kv, kv_scale, swa, sink, None,
                  **kw)
+
+
+# -------------------------------------------------------------------- prefill
+def prefill_workspace(T: int, Nmax: int, H: int, k: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace (the parts that must start at zero are left zeroed)."""
+    n = lib().csa_prefill_workspace_size(T, Nmax, H, k)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+
+
+def prefill(P: int, m: int, k: int, *, a, b, za, zb, bias, kv, kv_scale, q_fp4, q_sf, w,
+            k_fp4, k_sf, q, sink, prev_b=None, prev_zb=None, swa_prefix=None, norm_w=None,
+            tau: float = 0.0, rope_base: float = 10000.0, eps: float = 1e-6,
+            derotate: bool = True, workspace=None, out=None, lse: bool = False,
+            idx: bool = False, dev_status=None, stream=None):
+    """Causal CSA prefill of the T new tokens after a P-token prefix (one sequence).
+    kv / kv_scale [Nmax] are updated in place with the new entries. Returns out
+    [T][H][512] bf16 and, when asked, lse [T][H] and the selected sets idx [T][k]."""
+    T = a.shape[0]
+    H, H_I = q.shape[1], q_fp4.shape[1]
+    Nmax = kv.shape[0]
+    dev = q.device
+    if workspace is None:
+        workspace = prefill_workspace(T, Nmax, H, k, dev)
+    if out is None:
+        out = torch.empty((T, H, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    l = torch.empty((T, H), dtype=torch.float32, device=dev) if lse else None
+    ix = torch.empty((T, k), dtype=torch.int32, device=dev) if idx else None
+    args = PrefillArgs(P, T, m, H, H_I, k, Nmax, tau, rope_base, eps, int(derotate),
+                       _ptr(a, elem=2, name="a"), _ptr(b, elem=2, name="b"),
+                       _ptr(za, elem=4, name="za"), _ptr(zb, elem=4, name="zb"),
+                       _ptr(bias, elem=4, name="bias"), _ptr(norm_w, elem=4, name="norm_w"),
+                       _ptr(prev_b, elem=2, name="prev_b"),
+                       _ptr(prev_zb, elem=4, name="prev_zb"), _ptr(kv, elem=1, name="kv"),
+                       _ptr(kv_scale, elem=4, name="kv_scale"),
+                       _ptr(q_fp4, elem=1, name="q_fp4"), _ptr(q_sf, elem=1, name="q_sf"),
+                       _ptr(w, elem=4, name="w"), _ptr(k_fp4, elem=1, name="k_fp4"),
+                       _ptr(k_sf, elem=1, name="k_sf"), _ptr(q, elem=2, name="q"),
+                       _ptr(sink, elem=4, name="sink"),
+                       _ptr(swa_prefix, elem=2, name="swa_prefix"),
+                       _ptr(out, elem=2, name="out"), _ptr(l, elem=4, name="lse"),
+                       _ptr(ix, elem=4, name="idx"),
+                       _ptr(dev_status, elem=4, name="dev_status"))
+    _check(lib().csa_prefill(C.byref(args), workspace.data_ptr(), workspace.numel(),
+                             _stream(stream)), "csa_prefill")
+    res = [out]
+    if lse:
+        res.append(l)
+    if idx:
+        res.append(ix)
+    return res[0] if len(res) == 1 else tuple(res)

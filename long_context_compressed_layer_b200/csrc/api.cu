@@ -9,11 +9,14 @@
 namespace csa {
 cudaError_t launch_compress(const csa_compress_args& a, cudaStream_t stream);
 cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
-                                const CUtensorMap& kmap, cudaStream_t stream);
+                                const CUtensorMap& kmap, cudaStream_t stream, int kshared);
 size_t ix_workspace_size(int B, int64_t Nmax, int k);
 size_t at_workspace_size(int B, int H, int rows_max);
+cudaError_t launch_prefill_prep(const csa_prefill_args& a, uint16_t* lin, int32_t* n_all,
+                                int32_t* pos_all, cudaStream_t stream);
 cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* workspace,
-                        const CUtensorMap& qmap, cudaStream_t stream);
+                        const CUtensorMap& qmap, cudaStream_t stream, int64_t kv_bstride,
+                        int swa_linear, int64_t swa_base);
 
 namespace {
 
@@ -63,6 +66,67 @@ void* noalloc_scratch() {
     cache[dev].store(p, std::memory_order_release);
   }
   return p;
+}
+
+// Queries of a prefill handled per indexer / attention launch (the indexer keeps one
+// prefix-sum slot per query in shared memory).
+constexpr int kPrefillChunk = 1024;
+
+struct PrefillWs {
+  char* ix;           // indexer workspace for kPrefillChunk queries (kept zeroed)
+  int32_t* n_all;     // [T]
+  int32_t* pos_all;   // [T]
+  uint16_t* lin;      // [T + 127][512] window rows in position order
+  int32_t* idx;       // [chunk][k] selected sets when the caller passes none
+  char* at;           // attention workspace for one chunk
+};
+
+size_t prefill_ws_layout(int T, int64_t Nmax, int H, int k, char* base, PrefillWs* w) {
+  const int qc = T < kPrefillChunk ? (T > 0 ? T : 1) : kPrefillChunk;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += (bytes + 255) & ~(size_t)255;
+    return p;
+  };
+  char* ix = take(ix_workspace_size(qc, Nmax, k));
+  char* n_all = take((size_t)T * 4);
+  char* pos_all = take((size_t)T * 4);
+  char* lin = take(((size_t)T + CSA_WINDOW - 1) * CSA_HEAD_DIM * 2);
+  char* idx = take((size_t)qc * k * 4);
+  char* at = take(at_workspace_size(qc, H, k + CSA_WINDOW));
+  if (w) {
+    w->ix = ix;
+    w->n_all = reinterpret_cast<int32_t*>(n_all);
+    w->pos_all = reinterpret_cast<int32_t*>(pos_all);
+    w->lin = reinterpret_cast<uint16_t*>(lin);
+    w->idx = reinterpret_cast<int32_t*>(idx);
+    w->at = at;
+  }
+  return off;
+}
+
+bool encode_q_map(EncodeTiledFn enc, CUtensorMap* qmap, const uint16_t* q, int64_t rows, int H) {
+  const cuuint64_t dims[2] = {CSA_HEAD_DIM, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {CSA_HEAD_DIM * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)H};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(qmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(q), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+bool encode_key_map(EncodeTiledFn enc, CUtensorMap* kmap, const uint8_t* k_fp4, int64_t Nmax,
+                    int64_t B) {
+  const cuuint64_t dims[3] = {64, (cuuint64_t)Nmax, (cuuint64_t)B};
+  const cuuint64_t strides[2] = {64, (cuuint64_t)Nmax * 64};
+  const cuuint32_t box[3] = {64, 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(k_fp4), dims, strides,
+             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -142,7 +206,7 @@ int csa_indexer_topk(const csa_topk_args* a, void* ws, size_t ws_bytes, csa_stre
       return CSA_ERR_CUDA;
   }
   return cuda_status(
-      launch_indexer_topk(*a, ws, sms, kmap, reinterpret_cast<cudaStream_t>(stream)));
+      launch_indexer_topk(*a, ws, sms, kmap, reinterpret_cast<cudaStream_t>(stream), 0));
 }
 
 size_t csa_attn_workspace_size(int32_t B, int32_t H, int32_t rows_max) {
@@ -182,7 +246,8 @@ static int attn_common(const csa_attn_args* a, int sparse, void* ws, size_t ws_b
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return CSA_ERR_CUDA;
   return cuda_status(
-      launch_attn(*a, sparse, rows_max, ws, qmap, reinterpret_cast<cudaStream_t>(stream)));
+      launch_attn(*a, sparse, rows_max, ws, qmap, reinterpret_cast<cudaStream_t>(stream), a->Nmax,
+                  0, 0));
 }
 
 int csa_sparse_attn_decode(const csa_attn_args* a, void* ws, size_t ws_bytes,
@@ -192,6 +257,117 @@ int csa_sparse_attn_decode(const csa_attn_args* a, void* ws, size_t ws_bytes,
 
 int hca_attn_decode(const csa_attn_args* a, void* ws, size_t ws_bytes, csa_stream_t stream) {
   return attn_common(a, 0, ws, ws_bytes, stream);
+}
+
+size_t csa_prefill_workspace_size(int32_t T, int64_t Nmax, int32_t H, int32_t k) {
+  if (T < 0 || Nmax < 0 || H < 1 || k < 1) return 0;
+  return prefill_ws_layout(T, Nmax, H, k, nullptr, nullptr);
+}
+
+int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream_t stream_) {
+  if (!a) return CSA_ERR_INVALID_ARG;
+  if (a->P < 0 || a->T < 0 || a->m < 1 || a->m > 128 || a->P % a->m || a->Nmax < 0 ||
+      a->Nmax % 128 || (a->P + a->T) / a->m > a->Nmax || !(a->eps >= 0.f) ||
+      !(a->rope_base > 0.f) || !(a->tau >= 0.f) || (a->derotate != 0 && a->derotate != 1) ||
+      a->k < 1)
+    return CSA_ERR_INVALID_ARG;
+  if ((a->H != 64 && a->H != 128) || (a->H_I != 16 && a->H_I != 32 && a->H_I != 64) ||
+      a->k > 2048 || a->P + a->T >= ((int64_t)1 << 31) || a->Nmax > ((int64_t)1 << 30))
+    return CSA_ERR_UNSUPPORTED;
+  if (a->T == 0) return CSA_OK;
+  if (!ok_ptr(a->a) || !ok_ptr(a->b) || !ok_ptr(a->za) || !ok_ptr(a->zb) || !ok_ptr(a->bias) ||
+      !ok_ptr(a->kv) || !ok_ptr(a->kv_scale) || !ok_ptr(a->q_fp4) || !ok_ptr(a->q_sf) ||
+      !ok_ptr(a->w) || !ok_ptr(a->k_fp4) || !ok_ptr(a->k_sf) || !ok_ptr(a->q) ||
+      !ok_ptr(a->sink) || !ok_ptr(a->out) || !ok_opt(a->norm_w) || !ok_opt(a->lse) ||
+      !ok_opt(a->idx) || (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)))
+    return CSA_ERR_INVALID_ARG;
+  if (a->P > 0 && (!ok_ptr(a->prev_b) || !ok_ptr(a->prev_zb) || !ok_ptr(a->swa_prefix)))
+    return CSA_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255) ||
+      ws_bytes < prefill_ws_layout(a->T, a->Nmax, a->H, a->k, nullptr, nullptr))
+    return CSA_ERR_WORKSPACE;
+  const int sms = num_sms();
+  EncodeTiledFn enc = encode_fn();
+  if (sms <= 0 || !enc) return CSA_ERR_CUDA;
+  cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
+  PrefillWs w;
+  prefill_ws_layout(a->T, a->Nmax, a->H, a->k, reinterpret_cast<char*>(ws), &w);
+
+  // 1. the new blocks' entries
+  csa_compress_args c;
+  std::memset(&c, 0, sizeof(c));
+  c.B = 1;
+  c.T = a->T;
+  c.m = a->m;
+  c.overlap = 1;
+  c.pos0 = a->P;
+  c.rope_base = a->rope_base;
+  c.eps = a->eps;
+  c.a = a->a;
+  c.b = a->b;
+  c.za = a->za;
+  c.zb = a->zb;
+  c.bias = a->bias;
+  c.norm_w = a->norm_w;
+  c.prev_b = a->prev_b;
+  c.prev_zb = a->prev_zb;
+  c.kv = a->kv;
+  c.kv_scale = a->kv_scale;
+  c.Nmax = a->Nmax;
+  cudaError_t e = launch_compress(c, stream);
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  // 2. per-query lengths, positions and the window rows in position order
+  e = launch_prefill_prep(*a, w.lin, w.n_all, w.pos_all, stream);
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  // 3. per chunk of queries: indexer top-k over the shared keys, then attention
+  CUtensorMap kmap;
+  if (!encode_key_map(enc, &kmap, a->k_fp4, a->Nmax, 1)) return CSA_ERR_CUDA;
+  for (int c0 = 0; c0 < a->T; c0 += kPrefillChunk) {
+    const int nq = a->T - c0 < kPrefillChunk ? a->T - c0 : kPrefillChunk;
+    int32_t* idx = a->idx ? a->idx + (size_t)c0 * a->k : w.idx;
+    csa_topk_args t;
+    std::memset(&t, 0, sizeof(t));
+    t.B = nq;
+    t.H_I = a->H_I;
+    t.k = a->k;
+    t.Nmax = a->Nmax;
+    t.n_entries = w.n_all + c0;
+    t.q_fp4 = a->q_fp4 + (size_t)c0 * a->H_I * 64;
+    t.q_sf = a->q_sf + (size_t)c0 * a->H_I * 4;
+    t.w = a->w + (size_t)c0 * a->H_I;
+    t.k_fp4 = a->k_fp4;
+    t.k_sf = a->k_sf;
+    t.idx = idx;
+    t.dev_status = a->dev_status;
+    e = launch_indexer_topk(t, w.ix, sms, kmap, stream, 1);
+    if (e != cudaSuccess) return CSA_ERR_CUDA;
+    csa_attn_args at;
+    std::memset(&at, 0, sizeof(at));
+    at.B = nq;
+    at.H = a->H;
+    at.k = a->k;
+    at.Nmax = a->Nmax;
+    at.q = a->q + (size_t)c0 * a->H * CSA_HEAD_DIM;
+    at.pos = w.pos_all + c0;
+    at.idx = idx;
+    at.n_entries = w.n_all + c0;
+    at.kv = a->kv;
+    at.kv_scale = a->kv_scale;
+    at.swa = w.lin;
+    at.sink = a->sink;
+    at.tau = a->tau;
+    at.rope_base = a->rope_base;
+    at.derotate = a->derotate;
+    at.out = a->out + (size_t)c0 * a->H * CSA_HEAD_DIM;
+    at.lse = a->lse ? a->lse + (size_t)c0 * a->H : nullptr;
+    at.dev_status = a->dev_status;
+    CUtensorMap qmap;
+    if (!encode_q_map(enc, &qmap, at.q, (int64_t)nq * a->H, a->H)) return CSA_ERR_CUDA;
+    e = launch_attn(at, 1, a->k + CSA_WINDOW, w.at, qmap, stream, 0, 1,
+                    a->P - (CSA_WINDOW - 1));
+    if (e != cudaSuccess) return CSA_ERR_CUDA;
+  }
+  return CSA_OK;
 }
 
 int csa_sparse_attn_decode_noalloc(const csa_attn_args* a, csa_stream_t stream) {

@@ -43,6 +43,9 @@ struct AtSmem {
 struct AtParams {
   int B, H, k, sparse, C;  // C = chunks per sequence in the workspace
   int64_t Nmax;
+  int64_t kv_bstride;      // entries between sequences in kv / kv_scale (0: one shared cache)
+  int swa_linear;          // 0: swa is a [B][128] ring; 1: swa holds consecutive positions
+  int64_t swa_base;        // linear mode: position of swa row 0 (shared by the batch)
   const int32_t* pos;
   const int32_t* idx;
   const int32_t* n_entries;
@@ -141,8 +144,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       const int j = p.sparse ? jsel : r;
       if (j >= 0 && j < n) {
         kind = 1;
-        src = p.kv + ((size_t)b * p.Nmax + j) * kRow;
-        s.scl[tid] = p.kv_scale + (size_t)b * p.Nmax + j;
+        src = p.kv + ((size_t)b * p.kv_bstride + j) * kRow;
+        s.scl[tid] = p.kv_scale + (size_t)b * p.kv_bstride + j;
       } else if (j != -1) {
         report(p.dev_status, CSA_ERR_DEVICE);
       }
@@ -150,7 +153,9 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       const int pp = t - (kWin - 1) + (r - nwin_first);
       if (pp >= 0) {
         kind = 2;
-        src = reinterpret_cast<const uint8_t*>(p.swa + ((size_t)b * kWin + (pp % kWin)) * kD);
+        const size_t wrow = p.swa_linear ? (size_t)(pp - p.swa_base)
+                                         : (size_t)b * kWin + (pp % kWin);
+        src = reinterpret_cast<const uint8_t*>(p.swa + wrow * kD);
       }
     }
     s.kind[tid] = kind;
@@ -425,7 +430,8 @@ size_t at_workspace_size(int B, int H, int rows_max) {
 }
 
 cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* workspace,
-                        const CUtensorMap& qmap, cudaStream_t stream) {
+                        const CUtensorMap& qmap, cudaStream_t stream, int64_t kv_bstride,
+                        int swa_linear, int64_t swa_base) {
   AtParams p;
   p.B = a.B;
   p.H = a.H;
@@ -433,6 +439,9 @@ cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* 
   p.sparse = sparse;
   p.C = (rows_max + kAtRows - 1) / kAtRows;
   p.Nmax = a.Nmax;
+  p.kv_bstride = kv_bstride;
+  p.swa_linear = swa_linear;
+  p.swa_base = swa_base;
   p.pos = a.pos;
   p.idx = a.idx;
   p.n_entries = a.n_entries;

@@ -74,17 +74,25 @@ struct IxSmem {
   uint32_t tmem_base;
 };
 
-// Workspace layout of csa_indexer_topk (all regions 256-byte aligned).
+// Workspace layout of csa_indexer_topk (all regions 256-byte aligned). Everything that must
+// be zero when a call starts sits at the front at offsets that do not depend on B: the
+// grid barrier, then one fixed-size block per sequence (counters, rule, histogram). A call
+// with fewer sequences therefore finds its blocks where a larger call left them zeroed.
+constexpr int kSeqWords = 8 + kHist;  // per-sequence block: counters[4], rule[4], hist
+
 struct IxWs {
-  float* scores;        // [B][Nmax]
-  uint32_t* hist;       // [B][kHist]
-  uint32_t* counters;   // [B][4]: candidate count, ticket
   uint32_t* grid_bar;   // [2]: arrival count, generation (grid-wide barrier)
+  uint32_t* seq;        // [B][kSeqWords]
   uint32_t* slice_cnt;  // [B][S]: above-bin count per slice, then the slice's output offset
-  uint32_t* rule;       // [B][4]: cut key, cut index, selected count
+  float* scores;        // [B][Nmax]
   uint64_t* cand;       // [B][Nmax]: (key << 32) | index of the in-bin candidates
   int S;                // slices per sequence
+  // counters: candidate count, ticket; rule: cut key, cut index, selected count, ready flag
+  __device__ uint32_t* counters(int b) const { return seq + (size_t)b * kSeqWords; }
+  __device__ uint32_t* rule(int b) const { return seq + (size_t)b * kSeqWords + 4; }
+  __device__ uint32_t* hist(int b) const { return seq + (size_t)b * kSeqWords + 8; }
 };
+static_assert((kSeqWords * 4) % 16 == 0, "histograms stay 16-byte aligned");
 
 __host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
 
@@ -103,20 +111,17 @@ __host__ __device__ inline size_t ix_ws_layout(int B, int64_t Nmax, int k, char*
     off += align256(bytes);
     return p;
   };
-  char* p0 = take((size_t)B * Nmax * 4);
-  char* p1 = take((size_t)B * kHist * 4);
-  char* p2 = take((size_t)B * 16 + 8);
-  char* p3 = take((size_t)B * S * 4);
-  char* p4 = take((size_t)B * 16);
-  char* p5 = take((size_t)B * Nmax * 8);
+  char* p0 = take(8);
+  char* p1 = take((size_t)B * kSeqWords * 4);
+  char* p2 = take((size_t)B * S * 4);
+  char* p3 = take((size_t)B * Nmax * 4);
+  char* p4 = take((size_t)B * Nmax * 8);
   if (ws) {
-    ws->scores = (float*)p0;
-    ws->hist = (uint32_t*)p1;
-    ws->counters = (uint32_t*)p2;
-    ws->grid_bar = (uint32_t*)(p2 + (size_t)B * 16);
-    ws->slice_cnt = (uint32_t*)p3;
-    ws->rule = (uint32_t*)p4;
-    ws->cand = (uint64_t*)p5;
+    ws->grid_bar = (uint32_t*)p0;
+    ws->seq = (uint32_t*)p1;
+    ws->slice_cnt = (uint32_t*)p2;
+    ws->scores = (float*)p3;
+    ws->cand = (uint64_t*)p4;
     ws->S = S;
   }
   return off;
@@ -128,7 +133,8 @@ size_t ix_workspace_size(int B, int64_t Nmax, int k) {
 
 struct IxParams {
   int B, H_I, k;
-  int fused;  // 1: the selection follows in this (cooperative) launch
+  int fused;    // 1: the selection follows in this (cooperative) launch
+  int kshared;  // 1: every query scores the same key rows (the queries of one prefill)
   int64_t Nmax;
   const int32_t* n_entries;
   const uint8_t* q_fp4;
@@ -254,9 +260,10 @@ __device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
           s.abort = 1;
           break;
         }
+        const int kb = p.kshared ? 0 : b;  // key sequence
         mbar_arrive_expect_tx(&s.full[st], kIxKeyBytes + kIxSfBytes);
-        tma_load_3d(s.keys[st], &kmap, &s.full[st], 0, t * kIxTile, b);
-        bulk_load(s.ksf[st], p.k_sf + ((size_t)b * (p.Nmax / kIxTile) + t) * kIxSfBytes,
+        tma_load_3d(s.keys[st], &kmap, &s.full[st], 0, t * kIxTile, kb);
+        bulk_load(s.ksf[st], p.k_sf + ((size_t)kb * (p.Nmax / kIxTile) + t) * kIxSfBytes,
                   kIxSfBytes, &s.full[st]);
       }
       // drain: every copy this warp issued has landed before the CTA winds down
@@ -352,7 +359,7 @@ __device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
     float w[kIxN];
     auto flush = [&](int bb) {  // warp-local: add the warp's counts to the global histogram
       __syncwarp();
-      uint32_t* gh = p.ws.hist + (size_t)bb * kHist;
+      uint32_t* gh = p.ws.hist(bb);
       for (int i = lane; i < kHist / 2; i += 32) {
         const uint32_t v = hist[i];
         if (v) {
@@ -553,13 +560,13 @@ __device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb
   const int n = clamp_n(p.n_entries[b], p.Nmax, p.dev_status);
   const int k_eff = n < p.k ? n : p.k;
   const int S_b = slices_of(n);
-  uint32_t* cnt = p.ws.counters + (size_t)b * 4;
+  uint32_t* cnt = p.ws.counters(b);
   uint32_t* scnt = p.ws.slice_cnt + (size_t)b * p.ws.S;
   const float* sc = p.ws.scores + (size_t)b * p.Nmax;
 
   if (tid == 0) { x.tbin = -1; x.above = 0; }
   if (n > p.k) {
-    const uint4* gh = reinterpret_cast<const uint4*>(p.ws.hist + (size_t)b * kHist);
+    const uint4* gh = reinterpret_cast<const uint4*>(p.ws.hist(b));
     constexpr int nv = kHist / 4, vper = (nv + kSelThreads - 1) / kSelThreads;
     uint4 hv[vper];  // every load in flight before any is stored
 #pragma unroll
@@ -724,7 +731,7 @@ __device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb
     __syncthreads();
   }
   if (tid == 0) {
-    uint32_t* r = p.ws.rule + (size_t)b * 4;
+    uint32_t* r = p.ws.rule(b);
     r[0] = cut_key;
     r[1] = (uint32_t)cut_idx;
     r[2] = (uint32_t)k_eff;
@@ -732,11 +739,11 @@ __device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb
     cnt[0] = 0;
     cnt[1] = 0;
   }
-  uint32_t* gh = p.ws.hist + (size_t)b * kHist;
+  uint32_t* gh = p.ws.hist(b);
   for (int i = tid; i < kHist; i += kSelThreads) gh[i] = 0;
   __syncthreads();
   if (tid == 0 && p.fused) {  // publish the rule and offsets of this sequence
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.ws.rule + (size_t)b * 4 + 3),
+    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.ws.rule(b) + 3),
                  "r"(ready_gen)
                  : "memory");
   }
@@ -749,7 +756,7 @@ __device__ void select_write(const IxParams& p, SelScratch& x, int b, int sb) {
   const int tid = threadIdx.x;
   int n = p.n_entries[b];
   n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
-  const uint32_t* r = p.ws.rule + (size_t)b * 4;
+  const uint32_t* r = p.ws.rule(b);
   const uint32_t cut_key = __ldcg(r), k_eff = __ldcg(r + 2);
   const int32_t cut_idx = (int32_t)__ldcg(r + 1);
   const uint32_t off = __ldcg(p.ws.slice_cnt + (size_t)b * p.ws.S + sb);
@@ -815,7 +822,7 @@ __device__ void select_fused(const IxParams& p, uint8_t* scratch) {
     bool ok = true;
     if (threadIdx.x == 0) {
       const uint64_t t0 = globaltimer();
-      while (ld_acquire(p.ws.rule + (size_t)b * 4 + 3) != ready_gen) {
+      while (ld_acquire(p.ws.rule(b) + 3) != ready_gen) {
         if (globaltimer() - t0 > kWaitLimitNs) {
           report(p.dev_status, CSA_ERR_TIMEOUT);
           ok = false;
@@ -852,10 +859,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_write_kernel(IxParams p) {
 
 // ------------------------------------------------------------------- launch
 cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
-                                const CUtensorMap& kmap, cudaStream_t stream) {
+                                const CUtensorMap& kmap, cudaStream_t stream, int kshared) {
   IxWs ws;
   ix_ws_layout(a.B, a.Nmax, a.k, (char*)workspace, &ws);
-  IxParams p{a.B, a.H_I, a.k, 1, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
+  IxParams p{a.B, a.H_I, a.k, 1, kshared, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
              a.idx, a.scores, a.dev_status};
   const size_t smem = sizeof(IxSmem) + 1024;
   static int configured = -1;

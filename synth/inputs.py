@@ -252,3 +252,80 @@ def prefill_inputs(P: int, T: int, m: int, H: int, H_I: int, seed: int) -> dict:
         out["prev_b"] = tok["prev_b"][0]
         out["prev_zb"] = tok["prev_zb"][0]
     return out
+
+
+# ------------------------------------------------------- device-side generation
+def prefill_inputs_device(P: int, T: int, m: int, H: int, H_I: int, seed: int,
+                          device="cuda") -> dict:
+    """The bundle of prefill_inputs drawn on the GPU with torch's seeded generator, for
+    sizes where host generation would take minutes (the 64K-token prefill holds 4.3 G query
+    values). Same distributions as the host generators (bf16 by truncating float32 N(0,1),
+    E2M1 magnitudes and E4M3 exponents through the same 65536-entry lookup tables, E8M0
+    in 124..130, w ~ U(0,1)); a different random stream, so values differ from
+    prefill_inputs with the same seed. The stored prefix cache and the indexer keys come
+    from the host generators (they are small). Returns torch tensors on `device`."""
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    rng = np.random.default_rng(seed)
+    Nmax = round_up(max((P + T) // m, 1), 128)
+    CH = 1 << 26  # elements per generation chunk (bounds the temporaries)
+
+    def chunked(n, fn, dtype):
+        out = torch.empty(n, dtype=dtype, device=device)
+        for s in range(0, n, CH):
+            e = min(n, s + CH)
+            out[s:e] = fn(e - s)
+        return out
+
+    def bf16n(shape):
+        n = int(np.prod(shape))
+        f = lambda c: (torch.randn(c, generator=g, device=device).view(torch.int32) >> 16) \
+            .to(torch.int16)
+        return chunked(n, f, torch.int16).view(shape)
+
+    def lut_of(p):
+        edges = np.cumsum(p) / p.sum()
+        u = (np.arange(65536, dtype=np.float64) + 0.5) / 65536.0
+        lut = np.searchsorted(edges, u, side="right").clip(0, len(p) - 1).astype(np.uint8)
+        return torch.from_numpy(lut).to(device)
+
+    mag_lut = lut_of(_E2M1_MAG_P)
+
+    def fp4_packed(shape):  # shape ends with the element count; returns packed bytes
+        n = int(np.prod(shape)) // 2
+
+        def f(c):
+            lo = mag_lut[torch.randint(0, 65536, (c,), generator=g, device=device)] | \
+                (torch.randint(0, 2, (c,), generator=g, device=device, dtype=torch.uint8) << 3)
+            hi = mag_lut[torch.randint(0, 65536, (c,), generator=g, device=device)] | \
+                (torch.randint(0, 2, (c,), generator=g, device=device, dtype=torch.uint8) << 3)
+            return lo | (hi << 4)
+        return chunked(n, f, torch.uint8).view(*shape[:-1], shape[-1] // 2)
+
+    kv, scale = kv_cache(rng, 1, Nmax)
+    n_all = np.array([(P + T) // m], dtype=np.int32)
+    ix = indexer_inputs(rng, 1, H_I, Nmax, n_all)
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(
+        x.view(np.int16) if x.dtype == np.uint16 else x)).to(device)
+    out = {
+        "P": P, "T": T, "m": m, "H": H, "H_I": H_I, "Nmax": Nmax,
+        "kv": t(kv[0]), "kv_scale": t(scale[0]),
+        "k_fp4": t(ix["k_fp4"][0]), "k_sf": t(ix["k_sf"][0]),
+        "q_fp4": fp4_packed((T, H_I, D_I)),
+        "q_sf": torch.randint(124, 131, (T, H_I, 4), generator=g, device=device,
+                              dtype=torch.uint8),
+        "w": torch.rand((T, H_I), generator=g, device=device),
+        "q": bf16n((T, H, D)),
+        "sink": torch.randn(H, generator=g, device=device),
+        "swa_prefix": bf16n((W_SWA, D)),
+        "a": bf16n((T, D)), "b": bf16n((T, D)),
+        "za": torch.randn((T, D), generator=g, device=device),
+        "zb": torch.randn((T, D), generator=g, device=device),
+        "bias": torch.randn(2 * m, generator=g, device=device) * 0.1,
+    }
+    if P > 0:
+        out["prev_b"] = bf16n((m, D))
+        out["prev_zb"] = torch.randn((m, D), generator=g, device=device)
+    return out

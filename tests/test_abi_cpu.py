@@ -122,6 +122,35 @@ def test_compress_rejects_on_host(L):
     assert f(args(T=3)) == csa.CSA_OK  # no complete block: nothing to do
 
 
+def _prefill_args(**over):
+    a = csa.PrefillArgs(4096, 300, 4, 128, 64, 1024, 1152, 0.0, 10000.0, 1e-6, 1,
+                        *([FAKE] * 5), None, FAKE, FAKE, *([FAKE] * 10), FAKE, None,
+                        None, None)
+    for k, v in over.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_prefill_rejects_on_host(L):
+    ws_ok = L.csa_prefill_workspace_size(300, 1152, 128, 1024)
+    assert ws_ok > 300 * 4 * 2 + (300 + 127) * 1024  # lengths, positions, window rows
+    f = lambda a, ws=FAKE, n=ws_ok: L.csa_prefill(C.byref(a), ws, n, None)
+    assert L.csa_prefill(None, FAKE, ws_ok, None) == csa.CSA_ERR_INVALID_ARG
+    assert f(_prefill_args(P=4094)) == csa.CSA_ERR_INVALID_ARG   # not a block boundary
+    assert f(_prefill_args(Nmax=1100)) == csa.CSA_ERR_INVALID_ARG  # not a multiple of 128
+    assert f(_prefill_args(Nmax=1024)) == csa.CSA_ERR_INVALID_ARG  # 1099 entries do not fit
+    assert f(_prefill_args(k=0)) == csa.CSA_ERR_INVALID_ARG
+    assert f(_prefill_args(H=96)) == csa.CSA_ERR_UNSUPPORTED
+    assert f(_prefill_args(H_I=8)) == csa.CSA_ERR_UNSUPPORTED
+    assert f(_prefill_args(k=4096)) == csa.CSA_ERR_UNSUPPORTED
+    assert f(_prefill_args(swa_prefix=None)) == csa.CSA_ERR_INVALID_ARG  # P > 0 needs it
+    assert f(_prefill_args(prev_b=None)) == csa.CSA_ERR_INVALID_ARG
+    assert f(_prefill_args(q=FAKE + 2)) == csa.CSA_ERR_INVALID_ARG
+    assert f(_prefill_args(), n=ws_ok - 1) == csa.CSA_ERR_WORKSPACE
+    assert f(_prefill_args(), ws=FAKE + 64) == csa.CSA_ERR_WORKSPACE
+    assert f(_prefill_args(T=0)) == csa.CSA_OK  # nothing to do
+
+
 def test_cuda_sources_are_sm100a_only():
     src = open(os.path.join(ROOT, "long_context_compressed_layer_b200", "build.py")).read()
     assert "arch=compute_100a,code=sm_100a" in src

@@ -157,6 +157,28 @@ def test_indexer_workspace_stays_clean_across_calls():
         np.testing.assert_array_equal(again, first)
 
 
+def test_indexer_workspace_shared_across_batch_sizes():
+    # one workspace sized for the largest call serves smaller batches in between
+    rng = np.random.default_rng(21)
+    big_n = np.array([4096, 3000, 2500], np.int32)
+    big = synth.indexer_inputs(rng, 3, 64, 4096, big_n)
+    small_n = np.array([1500], np.int32)
+    small = synth.indexer_inputs(rng, 1, 64, 4096, small_n)
+    ws = csa.indexer_topk_workspace(3, 4096, 512)
+
+    def run(ix, n):
+        return host(csa.indexer_topk(dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]),
+                                     dev(ix["k_fp4"]), dev(ix["k_sf"]), 512, workspace=ws))
+
+    first = run(big, big_n)
+    one = run(small, small_n)
+    again = run(big, big_n)
+    np.testing.assert_array_equal(again, first)
+    ora = oracle.indexer_scores(small_n, small["q_fp4"], small["q_sf"], small["w"],
+                                small["k_fp4"], small["k_sf"])
+    assert compare.compare_topk(one[0], ora[0], 1500, 512, what="small batch") <= 1
+
+
 # ------------------------------------------------------------------ attention
 def _attn_case(B, H, Nmax, n, pos, k=None, seed=0, sink_override=None):
     rng = np.random.default_rng(seed)

@@ -1,0 +1,119 @@
+"""CUDA prefill (csa_prefill) vs the fp64 oracle's prefill on seeded inputs (needs a B200)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import inputs as synth
+from tests import compare
+
+pytestmark = pytest.mark.gpu
+
+csa = pytest.importorskip("long_context_compressed_layer_b200")
+
+
+def dev(x):
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.uint16:
+        x = x.view(np.int16)
+    return torch.from_numpy(x).cuda()
+
+
+def host(t):
+    return t.cpu().numpy()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    csa.lib()
+
+
+def run_prefill(inp, k, derotate=True):
+    kv, sc = dev(inp["kv"]), dev(inp["kv_scale"])
+    opt = {x: dev(inp[x]) for x in ("prev_b", "prev_zb") if x in inp}
+    if inp["P"] > 0:
+        opt["swa_prefix"] = dev(inp["swa_prefix"])
+    out, lse, idx = csa.prefill(
+        inp["P"], inp["m"], k, a=dev(inp["a"]), b=dev(inp["b"]), za=dev(inp["za"]),
+        zb=dev(inp["zb"]), bias=dev(inp["bias"]), kv=kv, kv_scale=sc, q_fp4=dev(inp["q_fp4"]),
+        q_sf=dev(inp["q_sf"]), w=dev(inp["w"]), k_fp4=dev(inp["k_fp4"]), k_sf=dev(inp["k_sf"]),
+        q=dev(inp["q"]), sink=dev(inp["sink"]), derotate=derotate, lse=True, idx=True, **opt)
+    torch.cuda.synchronize()
+    return dict(out=out.float().cpu().numpy(), lse=host(lse), idx=host(idx), kv=host(kv),
+                kv_scale=host(sc))
+
+
+def check_rows(inp, k, got, rows, ora):
+    P, m = inp["P"], inp["m"]
+    flips = 0
+    for i, r in enumerate(rows):
+        n = (P + r + 1) // m
+        s = oracle.indexer_scores(np.array([n], np.int32), inp["q_fp4"][r:r + 1],
+                                  inp["q_sf"][r:r + 1], inp["w"][r:r + 1],
+                                  inp["k_fp4"][None], inp["k_sf"][None])[0]
+        flips += compare.compare_topk(got["idx"][r], s, n, k, what=f"row {r}")
+    assert flips <= 2
+    compare.close(got["out"][rows], ora["out"], what="prefill out")
+    np.testing.assert_allclose(got["lse"][rows], ora["lse"], rtol=1e-4, atol=1e-4)
+
+
+def check_cache(inp, got, ora):
+    P, T, m = inp["P"], inp["T"], inp["m"]
+    n0, n1 = P // m, (P + T) // m
+    np.testing.assert_array_equal(got["kv"][:n0], inp["kv"][:n0])  # prefix rows untouched
+    np.testing.assert_allclose(got["kv_scale"][n0:n1], ora["kv_scale"][n0:n1], rtol=1e-5)
+    diff = got["kv"][n0:n1] != ora["kv"][n0:n1]
+    assert diff.sum() <= max(4, diff.size // 5000), f"{diff.sum()} stored codes differ"
+
+
+@pytest.mark.parametrize("P,T,H,H_I,k", [
+    (512, 301, 64, 16, 64),     # a tail of one token; every row checked
+    (4096, 160, 128, 64, 1024), # n(t) around k: the set is everything, then a true top-k
+])
+def test_prefill_small_all_rows(P, T, H, H_I, k):
+    inp = synth.prefill_inputs(P, T, 4, H, H_I, seed=P + T)
+    got = run_prefill(inp, k)
+    rows = np.arange(T, dtype=np.int32)
+    ora = oracle.prefill(inp, k, rows)
+    check_cache(inp, got, ora)
+    check_rows(inp, k, got, rows, ora)
+
+
+def test_prefill_from_empty_prefix_over_two_query_chunks():
+    # P = 0: the first queries see no entry at all (n = 0) and a short window; 1100 queries
+    # span two launches of 1024
+    inp = synth.prefill_inputs(0, 1100, 4, 128, 32, seed=11)
+    got = run_prefill(inp, 128)
+    rows = np.array([0, 1, 2, 3, 4, 5, 127, 128, 511, 512, 1022, 1023, 1024, 1025, 1099],
+                    np.int32)
+    ora = oracle.prefill(inp, 128, rows)
+    check_cache(inp, got, ora)
+    check_rows(inp, 128, got, rows, ora)
+    assert (got["idx"][0] == -1).all() and (got["idx"][4][1:] == -1).all()
+
+
+def test_prefill_long_prefix_sampled_rows():
+    # the 1M-class shape scaled down: H = 128, H_I = 64, k = 1024, n(t) ~ 4.1-4.5K
+    P, T, k = 16384, 1536, 1024
+    inp = synth.prefill_inputs(P, T, 4, 128, 64, seed=4)
+    got = run_prefill(inp, k)
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, 1, 2, 3, 1023, 1024, T - 1],
+                                     rng.choice(T, 17, replace=False)])).astype(np.int32)
+    ora = oracle.prefill(inp, k, rows)
+    check_cache(inp, got, ora)
+    check_rows(inp, k, got, rows, ora)
+
+
+def test_prefill_without_derotation_and_deterministic():
+    inp = synth.prefill_inputs(1024, 200, 4, 64, 16, seed=9)
+    a = run_prefill(inp, 128, derotate=False)
+    b = run_prefill(inp, 128, derotate=False)
+    for key in ("out", "lse", "idx", "kv"):
+        np.testing.assert_array_equal(a[key], b[key])
+    rows = np.array([0, 57, 199], np.int32)
+    ora = oracle.prefill(inp, 128, rows, derotate=False)
+    check_rows(inp, 128, a, rows, ora)
