@@ -143,6 +143,23 @@ def prefill_flops(P: int, T: int, m: int, H: int, H_I: int, k: int) -> tuple[int
     return int(2 * H_I * 128 * n.sum()), int(4 * H * 512 * rows.sum())
 
 
+def max_over_ranks(vals: list[float], world: int, device) -> list[float]:
+    """Per-rank timings -> their maxima over all ranks (one all-reduce of a few floats,
+    outside the data path)."""
+    if world <= 1:
+        return list(vals)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor(vals, dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(x) for x in t]
+
+
+def whole_job_rate(units_per_rank: int, world: int, ms: float) -> float:
+    """Units processed by all ranks per second, from the slowest rank's time."""
+    return world * units_per_rank / (ms * 1e-3)
+
+
 def bench_prefill(args, rank: int, world: int, local: int) -> None:
     import torch
 
@@ -441,13 +458,9 @@ def main():
     e2e_graphs = [capture(lambda c=c: e2e_step(c), GRAPH_STEPS) for c in copies]
     e2e_ms = time_graphs(e2e_graphs, nprobe)
 
-    ms_step = ms_total / steps_run
-    if world > 1:
-        t = torch.tensor([ms_step, e2e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_step, e2e_ms = float(t[0]), float(t[1])
-    value = world * B / (ms_step * 1e-3)
-    e2e_value = world * B / (e2e_ms * 1e-3)
+    ms_step, e2e_ms = max_over_ranks([ms_total / steps_run, e2e_ms], world, "cuda")
+    value = whole_job_rate(B, world, ms_step)
+    e2e_value = whole_job_rate(B, world, e2e_ms)
 
     if rank == 0:
         idx_bytes, step_bytes = algorithmic_bytes(d)

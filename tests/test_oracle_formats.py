@@ -1,5 +1,7 @@
 """Pins of the oracle's number formats against library casts and the OCP tables."""
 
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -98,6 +100,28 @@ def test_key_scale_offsets_form_a_bijection_per_group():
     # entry r0 + 32*r1 keeps its four scales in one 32-bit word: 16*r0 + 4*r1
     assert [oracle.key_sf_offset(37, s) for s in range(4)] == [16 * 5 + 4 + s for s in range(4)]
     assert oracle.key_sf_offset(128 + 96 + 31, 3) == 512 + 16 * 31 + 12 + 3
+
+
+def _page_ratios():
+    path = os.path.join(os.path.dirname(__file__), "golden", "page_ratios.txt")
+    out = {}
+    for line in open(path):
+        if line.strip() and not line.startswith("#"):
+            name, value, tol = line.split()[:3]
+            out[name] = (float(value), float(tol))
+    return out
+
+
+def test_stored_format_reproduces_the_ratios_the_pages_state():
+    r = _page_ratios()
+    entry = 448 + 64 * 2 + 4  # stored entry: E4M3 dims + BF16 RoPE dims + fp32 scale
+    csa_tok = (entry + 64 + 4) / 4  # CSA entry and its FP4 indexer key per 4 tokens
+    hca_tok = entry / 128
+    gqa8_tok = 8 * 128 * 2 * 2
+    v, tol = r["kv_cache_vs_bf16_gqa8"]
+    assert abs((csa_tok + hca_tok) / 2 / gqa8_tok - v) <= tol
+    v, tol = r["fp8_bf16_split_vs_all_bf16"]
+    assert abs((448 + 64 * 2) / (512 * 2) - v) <= tol
 
 
 def test_storage_arithmetic_matches_pages():
