@@ -9,14 +9,17 @@
 namespace csa {
 cudaError_t launch_compress(const csa_compress_args& a, cudaStream_t stream);
 cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
-                                const CUtensorMap& kmap, cudaStream_t stream, int kshared);
+                                const CUtensorMap& kmap, cudaStream_t stream);
 size_t ix_workspace_size(int B, int64_t Nmax, int k);
+cudaError_t launch_prefill_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
+                                        const CUtensorMap& kmap, cudaStream_t stream);
 size_t at_workspace_size(int B, int H, int rows_max);
+cudaError_t launch_prefill_attn(const csa_attn_args& a, int64_t swa_base, const CUtensorMap& qmap,
+                                cudaStream_t stream);
 cudaError_t launch_prefill_prep(const csa_prefill_args& a, uint16_t* lin, int32_t* n_all,
                                 int32_t* pos_all, cudaStream_t stream);
 cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* workspace,
-                        const CUtensorMap& qmap, cudaStream_t stream, int64_t kv_bstride,
-                        int swa_linear, int64_t swa_base);
+                        const CUtensorMap& qmap, cudaStream_t stream);
 
 namespace {
 
@@ -78,7 +81,6 @@ struct PrefillWs {
   int32_t* pos_all;   // [T]
   uint16_t* lin;      // [T + 127][512] window rows in position order
   int32_t* idx;       // [chunk][k] selected sets when the caller passes none
-  char* at;           // attention workspace for one chunk
 };
 
 size_t prefill_ws_layout(int T, int64_t Nmax, int H, int k, char* base, PrefillWs* w) {
@@ -94,14 +96,13 @@ size_t prefill_ws_layout(int T, int64_t Nmax, int H, int k, char* base, PrefillW
   char* pos_all = take((size_t)T * 4);
   char* lin = take(((size_t)T + CSA_WINDOW - 1) * CSA_HEAD_DIM * 2);
   char* idx = take((size_t)qc * k * 4);
-  char* at = take(at_workspace_size(qc, H, k + CSA_WINDOW));
+  (void)H;
   if (w) {
     w->ix = ix;
     w->n_all = reinterpret_cast<int32_t*>(n_all);
     w->pos_all = reinterpret_cast<int32_t*>(pos_all);
     w->lin = reinterpret_cast<uint16_t*>(lin);
     w->idx = reinterpret_cast<int32_t*>(idx);
-    w->at = at;
   }
   return off;
 }
@@ -206,7 +207,7 @@ int csa_indexer_topk(const csa_topk_args* a, void* ws, size_t ws_bytes, csa_stre
       return CSA_ERR_CUDA;
   }
   return cuda_status(
-      launch_indexer_topk(*a, ws, sms, kmap, reinterpret_cast<cudaStream_t>(stream), 0));
+      launch_indexer_topk(*a, ws, sms, kmap, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t csa_attn_workspace_size(int32_t B, int32_t H, int32_t rows_max) {
@@ -246,8 +247,7 @@ static int attn_common(const csa_attn_args* a, int sparse, void* ws, size_t ws_b
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return CSA_ERR_CUDA;
   return cuda_status(
-      launch_attn(*a, sparse, rows_max, ws, qmap, reinterpret_cast<cudaStream_t>(stream), a->Nmax,
-                  0, 0));
+      launch_attn(*a, sparse, rows_max, ws, qmap, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int csa_sparse_attn_decode(const csa_attn_args* a, void* ws, size_t ws_bytes,
@@ -339,7 +339,7 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
     t.k_sf = a->k_sf;
     t.idx = idx;
     t.dev_status = a->dev_status;
-    e = launch_indexer_topk(t, w.ix, sms, kmap, stream, 1);
+    e = launch_prefill_indexer_topk(t, w.ix, sms, kmap, stream);
     if (e != cudaSuccess) return CSA_ERR_CUDA;
     csa_attn_args at;
     std::memset(&at, 0, sizeof(at));
@@ -363,8 +363,7 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
     at.dev_status = a->dev_status;
     CUtensorMap qmap;
     if (!encode_q_map(enc, &qmap, at.q, (int64_t)nq * a->H, a->H)) return CSA_ERR_CUDA;
-    e = launch_attn(at, 1, a->k + CSA_WINDOW, w.at, qmap, stream, 0, 1,
-                    a->P - (CSA_WINDOW - 1));
+    e = launch_prefill_attn(at, a->P - (CSA_WINDOW - 1), qmap, stream);
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
   return CSA_OK;

@@ -43,9 +43,6 @@ struct AtSmem {
 struct AtParams {
   int B, H, k, sparse, C;  // C = chunks per sequence in the workspace
   int64_t Nmax;
-  int64_t kv_bstride;      // entries between sequences in kv / kv_scale (0: one shared cache)
-  int swa_linear;          // 0: swa is a [B][128] ring; 1: swa holds consecutive positions
-  int64_t swa_base;        // linear mode: position of swa row 0 (shared by the batch)
   const int32_t* pos;
   const int32_t* idx;
   const int32_t* n_entries;
@@ -144,8 +141,8 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       const int j = p.sparse ? jsel : r;
       if (j >= 0 && j < n) {
         kind = 1;
-        src = p.kv + ((size_t)b * p.kv_bstride + j) * kRow;
-        s.scl[tid] = p.kv_scale + (size_t)b * p.kv_bstride + j;
+        src = p.kv + ((size_t)b * p.Nmax + j) * kRow;
+        s.scl[tid] = p.kv_scale + (size_t)b * p.Nmax + j;
       } else if (j != -1) {
         report(p.dev_status, CSA_ERR_DEVICE);
       }
@@ -153,9 +150,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       const int pp = t - (kWin - 1) + (r - nwin_first);
       if (pp >= 0) {
         kind = 2;
-        const size_t wrow = p.swa_linear ? (size_t)(pp - p.swa_base)
-                                         : (size_t)b * kWin + (pp % kWin);
-        src = reinterpret_cast<const uint8_t*>(p.swa + wrow * kD);
+        src = reinterpret_cast<const uint8_t*>(p.swa + ((size_t)b * kWin + (pp % kWin)) * kD);
       }
     }
     s.kind[tid] = kind;
@@ -421,6 +416,376 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AtParams p) {
   *reinterpret_cast<uint2*>(p.out + ((size_t)b * p.H + h) * kD + d0) = packed;
 }
 
+// ------------------------------------------------------------- prefill attention
+// A prefill has many queries over one cache, so each query keeps its Q on chip and walks
+// its whole row list: one CTA per (query, half of the 512 output dims). Rows come in
+// chunks of 32 through a double buffer:
+//   warps 0-3  gather and dequantise the chunk's rows to FP16 (full 512 dims, the same
+//              swizzled layout as the decode kernel);
+//   warp 4     issues S = Q V^T (M = 128 heads, N = 32, K = 512) into a TMEM buffer, then,
+//              once the chunk's P is ready, O[:, half] += P V[:, half] (N = 256, K = 32);
+//   warps 5-8  one thread per head: online softmax in the base-2 domain with a lazy
+//              rescale (O and the running sum are rescaled in TMEM only when the running
+//              maximum grows by more than 2^8), P written as FP16.
+// At the end the softmax threads divide by the running sum plus the sink term, de-rotate
+// the RoPE dims and store BF16 (and lse). S is computed by both CTAs of a query (each
+// needs all 512 dims of the products); O is split so that it fits TMEM next to S.
+constexpr int kPaRows = 32;
+constexpr int kPaThreads = 32 * 9;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct PaSmem {
+  uint8_t q[8][128 * 128];             // Q FP16: 8 K-blocks [128 heads x 64 dims], 128-B swizzle
+  uint8_t v[2][8][kPaRows * 128];      // rows FP16: 8 dim-blocks [32 rows x 64 dims]
+  uint8_t pm[2][128 * 64];             // P FP16 [128 heads x 32 rows], 64-B swizzle
+  int kind[2][kPaRows];
+  uint64_t q_full, v_full[2], v_free[2], s_full[2], p_full[2], o_done, done;
+  uint32_t tmem_base;
+  volatile int abort;
+};
+
+struct PaParams {
+  int H, k;
+  int64_t Nmax;
+  const int32_t* pos;
+  const int32_t* idx;
+  const int32_t* n_entries;
+  const uint8_t* kv;
+  const float* kv_scale;
+  const uint16_t* swa;  // window rows in position order, row 0 = position swa_base
+  int64_t swa_base;
+  const float* sink;
+  float tau, rope_base;
+  int derotate;
+  uint16_t* out;
+  float* lse;
+  int32_t* dev_status;
+};
+
+__device__ __forceinline__ void pa_store_v(PaSmem& s, int buf, int r, int ch, uint4 v) {
+  *reinterpret_cast<uint4*>(&s.v[buf][ch >> 3][r * 128 + (((ch & 7) ^ (r & 7)) << 4)]) = v;
+}
+
+__global__ void __launch_bounds__(kPaThreads, 1)
+    prefill_attn_kernel(const __grid_constant__ CUtensorMap qmap, PaParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  PaSmem& s = *reinterpret_cast<PaSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int b = blockIdx.x >> 1, hf = blockIdx.x & 1, tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
+  pdl_wait();
+  pdl_trigger();
+  int n = p.n_entries[b];
+  const int t = p.pos[b];
+  if (n < 0 || n > p.Nmax) {
+    if (tid == 0) report(p.dev_status, CSA_ERR_DEVICE);
+    n = n < 0 ? 0 : (int)p.Nmax;
+  }
+  const int rows_total = p.k + kWin;
+  const int nchunks = (rows_total + kPaRows - 1) / kPaRows;
+  if (tid == 0) {
+    mbar_init(&s.q_full, 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.v_full[i], 128);
+      mbar_init(&s.v_free[i], 1);
+      mbar_init(&s.s_full[i], 1);
+      mbar_init(&s.p_full[i], 128);
+    }
+    mbar_init(&s.o_done, 1);
+    mbar_init(&s.done, 1);
+    s.abort = 0;
+    mbar_fence_init();
+    prefetch_tensormap(&qmap);
+    mbar_arrive_expect_tx(&s.q_full, (uint32_t)p.H * kD * 2);
+    for (int blk = 0; blk < 8; ++blk) tma_load_2d(s.q[blk], &qmap, &s.q_full, blk * 64, b * p.H);
+  }
+  if (warp == 4) tmem_alloc(&s.tmem_base, 512);
+  if (p.H < 128) {  // Q rows H..127 are zero padding
+    for (int i = tid; i < 8 * (128 - p.H) * 8; i += kPaThreads) {
+      const int blk = i / ((128 - p.H) * 8), rem = i % ((128 - p.H) * 8);
+      *reinterpret_cast<uint4*>(&s.q[blk][p.H * 128 + rem * 16]) = make_uint4(0, 0, 0, 0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  const uint32_t t_o = tmem, t_s0 = tmem + 256;
+
+  if (warp < 4) {
+    // ---------------------------------------------------------- gather (128 threads)
+    const int pt = tid;  // 0..127
+    bool ok = mbar_wait(&s.q_full, 0, p.dev_status);
+    if (!ok) s.abort = 1;
+    for (int i = pt; i < 8 * p.H * 8; i += 128) {  // widen Q to FP16 in place
+      uint4* c16 = reinterpret_cast<uint4*>(&s.q[i / (p.H * 8)][(i % (p.H * 8)) * 16]);
+      *c16 = bf16x8_to_f16x8(*c16);
+    }
+    const int r = pt >> 2, qd = pt & 3;
+    for (int c = 0; c < nchunks; ++c) {
+      const int buf = c & 1;
+      if (s.abort || !mbar_wait(&s.v_free[buf], ((c >> 1) & 1) ^ 1, p.dev_status)) {
+        s.abort = 1;
+        break;
+      }
+      const int rl = c * kPaRows + r;  // position in the row list
+      int kind = 0;
+      const uint8_t* src = nullptr;
+      float scl = 0.f;
+      if (rl < p.k) {
+        const int j = p.idx[(size_t)b * p.k + rl];
+        if (j >= 0 && j < n) {
+          kind = 1;
+          src = p.kv + (size_t)j * kRow;
+          scl = __ldg(p.kv_scale + j);
+        } else if (j != -1 && qd == 0) {
+          report(p.dev_status, CSA_ERR_DEVICE);
+        }
+      } else if (rl < rows_total) {
+        const int pp = t - (kWin - 1) + (rl - p.k);
+        if (pp >= 0) {
+          kind = 2;
+          src = reinterpret_cast<const uint8_t*>(p.swa + (size_t)(pp - p.swa_base) * kD);
+        }
+      }
+      const int units = kind == 1 ? 36 : (kind == 2 ? 64 : 0);
+      uint4 bufv[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const int u = qd + 4 * i;
+        bufv[i] = u < units ? __ldg(reinterpret_cast<const uint4*>(src + 16 * u))
+                            : make_uint4(0, 0, 0, 0);
+      }
+      if (kind == 1) {
+#pragma unroll
+        for (int i = 0; i < 9; ++i) {
+          const int u = qd + 4 * i;
+          if (u < 28) {
+            uint4 lo, hi;
+            e4m3x16_to_f16(bufv[i], scl, &lo, &hi);
+            pa_store_v(s, buf, r, 2 * u, lo);
+            pa_store_v(s, buf, r, 2 * u + 1, hi);
+          } else {
+            pa_store_v(s, buf, r, 28 + u, bf16x8_to_f16x8(bufv[i]));
+          }
+        }
+      } else if (kind == 2) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pa_store_v(s, buf, r, qd + 4 * i, bf16x8_to_f16x8(bufv[i]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) pa_store_v(s, buf, r, qd + 4 * i, make_uint4(0, 0, 0, 0));
+      }
+      if (qd == 0) s.kind[buf][r] = kind;
+      fence_async_smem();
+      mbar_arrive(&s.v_full[buf]);
+    }
+  } else if (warp == 4) {
+    // ---------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      const uint32_t id_s = idesc_f16(128, kPaRows, false);
+      const uint32_t id_o = idesc_f16(128, 256, true);
+      auto issue_pv = [&](int c) -> bool {
+        const int cb = c & 1;
+        if (s.abort || !mbar_wait(&s.p_full[cb], (c >> 1) & 1, p.dev_status)) return false;
+        tc_fence_after();
+        for (int kk = 0; kk < 2; ++kk)
+          mma_f16(t_o, smem_desc(smem_u32(s.pm[cb]) + kk * 32, 16, 512, kSwizzle64B),
+                  smem_desc(smem_u32(s.v[cb][hf * 4]) + kk * 2048, kPaRows * 128, 1024,
+                            kSwizzle128B),
+                  id_o, (c > 0 || kk > 0) ? 1u : 0u);
+        mma_commit(&s.v_free[cb]);
+        mma_commit(&s.o_done);
+        return true;
+      };
+      bool ok = true;
+      for (int c = 0; c < nchunks && ok; ++c) {
+        const int buf = c & 1;
+        if (s.abort || !mbar_wait(&s.v_full[buf], (c >> 1) & 1, p.dev_status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t t_s = t_s0 + kPaRows * buf;
+        for (int kk = 0; kk < 32; ++kk) {
+          const uint32_t off = (kk & 3) * 32;
+          mma_f16(t_s, smem_desc(smem_u32(s.q[kk >> 2]) + off, 16, 1024, kSwizzle128B),
+                  smem_desc(smem_u32(s.v[buf][kk >> 2]) + off, 16, 1024, kSwizzle128B), id_s,
+                  kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&s.s_full[buf]);
+        if (c > 0) ok = issue_pv(c - 1);
+      }
+      if (ok) ok = issue_pv(nchunks - 1);
+      if (!ok) s.abort = 1;
+      mma_commit(&s.done);
+      mbar_wait(&s.done, 0, p.dev_status);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax (128 threads)
+    const int quad = warp & 3, h = quad * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(quad * 32) << 16;
+    const float scale2 = p.tau * kLog2e;
+    float m_run = -INFINITY, l_run = 0.f;
+    bool ok = true;
+    for (int c = 0; c < nchunks; ++c) {
+      const int buf = c & 1, ph = (c >> 1) & 1;
+      bool w = true;
+      if (lane == 0)
+        w = !s.abort && mbar_wait(&s.s_full[buf], ph, p.dev_status) &&
+            mbar_wait(&s.v_full[buf], ph, p.dev_status) &&
+            (c == 0 || mbar_wait(&s.o_done, (c - 1) & 1, p.dev_status));
+      if (!__shfl_sync(0xffffffffu, w, 0)) {
+        s.abort = 1;
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[32];
+      tmem_ld32(t_s0 + kPaRows * buf + lane_off, r);
+      tmem_ld_wait();
+      float lg[kPaRows];
+      float m_c = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < kPaRows; ++e) {
+        lg[e] = s.kind[buf][e] ? __uint_as_float(r[e]) * scale2 : -INFINITY;
+        m_c = fmaxf(m_c, lg[e]);
+      }
+      // lazy rescale: move the reference maximum only when it grows by more than 2^8
+      const bool need = m_c > -INFINITY && (m_run == -INFINITY || m_c > m_run + 8.f);
+      if (__any_sync(0xffffffffu, need)) {
+        const float f = need ? (m_run == -INFINITY ? 0.f : exp2f(m_run - m_c)) : 1.f;
+        if (need) {
+          l_run *= f;
+          m_run = m_c;
+        }
+        if (c > 0) {  // O holds chunks 0..c-1 (complete: o_done was waited above)
+          for (int cc = 0; cc < 8; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(t_o + lane_off + cc * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(t_o + lane_off + cc * 32, o);
+          }
+          tmem_st_wait();
+        }
+      }
+      uint8_t* prow = s.pm[buf] + h * 64;
+      float lsum = 0.f;
+#pragma unroll
+      for (int ch = 0; ch < 4; ++ch) {
+        uint32_t wv[4];
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const int e = ch * 8 + 2 * e2;
+          const float p0 = (m_run == -INFINITY || lg[e] == -INFINITY) ? 0.f : exp2f(lg[e] - m_run);
+          const float p1 =
+              (m_run == -INFINITY || lg[e + 1] == -INFINITY) ? 0.f : exp2f(lg[e + 1] - m_run);
+          lsum += p0 + p1;
+          wv[e2] = pack_half2(p0, p1);
+        }
+        *reinterpret_cast<uint4*>(prow + ((ch ^ ((h >> 1) & 3)) << 4)) =
+            make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      }
+      l_run += lsum;
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(&s.p_full[buf]);
+    }
+    // every PV has completed: normalise, de-rotate, store
+    bool fin = ok;
+    if (lane == 0 && fin) fin = mbar_wait(&s.o_done, (nchunks - 1) & 1, p.dev_status);
+    fin = __shfl_sync(0xffffffffu, fin, 0) != 0;
+    if (fin) {
+      tc_fence_after();
+      const float sink2 = p.sink[h < p.H ? h : 0] * kLog2e;
+      float Z = l_run;
+      if (sink2 != -INFINITY) Z += (m_run == -INFINITY) ? (sink2 == INFINITY ? INFINITY : exp2f(sink2))
+                                                        : exp2f(sink2 - m_run);
+      const float inv = Z > 0.f ? 1.f / Z : 0.f;
+      for (int cc = 0; cc < 8; ++cc) {
+        uint32_t o[32];
+        tmem_ld32(t_o + lane_off + cc * 32, o);
+        tmem_ld_wait();
+        float v[32];
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
+        const int d0 = hf * 256 + cc * 32;
+        if (p.derotate && d0 >= kNope) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            float cs, sn;
+            rope_cos_sin((double)t, (d0 + e - kNope) >> 1, (double)p.rope_base, &cs, &sn);
+            const float x0 = v[e], x1 = v[e + 1];
+            v[e] = x0 * cs + x1 * sn;
+            v[e + 1] = -x0 * sn + x1 * cs;
+          }
+        }
+        if (h < p.H) {
+          uint4* dst = reinterpret_cast<uint4*>(p.out + ((size_t)b * p.H + h) * kD + d0);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              w4[e] = (uint32_t)f32_to_bf16_bits(v[q4 * 8 + 2 * e]) |
+                      ((uint32_t)f32_to_bf16_bits(v[q4 * 8 + 2 * e + 1]) << 16);
+            dst[q4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          }
+        }
+      }
+      if (hf == 0 && h < p.H && p.lse) {
+        float l;
+        if (Z == INFINITY) l = INFINITY;
+        else if (Z <= 0.f) l = -INFINITY;
+        else l = (m_run == -INFINITY ? log2f(Z) : m_run + log2f(Z)) / kLog2e;
+        p.lse[(size_t)b * p.H + h] = l;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+cudaError_t launch_prefill_attn(const csa_attn_args& a, int64_t swa_base, const CUtensorMap& qmap,
+                                cudaStream_t stream) {
+  PaParams p;
+  p.H = a.H;
+  p.k = a.k;
+  p.Nmax = a.Nmax;
+  p.pos = a.pos;
+  p.idx = a.idx;
+  p.n_entries = a.n_entries;
+  p.kv = a.kv;
+  p.kv_scale = a.kv_scale;
+  p.swa = a.swa;
+  p.swa_base = swa_base;
+  p.sink = a.sink;
+  p.tau = a.tau > 0.f ? a.tau : 0.044194173824159216f;
+  p.rope_base = a.rope_base;
+  p.derotate = a.derotate;
+  p.out = a.out;
+  p.lse = a.lse;
+  p.dev_status = a.dev_status;
+  const size_t smem = sizeof(PaSmem) + 1024;
+  static int configured = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured != dev) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = dev;
+  }
+  return launch_pdl(prefill_attn_kernel, dim3(2 * a.B), dim3(kPaThreads), smem, stream, qmap, p);
+}
+
 size_t at_smem_bytes() { return sizeof(AtSmem) + 1024; }
 
 size_t at_workspace_size(int B, int H, int rows_max) {
@@ -430,8 +795,7 @@ size_t at_workspace_size(int B, int H, int rows_max) {
 }
 
 cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* workspace,
-                        const CUtensorMap& qmap, cudaStream_t stream, int64_t kv_bstride,
-                        int swa_linear, int64_t swa_base) {
+                        const CUtensorMap& qmap, cudaStream_t stream) {
   AtParams p;
   p.B = a.B;
   p.H = a.H;
@@ -439,9 +803,6 @@ cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* 
   p.sparse = sparse;
   p.C = (rows_max + kAtRows - 1) / kAtRows;
   p.Nmax = a.Nmax;
-  p.kv_bstride = kv_bstride;
-  p.swa_linear = swa_linear;
-  p.swa_base = swa_base;
   p.pos = a.pos;
   p.idx = a.idx;
   p.n_entries = a.n_entries;

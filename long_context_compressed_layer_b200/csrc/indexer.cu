@@ -78,7 +78,12 @@ struct IxSmem {
 // be zero when a call starts sits at the front at offsets that do not depend on B: the
 // grid barrier, then one fixed-size block per sequence (counters, rule, histogram). A call
 // with fewer sequences therefore finds its blocks where a larger call left them zeroed.
-constexpr int kSeqWords = 8 + kHist;  // per-sequence block: counters[4], rule[4], hist
+// The global histogram of a sequence is kept in kHistRep copies: the epilogue warps of
+// every CTA add into copy (pipeline * 4 + warp) % kHistRep, so the atomics that land on
+// one hot bin are spread over kHistRep addresses instead of queueing on one; the
+// selection sums the copies.
+constexpr int kHistRep = 8;
+constexpr int kSeqWords = 8 + kHistRep * kHist;  // counters[4], rule[4], hist copies
 
 struct IxWs {
   uint32_t* grid_bar;   // [2]: arrival count, generation (grid-wide barrier)
@@ -90,7 +95,7 @@ struct IxWs {
   // counters: candidate count, ticket; rule: cut key, cut index, selected count, ready flag
   __device__ uint32_t* counters(int b) const { return seq + (size_t)b * kSeqWords; }
   __device__ uint32_t* rule(int b) const { return seq + (size_t)b * kSeqWords + 4; }
-  __device__ uint32_t* hist(int b) const { return seq + (size_t)b * kSeqWords + 8; }
+  __device__ uint32_t* hist(int b) const { return seq + (size_t)b * kSeqWords + 8; }  // [kHistRep][kHist]
 };
 static_assert((kSeqWords * 4) % 16 == 0, "histograms stay 16-byte aligned");
 
@@ -133,8 +138,7 @@ size_t ix_workspace_size(int B, int64_t Nmax, int k) {
 
 struct IxParams {
   int B, H_I, k;
-  int fused;    // 1: the selection follows in this (cooperative) launch
-  int kshared;  // 1: every query scores the same key rows (the queries of one prefill)
+  int fused;  // 1: the selection follows in this (cooperative) launch
   int64_t Nmax;
   const int32_t* n_entries;
   const uint8_t* q_fp4;
@@ -260,10 +264,9 @@ __device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
           s.abort = 1;
           break;
         }
-        const int kb = p.kshared ? 0 : b;  // key sequence
         mbar_arrive_expect_tx(&s.full[st], kIxKeyBytes + kIxSfBytes);
-        tma_load_3d(s.keys[st], &kmap, &s.full[st], 0, t * kIxTile, kb);
-        bulk_load(s.ksf[st], p.k_sf + ((size_t)kb * (p.Nmax / kIxTile) + t) * kIxSfBytes,
+        tma_load_3d(s.keys[st], &kmap, &s.full[st], 0, t * kIxTile, b);
+        bulk_load(s.ksf[st], p.k_sf + ((size_t)b * (p.Nmax / kIxTile) + t) * kIxSfBytes,
                   kIxSfBytes, &s.full[st]);
       }
       // drain: every copy this warp issued has landed before the CTA winds down
@@ -357,9 +360,9 @@ __device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
     uint32_t* hist = s.hist[ew];
     int b = -1, n_b = 0, since_flush = 0;
     float w[kIxN];
-    auto flush = [&](int bb) {  // warp-local: add the warp's counts to the global histogram
+    auto flush = [&](int bb) {  // warp-local: add the warp's counts to its histogram copy
       __syncwarp();
-      uint32_t* gh = p.ws.hist(bb);
+      uint32_t* gh = p.ws.hist(bb) + (size_t)((warp % kIxPipeWarps + kIxEpiWarps * (warp / kIxPipeWarps)) % kHistRep) * kHist;
       for (int i = lane; i < kHist / 2; i += 32) {
         const uint32_t v = hist[i];
         if (v) {
@@ -473,21 +476,20 @@ __device__ __forceinline__ void load_scores(const float* sc, int j, int end,
     }
   } else {
 #pragma unroll
-    for (int e = 0; e < kSelPer; ++e) v[e] = j + e < end ? __ldcg(sc + j + e) : 0.f;
+    for (int e = 0; e < kSelPer; ++e) v[e] = 0.f;
+    if (j < end) {  // the ragged end of the last slice: plain loads of what exists
+      float t[kSelPer];
+#pragma unroll
+      for (int e = 0; e < kSelPer; ++e) t[e] = j + e < end ? __ldcg(sc + j + e) : 0.f;
+#pragma unroll
+      for (int e = 0; e < kSelPer; ++e) v[e] = t[e];
+    }
   }
 }
 
-__device__ __forceinline__ void warp_append(bool pred, uint32_t* counter, uint32_t* slot_out) {
-  const uint32_t m = __ballot_sync(0xffffffffu, pred);
-  uint32_t base = 0;
-  const int lane = threadIdx.x & 31;
-  if (m) {
-    const int leader = __ffs(m) - 1;
-    if (lane == leader) base = atomicAdd(counter, __popc(m));
-    base = __shfl_sync(0xffffffffu, base, leader);
-  }
-  *slot_out = base + __popc(m & ((1u << lane) - 1));
-}
+// The selection runs once per CTA, so its code is executed cold: it is kept compact
+// (non-inlined steps, no per-element atomics in unrolled loops) to limit instruction
+// fetch stalls.
 
 // Candidates come from shared memory (staged) or, past its capacity, from global memory.
 __device__ __forceinline__ uint64_t cand_at(const uint64_t* cand, uint32_t i, bool staged) {
@@ -498,7 +500,7 @@ __device__ __forceinline__ uint64_t cand_at(const uint64_t* cand, uint32_t i, bo
 // `mask`, histogram the digit (field >> shift) & (2^bits - 1) and find the digit where the
 // running count (from the top when `descending`, else from the bottom) reaches *remaining.
 // Updates *prefix / *remaining (shared). Field: key = cand >> 32 (hi) or index (lo).
-__device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, bool hi,
+__device__ __noinline__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, bool hi,
                            uint32_t key_eq, bool need_key_eq, uint32_t mask, int shift,
                            int bits, bool descending, uint32_t* prefix, uint32_t* remaining,
                            uint32_t* h, uint32_t* digit_pop = nullptr) {
@@ -554,8 +556,8 @@ __device__ __forceinline__ int slices_of(int n) {
 // Phase 1 of the selection for slice sb of sequence b: the threshold bin (highest bin whose
 // suffix count reaches k), the slice's count above it and its in-bin candidates. The last
 // slice of the sequence to finish resolves the exact cut (finalize).
-__device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb,
-                                 uint32_t ready_gen) {
+__device__ __noinline__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb,
+                                              uint32_t ready_gen) {
   const int tid = threadIdx.x;
   const int n = clamp_n(p.n_entries[b], p.Nmax, p.dev_status);
   const int k_eff = n < p.k ? n : p.k;
@@ -568,16 +570,20 @@ __device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb
   if (n > p.k) {
     const uint4* gh = reinterpret_cast<const uint4*>(p.ws.hist(b));
     constexpr int nv = kHist / 4, vper = (nv + kSelThreads - 1) / kSelThreads;
-    uint4 hv[vper];  // every load in flight before any is stored
 #pragma unroll
     for (int i = 0; i < vper; ++i) {
       const int q = tid + i * kSelThreads;
-      hv[i] = q < nv ? __ldcg(gh + q) : make_uint4(0, 0, 0, 0);
-    }
+      if (q < nv) {
+        uint4 hv[kHistRep];  // every copy's load in flight before any is summed
 #pragma unroll
-    for (int i = 0; i < vper; ++i) {
-      const int q = tid + i * kSelThreads;
-      if (q < nv) reinterpret_cast<uint4*>(x.h)[q] = hv[i];
+        for (int r = 0; r < kHistRep; ++r) hv[r] = __ldcg(gh + r * nv + q);
+        uint4 t = hv[0];
+#pragma unroll
+        for (int r = 1; r < kHistRep; ++r) {
+          t.x += hv[r].x; t.y += hv[r].y; t.z += hv[r].z; t.w += hv[r].w;
+        }
+        reinterpret_cast<uint4*>(x.h)[q] = t;
+      }
     }
     __syncthreads();
     constexpr int per = (kHist + kSelThreads - 1) / kSelThreads;  // thread 0 holds the top
@@ -605,18 +611,32 @@ __device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb
   const int jt = j0 + tid * kSelPer;
   float v[kSelPer];
   load_scores(sc, jt, j1, v);
-  uint32_t above = 0;
+  uint32_t above = 0, eqm = 0;
 #pragma unroll
   for (int e = 0; e < kSelPer; ++e) {
-    const int j = jt + e;
-    const bool in = j < j1;
-    const uint32_t key = float_key(v[e]);
-    const int bin = in ? (int)(key >> (32 - kHistBits)) : -2;
+    const bool in = jt + e < j1;
+    const int bin = in ? (int)(float_key(v[e]) >> kLowBits) : -2;
     above += (in && bin > tbin) ? 1u : 0u;
-    const bool eq = in && bin == tbin;
-    uint32_t slot;
-    warp_append(eq, &cnt[0], &slot);
-    if (eq) {
+    eqm |= (uint32_t)(in && bin == tbin) << e;
+  }
+  {  // append this thread's in-bin candidates: one counter atomic per warp
+    const int lane = tid & 31;
+    const uint32_t ne = __popc(eqm);
+    uint32_t incl = ne;
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const uint32_t wtotal = __shfl_sync(0xffffffffu, incl, 31);
+    uint32_t base = 0;
+    if (wtotal) {
+      if (lane == 31) base = atomicAdd(&cnt[0], wtotal);
+      base = __shfl_sync(0xffffffffu, base, 31);
+    }
+    uint32_t slot = base + incl - ne;
+    for (uint32_t m = eqm; m; m &= m - 1, ++slot) {
+      const int j = jt + __ffs(m) - 1;
+      const uint32_t key = float_key(__ldcg(sc + j));
       if (slot < (uint32_t)p.Nmax) p.ws.cand[(size_t)b * p.Nmax + slot] = ((uint64_t)key << 32) | (uint32_t)j;
       else report(p.dev_status, CSA_ERR_DEVICE);
     }
@@ -740,7 +760,8 @@ __device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb
     cnt[1] = 0;
   }
   uint32_t* gh = p.ws.hist(b);
-  for (int i = tid; i < kHist; i += kSelThreads) gh[i] = 0;
+  for (int i = tid; i < kHistRep * kHist / 4; i += kSelThreads)
+    reinterpret_cast<uint4*>(gh)[i] = make_uint4(0, 0, 0, 0);
   __syncthreads();
   if (tid == 0 && p.fused) {  // publish the rule and offsets of this sequence
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.ws.rule(b) + 3),
@@ -752,7 +773,7 @@ __device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb
 }
 
 // Phase 2: slice sb of sequence b writes its selected entries, in index order, at its offset.
-__device__ void select_write(const IxParams& p, SelScratch& x, int b, int sb) {
+__device__ __noinline__ void select_write(const IxParams& p, SelScratch& x, int b, int sb) {
   const int tid = threadIdx.x;
   int n = p.n_entries[b];
   n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
@@ -776,16 +797,13 @@ __device__ void select_write(const IxParams& p, SelScratch& x, int b, int sb) {
   const uint32_t mine = __popc(mask);
   const uint32_t incl = block_incl_scan(mine, x.tmp, nullptr);
   uint32_t slot = off + incl - mine;
-#pragma unroll
-  for (int e = 0; e < kSelPer; ++e) {
-    if (mask & (1u << e)) {
-      if (slot < (uint32_t)p.k) {
-        out[slot] = jt + e;
-        if (p.scores_out) p.scores_out[(size_t)b * p.k + slot] = v[e];
-      } else {
-        report(p.dev_status, CSA_ERR_DEVICE);
-      }
-      ++slot;
+  for (uint32_t m = mask; m; m &= m - 1, ++slot) {
+    const int j = jt + __ffs(m) - 1;
+    if (slot < (uint32_t)p.k) {
+      out[slot] = j;
+      if (p.scores_out) p.scores_out[(size_t)b * p.k + slot] = __ldcg(sc + j);
+    } else {
+      report(p.dev_status, CSA_ERR_DEVICE);
     }
   }
   if (sb == 0) {
@@ -857,12 +875,310 @@ __global__ void __launch_bounds__(kSelThreads) topk_write_kernel(IxParams p) {
   if (sb < slices_of(n)) select_write(p, *reinterpret_cast<SelScratch*>(raw), b, sb);
 }
 
+// ------------------------------------------------------------- prefill scoring
+// In a prefill every query of the call scores the same key array (one sequence), so the
+// key stream is shared: a 128-entry key tile is loaded once for a group of kPxQ
+// consecutive queries and meets their kPxQ x 64 heads in kPxQ block-scaled MMAs
+// (D[128 entries x 64 heads] each, 2 x K = 64), instead of once per query. The roles are
+// those of the decode kernel with one pipeline per CTA: a TMA producer warp, a tcgen05
+// issuer warp that also stages each group's queries and scales, and eight epilogue warps
+// in two groups of four taking alternate tiles (accumulator buffer = tile parity). An
+// epilogue thread owns one entry and forms its kPxQ scores, masked by each query's own
+// eligible count, and counts them into per-warp, per-query histograms. The selection then
+// runs as the two stand-alone kernels, one CTA per (slice, query).
+constexpr int kPxQ = 3;                     // queries per group
+constexpr int kPxStages = 6;
+constexpr int kPxNbuf = 2;                  // accumulator buffers (one per epilogue group)
+constexpr int kPxEpiWarps = 8;
+constexpr int kPxThreads = 32 * (2 + kPxEpiWarps);
+constexpr int kPxGroupCols = kPxQ * kIxN;   // TMEM columns of one buffer
+constexpr int kPxTmemCols = 512;
+constexpr int kPxMaxG = (kIxMaxB + kPxQ - 1) / kPxQ;
+static_assert(kPxNbuf * kPxGroupCols + 8 + 8 * kPxQ <= kPxTmemCols, "TMEM budget");
+
+struct alignas(1024) PxSmem {
+  uint8_t keys[kPxStages][kIxKeyBytes];
+  uint8_t q[2][kPxQ][kIxN * 64];
+  uint32_t hist[kPxEpiWarps][kPxQ][kHist / 2];
+  uint8_t ksf[kPxStages][kIxSfBytes];
+  uint8_t qsf[2][kPxQ][512];
+  float w[kPxEpiWarps][kPxQ][kIxN];
+  int32_t prefix[kPxMaxG + 1];
+  uint64_t full[kPxStages], empty[kPxStages];
+  uint64_t acc_full[kPxNbuf], acc_empty[kPxNbuf], q_free[2], done;
+  uint32_t tmem_base;
+  volatile int abort;
+};
+
+__global__ void __launch_bounds__(kPxThreads, 1)
+    prefill_score_kernel(const __grid_constant__ CUtensorMap kmap, IxParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  PxSmem& s = *reinterpret_cast<PxSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = (p.B + kPxQ - 1) / kPxQ;
+  if (warp == 1 && lane == 0) {
+    for (int i = 0; i < kPxStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], 1);
+    }
+    for (int i = 0; i < kPxNbuf; ++i) {
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_empty[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) mbar_init(&s.q_free[i], 1);
+    mbar_init(&s.done, 1);
+    s.abort = 0;
+    mbar_fence_init();
+  }
+  if (threadIdx.x == 0) prefetch_tensormap(&kmap);
+  {
+    uint32_t* hz = &s.hist[0][0][0];
+    for (int i = threadIdx.x; i < kPxEpiWarps * kPxQ * kHist / 2; i += kPxThreads) hz[i] = 0;
+  }
+  if (warp == 1) tmem_alloc(&s.tmem_base, kPxTmemCols);
+  pdl_wait();
+  pdl_trigger();
+  // group g holds queries kPxQ*g .. kPxQ*g + kPxQ - 1 and ceil(max n / 128) key tiles
+  if (warp == 0) {
+    int carry = 0;
+    if (lane == 0) s.prefix[0] = 0;
+    for (int base = 0; base < G; base += 32) {
+      const int g = base + lane;
+      int v = 0;
+      if (g < G) {
+        int nmax = 0;
+        for (int qq = 0; qq < kPxQ; ++qq) {
+          const int qi = kPxQ * g + qq;
+          if (qi < p.B) nmax = max(nmax, clamp_n(p.n_entries[qi], p.Nmax, p.dev_status));
+        }
+        v = (nmax + kIxTile - 1) / kIxTile;
+      }
+      int incl = v;
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      if (g < G) s.prefix[g + 1] = carry + incl;
+      carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const int total = s.prefix[G];
+  const int g0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
+  const int g1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
+  const uint32_t tmem = s.tmem_base;
+  const uint32_t t_sfa = tmem + kPxNbuf * kPxGroupCols;
+  int gr0 = 0;  // first group of this CTA
+  if (g0 < g1)
+    while (s.prefix[gr0 + 1] <= g0) ++gr0;
+
+  if (g0 < g1 && warp == 0) {
+    // ---------------------------------------------------------------- producer
+    if (lane == 0) {
+      int gr = gr0, it = 0;
+      for (int g = g0; g < g1; ++g, ++it) {
+        while (s.prefix[gr + 1] <= g) ++gr;
+        const int t = g - s.prefix[gr];
+        const int st = it % kPxStages;
+        if (s.abort || !mbar_wait(&s.empty[st], ((it / kPxStages) & 1) ^ 1, p.dev_status)) {
+          s.abort = 1;
+          break;
+        }
+        mbar_arrive_expect_tx(&s.full[st], kIxKeyBytes + kIxSfBytes);
+        tma_load_3d(s.keys[st], &kmap, &s.full[st], 0, t * kIxTile, 0);
+        bulk_load(s.ksf[st], p.k_sf + (size_t)t * kIxSfBytes, kIxSfBytes, &s.full[st]);
+      }
+      const int issued = it;
+      for (int i = issued - kPxStages < 0 ? 0 : issued - kPxStages; i < issued; ++i)
+        mbar_wait(&s.full[i % kPxStages], (i / kPxStages) & 1, p.dev_status);
+    }
+  } else if (g0 < g1 && warp == 1) {
+    // ---------------------------------------------------------------- MMA issuer
+    int gr = -1, ngr = -1, it = 0;
+    uint32_t qslot = 0;
+    for (int g = g0; g < g1; ++g, ++it) {
+      int nb = gr < 0 ? gr0 : gr;
+      while (s.prefix[nb + 1] <= g) ++nb;
+      if (nb != gr) {  // stage the group's queries (B operands) and their scales
+        if (gr >= 0 && lane == 0) mma_commit(&s.q_free[qslot]);
+        gr = nb;
+        ++ngr;
+        qslot = ngr & 1;
+        bool ok = true;
+        if (lane == 0)
+          ok = !s.abort && mbar_wait(&s.q_free[qslot], ((ngr >> 1) & 1) ^ 1, p.dev_status);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) { s.abort = 1; break; }
+        for (int qq = 0; qq < kPxQ; ++qq) {
+          const int qi = kPxQ * gr + qq;
+          const bool has = qi < p.B;
+          const uint8_t* qsrc = p.q_fp4 + (size_t)(has ? qi : 0) * p.H_I * 64;
+          for (int c = lane; c < kIxN * 4; c += 32) {  // 16-byte chunks, 64-byte swizzle
+            const int r = c >> 2, ch = c & 3;
+            uint4 v = make_uint4(0, 0, 0, 0);
+            if (has && r < p.H_I) v = *reinterpret_cast<const uint4*>(qsrc + r * 64 + ch * 16);
+            *reinterpret_cast<uint4*>(&s.q[qslot][qq][r * 64 + ((ch ^ ((r >> 1) & 3)) << 4)]) = v;
+          }
+          uint32_t wv[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int n = lane + 32 * j;
+            wv[j] = (has && n < p.H_I)
+                        ? *reinterpret_cast<const uint32_t*>(p.q_sf + ((size_t)qi * p.H_I + n) * 4)
+                        : 0x7F7F7F7Fu;
+          }
+          *reinterpret_cast<uint4*>(&s.qsf[qslot][qq][lane * 16]) =
+              make_uint4(wv[0], wv[1], wv[2], wv[3]);
+        }
+        fence_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tc_fence_after();
+          for (int qq = 0; qq < kPxQ; ++qq)
+            tmem_cp_32x128b_x4(t_sfa + 8 + 8 * qq,
+                               smem_desc(smem_u32(s.qsf[qslot][qq]), 0, 128, kSwizzleNone));
+        }
+      }
+      if (lane == 0) {
+        const int st = it % kPxStages, bb = it % kPxNbuf;
+        bool ok = !s.abort;
+        if (ok) {
+          ok = mbar_wait(&s.acc_empty[bb], ((it / kPxNbuf) & 1) ^ 1, p.dev_status);
+          tc_fence_after();
+        }
+        ok = ok && mbar_wait(&s.full[st], (it / kPxStages) & 1, p.dev_status);
+        if (!ok) {
+          s.abort = 1;
+        } else {
+          tmem_cp_32x128b_x4(t_sfa, smem_desc(smem_u32(s.ksf[st]), 0, 128, kSwizzleNone));
+          const uint32_t ka = smem_u32(s.keys[st]);
+          for (int qq = 0; qq < kPxQ; ++qq) {
+            const uint32_t qa = smem_u32(s.q[qslot][qq]);
+#pragma unroll
+            for (int kh = 0; kh < 2; ++kh)
+              mma_mxf4(tmem + bb * kPxGroupCols + qq * kIxN,
+                       smem_desc(ka + 32 * kh, 16, 512, kSwizzle64B),
+                       smem_desc(qa + 32 * kh, 16, 512, kSwizzle64B),
+                       idesc_mxf4(kIxTile, kIxN, 2 * kh), t_sfa, t_sfa + 8 + 8 * qq, kh);
+          }
+          mma_commit(&s.empty[st]);
+          mma_commit(&s.acc_full[bb]);
+        }
+      }
+      if (__shfl_sync(0xffffffffu, s.abort, 0)) break;
+    }
+    if (lane == 0) {
+      mma_commit(&s.done);
+      mbar_wait(&s.done, 0, p.dev_status);
+    }
+    __syncwarp();
+  } else if (g0 < g1) {
+    // ---------------------------------------------------------------- epilogue
+    const int ew = warp - 2, grp = ew >> 2, quad = warp & 3, row = quad * 32 + lane;
+    const int ntiles = g1 - g0;
+    const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+    float* wq = &s.w[ew][0][0];
+    int gr = -1, since_flush = 0, gseq = gr0;
+    int nq[kPxQ];
+    auto flush = [&](int gg) {
+      __syncwarp();
+      for (int qq = 0; qq < kPxQ; ++qq) {
+        const int qi = kPxQ * gg + qq;
+        uint32_t* hist = s.hist[ew][qq];
+        uint32_t* gh = qi < p.B ? p.ws.hist(qi) + (size_t)(ew % kHistRep) * kHist : nullptr;
+        for (int i = lane; i < kHist / 2; i += 32) {
+          const uint32_t v = hist[i];
+          if (v) {
+            if (gh) {
+              if (v & 0xFFFFu) atomicAdd(gh + 2 * i, v & 0xFFFFu);
+              if (v >> 16) atomicAdd(gh + 2 * i + 1, v >> 16);
+            }
+            hist[i] = 0;
+          }
+        }
+      }
+      __syncwarp();
+    };
+    for (int it = grp; it < ntiles; it += kPxNbuf) {
+      const int bb = it % kPxNbuf;
+      bool ok = true;
+      if (lane == 0)
+        ok = !s.abort && mbar_wait(&s.acc_full[bb], (it / kPxNbuf) & 1, p.dev_status);
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
+        s.abort = 1;
+        break;
+      }
+      tc_fence_after();
+      const int g = g0 + it;
+      while (s.prefix[gseq + 1] <= g) ++gseq;
+      if (gseq != gr || since_flush >= 2000) {
+        if (gr >= 0) flush(gr);
+        since_flush = 0;
+        gr = gseq;
+        for (int qq = 0; qq < kPxQ; ++qq) {
+          const int qi = kPxQ * gr + qq;
+          nq[qq] = qi < p.B ? clamp_n(p.n_entries[qi], p.Nmax, nullptr) : 0;
+          for (int h = lane; h < kIxN; h += 32)
+            wq[qq * kIxN + h] = (qi < p.B && h < p.H_I) ? __ldg(p.w + (size_t)qi * p.H_I + h) : 0.f;
+        }
+        __syncwarp();
+      }
+      ++since_flush;
+      const int j = (g - s.prefix[gr]) * kIxTile + row;
+      for (int qq = 0; qq < kPxQ; ++qq) {
+        uint32_t r[2][32];
+        const uint32_t ta = lane_base + bb * kPxGroupCols + qq * kIxN;
+        tmem_ld32(ta, r[0]);
+        tmem_ld32(ta + 32, r[1]);
+        tmem_ld_wait();
+        const float4* w4 = reinterpret_cast<const float4*>(wq + qq * kIxN);
+        float part[8];
+#pragma unroll
+        for (int k8 = 0; k8 < 8; ++k8) part[k8] = 0.f;
+#pragma unroll
+        for (int h4 = 0; h4 < kIxN / 4; ++h4) {
+          const float4 wv = w4[h4];
+          const int h = 4 * h4;
+          part[h & 7] = fmaf(wv.x, fmaxf(__uint_as_float(r[h >> 5][h & 31]), 0.f), part[h & 7]);
+          part[(h + 1) & 7] =
+              fmaf(wv.y, fmaxf(__uint_as_float(r[(h + 1) >> 5][(h + 1) & 31]), 0.f), part[(h + 1) & 7]);
+          part[(h + 2) & 7] =
+              fmaf(wv.z, fmaxf(__uint_as_float(r[(h + 2) >> 5][(h + 2) & 31]), 0.f), part[(h + 2) & 7]);
+          part[(h + 3) & 7] =
+              fmaf(wv.w, fmaxf(__uint_as_float(r[(h + 3) >> 5][(h + 3) & 31]), 0.f), part[(h + 3) & 7]);
+        }
+        const float sc = ((part[0] + part[1]) + (part[2] + part[3])) +
+                         ((part[4] + part[5]) + (part[6] + part[7]));
+        if (j < nq[qq]) {
+          const int qi = kPxQ * gr + qq;
+          p.ws.scores[(size_t)qi * p.Nmax + j] = sc;
+          const uint32_t bin = float_key(sc) >> kLowBits;
+          atomicAdd(&s.hist[ew][qq][bin >> 1], 1u << (16 * (bin & 1)));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.acc_empty[bb]);
+    }
+    if (gr >= 0) flush(gr);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kPxTmemCols);
+  }
+}
+
 // ------------------------------------------------------------------- launch
 cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
-                                const CUtensorMap& kmap, cudaStream_t stream, int kshared) {
+                                const CUtensorMap& kmap, cudaStream_t stream) {
   IxWs ws;
   ix_ws_layout(a.B, a.Nmax, a.k, (char*)workspace, &ws);
-  IxParams p{a.B, a.H_I, a.k, 1, kshared, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
+  IxParams p{a.B, a.H_I, a.k, 1, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
              a.idx, a.scores, a.dev_status};
   const size_t smem = sizeof(IxSmem) + 1024;
   static int configured = -1;
@@ -909,5 +1225,32 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
 }
 
 size_t ix_smem_bytes() { return sizeof(IxSmem) + 1024; }
+
+// Indexer top-k of the queries of one prefill (all scoring the same keys): the shared-key
+// scoring kernel, then the two selection kernels.
+cudaError_t launch_prefill_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
+                                        const CUtensorMap& kmap, cudaStream_t stream) {
+  IxWs ws;
+  ix_ws_layout(a.B, a.Nmax, a.k, (char*)workspace, &ws);
+  IxParams p{a.B, a.H_I, a.k, 0, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
+             a.idx, a.scores, a.dev_status};
+  const size_t smem = sizeof(PxSmem) + 1024;
+  static int configured = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (configured != dev) {
+    cudaError_t e = cudaFuncSetAttribute(prefill_score_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured = dev;
+  }
+  cudaError_t e = launch_pdl(prefill_score_kernel, dim3(num_sms), dim3(kPxThreads), smem,
+                             stream, kmap, p);
+  if (e != cudaSuccess) return e;
+  dim3 g2((unsigned)ws.S, a.B);
+  e = launch_pdl(topk_threshold_kernel, g2, dim3(kSelThreads), 0, stream, p);
+  if (e != cudaSuccess) return e;
+  return launch_pdl(topk_write_kernel, g2, dim3(kSelThreads), 0, stream, p);
+}
 
 }  // namespace csa
