@@ -14,9 +14,11 @@ size_t ix_workspace_size(int B, int64_t Nmax, int k);
 cudaError_t launch_prefill_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
                                         const CUtensorMap& kmap, cudaStream_t stream);
 size_t at_workspace_size(int B, int H, int rows_max);
-cudaError_t launch_prefill_attn(const csa_attn_args& a, int64_t swa_base, const CUtensorMap& qmap,
-                                cudaStream_t stream);
-cudaError_t launch_prefill_prep(const csa_prefill_args& a, uint16_t* lin, int32_t* n_all,
+cudaError_t launch_prefill_attn(const csa_attn_args& a, const __half* rows16, int64_t swa_base,
+                                const CUtensorMap& qmap, cudaStream_t stream);
+cudaError_t launch_prefill_rows16(const uint8_t* kv, const float* kv_scale, int64_t n,
+                                  __half* rows16, cudaStream_t stream);
+cudaError_t launch_prefill_prep(const csa_prefill_args& a, __half* lin, int32_t* n_all,
                                 int32_t* pos_all, cudaStream_t stream);
 cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* workspace,
                         const CUtensorMap& qmap, cudaStream_t stream);
@@ -79,7 +81,7 @@ struct PrefillWs {
   char* ix;           // indexer workspace for kPrefillChunk queries (kept zeroed)
   int32_t* n_all;     // [T]
   int32_t* pos_all;   // [T]
-  uint16_t* lin;      // [T + 127][512] window rows in position order
+  __half* rows16;     // FP16 rows: [Nmax] entries, then [T + 127] window rows in position order
   int32_t* idx;       // [chunk][k] selected sets when the caller passes none
 };
 
@@ -94,14 +96,14 @@ size_t prefill_ws_layout(int T, int64_t Nmax, int H, int k, char* base, PrefillW
   char* ix = take(ix_workspace_size(qc, Nmax, k));
   char* n_all = take((size_t)T * 4);
   char* pos_all = take((size_t)T * 4);
-  char* lin = take(((size_t)T + CSA_WINDOW - 1) * CSA_HEAD_DIM * 2);
+  char* rows16 = take(((size_t)Nmax + T + CSA_WINDOW - 1) * CSA_HEAD_DIM * 2);
   char* idx = take((size_t)qc * k * 4);
   (void)H;
   if (w) {
     w->ix = ix;
     w->n_all = reinterpret_cast<int32_t*>(n_all);
     w->pos_all = reinterpret_cast<int32_t*>(pos_all);
-    w->lin = reinterpret_cast<uint16_t*>(lin);
+    w->rows16 = reinterpret_cast<__half*>(rows16);
     w->idx = reinterpret_cast<int32_t*>(idx);
   }
   return off;
@@ -316,8 +318,12 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
   c.Nmax = a->Nmax;
   cudaError_t e = launch_compress(c, stream);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
-  // 2. per-query lengths, positions and the window rows in position order
-  e = launch_prefill_prep(*a, w.lin, w.n_all, w.pos_all, stream);
+  // 2. per-query lengths, positions; FP16 rows of the entries and of the window in
+  //    position order
+  e = launch_prefill_prep(*a, w.rows16 + (size_t)a->Nmax * CSA_HEAD_DIM, w.n_all, w.pos_all,
+                          stream);
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  e = launch_prefill_rows16(a->kv, a->kv_scale, (a->P + a->T) / a->m, w.rows16, stream);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   // 3. per chunk of queries: indexer top-k over the shared keys, then attention
   CUtensorMap kmap;
@@ -353,7 +359,7 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
     at.n_entries = w.n_all + c0;
     at.kv = a->kv;
     at.kv_scale = a->kv_scale;
-    at.swa = w.lin;
+    at.swa = nullptr;
     at.sink = a->sink;
     at.tau = a->tau;
     at.rope_base = a->rope_base;
@@ -363,7 +369,7 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
     at.dev_status = a->dev_status;
     CUtensorMap qmap;
     if (!encode_q_map(enc, &qmap, at.q, (int64_t)nq * a->H, a->H)) return CSA_ERR_CUDA;
-    e = launch_prefill_attn(at, a->P - (CSA_WINDOW - 1), qmap, stream);
+    e = launch_prefill_attn(at, w.rows16, a->P - (CSA_WINDOW - 1), qmap, stream);
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
   return CSA_OK;

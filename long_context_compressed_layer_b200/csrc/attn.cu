@@ -418,10 +418,11 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AtParams p) {
 
 // ------------------------------------------------------------- prefill attention
 // A prefill has many queries over one cache, so each query keeps its Q on chip and walks
-// its whole row list: one CTA per (query, half of the 512 output dims). Rows come in
-// chunks of 32 through a double buffer:
-//   warps 0-3  gather and dequantise the chunk's rows to FP16 (full 512 dims, the same
-//              swizzled layout as the decode kernel);
+// its whole row list: one CTA per (query, half of the 512 output dims). The cache entries
+// and the window rows are dequantised to FP16 once per call (prefill_rows16_kernel), so the
+// per-query gather is a plain copy. Rows come in chunks of 32 through a double buffer:
+//   warps 0-3  gather the chunk's rows with 16-byte cp.async copies straight into the
+//              swizzled layout of the decode kernel (no register staging);
 //   warp 4     issues S = Q V^T (M = 128 heads, N = 32, K = 512) into a TMEM buffer, then,
 //              once the chunk's P is ready, O[:, half] += P V[:, half] (N = 256, K = 32);
 //   warps 5-8  one thread per head: online softmax in the base-2 domain with a lazy
@@ -439,7 +440,7 @@ struct PaSmem {
   uint8_t v[2][8][kPaRows * 128];      // rows FP16: 8 dim-blocks [32 rows x 64 dims]
   uint8_t pm[2][128 * 64];             // P FP16 [128 heads x 32 rows], 64-B swizzle
   int kind[2][kPaRows];
-  uint64_t q_full, v_full[2], v_free[2], s_full[2], p_full[2], o_done, done;
+  uint64_t q_full, v_full[2], v_free[2], s_full[2], p_full[2], o_done[2], done;
   uint32_t tmem_base;
   volatile int abort;
 };
@@ -450,9 +451,7 @@ struct PaParams {
   const int32_t* pos;
   const int32_t* idx;
   const int32_t* n_entries;
-  const uint8_t* kv;
-  const float* kv_scale;
-  const uint16_t* swa;  // window rows in position order, row 0 = position swa_base
+  const __half* rows16;  // FP16 rows: entries 0..Nmax-1, then window positions from swa_base
   int64_t swa_base;
   const float* sink;
   float tau, rope_base;
@@ -490,8 +489,8 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       mbar_init(&s.v_free[i], 1);
       mbar_init(&s.s_full[i], 1);
       mbar_init(&s.p_full[i], 128);
+      mbar_init(&s.o_done[i], 1);  // P V of the chunks with this parity
     }
-    mbar_init(&s.o_done, 1);
     mbar_init(&s.done, 1);
     s.abort = 0;
     mbar_fence_init();
@@ -522,6 +521,8 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       *c16 = bf16x8_to_f16x8(*c16);
     }
     const int r = pt >> 2, qd = pt & 3;
+    const int64_t self_row = p.Nmax + (t - p.swa_base);  // always present: stands in for
+                                                         // rows that carry no weight
     for (int c = 0; c < nchunks; ++c) {
       const int buf = c & 1;
       if (s.abort || !mbar_wait(&s.v_free[buf], ((c >> 1) & 1) ^ 1, p.dev_status)) {
@@ -530,14 +531,12 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       }
       const int rl = c * kPaRows + r;  // position in the row list
       int kind = 0;
-      const uint8_t* src = nullptr;
-      float scl = 0.f;
+      int64_t row = self_row;
       if (rl < p.k) {
         const int j = p.idx[(size_t)b * p.k + rl];
         if (j >= 0 && j < n) {
           kind = 1;
-          src = p.kv + (size_t)j * kRow;
-          scl = __ldg(p.kv_scale + j);
+          row = j;
         } else if (j != -1 && qd == 0) {
           report(p.dev_status, CSA_ERR_DEVICE);
         }
@@ -545,39 +544,22 @@ __global__ void __launch_bounds__(kPaThreads, 1)
         const int pp = t - (kWin - 1) + (rl - p.k);
         if (pp >= 0) {
           kind = 2;
-          src = reinterpret_cast<const uint8_t*>(p.swa + (size_t)(pp - p.swa_base) * kD);
+          row = p.Nmax + (pp - p.swa_base);
         }
       }
-      const int units = kind == 1 ? 36 : (kind == 2 ? 64 : 0);
-      uint4 bufv[16];
+      const __half* src = p.rows16 + row * kD;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        const int u = qd + 4 * i;
-        bufv[i] = u < units ? __ldg(reinterpret_cast<const uint4*>(src + 16 * u))
-                            : make_uint4(0, 0, 0, 0);
+        const int u = qd + 4 * i;  // 16-byte piece = 8 dims
+        const uint32_t dst =
+            smem_u32(&s.v[buf][u >> 3][r * 128 + (((u & 7) ^ (r & 7)) << 4)]);
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src + 8 * u)
+                     : "memory");
       }
-      if (kind == 1) {
-#pragma unroll
-        for (int i = 0; i < 9; ++i) {
-          const int u = qd + 4 * i;
-          if (u < 28) {
-            uint4 lo, hi;
-            e4m3x16_to_f16(bufv[i], scl, &lo, &hi);
-            pa_store_v(s, buf, r, 2 * u, lo);
-            pa_store_v(s, buf, r, 2 * u + 1, hi);
-          } else {
-            pa_store_v(s, buf, r, 28 + u, bf16x8_to_f16x8(bufv[i]));
-          }
-        }
-      } else if (kind == 2) {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pa_store_v(s, buf, r, qd + 4 * i, bf16x8_to_f16x8(bufv[i]));
-      } else {
-#pragma unroll
-        for (int i = 0; i < 16; ++i) pa_store_v(s, buf, r, qd + 4 * i, make_uint4(0, 0, 0, 0));
-      }
+      asm volatile("cp.async.commit_group;" ::: "memory");
       if (qd == 0) s.kind[buf][r] = kind;
-      fence_async_smem();
+      asm volatile("cp.async.wait_group 0;" ::: "memory");
+      fence_async_smem();  // the copies (and the widened Q) are read by tcgen05.mma
       mbar_arrive(&s.v_full[buf]);
     }
   } else if (warp == 4) {
@@ -595,7 +577,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
                             kSwizzle128B),
                   id_o, (c > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&s.v_free[cb]);
-        mma_commit(&s.o_done);
+        mma_commit(&s.o_done[cb]);
         return true;
       };
       bool ok = true;
@@ -629,14 +611,22 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     const float scale2 = p.tau * kLog2e;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
+    // P V of chunk c completes phase c >> 1 of o_done[c & 1]; the next phase of that
+    // barrier needs this warp's P of chunk c + 2, so a wait never trails by two phases
+    auto wait_pv = [&](int c) -> bool {
+      bool w = true;
+      if (lane == 0) w = mbar_wait(&s.o_done[c & 1], (c >> 1) & 1, p.dev_status);
+      return __shfl_sync(0xffffffffu, w, 0) != 0;
+    };
     for (int c = 0; c < nchunks; ++c) {
       const int buf = c & 1, ph = (c >> 1) & 1;
       bool w = true;
       if (lane == 0)
         w = !s.abort && mbar_wait(&s.s_full[buf], ph, p.dev_status) &&
-            mbar_wait(&s.v_full[buf], ph, p.dev_status) &&
-            (c == 0 || mbar_wait(&s.o_done, (c - 1) & 1, p.dev_status));
-      if (!__shfl_sync(0xffffffffu, w, 0)) {
+            mbar_wait(&s.v_full[buf], ph, p.dev_status);
+      w = __shfl_sync(0xffffffffu, w, 0) != 0;
+      if (w && c >= 2) w = wait_pv(c - 2);  // P[buf] was last read by P V of chunk c-2
+      if (!w) {
         s.abort = 1;
         ok = false;
         break;
@@ -655,12 +645,17 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       // lazy rescale: move the reference maximum only when it grows by more than 2^8
       const bool need = m_c > -INFINITY && (m_run == -INFINITY || m_c > m_run + 8.f);
       if (__any_sync(0xffffffffu, need)) {
+        if (c > 0 && !wait_pv(c - 1)) {  // O must hold chunks 0..c-1 before it is rescaled
+          s.abort = 1;
+          ok = false;
+          break;
+        }
         const float f = need ? (m_run == -INFINITY ? 0.f : exp2f(m_run - m_c)) : 1.f;
         if (need) {
           l_run *= f;
           m_run = m_c;
         }
-        if (c > 0) {  // O holds chunks 0..c-1 (complete: o_done was waited above)
+        if (c > 0) {
           for (int cc = 0; cc < 8; ++cc) {
             uint32_t o[32];
             tmem_ld32(t_o + lane_off + cc * 32, o);
@@ -695,9 +690,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       mbar_arrive(&s.p_full[buf]);
     }
     // every PV has completed: normalise, de-rotate, store
-    bool fin = ok;
-    if (lane == 0 && fin) fin = mbar_wait(&s.o_done, (nchunks - 1) & 1, p.dev_status);
-    fin = __shfl_sync(0xffffffffu, fin, 0) != 0;
+    const bool fin = ok && wait_pv(nchunks - 1);
     if (fin) {
       tc_fence_after();
       const float sink2 = p.sink[h < p.H ? h : 0] * kLog2e;
@@ -753,8 +746,40 @@ __global__ void __launch_bounds__(kPaThreads, 1)
   }
 }
 
-cudaError_t launch_prefill_attn(const csa_attn_args& a, int64_t swa_base, const CUtensorMap& qmap,
-                                cudaStream_t stream) {
+// Dequantise stored entries 0 .. n-1 to FP16 rows (E4M3 code x entry scale rounded once,
+// BF16 RoPE dims widened exactly): the same values the decode gather stages. One warp
+// per entry; lanes 0-27 take 16 E4M3 dims each, lanes 28-31 take 16 BF16 dims each.
+__global__ void __launch_bounds__(256) prefill_rows16_kernel(const uint8_t* kv, const float* kv_scale,
+                                                             int64_t n, __half* rows16) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t j = (int64_t)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (j >= n) return;
+  const uint8_t* row = kv + j * kRow;
+  uint4* dst = reinterpret_cast<uint4*>(rows16 + j * kD);
+  if (lane < 28) {
+    uint4 lo, hi;
+    e4m3x16_to_f16(*reinterpret_cast<const uint4*>(row + 16 * lane), __ldg(kv_scale + j), &lo, &hi);
+    dst[2 * lane] = lo;
+    dst[2 * lane + 1] = hi;
+  } else {
+    const int q = lane - 28;
+    const uint4* src = reinterpret_cast<const uint4*>(row + kNope + 32 * q);
+    dst[56 + 2 * q] = bf16x8_to_f16x8(src[0]);
+    dst[56 + 2 * q + 1] = bf16x8_to_f16x8(src[1]);
+  }
+}
+
+cudaError_t launch_prefill_rows16(const uint8_t* kv, const float* kv_scale, int64_t n,
+                                  __half* rows16, cudaStream_t stream) {
+  if (n <= 0) return cudaSuccess;
+  return launch_pdl(prefill_rows16_kernel, dim3((unsigned)((n + 7) / 8)), dim3(256), 0, stream,
+                    kv, kv_scale, n, rows16);
+}
+
+cudaError_t launch_prefill_attn(const csa_attn_args& a, const __half* rows16, int64_t swa_base,
+                                const CUtensorMap& qmap, cudaStream_t stream) {
   PaParams p;
   p.H = a.H;
   p.k = a.k;
@@ -762,9 +787,7 @@ cudaError_t launch_prefill_attn(const csa_attn_args& a, int64_t swa_base, const 
   p.pos = a.pos;
   p.idx = a.idx;
   p.n_entries = a.n_entries;
-  p.kv = a.kv;
-  p.kv_scale = a.kv_scale;
-  p.swa = a.swa;
+  p.rows16 = rows16;
   p.swa_base = swa_base;
   p.sink = a.sink;
   p.tau = a.tau > 0.f ? a.tau : 0.044194173824159216f;

@@ -7,16 +7,27 @@
 //   n_all[r]  = floor((P + r + 1) / m), the entries eligible at position t = P + r;
 //   pos_all[r] = P + r;
 //   lin[i], i = 0 .. T + 126: the window row of position P - 127 + i in consecutive order,
-//     copied from the prefix ring swa_prefix[p % 128] for p < P (rows of negative
+//     taken from the prefix ring swa_prefix[p % 128] for p < P (rows of negative
 //     positions are never read and are left as they are), and for p >= P formed from the
 //     token itself: RMSNorm (fp32, eps, optional weight) of a[p - P], RoPE at position p
-//     on the interleaved pairs of dims 448..511, rounded to BF16.
+//     on the interleaved pairs of dims 448..511, rounded to BF16. The rows are stored
+//     widened to FP16 (exact for the BF16 values of normalised rows), the form the
+//     attention kernel stages.
 // One warp per row; lane l owns dims 16l .. 16l + 15 (two 16-byte loads and stores), so a
 // 1 KB row moves in one coalesced pass. The squares are summed per lane, then by a fixed
 // butterfly, so the result does not depend on scheduling.
 #include "common.cuh"
 
 namespace csa {
+
+// 8 BF16 values -> 8 FP16 values (the same conversion the attention staging applies)
+__device__ __forceinline__ uint4 bf16x8_widen(uint4 v) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    w[e] = pack_half2(bf16_bits_to_f32(w[e] & 0xFFFF), bf16_bits_to_f32(w[e] >> 16));
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
 
 struct PrepParams {
   int64_t P;
@@ -25,7 +36,7 @@ struct PrepParams {
   const uint16_t* a;
   const float* norm_w;
   const uint16_t* swa_prefix;
-  uint16_t* lin;
+  __half* lin;
   int32_t* n_all;
   int32_t* pos_all;
 };
@@ -46,8 +57,8 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(PrepParams p) {
   if (pp < 0) return;
   if (pp < p.P) {
     const uint4* src = reinterpret_cast<const uint4*>(p.swa_prefix + (pp % kWin) * kD + 16 * lane);
-    dst[0] = src[0];
-    dst[1] = src[1];
+    dst[0] = bf16x8_widen(src[0]);
+    dst[1] = bf16x8_widen(src[1]);
     return;
   }
   const uint4* src = reinterpret_cast<const uint4*>(p.a + (pp - p.P) * kD + 16 * lane);
@@ -79,13 +90,14 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(PrepParams p) {
   }
   uint32_t o[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e)
-    o[e] = (uint32_t)f32_to_bf16_bits(y[2 * e]) | ((uint32_t)f32_to_bf16_bits(y[2 * e + 1]) << 16);
+  for (int e = 0; e < 8; ++e)  // the BF16 window value, then its exact FP16 form
+    o[e] = pack_half2(bf16_bits_to_f32(f32_to_bf16_bits(y[2 * e])),
+                      bf16_bits_to_f32(f32_to_bf16_bits(y[2 * e + 1])));
   dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
   dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-cudaError_t launch_prefill_prep(const csa_prefill_args& a, uint16_t* lin, int32_t* n_all,
+cudaError_t launch_prefill_prep(const csa_prefill_args& a, __half* lin, int32_t* n_all,
                                 int32_t* pos_all, cudaStream_t stream) {
   PrepParams p{a.P, a.T, a.m, a.eps, a.rope_base, a.a, a.norm_w, a.swa_prefix, lin, n_all,
                pos_all};

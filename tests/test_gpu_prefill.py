@@ -36,12 +36,15 @@ def run_prefill(inp, k, derotate=True):
     opt = {x: dev(inp[x]) for x in ("prev_b", "prev_zb") if x in inp}
     if inp["P"] > 0:
         opt["swa_prefix"] = dev(inp["swa_prefix"])
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
     out, lse, idx = csa.prefill(
         inp["P"], inp["m"], k, a=dev(inp["a"]), b=dev(inp["b"]), za=dev(inp["za"]),
         zb=dev(inp["zb"]), bias=dev(inp["bias"]), kv=kv, kv_scale=sc, q_fp4=dev(inp["q_fp4"]),
         q_sf=dev(inp["q_sf"]), w=dev(inp["w"]), k_fp4=dev(inp["k_fp4"]), k_sf=dev(inp["k_sf"]),
-        q=dev(inp["q"]), sink=dev(inp["sink"]), derotate=derotate, lse=True, idx=True, **opt)
+        q=dev(inp["q"]), sink=dev(inp["sink"]), derotate=derotate, lse=True, idx=True,
+        dev_status=st, **opt)
     torch.cuda.synchronize()
+    assert int(st.item()) == 0, f"device status {int(st.item())}"
     return dict(out=out.float().cpu().numpy(), lse=host(lse), idx=host(idx), kv=host(kv),
                 kv_scale=host(sc))
 
