@@ -78,12 +78,7 @@ struct IxSmem {
 // be zero when a call starts sits at the front at offsets that do not depend on B: the
 // grid barrier, then one fixed-size block per sequence (counters, rule, histogram). A call
 // with fewer sequences therefore finds its blocks where a larger call left them zeroed.
-// The global histogram of a sequence is kept in kHistRep copies: the epilogue warps of
-// every CTA add into copy (pipeline * 4 + warp) % kHistRep, so the atomics that land on
-// one hot bin are spread over kHistRep addresses instead of queueing on one; the
-// selection sums the copies.
-constexpr int kHistRep = 8;
-constexpr int kSeqWords = 8 + kHistRep * kHist;  // counters[4], rule[4], hist copies
+constexpr int kSeqWords = 8 + kHist;  // per-sequence block: counters[4], rule[4], hist
 
 struct IxWs {
   uint32_t* grid_bar;   // [2]: arrival count, generation (grid-wide barrier)
@@ -95,7 +90,7 @@ struct IxWs {
   // counters: candidate count, ticket; rule: cut key, cut index, selected count, ready flag
   __device__ uint32_t* counters(int b) const { return seq + (size_t)b * kSeqWords; }
   __device__ uint32_t* rule(int b) const { return seq + (size_t)b * kSeqWords + 4; }
-  __device__ uint32_t* hist(int b) const { return seq + (size_t)b * kSeqWords + 8; }  // [kHistRep][kHist]
+  __device__ uint32_t* hist(int b) const { return seq + (size_t)b * kSeqWords + 8; }
 };
 static_assert((kSeqWords * 4) % 16 == 0, "histograms stay 16-byte aligned");
 
@@ -360,9 +355,9 @@ __device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
     uint32_t* hist = s.hist[ew];
     int b = -1, n_b = 0, since_flush = 0;
     float w[kIxN];
-    auto flush = [&](int bb) {  // warp-local: add the warp's counts to its histogram copy
+    auto flush = [&](int bb) {  // warp-local: add the warp's counts to the global histogram
       __syncwarp();
-      uint32_t* gh = p.ws.hist(bb) + (size_t)((warp % kIxPipeWarps + kIxEpiWarps * (warp / kIxPipeWarps)) % kHistRep) * kHist;
+      uint32_t* gh = p.ws.hist(bb);
       for (int i = lane; i < kHist / 2; i += 32) {
         const uint32_t v = hist[i];
         if (v) {
@@ -476,20 +471,21 @@ __device__ __forceinline__ void load_scores(const float* sc, int j, int end,
     }
   } else {
 #pragma unroll
-    for (int e = 0; e < kSelPer; ++e) v[e] = 0.f;
-    if (j < end) {  // the ragged end of the last slice: plain loads of what exists
-      float t[kSelPer];
-#pragma unroll
-      for (int e = 0; e < kSelPer; ++e) t[e] = j + e < end ? __ldcg(sc + j + e) : 0.f;
-#pragma unroll
-      for (int e = 0; e < kSelPer; ++e) v[e] = t[e];
-    }
+    for (int e = 0; e < kSelPer; ++e) v[e] = j + e < end ? __ldcg(sc + j + e) : 0.f;
   }
 }
 
-// The selection runs once per CTA, so its code is executed cold: it is kept compact
-// (non-inlined steps, no per-element atomics in unrolled loops) to limit instruction
-// fetch stalls.
+__device__ __forceinline__ void warp_append(bool pred, uint32_t* counter, uint32_t* slot_out) {
+  const uint32_t m = __ballot_sync(0xffffffffu, pred);
+  uint32_t base = 0;
+  const int lane = threadIdx.x & 31;
+  if (m) {
+    const int leader = __ffs(m) - 1;
+    if (lane == leader) base = atomicAdd(counter, __popc(m));
+    base = __shfl_sync(0xffffffffu, base, leader);
+  }
+  *slot_out = base + __popc(m & ((1u << lane) - 1));
+}
 
 // Candidates come from shared memory (staged) or, past its capacity, from global memory.
 __device__ __forceinline__ uint64_t cand_at(const uint64_t* cand, uint32_t i, bool staged) {
@@ -500,7 +496,7 @@ __device__ __forceinline__ uint64_t cand_at(const uint64_t* cand, uint32_t i, bo
 // `mask`, histogram the digit (field >> shift) & (2^bits - 1) and find the digit where the
 // running count (from the top when `descending`, else from the bottom) reaches *remaining.
 // Updates *prefix / *remaining (shared). Field: key = cand >> 32 (hi) or index (lo).
-__device__ __noinline__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, bool hi,
+__device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, bool hi,
                            uint32_t key_eq, bool need_key_eq, uint32_t mask, int shift,
                            int bits, bool descending, uint32_t* prefix, uint32_t* remaining,
                            uint32_t* h, uint32_t* digit_pop = nullptr) {
@@ -556,8 +552,8 @@ __device__ __forceinline__ int slices_of(int n) {
 // Phase 1 of the selection for slice sb of sequence b: the threshold bin (highest bin whose
 // suffix count reaches k), the slice's count above it and its in-bin candidates. The last
 // slice of the sequence to finish resolves the exact cut (finalize).
-__device__ __noinline__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb,
-                                              uint32_t ready_gen) {
+__device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb,
+                                 uint32_t ready_gen) {
   const int tid = threadIdx.x;
   const int n = clamp_n(p.n_entries[b], p.Nmax, p.dev_status);
   const int k_eff = n < p.k ? n : p.k;
@@ -570,20 +566,16 @@ __device__ __noinline__ void select_threshold(const IxParams& p, SelScratch& x, 
   if (n > p.k) {
     const uint4* gh = reinterpret_cast<const uint4*>(p.ws.hist(b));
     constexpr int nv = kHist / 4, vper = (nv + kSelThreads - 1) / kSelThreads;
+    uint4 hv[vper];  // every load in flight before any is stored
 #pragma unroll
     for (int i = 0; i < vper; ++i) {
       const int q = tid + i * kSelThreads;
-      if (q < nv) {
-        uint4 hv[kHistRep];  // every copy's load in flight before any is summed
+      hv[i] = q < nv ? __ldcg(gh + q) : make_uint4(0, 0, 0, 0);
+    }
 #pragma unroll
-        for (int r = 0; r < kHistRep; ++r) hv[r] = __ldcg(gh + r * nv + q);
-        uint4 t = hv[0];
-#pragma unroll
-        for (int r = 1; r < kHistRep; ++r) {
-          t.x += hv[r].x; t.y += hv[r].y; t.z += hv[r].z; t.w += hv[r].w;
-        }
-        reinterpret_cast<uint4*>(x.h)[q] = t;
-      }
+    for (int i = 0; i < vper; ++i) {
+      const int q = tid + i * kSelThreads;
+      if (q < nv) reinterpret_cast<uint4*>(x.h)[q] = hv[i];
     }
     __syncthreads();
     constexpr int per = (kHist + kSelThreads - 1) / kSelThreads;  // thread 0 holds the top
@@ -611,32 +603,18 @@ __device__ __noinline__ void select_threshold(const IxParams& p, SelScratch& x, 
   const int jt = j0 + tid * kSelPer;
   float v[kSelPer];
   load_scores(sc, jt, j1, v);
-  uint32_t above = 0, eqm = 0;
+  uint32_t above = 0;
 #pragma unroll
   for (int e = 0; e < kSelPer; ++e) {
-    const bool in = jt + e < j1;
-    const int bin = in ? (int)(float_key(v[e]) >> kLowBits) : -2;
+    const int j = jt + e;
+    const bool in = j < j1;
+    const uint32_t key = float_key(v[e]);
+    const int bin = in ? (int)(key >> (32 - kHistBits)) : -2;
     above += (in && bin > tbin) ? 1u : 0u;
-    eqm |= (uint32_t)(in && bin == tbin) << e;
-  }
-  {  // append this thread's in-bin candidates: one counter atomic per warp
-    const int lane = tid & 31;
-    const uint32_t ne = __popc(eqm);
-    uint32_t incl = ne;
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += y;
-    }
-    const uint32_t wtotal = __shfl_sync(0xffffffffu, incl, 31);
-    uint32_t base = 0;
-    if (wtotal) {
-      if (lane == 31) base = atomicAdd(&cnt[0], wtotal);
-      base = __shfl_sync(0xffffffffu, base, 31);
-    }
-    uint32_t slot = base + incl - ne;
-    for (uint32_t m = eqm; m; m &= m - 1, ++slot) {
-      const int j = jt + __ffs(m) - 1;
-      const uint32_t key = float_key(__ldcg(sc + j));
+    const bool eq = in && bin == tbin;
+    uint32_t slot;
+    warp_append(eq, &cnt[0], &slot);
+    if (eq) {
       if (slot < (uint32_t)p.Nmax) p.ws.cand[(size_t)b * p.Nmax + slot] = ((uint64_t)key << 32) | (uint32_t)j;
       else report(p.dev_status, CSA_ERR_DEVICE);
     }
@@ -760,8 +738,7 @@ __device__ __noinline__ void select_threshold(const IxParams& p, SelScratch& x, 
     cnt[1] = 0;
   }
   uint32_t* gh = p.ws.hist(b);
-  for (int i = tid; i < kHistRep * kHist / 4; i += kSelThreads)
-    reinterpret_cast<uint4*>(gh)[i] = make_uint4(0, 0, 0, 0);
+  for (int i = tid; i < kHist; i += kSelThreads) gh[i] = 0;
   __syncthreads();
   if (tid == 0 && p.fused) {  // publish the rule and offsets of this sequence
     asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.ws.rule(b) + 3),
@@ -773,7 +750,7 @@ __device__ __noinline__ void select_threshold(const IxParams& p, SelScratch& x, 
 }
 
 // Phase 2: slice sb of sequence b writes its selected entries, in index order, at its offset.
-__device__ __noinline__ void select_write(const IxParams& p, SelScratch& x, int b, int sb) {
+__device__ void select_write(const IxParams& p, SelScratch& x, int b, int sb) {
   const int tid = threadIdx.x;
   int n = p.n_entries[b];
   n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
@@ -797,13 +774,16 @@ __device__ __noinline__ void select_write(const IxParams& p, SelScratch& x, int 
   const uint32_t mine = __popc(mask);
   const uint32_t incl = block_incl_scan(mine, x.tmp, nullptr);
   uint32_t slot = off + incl - mine;
-  for (uint32_t m = mask; m; m &= m - 1, ++slot) {
-    const int j = jt + __ffs(m) - 1;
-    if (slot < (uint32_t)p.k) {
-      out[slot] = j;
-      if (p.scores_out) p.scores_out[(size_t)b * p.k + slot] = __ldcg(sc + j);
-    } else {
-      report(p.dev_status, CSA_ERR_DEVICE);
+#pragma unroll
+  for (int e = 0; e < kSelPer; ++e) {
+    if (mask & (1u << e)) {
+      if (slot < (uint32_t)p.k) {
+        out[slot] = jt + e;
+        if (p.scores_out) p.scores_out[(size_t)b * p.k + slot] = v[e];
+      } else {
+        report(p.dev_status, CSA_ERR_DEVICE);
+      }
+      ++slot;
     }
   }
   if (sb == 0) {
@@ -1088,7 +1068,7 @@ __global__ void __launch_bounds__(kPxThreads, 1)
       for (int qq = 0; qq < kPxQ; ++qq) {
         const int qi = kPxQ * gg + qq;
         uint32_t* hist = s.hist[ew][qq];
-        uint32_t* gh = qi < p.B ? p.ws.hist(qi) + (size_t)(ew % kHistRep) * kHist : nullptr;
+        uint32_t* gh = qi < p.B ? p.ws.hist(qi) : nullptr;
         for (int i = lane; i < kHist / 2; i += 32) {
           const uint32_t v = hist[i];
           if (v) {
@@ -1173,6 +1153,170 @@ __global__ void __launch_bounds__(kPxThreads, 1)
   }
 }
 
+// One CTA per query: the whole selection of a query whose eligible count is small enough
+// for one CTA to scan (the queries of a prefill). The histogram gives the threshold bin;
+// pass 1 reads the scores in 1536-entry tiles (one float4 per thread), counts the entries
+// above the bin and collects the in-bin candidates in shared memory; the radix select of
+// the decode path fixes the exact cut; pass 2 reads the tiles again in index order and
+// writes the selected indices at offsets from a block scan, so the output is ascending.
+// It leaves the query's histogram zeroed.
+constexpr int kQsTile = kSelThreads * 4;
+
+__global__ void __launch_bounds__(kSelThreads) topk_query_kernel(IxParams p) {
+  __shared__ __align__(16) uint8_t raw[sizeof(SelScratch)];
+  SelScratch& x = *reinterpret_cast<SelScratch*>(raw);
+  pdl_wait();
+  pdl_trigger();
+  const int b = blockIdx.x, tid = threadIdx.x;
+  const int n = clamp_n(p.n_entries[b], p.Nmax, p.dev_status);
+  const int k_eff = n < p.k ? n : p.k;
+  const float* sc = p.ws.scores + (size_t)b * p.Nmax;
+  uint32_t* gh = p.ws.hist(b);
+  if (tid == 0) { x.tbin = -1; x.above = 0; x.pop = 0; }
+  if (n > p.k) {
+    for (int i = tid; i < kHist; i += kSelThreads) x.h[i] = __ldcg(gh + i);
+    __syncthreads();
+    constexpr int per = (kHist + kSelThreads - 1) / kSelThreads;
+    uint32_t mine = 0;
+    for (int i = 0; i < per; ++i) {
+      const int r = tid * per + i;
+      if (r < kHist) mine += x.h[kHist - 1 - r];
+    }
+    const uint32_t incl = block_incl_scan(mine, x.tmp, nullptr);
+    if (incl >= (uint32_t)p.k && incl - mine < (uint32_t)p.k) {
+      uint32_t cum = incl - mine;
+      for (int i = 0; i < per; ++i) {
+        const int r = tid * per + i;
+        if (r >= kHist) break;
+        const int bin = kHist - 1 - r;
+        if (cum + x.h[bin] >= (uint32_t)p.k) { x.tbin = bin; break; }
+        cum += x.h[bin];
+      }
+    }
+  }
+  __syncthreads();
+  const int tbin = x.tbin;
+  uint32_t cut_key = 0u;
+  int32_t cut_idx = 0x7FFFFFFF;  // tbin < 0: every eligible entry is selected
+  if (tbin >= 0) {
+    // pass 1: count above the bin, collect the bin's candidates (x.pop counts them; past
+    // the shared capacity they go to the global candidate list)
+    uint64_t* gcand = p.ws.cand + (size_t)b * p.Nmax;
+    uint32_t above = 0;
+    for (int j0 = 0; j0 < n; j0 += kQsTile) {
+      const int j = j0 + 4 * tid;
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+      if (j + 4 <= n) {
+        const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + j));
+        v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+      } else {
+        for (int e = 0; e < 4; ++e) v[e] = j + e < n ? __ldcg(sc + j + e) : 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        if (j + e >= n) continue;
+        const uint32_t key = float_key(v[e]);
+        const int bin = (int)(key >> kLowBits);
+        above += bin > tbin ? 1u : 0u;
+        if (bin == tbin) {
+          const uint32_t slot = atomicAdd(&x.pop, 1u);
+          const uint64_t c = ((uint64_t)key << 32) | (uint32_t)(j + e);
+          if (slot < kCandStage) x.cand[slot] = c;
+          if (slot < (uint32_t)p.Nmax) gcand[slot] = c;  // complete list for overflow
+        }
+      }
+    }
+    for (int o = 16; o > 0; o >>= 1) above += __shfl_xor_sync(0xffffffffu, above, o);
+    if ((tid & 31) == 0 && above) atomicAdd(&x.above, above);
+    __syncthreads();
+    const uint32_t above_total = x.above;
+    uint32_t n_cand = x.pop;
+    if (n_cand > (uint32_t)p.Nmax) n_cand = (uint32_t)p.Nmax;
+    const bool staged = n_cand <= kCandStage;
+    const uint64_t* cand = staged ? x.cand : gcand;
+    if (!staged) __threadfence_block();
+    const uint32_t need = (uint32_t)k_eff > above_total ? (uint32_t)k_eff - above_total : 0u;
+    if (need == 0) {
+      cut_key = ((uint32_t)(tbin + 1) << kLowBits) - 1u;
+      cut_idx = -1;
+    } else if (need >= n_cand) {
+      if (need > n_cand) report(p.dev_status, CSA_ERR_DEVICE);
+      cut_key = (uint32_t)tbin << kLowBits;
+      cut_idx = 0x7FFFFFFF;
+    } else {
+      __syncthreads();
+      if (tid == 0) { x.prefix = (uint32_t)tbin << kLowBits; x.rem = need; }
+      __syncthreads();
+      radix_step(cand, staged, n_cand, true, 0, false, ~0u << kLowBits, kLowBits - 8, 8, true,
+                 &x.prefix, &x.rem, x.h);
+      radix_step(cand, staged, n_cand, true, 0, false, ~0u << (kLowBits - 8), kLowBits - 16, 8,
+                 true, &x.prefix, &x.rem, x.h);
+      radix_step(cand, staged, n_cand, true, 0, false, ~0u << (kLowBits - 16), 0, kLowBits - 16,
+                 true, &x.prefix, &x.rem, x.h, &x.sum);
+      cut_key = x.prefix;
+      if (x.sum == x.rem) {
+        cut_idx = 0x7FFFFFFF;
+      } else {
+        __syncthreads();
+        if (tid == 0) x.prefix = 0;
+        __syncthreads();
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0u, 24, 8, false, &x.prefix,
+                   &x.rem, x.h);
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFF000000u, 16, 8, false,
+                   &x.prefix, &x.rem, x.h);
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFFFF0000u, 8, 8, false,
+                   &x.prefix, &x.rem, x.h);
+        radix_step(cand, staged, n_cand, false, cut_key, true, 0xFFFFFF00u, 0, 8, false,
+                   &x.prefix, &x.rem, x.h);
+        cut_idx = (int32_t)x.prefix;
+      }
+    }
+  }
+  // pass 2: ordered write
+  int32_t* out = p.idx + (size_t)b * p.k;
+  uint32_t base = 0;
+  for (int j0 = 0; j0 < n; j0 += kQsTile) {
+    const int j = j0 + 4 * tid;
+    float v[4] = {0.f, 0.f, 0.f, 0.f};
+    if (j + 4 <= n) {
+      const float4 f = __ldcg(reinterpret_cast<const float4*>(sc + j));
+      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    } else {
+      for (int e = 0; e < 4; ++e) v[e] = j + e < n ? __ldcg(sc + j + e) : 0.f;
+    }
+    uint32_t mask = 0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t key = float_key(v[e]);
+      if (j + e < n && (key > cut_key || (key == cut_key && j + e <= cut_idx))) mask |= 1u << e;
+    }
+    const uint32_t mine = __popc(mask);
+    uint32_t tot;
+    const uint32_t incl = block_incl_scan(mine, x.tmp, &tot);
+    uint32_t slot = base + incl - mine;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      if (mask & (1u << e)) {
+        if (slot < (uint32_t)p.k) {
+          out[slot] = j + e;
+          if (p.scores_out) p.scores_out[(size_t)b * p.k + slot] = v[e];
+        } else {
+          report(p.dev_status, CSA_ERR_DEVICE);
+        }
+        ++slot;
+      }
+    }
+    base += tot;
+    __syncthreads();  // x.tmp is reused by the next tile's scan
+  }
+  if (base != (uint32_t)k_eff && tid == 0) report(p.dev_status, CSA_ERR_DEVICE);
+  for (int i = k_eff + tid; i < p.k; i += kSelThreads) {
+    out[i] = -1;
+    if (p.scores_out) p.scores_out[(size_t)b * p.k + i] = __int_as_float(0x7fc00000);
+  }
+  for (int i = tid; i < kHist; i += kSelThreads) gh[i] = 0;
+}
+
 // ------------------------------------------------------------------- launch
 cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
                                 const CUtensorMap& kmap, cudaStream_t stream) {
@@ -1247,10 +1391,7 @@ cudaError_t launch_prefill_indexer_topk(const csa_topk_args& a, void* workspace,
   cudaError_t e = launch_pdl(prefill_score_kernel, dim3(num_sms), dim3(kPxThreads), smem,
                              stream, kmap, p);
   if (e != cudaSuccess) return e;
-  dim3 g2((unsigned)ws.S, a.B);
-  e = launch_pdl(topk_threshold_kernel, g2, dim3(kSelThreads), 0, stream, p);
-  if (e != cudaSuccess) return e;
-  return launch_pdl(topk_write_kernel, g2, dim3(kSelThreads), 0, stream, p);
+  return launch_pdl(topk_query_kernel, dim3(a.B), dim3(kSelThreads), 0, stream, p);
 }
 
 }  // namespace csa
