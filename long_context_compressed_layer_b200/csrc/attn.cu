@@ -420,27 +420,30 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AtParams p) {
 // A prefill has many queries over one cache, so each query keeps its Q on chip and walks
 // its whole row list: one CTA per (query, half of the 512 output dims). The cache entries
 // and the window rows are dequantised to FP16 once per call (prefill_rows16_kernel), so the
-// per-query gather is a plain copy. Rows come in chunks of 32 through a double buffer:
+// per-query gather is a plain copy. Rows come in chunks of 32 through a triple buffer:
 //   warps 0-3  gather the chunk's rows with 16-byte cp.async copies straight into the
 //              swizzled layout of the decode kernel (no register staging);
 //   warp 4     issues S = Q V^T (M = 128 heads, N = 32, K = 512) into a TMEM buffer, then,
 //              once the chunk's P is ready, O[:, half] += P V[:, half] (N = 256, K = 32);
 //   warps 5-8  one thread per head: online softmax in the base-2 domain with a lazy
 //              rescale (O and the running sum are rescaled in TMEM only when the running
-//              maximum grows by more than 2^8), P written as FP16.
+//              maximum grows by more than 2^8); P is written as FP16 into the chunk's own
+//              S columns in TMEM, and the P V product reads its A operand from there, so
+//              shared memory holds only Q and the three row buffers.
 // At the end the softmax threads divide by the running sum plus the sink term, de-rotate
 // the RoPE dims and store BF16 (and lse). S is computed by both CTAs of a query (each
 // needs all 512 dims of the products); O is split so that it fits TMEM next to S.
 constexpr int kPaRows = 32;
+constexpr int kPaBufs = 3;
 constexpr int kPaThreads = 32 * 9;
 constexpr float kLog2e = 1.4426950408889634f;
 
 struct PaSmem {
   uint8_t q[8][128 * 128];             // Q FP16: 8 K-blocks [128 heads x 64 dims], 128-B swizzle
-  uint8_t v[2][8][kPaRows * 128];      // rows FP16: 8 dim-blocks [32 rows x 64 dims]
-  uint8_t pm[2][128 * 64];             // P FP16 [128 heads x 32 rows], 64-B swizzle
-  int kind[2][kPaRows];
-  uint64_t q_full, v_full[2], v_free[2], s_full[2], p_full[2], o_done[2], done;
+  uint8_t v[kPaBufs][8][kPaRows * 128];  // rows FP16: 8 dim-blocks [32 rows x 64 dims]
+  int kind[kPaBufs][kPaRows];
+  uint64_t q_full, v_full[kPaBufs], v_free[kPaBufs], s_full[kPaBufs], p_full[kPaBufs],
+      o_done[kPaBufs], done;
   uint32_t tmem_base;
   volatile int abort;
 };
@@ -484,7 +487,7 @@ __global__ void __launch_bounds__(kPaThreads, 1)
   const int nchunks = (rows_total + kPaRows - 1) / kPaRows;
   if (tid == 0) {
     mbar_init(&s.q_full, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kPaBufs; ++i) {
       mbar_init(&s.v_full[i], 128);
       mbar_init(&s.v_free[i], 1);
       mbar_init(&s.s_full[i], 1);
@@ -524,8 +527,8 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     const int64_t self_row = p.Nmax + (t - p.swa_base);  // always present: stands in for
                                                          // rows that carry no weight
     for (int c = 0; c < nchunks; ++c) {
-      const int buf = c & 1;
-      if (s.abort || !mbar_wait(&s.v_free[buf], ((c >> 1) & 1) ^ 1, p.dev_status)) {
+      const int buf = c % kPaBufs;
+      if (s.abort || !mbar_wait(&s.v_free[buf], ((c / kPaBufs) & 1) ^ 1, p.dev_status)) {
         s.abort = 1;
         break;
       }
@@ -568,22 +571,22 @@ __global__ void __launch_bounds__(kPaThreads, 1)
       const uint32_t id_s = idesc_f16(128, kPaRows, false);
       const uint32_t id_o = idesc_f16(128, 256, true);
       auto issue_pv = [&](int c) -> bool {
-        const int cb = c & 1;
-        if (s.abort || !mbar_wait(&s.p_full[cb], (c >> 1) & 1, p.dev_status)) return false;
+        const int cb = c % kPaBufs;
+        if (s.abort || !mbar_wait(&s.p_full[cb], (c / kPaBufs) & 1, p.dev_status)) return false;
         tc_fence_after();
-        for (int kk = 0; kk < 2; ++kk)
-          mma_f16(t_o, smem_desc(smem_u32(s.pm[cb]) + kk * 32, 16, 512, kSwizzle64B),
-                  smem_desc(smem_u32(s.v[cb][hf * 4]) + kk * 2048, kPaRows * 128, 1024,
-                            kSwizzle128B),
-                  id_o, (c > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < 2; ++kk)  // A = P: 16 rows (8 columns) per step
+          mma_f16_ts(t_o, t_s0 + kPaRows * cb + kk * 8,
+                     smem_desc(smem_u32(s.v[cb][hf * 4]) + kk * 2048, kPaRows * 128, 1024,
+                               kSwizzle128B),
+                     id_o, (c > 0 || kk > 0) ? 1u : 0u);
         mma_commit(&s.v_free[cb]);
         mma_commit(&s.o_done[cb]);
         return true;
       };
       bool ok = true;
       for (int c = 0; c < nchunks && ok; ++c) {
-        const int buf = c & 1;
-        if (s.abort || !mbar_wait(&s.v_full[buf], (c >> 1) & 1, p.dev_status)) {
+        const int buf = c % kPaBufs;
+        if (s.abort || !mbar_wait(&s.v_full[buf], (c / kPaBufs) & 1, p.dev_status)) {
           ok = false;
           break;
         }
@@ -611,21 +614,20 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     const float scale2 = p.tau * kLog2e;
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    // P V of chunk c completes phase c >> 1 of o_done[c & 1]; the next phase of that
-    // barrier needs this warp's P of chunk c + 2, so a wait never trails by two phases
+    // P V of chunk c completes phase c / kPaBufs of o_done[c % kPaBufs]; the next phase of
+    // that barrier needs this warp's P of chunk c + kPaBufs, so a wait never trails by two
     auto wait_pv = [&](int c) -> bool {
       bool w = true;
-      if (lane == 0) w = mbar_wait(&s.o_done[c & 1], (c >> 1) & 1, p.dev_status);
+      if (lane == 0) w = mbar_wait(&s.o_done[c % kPaBufs], (c / kPaBufs) & 1, p.dev_status);
       return __shfl_sync(0xffffffffu, w, 0) != 0;
     };
     for (int c = 0; c < nchunks; ++c) {
-      const int buf = c & 1, ph = (c >> 1) & 1;
+      const int buf = c % kPaBufs, ph = (c / kPaBufs) & 1;
       bool w = true;
       if (lane == 0)
         w = !s.abort && mbar_wait(&s.s_full[buf], ph, p.dev_status) &&
             mbar_wait(&s.v_full[buf], ph, p.dev_status);
       w = __shfl_sync(0xffffffffu, w, 0) != 0;
-      if (w && c >= 2) w = wait_pv(c - 2);  // P[buf] was last read by P V of chunk c-2
       if (!w) {
         s.abort = 1;
         ok = false;
@@ -667,25 +669,23 @@ __global__ void __launch_bounds__(kPaThreads, 1)
           tmem_st_wait();
         }
       }
-      uint8_t* prow = s.pm[buf] + h * 64;
+      // P (FP16) over the chunk's S columns: S was read into registers above, and the
+      // previous P in these columns belonged to chunk c - kPaBufs, whose P V completed
+      // before S of this chunk was issued
+      uint32_t pw[kPaRows / 2];
       float lsum = 0.f;
 #pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        uint32_t wv[4];
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const int e = ch * 8 + 2 * e2;
-          const float p0 = (m_run == -INFINITY || lg[e] == -INFINITY) ? 0.f : exp2f(lg[e] - m_run);
-          const float p1 =
-              (m_run == -INFINITY || lg[e + 1] == -INFINITY) ? 0.f : exp2f(lg[e + 1] - m_run);
-          lsum += p0 + p1;
-          wv[e2] = pack_half2(p0, p1);
-        }
-        *reinterpret_cast<uint4*>(prow + ((ch ^ ((h >> 1) & 3)) << 4)) =
-            make_uint4(wv[0], wv[1], wv[2], wv[3]);
+      for (int e2 = 0; e2 < kPaRows / 2; ++e2) {
+        const int e = 2 * e2;
+        const float p0 = (m_run == -INFINITY || lg[e] == -INFINITY) ? 0.f : exp2f(lg[e] - m_run);
+        const float p1 =
+            (m_run == -INFINITY || lg[e + 1] == -INFINITY) ? 0.f : exp2f(lg[e + 1] - m_run);
+        lsum += p0 + p1;
+        pw[e2] = pack_half2(p0, p1);
       }
+      tmem_st16(t_s0 + kPaRows * buf + lane_off, pw);
+      tmem_st_wait();
       l_run += lsum;
-      fence_async_smem();
       tc_fence_before();
       mbar_arrive(&s.p_full[buf]);
     }
