@@ -407,8 +407,10 @@ __device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
 #pragma unroll
         for (int k8 = 0; k8 < 8; ++k8) part[k8] = 0.f;
 #pragma unroll
-        for (int h = 0; h < kIxN; ++h)
-          part[h & 7] = fmaf(w[h], fmaxf(__uint_as_float(r[h >> 5][h & 31]), 0.f), part[h & 7]);
+        for (int h = 0; h < kIxN; h += 2)  // heads h, h+1 -> partial sums h & 7, (h+1) & 7
+          fma2(part[h & 7], part[(h + 1) & 7], w[h], w[h + 1],
+               fmaxf(__uint_as_float(r[h >> 5][h & 31]), 0.f),
+               fmaxf(__uint_as_float(r[(h + 1) >> 5][(h + 1) & 31]), 0.f));
         const float sc = ((part[0] + part[1]) + (part[2] + part[3])) +
                          ((part[4] + part[5]) + (part[6] + part[7]));
         const int j = (g - prefix[b]) * kIxTile + row;
@@ -1122,13 +1124,12 @@ __global__ void __launch_bounds__(kPxThreads, 1)
         for (int h4 = 0; h4 < kIxN / 4; ++h4) {
           const float4 wv = w4[h4];
           const int h = 4 * h4;
-          part[h & 7] = fmaf(wv.x, fmaxf(__uint_as_float(r[h >> 5][h & 31]), 0.f), part[h & 7]);
-          part[(h + 1) & 7] =
-              fmaf(wv.y, fmaxf(__uint_as_float(r[(h + 1) >> 5][(h + 1) & 31]), 0.f), part[(h + 1) & 7]);
-          part[(h + 2) & 7] =
-              fmaf(wv.z, fmaxf(__uint_as_float(r[(h + 2) >> 5][(h + 2) & 31]), 0.f), part[(h + 2) & 7]);
-          part[(h + 3) & 7] =
-              fmaf(wv.w, fmaxf(__uint_as_float(r[(h + 3) >> 5][(h + 3) & 31]), 0.f), part[(h + 3) & 7]);
+          fma2(part[h & 7], part[(h + 1) & 7], wv.x, wv.y,
+               fmaxf(__uint_as_float(r[h >> 5][h & 31]), 0.f),
+               fmaxf(__uint_as_float(r[(h + 1) >> 5][(h + 1) & 31]), 0.f));
+          fma2(part[(h + 2) & 7], part[(h + 3) & 7], wv.z, wv.w,
+               fmaxf(__uint_as_float(r[(h + 2) >> 5][(h + 2) & 31]), 0.f),
+               fmaxf(__uint_as_float(r[(h + 3) >> 5][(h + 3) & 31]), 0.f));
         }
         const float sc = ((part[0] + part[1]) + (part[2] + part[3])) +
                          ((part[4] + part[5]) + (part[6] + part[7]));
