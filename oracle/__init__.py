@@ -67,6 +67,8 @@ def lib():
             L.or_indexer_scores.argtypes = [i, i, i64, i32, u8, u8, f32, u8, u8, f64, i]
             L.or_topk.restype = i
             L.or_topk.argtypes = [i64, i, f64, i32]
+            L.or_topk_bf16.restype = i
+            L.or_topk_bf16.argtypes = [i64, i, f64, i32]
             L.or_attention.restype = i
             L.or_attention.argtypes = [i, i, i, i64, i, u16, i32, i32, i32, u8, f32, u16,
                                        f32, d, d, i, f64, f64, i]
@@ -175,6 +177,15 @@ def topk(scores: np.ndarray, n: int, k: int) -> np.ndarray:
     s = _c(np.asarray(scores[:n], dtype=np.float64), np.float64)
     idx = np.empty(k, dtype=np.int32)
     if lib().or_topk(n, k, _p(s, C.c_double), _p(idx, C.c_int32)):
+        raise ValueError("oracle topk rejected its arguments")
+    return idx
+
+
+def topk_bf16(scores: np.ndarray, n: int, k: int) -> np.ndarray:
+    """Top-k on the scores rounded to BF16 (ties in the rounded value broken by index)."""
+    s = _c(np.asarray(scores[:n], dtype=np.float64), np.float64)
+    idx = np.empty(k, dtype=np.int32)
+    if lib().or_topk_bf16(n, k, _p(s, C.c_double), _p(idx, C.c_int32)):
         raise ValueError("oracle topk rejected its arguments")
     return idx
 

@@ -317,6 +317,17 @@ int or_topk(int64_t n, int k, const double* scores, int32_t* idx) {
   return 0;
 }
 
+// Top-k on BF16 index scores [walkthrough §3.4: the index scores are quantised from FP32
+// to BF16 before the top-k selector]: every score is rounded to BF16 (nearest even) and
+// the selection of or_topk runs on the rounded values, so entries whose scores round to
+// the same BF16 value are ordered by index.
+int or_topk_bf16(int64_t n, int k, const double* scores, int32_t* idx) {
+  if (n < 0 || k < 1) return -1;
+  std::vector<double> r((size_t)n);
+  for (int64_t j = 0; j < n; ++j) r[(size_t)j] = or_bf16_decode(or_bf16_encode(scores[j]));
+  return or_topk(n, k, r.data(), idx);
+}
+
 // --------------------------------------------------------------- attention
 // Shared-KV MQA for one query token per sequence [tutorial, Hybrid Attention: shared
 // key-value MQA, every head reads the same entry as key and value]; the row set is

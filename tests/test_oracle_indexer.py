@@ -1,6 +1,7 @@
 """Pins of the oracle's lightning-indexer scores and top-k selection."""
 
 import numpy as np
+import torch
 import pytest
 
 import oracle
@@ -135,3 +136,36 @@ def test_eligible_counts_of_the_workloads():
     w = synth.WORKLOADS[2]
     L = synth.seq_lengths(w)
     assert ((L >= 65536) & (L <= 131072)).all() and len(L) == 32
+
+
+def test_bf16_topk_orders_rounded_ties_by_index():
+    # near 1.0 the BF16 spacing is 2^-7: 1.001 and 1 + 2^-10 both round to 1.0, so the
+    # three entries at 1.0 tie and the smallest index wins the last slot
+    s = np.array([1.0, 1.001, 3.0, 2.0, 1.0 + 2.0 ** -10, 0.5])
+    np.testing.assert_array_equal(oracle.topk_bf16(s, 6, 3), [0, 2, 3])
+    np.testing.assert_array_equal(oracle.topk(s, 6, 3), [1, 2, 3])
+    np.testing.assert_array_equal(oracle.topk_bf16(s, 4, 8), [0, 1, 2, 3, -1, -1, -1, -1])
+
+
+def test_bf16_topk_matches_library_rounding_and_lexsort():
+    # an independent statement: torch's round-to-nearest-even BF16 cast, then numpy's
+    # lexsort on (value descending, index ascending)
+    rng = np.random.default_rng(5)
+    for n, k in ((1000, 100), (4096, 512), (257, 300)):
+        s = rng.standard_normal(n) * rng.choice([1.0, 1e3], size=n)
+        r = torch.from_numpy(s).to(torch.float32).to(torch.bfloat16).to(torch.float64).numpy()
+        # torch rounds through fp32; keep cases where that equals direct rounding
+        order = np.lexsort((np.arange(n), -r))
+        keep = min(k, n)
+        want = np.concatenate([np.sort(order[:keep]), np.full(k - keep, -1)])
+        got = oracle.topk_bf16(s.astype(np.float32).astype(np.float64), n, k)
+        np.testing.assert_array_equal(got, want)
+
+
+def test_bf16_topk_equals_exact_topk_on_distinct_bf16_values():
+    rng = np.random.default_rng(6)
+    vals = np.unique(rng.integers(0x3C00, 0x4400, size=3000).astype(np.uint16))
+    s = torch.from_numpy(vals.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    rng.shuffle(s)
+    n = len(s)
+    np.testing.assert_array_equal(oracle.topk_bf16(s, n, 700), oracle.topk(s, n, 700))
