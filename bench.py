@@ -432,6 +432,23 @@ def main():
     nprobe = max(4, min(replays, 256))
     t_idx = time_graphs(idx_graphs, nprobe)
     t_att = time_graphs(att_graphs, nprobe)
+
+    # the selection on BF16-rounded index scores: its call time, and how much of the fp32
+    # selection it keeps (recall) on the first device copy
+    idx_bf = torch.empty_like(idx)
+
+    def step_idx_bf(c):
+        csa.indexer_topk(c["n_entries"], c["q_fp4"], c["q_sf"], c["w"], c["k_fp4"], c["k_sf"],
+                         k, workspace=ws_idx, idx=idx_bf, dev_status=status, bf16_scores=True)
+
+    bf_graphs = [capture(lambda c=c: step_idx_bf(c), GRAPH_STEPS) for c in copies]
+    t_idx_bf = time_graphs(bf_graphs, nprobe)
+    step_idx(copies[0])
+    step_idx_bf(copies[0])
+    torch.cuda.synchronize()
+    a32, a16 = idx.cpu().numpy(), idx_bf.cpu().numpy()
+    recall = float(np.mean([len(np.intersect1d(a32[b][a32[b] >= 0], a16[b][a16[b] >= 0])) /
+                            max(1, int((a32[b] >= 0).sum())) for b in range(B)]))
     clocks = sampler.stop()
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during the benchmark")
@@ -481,6 +498,8 @@ def main():
                        "step_achieved_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
                        "step_frac_of_peak": step_bytes / (ms_step * 1e-3) / 1e9 / pk["hbm_gbs"],
                        "indexer_topk_ms": t_idx, "sparse_attn_ms": t_att,
+                       "bf16_index_scores": {"indexer_topk_ms": t_idx_bf,
+                                             "recall_of_fp32_topk": recall},
                        "launch": f"CUDA graphs of {GRAPH_STEPS} steps, programmatic dependent launch"},
             "roofline": {"bound": "hbm", "kernel": "csa_indexer_topk (score + select)",
                          "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",

@@ -149,6 +149,14 @@ size_t csa_indexer_topk_workspace_size(int32_t B, int64_t Nmax, int32_t k);
 int csa_indexer_topk(const csa_topk_args* args, void* workspace, size_t workspace_bytes,
                      csa_stream_t stream);
 
+/* csa_indexer_topk_bf16: csa_indexer_topk with every score rounded to BF16 (nearest even)
+ * before selection (walkthrough §3.4: the index scores are quantised from FP32 to BF16
+ * for the top-k selector). Scores that round to the same BF16 value are ordered by
+ * index. Same arguments, workspace and errors; `scores`, when given, returns the
+ * rounded values. */
+int csa_indexer_topk_bf16(const csa_topk_args* args, void* workspace, size_t workspace_bytes,
+                          csa_stream_t stream);
+
 /* ------------------------------------------------------------------------------------
  * csa_sparse_attn_decode / hca_attn_decode: one query token per sequence.
  * (tutorial "Hybrid Attention": shared key-value MQA; walkthrough §2.2: the 128 most

@@ -60,7 +60,7 @@ class PrefillArgs(C.Structure):
 
 
 EXPORTS = ["csa_status_string", "csa_compress", "csa_indexer_topk_workspace_size",
-           "csa_indexer_topk", "csa_attn_workspace_size", "csa_sparse_attn_decode",
+           "csa_indexer_topk", "csa_indexer_topk_bf16", "csa_attn_workspace_size", "csa_sparse_attn_decode",
            "hca_attn_decode", "csa_sparse_attn_decode_noalloc", "csa_prefill_workspace_size",
            "csa_prefill"]
 
@@ -83,8 +83,9 @@ def lib() -> C.CDLL:
         L.csa_compress.argtypes = [C.POINTER(CompressArgs), _vp]
         L.csa_indexer_topk_workspace_size.restype = C.c_size_t
         L.csa_indexer_topk_workspace_size.argtypes = [C.c_int32, C.c_int64, C.c_int32]
-        L.csa_indexer_topk.restype = C.c_int
-        L.csa_indexer_topk.argtypes = [C.POINTER(TopkArgs), _vp, C.c_size_t, _vp]
+        for f in ("csa_indexer_topk", "csa_indexer_topk_bf16"):
+            getattr(L, f).restype = C.c_int
+            getattr(L, f).argtypes = [C.POINTER(TopkArgs), _vp, C.c_size_t, _vp]
         L.csa_attn_workspace_size.restype = C.c_size_t
         L.csa_attn_workspace_size.argtypes = [C.c_int32, C.c_int32, C.c_int32]
         for f in ("csa_sparse_attn_decode", "hca_attn_decode"):
@@ -164,8 +165,9 @@ def indexer_topk_workspace(B: int, Nmax: int, k: int, device="cuda") -> torch.Te
 
 
 def indexer_topk(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, k: int, *, workspace=None, idx=None,
-                 scores: bool = False, dev_status=None, stream=None):
-    """Top-k entry indices [B][k] (ascending, -1 padded) and optionally their scores."""
+                 scores: bool = False, bf16_scores: bool = False, dev_status=None, stream=None):
+    """Top-k entry indices [B][k] (ascending, -1 padded) and optionally their scores.
+    bf16_scores selects on scores rounded to BF16 (csa_indexer_topk_bf16)."""
     B, H_I, _ = q_fp4.shape
     Nmax = k_fp4.shape[1]
     dev = q_fp4.device
@@ -179,8 +181,9 @@ def indexer_topk(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, k: int, *, workspace=No
                     _ptr(w, elem=4, name="w"), _ptr(k_fp4, elem=1, name="k_fp4"),
                     _ptr(k_sf, elem=1, name="k_sf"), _ptr(idx, elem=4, name="idx"),
                     _ptr(sc, elem=4, name="scores"), _ptr(dev_status, elem=4, name="dev_status"))
-    _check(lib().csa_indexer_topk(C.byref(args), workspace.data_ptr(), workspace.numel(),
-                                  _stream(stream)), "csa_indexer_topk")
+    fn = "csa_indexer_topk_bf16" if bf16_scores else "csa_indexer_topk"
+    _check(getattr(lib(), fn)(C.byref(args), workspace.data_ptr(), workspace.numel(),
+                              _stream(stream)), fn)
     return (idx, sc) if scores else idx
 
 

@@ -9,7 +9,7 @@
 namespace csa {
 cudaError_t launch_compress(const csa_compress_args& a, cudaStream_t stream);
 cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
-                                const CUtensorMap& kmap, cudaStream_t stream);
+                                const CUtensorMap& kmap, cudaStream_t stream, int bf16);
 size_t ix_workspace_size(int B, int64_t Nmax, int k);
 cudaError_t launch_prefill_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
                                         const CUtensorMap& kmap, cudaStream_t stream);
@@ -177,7 +177,8 @@ size_t csa_indexer_topk_workspace_size(int32_t B, int64_t Nmax, int32_t k) {
   return ix_workspace_size(B, Nmax, k);
 }
 
-int csa_indexer_topk(const csa_topk_args* a, void* ws, size_t ws_bytes, csa_stream_t stream) {
+static int indexer_common(const csa_topk_args* a, void* ws, size_t ws_bytes,
+                          csa_stream_t stream, int bf16) {
   if (!a) return CSA_ERR_INVALID_ARG;
   if (a->B < 0 || a->k < 1 || a->Nmax < 0 || a->Nmax % 128 != 0) return CSA_ERR_INVALID_ARG;
   if (a->H_I != 16 && a->H_I != 32 && a->H_I != 64) return CSA_ERR_UNSUPPORTED;
@@ -209,7 +210,16 @@ int csa_indexer_topk(const csa_topk_args* a, void* ws, size_t ws_bytes, csa_stre
       return CSA_ERR_CUDA;
   }
   return cuda_status(
-      launch_indexer_topk(*a, ws, sms, kmap, reinterpret_cast<cudaStream_t>(stream)));
+      launch_indexer_topk(*a, ws, sms, kmap, reinterpret_cast<cudaStream_t>(stream), bf16));
+}
+
+int csa_indexer_topk(const csa_topk_args* a, void* ws, size_t ws_bytes, csa_stream_t stream) {
+  return indexer_common(a, ws, ws_bytes, stream, 0);
+}
+
+int csa_indexer_topk_bf16(const csa_topk_args* a, void* ws, size_t ws_bytes,
+                          csa_stream_t stream) {
+  return indexer_common(a, ws, ws_bytes, stream, 1);
 }
 
 size_t csa_attn_workspace_size(int32_t B, int32_t H, int32_t rows_max) {

@@ -134,6 +134,7 @@ size_t ix_workspace_size(int B, int64_t Nmax, int k) {
 struct IxParams {
   int B, H_I, k;
   int fused;  // 1: the selection follows in this (cooperative) launch
+  int bf16;   // 1: scores are rounded to BF16 before they are stored and selected
   int64_t Nmax;
   const int32_t* n_entries;
   const uint8_t* q_fp4;
@@ -411,8 +412,9 @@ __device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
           fma2(part[h & 7], part[(h + 1) & 7], w[h], w[h + 1],
                fmaxf(__uint_as_float(r[h >> 5][h & 31]), 0.f),
                fmaxf(__uint_as_float(r[(h + 1) >> 5][(h + 1) & 31]), 0.f));
-        const float sc = ((part[0] + part[1]) + (part[2] + part[3])) +
-                         ((part[4] + part[5]) + (part[6] + part[7]));
+        float sc = ((part[0] + part[1]) + (part[2] + part[3])) +
+                   ((part[4] + part[5]) + (part[6] + part[7]));
+        if (p.bf16) sc = bf16_bits_to_f32(f32_to_bf16_bits(sc));
         const int j = (g - prefix[b]) * kIxTile + row;
         if (j < n_b) {
           p.ws.scores[(size_t)b * p.Nmax + j] = sc;
@@ -1320,10 +1322,10 @@ __global__ void __launch_bounds__(kSelThreads) topk_query_kernel(IxParams p) {
 
 // ------------------------------------------------------------------- launch
 cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
-                                const CUtensorMap& kmap, cudaStream_t stream) {
+                                const CUtensorMap& kmap, cudaStream_t stream, int bf16) {
   IxWs ws;
   ix_ws_layout(a.B, a.Nmax, a.k, (char*)workspace, &ws);
-  IxParams p{a.B, a.H_I, a.k, 1, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
+  IxParams p{a.B, a.H_I, a.k, 1, bf16, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
              a.idx, a.scores, a.dev_status};
   const size_t smem = sizeof(IxSmem) + 1024;
   static int configured = -1;
@@ -1377,7 +1379,7 @@ cudaError_t launch_prefill_indexer_topk(const csa_topk_args& a, void* workspace,
                                         const CUtensorMap& kmap, cudaStream_t stream) {
   IxWs ws;
   ix_ws_layout(a.B, a.Nmax, a.k, (char*)workspace, &ws);
-  IxParams p{a.B, a.H_I, a.k, 0, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
+  IxParams p{a.B, a.H_I, a.k, 0, 0, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
              a.idx, a.scores, a.dev_status};
   const size_t smem = sizeof(PxSmem) + 1024;
   static int configured = -1;

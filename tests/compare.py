@@ -86,3 +86,33 @@ def compare_topk(idx_gpu, scores_ora, n, k, what=""):
     extra = np.setdiff1d(g, want)
     assert (s[extra] >= sk * (1 - 10 * TIE_REL)).all(), f"{what}: a chosen entry is far below the k-th"
     return int(len(extra))
+
+
+def _bf16_round(x):
+    import torch
+    return torch.from_numpy(np.asarray(x, dtype=np.float64)).to(torch.bfloat16).to(
+        torch.float64).numpy()
+
+
+def compare_topk_bf16(idx_gpu, scores_ora, n, k, what=""):
+    """One sequence of the BF16-score selection -> number of tolerated mismatches.
+    The GPU rounds its fp32 score to BF16, the oracle its fp64 score, so an entry whose
+    score sits next to a BF16 rounding midpoint may land one BF16 step apart; the sets may
+    differ only in entries within one BF16 step of the boundary value."""
+    import oracle
+    want = oracle.topk_bf16(np.asarray(scores_ora[:n], dtype=np.float64), n, k)
+    got = np.asarray(idx_gpu)
+    keep = min(k, n)
+    assert (got[keep:] == -1).all(), f"{what}: padding"
+    g = got[:keep]
+    assert (np.diff(g) > 0).all(), f"{what}: not strictly ascending"
+    if np.array_equal(g, want[:keep]):
+        return 0
+    assert n > k, what
+    r = _bf16_round(scores_ora[:n])
+    rk = np.sort(r)[::-1][k - 1]
+    step = np.abs(rk) * 2.0 ** -7
+    diff = np.setxor1d(g, want[:keep])
+    assert (np.abs(r[diff] - rk) <= step).all(), \
+        f"{what}: a differing entry is more than one BF16 step from the boundary"
+    return int(len(diff))

@@ -103,6 +103,32 @@ def test_indexer_topk_matches_oracle(B, H_I, Nmax, n, k, planted):
     assert total <= 2
 
 
+@pytest.mark.parametrize("B,H_I,Nmax,n,k,planted", [
+    (1, 16, 2048, [2048], 512, 0),
+    (3, 64, 4096, [4096, 2999, 130], 512, 0),
+    (2, 64, 16384, [16384, 12345], 1024, 8),
+])
+def test_indexer_topk_bf16_scores_match_oracle(B, H_I, Nmax, n, k, planted):
+    rng = np.random.default_rng(B * 11 + k)
+    n = np.asarray(n, dtype=np.int32)
+    ix = synth.indexer_inputs(rng, B, H_I, Nmax, n, planted)
+    idx, sc = csa.indexer_topk(dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]),
+                               dev(ix["k_fp4"]), dev(ix["k_sf"]), k, scores=True,
+                               bf16_scores=True)
+    torch.cuda.synchronize()
+    idx, sc = host(idx), host(sc)
+    ora = oracle.indexer_scores(n, ix["q_fp4"], ix["q_sf"], ix["w"], ix["k_fp4"], ix["k_sf"])
+    total = 0
+    for b in range(B):
+        total += compare.compare_topk_bf16(idx[b], ora[b], int(n[b]), k, what=f"seq {b}")
+        sel = idx[b][idx[b] >= 0]
+        want = compare._bf16_round(ora[b][sel])
+        # each returned score is a BF16 value within one BF16 step of the oracle's
+        assert (compare._bf16_round(sc[b][: len(sel)]) == sc[b][: len(sel)]).all()
+        np.testing.assert_allclose(sc[b][: len(sel)], want, rtol=2.0 ** -7, atol=1e-6)
+    assert total <= 2 * B
+
+
 def test_indexer_scores_exact_on_integer_case():
     # unit scales, w = 1: every score is a multiple of 1/4 below 2^24, exact in fp32
     B, H_I, Nmax, k = 1, 64, 1024, 1024
