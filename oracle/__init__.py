@@ -67,6 +67,13 @@ def lib():
             L.or_indexer_scores.argtypes = [i, i, i64, i32, u8, u8, f32, u8, u8, f64, i]
             L.or_topk.restype = i
             L.or_topk.argtypes = [i64, i, f64, i32]
+            L.or_e2m1_encode.restype = C.c_uint8
+            L.or_e2m1_encode.argtypes = [d]
+            L.or_mxfp4_block.restype = None
+            L.or_mxfp4_block.argtypes = [f64, u8, u8]
+            L.or_compress_index_keys.restype = i
+            L.or_compress_index_keys.argtypes = [i, i, i, i, i64, u16, u16, f32, f32, f32, u16,
+                                                 f32, i64, u8, u8, f64]
             L.or_topk_bf16.restype = i
             L.or_topk_bf16.argtypes = [i64, i, f64, i32]
             L.or_attention.restype = i
@@ -179,6 +186,42 @@ def topk(scores: np.ndarray, n: int, k: int) -> np.ndarray:
     if lib().or_topk(n, k, _p(s, C.c_double), _p(idx, C.c_int32)):
         raise ValueError("oracle topk rejected its arguments")
     return idx
+
+
+def e2m1_encode(x):
+    return np.vectorize(lambda v: lib().or_e2m1_encode(float(v)), otypes=[np.uint8])(x)
+
+
+def mxfp4_block(v) -> tuple[np.ndarray, int]:
+    """32 values -> (32 E2M1 codes, E8M0 scale code)."""
+    v = _c(np.asarray(v, dtype=np.float64), np.float64)
+    nib = np.empty(32, dtype=np.uint8)
+    sf = np.zeros(1, dtype=np.uint8)
+    lib().or_mxfp4_block(_p(v, C.c_double), _p(nib, C.c_uint8), _p(sf, C.c_uint8))
+    return nib, int(sf[0])
+
+
+def compress_index_keys(a, za, bias, m: int, overlap: bool, Nmax: int, b=None, zb=None,
+                        pos0: int = 0, prev_b=None, prev_zb=None):
+    """[B][T][128] indexer-key streams -> (k_fp4 [B][Nmax][64], k_sf [B][Nmax/128*512],
+    y [B][N][128]); rows pos0/m .. pos0/m + N - 1 are written, the rest stay zero."""
+    B, T, _ = a.shape
+    N = T // m
+    k_fp4 = np.zeros((B, Nmax, 64), dtype=np.uint8)
+    k_sf = np.zeros((B, Nmax // 128 * 512), dtype=np.uint8)
+    y = np.empty((B, N, 128))
+    g = {x: _c(v, t) for x, v, t in (("a", a, np.uint16), ("b", b, np.uint16),
+                                      ("za", za, np.float32), ("zb", zb, np.float32),
+                                      ("bias", bias, np.float32), ("pb", prev_b, np.uint16),
+                                      ("pz", prev_zb, np.float32))}
+    rc = lib().or_compress_index_keys(
+        B, T, m, int(overlap), pos0, _p(g["a"], C.c_uint16), _p(g["b"], C.c_uint16),
+        _p(g["za"], C.c_float), _p(g["zb"], C.c_float), _p(g["bias"], C.c_float),
+        _p(g["pb"], C.c_uint16), _p(g["pz"], C.c_float), Nmax, _p(k_fp4, C.c_uint8),
+        _p(k_sf, C.c_uint8), _p(y, C.c_double))
+    if rc:
+        raise ValueError("oracle key compression rejected its arguments")
+    return k_fp4, k_sf, y
 
 
 def topk_bf16(scores: np.ndarray, n: int, k: int) -> np.ndarray:

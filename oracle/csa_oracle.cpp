@@ -128,6 +128,40 @@ double or_e8m0_decode(uint8_t e) {
   return std::ldexp(1.0, (int)e - 127);
 }
 
+// OCP MX FP4 E2M1 code of x: the nearest of {0, .5, 1, 1.5, 2, 3, 4, 6} with the sign of
+// x, ties to the code with an even mantissa bit, magnitudes above 6 saturating to 6.
+uint8_t or_e2m1_encode(double x) {
+  const uint8_t sign = std::signbit(x) ? 8 : 0;
+  const double a = std::fabs(x);
+  uint8_t c;
+  if (a <= 0.25) c = 0;        // 0.25 ties to 0 (even)
+  else if (a < 0.75) c = 1;    // 0.75 ties to 1.0
+  else if (a <= 1.25) c = 2;   // 1.25 ties to 1.0
+  else if (a < 1.75) c = 3;    // 1.75 ties to 2.0
+  else if (a <= 2.5) c = 4;    // 2.5 ties to 2.0
+  else if (a < 3.5) c = 5;     // 3.5 ties to 4.0
+  else if (a <= 5.0) c = 6;    // 5.0 ties to 4.0
+  else c = 7;
+  return sign | c;
+}
+
+// MXFP4 quantisation of one 32-element block [OCP MX spec, the MX conversion rule]:
+// shared exponent e = floor(log2(max |v|)) - 2 (2 is the largest E2M1 exponent), stored
+// as the E8M0 code e + 127 (clamped to 0..254); elements are E2M1(v / 2^e). A block of
+// zeros gets code 0.
+void or_mxfp4_block(const double* v, uint8_t* nib, uint8_t* sf) {
+  double amax = 0.0;
+  for (int i = 0; i < 32; ++i) amax = std::max(amax, std::fabs(v[i]));
+  int e = -127;
+  if (amax > 0.0) {
+    int ex;
+    std::frexp(amax, &ex);  // amax = f * 2^ex with f in [0.5, 1): floor(log2 amax) = ex - 1
+    e = std::min(127, std::max(-127, ex - 1 - 2));
+  }
+  *sf = (uint8_t)(e + 127);
+  for (int i = 0; i < 32; ++i) nib[i] = or_e2m1_encode(std::ldexp(v[i], -e));
+}
+
 // Byte offset of the E8M0 scale of entry j, 32-element block s, in the indexer-key
 // scale array. Keys are grouped 128 to a 512-byte group; inside a group entry
 // j = r0 + 32*r1 (r0 < 32, r1 < 4) keeps its four block scales at 16*r0 + 4*r1 + s.
@@ -230,6 +264,75 @@ int or_compress(int B, int T, int m, int overlap, int64_t pos0, double rope_base
           std::memcpy(row + kNope + 2 * (d - kNope), &h, 2);
         }
       }
+    }
+  }
+  return 0;
+}
+
+// Indexer-key compression (R21-R23) [walkthrough §2.2: the lightning indexer scores the
+// compressed entries, so each entry needs an indexer key; §3.4: the indexer QK path is
+// FP4]: the 128-dim indexer-key stream of the T tokens at pos0 .. pos0+T-1 is merged with
+// the gated softmax of or_compress (same candidate slots and bias layout, R1-R3), with no
+// norm and no RoPE (R22), and each entry is stored as MXFP4 (R23): 64 bytes of E2M1
+// codes (element 2i in the low nibble of byte i) at row pos0/m + i of k_fp4 [B][Nmax][64]
+// and four E8M0 block scales at or_key_sf_offset(row, s) of k_sf [B][Nmax/128][512].
+// y_out [B][N][128] (nullable) is the merged entry before quantisation.
+int or_compress_index_keys(int B, int T, int m, int overlap, int64_t pos0,
+                           const uint16_t* a, const uint16_t* b, const float* za,
+                           const float* zb, const float* bias, const uint16_t* prev_b,
+                           const float* prev_zb, int64_t Nmax, uint8_t* k_fp4, uint8_t* k_sf,
+                           double* y_out) {
+  if (B < 0 || T < 0 || m < 1 || pos0 < 0 || pos0 % m != 0 || Nmax % 128 != 0) return -1;
+  if (!a || !za || !bias) return -1;
+  if (overlap && (!b || !zb)) return -1;
+  if (overlap && pos0 > 0 && (!prev_b || !prev_zb)) return -1;
+  const int N = T / m;
+  if (pos0 / m + N > Nmax) return -1;
+  std::vector<double> xs, zs, y(kDI);
+  std::vector<uint8_t> nib(kDI);
+  for (int bb = 0; bb < B; ++bb) {
+    for (int i = 0; i < N; ++i) {
+      for (int d = 0; d < kDI; ++d) {
+        xs.clear();
+        zs.clear();
+        for (int r = 0; r < m; ++r) {  // own block, slots 0..m-1
+          const size_t o = ((size_t)bb * T + (int64_t)m * i + r) * kDI + d;
+          xs.push_back(or_bf16_decode(a[o]));
+          zs.push_back((double)za[o] + (double)bias[r]);
+        }
+        if (overlap) {  // previous block, slots m..2m-1
+          for (int r = 0; r < m; ++r) {
+            if (i > 0) {
+              const size_t o = ((size_t)bb * T + (int64_t)m * (i - 1) + r) * kDI + d;
+              xs.push_back(or_bf16_decode(b[o]));
+              zs.push_back((double)zb[o] + (double)bias[m + r]);
+            } else if (pos0 > 0) {
+              const size_t o = ((size_t)bb * m + r) * kDI + d;
+              xs.push_back(or_bf16_decode(prev_b[o]));
+              zs.push_back((double)prev_zb[o] + (double)bias[m + r]);
+            }
+          }
+        }
+        double zmax = -kInf;
+        for (double z : zs) zmax = std::max(zmax, z);
+        double den = 0.0, num = 0.0;
+        for (size_t c = 0; c < zs.size(); ++c) {
+          const double g = std::exp(zs[c] - zmax);
+          den += g;
+          num += g * xs[c];
+        }
+        y[d] = num / den;
+      }
+      if (y_out) std::memcpy(y_out + ((size_t)bb * N + i) * kDI, y.data(), kDI * sizeof(double));
+      const int64_t row = pos0 / m + i;
+      uint8_t* krow = k_fp4 + ((size_t)bb * Nmax + row) * (kDI / 2);
+      uint8_t* sfb = k_sf + (size_t)bb * (Nmax / 128) * 512;
+      for (int s = 0; s < kDI / 32; ++s) {
+        uint8_t code;
+        or_mxfp4_block(y.data() + 32 * s, nib.data() + 32 * s, &code);
+        sfb[or_key_sf_offset(row, s)] = code;
+      }
+      for (int j = 0; j < kDI / 2; ++j) krow[j] = (uint8_t)(nib[2 * j] | (nib[2 * j + 1] << 4));
     }
   }
   return 0;

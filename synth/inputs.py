@@ -127,22 +127,23 @@ def e8m0_codes(rng: np.random.Generator, shape, lo: int = 124, hi: int = 130) ->
 
 # ------------------------------------------------------------- input bundles
 def compress_inputs(B: int, T: int, m: int, overlap: bool, seed: int,
-                    pos0: int = 0) -> dict:
-    """Token streams for one compression call: a, b bf16 [B][T][512], gate logits za, zb
-    float32 [B][T][512] ~ N(0,1), bias [2m] (CSA) or [m] (HCA) ~ N(0, 0.1), and when
-    pos0 > 0 the previous block's tail prev_b / prev_zb [B][m][512]."""
+                    pos0: int = 0, dim: int = D) -> dict:
+    """Token streams for one compression call: a, b bf16 [B][T][dim], gate logits za, zb
+    float32 [B][T][dim] ~ N(0,1), bias [2m] (CSA) or [m] (HCA) ~ N(0, 0.1), and when
+    pos0 > 0 the previous block's tail prev_b / prev_zb [B][m][dim]. dim is 512 for the
+    KV stream and 128 for the indexer-key stream."""
     rng = np.random.default_rng(seed)
     out = {
-        "a": bf16_normal(rng, (B, T, D)),
-        "za": rng.standard_normal((B, T, D), dtype=np.float32),
+        "a": bf16_normal(rng, (B, T, dim)),
+        "za": rng.standard_normal((B, T, dim), dtype=np.float32),
         "bias": (rng.standard_normal(2 * m if overlap else m) * 0.1).astype(np.float32),
     }
     if overlap:
-        out["b"] = bf16_normal(rng, (B, T, D))
-        out["zb"] = rng.standard_normal((B, T, D), dtype=np.float32)
+        out["b"] = bf16_normal(rng, (B, T, dim))
+        out["zb"] = rng.standard_normal((B, T, dim), dtype=np.float32)
         if pos0 > 0:
-            out["prev_b"] = bf16_normal(rng, (B, m, D))
-            out["prev_zb"] = rng.standard_normal((B, m, D), dtype=np.float32)
+            out["prev_b"] = bf16_normal(rng, (B, m, dim))
+            out["prev_zb"] = rng.standard_normal((B, m, dim), dtype=np.float32)
     return out
 
 
