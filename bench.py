@@ -117,13 +117,13 @@ class ClockSampler:
 
 def ncu_traffic() -> dict | None:
     """DRAM bytes per launch of the indexer call from the committed ncu summary, if it was
-    taken on the current kernel sources."""
+    taken on the current sources of that kernel."""
     p = os.path.join(ROOT, "profiles", "indexer_topk_csa_decode_pro_1m.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     from long_context_compressed_layer_b200 import build as b
-    if d.get("sources_sha") != b.sources_sha():
+    if d.get("sources_sha") != b.sources_sha(d.get("sources")):
         return None
     return d
 
@@ -200,6 +200,31 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during the benchmark")
 
+    # the indexer keys of the new blocks (csa_compress_index_keys over the 65,536 new
+    # tokens -> 16,384 MXFP4 keys): an HBM stream of 6,144 bytes read and 68 written per key
+    ik_fp4 = torch.zeros((1, d["Nmax"], 64), dtype=torch.uint8, device="cuda")
+    ik_sf = torch.zeros((1, d["Nmax"] // 128 * 512), dtype=torch.uint8, device="cuda")
+
+    def ikeys():
+        csa.compress_index_keys(d["ia"][None], d["iza"][None], d["ibias"], w.m, True,
+                                b=d["ib"][None], zb=d["izb"][None], pos0=w.P,
+                                prev_b=d["iprev_b"][None], prev_zb=d["iprev_zb"][None],
+                                k_fp4=ik_fp4, k_sf=ik_sf)
+
+    for _ in range(3):
+        ikeys()
+    k0, k1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    k0.record(stream)
+    for _ in range(20):
+        ikeys()
+    k1.record(stream)
+    torch.cuda.synchronize()
+    ik_ms = k0.elapsed_time(k1) / 20
+    n_keys = T // w.m
+    ik_bytes = n_keys * (2 * w.m * 128 * 6 + 68)
+    hbm = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"] if os.path.exists(
+        os.path.join(ROOT, "MEASURED_PEAKS.json")) else 6650.0
+
     # end to end: the new tokens' inputs go up from pinned host memory and the output
     # comes back, around the same call
     up = ("a", "b", "za", "zb", "q", "q_fp4", "q_sf", "w")
@@ -234,7 +259,11 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
         "config": {"workload": w.name, "prefix_tokens": w.P, "new_tokens": T, "heads": w.H,
                    "indexer_heads": w.H_I, "top_k": k, "window": 128,
                    "l2": "inputs larger than L2 (8.6 GB of queries)",
-                   "fp4_tflop": f4 / 1e12, "bf16_tflop": f16 / 1e12},
+                   "fp4_tflop": f4 / 1e12, "bf16_tflop": f16 / 1e12,
+                   "index_key_compress": {"ms": ik_ms, "keys": n_keys,
+                                          "algorithmic_bytes": ik_bytes,
+                                          "gbs": ik_bytes / (ik_ms * 1e-3) / 1e9,
+                                          "frac_of_hbm": ik_bytes / (ik_ms * 1e-3) / 1e9 / hbm}},
         "roofline": {"bound": "tensor", "kernel": "csa_prefill (whole call)",
                      "achieved": eq_tflops, "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": eq_tflops / bf16_peak,

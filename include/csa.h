@@ -108,6 +108,40 @@ typedef struct {
 int csa_compress(const csa_compress_args* args, csa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * csa_compress_index_keys: the indexer keys of the compressed entries.
+ * (walkthrough §2.2: the lightning indexer scores the compressed entries; §3.4: its QK
+ * path is FP4.) The pages do not spell out how the indexer keys are built; this call
+ * applies the gated merge of csa_compress (same candidate slots, bias layout and
+ * previous-block handling) to a 128-dim indexer-key stream, with no norm and no RoPE,
+ * and stores each entry as MXFP4 exactly as csa_indexer_topk reads it:
+ *   per 32-element block s: e = floor(log2(max |y|)) - 2 (E8M0 code e + 127, clamped
+ *   to 0..254; an all-zero block gets code 0), codes = E2M1(y / 2^e) rounded to nearest
+ *   (ties to the even code) and saturated at +-6; element 2i in the low nibble of byte i
+ *   of k_fp4 row pos0/m + i, the scale at the grouped k_sf position of that row.
+ * Computed in fp32. Nmax must be a multiple of 128.
+ */
+typedef struct {
+  int32_t B;
+  int32_t T;
+  int32_t m;
+  int32_t overlap;
+  int64_t pos0;
+  const uint16_t* a;      /* bf16 [B][T][128] */
+  const uint16_t* b;      /* bf16 [B][T][128]; NULL when overlap == 0 */
+  const float* za;        /* [B][T][128] */
+  const float* zb;        /* [B][T][128]; NULL when overlap == 0 */
+  const float* bias;      /* [2m] (overlap) or [m] */
+  const uint16_t* prev_b; /* bf16 [B][m][128] (overlap, pos0 > 0) */
+  const float* prev_zb;   /* [B][m][128] */
+  uint8_t* k_fp4;         /* out [B][Nmax][64] */
+  uint8_t* k_sf;          /* out [B][Nmax/128][512] */
+  int64_t Nmax;           /* multiple of 128; pos0/m + N <= Nmax */
+  float* dbg;             /* optional out [B][N][128]: y before quantisation */
+} csa_ikey_args;
+
+int csa_compress_index_keys(const csa_ikey_args* args, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * csa_indexer_topk: lightning-indexer scores of every eligible entry and the top-k set.
  * (walkthrough §2.2: the indexer scores compressed entries, each query keeps the top-k,
  * one set shared by all heads; §3.4 and chooseai §二: the indexer QK path is MXFP4.)

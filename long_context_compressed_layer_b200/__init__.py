@@ -33,6 +33,13 @@ class CompressArgs(C.Structure):
                 ("kv_scale", _vp), ("Nmax", C.c_int64), ("dbg", _vp)]
 
 
+class IkeyArgs(C.Structure):
+    _fields_ = [("B", C.c_int32), ("T", C.c_int32), ("m", C.c_int32), ("overlap", C.c_int32),
+                ("pos0", C.c_int64), ("a", _vp), ("b", _vp), ("za", _vp), ("zb", _vp),
+                ("bias", _vp), ("prev_b", _vp), ("prev_zb", _vp), ("k_fp4", _vp),
+                ("k_sf", _vp), ("Nmax", C.c_int64), ("dbg", _vp)]
+
+
 class TopkArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("H_I", C.c_int32), ("k", C.c_int32), ("Nmax", C.c_int64),
                 ("n_entries", _vp), ("q_fp4", _vp), ("q_sf", _vp), ("w", _vp),
@@ -59,7 +66,8 @@ class PrefillArgs(C.Structure):
                 ("lse", _vp), ("idx", _vp), ("dev_status", _vp)]
 
 
-EXPORTS = ["csa_status_string", "csa_compress", "csa_indexer_topk_workspace_size",
+EXPORTS = ["csa_status_string", "csa_compress", "csa_compress_index_keys",
+           "csa_indexer_topk_workspace_size",
            "csa_indexer_topk", "csa_indexer_topk_bf16", "csa_attn_workspace_size", "csa_sparse_attn_decode",
            "hca_attn_decode", "csa_sparse_attn_decode_noalloc", "csa_prefill_workspace_size",
            "csa_prefill"]
@@ -81,6 +89,8 @@ def lib() -> C.CDLL:
         L.csa_status_string.argtypes = [C.c_int]
         L.csa_compress.restype = C.c_int
         L.csa_compress.argtypes = [C.POINTER(CompressArgs), _vp]
+        L.csa_compress_index_keys.restype = C.c_int
+        L.csa_compress_index_keys.argtypes = [C.POINTER(IkeyArgs), _vp]
         L.csa_indexer_topk_workspace_size.restype = C.c_size_t
         L.csa_indexer_topk_workspace_size.argtypes = [C.c_int32, C.c_int64, C.c_int32]
         for f in ("csa_indexer_topk", "csa_indexer_topk_bf16"):
@@ -155,6 +165,33 @@ def compress(a, za, bias, m: int, overlap: bool, *, b=None, zb=None, pos0: int =
                         Nmax, _ptr(d, elem=4, name="dbg"))
     _check(lib().csa_compress(C.byref(args), _stream(stream)), "csa_compress")
     return kv, kv_scale, d
+
+
+def compress_index_keys(a, za, bias, m: int, overlap: bool, *, b=None, zb=None, pos0: int = 0,
+                        prev_b=None, prev_zb=None, k_fp4=None, k_sf=None,
+                        Nmax: int | None = None, dbg: bool = False, stream=None):
+    """Compress a [B][T][128] indexer-key stream into MXFP4 keys at rows pos0/m ...
+    Returns (k_fp4 [B][Nmax][64], k_sf [B][Nmax/128*512], dbg [B][N][128] or None);
+    k_fp4 / k_sf are written in place when given."""
+    B, T, _ = a.shape
+    N = T // m
+    if Nmax is None:
+        Nmax = k_fp4.shape[1] if k_fp4 is not None else -(-(pos0 // m + N) // 128) * 128
+    dev = a.device
+    if k_fp4 is None:
+        k_fp4 = torch.zeros((B, Nmax, 64), dtype=torch.uint8, device=dev)
+    if k_sf is None:
+        k_sf = torch.zeros((B, Nmax // 128 * 512), dtype=torch.uint8, device=dev)
+    d = torch.empty((B, N, INDEX_DIM), dtype=torch.float32, device=dev) if dbg else None
+    args = IkeyArgs(B, T, m, int(overlap), pos0, _ptr(a, elem=2, name="a"),
+                    _ptr(b, elem=2, name="b"), _ptr(za, elem=4, name="za"),
+                    _ptr(zb, elem=4, name="zb"), _ptr(bias, elem=4, name="bias"),
+                    _ptr(prev_b, elem=2, name="prev_b"), _ptr(prev_zb, elem=4, name="prev_zb"),
+                    _ptr(k_fp4, elem=1, name="k_fp4"), _ptr(k_sf, elem=1, name="k_sf"), Nmax,
+                    _ptr(d, elem=4, name="dbg"))
+    _check(lib().csa_compress_index_keys(C.byref(args), _stream(stream)),
+           "csa_compress_index_keys")
+    return k_fp4, k_sf, d
 
 
 # ------------------------------------------------------------- indexer top-k

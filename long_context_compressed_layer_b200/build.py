@@ -24,13 +24,16 @@ def sources() -> list[str]:
     return sorted(glob.glob(os.path.join(HERE, "csrc", "*.cu")))
 
 
-def sources_sha() -> str:
-    """Hash of the kernel sources and the ABI header (ties profiles to the code they used)."""
+def sources_sha(files: list[str] | None = None) -> str:
+    """Hash of kernel sources (ties a profile to the code it measured): the given files
+    under csrc/, or every source plus the ABI header."""
     import hashlib
 
     h = hashlib.sha256()
-    for f in sorted(glob.glob(os.path.join(HERE, "csrc", "*"))) + [
-            os.path.join(HERE, "..", "include", "csa.h")]:
+    paths = ([os.path.join(HERE, "csrc", f) for f in files] if files else
+             sorted(glob.glob(os.path.join(HERE, "csrc", "*"))) +
+             [os.path.join(HERE, "..", "include", "csa.h")])
+    for f in paths:
         h.update(open(f, "rb").read())
     return h.hexdigest()[:16]
 

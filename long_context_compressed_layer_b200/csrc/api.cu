@@ -8,6 +8,7 @@
 
 namespace csa {
 cudaError_t launch_compress(const csa_compress_args& a, cudaStream_t stream);
+cudaError_t launch_ikey_compress(const csa_ikey_args& a, cudaStream_t stream);
 cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
                                 const CUtensorMap& kmap, cudaStream_t stream, int bf16);
 size_t ix_workspace_size(int B, int64_t Nmax, int k);
@@ -170,6 +171,25 @@ int csa_compress(const csa_compress_args* a, csa_stream_t stream) {
     if (a->pos0 > 0 && (!ok_ptr(a->prev_b) || !ok_ptr(a->prev_zb))) return CSA_ERR_INVALID_ARG;
   }
   return cuda_status(launch_compress(*a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csa_compress_index_keys(const csa_ikey_args* a, csa_stream_t stream) {
+  if (!a) return CSA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->T < 0 || a->m < 1 || a->m > 128 || a->pos0 < 0 || a->pos0 % a->m ||
+      a->Nmax < 0 || a->Nmax % 128 || (a->overlap != 0 && a->overlap != 1))
+    return CSA_ERR_INVALID_ARG;
+  if (a->B > 65535) return CSA_ERR_UNSUPPORTED;
+  const int N = a->T / a->m;
+  if (a->pos0 / a->m + N > a->Nmax) return CSA_ERR_INVALID_ARG;
+  if (a->B == 0 || N == 0) return CSA_OK;
+  if (!ok_ptr(a->a) || !ok_ptr(a->za) || !ok_ptr(a->bias) || !ok_ptr(a->k_fp4) ||
+      !ok_ptr(a->k_sf) || !ok_opt(a->dbg))
+    return CSA_ERR_INVALID_ARG;
+  if (a->overlap) {
+    if (!ok_ptr(a->b) || !ok_ptr(a->zb)) return CSA_ERR_INVALID_ARG;
+    if (a->pos0 > 0 && (!ok_ptr(a->prev_b) || !ok_ptr(a->prev_zb))) return CSA_ERR_INVALID_ARG;
+  }
+  return cuda_status(launch_ikey_compress(*a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t csa_indexer_topk_workspace_size(int32_t B, int64_t Nmax, int32_t k) {

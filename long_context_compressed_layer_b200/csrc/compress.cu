@@ -151,6 +151,94 @@ __global__ void __launch_bounds__(128) compress_kernel(csa_compress_args a, int 
   if (tid == 0) a.kv_scale[row] = scale;
 }
 
+// Indexer-key compression: the same gated merge on the 128-dim indexer-key stream (no norm,
+// no RoPE), stored as MXFP4 for the FP4 indexer (walkthrough §3.4). One CTA of 128
+// threads per entry, thread d owning dim d, so each warp holds one 32-element block:
+// the block maximum is a warp reduction, the shared exponent floor(log2 amax) - 2 comes
+// from frexpf, scaling by a power of two is exact, and each element is rounded to the
+// nearest E2M1 value (ties to the even code, saturating at 6). Lanes pair their nibbles
+// with a shuffle (element 2i in the low nibble).
+__device__ __forceinline__ uint32_t e2m1_code(float x) {
+  const uint32_t sign = __float_as_uint(x) >> 31 ? 8u : 0u;
+  const float a = fabsf(x);
+  uint32_t c;
+  if (a <= 0.25f) c = 0;
+  else if (a < 0.75f) c = 1;
+  else if (a <= 1.25f) c = 2;
+  else if (a < 1.75f) c = 3;
+  else if (a <= 2.5f) c = 4;
+  else if (a < 3.5f) c = 5;
+  else if (a <= 5.0f) c = 6;
+  else c = 7;
+  return sign | c;
+}
+
+__global__ void __launch_bounds__(128) ikey_compress_kernel(csa_ikey_args a, int N) {
+  const int i = blockIdx.x, b = blockIdx.y, d = threadIdx.x, lane = d & 31, s = d >> 5;
+  constexpr int kDI = CSA_INDEX_DIM;
+  const int m = a.m;
+  pdl_wait();
+  pdl_trigger();
+  const size_t tok0 = (size_t)b * a.T + (size_t)m * i;
+  float mx = -INFINITY, den = 0.f, num = 0.f;
+  auto add = [&](uint16_t xb, float z) {
+    const float x = bf16_bits_to_f32(xb);
+    if (z > mx) {
+      const float r = expf(mx - z);  // 0 on the first candidate
+      den = den * r + 1.f;
+      num = num * r + x;
+      mx = z;
+    } else {
+      const float g = expf(z - mx);
+      den += g;
+      num += g * x;
+    }
+  };
+  for (int r = 0; r < m; ++r) {
+    const size_t o = (tok0 + r) * kDI + d;
+    add(a.a[o], a.za[o] + __ldg(a.bias + r));
+  }
+  if (a.overlap) {
+    const uint16_t* pb = nullptr;
+    const float* pz = nullptr;
+    if (i > 0) {
+      pb = a.b + (tok0 - m) * kDI;
+      pz = a.zb + (tok0 - m) * kDI;
+    } else if (a.pos0 > 0) {
+      pb = a.prev_b + (size_t)b * m * kDI;
+      pz = a.prev_zb + (size_t)b * m * kDI;
+    }
+    if (pb)
+      for (int r = 0; r < m; ++r) add(pb[(size_t)r * kDI + d], pz[(size_t)r * kDI + d] + __ldg(a.bias + m + r));
+  }
+  const float y = __fdiv_rn(num, den);
+  if (a.dbg) a.dbg[((size_t)b * N + i) * kDI + d] = y;
+  float amax = fabsf(y);
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  int e = -127;
+  if (amax > 0.f) {
+    int ex;
+    frexpf(amax, &ex);  // amax = f * 2^ex, f in [0.5, 1): floor(log2 amax) = ex - 1
+    e = min(127, max(-127, ex - 3));
+  }
+  const uint32_t nib = e2m1_code(ldexpf(y, -e));
+  const uint32_t hi = __shfl_down_sync(0xffffffffu, nib, 1);
+  const int64_t row = a.pos0 / m + i;
+  if ((lane & 1) == 0)
+    a.k_fp4[((size_t)b * a.Nmax + row) * (kDI / 2) + 16 * s + (lane >> 1)] = (uint8_t)(nib | (hi << 4));
+  if (lane == 0) {
+    const int64_t g = row / 128, r = row % 128;
+    a.k_sf[(size_t)b * (a.Nmax / 128) * 512 + g * 512 + 16 * (r % 32) + 4 * (r / 32) + s] =
+        (uint8_t)(e + 127);
+  }
+}
+
+cudaError_t launch_ikey_compress(const csa_ikey_args& a, cudaStream_t stream) {
+  const int N = a.T / a.m;
+  if (N == 0 || a.B == 0) return cudaSuccess;
+  return launch_pdl(ikey_compress_kernel, dim3(N, a.B), dim3(128), 0, stream, a, N);
+}
+
 cudaError_t launch_compress(const csa_compress_args& a, cudaStream_t stream) {
   const int N = a.T / a.m;
   if (N == 0 || a.B == 0) return cudaSuccess;

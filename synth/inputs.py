@@ -326,7 +326,14 @@ def prefill_inputs_device(P: int, T: int, m: int, H: int, H_I: int, seed: int,
         "zb": torch.randn((T, D), generator=g, device=device),
         "bias": torch.randn(2 * m, generator=g, device=device) * 0.1,
     }
+    # the indexer-key stream of the new tokens (128 dims), for the key compressor
+    out["ia"], out["ib"] = bf16n((T, D_I)), bf16n((T, D_I))
+    out["iza"] = torch.randn((T, D_I), generator=g, device=device)
+    out["izb"] = torch.randn((T, D_I), generator=g, device=device)
+    out["ibias"] = torch.randn(2 * m, generator=g, device=device) * 0.1
     if P > 0:
         out["prev_b"] = bf16n((m, D))
         out["prev_zb"] = torch.randn((m, D), generator=g, device=device)
+        out["iprev_b"] = bf16n((m, D_I))
+        out["iprev_zb"] = torch.randn((m, D_I), generator=g, device=device)
     return out

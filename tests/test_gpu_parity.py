@@ -74,6 +74,54 @@ def test_compress_workload0_full():
     assert flips <= kv.size // 5000
 
 
+# ------------------------------------------------------- indexer-key compression
+_E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+
+
+@pytest.mark.parametrize("B,T,m,pos0", [
+    (2, 4 * 37 + 3, 4, 0),      # ragged tail, first entry without a previous block
+    (1, 4 * 64, 4, 4096),       # previous block from the caller's tail
+    (1, 8192, 4, 0),            # the 8K stream of the tiny decode workload -> 2048 keys
+])
+def test_index_key_compression_matches_oracle(B, T, m, pos0):
+    inp = synth.compress_inputs(B, T, m, True, seed=300 + T, pos0=pos0, dim=128)
+    N = T // m
+    Nmax = -(-(pos0 // m + N) // 128) * 128
+    kf, ks, dbg = csa.compress_index_keys(
+        dev(inp["a"]), dev(inp["za"]), dev(inp["bias"]), m, True, b=dev(inp["b"]),
+        zb=dev(inp["zb"]), pos0=pos0, prev_b=dev(inp["prev_b"]) if pos0 else None,
+        prev_zb=dev(inp["prev_zb"]) if pos0 else None, Nmax=Nmax, dbg=True)
+    torch.cuda.synchronize()
+    kf, ks, dbg = host(kf), host(ks), host(dbg)
+    okf, oks, oy = oracle.compress_index_keys(
+        inp["a"], inp["za"], inp["bias"], m, True, Nmax, b=inp["b"], zb=inp["zb"], pos0=pos0,
+        prev_b=inp.get("prev_b"), prev_zb=inp.get("prev_zb"))
+    np.testing.assert_allclose(dbg, oy, rtol=1e-5, atol=1e-5)
+    flips = 0
+    n0 = pos0 // m
+    for bb in range(B):
+        for i in range(N):
+            row = n0 + i
+            g = np.stack([kf[bb, row] & 15, kf[bb, row] >> 4], axis=1).reshape(128)
+            o = np.stack([okf[bb, row] & 15, okf[bb, row] >> 4], axis=1).reshape(128)
+            for sblk in range(4):
+                off = oracle.key_sf_offset(row, sblk)
+                y = oy[bb, i, 32 * sblk:32 * sblk + 32]
+                amax = np.abs(y).max()
+                if ks[bb, off] != oks[bb, off]:  # only at a power-of-two block maximum
+                    assert amax > 0 and abs(np.log2(amax) - np.round(np.log2(amax))) < 1e-6
+                    flips += 1
+                    continue
+                d = g[32 * sblk:32 * sblk + 32] != o[32 * sblk:32 * sblk + 32]
+                if d.any():
+                    X = 2.0 ** (int(oks[bb, off]) - 127)
+                    r = np.abs(y[d]) / X
+                    near = np.min(np.abs(r[:, None] - _E2M1_MIDS[None, :]), axis=1) <= 1e-5 * r
+                    assert near.all(), f"entry {row} block {sblk}: code differs off a midpoint"
+                    flips += int(d.sum())
+    assert flips <= max(2, N * B // 500)
+
+
 # ------------------------------------------------------------- indexer top-k
 def _topk_case(B, H_I, Nmax, n, k, planted=0, seed=0):
     rng = np.random.default_rng(seed)
