@@ -74,6 +74,8 @@ def lib():
             L.or_compress_index_keys.restype = i
             L.or_compress_index_keys.argtypes = [i, i, i, i, i64, u16, u16, f32, f32, f32, u16,
                                                  f32, i64, u8, u8, f64]
+            L.or_indexer_query.restype = i
+            L.or_indexer_query.argtypes = [i, i, i, u16, u16, u8, u8, f64]
             L.or_topk_bf16.restype = i
             L.or_topk_bf16.argtypes = [i64, i, f64, i32]
             L.or_attention.restype = i
@@ -222,6 +224,20 @@ def compress_index_keys(a, za, bias, m: int, overlap: bool, Nmax: int, b=None, z
     if rc:
         raise ValueError("oracle key compression rejected its arguments")
     return k_fp4, k_sf, y
+
+
+def indexer_query(c, W, H_I: int):
+    """c bf16 [T][r], W bf16 [H_I * 128][r] -> (q_fp4 [T][H_I][64], q_sf [T][H_I][4],
+    y [T][H_I * 128])."""
+    T, r = c.shape
+    q_fp4 = np.empty((T, H_I, 64), dtype=np.uint8)
+    q_sf = np.empty((T, H_I, 4), dtype=np.uint8)
+    y = np.empty((T, H_I * 128))
+    cc, ww = _c(c, np.uint16), _c(W, np.uint16)
+    if lib().or_indexer_query(T, r, H_I, _p(cc, C.c_uint16), _p(ww, C.c_uint16),
+                              _p(q_fp4, C.c_uint8), _p(q_sf, C.c_uint8), _p(y, C.c_double)):
+        raise ValueError("oracle indexer query rejected its arguments")
+    return q_fp4, q_sf, y
 
 
 def topk_bf16(scores: np.ndarray, n: int, k: int) -> np.ndarray:

@@ -338,6 +338,38 @@ int or_compress_index_keys(int B, int T, int m, int overlap, int64_t pos0,
   return 0;
 }
 
+// Indexer queries (R24) [walkthrough §2.2: the lightning indexer uses a low-rank query,
+// down-projected and then up-projected into its heads, the down projection shared with
+// the main attention; §3.4: its QK path is FP4]: for every token t the H_I x 128 query
+// values are y[t][o] = sum_j W[o][j] * c[t][j] over the r-dim latent c (both BF16), with
+// no norm and no RoPE, stored per head as MXFP4 (R23): q_fp4 [T][H_I][64] (element 2i in
+// the low nibble of byte i), q_sf [T][H_I][4]. y_out [T][H_I * 128] is nullable.
+int or_indexer_query(int T, int r, int H_I, const uint16_t* c, const uint16_t* W,
+                     uint8_t* q_fp4, uint8_t* q_sf, double* y_out) {
+  if (T < 0 || r < 1 || H_I < 1 || !c || !W || !q_fp4 || !q_sf) return -1;
+  const int O = H_I * kDI;
+  std::vector<double> y(O), cw((size_t)r);
+  std::vector<uint8_t> nib(kDI);
+  for (int t = 0; t < T; ++t) {
+    for (int j = 0; j < r; ++j) cw[(size_t)j] = or_bf16_decode(c[(size_t)t * r + j]);
+    for (int o = 0; o < O; ++o) {
+      double acc = 0.0;
+      const uint16_t* w = W + (size_t)o * r;
+      for (int j = 0; j < r; ++j) acc += or_bf16_decode(w[j]) * cw[(size_t)j];
+      y[(size_t)o] = acc;
+    }
+    if (y_out) std::memcpy(y_out + (size_t)t * O, y.data(), O * sizeof(double));
+    for (int h = 0; h < H_I; ++h) {
+      for (int sb = 0; sb < kDI / 32; ++sb)
+        or_mxfp4_block(y.data() + (size_t)h * kDI + 32 * sb, nib.data() + 32 * sb,
+                       q_sf + ((size_t)t * H_I + h) * 4 + sb);
+      uint8_t* row = q_fp4 + ((size_t)t * H_I + h) * (kDI / 2);
+      for (int j = 0; j < kDI / 2; ++j) row[j] = (uint8_t)(nib[2 * j] | (nib[2 * j + 1] << 4));
+    }
+  }
+  return 0;
+}
+
 // Dequantise one stored entry (448 E4M3 codes times the entry scale, then 64 bf16).
 void or_dequant_row(const uint8_t* row, float scale, double* v) {
   for (int d = 0; d < kNope; ++d) v[d] = or_e4m3_decode(row[d]) * (double)scale;

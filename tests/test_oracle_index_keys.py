@@ -102,3 +102,20 @@ def test_stored_keys_are_the_mxfp4_of_the_merge_in_the_indexer_layout():
                              * 2.0 ** (oracle.mxfp4_block(y[0, i, 32 * t:32 * t + 32])[1] - 127)
                              for t in range(4)])
         assert abs(s[128 + i] - max(0.0, dq.sum())) <= 1e-9 * max(1.0, abs(dq).sum())
+
+
+def test_indexer_query_is_the_library_matmul_then_mxfp4_per_head():
+    rng = np.random.default_rng(8)
+    T, r, H_I = 37, 192, 4
+    c = synth.bf16_normal(rng, (T, r))
+    W = synth.bf16_normal(rng, (H_I * 128, r), std=r ** -0.5)
+    q_fp4, q_sf, y = oracle.indexer_query(c, W, H_I)
+    want = indep.bf16_to_f64(c) @ indep.bf16_to_f64(W).T  # numpy's matmul in fp64
+    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-12)
+    for t in (0, 17, 36):
+        for h in range(H_I):
+            codes = np.stack([q_fp4[t, h] & 15, q_fp4[t, h] >> 4], axis=1).reshape(128)
+            for s in range(4):
+                nib, sf = oracle.mxfp4_block(y[t, h * 128 + 32 * s:h * 128 + 32 * s + 32])
+                np.testing.assert_array_equal(codes[32 * s:32 * s + 32], nib)
+                assert q_sf[t, h, s] == sf
