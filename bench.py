@@ -225,6 +225,30 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
     hbm = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))["hbm_gbs"] if os.path.exists(
         os.path.join(ROOT, "MEASURED_PEAKS.json")) else 6650.0
 
+    # the indexer queries of the new tokens (csa_indexer_query: a [65,536 x 1536] x
+    # [1536 x 8192] BF16 product quantised to MXFP4 per head), timed alone
+    g = torch.Generator(device="cuda")
+    g.manual_seed(w.seed + 17)
+    rq = 1536
+    cq = torch.randn((T, rq), generator=g, device="cuda").to(torch.bfloat16)
+    Wq = (torch.randn((w.H_I * 128, rq), generator=g, device="cuda") * rq ** -0.5).to(
+        torch.bfloat16)
+    qf_out = torch.empty((T, w.H_I, 64), dtype=torch.uint8, device="cuda")
+    qs_out = torch.empty((T, w.H_I, 4), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        csa.indexer_query(cq, Wq, w.H_I, q_fp4=qf_out, q_sf=qs_out)
+    k0.record(stream)
+    for _ in range(10):
+        csa.indexer_query(cq, Wq, w.H_I, q_fp4=qf_out, q_sf=qs_out)
+    k1.record(stream)
+    torch.cuda.synchronize()
+    iq_ms = k0.elapsed_time(k1) / 10
+    iq_flop = 2 * T * rq * w.H_I * 128
+    peaks_file = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    pkd = json.load(open(peaks_file)) if os.path.exists(peaks_file) else {}
+    bf16_burst = pkd.get("bf16_tflops", 1590.0)  # a kernel timed alone: the burst figure
+    del cq, Wq
+
     # end to end: the new tokens' inputs go up from pinned host memory and the output
     # comes back, around the same call
     up = ("a", "b", "za", "zb", "q", "q_fp4", "q_sf", "w")
@@ -263,7 +287,11 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
                    "index_key_compress": {"ms": ik_ms, "keys": n_keys,
                                           "algorithmic_bytes": ik_bytes,
                                           "gbs": ik_bytes / (ik_ms * 1e-3) / 1e9,
-                                          "frac_of_hbm": ik_bytes / (ik_ms * 1e-3) / 1e9 / hbm}},
+                                          "frac_of_hbm": ik_bytes / (ik_ms * 1e-3) / 1e9 / hbm},
+                   "index_query": {"ms": iq_ms, "latent_dim": rq, "tflop": iq_flop / 1e12,
+                                   "tflops": iq_flop / (iq_ms * 1e-3) / 1e12,
+                                   "frac_of_bf16_burst": iq_flop / (iq_ms * 1e-3) / 1e12
+                                   / bf16_burst}},
         "roofline": {"bound": "tensor", "kernel": "csa_prefill (whole call)",
                      "achieved": eq_tflops, "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": eq_tflops / bf16_peak,

@@ -142,6 +142,31 @@ typedef struct {
 int csa_compress_index_keys(const csa_ikey_args* args, csa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * csa_indexer_query: the indexer queries of T tokens (walkthrough §2.2: low-rank indexer
+ * queries, down-projected then up-projected into the indexer heads, the down projection
+ * shared with the main attention; §3.4: FP4 QK path).
+ *   y[t][o] = sum_j W[o][j] * c[t][j],  o < H_I * 128,  j < r
+ * with c the query latent and W the up-projection (both BF16; BF16 tensor-core products,
+ * fp32 accumulation), no norm and no RoPE, stored per head as MXFP4 with the rule of
+ * csa_compress_index_keys: q_fp4 [T][H_I][64] (element 2i in the low nibble of byte i),
+ * q_sf [T][H_I][4] -- the query layout of csa_indexer_topk. r is a multiple of 64
+ * (at most 16384), H_I in {16, 32, 64}.
+ */
+typedef struct {
+  int32_t T;              /* tokens */
+  int32_t r;              /* latent dims, multiple of 64 */
+  int32_t H_I;            /* indexer heads: 16, 32 or 64 */
+  const uint16_t* c;      /* bf16 [T][r] */
+  const uint16_t* W;      /* bf16 [H_I * 128][r] */
+  uint8_t* q_fp4;         /* out [T][H_I][64] */
+  uint8_t* q_sf;          /* out [T][H_I][4] */
+  float* dbg;             /* optional out [T][H_I * 128]: y before quantisation */
+  int32_t* dev_status;    /* optional device word */
+} csa_iquery_args;
+
+int csa_indexer_query(const csa_iquery_args* args, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * csa_indexer_topk: lightning-indexer scores of every eligible entry and the top-k set.
  * (walkthrough §2.2: the indexer scores compressed entries, each query keeps the top-k,
  * one set shared by all heads; §3.4 and chooseai §二: the indexer QK path is MXFP4.)

@@ -40,6 +40,11 @@ class IkeyArgs(C.Structure):
                 ("k_sf", _vp), ("Nmax", C.c_int64), ("dbg", _vp)]
 
 
+class IqueryArgs(C.Structure):
+    _fields_ = [("T", C.c_int32), ("r", C.c_int32), ("H_I", C.c_int32), ("c", _vp), ("W", _vp),
+                ("q_fp4", _vp), ("q_sf", _vp), ("dbg", _vp), ("dev_status", _vp)]
+
+
 class TopkArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("H_I", C.c_int32), ("k", C.c_int32), ("Nmax", C.c_int64),
                 ("n_entries", _vp), ("q_fp4", _vp), ("q_sf", _vp), ("w", _vp),
@@ -67,7 +72,7 @@ class PrefillArgs(C.Structure):
 
 
 EXPORTS = ["csa_status_string", "csa_compress", "csa_compress_index_keys",
-           "csa_indexer_topk_workspace_size",
+           "csa_indexer_query", "csa_indexer_topk_workspace_size",
            "csa_indexer_topk", "csa_indexer_topk_bf16", "csa_attn_workspace_size", "csa_sparse_attn_decode",
            "hca_attn_decode", "csa_sparse_attn_decode_noalloc", "csa_prefill_workspace_size",
            "csa_prefill"]
@@ -91,6 +96,8 @@ def lib() -> C.CDLL:
         L.csa_compress.argtypes = [C.POINTER(CompressArgs), _vp]
         L.csa_compress_index_keys.restype = C.c_int
         L.csa_compress_index_keys.argtypes = [C.POINTER(IkeyArgs), _vp]
+        L.csa_indexer_query.restype = C.c_int
+        L.csa_indexer_query.argtypes = [C.POINTER(IqueryArgs), _vp]
         L.csa_indexer_topk_workspace_size.restype = C.c_size_t
         L.csa_indexer_topk_workspace_size.argtypes = [C.c_int32, C.c_int64, C.c_int32]
         for f in ("csa_indexer_topk", "csa_indexer_topk_bf16"):
@@ -192,6 +199,24 @@ def compress_index_keys(a, za, bias, m: int, overlap: bool, *, b=None, zb=None, 
     _check(lib().csa_compress_index_keys(C.byref(args), _stream(stream)),
            "csa_compress_index_keys")
     return k_fp4, k_sf, d
+
+
+def indexer_query(c, W, H_I: int, *, q_fp4=None, q_sf=None, dbg: bool = False,
+                  dev_status=None, stream=None):
+    """Indexer queries of T tokens: c bf16 [T][r], W bf16 [H_I * 128][r] -> (q_fp4
+    [T][H_I][64], q_sf [T][H_I][4], dbg [T][H_I * 128] or None)."""
+    T, r = c.shape
+    dev = c.device
+    if q_fp4 is None:
+        q_fp4 = torch.empty((T, H_I, 64), dtype=torch.uint8, device=dev)
+    if q_sf is None:
+        q_sf = torch.empty((T, H_I, 4), dtype=torch.uint8, device=dev)
+    d = torch.empty((T, H_I * 128), dtype=torch.float32, device=dev) if dbg else None
+    args = IqueryArgs(T, r, H_I, _ptr(c, elem=2, name="c"), _ptr(W, elem=2, name="W"),
+                      _ptr(q_fp4, elem=1, name="q_fp4"), _ptr(q_sf, elem=1, name="q_sf"),
+                      _ptr(d, elem=4, name="dbg"), _ptr(dev_status, elem=4, name="dev_status"))
+    _check(lib().csa_indexer_query(C.byref(args), _stream(stream)), "csa_indexer_query")
+    return q_fp4, q_sf, d
 
 
 # ------------------------------------------------------------- indexer top-k

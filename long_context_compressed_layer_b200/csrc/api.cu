@@ -9,6 +9,8 @@
 namespace csa {
 cudaError_t launch_compress(const csa_compress_args& a, cudaStream_t stream);
 cudaError_t launch_ikey_compress(const csa_ikey_args& a, cudaStream_t stream);
+cudaError_t launch_iquery(const csa_iquery_args& a, const CUtensorMap& cmap,
+                          const CUtensorMap& wmap, cudaStream_t stream);
 cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
                                 const CUtensorMap& kmap, cudaStream_t stream, int bf16);
 size_t ix_workspace_size(int B, int64_t Nmax, int k);
@@ -190,6 +192,32 @@ int csa_compress_index_keys(const csa_ikey_args* a, csa_stream_t stream) {
     if (a->pos0 > 0 && (!ok_ptr(a->prev_b) || !ok_ptr(a->prev_zb))) return CSA_ERR_INVALID_ARG;
   }
   return cuda_status(launch_ikey_compress(*a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csa_indexer_query(const csa_iquery_args* a, csa_stream_t stream) {
+  if (!a) return CSA_ERR_INVALID_ARG;
+  if (a->T < 0 || a->r < 64 || a->r % 64) return CSA_ERR_INVALID_ARG;
+  if (a->r > 16384 || (a->H_I != 16 && a->H_I != 32 && a->H_I != 64)) return CSA_ERR_UNSUPPORTED;
+  if (a->T == 0) return CSA_OK;
+  if (!ok_ptr(a->c) || !ok_ptr(a->W) || !ok_ptr(a->q_fp4) || !ok_ptr(a->q_sf) ||
+      !ok_opt(a->dbg) || (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)))
+    return CSA_ERR_INVALID_ARG;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return CSA_ERR_CUDA;
+  CUtensorMap cmap, wmap;
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const cuuint64_t cdims[2] = {(cuuint64_t)a->r, (cuuint64_t)a->T};
+  const cuuint64_t wdims[2] = {(cuuint64_t)a->r, (cuuint64_t)a->H_I * 128};
+  const cuuint64_t strides[1] = {(cuuint64_t)a->r * 2};
+  if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a->c), cdims,
+          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+      enc(&wmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(a->W), wdims,
+          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return CSA_ERR_CUDA;
+  return cuda_status(launch_iquery(*a, cmap, wmap, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t csa_indexer_topk_workspace_size(int32_t B, int64_t Nmax, int32_t k) {

@@ -399,6 +399,32 @@ __device__ __forceinline__ void fma2(float& acc0, float& acc1, float w0, float w
   asm("mov.b64 {%0, %1}, %2;" : "=f"(acc0), "=f"(acc1) : "l"(a));
 }
 
+// OCP MX FP4 E2M1 code of x: the nearest of {0, .5, 1, 1.5, 2, 3, 4, 6} with the sign of
+// x, ties to the code with an even mantissa bit, magnitudes above 6 saturating to 6.
+__device__ __forceinline__ uint32_t e2m1_code(float x) {
+  const uint32_t sign = __float_as_uint(x) >> 31 ? 8u : 0u;
+  const float a = fabsf(x);
+  uint32_t c;
+  if (a <= 0.25f) c = 0;
+  else if (a < 0.75f) c = 1;
+  else if (a <= 1.25f) c = 2;
+  else if (a < 1.75f) c = 3;
+  else if (a <= 2.5f) c = 4;
+  else if (a < 3.5f) c = 5;
+  else if (a <= 5.0f) c = 6;
+  else c = 7;
+  return sign | c;
+}
+
+// MXFP4 shared exponent of a 32-element block with maximum magnitude amax:
+// floor(log2 amax) - 2 clamped to [-127, 127] (E8M0 code = e + 127); -127 for zero.
+__device__ __forceinline__ int mxfp4_exponent(float amax) {
+  if (!(amax > 0.f)) return -127;
+  int ex;
+  frexpf(amax, &ex);  // amax = f * 2^ex, f in [0.5, 1): floor(log2 amax) = ex - 1
+  return min(127, max(-127, ex - 3));
+}
+
 // Order-preserving map of a float onto uint32 (larger float -> larger key).
 __device__ __forceinline__ uint32_t float_key(float f) {
   const uint32_t u = __float_as_uint(f);

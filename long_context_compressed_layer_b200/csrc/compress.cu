@@ -158,21 +158,6 @@ __global__ void __launch_bounds__(128) compress_kernel(csa_compress_args a, int 
 // from frexpf, scaling by a power of two is exact, and each element is rounded to the
 // nearest E2M1 value (ties to the even code, saturating at 6). Lanes pair their nibbles
 // with a shuffle (element 2i in the low nibble).
-__device__ __forceinline__ uint32_t e2m1_code(float x) {
-  const uint32_t sign = __float_as_uint(x) >> 31 ? 8u : 0u;
-  const float a = fabsf(x);
-  uint32_t c;
-  if (a <= 0.25f) c = 0;
-  else if (a < 0.75f) c = 1;
-  else if (a <= 1.25f) c = 2;
-  else if (a < 1.75f) c = 3;
-  else if (a <= 2.5f) c = 4;
-  else if (a < 3.5f) c = 5;
-  else if (a <= 5.0f) c = 6;
-  else c = 7;
-  return sign | c;
-}
-
 __global__ void __launch_bounds__(128) ikey_compress_kernel(csa_ikey_args a, int N) {
   const int i = blockIdx.x, b = blockIdx.y, d = threadIdx.x, lane = d & 31, s = d >> 5;
   constexpr int kDI = CSA_INDEX_DIM;
@@ -215,12 +200,7 @@ __global__ void __launch_bounds__(128) ikey_compress_kernel(csa_ikey_args a, int
   if (a.dbg) a.dbg[((size_t)b * N + i) * kDI + d] = y;
   float amax = fabsf(y);
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  int e = -127;
-  if (amax > 0.f) {
-    int ex;
-    frexpf(amax, &ex);  // amax = f * 2^ex, f in [0.5, 1): floor(log2 amax) = ex - 1
-    e = min(127, max(-127, ex - 3));
-  }
+  const int e = mxfp4_exponent(amax);
   const uint32_t nib = e2m1_code(ldexpf(y, -e));
   const uint32_t hi = __shfl_down_sync(0xffffffffu, nib, 1);
   const int64_t row = a.pos0 / m + i;

@@ -122,6 +122,44 @@ def test_index_key_compression_matches_oracle(B, T, m, pos0):
     assert flips <= max(2, N * B // 500)
 
 
+@pytest.mark.parametrize("T,r,H_I", [
+    (300, 256, 16),    # three token tiles, the last one ragged
+    (4, 1536, 64),     # one decode step of the 1M workload, latent rank 1536
+    (129, 64, 32),     # a single K block
+])
+def test_indexer_query_matches_oracle(T, r, H_I):
+    rng = np.random.default_rng(T + r)
+    c = synth.bf16_normal(rng, (T, r))
+    W = synth.bf16_normal(rng, (H_I * 128, r), std=r ** -0.5)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    qf, qs, dbg = csa.indexer_query(dev(c), dev(W), H_I, dbg=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    qf, qs, dbg = host(qf), host(qs), host(dbg)
+    of, os_, y = oracle.indexer_query(c, W, H_I)
+    np.testing.assert_allclose(dbg, y, rtol=1e-4, atol=1e-4)
+    flips = 0
+    for t in range(T):
+        for h in range(H_I):
+            g = np.stack([qf[t, h] & 15, qf[t, h] >> 4], axis=1).reshape(128)
+            o = np.stack([of[t, h] & 15, of[t, h] >> 4], axis=1).reshape(128)
+            for sblk in range(4):
+                yb = y[t, h * 128 + 32 * sblk:h * 128 + 32 * sblk + 32]
+                if qs[t, h, sblk] != os_[t, h, sblk]:
+                    amax = np.abs(yb).max()
+                    assert abs(np.log2(amax) - np.round(np.log2(amax))) < 1e-5
+                    flips += 1
+                    continue
+                d = g[32 * sblk:32 * sblk + 32] != o[32 * sblk:32 * sblk + 32]
+                if d.any():
+                    X = 2.0 ** (int(os_[t, h, sblk]) - 127)
+                    rr = np.abs(yb[d]) / X
+                    near = np.min(np.abs(rr[:, None] - _E2M1_MIDS[None, :]), axis=1) <= 1e-4 * rr
+                    assert near.all(), f"token {t} head {h} block {sblk}: code off a midpoint"
+                    flips += int(d.sum())
+    assert flips <= max(4, T * H_I * 128 // 2000)
+
+
 # ------------------------------------------------------------- indexer top-k
 def _topk_case(B, H_I, Nmax, n, k, planted=0, seed=0):
     rng = np.random.default_rng(seed)
