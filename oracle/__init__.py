@@ -76,6 +76,8 @@ def lib():
                                                  f32, i64, u8, u8, f64]
             L.or_indexer_query.restype = i
             L.or_indexer_query.argtypes = [i, i, i, u16, u16, u8, u8, f64]
+            L.or_grouped_out_proj.restype = i
+            L.or_grouped_out_proj.argtypes = [i, i, i, i, i, u16, u16, u16, f64, f64]
             L.or_topk_bf16.restype = i
             L.or_topk_bf16.argtypes = [i64, i, f64, i32]
             L.or_attention.restype = i
@@ -238,6 +240,21 @@ def indexer_query(c, W, H_I: int):
                               _p(q_fp4, C.c_uint8), _p(q_sf, C.c_uint8), _p(y, C.c_double)):
         raise ValueError("oracle indexer query rejected its arguments")
     return q_fp4, q_sf, y
+
+
+def grouped_out_proj(attn, Wg, Wo):
+    """attn bf16 [T][H][512], Wg bf16 [G][d_g][H/G*512], Wo bf16 [d_model][G*d_g] ->
+    (out [T][d_model], mid [T][G*d_g]) in float64."""
+    T, H, _ = attn.shape
+    G, d_g, _ = Wg.shape
+    d_model = Wo.shape[0]
+    out = np.empty((T, d_model))
+    mid = np.empty((T, G * d_g))
+    a, g, o = _c(attn, np.uint16), _c(Wg, np.uint16), _c(Wo, np.uint16)
+    if lib().or_grouped_out_proj(T, H, G, d_g, d_model, _p(a, C.c_uint16), _p(g, C.c_uint16),
+                                 _p(o, C.c_uint16), _p(out, C.c_double), _p(mid, C.c_double)):
+        raise ValueError("oracle output projection rejected its arguments")
+    return out, mid
 
 
 def topk_bf16(scores: np.ndarray, n: int, k: int) -> np.ndarray:

@@ -370,6 +370,40 @@ int or_indexer_query(int T, int r, int H_I, const uint16_t* c, const uint16_t* W
   return 0;
 }
 
+// Grouped output projection (R25) [walkthrough §2.2: with many query heads the output
+// projection first reduces each group of heads, then projects the concatenation; the
+// tutorial's Hybrid Attention section names it as the step after the shared-KV MQA]:
+// the H heads of a token form G groups of H/G consecutive heads; group g's concatenated
+// outputs x_g (H/G * 512 values) give mid_g = Wg[g] x_g (d_g values), rounded to BF16;
+// then out = Wo [mid_0 .. mid_{G-1}] (d_model values). attn bf16 [T][H][512],
+// Wg bf16 [G][d_g][H/G * 512], Wo bf16 [d_model][G * d_g]; out [T][d_model] and
+// mid [T][G * d_g] (after the BF16 rounding, nullable) in double.
+int or_grouped_out_proj(int T, int H, int G, int d_g, int d_model, const uint16_t* attn,
+                        const uint16_t* Wg, const uint16_t* Wo, double* out, double* mid) {
+  if (T < 0 || H < 1 || G < 1 || H % G || d_g < 1 || d_model < 1 || !attn || !Wg || !Wo || !out)
+    return -1;
+  const int K1 = H / G * kD, M = G * d_g;
+  std::vector<double> x((size_t)H * kD), md((size_t)M);
+  for (int t = 0; t < T; ++t) {
+    for (size_t i = 0; i < x.size(); ++i) x[i] = or_bf16_decode(attn[(size_t)t * H * kD + i]);
+    for (int g = 0; g < G; ++g)
+      for (int o = 0; o < d_g; ++o) {
+        const uint16_t* w = Wg + ((size_t)g * d_g + o) * K1;
+        double acc = 0.0;
+        for (int j = 0; j < K1; ++j) acc += or_bf16_decode(w[j]) * x[(size_t)g * K1 + j];
+        md[(size_t)g * d_g + o] = or_bf16_decode(or_bf16_encode(acc));
+      }
+    if (mid) std::memcpy(mid + (size_t)t * M, md.data(), M * sizeof(double));
+    for (int o = 0; o < d_model; ++o) {
+      const uint16_t* w = Wo + (size_t)o * M;
+      double acc = 0.0;
+      for (int j = 0; j < M; ++j) acc += or_bf16_decode(w[j]) * md[(size_t)j];
+      out[(size_t)t * d_model + o] = acc;
+    }
+  }
+  return 0;
+}
+
 // Dequantise one stored entry (448 E4M3 codes times the entry scale, then 64 bf16).
 void or_dequant_row(const uint8_t* row, float scale, double* v) {
   for (int d = 0; d < kNope; ++d) v[d] = or_e4m3_decode(row[d]) * (double)scale;
