@@ -249,6 +249,25 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
     bf16_burst = pkd.get("bf16_tflops", 1590.0)  # a kernel timed alone: the burst figure
     del cq, Wq
 
+    # the grouped output projection of the prefill's attention output (16 groups of 8
+    # heads reduced to 1024 each, then 16,384 -> 7168), timed alone
+    G, d_g, d_model = 16, 1024, 7168
+    K1 = w.H // G * 512
+    Wg = (torch.randn((G, d_g, K1), generator=g, device="cuda") * K1 ** -0.5).to(torch.bfloat16)
+    Wo = (torch.randn((d_model, G * d_g), generator=g, device="cuda") * (G * d_g) ** -0.5).to(
+        torch.bfloat16)
+    op_out = torch.empty((T, d_model), dtype=torch.bfloat16, device="cuda")
+    op_ws = torch.empty(T * G * d_g * 2 + 256, dtype=torch.uint8, device="cuda")
+    csa.grouped_out_proj(out, Wg, Wo, workspace=op_ws, out=op_out)
+    k0.record(stream)
+    for _ in range(3):
+        csa.grouped_out_proj(out, Wg, Wo, workspace=op_ws, out=op_out)
+    k1.record(stream)
+    torch.cuda.synchronize()
+    op_ms = k0.elapsed_time(k1) / 3
+    op_flop = 2 * T * (G * d_g * K1 + d_model * G * d_g)
+    del Wg, Wo, op_out, op_ws
+
     # end to end: the new tokens' inputs go up from pinned host memory and the output
     # comes back, around the same call
     up = ("a", "b", "za", "zb", "q", "q_fp4", "q_sf", "w")
@@ -291,7 +310,12 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
                    "index_query": {"ms": iq_ms, "latent_dim": rq, "tflop": iq_flop / 1e12,
                                    "tflops": iq_flop / (iq_ms * 1e-3) / 1e12,
                                    "frac_of_bf16_burst": iq_flop / (iq_ms * 1e-3) / 1e12
-                                   / bf16_burst}},
+                                   / bf16_burst},
+                   "grouped_out_proj": {"ms": op_ms, "groups": G, "group_rank": d_g,
+                                        "d_model": d_model, "tflop": op_flop / 1e12,
+                                        "tflops": op_flop / (op_ms * 1e-3) / 1e12,
+                                        "frac_of_bf16_burst": op_flop / (op_ms * 1e-3) / 1e12
+                                        / bf16_burst}},
         "roofline": {"bound": "tensor", "kernel": "csa_prefill (whole call)",
                      "achieved": eq_tflops, "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": eq_tflops / bf16_peak,

@@ -329,6 +329,35 @@ int csa_prefill(const csa_prefill_args* args, void* workspace, size_t workspace_
                 csa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * csa_grouped_out_proj: the grouped output projection after the attention (walkthrough
+ * §2.2: the heads are reduced group by group, then the concatenation is projected).
+ * The H heads of a token form G groups of H/G consecutive heads:
+ *   mid[t][g*d_g + o] = BF16( sum_j Wg[g][o][j] * attn[t][g*H/G*512 + j] )
+ *   out[t][o]         = BF16( sum_j Wo[o][j] * mid[t][j] )
+ * BF16 tensor-core products with fp32 accumulation. attn bf16 [T][H][512] (the
+ * attention output), Wg bf16 [G][d_g][H/G * 512], Wo bf16 [d_model][G * d_g],
+ * out bf16 [T][d_model]; the workspace holds mid [T][G * d_g]
+ * (csa_grouped_out_proj_workspace_size). H in {64, 128}, G divides H, d_g and d_model
+ * multiples of 128.
+ */
+typedef struct {
+  int32_t T;
+  int32_t H;
+  int32_t G;
+  int32_t d_g;
+  int32_t d_model;
+  const uint16_t* attn;
+  const uint16_t* Wg;
+  const uint16_t* Wo;
+  uint16_t* out;
+  int32_t* dev_status;   /* optional device word */
+} csa_oproj_args;
+
+size_t csa_grouped_out_proj_workspace_size(int32_t T, int32_t G, int32_t d_g);
+int csa_grouped_out_proj(const csa_oproj_args* args, void* workspace, size_t workspace_bytes,
+                         csa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * csa_sparse_attn_decode_noalloc: csa_sparse_attn_decode without a workspace argument.
  * The pages have no counterpart: this is an interface convenience, not part of the method.
  *

@@ -45,6 +45,12 @@ class IqueryArgs(C.Structure):
                 ("q_fp4", _vp), ("q_sf", _vp), ("dbg", _vp), ("dev_status", _vp)]
 
 
+class OprojArgs(C.Structure):
+    _fields_ = [("T", C.c_int32), ("H", C.c_int32), ("G", C.c_int32), ("d_g", C.c_int32),
+                ("d_model", C.c_int32), ("attn", _vp), ("Wg", _vp), ("Wo", _vp), ("out", _vp),
+                ("dev_status", _vp)]
+
+
 class TopkArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("H_I", C.c_int32), ("k", C.c_int32), ("Nmax", C.c_int64),
                 ("n_entries", _vp), ("q_fp4", _vp), ("q_sf", _vp), ("w", _vp),
@@ -72,7 +78,8 @@ class PrefillArgs(C.Structure):
 
 
 EXPORTS = ["csa_status_string", "csa_compress", "csa_compress_index_keys",
-           "csa_indexer_query", "csa_indexer_topk_workspace_size",
+           "csa_indexer_query", "csa_grouped_out_proj_workspace_size", "csa_grouped_out_proj",
+           "csa_indexer_topk_workspace_size",
            "csa_indexer_topk", "csa_indexer_topk_bf16", "csa_attn_workspace_size", "csa_sparse_attn_decode",
            "hca_attn_decode", "csa_sparse_attn_decode_noalloc", "csa_prefill_workspace_size",
            "csa_prefill"]
@@ -98,6 +105,10 @@ def lib() -> C.CDLL:
         L.csa_compress_index_keys.argtypes = [C.POINTER(IkeyArgs), _vp]
         L.csa_indexer_query.restype = C.c_int
         L.csa_indexer_query.argtypes = [C.POINTER(IqueryArgs), _vp]
+        L.csa_grouped_out_proj_workspace_size.restype = C.c_size_t
+        L.csa_grouped_out_proj_workspace_size.argtypes = [C.c_int32, C.c_int32, C.c_int32]
+        L.csa_grouped_out_proj.restype = C.c_int
+        L.csa_grouped_out_proj.argtypes = [C.POINTER(OprojArgs), _vp, C.c_size_t, _vp]
         L.csa_indexer_topk_workspace_size.restype = C.c_size_t
         L.csa_indexer_topk_workspace_size.argtypes = [C.c_int32, C.c_int64, C.c_int32]
         for f in ("csa_indexer_topk", "csa_indexer_topk_bf16"):
@@ -217,6 +228,26 @@ def indexer_query(c, W, H_I: int, *, q_fp4=None, q_sf=None, dbg: bool = False,
                       _ptr(d, elem=4, name="dbg"), _ptr(dev_status, elem=4, name="dev_status"))
     _check(lib().csa_indexer_query(C.byref(args), _stream(stream)), "csa_indexer_query")
     return q_fp4, q_sf, d
+
+
+def grouped_out_proj(attn, Wg, Wo, *, workspace=None, out=None, dev_status=None, stream=None):
+    """attn bf16 [T][H][512], Wg bf16 [G][d_g][H/G*512], Wo bf16 [d_model][G*d_g] ->
+    out bf16 [T][d_model]."""
+    T, H, _ = attn.shape
+    G, d_g, _ = Wg.shape
+    d_model = Wo.shape[0]
+    dev = attn.device
+    if workspace is None:
+        n = lib().csa_grouped_out_proj_workspace_size(T, G, d_g)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=dev)
+    if out is None:
+        out = torch.empty((T, d_model), dtype=torch.bfloat16, device=dev)
+    args = OprojArgs(T, H, G, d_g, d_model, _ptr(attn, elem=2, name="attn"),
+                     _ptr(Wg, elem=2, name="Wg"), _ptr(Wo, elem=2, name="Wo"),
+                     _ptr(out, elem=2, name="out"), _ptr(dev_status, elem=4, name="dev_status"))
+    _check(lib().csa_grouped_out_proj(C.byref(args), workspace.data_ptr(), workspace.numel(),
+                                      _stream(stream)), "csa_grouped_out_proj")
+    return out
 
 
 # ------------------------------------------------------------- indexer top-k

@@ -9,6 +9,9 @@
 namespace csa {
 cudaError_t launch_compress(const csa_compress_args& a, cudaStream_t stream);
 cudaError_t launch_ikey_compress(const csa_ikey_args& a, cudaStream_t stream);
+cudaError_t launch_gemm_bf16(const CUtensorMap& amap, const CUtensorMap& bmap, int M, int N,
+                             int K, int G, int a_x_group, int b_y_group, int64_t c_x_group,
+                             uint16_t* C, int64_t ldc, int32_t* dev_status, cudaStream_t stream);
 cudaError_t launch_iquery(const csa_iquery_args& a, const CUtensorMap& cmap,
                           const CUtensorMap& wmap, cudaStream_t stream);
 cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
@@ -123,6 +126,19 @@ bool encode_q_map(EncodeTiledFn enc, CUtensorMap* qmap, const uint16_t* q, int64
          CUDA_SUCCESS;
 }
 
+// A BF16 matrix [rows][cols] (row-major) read in 64 x 128 boxes with the 128-byte swizzle.
+bool encode_bf16_map(EncodeTiledFn enc, CUtensorMap* map, const uint16_t* base, int64_t cols,
+                     int64_t rows) {
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<uint16_t*>(base), dims,
+             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 bool encode_key_map(EncodeTiledFn enc, CUtensorMap* kmap, const uint8_t* k_fp4, int64_t Nmax,
                     int64_t B) {
   const cuuint64_t dims[3] = {64, (cuuint64_t)Nmax, (cuuint64_t)B};
@@ -218,6 +234,43 @@ int csa_indexer_query(const csa_iquery_args* a, csa_stream_t stream) {
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return CSA_ERR_CUDA;
   return cuda_status(launch_iquery(*a, cmap, wmap, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+size_t csa_grouped_out_proj_workspace_size(int32_t T, int32_t G, int32_t d_g) {
+  if (T < 0 || G < 1 || d_g < 1) return 0;
+  return (((size_t)T * G * d_g * 2) + 255) & ~(size_t)255;
+}
+
+int csa_grouped_out_proj(const csa_oproj_args* a, void* ws, size_t ws_bytes,
+                         csa_stream_t stream) {
+  if (!a) return CSA_ERR_INVALID_ARG;
+  if (a->T < 0 || a->G < 1 || a->d_g < 1 || a->d_model < 1) return CSA_ERR_INVALID_ARG;
+  if ((a->H != 64 && a->H != 128) || a->H % a->G || a->d_g % 128 || a->d_model % 128 ||
+      (int64_t)a->G * a->d_g > 65536)
+    return CSA_ERR_UNSUPPORTED;
+  if (a->T == 0) return CSA_OK;
+  if (!ok_ptr(a->attn) || !ok_ptr(a->Wg) || !ok_ptr(a->Wo) || !ok_ptr(a->out) ||
+      (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)))
+    return CSA_ERR_INVALID_ARG;
+  if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255) ||
+      ws_bytes < csa_grouped_out_proj_workspace_size(a->T, a->G, a->d_g))
+    return CSA_ERR_WORKSPACE;
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return CSA_ERR_CUDA;
+  const int K1 = a->H / a->G * CSA_HEAD_DIM, M = a->G * a->d_g;
+  uint16_t* mid = reinterpret_cast<uint16_t*>(ws);
+  CUtensorMap m_attn, m_wg, m_mid, m_wo;
+  if (!encode_bf16_map(enc, &m_attn, a->attn, (int64_t)a->H * CSA_HEAD_DIM, a->T) ||
+      !encode_bf16_map(enc, &m_wg, a->Wg, K1, (int64_t)a->G * a->d_g) ||
+      !encode_bf16_map(enc, &m_mid, mid, M, a->T) ||
+      !encode_bf16_map(enc, &m_wo, a->Wo, M, a->d_model))
+    return CSA_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_gemm_bf16(m_attn, m_wg, a->T, a->d_g, K1, a->G, K1, a->d_g, a->d_g,
+                                   mid, M, a->dev_status, st);
+  if (e != cudaSuccess) return CSA_ERR_CUDA;
+  return cuda_status(launch_gemm_bf16(m_mid, m_wo, a->T, a->d_model, M, 1, 0, 0, 0, a->out,
+                                      a->d_model, a->dev_status, st));
 }
 
 size_t csa_indexer_topk_workspace_size(int32_t B, int64_t Nmax, int32_t k) {

@@ -160,6 +160,26 @@ def test_indexer_query_matches_oracle(T, r, H_I):
     assert flips <= max(4, T * H_I * 128 // 2000)
 
 
+# -------------------------------------------------------- grouped output projection
+@pytest.mark.parametrize("T,H,G,d_g,d_model", [
+    (200, 64, 16, 128, 256),     # two token tiles, the second ragged
+    (4, 128, 16, 1024, 1024),    # one decode step of the 1M workload's heads
+    (130, 128, 8, 256, 384),
+])
+def test_grouped_out_proj_matches_oracle(T, H, G, d_g, d_model):
+    rng = np.random.default_rng(T + H + G)
+    attn = synth.bf16_normal(rng, (T, H, 512))
+    K1 = H // G * 512
+    Wg = synth.bf16_normal(rng, (G, d_g, K1), std=0.5 * K1 ** -0.5)
+    Wo = synth.bf16_normal(rng, (d_model, G * d_g), std=0.5 * (G * d_g) ** -0.5)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out = csa.grouped_out_proj(dev(attn), dev(Wg), dev(Wo), dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    want, _ = oracle.grouped_out_proj(attn, Wg, Wo)
+    compare.close(out.float().cpu().numpy(), want, what="grouped output projection")
+
+
 # ------------------------------------------------------------- indexer top-k
 def _topk_case(B, H_I, Nmax, n, k, planted=0, seed=0):
     rng = np.random.default_rng(seed)
