@@ -108,6 +108,63 @@ typedef struct {
 int csa_compress(const csa_compress_args* args, csa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
+ * csa_decode_append: one decode step's update of the per-sequence state (walkthrough
+ * §3.5: the state cache holds the 128 window tokens and the tail of the unfinished
+ * block, the classical cache the compressed entries).
+ * For each sequence b with new token t = pos[b]:
+ *   - a / za go to tail row t % m of tail_a / tail_za [B][m][512]; b / zb (overlap) to
+ *     row t % m of slot (t / m) & 1 of the two-block ring tail_b / tail_zb [B][2][m][512]
+ *     (the slot of block i - 1 is block i's previous block);
+ *   - the window row of t (RMSNorm, RoPE at t, BF16, as csa_prefill's) is written to
+ *     swa[b][t % 128];
+ *   - when t % m == m - 1 the block t / m is compressed from the tails exactly as
+ *     csa_compress (previous block from the ring when t / m > 0 and overlap = 1) into row
+ *     t / m of kv / kv_scale, n_entries[b] = t / m + 1, and when the indexer-key stream
+ *     is given (ia != NULL) its key is compressed as csa_compress_index_keys into
+ *     k_fp4 / k_sf from the tails itail_* ([B][m][128], ring [B][2][m][128]).
+ * The state buffers are the caller's; a sequence starting mid-stream must hold its
+ * previous block in the ring slot of block t / m - 1. A position whose block would not
+ * fit Nmax is reported through dev_status and skipped.
+ */
+typedef struct {
+  int32_t B;
+  int32_t m;               /* block size: 4 for CSA, 128 for HCA */
+  int32_t overlap;         /* 1: CSA overlapping merge */
+  float rope_base;
+  float eps;
+  const int32_t* pos;      /* [B] position of the new token */
+  const uint16_t* a;       /* bf16 [B][512] */
+  const uint16_t* b;       /* bf16 [B][512] (overlap) */
+  const float* za;         /* [B][512] */
+  const float* zb;         /* [B][512] (overlap) */
+  const float* bias;       /* [2m] or [m] */
+  const float* norm_w;     /* [512] or NULL */
+  uint16_t* tail_a;        /* state bf16 [B][m][512] */
+  float* tail_za;          /* state [B][m][512] */
+  uint16_t* tail_b;        /* state bf16 [B][2][m][512] (overlap) */
+  float* tail_zb;          /* state [B][2][m][512] (overlap) */
+  uint16_t* swa;           /* state bf16 [B][128][512] window ring */
+  uint8_t* kv;             /* cache [B][Nmax][576] */
+  float* kv_scale;         /* cache [B][Nmax] */
+  int64_t Nmax;            /* entry capacity, multiple of 128 */
+  int32_t* n_entries;      /* [B] updated when a block closes */
+  const uint16_t* ia;      /* optional indexer-key stream: bf16 [B][128] (NULL: none) */
+  const uint16_t* ib;
+  const float* iza;
+  const float* izb;
+  const float* ibias;      /* [2m] */
+  uint16_t* itail_a;       /* state bf16 [B][m][128] */
+  float* itail_za;         /* state [B][m][128] */
+  uint16_t* itail_b;       /* state bf16 [B][2][m][128] */
+  float* itail_zb;         /* state [B][2][m][128] */
+  uint8_t* k_fp4;          /* [B][Nmax][64] */
+  uint8_t* k_sf;           /* [B][Nmax/128][512] */
+  int32_t* dev_status;     /* optional device word */
+} csa_append_args;
+
+int csa_decode_append(const csa_append_args* args, csa_stream_t stream);
+
+/* ------------------------------------------------------------------------------------
  * csa_compress_index_keys: the indexer keys of the compressed entries.
  * (walkthrough §2.2: the lightning indexer scores the compressed entries; §3.4: its QK
  * path is FP4.) The pages do not spell out how the indexer keys are built; this call

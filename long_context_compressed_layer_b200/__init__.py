@@ -51,6 +51,17 @@ class OprojArgs(C.Structure):
                 ("dev_status", _vp)]
 
 
+class AppendArgs(C.Structure):
+    _fields_ = [("B", C.c_int32), ("m", C.c_int32), ("overlap", C.c_int32),
+                ("rope_base", C.c_float), ("eps", C.c_float), ("pos", _vp), ("a", _vp),
+                ("b", _vp), ("za", _vp), ("zb", _vp), ("bias", _vp), ("norm_w", _vp),
+                ("tail_a", _vp), ("tail_za", _vp), ("tail_b", _vp), ("tail_zb", _vp),
+                ("swa", _vp), ("kv", _vp), ("kv_scale", _vp), ("Nmax", C.c_int64),
+                ("n_entries", _vp), ("ia", _vp), ("ib", _vp), ("iza", _vp), ("izb", _vp),
+                ("ibias", _vp), ("itail_a", _vp), ("itail_za", _vp), ("itail_b", _vp),
+                ("itail_zb", _vp), ("k_fp4", _vp), ("k_sf", _vp), ("dev_status", _vp)]
+
+
 class TopkArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("H_I", C.c_int32), ("k", C.c_int32), ("Nmax", C.c_int64),
                 ("n_entries", _vp), ("q_fp4", _vp), ("q_sf", _vp), ("w", _vp),
@@ -77,7 +88,7 @@ class PrefillArgs(C.Structure):
                 ("lse", _vp), ("idx", _vp), ("dev_status", _vp)]
 
 
-EXPORTS = ["csa_status_string", "csa_compress", "csa_compress_index_keys",
+EXPORTS = ["csa_status_string", "csa_compress", "csa_compress_index_keys", "csa_decode_append",
            "csa_indexer_query", "csa_grouped_out_proj_workspace_size", "csa_grouped_out_proj",
            "csa_indexer_topk_workspace_size",
            "csa_indexer_topk", "csa_indexer_topk_bf16", "csa_attn_workspace_size", "csa_sparse_attn_decode",
@@ -101,6 +112,8 @@ def lib() -> C.CDLL:
         L.csa_status_string.argtypes = [C.c_int]
         L.csa_compress.restype = C.c_int
         L.csa_compress.argtypes = [C.POINTER(CompressArgs), _vp]
+        L.csa_decode_append.restype = C.c_int
+        L.csa_decode_append.argtypes = [C.POINTER(AppendArgs), _vp]
         L.csa_compress_index_keys.restype = C.c_int
         L.csa_compress_index_keys.argtypes = [C.POINTER(IkeyArgs), _vp]
         L.csa_indexer_query.restype = C.c_int
@@ -183,6 +196,51 @@ def compress(a, za, bias, m: int, overlap: bool, *, b=None, zb=None, pos0: int =
                         Nmax, _ptr(d, elem=4, name="dbg"))
     _check(lib().csa_compress(C.byref(args), _stream(stream)), "csa_compress")
     return kv, kv_scale, d
+
+
+def new_decode_state(B: int, Nmax: int, m: int = 4, index_keys: bool = True, device="cuda"):
+    """Zeroed per-sequence decode state: block tails, the window ring, the compressed cache
+    and (optionally) the indexer-key tails and keys."""
+    z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=device)
+    st = {"tail_a": z((B, m, HEAD_DIM), torch.int16), "tail_za": z((B, m, HEAD_DIM), torch.float32),
+          "tail_b": z((B, 2, m, HEAD_DIM), torch.int16),
+          "tail_zb": z((B, 2, m, HEAD_DIM), torch.float32),
+          "swa": z((B, WINDOW, HEAD_DIM), torch.int16), "kv": z((B, Nmax, ROW_BYTES), torch.uint8),
+          "kv_scale": z((B, Nmax), torch.float32), "n_entries": z((B,), torch.int32)}
+    if index_keys:
+        st.update({"itail_a": z((B, m, INDEX_DIM), torch.int16),
+                   "itail_za": z((B, m, INDEX_DIM), torch.float32),
+                   "itail_b": z((B, 2, m, INDEX_DIM), torch.int16),
+                   "itail_zb": z((B, 2, m, INDEX_DIM), torch.float32),
+                   "k_fp4": z((B, Nmax, 64), torch.uint8),
+                   "k_sf": z((B, Nmax // 128 * 512), torch.uint8)})
+    return st
+
+
+def decode_append(pos, a, za, bias, state, *, b=None, zb=None, m: int = 4, overlap: bool = True,
+                  norm_w=None, rope_base: float = 10000.0, eps: float = 1e-6, ia=None, ib=None,
+                  iza=None, izb=None, ibias=None, dev_status=None, stream=None):
+    """Append one token per sequence (a, b bf16 [B][512]; za, zb [B][512]; ia.. [B][128]) at
+    positions pos [B] to a state from new_decode_state."""
+    B = a.shape[0]
+    g = lambda k_, el: _ptr(state.get(k_), elem=el, name=k_)
+    args = AppendArgs(B, m, int(overlap), rope_base, eps, _ptr(pos, elem=4, name="pos"),
+                      _ptr(a, elem=2, name="a"), _ptr(b, elem=2, name="b"),
+                      _ptr(za, elem=4, name="za"), _ptr(zb, elem=4, name="zb"),
+                      _ptr(bias, elem=4, name="bias"), _ptr(norm_w, elem=4, name="norm_w"),
+                      g("tail_a", 2), g("tail_za", 4), g("tail_b", 2), g("tail_zb", 4),
+                      g("swa", 2), g("kv", 1), g("kv_scale", 4), state["kv"].shape[1],
+                      g("n_entries", 4), _ptr(ia, elem=2, name="ia"), _ptr(ib, elem=2, name="ib"),
+                      _ptr(iza, elem=4, name="iza"), _ptr(izb, elem=4, name="izb"),
+                      _ptr(ibias, elem=4, name="ibias"),
+                      g("itail_a", 2) if ia is not None else None,
+                      g("itail_za", 4) if ia is not None else None,
+                      g("itail_b", 2) if ia is not None else None,
+                      g("itail_zb", 4) if ia is not None else None,
+                      g("k_fp4", 1) if ia is not None else None,
+                      g("k_sf", 1) if ia is not None else None,
+                      _ptr(dev_status, elem=4, name="dev_status"))
+    _check(lib().csa_decode_append(C.byref(args), _stream(stream)), "csa_decode_append")
 
 
 def compress_index_keys(a, za, bias, m: int, overlap: bool, *, b=None, zb=None, pos0: int = 0,

@@ -9,6 +9,7 @@
 namespace csa {
 cudaError_t launch_compress(const csa_compress_args& a, cudaStream_t stream);
 cudaError_t launch_ikey_compress(const csa_ikey_args& a, cudaStream_t stream);
+cudaError_t launch_append(const csa_append_args& a, cudaStream_t stream);
 cudaError_t launch_gemm_bf16(const CUtensorMap& amap, const CUtensorMap& bmap, int M, int N,
                              int K, int G, int a_x_group, int b_y_group, int64_t c_x_group,
                              uint16_t* C, int64_t ldc, int32_t* dev_status, cudaStream_t stream);
@@ -189,6 +190,27 @@ int csa_compress(const csa_compress_args* a, csa_stream_t stream) {
     if (a->pos0 > 0 && (!ok_ptr(a->prev_b) || !ok_ptr(a->prev_zb))) return CSA_ERR_INVALID_ARG;
   }
   return cuda_status(launch_compress(*a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+int csa_decode_append(const csa_append_args* a, csa_stream_t stream) {
+  if (!a) return CSA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->m < 1 || a->m > 128 || a->Nmax < 0 || a->Nmax % 128 ||
+      (a->overlap != 0 && a->overlap != 1) || !(a->eps >= 0.f) || !(a->rope_base > 0.f))
+    return CSA_ERR_INVALID_ARG;
+  if (a->B > 65535) return CSA_ERR_UNSUPPORTED;
+  if (a->B == 0) return CSA_OK;
+  if (!ok_ptr(a->pos) || !ok_ptr(a->a) || !ok_ptr(a->za) || !ok_ptr(a->bias) ||
+      !ok_opt(a->norm_w) || !ok_ptr(a->tail_a) || !ok_ptr(a->tail_za) || !ok_ptr(a->swa) ||
+      !ok_ptr(a->kv) || !ok_ptr(a->kv_scale) || !ok_ptr(a->n_entries) ||
+      (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)))
+    return CSA_ERR_INVALID_ARG;
+  if (a->overlap && (!ok_ptr(a->b) || !ok_ptr(a->zb) || !ok_ptr(a->tail_b) || !ok_ptr(a->tail_zb)))
+    return CSA_ERR_INVALID_ARG;
+  if (a->ia && (!ok_ptr(a->ib) || !ok_ptr(a->iza) || !ok_ptr(a->izb) || !ok_ptr(a->ibias) ||
+                !ok_ptr(a->itail_a) || !ok_ptr(a->itail_za) || !ok_ptr(a->itail_b) ||
+                !ok_ptr(a->itail_zb) || !ok_ptr(a->k_fp4) || !ok_ptr(a->k_sf) || !a->overlap))
+    return CSA_ERR_INVALID_ARG;
+  return cuda_status(launch_append(*a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 int csa_compress_index_keys(const csa_ikey_args* a, csa_stream_t stream) {

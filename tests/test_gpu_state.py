@@ -1,0 +1,65 @@
+"""Decode-step state updates (csa_decode_append) against whole-stream compression."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from synth import inputs as synth
+
+pytestmark = pytest.mark.gpu
+
+csa = pytest.importorskip("long_context_compressed_layer_b200")
+
+
+def dev(x):
+    x = np.ascontiguousarray(x)
+    return torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).cuda()
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no GPU")
+    csa.lib()
+
+
+def test_token_by_token_appends_equal_whole_stream_compression():
+    B, S, m = 2, 4 * 37 + 2, 4  # 37 closed blocks, two tokens left in the tail
+    kvs = synth.compress_inputs(B, S, m, True, seed=61)
+    iks = synth.compress_inputs(B, S, m, True, seed=62, dim=128)
+    Nmax = 128
+    st = csa.new_decode_state(B, Nmax, m)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    d = {k: dev(v) for k, v in kvs.items()}
+    di = {k: dev(v) for k, v in iks.items()}
+    for t in range(S):
+        pos = torch.full((B,), t, dtype=torch.int32, device="cuda")
+        csa.decode_append(pos, d["a"][:, t].contiguous(), d["za"][:, t].contiguous(), d["bias"],
+                          st, b=d["b"][:, t].contiguous(), zb=d["zb"][:, t].contiguous(), m=m,
+                          ia=di["a"][:, t].contiguous(), ib=di["b"][:, t].contiguous(),
+                          iza=di["za"][:, t].contiguous(), izb=di["zb"][:, t].contiguous(),
+                          ibias=di["bias"], dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    assert (st["n_entries"].cpu().numpy() == S // m).all()
+    # the same entries and keys as the whole-stream calls (the same block arithmetic)
+    kv, sc, _ = csa.compress(d["a"], d["za"], d["bias"], m, True, b=d["b"], zb=d["zb"],
+                             Nmax=Nmax)
+    kf, ks, _ = csa.compress_index_keys(di["a"], di["za"], di["bias"], m, True, b=di["b"],
+                                        zb=di["zb"], Nmax=Nmax)
+    torch.cuda.synchronize()
+    n = S // m
+    assert torch.equal(st["kv"][:, :n], kv[:, :n]) and torch.equal(st["kv_scale"][:, :n],
+                                                                   sc[:, :n])
+    assert torch.equal(st["k_fp4"][:, :n], kf[:, :n]) and torch.equal(st["k_sf"], ks)
+    # the window ring holds the last 128 tokens' window rows
+    ring = st["swa"].cpu().numpy().view(np.uint16)
+    for bb in range(B):
+        for p in (S - 128, S - 57, S - 1):
+            want = oracle.swa_row(kvs["a"][bb, p], p)
+            got = ring[bb, p % 128]
+            wf = want.astype(np.uint32) << 16
+            gf = got.astype(np.uint32) << 16
+            np.testing.assert_allclose(gf.view(np.float32), wf.view(np.float32), rtol=2.0 ** -7,
+                                       atol=1e-6)
