@@ -158,3 +158,81 @@ def test_cuda_sources_are_sm100a_only():
         text = open(f).read()
         assert "multicast" not in text  # no TMA multicast anywhere
         assert "wgmma" not in text and "mma.sync" not in text
+
+
+def test_index_key_compression_rejects_on_host(L):
+    def args(**over):
+        a = csa.IkeyArgs(1, 64, 4, 1, 0, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, FAKE, FAKE,
+                         128, None)
+        for k, v in over.items():
+            setattr(a, k, v)
+        return a
+
+    f = lambda a: L.csa_compress_index_keys(C.byref(a), None)
+    assert L.csa_compress_index_keys(None, None) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(Nmax=100)) == csa.CSA_ERR_INVALID_ARG      # not a multiple of 128
+    assert f(args(pos0=6)) == csa.CSA_ERR_INVALID_ARG        # not a block boundary
+    assert f(args(pos0=512)) == csa.CSA_ERR_INVALID_ARG      # 144 entries > Nmax, no tail
+    assert f(args(b=None)) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(k_sf=FAKE + 4)) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(T=3)) == csa.CSA_OK                        # no complete block
+
+
+def test_indexer_query_rejects_on_host(L):
+    def args(**over):
+        a = csa.IqueryArgs(16, 1536, 64, FAKE, FAKE, FAKE, FAKE, None, None)
+        for k, v in over.items():
+            setattr(a, k, v)
+        return a
+
+    f = lambda a: L.csa_indexer_query(C.byref(a), None)
+    assert f(args(r=100)) == csa.CSA_ERR_INVALID_ARG   # not a multiple of 64
+    assert f(args(r=32768)) == csa.CSA_ERR_UNSUPPORTED
+    assert f(args(H_I=8)) == csa.CSA_ERR_UNSUPPORTED
+    assert f(args(W=None)) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(T=0)) == csa.CSA_OK
+
+
+def test_grouped_out_proj_rejects_on_host(L):
+    ws_ok = L.csa_grouped_out_proj_workspace_size(64, 16, 1024)
+    assert ws_ok >= 64 * 16 * 1024 * 2
+
+    def args(**over):
+        a = csa.OprojArgs(64, 128, 16, 1024, 7168, FAKE, FAKE, FAKE, FAKE, None)
+        for k, v in over.items():
+            setattr(a, k, v)
+        return a
+
+    f = lambda a, ws=FAKE, n=ws_ok: L.csa_grouped_out_proj(C.byref(a), ws, n, None)
+    assert f(args(G=3)) == csa.CSA_ERR_UNSUPPORTED        # does not divide 128 heads
+    assert f(args(d_g=1000)) == csa.CSA_ERR_UNSUPPORTED   # not a multiple of 128
+    assert f(args(H=96)) == csa.CSA_ERR_UNSUPPORTED
+    assert f(args(out=None)) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(), n=ws_ok - 1) == csa.CSA_ERR_WORKSPACE
+    assert f(args(T=0)) == csa.CSA_OK
+
+
+def test_decode_append_rejects_on_host(L):
+    def args(**over):
+        a = csa.AppendArgs(2, 4, 1, 10000.0, 1e-6, *([FAKE] * 6), None, *([FAKE] * 7), 128,
+                           FAKE, *([None] * 11), None)
+        for k, v in over.items():
+            setattr(a, k, v)
+        return a
+
+    f = lambda a: L.csa_decode_append(C.byref(a), None)
+    assert L.csa_decode_append(None, None) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(m=0)) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(Nmax=100)) == csa.CSA_ERR_INVALID_ARG
+    assert f(args(tail_b=None)) == csa.CSA_ERR_INVALID_ARG     # overlap needs the ring
+    assert f(args(ia=FAKE)) == csa.CSA_ERR_INVALID_ARG         # a key stream needs its state
+    assert f(args(B=0)) == csa.CSA_OK
+
+
+def test_bf16_index_scores_share_the_indexer_checks(L):
+    ws_ok = L.csa_indexer_topk_workspace_size(2, 1024, 512)
+    call = lambda a, ws=FAKE, n=ws_ok: L.csa_indexer_topk_bf16(C.byref(a), ws, n, None)
+    assert call(_topk_args(Nmax=1000)) == csa.CSA_ERR_INVALID_ARG
+    assert call(_topk_args(H_I=8)) == csa.CSA_ERR_UNSUPPORTED
+    assert call(_topk_args(), n=ws_ok - 1) == csa.CSA_ERR_WORKSPACE
+    assert call(_topk_args(B=0)) == csa.CSA_OK
