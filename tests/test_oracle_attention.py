@@ -213,3 +213,35 @@ def test_swa_row_at_position_zero_is_the_normalised_token():
     x = indep.bf16_to_f64(a)
     want = indep.f64_to_bf16(x / np.sqrt(np.mean(x * x) + 1e-6))
     np.testing.assert_array_equal(oracle.swa_row(a, 0), want)
+
+
+def test_online_blocking_over_any_split_equals_the_oracle():
+    # P-11: merging running (max, sum, output) over arbitrary blocks of the row list, the
+    # sink entering only the denominator, reproduces the oracle's result to 1e-12
+    d = _small_decode(9)
+    rng = np.random.default_rng(9)
+    got, lse = oracle.attention(d["q"], d["pos"], d["n"], d["kv"], d["sc"], d["swa"],
+                                d["sink"], derotate=False)
+    for b in range(2):
+        ent = indep.dequant_rows(d["kv"][b, : d["n"][b]], d["sc"][b, : d["n"][b]])
+        V = np.concatenate([ent, _window_rows(d["swa"][b], d["pos"][b])])
+        q = indep.bf16_to_f64(d["q"][b])
+        for _ in range(3):
+            perm = rng.permutation(len(V))
+            cuts = np.sort(rng.choice(np.arange(1, len(V)), size=7, replace=False))
+            M = np.full(q.shape[0], -np.inf)
+            S = np.zeros(q.shape[0])
+            O = np.zeros((q.shape[0], 512))
+            for blk in np.split(perm, cuts):
+                lg = TAU * q @ V[blk].T
+                mb = lg.max(1)
+                Mn = np.maximum(M, mb)
+                a = np.exp(M - Mn)
+                e = np.exp(lg - Mn[:, None])
+                S = S * a + e.sum(1)
+                O = O * a[:, None] + e @ V[blk]
+                M = Mn
+            sink = d["sink"].astype(np.float64)
+            Z = S + np.exp(sink - M)
+            np.testing.assert_allclose(O / Z[:, None], got[b], rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(M + np.log(Z), lse[b], rtol=1e-12)
