@@ -167,6 +167,12 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
     from synth import inputs as synth
 
     torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
     w = synth.WORKLOADS[PREFILL_ID]
     d = synth.prefill_inputs_device(w.P, w.T, w.m, w.H, w.H_I, seed=w.seed + 1000 * rank)
     T, k = w.T, w.k
@@ -189,12 +195,16 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
     for _ in range(max(args.warmup, 3)):
         step()
     torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
         step()
     e1.record(stream)
     torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
     clocks = sampler.stop()
     ms = e0.elapsed_time(e1) / args.steps
     if int(status.item()) != 0:
@@ -286,6 +296,9 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
     torch.cuda.synchronize()
     e2e_ms = x0.elapsed_time(x1) / args.steps
     d["kv"].copy_(kv0)
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, "cuda")
+    if world > 1:
+        dist.destroy_process_group()
     if rank != 0:
         return
     f4, f16 = prefill_flops(w.P, T, w.m, w.H, w.H_I, k)
@@ -295,7 +308,7 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
     # FP4 counts at the nominal 4x of dense BF16 (no FP4 peak is measured on this machine)
     eq_tflops = (f4 / 4 + f16) / (ms * 1e-3) / 1e12
     line = {
-        "metric": PREFILL_METRIC, "value": T / (ms * 1e-3), "unit": "tokens/s",
+        "metric": PREFILL_METRIC, "value": whole_job_rate(T, world, ms), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp4+fp16", "data": "synthetic",
@@ -323,7 +336,8 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
                                   if "bf16_tflops_sustained" in pk else "fallback"),
                      "traffic": None},
         "clocks": clocks,
-        "e2e": {"value": T / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s",
+                "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
     }
     print(json.dumps(line), flush=True)
