@@ -2,29 +2,34 @@
 // indexer queries score the compressed entries and each query keeps the top-k, one set
 // for all heads; §3.4 and chooseai.net §二: the indexer QK path runs in MXFP4).
 //
-// Kernel 1, indexer_score_kernel: a persistent (one CTA per SM), warp-specialised stream
-// over the FP4 keys.
-//   warp 0      TMA producer: 128-entry key tiles (128 x 64 B, 64-byte swizzle) and the
-//               tile's 512-byte scale group, into a 12-stage shared-memory ring;
-//   warp 1      tcgen05 issuer: copies the key scales into TMEM (tcgen05.cp), then two
-//               kind::mxf4 block-scaled MMAs (K = 64 each) give D[128 entries x 64 heads]
-//               in fp32 TMEM, four accumulators deep; it also stages each sequence's FP4
-//               queries (B operand) and their scales;
-//   warps 2..9  epilogue, two groups of four (one warp per TMEM lane quadrant) taking
-//               alternate tiles: one thread per entry reads its 64 head sums from TMEM and
-//               forms s = sum_h w_h * max(0, acc_h) in fp32 (w held in registers), writes it
-//               to the score workspace and counts its order-preserving key into the warp's
-//               own 4096-bin histogram (16-bit counters), flushed to the sequence's global
-//               histogram when the warp moves to another sequence.
-// Kernels 2-3, the selection (no sorting anywhere):
-//   topk_threshold_kernel: per sequence and 8192-entry slice, the histogram fixes the bin
+// indexer_score_kernel: a persistent, warp-specialised stream over the FP4 keys, launched
+// cooperatively with one CTA per SM. Each CTA runs two independent pipelines over two
+// halves of its contiguous range of (sequence, 128-entry tile) work items, each pipeline
+// with its own warps, shared-memory ring and half of TMEM:
+//   producer warp  TMA loads of the 128 x 64-byte key tile (64-byte swizzle) and the
+//                  tile's 512-byte scale group into a 6-stage ring;
+//   issuer warp    copies the key scales into TMEM (tcgen05.cp), issues two kind::mxf4
+//                  block-scaled MMAs (K = 64 each) giving D[128 entries x 64 heads] in fp32
+//                  TMEM, three accumulators deep, and stages each sequence's FP4 queries
+//                  (B operand) and their scales;
+//   4 epilogue warps  one per TMEM lane quadrant, one thread per entry: reads its 64 head
+//                  sums, forms s = sum_h w_h * max(0, acc_h) in fp32 (w in registers, head
+//                  pairs in packed FMAs; rounded to BF16 when asked), writes the score to
+//                  the workspace and counts its order-preserving key into the warp's own
+//                  2048-bin histogram (16-bit counters), flushed to the sequence's global
+//                  histogram when the warp moves to another sequence.
+// After a grid barrier the same CTAs select (no sorting anywhere):
+//   select_threshold: per sequence and 12,288-entry slice, the histogram fixes the bin
 //     that holds the k-th score (a parallel suffix scan); each CTA counts its entries above
 //     that bin and appends the in-bin candidates. The last CTA of a sequence (atomic ticket,
 //     no spinning) resolves the exact cut inside the bin by a radix select on the remaining
-//     20 key bits (ties broken by the smaller index), then turns the per-slice counts into
-//     output offsets and clears the histogram and counters for the next call;
-//   topk_write_kernel: every slice writes its selected entries in index order at its offset,
-//     so the output comes out ascending without a sort.
+//     21 key bits (ties broken by the smaller index), turns the per-slice counts into output
+//     offsets, clears the histogram and counters for the next call and publishes the cut;
+//   select_write: every slice writes its selected entries in index order at its offset, so
+//     the output comes out ascending without a sort.
+// If the cooperative launch is refused, scoring runs as an ordinary launch followed by the
+// same two steps as stand-alone kernels (topk_threshold_kernel, topk_write_kernel). The
+// prefill variant (prefill_score_kernel, topk_query_kernel) is described further down.
 #include "common.cuh"
 
 namespace csa {
@@ -869,7 +874,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_write_kernel(IxParams p) {
 // in two groups of four taking alternate tiles (accumulator buffer = tile parity). An
 // epilogue thread owns one entry and forms its kPxQ scores, masked by each query's own
 // eligible count, and counts them into per-warp, per-query histograms. The selection then
-// runs as the two stand-alone kernels, one CTA per (slice, query).
+// runs as topk_query_kernel, one CTA per query.
 constexpr int kPxQ = 3;                     // queries per group
 constexpr int kPxStages = 6;
 constexpr int kPxNbuf = 2;                  // accumulator buffers (one per epilogue group)
