@@ -6,7 +6,7 @@
 // Both stages are BF16 GEMM tiles C[128 x 128] = A[128 x K] B[128 x K]^T with fp32
 // accumulation in TMEM and a BF16 (round-to-nearest-even) epilogue: one CTA per
 // (row tile, column tile, group). Warp 0 streams 64-wide K blocks of A and B by TMA
-// (128-byte swizzle) into a 4-stage ring, warp 1 issues tcgen05.mma kind::f16 (BF16),
+// (128-byte swizzle) into a 3-stage ring (two CTAs fit an SM), warp 1 issues tcgen05.mma kind::f16 (BF16),
 // warps 2-5 (one per TMEM lane quadrant, one row per thread) convert and store. The
 // group index selects column offsets of A and C and a row offset of B, so stage 1 runs
 // all groups in one launch over the [T][H * 512] attention output.
@@ -14,7 +14,7 @@
 
 namespace csa {
 
-constexpr int kGmStages = 4;
+constexpr int kGmStages = 3;
 constexpr int kGmTile = 128;
 constexpr int kGmKBlk = 64;
 constexpr int kGmThreads = 192;

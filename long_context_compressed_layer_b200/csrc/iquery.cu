@@ -5,7 +5,7 @@
 //
 // One CTA per (128-token tile, indexer head): y[t][0..127] = sum_j W[h*128 + .][j] c[t][j]
 // is a 128 x 128 x r BF16 GEMM tile. Warp 0 streams the K blocks of c and W (64 BF16
-// each, 128-byte swizzle) by TMA into a 4-stage ring; warp 1 issues four
+// each, 128-byte swizzle) by TMA into a 3-stage ring (two CTAs fit an SM); warp 1 issues four
 // tcgen05.mma kind::f16 (BF16, K = 16) per block into 128 fp32 TMEM columns; warps 2-5
 // (one per TMEM lane quadrant, one token per thread) read the token's 128 values, and
 // per 32-value block form the MXFP4 shared exponent and E2M1 codes, writing 64 code
@@ -15,7 +15,7 @@
 
 namespace csa {
 
-constexpr int kIqStages = 4;
+constexpr int kIqStages = 3;
 constexpr int kIqTile = 128;   // tokens per CTA = MMA M; one head's 128 dims = MMA N
 constexpr int kIqKBlk = 64;    // BF16 elements per K block (one 128-byte swizzle row)
 constexpr int kIqThreads = 192;
