@@ -450,3 +450,32 @@ def test_workload1_hca_decode():
                                   d["swa"], d["sink"])
     compare.close(out.float().cpu().numpy(), want, what="workload 1")
     np.testing.assert_allclose(host(lse), wlse, rtol=1e-4, atol=1e-4)
+
+
+def test_workload3_full_size_decode():
+    """The 1M-context decode step at full size, through the calls bench.py times: every
+    sequence's top-k set against the oracle's scores, then the attention output of every
+    head against the oracle on the same quantised cache and the same sets."""
+    w = synth.WORKLOADS[3]
+    d = synth.decode_inputs(w)
+    n = d["n_entries"]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx, sc = csa.indexer_topk(dev(n), dev(d["q_fp4"]), dev(d["q_sf"]), dev(d["w"]),
+                               dev(d["k_fp4"]), dev(d["k_sf"]), w.k, scores=True,
+                               dev_status=status)
+    out, lse = csa.sparse_attn_decode(dev(d["q"]), dev(d["pos"]), dev(n), dev(d["kv"]),
+                                      dev(d["kv_scale"]), dev(d["swa"]), dev(d["sink"]), idx,
+                                      lse=True, dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    idx_h, sc_h = host(idx), host(sc)
+    ora_s = oracle.indexer_scores(n, d["q_fp4"], d["q_sf"], d["w"], d["k_fp4"], d["k_sf"])
+    flips = 0
+    for b in range(d["B"]):
+        flips += compare.compare_topk(idx_h[b], ora_s[b], int(n[b]), w.k, what=f"1M seq {b}")
+        np.testing.assert_allclose(sc_h[b], ora_s[b][idx_h[b]], rtol=2e-5, atol=1e-6)
+    assert flips <= 2 * d["B"]
+    want, wlse = oracle.attention(d["q"], d["pos"], n, d["kv"], d["kv_scale"], d["swa"],
+                                  d["sink"], idx=idx_h)
+    compare.close(out.float().cpu().numpy(), want, what="1M attention")
+    np.testing.assert_allclose(host(lse), wlse, rtol=1e-4, atol=1e-4)
