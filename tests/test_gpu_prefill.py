@@ -120,3 +120,49 @@ def test_prefill_without_derotation_and_deterministic():
     rows = np.array([0, 57, 199], np.int32)
     ora = oracle.prefill(inp, 128, rows, derotate=False)
     check_rows(inp, 128, a, rows, ora)
+
+
+def _host_inputs(d, rows):
+    """Host copies of a device-drawn prefill bundle for the oracle: every input except the
+    queries, which only the sampled rows need (the rest of the array stays untouched
+    zero pages)."""
+    def h(x):
+        x = x.cpu().numpy()
+        return x.view(np.uint16) if x.dtype == np.int16 else x
+
+    inp = {k: d[k] for k in ("P", "T", "m", "H", "H_I", "Nmax")}
+    for k in ("kv", "kv_scale", "k_fp4", "k_sf", "q_fp4", "q_sf", "w", "sink", "swa_prefix",
+              "a", "b", "za", "zb", "bias", "prev_b", "prev_zb"):
+        if k in d:
+            inp[k] = h(d[k])
+    q = np.zeros(tuple(d["q"].shape), dtype=np.uint16)
+    idx = torch.as_tensor(rows, dtype=torch.long, device=d["q"].device)
+    q[rows] = h(d["q"].index_select(0, idx))
+    inp["q"] = q
+    return inp
+
+
+@pytest.mark.slow
+def test_prefill_full_size_sampled_rows():
+    # the 64K-token prefill after a 192K-token prefix, as bench.py --workload prefill runs
+    # it, checked on rows at the start, chunk boundaries and the end
+    w = synth.WORKLOADS[4]
+    d = synth.prefill_inputs_device(w.P, w.T, w.m, w.H, w.H_I, seed=w.seed)
+    kv0 = d["kv"].clone()
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse, idx = csa.prefill(
+        w.P, w.m, w.k, a=d["a"], b=d["b"], za=d["za"], zb=d["zb"], bias=d["bias"], kv=d["kv"],
+        kv_scale=d["kv_scale"], q_fp4=d["q_fp4"], q_sf=d["q_sf"], w=d["w"], k_fp4=d["k_fp4"],
+        k_sf=d["k_sf"], q=d["q"], sink=d["sink"], prev_b=d["prev_b"], prev_zb=d["prev_zb"],
+        swa_prefix=d["swa_prefix"], lse=True, idx=True, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    rows = np.array([0, 1, 1023, 1024, 32767, 40000, w.T - 2, w.T - 1], np.int32)
+    kv_gpu = d["kv"]
+    d["kv"] = kv0  # the oracle compresses the new blocks itself from the prefix cache
+    inp = _host_inputs(d, rows)
+    ora = oracle.prefill(inp, w.k, rows)
+    got = dict(out=out.float().cpu().numpy(), lse=host(lse), idx=host(idx), kv=host(kv_gpu),
+               kv_scale=host(d["kv_scale"]))
+    check_cache(inp, got, ora)
+    check_rows(inp, w.k, got, rows, ora)
