@@ -35,21 +35,6 @@ __device__ __forceinline__ uint64_t globaltimer() {
   return t;
 }
 
-// Named barrier over `nthreads` threads that also ORs a flag across them: every
-// participant gets the same answer, so a decision taken on it never diverges.
-__device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool v) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 q, %1, 0;\n\t"
-      "bar.red.or.pred p, %2, %3, q;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)v), "r"(id), "r"(nthreads)
-      : "memory");
-  return r != 0;
-}
-
 // First error wins.
 __device__ __forceinline__ void report(int32_t* dev_status, int32_t code) {
   if (dev_status) atomicCAS(dev_status, 0, code);
@@ -429,10 +414,6 @@ __device__ __forceinline__ int mxfp4_exponent(float amax) {
 __device__ __forceinline__ uint32_t float_key(float f) {
   const uint32_t u = __float_as_uint(f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float key_float(uint32_t k) {
-  const uint32_t u = (k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k;
-  return __uint_as_float(u);
 }
 
 // RoPE angle p * base^(-j/32) reduced to [-pi, pi] in double precision, so that

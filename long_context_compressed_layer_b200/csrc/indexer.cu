@@ -1376,8 +1376,6 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
   return launch_pdl(topk_write_kernel, g2, dim3(kSelThreads), 0, stream, p);
 }
 
-size_t ix_smem_bytes() { return sizeof(IxSmem) + 1024; }
-
 // Indexer top-k of the queries of one prefill (all scoring the same keys): the shared-key
 // scoring kernel, then the two selection kernels.
 cudaError_t launch_prefill_indexer_topk(const csa_topk_args& a, void* workspace, int num_sms,
