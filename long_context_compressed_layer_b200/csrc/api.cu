@@ -509,11 +509,10 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
 }
 
 int csa_sparse_attn_decode_noalloc(const csa_attn_args* a, csa_stream_t stream) {
-  // Out-of-range sizes: let the ordinary checks pick the status (no workspace is passed,
-  // so nothing can launch).
-  if (!a || a->B <= 0 || a->B > 65535 || (a->H != 64 && a->H != 128) || a->k < 1 ||
-      a->k > 2048)
-    return attn_common(a, 1, nullptr, 0, stream);
+  // The ordinary checks first, with no workspace: they return before touching the device,
+  // and anything other than the missing workspace is the answer.
+  const int st = attn_common(a, 1, nullptr, 0, stream);
+  if (st != CSA_ERR_WORKSPACE) return st;
   if (at_workspace_size(a->B, a->H, a->k + CSA_WINDOW) > CSA_NOALLOC_SCRATCH_BYTES)
     return CSA_ERR_UNSUPPORTED;
   void* ws = noalloc_scratch();
