@@ -69,3 +69,32 @@ def dequant_rows(kv_rows, scale):
 def softmax(x, axis=-1):
     from scipy.special import softmax as sp_softmax
     return sp_softmax(x, axis=axis)
+
+
+def gated_merge(inp, m, overlap, pos0=0):
+    """The gated merge of a compression input bundle (streams a, b, logits za, zb, bias
+    [2m]) by the library softmax over an explicit candidate axis: entry i takes the m own
+    tokens of a with logits za + bias[:m] and, with overlap, the m previous-block tokens of
+    b (or of prev_b for the first entry of a later chunk) with logits zb + bias[m:]."""
+    a = bf16_to_f64(inp["a"])
+    B, T, D = a.shape
+    N = T // m
+    bias = inp["bias"].astype(np.float64)
+    e = np.empty((B, N, D))
+    for b in range(B):
+        for i in range(N):
+            xs = [a[b, m * i:m * i + m]]
+            zs = [inp["za"][b, m * i:m * i + m].astype(np.float64) + bias[:m, None]]
+            if overlap and (i > 0 or pos0 > 0):
+                if i > 0:
+                    xb = bf16_to_f64(inp["b"][b, m * (i - 1):m * i])
+                    zb = inp["zb"][b, m * (i - 1):m * i].astype(np.float64)
+                else:
+                    xb = bf16_to_f64(inp["prev_b"][b])
+                    zb = inp["prev_zb"][b].astype(np.float64)
+                xs.append(xb)
+                zs.append(zb + bias[m:, None])
+            x = np.concatenate(xs, 0)
+            z = np.concatenate(zs, 0)
+            e[b, i] = (softmax(z, axis=0) * x).sum(0)
+    return e

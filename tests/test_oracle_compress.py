@@ -8,32 +8,6 @@ from synth import inputs as synth
 from tests import indep
 
 
-def _merge_brute(inp, m, overlap, pos0=0):
-    """Gated merge by library softmax over an explicit candidate axis."""
-    a = indep.bf16_to_f64(inp["a"])
-    B, T, D = a.shape
-    N = T // m
-    bias = inp["bias"].astype(np.float64)
-    e = np.empty((B, N, D))
-    for b in range(B):
-        for i in range(N):
-            xs = [a[b, m * i:m * i + m]]
-            zs = [inp["za"][b, m * i:m * i + m].astype(np.float64) + bias[:m, None]]
-            if overlap and (i > 0 or pos0 > 0):
-                if i > 0:
-                    xb = indep.bf16_to_f64(inp["b"][b, m * (i - 1):m * i])
-                    zb = inp["zb"][b, m * (i - 1):m * i].astype(np.float64)
-                else:
-                    xb = indep.bf16_to_f64(inp["prev_b"][b])
-                    zb = inp["prev_zb"][b].astype(np.float64)
-                xs.append(xb)
-                zs.append(zb + bias[m:, None])
-            x = np.concatenate(xs, 0)
-            z = np.concatenate(zs, 0)
-            e[b, i] = (indep.softmax(z, axis=0) * x).sum(0)
-    return e
-
-
 @pytest.mark.parametrize("m,overlap,pos0", [(4, True, 0), (2, True, 8), (4, False, 0),
                                             (1, True, 4), (128, False, 0)])
 def test_merge_matches_library_softmax(m, overlap, pos0):
@@ -42,7 +16,7 @@ def test_merge_matches_library_softmax(m, overlap, pos0):
     r = oracle.compress(inp["a"], inp["za"], inp["bias"], m, overlap, b=inp.get("b"),
                         zb=inp.get("zb"), pos0=pos0, prev_b=inp.get("prev_b"),
                         prev_zb=inp.get("prev_zb"))
-    np.testing.assert_allclose(r["e"], _merge_brute(inp, m, overlap, pos0), rtol=1e-12,
+    np.testing.assert_allclose(r["e"], indep.gated_merge(inp, m, overlap, pos0), rtol=1e-12,
                                atol=1e-12)
 
 
@@ -92,6 +66,34 @@ def test_rmsnorm_closed_form_at_position_zero():
         ms = np.mean(e * e)
         np.testing.assert_allclose(y, e / np.sqrt(ms + 1e-6), rtol=1e-13)
         np.testing.assert_allclose(np.mean(y * y), ms / (ms + 1e-6), rtol=1e-12)
+
+
+def test_rmsnorm_weight_scales_each_normalised_dim():
+    # the optional RMSNorm weight multiplies dim d of the normalised entry by w[d]; with
+    # equal weights on the two dims of each RoPE pair the rotation commutes with it
+    rng = np.random.default_rng(12)
+    inp = synth.compress_inputs(2, 32, 4, True, seed=12)
+    w = rng.uniform(0.5, 2.0, 512).astype(np.float32)
+    w[449::2] = w[448::2]
+    base = oracle.compress(inp["a"], inp["za"], inp["bias"], 4, True, b=inp["b"], zb=inp["zb"])
+    wt = oracle.compress(inp["a"], inp["za"], inp["bias"], 4, True, b=inp["b"], zb=inp["zb"],
+                         norm_w=w)
+    np.testing.assert_array_equal(wt["e"], base["e"])
+    np.testing.assert_allclose(wt["y"], base["y"] * w.astype(np.float64), rtol=1e-13,
+                               atol=1e-15)
+
+
+def test_window_row_norm_weight_by_powers_of_two():
+    # powers of two scale binary floating point exactly, so the stored BF16 window row with
+    # such weights is the row without them times the weights
+    rng = np.random.default_rng(13)
+    a = synth.bf16_normal(rng, (512,))
+    w = (2.0 ** rng.integers(-2, 3, 512)).astype(np.float32)
+    w[449::2] = w[448::2]
+    for t in (0, 5, 1000):
+        plain = indep.bf16_to_f64(oracle.swa_row(a, t))
+        weighted = indep.bf16_to_f64(oracle.swa_row(a, t, norm_w=w))
+        np.testing.assert_array_equal(weighted, plain * w.astype(np.float64))
 
 
 def test_rope_pairs_keep_norm_and_turn_by_position():

@@ -2,6 +2,7 @@
 the gated merge on the 128-dim stream and the stored layout the indexer reads."""
 
 import numpy as np
+import pytest
 
 import oracle
 from synth import inputs as synth
@@ -74,6 +75,18 @@ def test_key_merge_with_uniform_gates_is_the_block_mean():
     want5 = (a[:, 20:24].sum(axis=1) + b[:, 16:20].sum(axis=1)) / 8
     np.testing.assert_allclose(y[:, 0], want0, rtol=1e-13, atol=1e-13)
     np.testing.assert_allclose(y[:, 5], want5, rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("m,pos0", [(4, 0), (4, 512), (2, 8)])
+def test_key_merge_matches_library_softmax(m, pos0):
+    # random gates and bias: every candidate slot keeps its own bias term
+    inp = synth.compress_inputs(2, 16 * m, m, True, seed=21 + m + pos0, dim=128, pos0=pos0)
+    Nmax = (pos0 // m + 16 + 127) // 128 * 128
+    _, _, y = oracle.compress_index_keys(inp["a"], inp["za"], inp["bias"], m, True, Nmax,
+                                         b=inp["b"], zb=inp["zb"], pos0=pos0,
+                                         prev_b=inp.get("prev_b"), prev_zb=inp.get("prev_zb"))
+    np.testing.assert_allclose(y, indep.gated_merge(inp, m, True, pos0), rtol=1e-12,
+                               atol=1e-12)
 
 
 def test_stored_keys_are_the_mxfp4_of_the_merge_in_the_indexer_layout():
