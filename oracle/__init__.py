@@ -306,8 +306,9 @@ def swa_row(a_row, t: int, rope_base: float = 10000.0, eps: float = 1e-6,
 
 def prefill(inp: dict, k: int, q_rows, tau: float | None = None, rope_base: float = 10000.0,
             eps: float = 1e-6, derotate: bool = True, nthreads: int = 0) -> dict:
-    """Evaluate the rows `q_rows` of a prefill described by a synth.prefill_inputs dict.
-    Returns out [nq][H][512], lse [nq][H], idx [nq][k] and the cache after compression."""
+    """Evaluate the rows `q_rows` of a prefill described by a synth.prefill_inputs dict
+    (with an optional RMSNorm weight under "norm_w"). Returns out [nq][H][512], lse [nq][H],
+    idx [nq][k] and the cache after compression."""
     P, T, m, H, H_I, Nmax = (inp[x] for x in ("P", "T", "m", "H", "H_I", "Nmax"))
     tau = 1.0 / np.sqrt(512.0) if tau is None else tau
     kv = np.array(inp["kv"], dtype=np.uint8, copy=True)
@@ -320,11 +321,11 @@ def prefill(inp: dict, k: int, q_rows, tau: float | None = None, rope_base: floa
         ("bias", np.float32), ("prev_b", np.uint16), ("prev_zb", np.float32),
         ("q_fp4", np.uint8), ("q_sf", np.uint8), ("w", np.float32), ("k_fp4", np.uint8),
         ("k_sf", np.uint8), ("q", np.uint16), ("sink", np.float32),
-        ("swa_prefix", np.uint16))}
+        ("swa_prefix", np.uint16), ("norm_w", np.float32))}
     U16, F32, U8 = C.c_uint16, C.c_float, C.c_uint8
     rc = lib().or_prefill(P, T, m, H, H_I, k, rope_base, eps, tau, int(derotate),
                           _p(g["a"], U16), _p(g["b"], U16), _p(g["za"], F32),
-                          _p(g["zb"], F32), _p(g["bias"], F32), None,
+                          _p(g["zb"], F32), _p(g["bias"], F32), _p(g["norm_w"], F32),
                           _p(g["prev_b"], U16), _p(g["prev_zb"], F32), _p(kv, U8),
                           _p(sc, F32), Nmax, _p(g["q_fp4"], U8), _p(g["q_sf"], U8),
                           _p(g["w"], F32), _p(g["k_fp4"], U8), _p(g["k_sf"], U8),

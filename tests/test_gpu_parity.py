@@ -33,7 +33,7 @@ def _gpu():
 
 
 # ------------------------------------------------------------------ compress
-def _run_compress(inp, m, overlap, pos0=0, Nmax=None):
+def _run_compress(inp, m, overlap, pos0=0, Nmax=None, norm_w=None):
     B, T, _ = inp["a"].shape
     N = T // m
     Nmax = Nmax or pos0 // m + N
@@ -42,7 +42,8 @@ def _run_compress(inp, m, overlap, pos0=0, Nmax=None):
                                zb=dev(inp["zb"]) if overlap else None, pos0=pos0,
                                prev_b=dev(inp["prev_b"]) if "prev_b" in inp else None,
                                prev_zb=dev(inp["prev_zb"]) if "prev_zb" in inp else None,
-                               Nmax=Nmax, dbg=True)
+                               Nmax=Nmax, dbg=True,
+                               norm_w=dev(norm_w) if norm_w is not None else None)
     torch.cuda.synchronize()
     n0 = pos0 // m
     return host(kv)[:, n0:n0 + N], host(sc)[:, n0:n0 + N], host(dbg)
@@ -62,6 +63,17 @@ def test_compress_matches_oracle(B, T, m, overlap, pos0):
                           zb=inp.get("zb"), pos0=pos0, prev_b=inp.get("prev_b"),
                           prev_zb=inp.get("prev_zb"))
     flips = compare.compare_entries(kv, sc, dbg, ora, what=f"compress m={m}")
+    assert flips <= max(4, kv.size // 5000)
+
+
+def test_compress_with_rmsnorm_weight():
+    # the optional RMSNorm weight (dims scaled after the norm, before RoPE)
+    inp = synth.compress_inputs(2, 4 * 40, 4, True, seed=131, pos0=256)
+    w = np.random.default_rng(131).uniform(0.5, 2.0, 512).astype(np.float32)
+    kv, sc, dbg = _run_compress(inp, 4, True, 256, norm_w=w)
+    ora = oracle.compress(inp["a"], inp["za"], inp["bias"], 4, True, b=inp["b"], zb=inp["zb"],
+                          pos0=256, prev_b=inp["prev_b"], prev_zb=inp["prev_zb"], norm_w=w)
+    flips = compare.compare_entries(kv, sc, dbg, ora, what="compress with norm weight")
     assert flips <= max(4, kv.size // 5000)
 
 

@@ -33,7 +33,7 @@ def _gpu():
 
 def run_prefill(inp, k, derotate=True):
     kv, sc = dev(inp["kv"]), dev(inp["kv_scale"])
-    opt = {x: dev(inp[x]) for x in ("prev_b", "prev_zb") if x in inp}
+    opt = {x: dev(inp[x]) for x in ("prev_b", "prev_zb", "norm_w") if x in inp}
     if inp["P"] > 0:
         opt["swa_prefix"] = dev(inp["swa_prefix"])
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -83,6 +83,17 @@ def test_prefill_small_all_rows(P, T, H, H_I, k):
     ora = oracle.prefill(inp, k, rows)
     check_cache(inp, got, ora)
     check_rows(inp, k, got, rows, ora)
+
+
+def test_prefill_with_rmsnorm_weight():
+    # the optional RMSNorm weight reaches the new entries and the new window rows
+    inp = synth.prefill_inputs(512, 200, 4, 64, 16, seed=23)
+    inp["norm_w"] = np.random.default_rng(23).uniform(0.5, 2.0, 512).astype(np.float32)
+    got = run_prefill(inp, 64)
+    rows = np.array([0, 1, 2, 3, 100, 127, 128, 199], np.int32)
+    ora = oracle.prefill(inp, 64, rows)
+    check_cache(inp, got, ora)
+    check_rows(inp, 64, got, rows, ora)
 
 
 def test_prefill_from_empty_prefix_over_two_query_chunks():

@@ -24,10 +24,14 @@ def _gpu():
     csa.lib()
 
 
-def test_token_by_token_appends_equal_whole_stream_compression():
+@pytest.mark.parametrize("weighted", [False, True])
+def test_token_by_token_appends_equal_whole_stream_compression(weighted):
     B, S, m = 2, 4 * 37 + 2, 4  # 37 closed blocks, two tokens left in the tail
     kvs = synth.compress_inputs(B, S, m, True, seed=61)
     iks = synth.compress_inputs(B, S, m, True, seed=62, dim=128)
+    # the optional RMSNorm weight of the entries and window rows
+    w = np.random.default_rng(61).uniform(0.5, 2.0, 512).astype(np.float32) if weighted else None
+    w_dev = dev(w) if weighted else None
     Nmax = 128
     st = csa.new_decode_state(B, Nmax, m)
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -39,13 +43,13 @@ def test_token_by_token_appends_equal_whole_stream_compression():
                           st, b=d["b"][:, t].contiguous(), zb=d["zb"][:, t].contiguous(), m=m,
                           ia=di["a"][:, t].contiguous(), ib=di["b"][:, t].contiguous(),
                           iza=di["za"][:, t].contiguous(), izb=di["zb"][:, t].contiguous(),
-                          ibias=di["bias"], dev_status=status)
+                          ibias=di["bias"], norm_w=w_dev, dev_status=status)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     assert (st["n_entries"].cpu().numpy() == S // m).all()
     # the same entries and keys as the whole-stream calls (the same block arithmetic)
     kv, sc, _ = csa.compress(d["a"], d["za"], d["bias"], m, True, b=d["b"], zb=d["zb"],
-                             Nmax=Nmax)
+                             Nmax=Nmax, norm_w=w_dev)
     kf, ks, _ = csa.compress_index_keys(di["a"], di["za"], di["bias"], m, True, b=di["b"],
                                         zb=di["zb"], Nmax=Nmax)
     torch.cuda.synchronize()
@@ -57,7 +61,7 @@ def test_token_by_token_appends_equal_whole_stream_compression():
     ring = st["swa"].cpu().numpy().view(np.uint16)
     for bb in range(B):
         for p in (S - 128, S - 57, S - 1):
-            want = oracle.swa_row(kvs["a"][bb, p], p)
+            want = oracle.swa_row(kvs["a"][bb, p], p, norm_w=w)
             got = ring[bb, p % 128]
             wf = want.astype(np.uint32) << 16
             gf = got.astype(np.uint32) << 16

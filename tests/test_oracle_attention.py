@@ -155,15 +155,21 @@ def test_bad_index_is_rejected():
 
 
 # ----------------------------------------------------------------- prefill
-def test_prefill_row_matches_independent_recomputation():
+@pytest.mark.parametrize("weighted", [False, True])
+def test_prefill_row_matches_independent_recomputation(weighted):
     P, T, m, H, H_I, k = 512, 64, 4, 2, 4, 40
     inp = synth.prefill_inputs(P, T, m, H, H_I, seed=10)
+    norm_w = None
+    if weighted:  # the optional RMSNorm weight reaches the entries and the window rows
+        norm_w = np.random.default_rng(10).uniform(0.5, 2.0, 512).astype(np.float32)
+        inp["norm_w"] = norm_w
     rows = [0, 1, 3, 4, 31, 63]
     r = oracle.prefill(inp, k, rows)
     # the new entries match a stand-alone compression of the new tokens
     comp = oracle.compress(inp["a"][None], inp["za"][None], inp["bias"], m, True,
                            b=inp["b"][None], zb=inp["zb"][None], pos0=P,
-                           prev_b=inp["prev_b"][None], prev_zb=inp["prev_zb"][None])
+                           prev_b=inp["prev_b"][None], prev_zb=inp["prev_zb"][None],
+                           norm_w=norm_w)
     n0 = P // m
     np.testing.assert_array_equal(r["kv"][n0:n0 + T // m], comp["kv"][0])
     np.testing.assert_array_equal(r["kv"][:n0], inp["kv"][:n0])
@@ -186,7 +192,8 @@ def test_prefill_row_matches_independent_recomputation():
             if p < P:
                 win.append(indep.bf16_to_f64(inp["swa_prefix"][p % 128]))
             else:
-                win.append(indep.bf16_to_f64(oracle.swa_row(inp["a"][p - P], p)))
+                win.append(indep.bf16_to_f64(oracle.swa_row(inp["a"][p - P], p,
+                                                            norm_w=norm_w)))
         V = np.concatenate([ent, np.array(win)])
         qh = indep.bf16_to_f64(inp["q"][row])
         full = np.concatenate([inp["sink"].astype(np.float64)[:, None], TAU * qh @ V.T], 1)
