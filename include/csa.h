@@ -340,8 +340,10 @@ int hca_attn_decode(const csa_attn_args* args, void* workspace, size_t workspace
  * kv_scale [Nmax]; q_fp4 [T][H_I][64]; q_sf [T][H_I][4]; w [T][H_I]; k_fp4 [Nmax][64];
  * k_sf [Nmax/128][512] (grouped as in csa_indexer_topk); q bf16 [T][H][512];
  * swa_prefix bf16 [128][512] (needed when P > 0); out bf16 [T][H][512]; lse [T][H];
- * idx [T][k]. m in 1..128, P % m == 0, Nmax a multiple of 128 with (P+T)/m <= Nmax,
- * H in {64, 128}, H_I in {16, 32, 64}, 1 <= k <= 2048.
+ * idx [T][k]. m in 1..128, P % m == 0, Nmax a positive multiple of 128 with
+ * (P+T)/m <= Nmax (the key array is read in 128-entry tiles, so it holds at least one
+ * tile even when no block is complete), H in {64, 128}, H_I in {16, 32, 64},
+ * 1 <= k <= 2048.
  * The workspace (csa_prefill_workspace_size) must be zero-filled once before its first
  * use; every call leaves the parts that must start at zero zeroed again.
  */
@@ -352,7 +354,7 @@ typedef struct {
   int32_t H;                  /* query heads: 64 or 128 */
   int32_t H_I;                /* indexer heads: 16, 32 or 64 */
   int32_t k;                  /* top-k */
-  int64_t Nmax;               /* entry capacity, multiple of 128 */
+  int64_t Nmax;               /* entry capacity, positive multiple of 128 */
   float tau;                  /* softmax scale; 0 selects 1/sqrt(512) */
   float rope_base;            /* 10000 */
   float eps;                  /* RMSNorm epsilon */

@@ -401,7 +401,7 @@ size_t csa_prefill_workspace_size(int32_t T, int64_t Nmax, int32_t H, int32_t k)
 
 int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream_t stream_) {
   if (!a) return CSA_ERR_INVALID_ARG;
-  if (a->P < 0 || a->T < 0 || a->m < 1 || a->m > 128 || a->P % a->m || a->Nmax < 0 ||
+  if (a->P < 0 || a->T < 0 || a->m < 1 || a->m > 128 || a->P % a->m || a->Nmax < 128 ||
       a->Nmax % 128 || (a->P + a->T) / a->m > a->Nmax || !(a->eps >= 0.f) ||
       !(a->rope_base > 0.f) || !(a->tau >= 0.f) || (a->derotate != 0 && a->derotate != 1) ||
       a->k < 1)

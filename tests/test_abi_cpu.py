@@ -139,6 +139,8 @@ def test_prefill_rejects_on_host(L):
     assert f(_prefill_args(P=4094)) == csa.CSA_ERR_INVALID_ARG   # not a block boundary
     assert f(_prefill_args(Nmax=1100)) == csa.CSA_ERR_INVALID_ARG  # not a multiple of 128
     assert f(_prefill_args(Nmax=1024)) == csa.CSA_ERR_INVALID_ARG  # 1099 entries do not fit
+    # no capacity at all, even with no complete block: rejected before any launch
+    assert f(_prefill_args(P=0, T=3, Nmax=0)) == csa.CSA_ERR_INVALID_ARG
     assert f(_prefill_args(k=0)) == csa.CSA_ERR_INVALID_ARG
     assert f(_prefill_args(H=96)) == csa.CSA_ERR_UNSUPPORTED
     assert f(_prefill_args(H_I=8)) == csa.CSA_ERR_UNSUPPORTED
