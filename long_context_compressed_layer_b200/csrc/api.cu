@@ -427,6 +427,8 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   PrefillWs w;
   prefill_ws_layout(a->T, a->Nmax, a->H, a->k, reinterpret_cast<char*>(ws), &w);
+  CUtensorMap kmap;  // encoded before the first launch, so a refusal leaves no partial work
+  if (!encode_key_map(enc, &kmap, a->k_fp4, a->Nmax, 1)) return CSA_ERR_CUDA;
 
   // 1. the new blocks' entries
   csa_compress_args c;
@@ -459,8 +461,6 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
   e = launch_prefill_rows16(a->kv, a->kv_scale, (a->P + a->T) / a->m, w.rows16, stream);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   // 3. per chunk of queries: indexer top-k over the shared keys, then attention
-  CUtensorMap kmap;
-  if (!encode_key_map(enc, &kmap, a->k_fp4, a->Nmax, 1)) return CSA_ERR_CUDA;
   for (int c0 = 0; c0 < a->T; c0 += kPrefillChunk) {
     const int nq = a->T - c0 < kPrefillChunk ? a->T - c0 : kPrefillChunk;
     int32_t* idx = a->idx ? a->idx + (size_t)c0 * a->k : w.idx;
