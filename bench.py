@@ -38,6 +38,10 @@ WORKLOAD_ID = 3
 METRIC = "CSA decode queries/s at 1M ctx; achieved HBM GB/s as % of B200 peak"
 UNIT = "queries/s"
 COPIES = 4
+# nominal B200 figures, reported beside the measured peaks: HBM3e bandwidth (HGX) and dense
+# BF16 tensor throughput
+NOMINAL_HBM_GBS = 7700.0
+NOMINAL_BF16_TFLOPS = 2250.0
 
 
 def algorithmic_bytes(d: dict) -> tuple[int, int]:
@@ -332,6 +336,8 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
         "roofline": {"bound": "tensor", "kernel": "csa_prefill (whole call)",
                      "achieved": eq_tflops, "peak": bf16_peak, "unit": "TFLOP/s",
                      "frac": eq_tflops / bf16_peak,
+                     "nominal_peak": NOMINAL_BF16_TFLOPS,
+                     "frac_of_nominal": eq_tflops / NOMINAL_BF16_TFLOPS,
                      "peak_src": ("measured sustained bf16; FP4 FLOPs weighted 1/4 (nominal ratio)"
                                   if "bf16_tflops_sustained" in pk else "fallback"),
                      "traffic": None},
@@ -599,6 +605,8 @@ def main():
             "roofline": {"bound": "hbm", "kernel": "csa_indexer_topk (score + select)",
                          "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "peak_src": pk["src"],
+                         "nominal_peak": NOMINAL_HBM_GBS,
+                         "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
                          "algorithmic_bytes_per_launch": idx_bytes,
                          "traffic": traffic["dram_bytes_per_launch"] if traffic else None},
             "clocks": clocks,
