@@ -346,7 +346,51 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
                 "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
     }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = prefill_cpu_baseline(d, w)
     print(json.dumps(line), flush=True)
+
+
+def prefill_cpu_baseline(d: dict, w, nrows: int = 128) -> dict:
+    """The oracle timed on a bounded sample of one prefill (inputs as drawn on the device,
+    copied to the host): its compression of every new block, then `nrows` query rows (the
+    first tokens, the edges of the 1024-query chunks, the last token and seeded random
+    ones). Tokens/s is extrapolated from the two times: T / (t_compress + T * t_row)."""
+    import torch
+
+    import oracle
+
+    T = d["T"]
+    fixed = [r for r in (0, 1, 2, 3, 1023, 1024, T - 1) if r < T]
+    rng = np.random.default_rng(w.seed)
+    extra = rng.choice(T, min(T, max(0, nrows - len(fixed))), replace=False)
+    rows = np.unique(np.concatenate([fixed, extra]).astype(np.int32))[:nrows]
+
+    def host(x):
+        x = x.cpu().numpy()
+        return x.view(np.uint16) if x.dtype == np.int16 else x
+
+    inp = {key: d[key] for key in ("P", "T", "m", "H", "H_I", "Nmax")}
+    for key in ("kv", "kv_scale", "k_fp4", "k_sf", "q_fp4", "q_sf", "w", "sink", "swa_prefix",
+                "a", "b", "za", "zb", "bias", "prev_b", "prev_zb"):
+        if key in d:
+            inp[key] = host(d[key])
+    q = np.zeros(tuple(d["q"].shape), dtype=np.uint16)  # only the sampled rows are read
+    q[rows] = host(d["q"].index_select(0, torch.as_tensor(rows, dtype=torch.long,
+                                                          device=d["q"].device)))
+    inp["q"] = q
+    t0 = time.perf_counter()
+    oracle.prefill(inp, w.k, np.zeros(0, np.int32))
+    t1 = time.perf_counter()
+    oracle.prefill(inp, w.k, rows)
+    t2 = time.perf_counter()
+    t_comp = t1 - t0
+    t_row = max(0.0, (t2 - t1) - t_comp) / len(rows)
+    return {"value": T / (t_comp + T * t_row), "unit": "tokens/s", "cores": os.cpu_count() or 1,
+            "kind": "oracle",
+            "sample": f"compression of all {T // d['m']} new blocks ({t_comp:.1f} s) and "
+                      f"{len(rows)} query rows ({t2 - t1 - t_comp:.1f} s), fp64, all host "
+                      "threads; tokens/s extrapolated per query row"}
 
 
 def run_reference(args, rank: int) -> None:

@@ -56,3 +56,17 @@ def test_reference_arm_runs_on_rank_zero_only():
                         "--steps", "1", "--warmup", "0"], env=env, capture_output=True,
                        text=True, timeout=120)
     assert r.returncode == 0 and r.stdout.strip() == ""
+
+
+def test_prefill_cpu_baseline_on_a_small_host_bundle():
+    # the prefill line's oracle leg, on inputs drawn by the device generator on the CPU
+    from types import SimpleNamespace
+
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth import inputs as synth
+
+    d = synth.prefill_inputs_device(512, 300, 4, 64, 16, seed=3, device="cpu")
+    r = bench.prefill_cpu_baseline(d, SimpleNamespace(k=64, seed=3), nrows=12)
+    assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0
+    assert r["cores"] >= 1 and "12 query rows" in r["sample"]
