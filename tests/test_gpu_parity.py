@@ -364,6 +364,8 @@ def _ora_attn(d, derotate=True):
     (2, 128, 4096, [4096, 3000], [16383, 12001], 1024),  # CSA, workload 3 heads
     (3, 64, 1024, [1024, 7, 0], [131071, 900, 50], None),  # HCA, ragged, early positions
     (1, 128, 256, [200], [803], 100),                     # CSA, k not a multiple of 64
+    (1, 128, 4096, [4096], [16383], 2048),                # CSA at the largest k
+    (1, 64, 8192, [8192], [1048575], None),               # HCA over a 1M-token context
 ])
 def test_attention_matches_oracle(B, H, Nmax, n, pos, k):
     d = _attn_case(B, H, Nmax, n, pos, k, seed=H + B)
