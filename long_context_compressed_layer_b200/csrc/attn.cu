@@ -797,15 +797,10 @@ cudaError_t launch_prefill_attn(const csa_attn_args& a, const __half* rows16, in
   p.lse = a.lse;
   p.dev_status = a.dev_status;
   const size_t smem = sizeof(PaSmem) + 1024;
-  static int configured = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured != dev) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_attn_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = dev;
-  }
+  static std::atomic<uint64_t> configured{0};
+  if (cudaError_t e = configure_smem_once(prefill_attn_kernel, smem, configured);
+      e != cudaSuccess)
+    return e;
   return launch_pdl(prefill_attn_kernel, dim3(2 * a.B), dim3(kPaThreads), smem, stream, qmap, p);
 }
 
@@ -843,15 +838,10 @@ cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* 
   p.part_ml = reinterpret_cast<float2*>(reinterpret_cast<char*>(workspace) + ((o + 255) & ~(size_t)255));
   p.dev_status = a.dev_status;
   const size_t smem = at_smem_bytes();
-  static int configured = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured != dev) {
-    cudaError_t e = cudaFuncSetAttribute(attn_chunk_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = dev;
-  }
+  static std::atomic<uint64_t> configured{0};
+  if (cudaError_t e = configure_smem_once(attn_chunk_kernel, smem, configured);
+      e != cudaSuccess)
+    return e;
   cudaError_t e = launch_pdl(attn_chunk_kernel, dim3(p.C, a.B), dim3(kAtThreads), smem, stream,
                              qmap, p);
   if (e != cudaSuccess) return e;

@@ -130,15 +130,10 @@ cudaError_t launch_gemm_bf16(const CUtensorMap& amap, const CUtensorMap& bmap, i
                              cudaStream_t stream) {
   GmParams p{M, K, a_x_group, b_y_group, c_x_group, C, ldc, dev_status};
   const size_t smem = sizeof(GmSmem) + 1024;
-  static int configured = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured != dev) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = dev;
-  }
+  static std::atomic<uint64_t> configured{0};
+  if (cudaError_t e = configure_smem_once(gemm_bf16_kernel, smem, configured);
+      e != cudaSuccess)
+    return e;
   dim3 grid((M + kGmTile - 1) / kGmTile, N / kGmTile, G);
   return launch_pdl(gemm_bf16_kernel, grid, dim3(kGmThreads), smem, stream, amap, bmap, p);
 }

@@ -1333,19 +1333,11 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
   IxParams p{a.B, a.H_I, a.k, 1, bf16, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
              a.idx, a.scores, a.dev_status};
   const size_t smem = sizeof(IxSmem) + 1024;
-  static int configured = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured != dev) {
-    cudaError_t e = cudaFuncSetAttribute(indexer_score_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    // the whole carveout as shared memory, so two CTAs fit on an SM
-    e = cudaFuncSetAttribute(indexer_score_kernel,
-                             cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    configured = dev;
-  }
+  // the whole carveout as shared memory, so two CTAs fit on an SM
+  static std::atomic<uint64_t> configured{0};
+  if (cudaError_t e = configure_smem_once(indexer_score_kernel, smem, configured, 100);
+      e != cudaSuccess)
+    return e;
   // Scoring and selection in one cooperative launch (every CTA resident, so the grid
   // barrier between the phases always completes); the runtime refuses a grid that cannot
   // be resident, and the selection then runs as two further kernels.
@@ -1385,15 +1377,10 @@ cudaError_t launch_prefill_indexer_topk(const csa_topk_args& a, void* workspace,
   IxParams p{a.B, a.H_I, a.k, 0, 0, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
              a.idx, a.scores, a.dev_status};
   const size_t smem = sizeof(PxSmem) + 1024;
-  static int configured = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured != dev) {
-    cudaError_t e = cudaFuncSetAttribute(prefill_score_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = dev;
-  }
+  static std::atomic<uint64_t> configured{0};
+  if (cudaError_t e = configure_smem_once(prefill_score_kernel, smem, configured);
+      e != cudaSuccess)
+    return e;
   cudaError_t e = launch_pdl(prefill_score_kernel, dim3(num_sms), dim3(kPxThreads), smem,
                              stream, kmap, p);
   if (e != cudaSuccess) return e;

@@ -144,15 +144,10 @@ cudaError_t launch_iquery(const csa_iquery_args& a, const CUtensorMap& cmap,
                           const CUtensorMap& wmap, cudaStream_t stream) {
   IqParams p{a.T, a.r, a.H_I, a.q_fp4, a.q_sf, a.dbg, a.dev_status};
   const size_t smem = sizeof(IqSmem) + 1024;
-  static int configured = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (configured != dev) {
-    cudaError_t e = cudaFuncSetAttribute(iquery_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    configured = dev;
-  }
+  static std::atomic<uint64_t> configured{0};
+  if (cudaError_t e = configure_smem_once(iquery_kernel, smem, configured);
+      e != cudaSuccess)
+    return e;
   dim3 grid((a.T + kIqTile - 1) / kIqTile, a.H_I);
   return launch_pdl(iquery_kernel, grid, dim3(kIqThreads), smem, stream, cmap, wmap, p);
 }
