@@ -78,3 +78,24 @@ def test_offsets_and_sizes_match_the_c_compiler(tmp_path):
             assert (d.offset, d.size) == (int(off), int(size)), f"{name}.{field}"
         seen += 1
     assert seen == sum(len(c._fields_) + 1 for c in BINDING.values())
+
+
+def test_every_entry_point_has_a_signature_of_the_declared_arity():
+    # ctypes passes whatever it is given when argtypes is unset and assumes an int result;
+    # every entry point the header declares gets its declared result type and as many
+    # argtypes as the declaration has parameters
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = re.findall(r"^\s*((?:const\s+)?[A-Za-z_][\w\s\*]*?)\b(\w+)\s*\(([^;{]*)\)\s*;",
+                       text, flags=re.M)
+    if not os.path.exists(csa.LIB_PATH):
+        pytest.skip("library not built")
+    L = csa.lib()
+    results = {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "const char*": ctypes.c_char_p}
+    assert decls
+    for ret, name, params in decls:
+        ret = re.sub(r"\s*\*", "*", " ".join(ret.split()))
+        params = params.strip()
+        arity = 0 if params in ("", "void") else params.count(",") + 1
+        fn = getattr(L, name)
+        assert fn.argtypes is not None and len(fn.argtypes) == arity, name
+        assert fn.restype is results[ret], (name, ret)
