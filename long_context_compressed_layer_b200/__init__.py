@@ -163,6 +163,20 @@ def _ptr(t: torch.Tensor | None, *, elem: int | None = None, name: str = "") -> 
     return t.data_ptr()
 
 
+def _sizes(**named) -> None:
+    """Each named (tensor, n): a given tensor must hold at least n elements, the count its
+    layout needs; a shorter buffer would let a kernel read or write past its end."""
+    for name, (t, n) in named.items():
+        if t is not None and t.numel() < n:
+            raise ValueError(f"{name}: expected at least {n} elements, got {t.numel()} "
+                             f"(shape {tuple(t.shape)})")
+
+
+def _dim(t, axis: int, n: int, name: str) -> None:
+    if t.shape[axis] != n:
+        raise ValueError(f"{name}: dimension {axis} must be {n}, got shape {tuple(t.shape)}")
+
+
 def _stream(stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -178,9 +192,15 @@ def compress(a, za, bias, m: int, overlap: bool, *, b=None, zb=None, pos0: int =
     Returns (kv [B][Nmax][576] uint8, kv_scale [B][Nmax] float32, dbg [B][N][512] or None);
     kv/kv_scale are written in place when given."""
     B, T, _ = a.shape
+    _dim(a, 2, HEAD_DIM, "a")
     N = T // m
     if Nmax is None:
         Nmax = kv.shape[1] if kv is not None else pos0 // m + N
+    tok = B * T * HEAD_DIM
+    _sizes(za=(za, tok), b=(b, tok), zb=(zb, tok), bias=(bias, 2 * m if overlap else m),
+           norm_w=(norm_w, HEAD_DIM), prev_b=(prev_b, B * m * HEAD_DIM),
+           prev_zb=(prev_zb, B * m * HEAD_DIM), kv=(kv, B * Nmax * ROW_BYTES),
+           kv_scale=(kv_scale, B * Nmax))
     dev = a.device
     if kv is None:
         kv = torch.zeros((B, Nmax, ROW_BYTES), dtype=torch.uint8, device=dev)
@@ -223,6 +243,23 @@ def decode_append(pos, a, za, bias, state, *, b=None, zb=None, m: int = 4, overl
     """Append one token per sequence (a, b bf16 [B][512]; za, zb [B][512]; ia.. [B][128]) at
     positions pos [B] to a state from new_decode_state."""
     B = a.shape[0]
+    _dim(a, -1, HEAD_DIM, "a")
+    Nmax = state["kv"].shape[1]
+    row, irow = B * HEAD_DIM, B * INDEX_DIM
+    _sizes(pos=(pos, B), za=(za, row), b=(b, row), zb=(zb, row),
+           bias=(bias, 2 * m if overlap else m), norm_w=(norm_w, HEAD_DIM), ia=(ia, irow),
+           ib=(ib, irow), iza=(iza, irow), izb=(izb, irow), ibias=(ibias, 2 * m),
+           tail_a=(state["tail_a"], B * m * HEAD_DIM), tail_za=(state["tail_za"], B * m * HEAD_DIM),
+           tail_b=(state.get("tail_b"), 2 * B * m * HEAD_DIM),
+           tail_zb=(state.get("tail_zb"), 2 * B * m * HEAD_DIM),
+           swa=(state["swa"], B * WINDOW * HEAD_DIM), kv=(state["kv"], B * Nmax * ROW_BYTES),
+           kv_scale=(state["kv_scale"], B * Nmax), n_entries=(state["n_entries"], B))
+    if ia is not None:
+        _sizes(itail_a=(state["itail_a"], B * m * INDEX_DIM),
+               itail_za=(state["itail_za"], B * m * INDEX_DIM),
+               itail_b=(state["itail_b"], 2 * B * m * INDEX_DIM),
+               itail_zb=(state["itail_zb"], 2 * B * m * INDEX_DIM),
+               k_fp4=(state["k_fp4"], B * Nmax * 64), k_sf=(state["k_sf"], B * Nmax // 128 * 512))
     g = lambda k_, el: _ptr(state.get(k_), elem=el, name=k_)
     args = AppendArgs(B, m, int(overlap), rope_base, eps, _ptr(pos, elem=4, name="pos"),
                       _ptr(a, elem=2, name="a"), _ptr(b, elem=2, name="b"),
@@ -250,9 +287,14 @@ def compress_index_keys(a, za, bias, m: int, overlap: bool, *, b=None, zb=None, 
     Returns (k_fp4 [B][Nmax][64], k_sf [B][Nmax/128*512], dbg [B][N][128] or None);
     k_fp4 / k_sf are written in place when given."""
     B, T, _ = a.shape
+    _dim(a, 2, INDEX_DIM, "a")
     N = T // m
     if Nmax is None:
         Nmax = k_fp4.shape[1] if k_fp4 is not None else -(-(pos0 // m + N) // 128) * 128
+    tok = B * T * INDEX_DIM
+    _sizes(za=(za, tok), b=(b, tok), zb=(zb, tok), bias=(bias, 2 * m if overlap else m),
+           prev_b=(prev_b, B * m * INDEX_DIM), prev_zb=(prev_zb, B * m * INDEX_DIM),
+           k_fp4=(k_fp4, B * Nmax * 64), k_sf=(k_sf, B * Nmax // 128 * 512))
     dev = a.device
     if k_fp4 is None:
         k_fp4 = torch.zeros((B, Nmax, 64), dtype=torch.uint8, device=dev)
@@ -275,6 +317,7 @@ def indexer_query(c, W, H_I: int, *, q_fp4=None, q_sf=None, dbg: bool = False,
     """Indexer queries of T tokens: c bf16 [T][r], W bf16 [H_I * 128][r] -> (q_fp4
     [T][H_I][64], q_sf [T][H_I][4], dbg [T][H_I * 128] or None)."""
     T, r = c.shape
+    _sizes(W=(W, H_I * INDEX_DIM * r), q_fp4=(q_fp4, T * H_I * 64), q_sf=(q_sf, T * H_I * 4))
     dev = c.device
     if q_fp4 is None:
         q_fp4 = torch.empty((T, H_I, 64), dtype=torch.uint8, device=dev)
@@ -292,8 +335,11 @@ def grouped_out_proj(attn, Wg, Wo, *, workspace=None, out=None, dev_status=None,
     """attn bf16 [T][H][512], Wg bf16 [G][d_g][H/G*512], Wo bf16 [d_model][G*d_g] ->
     out bf16 [T][d_model]."""
     T, H, _ = attn.shape
+    _dim(attn, 2, HEAD_DIM, "attn")
     G, d_g, _ = Wg.shape
     d_model = Wo.shape[0]
+    _sizes(Wg=(Wg, G * d_g * (H // G) * HEAD_DIM), Wo=(Wo, d_model * G * d_g),
+           out=(out, T * d_model))
     dev = attn.device
     if workspace is None:
         n = lib().csa_grouped_out_proj_workspace_size(T, G, d_g)
@@ -320,7 +366,10 @@ def indexer_topk(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, k: int, *, workspace=No
     """Top-k entry indices [B][k] (ascending, -1 padded) and optionally their scores.
     bf16_scores selects on scores rounded to BF16 (csa_indexer_topk_bf16)."""
     B, H_I, _ = q_fp4.shape
+    _dim(q_fp4, 2, 64, "q_fp4")
     Nmax = k_fp4.shape[1]
+    _sizes(n_entries=(n_entries, B), q_sf=(q_sf, B * H_I * 4), w=(w, B * H_I),
+           k_fp4=(k_fp4, B * Nmax * 64), k_sf=(k_sf, B * Nmax // 128 * 512), idx=(idx, B * k))
     dev = q_fp4.device
     if workspace is None:
         workspace = indexer_topk_workspace(B, Nmax, k, dev)
@@ -348,8 +397,12 @@ def _attn(fn: str, sparse: bool, q, pos, n_entries, kv, kv_scale, swa, sink, idx
           tau: float = 0.0, rope_base: float = 10000.0, derotate: bool = True,
           workspace=None, out=None, lse: bool = False, dev_status=None, stream=None):
     B, H, _ = q.shape
+    _dim(q, 2, HEAD_DIM, "q")
     Nmax = kv.shape[1]
     k = idx.shape[1] if sparse else 0
+    _sizes(pos=(pos, B), n_entries=(n_entries, B), kv=(kv, B * Nmax * ROW_BYTES),
+           kv_scale=(kv_scale, B * Nmax), swa=(swa, B * WINDOW * HEAD_DIM), sink=(sink, H),
+           idx=(idx if sparse else None, B * k), out=(out, B * H * HEAD_DIM))
     dev = q.device
     noalloc = fn.endswith("_noalloc")
     if workspace is None and not noalloc:
@@ -411,6 +464,14 @@ def prefill(P: int, m: int, k: int, *, a, b, za, zb, bias, kv, kv_scale, q_fp4, 
     T = a.shape[0]
     H, H_I = q.shape[1], q_fp4.shape[1]
     Nmax = kv.shape[0]
+    tok = T * HEAD_DIM
+    _sizes(a=(a, tok), b=(b, tok), za=(za, tok), zb=(zb, tok), bias=(bias, 2 * m),
+           kv=(kv, Nmax * ROW_BYTES), kv_scale=(kv_scale, Nmax), q_fp4=(q_fp4, T * H_I * 64),
+           q_sf=(q_sf, T * H_I * 4), w=(w, T * H_I), k_fp4=(k_fp4, Nmax * 64),
+           k_sf=(k_sf, Nmax // 128 * 512), q=(q, T * H * HEAD_DIM), sink=(sink, H),
+           prev_b=(prev_b, m * HEAD_DIM), prev_zb=(prev_zb, m * HEAD_DIM),
+           swa_prefix=(swa_prefix, WINDOW * HEAD_DIM), norm_w=(norm_w, HEAD_DIM),
+           out=(out, T * H * HEAD_DIM))
     dev = q.device
     if workspace is None:
         workspace = prefill_workspace(T, Nmax, H, k, dev)
