@@ -158,6 +158,10 @@ def _ptr(t: torch.Tensor | None, *, elem: int | None = None, name: str = "") -> 
         return None
     if not t.is_cuda or not t.is_contiguous():
         raise ValueError(f"{name}: expected a contiguous CUDA tensor")
+    if t.device.index != torch.cuda.current_device():
+        # the kernels run on the current device and would dereference another GPU's memory
+        raise ValueError(f"{name}: on {t.device}, but the current device is "
+                         f"cuda:{torch.cuda.current_device()}")
     if elem is not None and t.element_size() != elem:
         raise ValueError(f"{name}: expected {elem}-byte elements, got {t.dtype}")
     return t.data_ptr()
