@@ -20,7 +20,7 @@
 //
 // Parity status: every function here is pinned by the CPU test suite against format
 // definitions, closed forms, invariants, textbook reductions or brute force; none is
-// "parity unpinned" against its own definition. The readings R1-R17 themselves are
+// "parity unpinned" against its own definition. The readings R1-R25 themselves are
 // not fixed by the pages and are pinned only to this statement.
 
 #include <algorithm>
