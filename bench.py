@@ -393,6 +393,157 @@ def prefill_cpu_baseline(d: dict, w, nrows: int = 128) -> dict:
                       "threads; tokens/s extrapolated per query row"}
 
 
+HCA_ID = 1
+HCA_METRIC = "HCA decode queries/s (8 sequences at 128K context, 1,024 entries each)"
+HCA_COPIES = 24  # 24 x 6.3 MB of streamed inputs: more than L2 across the rotation
+
+
+def hca_step_bytes(d: dict) -> int:
+    """Algorithmic bytes of one HCA decode step: per sequence every eligible row of 580 B
+    (576 B + fp32 scale), 128 window rows of 1 KB, Q and O (H x 1 KB each), the position
+    and length, and the H sink logits."""
+    H = d["workload"].H
+    n = d["n_entries"].astype(np.int64)
+    return int((n * 580).sum() + d["B"] * (128 * 1024 + 2 * H * 1024 + 8 + H * 4))
+
+
+def bench_hca(args, rank: int, world: int, local: int) -> None:
+    """The HCA decode (hca_attn_decode) of the 128K-context workload, replayed from CUDA
+    graphs over device copies of its inputs; roofline against the measured HBM copy rate."""
+    import torch
+
+    import long_context_compressed_layer_b200 as csa
+    from synth import inputs as synth
+
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    w = synth.WORKLOADS[HCA_ID]
+    d = synth.decode_inputs(w, seed=w.seed + 1000 * rank)
+    B, Nmax = d["B"], d["Nmax"]
+
+    def dev(x):
+        x = np.ascontiguousarray(x)
+        return torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).cuda()
+
+    streamed = ("kv", "kv_scale", "q", "swa")
+    base = {key: dev(d[key]) for key in streamed + ("n_entries", "pos", "sink")}
+    copies = [base] + [{key: (base[key].clone() if key in streamed else base[key])
+                        for key in base} for _ in range(HCA_COPIES - 1)]
+    ws = csa.attn_workspace(B, w.H, Nmax + 128)
+    out = torch.empty((B, w.H, 512), dtype=torch.bfloat16, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step(c):
+        csa.hca_attn_decode(c["q"], c["pos"], c["n_entries"], c["kv"], c["kv_scale"], c["swa"],
+                            c["sink"], workspace=ws, out=out, dev_status=status)
+
+    graph_steps = 8
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        s_cap = torch.cuda.Stream()
+        s_cap.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s_cap):
+            fn()  # warm the tensor-map / attribute caches outside the capture
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=s_cap):
+                for _ in range(graph_steps):
+                    fn()
+        torch.cuda.current_stream().wait_stream(s_cap)
+        torch.cuda.synchronize()
+        return g
+
+    def timed(graphs, n):
+        for i in range(max(3, len(graphs))):  # warm-up replays
+            graphs[i % len(graphs)].replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(n):
+            graphs[i % len(graphs)].replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return e0.elapsed_time(e1) / (n * graph_steps)
+
+    graphs = [capture(lambda c=c: step(c)) for c in copies]
+    replays = max(1, (args.steps + graph_steps - 1) // graph_steps)
+    sampler = ClockSampler(local)
+    sampler.start()
+    ms = timed(graphs, replays)
+    clocks = sampler.stop()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during the benchmark")
+
+    # end to end: the step's queries, positions and lengths go up from pinned host memory
+    # and the output comes back, inside the replayed graphs
+    q_inputs = ("q", "pos", "n_entries")
+    pinned = {key: base[key].cpu().pin_memory() for key in q_inputs}
+    dev_in = {key: torch.empty_like(base[key]) for key in q_inputs}
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def e2e_step(c):
+        for key in q_inputs:
+            dev_in[key].copy_(pinned[key], non_blocking=True)
+        step({**c, **dev_in})
+        out_h.copy_(out, non_blocking=True)
+
+    e2e_ms = timed([capture(lambda c=c: e2e_step(c)) for c in copies],
+                   max(4, min(replays, 256)))
+    ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, "cuda")
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    pk = peaks()
+    step_bytes = hca_step_bytes(d)
+    streamed_bytes = sum(base[key].numel() * base[key].element_size() for key in streamed)
+    achieved = step_bytes / (ms * 1e-3) / 1e9
+    line = {
+        "metric": HCA_METRIC, "value": whole_job_rate(B, world, ms), "unit": UNIT,
+        "n_gpus": world, "steps": replays * graph_steps, "warmup": max(3, HCA_COPIES) * graph_steps,
+        "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp16", "data": "synthetic",
+        "config": {"workload": w.name, "queries_per_step_per_gpu": B, "context": w.L,
+                   "entries_per_seq": int(d["n_entries"][0]), "heads": w.H, "window": 128,
+                   "l2": f"inputs rotated over {HCA_COPIES} device copies "
+                         f"({HCA_COPIES * streamed_bytes / 1e6:.0f} MB of streamed inputs)",
+                   "launch": f"CUDA graphs of {graph_steps} steps, programmatic dependent launch"},
+        "roofline": {"bound": "hbm", "kernel": "hca_attn_decode (chunk + combine kernels)",
+                     "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / pk["hbm_gbs"], "peak_src": pk["src"],
+                     "nominal_peak": NOMINAL_HBM_GBS,
+                     "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+                     "algorithmic_bytes_per_launch": step_bytes, "traffic": None},
+        "clocks": clocks,
+        "e2e": {"value": whole_job_rate(B, world, e2e_ms), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 2 * replays * graph_steps,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        import oracle
+
+        t0 = time.perf_counter()
+        oracle.attention(d["q"], d["pos"], d["n_entries"], d["kv"], d["kv_scale"], d["swa"],
+                         d["sink"])
+        dt = time.perf_counter() - t0
+        line["cpu_baseline"] = {"value": B / dt, "unit": UNIT, "cores": os.cpu_count() or 1,
+                                "kind": "oracle",
+                                "sample": f"one whole step ({B} queries), fp64, all host threads"}
+    print(json.dumps(line), flush=True)
+
+
 def run_reference(args, rank: int) -> None:
     """The fp64 CPU oracle, as it stands, on the host cores: each step is one decode query
     (one sequence of the workload: indexer over 262,144 entries, top-k, attention)."""
@@ -462,7 +613,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--copies", type=int, default=COPIES,
                     help="device copies of the streamed inputs rotated across steps")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "hca"])
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -473,6 +624,9 @@ def main():
         return
     if args.workload == "prefill":
         bench_prefill(args, rank, world, local)
+        return
+    if args.workload == "hca":
+        bench_hca(args, rank, world, local)
         return
 
     import torch

@@ -70,3 +70,14 @@ def test_prefill_cpu_baseline_on_a_small_host_bundle():
     r = bench.prefill_cpu_baseline(d, SimpleNamespace(k=64, seed=3), nrows=12)
     assert r["kind"] == "oracle" and r["unit"] == "tokens/s" and r["value"] > 0
     assert r["cores"] >= 1 and "12 query rows" in r["sample"]
+
+
+def test_hca_step_bytes_of_the_128k_workload():
+    # 8 sequences x (1,024 rows x 580 B + 128 window rows x 1 KB + Q and O of 64 heads x
+    # 1 KB + position and length + 64 sink logits)
+    sys.path.insert(0, ROOT)
+    import bench
+    from synth import inputs as synth
+
+    d = synth.decode_inputs(synth.WORKLOADS[bench.HCA_ID])
+    assert bench.hca_step_bytes(d) == 8 * (1024 * 580 + 128 * 1024 + 2 * 64 * 1024 + 8 + 256)
