@@ -345,6 +345,10 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
         "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s",
                 "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        # per call: compression of the new blocks, the window-row prep, the FP16 entry rows,
+        # then per 1024 queries the scoring, selection and attention kernels
+        "gpu_launches": args.steps * ((1 if T // w.m else 0) + 1 + (1 if (w.P + T) // w.m else 0)
+                                      + 3 * (-(-T // 1024))),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = prefill_cpu_baseline(d, w)
