@@ -1,0 +1,89 @@
+"""bench.py's host flow on the CPU, device objects faked (tests/fake_device.py): every mode
+runs to its JSON line, and the line carries every key of the benchmark contract. The
+numbers are meaningless here; a B200 run produces the real ones."""
+
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+RUN = """
+import sys
+sys.path.insert(0, {root!r})
+import tests.fake_device as fd
+fd.install()
+import bench
+from synth import inputs as synth
+bench.ClockSampler.start = lambda self: None
+bench.ClockSampler.stop = lambda self: {{"sm_mhz": None, "sm_max_mhz": None, "reasons": []}}
+if {small_prefill}:  # the 64K-token prefill's queries would need 8.6 GB of host memory
+    synth.WORKLOADS[4] = synth.Workload("small_prefill", "prefill", B=1, m=4, H=128, H_I=64,
+                                        k=1024, P=512, T=1100, seed=4)
+    import torch
+    real = synth.prefill_inputs_device
+    synth.prefill_inputs_device = lambda *a, device="cuda", **k: {{
+        key: v.to("meta") if isinstance(v, torch.Tensor) else v
+        for key, v in real(*a, device="cpu", **k).items()}}
+sys.argv = ["bench.py"] + {argv!r}
+bench.main()
+"""
+
+
+def _line(argv, small_prefill=False):
+    code = RUN.format(root=ROOT, argv=argv, small_prefill=small_prefill)
+    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout[-2000:]
+    return json.loads(lines[0])
+
+
+def _contract(d, cpu_baseline=True):
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+                "roofline", "clocks", "e2e", "gpu_launches"):
+        assert key in d, key
+    assert "workload" in d["config"]
+    for key in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
+        assert key in d["roofline"], key
+    for key in ("sm_mhz", "sm_max_mhz", "reasons"):
+        assert key in d["clocks"], key
+    for key in ("value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"):
+        assert key in d["e2e"], key
+    assert d["e2e"]["h2d_bytes_per_step"] > 0 and d["e2e"]["d2h_bytes_per_step"] > 0
+    assert d["gpu_launches"] > 0 and d["n_gpus"] == 1
+    if cpu_baseline:
+        for key in ("value", "unit", "cores", "kind", "sample"):
+            assert key in d["cpu_baseline"], key
+
+
+@pytest.mark.slow
+def test_default_decode_line():
+    d = _line(["--steps", "16", "--warmup", "3"])
+    _contract(d)
+    assert d["config"]["workload"] == "csa_decode_pro_1m" and d["roofline"]["bound"] == "hbm"
+    assert d["roofline"]["algorithmic_bytes_per_launch"] == 71338000
+
+
+def test_hca_line():
+    d = _line(["--workload", "hca", "--steps", "16", "--warmup", "3"])
+    _contract(d)
+    assert d["config"]["workload"] == "hca_decode_128k"
+
+
+def test_prefill_line():
+    d = _line(["--workload", "prefill", "--steps", "2", "--warmup", "3"], small_prefill=True)
+    _contract(d)
+    assert d["roofline"]["bound"] == "tensor"
+
+
+def test_reference_line():
+    d = _line(["--impl", "reference", "--steps", "1", "--warmup", "0"])
+    assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle"
+    assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
