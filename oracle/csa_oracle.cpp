@@ -15,13 +15,13 @@
 //                  sections "Hybrid Attention", "Partial RoPE", "Attention sink", "低精度路径"
 //
 // The pages give prose only: no formula, constant or worked example for the layer.
-// Every precise choice below that the prose leaves open is a numbered reading (R#);
-// the list of readings and their reasons lives with the design notes.
+// Every precise choice below that the prose leaves open is marked as a reading: the
+// plainest choice that the rest of the pages support, stated where it is made.
 //
 // Parity status: every function here is pinned by the CPU test suite against format
 // definitions, closed forms, invariants, textbook reductions or brute force; none is
-// "parity unpinned" against its own definition. The readings R1-R25 themselves are
-// not fixed by the pages and are pinned only to this statement.
+// "parity unpinned" against its own definition. The readings themselves are not fixed
+// by the pages and are pinned only to this statement.
 
 #include <algorithm>
 #include <cmath>
@@ -99,7 +99,7 @@ double or_e4m3_decode(uint8_t c) {
   return s ? -v : v;
 }
 
-// Round-to-nearest-even, saturating to +-448 (R7: the cache never stores NaN for
+// Round-to-nearest-even, saturating to +-448 (a reading: the cache never stores NaN for
 // finite inputs).
 uint8_t or_e4m3_encode(double x) {
   if (std::isnan(x)) return 0x7F;
@@ -172,19 +172,21 @@ size_t or_key_sf_offset(int64_t j, int s) {
 
 // ------------------------------------------------------------ compression
 // One call compresses the T tokens at absolute positions pos0 .. pos0+T-1 of each of
-// B sequences (pos0 a multiple of m) into N = floor(T/m) entries (R3: only complete
-// blocks are emitted), entry i covering tokens pos0+m*i .. pos0+m*i+m-1.
+// B sequences (pos0 a multiple of m) into N = floor(T/m) entries (a reading: only
+// complete blocks are emitted), entry i covering tokens pos0+m*i .. pos0+m*i+m-1.
 //
 // Gated merge [walkthrough §2.2: two independent KV sequences merged with
 // softmax-normalised gate weights, adjacent blocks overlap; chooseai 一: softmax with a
 // positional bias]: for every dim d the candidates are the m own-block tokens of `a`
 // with logits za + bias[r] and, when overlap = 1 (CSA), the m previous-block tokens of
-// `b` with logits zb + bias[m + r] (R1). The very first block of a sequence has no
-// previous block (R2); the first block of a later chunk takes it from prev_b/prev_zb.
-// Then RMSNorm (R4) [walkthrough §2.3: RMSNorm on the KV entries], RoPE on the last 64
-// dims at the entry's block-start position (R5, R6) [digest 2.: partial RoPE on the
-// last 64 dims], and the split store (R7): dims 0..447 as E4M3 of y/scale with
-// scale = amax/448, dims 448..511 as bf16 [chooseai 一: RoPE dims BF16, the rest FP8].
+// `b` with logits zb + bias[m + r] (the slot order is a reading). The very first block
+// of a sequence has no previous block (a reading); the first block of a later chunk
+// takes it from prev_b/prev_zb. Then RMSNorm (eps and the optional weight are readings)
+// [walkthrough §2.3: RMSNorm on the KV entries], RoPE on the last 64 dims at the entry's
+// block-start position (pairing, base and position are readings) [digest 2.: partial
+// RoPE on the last 64 dims], and the split store (its scale rule is a reading): dims
+// 0..447 as E4M3 of y/scale with scale = amax/448, dims 448..511 as bf16 [chooseai 一:
+// RoPE dims BF16, the rest FP8].
 //
 // Outputs (each nullable): e_out [B][N][512] merged entry before the norm,
 // y_out [B][N][512] final pre-quantisation value, kv [B][N][576], kv_scale [B][N].
@@ -269,13 +271,14 @@ int or_compress(int B, int T, int m, int overlap, int64_t pos0, double rope_base
   return 0;
 }
 
-// Indexer-key compression (R21-R23) [walkthrough §2.2: the lightning indexer scores the
-// compressed entries, so each entry needs an indexer key; §3.4: the indexer QK path is
-// FP4]: the 128-dim indexer-key stream of the T tokens at pos0 .. pos0+T-1 is merged with
-// the gated softmax of or_compress (same candidate slots and bias layout, R1-R3), with no
-// norm and no RoPE (R22), and each entry is stored as MXFP4 (R23): 64 bytes of E2M1
-// codes (element 2i in the low nibble of byte i) at row pos0/m + i of k_fp4 [B][Nmax][64]
-// and four E8M0 block scales at or_key_sf_offset(row, s) of k_sf [B][Nmax/128][512].
+// Indexer-key compression (readings throughout) [walkthrough §2.2: the lightning indexer
+// scores the compressed entries, so each entry needs an indexer key; §3.4: the indexer
+// QK path is FP4]: the 128-dim indexer-key stream of the T tokens at pos0 .. pos0+T-1 is
+// merged with the gated softmax of or_compress (same candidate slots and bias layout),
+// with no norm and no RoPE (the pages name neither for the indexer), and each entry is
+// stored as MXFP4 (the OCP MX conversion rule): 64 bytes of E2M1 codes (element 2i in the
+// low nibble of byte i) at row pos0/m + i of k_fp4 [B][Nmax][64] and four E8M0 block
+// scales at or_key_sf_offset(row, s) of k_sf [B][Nmax/128][512].
 // y_out [B][N][128] (nullable) is the merged entry before quantisation.
 int or_compress_index_keys(int B, int T, int m, int overlap, int64_t pos0,
                            const uint16_t* a, const uint16_t* b, const float* za,
@@ -338,11 +341,11 @@ int or_compress_index_keys(int B, int T, int m, int overlap, int64_t pos0,
   return 0;
 }
 
-// Indexer queries (R24) [walkthrough §2.2: the lightning indexer uses a low-rank query,
+// Indexer queries (a reading) [walkthrough §2.2: the lightning indexer uses a low-rank query,
 // down-projected and then up-projected into its heads, the down projection shared with
 // the main attention; §3.4: its QK path is FP4]: for every token t the H_I x 128 query
 // values are y[t][o] = sum_j W[o][j] * c[t][j] over the r-dim latent c (both BF16), with
-// no norm and no RoPE, stored per head as MXFP4 (R23): q_fp4 [T][H_I][64] (element 2i in
+// no norm and no RoPE, stored per head as MXFP4 (as the keys): q_fp4 [T][H_I][64] (element 2i in
 // the low nibble of byte i), q_sf [T][H_I][4]. y_out [T][H_I * 128] is nullable.
 int or_indexer_query(int T, int r, int H_I, const uint16_t* c, const uint16_t* W,
                      uint8_t* q_fp4, uint8_t* q_sf, double* y_out) {
@@ -370,7 +373,8 @@ int or_indexer_query(int T, int r, int H_I, const uint16_t* c, const uint16_t* W
   return 0;
 }
 
-// Grouped output projection (R25) [walkthrough §2.2: with many query heads the output
+// Grouped output projection (a reading: the pages give neither the group count nor the
+// group width) [walkthrough §2.2: with many query heads the output
 // projection first reduces each group of heads, then projects the concatenation; the
 // tutorial's Hybrid Attention section names it as the step after the shared-KV MQA]:
 // the H heads of a token form G groups of H/G consecutive heads; group g's concatenated
@@ -420,7 +424,8 @@ void or_dequant_row(const uint8_t* row, float scale, double* v) {
 // path runs in FP4 (MXFP4)]:
 //   s_j = sum_h w_h * max(0, sum_d q[h][d] * k[j][d])
 // with q and k decoded from E2M1 codes (element d in the low nibble of byte d/2 when d
-// is even) times their E8M0 block scale (one per 32 elements). No further scale (R9).
+// is even) times their E8M0 block scale (one per 32 elements). No further scale (a
+// reading: a positive scale cannot change the top-k).
 // scores [B][Nmax]: entries j >= n_entries[b] are set to NaN.
 int or_indexer_scores(int B, int H_I, int64_t Nmax, const int32_t* n_entries,
                       const uint8_t* q_fp4, const uint8_t* q_sf, const float* w,
@@ -503,12 +508,12 @@ int or_topk_bf16(int64_t n, int k, const double* scores, int32_t* idx) {
 // the selected entries (CSA, sparse = 1) or all n_entries[b] entries (HCA, sparse = 0)
 // [chooseai 一: HCA attends densely, no top-k], plus the sliding-window tokens
 // max(0,t-127)..t [walkthrough §2.2: the most recent 128 uncompressed tokens join the
-// core attention] read from the ring swa[b][p % 128] (R8, R13), with the sink logit
+// core attention] read from the ring swa[b][p % 128] (readings), with the sink logit
 // sigma_h added to the denominator only [digest 2.: learnable sink logit, the scores
 // may sum to less than 1]:
 //   l_j = tau * q_h . v_j,  Z = exp(sigma_h) + sum_j exp(l_j),  o_h = sum_j exp(l_j)/Z v_j
-// (R12: tau given by the caller, sink unscaled). lse = log Z. When derotate = 1 the
-// last 64 output dims are rotated by -t*theta (R15) [tutorial, Partial RoPE: the
+// (a reading: tau given by the caller, sink unscaled). lse = log Z. When derotate = 1 the
+// last 64 output dims are rotated by -t*theta (a reading) [tutorial, Partial RoPE: the
 // output is processed so absolute position does not leak into the value output].
 // out [B][H][512], lse [B][H]. Returns 0, or -1 for an out-of-range index.
 int or_attention(int B, int H, int k, int64_t Nmax, int sparse, const uint16_t* q,
@@ -596,7 +601,7 @@ int or_attention(int B, int H, int k, int64_t Nmax, int sparse, const uint16_t* 
 }
 
 // ------------------------------------------------------------------ prefill
-// Sliding-window row of token t (R8): the raw KV a[t] goes through the same RMSNorm
+// Sliding-window row of token t (a reading): the raw KV a[t] goes through the same RMSNorm
 // and the RoPE rotation at position t as an entry, and is stored as bf16.
 void or_swa_row(const uint16_t* a_row, int64_t t, double rope_base, double eps,
                 const float* norm_w, uint16_t* out_row) {
@@ -623,7 +628,7 @@ void or_swa_row(const uint16_t* a_row, int64_t t, double rope_base, double eps,
 // unfinished block; the classical cache holds the compressed entries]. Compression of
 // the new blocks is part of the pass: entries P/m .. (P+T)/m - 1 are written into
 // kv/kv_scale (rows 0 .. P/m - 1 are the cached prefix). Then, for every requested
-// query row r (token t = P + r): n(t) = floor((t+1)/m) eligible entries (R11), indexer
+// query row r (token t = P + r): n(t) = floor((t+1)/m) eligible entries (a reading), indexer
 // scores over them, top-k, and the attention of or_attention over the selected
 // entries plus the window t-127..t, whose rows come from swa_prefix (ring slot p % 128)
 // for p < P and from or_swa_row of the new tokens for p >= P.

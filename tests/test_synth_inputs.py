@@ -1,4 +1,7 @@
-"""The seeded input generators follow the recipe the design notes state (no GPU)."""
+"""The seeded input generators draw what they promise (no GPU): E4M3 codes never NaN and
+near the top of the range, E2M1 magnitudes from the table with balanced signs, E8M0 codes
+in their stated range, the workloads' shapes and lengths, planted runs of 16 with large
+keys, and a device generator that matches the host distributions."""
 
 import numpy as np
 import torch
