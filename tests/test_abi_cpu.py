@@ -53,6 +53,32 @@ def test_workspace_sizes_are_host_only(L):
     assert L.csa_attn_workspace_size(1, 0, 10) == 0
 
 
+def test_workspace_sizes_grow_with_every_argument(L):
+    # one workspace serves every smaller problem (the header's promise), so no size may
+    # shrink when a dimension grows; sizes come in whole 256-byte blocks
+    ix = L.csa_indexer_topk_workspace_size
+    at = L.csa_attn_workspace_size
+    pf = L.csa_prefill_workspace_size
+    op = L.csa_grouped_out_proj_workspace_size
+    for B in (1, 2, 4, 32, 1024):
+        for N in (128, 4096, 262144):
+            for k in (1, 512, 2048):
+                v = ix(B, N, k)
+                assert v % 256 == 0
+                assert v <= ix(2 * B, N, k) and v <= ix(B, 2 * N, k) and v <= ix(B, N, 2 * k)
+    for B in (1, 4, 32):
+        for H in (64, 128):
+            for rows in (129, 1152, 2176, 8320):
+                v = at(B, H, rows)
+                assert v % 256 == 0 and v <= at(2 * B, H, rows) and v <= at(B, H, rows + 64)
+    for T in (1, 1024, 1100, 65536):
+        for N in (128, 65536):
+            v = pf(T, N, 128, 1024)
+            assert v % 256 == 0 and v <= pf(T + 1, N, 128, 1024) and v <= pf(T, N + 128, 128, 1024)
+            assert v >= ix(min(T, 1024), N, 1024)  # holds the indexer workspace of one chunk
+    assert op(100, 16, 1024) <= op(101, 16, 1024) and op(1, 1, 1) % 256 == 0
+
+
 FAKE = 1 << 20  # a 256-aligned non-null address: never dereferenced on a rejected call
 
 
