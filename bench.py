@@ -447,7 +447,7 @@ def bench_hca(args, rank: int, world: int, local: int) -> None:
         csa.hca_attn_decode(c["q"], c["pos"], c["n_entries"], c["kv"], c["kv_scale"], c["swa"],
                             c["sink"], workspace=ws, out=out, dev_status=status)
 
-    graph_steps = 8
+    graph_steps = next(g for g in (8, 4, 2, 1) if args.steps % g == 0)  # exactly --steps
 
     def capture(fn):
         g = torch.cuda.CUDAGraph()
@@ -694,7 +694,9 @@ def main():
         torch.cuda.synchronize()
         return g
 
-    GRAPH_STEPS = 8
+    # graphs of 8 steps when --steps allows it, else of the largest power of two dividing
+    # it, so that the timed region runs exactly --steps steps
+    GRAPH_STEPS = next(g for g in (8, 4, 2, 1) if args.steps % g == 0)
     step_graphs = [capture(lambda c=c: step(c), GRAPH_STEPS) for c in copies]
     idx_graphs = [capture(lambda c=c: step_idx(c), GRAPH_STEPS) for c in copies]
     att_graphs = [capture(lambda c=c: step_att(c), GRAPH_STEPS) for c in copies]

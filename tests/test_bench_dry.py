@@ -64,16 +64,18 @@ def _contract(d, cpu_baseline=True):
 
 @pytest.mark.slow
 def test_default_decode_line():
-    d = _line(["--steps", "16", "--warmup", "3"])
+    d = _line(["--steps", "20", "--warmup", "3"])
     _contract(d)
+    assert d["steps"] == 20
     assert d["config"]["workload"] == "csa_decode_pro_1m" and d["roofline"]["bound"] == "hbm"
     assert d["roofline"]["algorithmic_bytes_per_launch"] == 71338000
 
 
 def test_hca_line():
-    d = _line(["--workload", "hca", "--steps", "16", "--warmup", "3"])
+    d = _line(["--workload", "hca", "--steps", "20", "--warmup", "3"])
     _contract(d)
     assert d["config"]["workload"] == "hca_decode_128k"
+    assert d["steps"] == 20  # graphs of 4 steps: exactly the steps asked for
 
 
 def test_prefill_line():
