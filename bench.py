@@ -9,13 +9,15 @@ Metric: decode queries/s (whole job). Inputs are synthetic and seeded; four devi
 of the streamed inputs are rotated so that consecutive steps never hit in L2.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                       [--workload decode|prefill]
+                       [--workload decode|prefill|hca]
 Under torchrun every rank runs its own 4-sequence batch (weak scaling, no collective on
 the data path); rank 0 prints one JSON line.
 
 --workload prefill times csa_prefill instead: 65,536 new tokens after a 196,608-token
 prefix (one sequence, 128 heads, indexer 64 heads, top-k 1024); one step is the whole
 prefill call (compression, indexer top-k and attention for every new token).
+--workload hca times hca_attn_decode: 8 sequences at 128K context (1,024 entries each,
+64 heads), dense MQA over every entry + window + sink, graphs over 24 device copies.
 """
 
 from __future__ import annotations
