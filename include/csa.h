@@ -127,11 +127,11 @@ int csa_compress(const csa_compress_args* args, csa_stream_t stream);
  * fit Nmax is reported through dev_status and skipped.
  */
 typedef struct {
-  int32_t B;
+  int32_t B;               /* sequences, one new token each */
   int32_t m;               /* block size: 4 for CSA, 128 for HCA */
   int32_t overlap;         /* 1: CSA overlapping merge */
-  float rope_base;
-  float eps;
+  float rope_base;         /* 10000 */
+  float eps;               /* RMSNorm epsilon of entries and window rows */
   const int32_t* pos;      /* [B] position of the new token */
   const uint16_t* a;       /* bf16 [B][512] */
   const uint16_t* b;       /* bf16 [B][512] (overlap) */
@@ -149,9 +149,9 @@ typedef struct {
   int64_t Nmax;            /* entry capacity, multiple of 128 */
   int32_t* n_entries;      /* [B] updated when a block closes */
   const uint16_t* ia;      /* optional indexer-key stream: bf16 [B][128] (NULL: none) */
-  const uint16_t* ib;
-  const float* iza;
-  const float* izb;
+  const uint16_t* ib;      /* bf16 [B][128]: the key stream of the previous-block slots (as b) */
+  const float* iza;        /* [B][128] gate logits paired with ia */
+  const float* izb;        /* [B][128] gate logits paired with ib */
   const float* ibias;      /* [2m] */
   uint16_t* itail_a;       /* state bf16 [B][m][128] */
   float* itail_za;         /* state [B][m][128] */
@@ -178,11 +178,11 @@ int csa_decode_append(const csa_append_args* args, csa_stream_t stream);
  * Computed in fp32. Nmax must be a multiple of 128.
  */
 typedef struct {
-  int32_t B;
-  int32_t T;
-  int32_t m;
-  int32_t overlap;
-  int64_t pos0;
+  int32_t B;              /* sequences */
+  int32_t T;              /* tokens per sequence in this call (row pitch of a, b, za, zb) */
+  int32_t m;              /* block size (4 for CSA) */
+  int32_t overlap;        /* 1: overlapping merge (needs b, zb); 0: own block only */
+  int64_t pos0;           /* absolute position of token 0, a multiple of m */
   const uint16_t* a;      /* bf16 [B][T][128] */
   const uint16_t* b;      /* bf16 [B][T][128]; NULL when overlap == 0 */
   const float* za;        /* [B][T][128] */
@@ -246,7 +246,7 @@ int csa_indexer_query(const csa_iquery_args* args, csa_stream_t stream);
  * that share a workspace must not overlap on the device.
  */
 typedef struct {
-  int32_t B;
+  int32_t B;              /* queries (one per sequence) */
   int32_t H_I;                /* indexer heads: 16, 32 or 64 */
   int32_t k;                  /* top-k */
   int64_t Nmax;               /* entry capacity per sequence, multiple of 128 */
@@ -292,7 +292,7 @@ int csa_indexer_topk_bf16(const csa_topk_args* args, void* workspace, size_t wor
  * H in {64, 128}. k <= 2048 (CSA); n_entries <= Nmax (HCA, any size).
  */
 typedef struct {
-  int32_t B;
+  int32_t B;              /* queries (one per sequence) */
   int32_t H;                  /* query heads: 64 or 128 */
   int32_t k;                  /* CSA: selected entries per sequence; ignored by HCA */
   int64_t Nmax;               /* entry capacity per sequence */
@@ -360,24 +360,24 @@ typedef struct {
   float eps;                  /* RMSNorm epsilon */
   int32_t derotate;           /* 1: de-rotate the last 64 output dims by t */
   const uint16_t* a;          /* new tokens (see Layouts) */
-  const uint16_t* b;
-  const float* za;
-  const float* zb;
-  const float* bias;
+  const uint16_t* b;          /* bf16 [T][512], the previous-block stream */
+  const float* za;            /* [T][512] gate logits paired with a */
+  const float* zb;            /* [T][512] gate logits paired with b */
+  const float* bias;          /* [2m] slot bias */
   const float* norm_w;        /* [512] or NULL = ones (entries and window rows) */
-  const uint16_t* prev_b;
-  const float* prev_zb;
+  const uint16_t* prev_b;     /* bf16 [m][512]: tokens P-m .. P-1 of b (P > 0) */
+  const float* prev_zb;       /* [m][512] (P > 0) */
   uint8_t* kv;                /* in: prefix rows; out: the new rows */
-  float* kv_scale;
-  const uint8_t* q_fp4;
-  const uint8_t* q_sf;
-  const float* w;
-  const uint8_t* k_fp4;
-  const uint8_t* k_sf;
-  const uint16_t* q;
+  float* kv_scale;            /* [Nmax], as kv */
+  const uint8_t* q_fp4;       /* [T][H_I][64] MXFP4 indexer queries */
+  const uint8_t* q_sf;        /* [T][H_I][4] E8M0 scales */
+  const float* w;             /* [T][H_I] indexer head weights */
+  const uint8_t* k_fp4;       /* [Nmax][64] indexer keys of every entry up to (P+T)/m */
+  const uint8_t* k_sf;        /* [Nmax/128][512] grouped key scales */
+  const uint16_t* q;          /* bf16 [T][H][512] queries (RMS-normalised, rotated at t) */
   const float* sink;          /* [H] */
-  const uint16_t* swa_prefix;
-  uint16_t* out;
+  const uint16_t* swa_prefix; /* bf16 [128][512] window ring of the prefix (P > 0) */
+  uint16_t* out;              /* out bf16 [T][H][512] */
   float* lse;                 /* optional */
   int32_t* idx;               /* optional: the selected sets */
   int32_t* dev_status;        /* optional device word */
@@ -400,15 +400,15 @@ int csa_prefill(const csa_prefill_args* args, void* workspace, size_t workspace_
  * multiples of 128.
  */
 typedef struct {
-  int32_t T;
-  int32_t H;
-  int32_t G;
-  int32_t d_g;
-  int32_t d_model;
-  const uint16_t* attn;
-  const uint16_t* Wg;
-  const uint16_t* Wo;
-  uint16_t* out;
+  int32_t T;             /* tokens */
+  int32_t H;             /* heads: 64 or 128 */
+  int32_t G;             /* groups of H/G consecutive heads */
+  int32_t d_g;           /* reduced width per group, multiple of 128 */
+  int32_t d_model;       /* output width, multiple of 128 */
+  const uint16_t* attn;  /* bf16 [T][H][512] attention output */
+  const uint16_t* Wg;    /* bf16 [G][d_g][H/G * 512] per-group reductions */
+  const uint16_t* Wo;    /* bf16 [d_model][G * d_g] output projection */
+  uint16_t* out;         /* out bf16 [T][d_model] */
   int32_t* dev_status;   /* optional device word */
 } csa_oproj_args;
 

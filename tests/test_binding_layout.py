@@ -99,3 +99,11 @@ def test_every_entry_point_has_a_signature_of_the_declared_arity():
         fn = getattr(L, name)
         assert fn.argtypes is not None and len(fn.argtypes) == arity, name
         assert fn.restype is results[ret], (name, ret)
+
+
+def test_every_header_field_is_documented():
+    # the boundary states each argument's meaning and layout next to it
+    text = open(HEADER).read()
+    for body, name in re.findall(r"typedef struct\s*\{(.*?)\}\s*(\w+)\s*;", text, flags=re.S):
+        bare = [ln.strip() for ln in body.splitlines() if ln.strip() and "/*" not in ln]
+        assert not bare, f"{name}: fields without a comment: {bare}"
