@@ -14,7 +14,8 @@ E2M1_TABLE = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
 
 def bf16_to_f64(h):
     h = np.asarray(h, dtype=np.uint16)
-    return (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    with np.errstate(invalid="ignore"):  # signalling-NaN codes widen to NaN, quietly
+        return (h.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
 
 
 def e4m3_to_f64(c):
