@@ -86,7 +86,7 @@ def lib():
             L.or_swa_row.restype = None
             L.or_swa_row.argtypes = [u16, i64, d, d, f32, u16]
             L.or_prefill.restype = i
-            L.or_prefill.argtypes = [i64, i, i, i, i, i, d, d, d, i, u16, u16, f32, f32, f32,
+            L.or_prefill.argtypes = [i64, i, i, i, i, i, d, d, d, i, i, u16, u16, f32, f32, f32,
                                      f32, u16, f32, u8, f32, i64, u8, u8, f32, u8, u8, u16,
                                      f32, u16, i, i32, f64, f64, i32, i]
             _lib = L
@@ -305,10 +305,12 @@ def swa_row(a_row, t: int, rope_base: float = 10000.0, eps: float = 1e-6,
 
 
 def prefill(inp: dict, k: int, q_rows, tau: float | None = None, rope_base: float = 10000.0,
-            eps: float = 1e-6, derotate: bool = True, nthreads: int = 0) -> dict:
+            eps: float = 1e-6, derotate: bool = True, strict: bool = False,
+            nthreads: int = 0) -> dict:
     """Evaluate the rows `q_rows` of a prefill described by a synth.prefill_inputs dict
     (with an optional RMSNorm weight under "norm_w"). Returns out [nq][H][512], lse [nq][H],
-    idx [nq][k] and the cache after compression."""
+    idx [nq][k] and the cache after compression. strict=True takes the eligibility
+    n(t) = floor(t/m) (blocks completed before t) instead of floor((t+1)/m)."""
     P, T, m, H, H_I, Nmax = (inp[x] for x in ("P", "T", "m", "H", "H_I", "Nmax"))
     tau = 1.0 / np.sqrt(512.0) if tau is None else tau
     kv = np.array(inp["kv"], dtype=np.uint8, copy=True)
@@ -323,7 +325,7 @@ def prefill(inp: dict, k: int, q_rows, tau: float | None = None, rope_base: floa
         ("k_sf", np.uint8), ("q", np.uint16), ("sink", np.float32),
         ("swa_prefix", np.uint16), ("norm_w", np.float32))}
     U16, F32, U8 = C.c_uint16, C.c_float, C.c_uint8
-    rc = lib().or_prefill(P, T, m, H, H_I, k, rope_base, eps, tau, int(derotate),
+    rc = lib().or_prefill(P, T, m, H, H_I, k, rope_base, eps, tau, int(derotate), int(strict),
                           _p(g["a"], U16), _p(g["b"], U16), _p(g["za"], F32),
                           _p(g["zb"], F32), _p(g["bias"], F32), _p(g["norm_w"], F32),
                           _p(g["prev_b"], U16), _p(g["prev_zb"], F32), _p(kv, U8),

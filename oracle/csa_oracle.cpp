@@ -628,15 +628,22 @@ void or_swa_row(const uint16_t* a_row, int64_t t, double rope_base, double eps,
 // unfinished block; the classical cache holds the compressed entries]. Compression of
 // the new blocks is part of the pass: entries P/m .. (P+T)/m - 1 are written into
 // kv/kv_scale (rows 0 .. P/m - 1 are the cached prefix). Then, for every requested
-// query row r (token t = P + r): n(t) = floor((t+1)/m) eligible entries (a reading), indexer
+// query row r (token t = P + r): n(t) eligible entries (a reading, below), indexer
 // scores over them, top-k, and the attention of or_attention over the selected
 // entries plus the window t-127..t, whose rows come from swa_prefix (ring slot p % 128)
 // for p < P and from or_swa_row of the new tokens for p >= P.
+// Eligibility (a reading; the pages say only that a query sees the compressed blocks that
+// are complete): by default the block whose last token is t itself counts, n(t) =
+// floor((t+1)/m), so a prefill row at t equals a decode step at t with the block just
+// closed, and the decode entry counts of the workloads (L/m entries at position L-1)
+// hold. strict_eligibility = 1 takes "completed before t": only blocks whose last token
+// lies before t count, n(t) = floor(t/m).
 // q_rows [nq] lists the rows to evaluate; out [nq][H][512], lse [nq][H], idx [nq][k].
 int or_prefill(int64_t P, int T, int m, int H, int H_I, int k, double rope_base,
-               double eps, double tau, int derotate, const uint16_t* a, const uint16_t* b,
-               const float* za, const float* zb, const float* bias, const float* norm_w,
-               const uint16_t* prev_b, const float* prev_zb, uint8_t* kv, float* kv_scale,
+               double eps, double tau, int derotate, int strict_eligibility, const uint16_t* a,
+               const uint16_t* b, const float* za, const float* zb, const float* bias,
+               const float* norm_w, const uint16_t* prev_b, const float* prev_zb, uint8_t* kv,
+               float* kv_scale,
                int64_t Nmax, const uint8_t* q_fp4, const uint8_t* q_sf, const float* w,
                const uint8_t* k_fp4, const uint8_t* k_sf, const uint16_t* q,
                const float* sink, const uint16_t* swa_prefix, int nq,
@@ -644,6 +651,7 @@ int or_prefill(int64_t P, int T, int m, int H, int H_I, int k, double rope_base,
                int nthreads) {
   if (P < 0 || T < 0 || m < 1 || P % m != 0 || (P + T) / m > Nmax) return -1;
   if (P > 0 && !swa_prefix) return -1;
+  if (strict_eligibility != 0 && strict_eligibility != 1) return -1;
   const int64_t n0 = P / m;
   int rc = or_compress(1, T, m, 1, P, rope_base, eps, a, b, za, zb, bias, norm_w, prev_b,
                        prev_zb, nullptr, nullptr, kv + (size_t)n0 * kRow, kv_scale + n0);
@@ -658,7 +666,7 @@ int or_prefill(int64_t P, int T, int m, int H, int H_I, int k, double rope_base,
     for (int i = tid; i < nq; i += nthreads) {
       const int r = q_rows[i];
       const int64_t t = P + r;
-      const int32_t n = (int32_t)((t + 1) / m);
+      const int32_t n = (int32_t)((strict_eligibility ? t : t + 1) / m);
       int32_t* sel = idx + (size_t)i * k;
       if (or_indexer_scores(1, H_I, Nmax, &n, q_fp4 + (size_t)r * H_I * (kDI / 2),
                             q_sf + (size_t)r * H_I * 4, w + (size_t)r * H_I, k_fp4, k_sf,

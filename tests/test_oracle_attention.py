@@ -155,8 +155,8 @@ def test_bad_index_is_rejected():
 
 
 # ----------------------------------------------------------------- prefill
-@pytest.mark.parametrize("weighted", [False, True])
-def test_prefill_row_matches_independent_recomputation(weighted):
+@pytest.mark.parametrize("weighted,strict", [(False, False), (True, False), (False, True)])
+def test_prefill_row_matches_independent_recomputation(weighted, strict):
     P, T, m, H, H_I, k = 512, 64, 4, 2, 4, 40
     inp = synth.prefill_inputs(P, T, m, H, H_I, seed=10)
     norm_w = None
@@ -164,7 +164,7 @@ def test_prefill_row_matches_independent_recomputation(weighted):
         norm_w = np.random.default_rng(10).uniform(0.5, 2.0, 512).astype(np.float32)
         inp["norm_w"] = norm_w
     rows = [0, 1, 3, 4, 31, 63]
-    r = oracle.prefill(inp, k, rows)
+    r = oracle.prefill(inp, k, rows, strict=strict)
     # the new entries match a stand-alone compression of the new tokens
     comp = oracle.compress(inp["a"][None], inp["za"][None], inp["bias"], m, True,
                            b=inp["b"][None], zb=inp["zb"][None], pos0=P,
@@ -179,7 +179,8 @@ def test_prefill_row_matches_independent_recomputation(weighted):
         indep.e8m0_to_f64(ks), 32, -1)
     for i, row in enumerate(rows):
         t = P + row
-        n = (t + 1) // m
+        # inclusive: the block whose last token is t counts; strict: blocks ending before t
+        n = t // m if strict else (t + 1) // m
         q = indep.e2m1_to_f64(indep.unpack_fp4(inp["q_fp4"][row])) * np.repeat(
             indep.e8m0_to_f64(inp["q_sf"][row]), 32, -1)
         s = np.maximum(kdec[:n] @ q.T, 0) @ inp["w"][row].astype(np.float64)
@@ -212,6 +213,31 @@ def test_prefill_eligibility_counts_the_block_ending_at_t():
         sel = r["idx"][t]
         assert (sel >= 0).sum() == (t + 1) // m
         assert sel[sel >= 0].max(initial=-1) == (t + 1) // m - 1
+
+
+def test_prefill_strict_eligibility_takes_blocks_completed_before_t():
+    # "completed before t": block i (tokens m*i .. m*i+m-1) is visible at t iff
+    # m*i + m - 1 < t; the block closing at t itself is not. Counted by hand for m = 4:
+    # t = 0..4 see 0 blocks, t = 4 is the first to see block 0 (its last token is 3).
+    P, T, m = 0, 16, 4
+    inp = synth.prefill_inputs(P, T, m, 1, 2, seed=11)
+    r = oracle.prefill(inp, 100, list(range(T)), strict=True)
+    want = [0, 0, 0, 0, 1, 1, 1, 1, 2, 2, 2, 2, 3, 3, 3, 3]
+    for t in range(T):
+        sel = r["idx"][t]
+        assert (sel >= 0).sum() == want[t]
+        assert sel[sel >= 0].max(initial=-1) == want[t] - 1
+
+
+def test_prefill_strict_row_at_t_equals_inclusive_row_at_t_minus_1_selection():
+    # with k >= n the set is every eligible entry, so under the strict reading the set at
+    # t is the inclusive reading's set at t - 1 (floor(t/m) = floor(((t-1)+1)/m))
+    P, T, m = 64, 40, 4
+    inp = synth.prefill_inputs(P, T, m, 2, 2, seed=13)
+    rows = list(range(1, T))
+    s = oracle.prefill(inp, 64, rows, strict=True)
+    i = oracle.prefill(inp, 64, [r - 1 for r in rows])
+    np.testing.assert_array_equal(s["idx"], i["idx"])
 
 
 def test_swa_row_at_position_zero_is_the_normalised_token():

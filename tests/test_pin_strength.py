@@ -246,8 +246,14 @@ MUTANTS = [
      "const uint16_t* qh = q + ((size_t)bb * H + h) * kD;",
      "const uint16_t* qh = q + ((size_t)bb * H) * kD;", 0),
     ("pf_n_off1",
-     "const int32_t n = (int32_t)((t + 1) / m);",
+     "const int32_t n = (int32_t)((strict_eligibility ? t : t + 1) / m);",
      "const int32_t n = (int32_t)(t / m);", 0),
+    ("pf_strict_ignored",
+     "const int32_t n = (int32_t)((strict_eligibility ? t : t + 1) / m);",
+     "const int32_t n = (int32_t)((t + 1) / m);", 0),
+    ("pf_strict_off1",
+     "const int32_t n = (int32_t)((strict_eligibility ? t : t + 1) / m);",
+     "const int32_t n = (int32_t)((strict_eligibility ? t - 1 : t + 1) / m);", 0),
     ("sw_pos",
      "const double c = std::cos((double)t * theta), s = std::sin((double)t * theta);\n"
      "    const double x0 = y[",
