@@ -327,13 +327,19 @@ int hca_attn_decode(const csa_attn_args* args, void* workspace, size_t workspace
  *    P/m .. (P+T)/m - 1 are written into kv / kv_scale; rows 0 .. P/m - 1 are the cached
  *    prefix and are only read. T may leave a tail of T % m tokens: their block is not
  *    emitted (it stays in the caller's state).
- * 2. For every new token t = P + r (r = 0 .. T-1), with n(t) = floor((t+1)/m) eligible
- *    entries: the indexer top-k over entries j < n(t) (as csa_indexer_topk, all queries
+ * 2. For every new token t = P + r (r = 0 .. T-1), with n(t) eligible entries (below):
+ *    the indexer top-k over entries j < n(t) (as csa_indexer_topk, all queries
  *    scoring the one key array k_fp4 / k_sf, which must hold the indexer keys of every
  *    entry up to (P+T)/m), then CSA attention over the selected entries, the window
  *    t-127 .. t and the sink (as csa_sparse_attn_decode with pos = t). Window rows of
  *    prefix positions come from the ring swa_prefix[p % 128]; window rows of new tokens
  *    are RMSNorm (eps, norm_w) then RoPE at position p of a[p - P], rounded to BF16.
+ *
+ * Eligibility: the pages say a query sees the compressed blocks that are complete. With
+ * strict_eligibility = 0 (the default reading) the block whose last token is t itself
+ * counts: n(t) = floor((t+1)/m), so a prefill row at t equals a decode step at t just after
+ * that block closed. With strict_eligibility = 1 only blocks completed before t count:
+ * n(t) = floor(t/m). The window t-127 .. t is the same under both.
  *
  * Layouts: a, b bf16 [T][512]; za, zb [T][512]; bias [2m]; prev_b bf16 [m][512] and
  * prev_zb [m][512] are the m tokens before P (needed when P > 0); kv [Nmax][576];
@@ -359,6 +365,7 @@ typedef struct {
   float rope_base;            /* 10000 */
   float eps;                  /* RMSNorm epsilon */
   int32_t derotate;           /* 1: de-rotate the last 64 output dims by t */
+  int32_t strict_eligibility; /* 0: n(t) = floor((t+1)/m); 1: n(t) = floor(t/m) */
   const uint16_t* a;          /* new tokens (see Layouts) */
   const uint16_t* b;          /* bf16 [T][512], the previous-block stream */
   const float* za;            /* [T][512] gate logits paired with a */

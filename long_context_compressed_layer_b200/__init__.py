@@ -81,6 +81,7 @@ class PrefillArgs(C.Structure):
     _fields_ = [("P", C.c_int64), ("T", C.c_int32), ("m", C.c_int32), ("H", C.c_int32),
                 ("H_I", C.c_int32), ("k", C.c_int32), ("Nmax", C.c_int64), ("tau", C.c_float),
                 ("rope_base", C.c_float), ("eps", C.c_float), ("derotate", C.c_int32),
+                ("strict_eligibility", C.c_int32),
                 ("a", _vp), ("b", _vp), ("za", _vp), ("zb", _vp), ("bias", _vp),
                 ("norm_w", _vp), ("prev_b", _vp), ("prev_zb", _vp), ("kv", _vp),
                 ("kv_scale", _vp), ("q_fp4", _vp), ("q_sf", _vp), ("w", _vp), ("k_fp4", _vp),
@@ -460,11 +461,13 @@ def prefill_workspace(T: int, Nmax: int, H: int, k: int, device="cuda") -> torch
 def prefill(P: int, m: int, k: int, *, a, b, za, zb, bias, kv, kv_scale, q_fp4, q_sf, w,
             k_fp4, k_sf, q, sink, prev_b=None, prev_zb=None, swa_prefix=None, norm_w=None,
             tau: float = 0.0, rope_base: float = 10000.0, eps: float = 1e-6,
-            derotate: bool = True, workspace=None, out=None, lse: bool = False,
-            idx: bool = False, dev_status=None, stream=None):
+            derotate: bool = True, strict_eligibility: bool = False, workspace=None,
+            out=None, lse: bool = False, idx: bool = False, dev_status=None, stream=None):
     """Causal CSA prefill of the T new tokens after a P-token prefix (one sequence).
     kv / kv_scale [Nmax] are updated in place with the new entries. Returns out
-    [T][H][512] bf16 and, when asked, lse [T][H] and the selected sets idx [T][k]."""
+    [T][H][512] bf16 and, when asked, lse [T][H] and the selected sets idx [T][k].
+    strict_eligibility: a query at t sees only blocks completed before t (floor(t/m)
+    entries) instead of also the block closing at t (floor((t+1)/m))."""
     T = a.shape[0]
     H, H_I = q.shape[1], q_fp4.shape[1]
     Nmax = kv.shape[0]
@@ -484,6 +487,7 @@ def prefill(P: int, m: int, k: int, *, a, b, za, zb, bias, kv, kv_scale, q_fp4, 
     l = torch.empty((T, H), dtype=torch.float32, device=dev) if lse else None
     ix = torch.empty((T, k), dtype=torch.int32, device=dev) if idx else None
     args = PrefillArgs(P, T, m, H, H_I, k, Nmax, tau, rope_base, eps, int(derotate),
+                       int(strict_eligibility),
                        _ptr(a, elem=2, name="a"), _ptr(b, elem=2, name="b"),
                        _ptr(za, elem=4, name="za"), _ptr(zb, elem=4, name="zb"),
                        _ptr(bias, elem=4, name="bias"), _ptr(norm_w, elem=4, name="norm_w"),

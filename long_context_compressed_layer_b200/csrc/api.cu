@@ -406,7 +406,7 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
   if (a->P < 0 || a->T < 0 || a->m < 1 || a->m > 128 || a->P % a->m || a->Nmax < 128 ||
       a->Nmax % 128 || (a->P + a->T) / a->m > a->Nmax || !(a->eps >= 0.f) ||
       !(a->rope_base > 0.f) || !(a->tau >= 0.f) || (a->derotate != 0 && a->derotate != 1) ||
-      a->k < 1)
+      (a->strict_eligibility != 0 && a->strict_eligibility != 1) || a->k < 1)
     return CSA_ERR_INVALID_ARG;
   if ((a->H != 64 && a->H != 128) || (a->H_I != 16 && a->H_I != 32 && a->H_I != 64) ||
       a->k > 2048 || a->P + a->T >= ((int64_t)1 << 31) || a->Nmax > ((int64_t)1 << 30))

@@ -4,7 +4,9 @@
 // state).
 //
 // prefill_prep_kernel writes, for the T new tokens of one sequence:
-//   n_all[r]  = floor((P + r + 1) / m), the entries eligible at position t = P + r;
+//   n_all[r]  = the entries eligible at position t = P + r: floor((t + 1) / m) when the
+//              block closing at t counts, floor(t / m) under the strict reading (only
+//              blocks completed before t);
 //   pos_all[r] = P + r;
 //   lin[i], i = 0 .. T + 126: the window row of position P - 127 + i in consecutive order,
 //     taken from the prefix ring swa_prefix[p % 128] for p < P (rows of negative
@@ -31,7 +33,7 @@ __device__ __forceinline__ uint4 bf16x8_widen(uint4 v) {
 
 struct PrepParams {
   int64_t P;
-  int T, m;
+  int T, m, strict;
   float eps, rope_base;
   const uint16_t* a;
   const float* norm_w;
@@ -47,7 +49,7 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(PrepParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (gtid < p.T) {
-    p.n_all[gtid] = (int32_t)((p.P + gtid + 1) / p.m);
+    p.n_all[gtid] = (int32_t)((p.P + gtid + (p.strict ? 0 : 1)) / p.m);
     p.pos_all[gtid] = (int32_t)(p.P + gtid);
   }
   const int64_t i = (int64_t)blockIdx.x * (blockDim.x / 32) + warp;
@@ -99,8 +101,8 @@ __global__ void __launch_bounds__(256) prefill_prep_kernel(PrepParams p) {
 
 cudaError_t launch_prefill_prep(const csa_prefill_args& a, __half* lin, int32_t* n_all,
                                 int32_t* pos_all, cudaStream_t stream) {
-  PrepParams p{a.P, a.T, a.m, a.eps, a.rope_base, a.a, a.norm_w, a.swa_prefix, lin, n_all,
-               pos_all};
+  PrepParams p{a.P, a.T, a.m, a.strict_eligibility, a.eps, a.rope_base, a.a, a.norm_w,
+               a.swa_prefix, lin, n_all, pos_all};
   const int64_t rows = (int64_t)a.T + kWin - 1;
   const int64_t blocks_rows = (rows + 7) / 8, blocks_ids = ((int64_t)a.T + 255) / 256;
   const int64_t blocks = blocks_rows > blocks_ids ? blocks_rows : blocks_ids;

@@ -149,7 +149,7 @@ def test_compress_rejects_on_host(L):
 
 
 def _prefill_args(**over):
-    a = csa.PrefillArgs(4096, 300, 4, 128, 64, 1024, 1152, 0.0, 10000.0, 1e-6, 1,
+    a = csa.PrefillArgs(4096, 300, 4, 128, 64, 1024, 1152, 0.0, 10000.0, 1e-6, 1, 0,
                         *([FAKE] * 5), None, FAKE, FAKE, *([FAKE] * 10), FAKE, None,
                         None, None)
     for k, v in over.items():
@@ -168,6 +168,7 @@ def test_prefill_rejects_on_host(L):
     # no capacity at all, even with no complete block: rejected before any launch
     assert f(_prefill_args(P=0, T=3, Nmax=0)) == csa.CSA_ERR_INVALID_ARG
     assert f(_prefill_args(k=0)) == csa.CSA_ERR_INVALID_ARG
+    assert f(_prefill_args(strict_eligibility=2)) == csa.CSA_ERR_INVALID_ARG
     assert f(_prefill_args(H=96)) == csa.CSA_ERR_UNSUPPORTED
     assert f(_prefill_args(H_I=8)) == csa.CSA_ERR_UNSUPPORTED
     assert f(_prefill_args(k=4096)) == csa.CSA_ERR_UNSUPPORTED

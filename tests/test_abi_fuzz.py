@@ -53,7 +53,7 @@ BASES = [
     (lambda: csa.AttnArgs(2, 128, 1024, 4096, F, F, F, F, F, F, F, F, 0.0, 10000.0, 1, F,
                           None, None),
      lambda a: L.csa_sparse_attn_decode_noalloc(C.byref(a), None)),
-    (lambda: csa.PrefillArgs(4096, 300, 4, 128, 64, 1024, 1152, 0.0, 10000.0, 1e-6, 1,
+    (lambda: csa.PrefillArgs(4096, 300, 4, 128, 64, 1024, 1152, 0.0, 10000.0, 1e-6, 1, 0,
                              *([F] * 5), None, F, F, *([F] * 10), F, None, None, None),
      lambda a: L.csa_prefill(C.byref(a), F, WS, None)),
 ]

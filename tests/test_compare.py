@@ -6,7 +6,7 @@ import pytest
 
 import oracle
 from synth import inputs as synth
-from tests import compare
+from tests import compare, indep
 
 
 def test_close_bounds_both_the_largest_error_and_the_relative_l2():
@@ -80,3 +80,88 @@ def test_bf16_topk_accepts_only_boundary_neighbours():
     wrong = np.sort(np.r_[want[:k - 1], far]) if far not in want else want
     with pytest.raises(AssertionError):
         compare.compare_topk_bf16(wrong, s, n, k)
+
+
+def test_code_flips_must_be_the_rounding_of_a_value_near_the_oracles():
+    # an E4M3 value placed exactly on the midpoint of two codes: either neighbour passes,
+    # a code two steps away does not (the older rule looked only at where the oracle's
+    # value lay and accepted any code there)
+    kv, sc, dbg, ora = _entries()
+    y = ora["y"].copy()
+    lo = int(kv[0, 1, 7]) & 0x7F
+    if lo in (0, 0x7E):
+        lo = 0x30
+    pair = indep.e4m3_to_f64(np.array([lo, lo + 1], dtype=np.uint8))
+    y[0, 1, 7] = (pair[0] + pair[1]) / 2 * float(sc[0, 1])
+    ref = kv.copy()
+    ref[0, 1, 7] = lo
+    for code, ok in ((lo, True), (lo + 1, True), (lo + 2, False), (lo - 1, False)):
+        got = ref.copy()
+        got[0, 1, 7] = code
+        if ok:
+            compare.check_codes(got, ref, y, sc)
+        else:
+            with pytest.raises(AssertionError, match="E4M3"):
+                compare.check_codes(got, ref, y, sc)
+
+
+def test_rotated_bf16_codes_follow_the_pair_norm_window():
+    # a rotated dim that nearly cancels (|v| = 1e-7 of its pair's norm): fp32 rounding of
+    # the pair moves it by several of its own BF16 steps, and the rule admits exactly the
+    # codes within 1e-5 of the pair norm, not arbitrary ones
+    kv, sc, dbg, ora = _entries()
+    y = ora["y"].copy()
+    y[0, 0, 448], y[0, 0, 449] = 1e-7, 1.0  # pair (x0, x1) with a tiny x0
+    ref = kv.copy()
+    ref[0, 0, 448:452] = np.frombuffer(indep.f64_to_bf16(np.array([1e-7, 1.0])).tobytes(),
+                                       np.uint8)
+    close_by = ref.copy()
+    close_by[0, 0, 448:452] = np.frombuffer(indep.f64_to_bf16(np.array([3e-6, 1.0])).tobytes(),
+                                            np.uint8)
+    assert compare.check_codes(close_by, ref, y, sc) == 1
+    far = ref.copy()
+    far[0, 0, 448:452] = np.frombuffer(indep.f64_to_bf16(np.array([3e-4, 1.0])).tobytes(),
+                                       np.uint8)
+    with pytest.raises(AssertionError, match="BF16"):
+        compare.check_codes(far, ref, y, sc)
+    sign = ref.copy()
+    sign[0, 0, 448:452] = np.frombuffer(indep.f64_to_bf16(np.array([-2e-5, 1.0])).tobytes(),
+                                        np.uint8)
+    with pytest.raises(AssertionError, match="BF16"):
+        compare.check_codes(sign, ref, y, sc)
+
+
+def test_mxfp4_rule_accepts_the_oracle_and_catches_planted_deviations():
+    inp = synth.compress_inputs(1, 64, 4, True, seed=5, dim=128)
+    kf, ks, y = oracle.compress_index_keys(inp["a"], inp["za"], inp["bias"], 4, True, 128,
+                                           b=inp["b"], zb=inp["zb"])
+    rows = np.arange(16)
+    sf = np.array([[ks[0, oracle.key_sf_offset(r, s)] for s in range(4)] for r in rows])
+    codes = compare.unpack_nibbles(kf[0, rows]).reshape(-1, 32)
+    yb = y[0].reshape(-1, 32)
+    assert compare.check_mxfp4(codes, codes, sf.reshape(-1), sf.reshape(-1), yb) == 0
+    # an element moved to the next code although the value is nowhere near a midpoint
+    X = np.ldexp(1.0, sf.reshape(-1).astype(np.int64) - 127)[:, None]
+    r = np.abs(yb / X)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    far = np.min(np.abs(r[..., None] - mids), axis=-1) > 0.1
+    blk, el = np.argwhere(far & (codes & 7 < 7) & (codes & 7 > 0))[0]
+    bad = codes.copy()
+    bad[blk, el] += 1
+    with pytest.raises(AssertionError, match="E2M1"):
+        compare.check_mxfp4(bad, codes, sf.reshape(-1), sf.reshape(-1), yb)
+    # a scale one step off on a block whose maximum is not a power of two
+    sfb = sf.reshape(-1).copy()
+    amax = np.abs(yb).max(axis=1)
+    i = int(np.argmax(np.abs(np.log2(amax) - np.round(np.log2(amax))) > 0.1))
+    sfb[i] += 1
+    with pytest.raises(AssertionError, match="scale"):
+        compare.check_mxfp4(codes, codes, sfb, sf.reshape(-1), yb)
+    # at an exact midpoint both neighbours pass
+    mid = yb.copy()
+    mid[0, 0] = 1.25 * X[0, 0]
+    two = codes.copy()
+    two[:1, :1] = 2
+    three = codes.copy()
+    three[:1, :1] = 3
+    assert compare.check_mxfp4(three, two, sf.reshape(-1), sf.reshape(-1), mid) <= 1

@@ -87,9 +87,6 @@ def test_compress_workload0_full():
 
 
 # ------------------------------------------------------- indexer-key compression
-_E2M1_MIDS = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
-
-
 @pytest.mark.parametrize("B,T,m,pos0", [
     (2, 4 * 37 + 3, 4, 0),      # ragged tail, first entry without a previous block
     (1, 4 * 64, 4, 4096),       # previous block from the caller's tail
@@ -109,28 +106,16 @@ def test_index_key_compression_matches_oracle(B, T, m, pos0):
         inp["a"], inp["za"], inp["bias"], m, True, Nmax, b=inp["b"], zb=inp["zb"], pos0=pos0,
         prev_b=inp.get("prev_b"), prev_zb=inp.get("prev_zb"))
     np.testing.assert_allclose(dbg, oy, rtol=1e-5, atol=1e-5)
-    flips = 0
     n0 = pos0 // m
+    rows = np.arange(n0, n0 + N)
+    flips = 0
     for bb in range(B):
-        for i in range(N):
-            row = n0 + i
-            g = np.stack([kf[bb, row] & 15, kf[bb, row] >> 4], axis=1).reshape(128)
-            o = np.stack([okf[bb, row] & 15, okf[bb, row] >> 4], axis=1).reshape(128)
-            for sblk in range(4):
-                off = oracle.key_sf_offset(row, sblk)
-                y = oy[bb, i, 32 * sblk:32 * sblk + 32]
-                amax = np.abs(y).max()
-                if ks[bb, off] != oks[bb, off]:  # only at a power-of-two block maximum
-                    assert amax > 0 and abs(np.log2(amax) - np.round(np.log2(amax))) < 1e-6
-                    flips += 1
-                    continue
-                d = g[32 * sblk:32 * sblk + 32] != o[32 * sblk:32 * sblk + 32]
-                if d.any():
-                    X = 2.0 ** (int(oks[bb, off]) - 127)
-                    r = np.abs(y[d]) / X
-                    near = np.min(np.abs(r[:, None] - _E2M1_MIDS[None, :]), axis=1) <= 1e-5 * r
-                    assert near.all(), f"entry {row} block {sblk}: code differs off a midpoint"
-                    flips += int(d.sum())
+        sf_g = np.array([[ks[bb, oracle.key_sf_offset(r, s)] for s in range(4)] for r in rows])
+        sf_o = np.array([[oks[bb, oracle.key_sf_offset(r, s)] for s in range(4)] for r in rows])
+        flips += compare.check_mxfp4(
+            compare.unpack_nibbles(kf[bb, rows]).reshape(-1, 32),
+            compare.unpack_nibbles(okf[bb, rows]).reshape(-1, 32), sf_g.reshape(-1),
+            sf_o.reshape(-1), oy[bb].reshape(-1, 32), what=f"index keys seq {bb}")
     assert flips <= max(2, N * B // 500)
 
 
@@ -150,25 +135,10 @@ def test_indexer_query_matches_oracle(T, r, H_I):
     qf, qs, dbg = host(qf), host(qs), host(dbg)
     of, os_, y = oracle.indexer_query(c, W, H_I)
     np.testing.assert_allclose(dbg, y, rtol=1e-4, atol=1e-4)
-    flips = 0
-    for t in range(T):
-        for h in range(H_I):
-            g = np.stack([qf[t, h] & 15, qf[t, h] >> 4], axis=1).reshape(128)
-            o = np.stack([of[t, h] & 15, of[t, h] >> 4], axis=1).reshape(128)
-            for sblk in range(4):
-                yb = y[t, h * 128 + 32 * sblk:h * 128 + 32 * sblk + 32]
-                if qs[t, h, sblk] != os_[t, h, sblk]:
-                    amax = np.abs(yb).max()
-                    assert abs(np.log2(amax) - np.round(np.log2(amax))) < 1e-5
-                    flips += 1
-                    continue
-                d = g[32 * sblk:32 * sblk + 32] != o[32 * sblk:32 * sblk + 32]
-                if d.any():
-                    X = 2.0 ** (int(os_[t, h, sblk]) - 127)
-                    rr = np.abs(yb[d]) / X
-                    near = np.min(np.abs(rr[:, None] - _E2M1_MIDS[None, :]), axis=1) <= 1e-4 * rr
-                    assert near.all(), f"token {t} head {h} block {sblk}: code off a midpoint"
-                    flips += int(d.sum())
+    flips = compare.check_mxfp4(compare.unpack_nibbles(qf).reshape(-1, 32),
+                                compare.unpack_nibbles(of).reshape(-1, 32), qs.reshape(-1),
+                                os_.reshape(-1), y.reshape(-1, 32), mid_rel=1e-4,
+                                sf_rel=1e-5, what="indexer queries")
     assert flips <= max(4, T * H_I * 128 // 2000)
 
 

@@ -31,7 +31,7 @@ def _gpu():
     csa.lib()
 
 
-def run_prefill(inp, k, derotate=True):
+def run_prefill(inp, k, derotate=True, strict=False):
     kv, sc = dev(inp["kv"]), dev(inp["kv_scale"])
     opt = {x: dev(inp[x]) for x in ("prev_b", "prev_zb", "norm_w") if x in inp}
     if inp["P"] > 0:
@@ -41,7 +41,8 @@ def run_prefill(inp, k, derotate=True):
         inp["P"], inp["m"], k, a=dev(inp["a"]), b=dev(inp["b"]), za=dev(inp["za"]),
         zb=dev(inp["zb"]), bias=dev(inp["bias"]), kv=kv, kv_scale=sc, q_fp4=dev(inp["q_fp4"]),
         q_sf=dev(inp["q_sf"]), w=dev(inp["w"]), k_fp4=dev(inp["k_fp4"]), k_sf=dev(inp["k_sf"]),
-        q=dev(inp["q"]), sink=dev(inp["sink"]), derotate=derotate, lse=True, idx=True,
+        q=dev(inp["q"]), sink=dev(inp["sink"]), derotate=derotate,
+        strict_eligibility=strict, lse=True, idx=True,
         dev_status=st, **opt)
     torch.cuda.synchronize()
     assert int(st.item()) == 0, f"device status {int(st.item())}"
@@ -49,11 +50,11 @@ def run_prefill(inp, k, derotate=True):
                 kv_scale=host(sc))
 
 
-def check_rows(inp, k, got, rows, ora):
+def check_rows(inp, k, got, rows, ora, strict=False):
     P, m = inp["P"], inp["m"]
     flips = 0
     for i, r in enumerate(rows):
-        n = (P + r + 1) // m
+        n = (P + r + (0 if strict else 1)) // m
         s = oracle.indexer_scores(np.array([n], np.int32), inp["q_fp4"][r:r + 1],
                                   inp["q_sf"][r:r + 1], inp["w"][r:r + 1],
                                   inp["k_fp4"][None], inp["k_sf"][None])[0]
@@ -68,8 +69,18 @@ def check_cache(inp, got, ora):
     n0, n1 = P // m, (P + T) // m
     np.testing.assert_array_equal(got["kv"][:n0], inp["kv"][:n0])  # prefix rows untouched
     np.testing.assert_allclose(got["kv_scale"][n0:n1], ora["kv_scale"][n0:n1], rtol=1e-5)
-    diff = got["kv"][n0:n1] != ora["kv"][n0:n1]
-    assert diff.sum() <= max(4, diff.size // 5000), f"{diff.sum()} stored codes differ"
+    if n1 == n0:
+        return
+    # the oracle's values before quantisation: its compression of the new tokens
+    comp = oracle.compress(inp["a"][None], inp["za"][None], inp["bias"], m, True,
+                           b=inp["b"][None], zb=inp["zb"][None], pos0=P,
+                           prev_b=inp["prev_b"][None] if P else None,
+                           prev_zb=inp["prev_zb"][None] if P else None,
+                           norm_w=inp.get("norm_w"))
+    np.testing.assert_array_equal(comp["kv"][0], ora["kv"][n0:n1])
+    flips = compare.check_codes(got["kv"][n0:n1], ora["kv"][n0:n1], comp["y"][0],
+                                ora["kv_scale"][n0:n1], what="prefill cache rows")
+    assert flips <= max(4, (n1 - n0) * 576 // 5000), f"{flips} stored codes differ"
 
 
 @pytest.mark.parametrize("P,T,H,H_I,k", [
@@ -83,6 +94,22 @@ def test_prefill_small_all_rows(P, T, H, H_I, k):
     ora = oracle.prefill(inp, k, rows)
     check_cache(inp, got, ora)
     check_rows(inp, k, got, rows, ora)
+
+
+@pytest.mark.parametrize("P,T,H,H_I,k", [
+    (0, 300, 64, 16, 64),       # from an empty prefix: t = 0..3 see nothing, t = 4 block 0
+    (4096, 160, 128, 64, 1024), # n(t) = floor(t/m) around k
+])
+def test_prefill_strict_eligibility_all_rows(P, T, H, H_I, k):
+    # the reading "only blocks completed before t": n(t) = floor(t/m)
+    inp = synth.prefill_inputs(P, T, 4, H, H_I, seed=P + T + 1)
+    got = run_prefill(inp, k, strict=True)
+    rows = np.arange(T, dtype=np.int32)
+    ora = oracle.prefill(inp, k, rows, strict=True)
+    check_cache(inp, got, ora)
+    check_rows(inp, k, got, rows, ora, strict=True)
+    n = (P + rows) // 4
+    assert ((got["idx"] >= 0).sum(axis=1) == np.minimum(n, k)).all()
 
 
 def test_prefill_with_rmsnorm_weight():

@@ -1,4 +1,5 @@
-"""Decode-step state updates (csa_decode_append) against whole-stream compression."""
+"""Decode-step state updates (csa_decode_append) against the oracle's whole-stream
+compression (and the library's own whole-stream calls)."""
 
 import numpy as np
 import pytest
@@ -6,6 +7,7 @@ import torch
 
 import oracle
 from synth import inputs as synth
+from tests import compare
 
 pytestmark = pytest.mark.gpu
 
@@ -47,13 +49,34 @@ def test_token_by_token_appends_equal_whole_stream_compression(weighted):
     torch.cuda.synchronize()
     assert int(status.item()) == 0
     assert (st["n_entries"].cpu().numpy() == S // m).all()
-    # the same entries and keys as the whole-stream calls (the same block arithmetic)
+    # the entries and keys against the oracle's whole-stream compression of the same tokens
+    n = S // m
+    ora = oracle.compress(kvs["a"], kvs["za"], kvs["bias"], m, True, b=kvs["b"], zb=kvs["zb"],
+                          norm_w=w)
+    kv_h, sc_h = st["kv"].cpu().numpy(), st["kv_scale"].cpu().numpy()
+    np.testing.assert_allclose(sc_h[:, :n], ora["kv_scale"], rtol=1e-5)
+    flips = compare.check_codes(kv_h[:, :n], ora["kv"], ora["y"], ora["kv_scale"],
+                                what="appended entries")
+    assert flips <= max(4, ora["kv"].size // 5000)
+    okf, oks, oy = oracle.compress_index_keys(iks["a"], iks["za"], iks["bias"], m, True, Nmax,
+                                              b=iks["b"], zb=iks["zb"])
+    kf_h, ks_h = st["k_fp4"].cpu().numpy(), st["k_sf"].cpu().numpy()
+    rows = np.arange(n)
+    kflips = 0
+    for bb in range(B):
+        sf_g = np.array([[ks_h[bb, oracle.key_sf_offset(r, s)] for s in range(4)] for r in rows])
+        sf_o = np.array([[oks[bb, oracle.key_sf_offset(r, s)] for s in range(4)] for r in rows])
+        kflips += compare.check_mxfp4(
+            compare.unpack_nibbles(kf_h[bb, rows]).reshape(-1, 32),
+            compare.unpack_nibbles(okf[bb, rows]).reshape(-1, 32), sf_g.reshape(-1),
+            sf_o.reshape(-1), oy[bb].reshape(-1, 32), what=f"appended keys seq {bb}")
+    assert kflips <= max(2, n * B // 500)
+    # and bit for bit the same as the library's whole-stream calls (one block arithmetic)
     kv, sc, _ = csa.compress(d["a"], d["za"], d["bias"], m, True, b=d["b"], zb=d["zb"],
                              Nmax=Nmax, norm_w=w_dev)
     kf, ks, _ = csa.compress_index_keys(di["a"], di["za"], di["bias"], m, True, b=di["b"],
                                         zb=di["zb"], Nmax=Nmax)
     torch.cuda.synchronize()
-    n = S // m
     assert torch.equal(st["kv"][:, :n], kv[:, :n]) and torch.equal(st["kv_scale"][:, :n],
                                                                    sc[:, :n])
     assert torch.equal(st["k_fp4"][:, :n], kf[:, :n]) and torch.equal(st["k_sf"], ks)
