@@ -18,6 +18,10 @@ prefix (one sequence, 128 heads, indexer 64 heads, top-k 1024); one step is the 
 prefill call (compression, indexer top-k and attention for every new token).
 --workload hca times hca_attn_decode: 8 sequences at 128K context (1,024 entries each,
 64 heads), dense MQA over every entry + window + sink, graphs over 24 device copies.
+--workload flash times the same CSA decode step as the default on the V4-Flash-shaped
+workload (32 sequences of 64K-128K tokens, 64 heads, indexer 64 heads, top-k 512), and
+--workload tiny on one 8K-token sequence (64 heads, indexer 16 heads, top-k 512); each
+rotates over enough device copies that one rotation exceeds twice the L2.
 """
 
 from __future__ import annotations
@@ -594,7 +598,7 @@ def cpu_baseline_sample(d_host, w) -> dict:
     """The oracle timed on a bounded sample: 2 decode queries of the workload."""
     import oracle
     cores = os.cpu_count() or 1
-    q = 2
+    q = min(2, d_host["B"])
     t0 = time.perf_counter()
     for b in range(q):
         sl = slice(b, b + 1)
@@ -607,7 +611,18 @@ def cpu_baseline_sample(d_host, w) -> dict:
                          d_host["sink"], idx=idx)
     dt = time.perf_counter() - t0
     return {"value": q / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{q} decode queries (sequences 0-1 of the workload), fp64, all host threads"}
+            "sample": f"{q} decode queries (the first sequences of the workload), fp64, all "
+                      "host threads"}
+
+
+# CSA decode workloads timed like the default one: the workload index in synth.WORKLOADS
+# and the metric name of its line
+DECODE_MODES = {
+    "decode": (WORKLOAD_ID, METRIC),
+    "flash": (2, "CSA decode queries/s (V4-Flash-shaped: 32 sequences of 64K-128K tokens)"),
+    "tiny": (0, "CSA decode queries/s (one sequence of 8K tokens, 64 heads, k = 512)"),
+}
+L2_BYTES = 126 << 20
 
 
 def main():
@@ -617,9 +632,11 @@ def main():
     ap.add_argument("--warmup", type=int, default=500)
     ap.add_argument("--impl", default="csa", choices=["csa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--copies", type=int, default=COPIES,
-                    help="device copies of the streamed inputs rotated across steps")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "hca"])
+    ap.add_argument("--copies", type=int, default=0,
+                    help="device copies of the streamed inputs rotated across steps "
+                         "(0: enough that one rotation exceeds twice the L2)")
+    ap.add_argument("--workload", default="decode",
+                    choices=sorted(DECODE_MODES) + ["prefill", "hca"])
     args = ap.parse_args()
 
     rank = int(os.environ.get("RANK", "0"))
@@ -646,7 +663,8 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
-    w = synth.WORKLOADS[WORKLOAD_ID]
+    wid, metric = DECODE_MODES[args.workload]
+    w = synth.WORKLOADS[wid]
     d = synth.decode_inputs(w, seed=w.seed + 1000 * rank)
     B, k, Nmax = d["B"], w.k, d["Nmax"]
 
@@ -656,7 +674,8 @@ def main():
 
     streamed = ("k_fp4", "k_sf", "kv", "kv_scale", "q_fp4", "q_sf", "w", "q", "swa")
     base = {key: dev(d[key]) for key in streamed + ("n_entries", "pos", "sink")}
-    ncopy = max(1, args.copies)
+    copy_bytes = sum(base[key].numel() * base[key].element_size() for key in streamed)
+    ncopy = args.copies if args.copies > 0 else min(512, max(COPIES, -(-2 * L2_BYTES // copy_bytes)))
     copies = [base] + [{key: (base[key].clone() if key in streamed else base[key])
                         for key in base} for _ in range(ncopy - 1)]
     ws_idx = csa.indexer_topk_workspace(B, Nmax, k)
@@ -792,7 +811,7 @@ def main():
         achieved = idx_bytes / (t_idx * 1e-3) / 1e9
         traffic = ncu_traffic()
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "metric": metric, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": steps_run, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp4+fp16",
             "data": "synthetic",
@@ -800,7 +819,7 @@ def main():
                        "entries_per_seq": int(d["n_entries"][0]), "heads": w.H,
                        "indexer_heads": w.H_I, "top_k": w.k, "window": 128,
                        "l2": f"inputs rotated over {ncopy} device copies "
-                             f"({ncopy * (Nmax * 68 * B) / 1e6:.0f} MB of streamed keys)",
+                             f"({ncopy * copy_bytes / 1e6:.0f} MB of streamed inputs)",
                        "step_algorithmic_bytes": step_bytes,
                        "step_achieved_gbs": step_bytes / (ms_step * 1e-3) / 1e9,
                        "step_frac_of_peak": step_bytes / (ms_step * 1e-3) / 1e9 / pk["hbm_gbs"],

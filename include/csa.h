@@ -240,11 +240,23 @@ int csa_indexer_query(const csa_iquery_args* args, csa_stream_t stream);
  * scale of entry j (j = 128g + 32r1 + r0), block s, sits at byte 16*r0 + 4*r1 + s of
  * group g -- the tensor-core scale-factor atom, so a group is copied as is.
  * Nmax must be a multiple of 128. 1 <= k <= 2048, H_I in {16, 32, 64}.
- * The workspace must be zero-filled once before its first use; every call leaves it
- * zeroed again. One workspace serves calls of any B and Nmax up to the sizes it was
- * created for (the parts kept at zero sit at offsets that do not depend on B). Calls
- * that share a workspace must not overlap on the device.
+ * The workspace must be zero-filled once before its first use; every call that ends with
+ * dev_status still zero leaves it zeroed again. After a call that reported
+ * CSA_ERR_TIMEOUT or CSA_ERR_DEVICE (or any call whose dev_status was not read), zero-fill
+ * the workspace again before reusing it: a call that gave up part-way leaves counts
+ * behind. One workspace serves calls of any B and Nmax up to the sizes it was created
+ * for (the parts kept at zero sit at offsets that do not depend on B). Calls that share a
+ * workspace must not overlap on the device.
+ *
+ * Scoring and selection normally run in one cooperative launch with one CTA per SM and
+ * two grid-wide barriers; if the runtime refuses that launch (for instance when other
+ * work holds SMs), scoring runs as an ordinary launch followed by two selection kernels,
+ * with the same results. `flags` = CSA_TOPK_SEPARATE_SELECT takes that second path on
+ * purpose (for testing it). `select_wait_ns` bounds each wait at the grid barriers of the
+ * cooperative path (0 = 2 s); a wait that runs out writes CSA_ERR_TIMEOUT to dev_status
+ * and the call returns with its outputs undefined.
  */
+#define CSA_TOPK_SEPARATE_SELECT 1u
 typedef struct {
   int32_t B;              /* queries (one per sequence) */
   int32_t H_I;                /* indexer heads: 16, 32 or 64 */
@@ -259,6 +271,8 @@ typedef struct {
   int32_t* idx;               /* out [B][k] ascending, -1 padded */
   float* scores;              /* optional out [B][k]: score of idx[b][i] (NaN for -1) */
   int32_t* dev_status;        /* optional device word, see conventions */
+  uint32_t flags;             /* 0 or CSA_TOPK_SEPARATE_SELECT */
+  int64_t select_wait_ns;     /* limit of a grid-barrier wait in ns; 0 = the default */
 } csa_topk_args;
 
 size_t csa_indexer_topk_workspace_size(int32_t B, int64_t Nmax, int32_t k);
@@ -434,9 +448,12 @@ int csa_grouped_out_proj(const csa_oproj_args* args, void* workspace, size_t wor
  *
  * Scratch comes from one file-scope device array of CSA_NOALLOC_SCRATCH_BYTES per device
  * (12 MiB; enough for B = 4, H = 128, k = 1024). Its address is looked up with
- * cudaGetSymbolAddress on the first call on each device and cached; make that first call
- * outside stream capture (for instance one ordinary call before capturing). Nothing in
- * the scratch has to start at zero: every partial result is written before it is read.
+ * cudaGetSymbolAddress on the first call on each device and cached together with the
+ * current context; a call under another context of that device (or after the device's
+ * primary context was reset) looks it up again. Make the first call of each device and
+ * context outside stream capture (for instance one ordinary call before capturing).
+ * Nothing in the scratch has to start at zero: every partial result is written before it
+ * is read.
  *
  * Results are the same as csa_sparse_attn_decode with a caller workspace (the same
  * kernels run). Arguments are checked as there; a problem whose scratch

@@ -21,6 +21,7 @@ HEAD_DIM, NOPE_DIM, ROPE_DIM, ROW_BYTES, INDEX_DIM, WINDOW = 512, 448, 64, 576, 
 
 CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_WORKSPACE = 0, 1, 2, 3
 CSA_ERR_CUDA, CSA_ERR_DEVICE, CSA_ERR_TIMEOUT = 4, 5, 6
+TOPK_SEPARATE_SELECT = 1
 
 _vp = C.c_void_p
 
@@ -66,7 +67,7 @@ class TopkArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("H_I", C.c_int32), ("k", C.c_int32), ("Nmax", C.c_int64),
                 ("n_entries", _vp), ("q_fp4", _vp), ("q_sf", _vp), ("w", _vp),
                 ("k_fp4", _vp), ("k_sf", _vp), ("idx", _vp), ("scores", _vp),
-                ("dev_status", _vp)]
+                ("dev_status", _vp), ("flags", C.c_uint32), ("select_wait_ns", C.c_int64)]
 
 
 class AttnArgs(C.Structure):
@@ -367,9 +368,14 @@ def indexer_topk_workspace(B: int, Nmax: int, k: int, device="cuda") -> torch.Te
 
 
 def indexer_topk(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, k: int, *, workspace=None, idx=None,
-                 scores: bool = False, bf16_scores: bool = False, dev_status=None, stream=None):
+                 scores: bool = False, bf16_scores: bool = False, dev_status=None,
+                 separate_select: bool = False, select_wait_ns: int = 0, stream=None):
     """Top-k entry indices [B][k] (ascending, -1 padded) and optionally their scores.
-    bf16_scores selects on scores rounded to BF16 (csa_indexer_topk_bf16)."""
+    bf16_scores selects on scores rounded to BF16 (csa_indexer_topk_bf16).
+    separate_select runs the selection as separate kernels instead of inside the
+    cooperative scoring launch; select_wait_ns bounds that launch's grid-barrier waits
+    (0 = the library default). After a call whose dev_status reports an error, zero-fill
+    the workspace before reusing it."""
     B, H_I, _ = q_fp4.shape
     _dim(q_fp4, 2, 64, "q_fp4")
     Nmax = k_fp4.shape[1]
@@ -385,7 +391,8 @@ def indexer_topk(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, k: int, *, workspace=No
                     _ptr(q_fp4, elem=1, name="q_fp4"), _ptr(q_sf, elem=1, name="q_sf"),
                     _ptr(w, elem=4, name="w"), _ptr(k_fp4, elem=1, name="k_fp4"),
                     _ptr(k_sf, elem=1, name="k_sf"), _ptr(idx, elem=4, name="idx"),
-                    _ptr(sc, elem=4, name="scores"), _ptr(dev_status, elem=4, name="dev_status"))
+                    _ptr(sc, elem=4, name="scores"), _ptr(dev_status, elem=4, name="dev_status"),
+                    TOPK_SEPARATE_SELECT if separate_select else 0, int(select_wait_ns))
     fn = "csa_indexer_topk_bf16" if bf16_scores else "csa_indexer_topk"
     _check(getattr(lib(), fn)(C.byref(args), workspace.data_ptr(), workspace.numel(),
                               _stream(stream)), fn)

@@ -66,19 +66,49 @@ bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA; }
 
 // Scratch of csa_sparse_attn_decode_noalloc: one array per device, zero-initialised when
-// the module loads. Its device address is cached per device after the first lookup.
+// the module loads. Its device address is looked up with cudaGetSymbolAddress and cached
+// per device together with the context it belongs to: a call under another context of
+// that device (or after the primary context was reset) looks it up again.
 __device__ __align__(256) unsigned char g_noalloc_scratch[CSA_NOALLOC_SCRATCH_BYTES];
 constexpr int kMaxDevices = 64;
 
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static const CtxGetCurrentFn fn = []() -> CtxGetCurrentFn {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      return reinterpret_cast<CtxGetCurrentFn>(p);
+    return nullptr;
+  }();
+  return fn;
+}
+
 void* noalloc_scratch() {
-  static std::atomic<void*> cache[kMaxDevices];
+  struct Slot {
+    std::atomic<void*> ctx{nullptr};
+    std::atomic<void*> ptr{nullptr};
+  };
+  static Slot cache[kMaxDevices];
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  void* p = cache[dev].load(std::memory_order_acquire);
-  if (!p) {
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
-    cache[dev].store(p, std::memory_order_release);
-  }
+  CtxGetCurrentFn get_ctx = ctx_get_current_fn();
+  if (!get_ctx) return nullptr;
+  CUcontext ctx = nullptr;  // null before the runtime has made its context current
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
+  Slot& s = cache[dev];
+  void* p = s.ptr.load(std::memory_order_acquire);
+  if (ctx && p && s.ctx.load(std::memory_order_acquire) == (void*)ctx) return p;
+  p = nullptr;  // the lookup also sets up the runtime's context when it is not yet current
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) return nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return nullptr;
+  // both words are rewritten on a change of context; a thread that reads a mixed pair
+  // looks the address up again, which returns the same value
+  s.ptr.store(nullptr, std::memory_order_release);
+  s.ctx.store((void*)ctx, std::memory_order_release);
+  s.ptr.store(p, std::memory_order_release);
   return p;
 }
 
@@ -305,7 +335,9 @@ size_t csa_indexer_topk_workspace_size(int32_t B, int64_t Nmax, int32_t k) {
 static int indexer_common(const csa_topk_args* a, void* ws, size_t ws_bytes,
                           csa_stream_t stream, int bf16) {
   if (!a) return CSA_ERR_INVALID_ARG;
-  if (a->B < 0 || a->k < 1 || a->Nmax < 0 || a->Nmax % 128 != 0) return CSA_ERR_INVALID_ARG;
+  if (a->B < 0 || a->k < 1 || a->Nmax < 0 || a->Nmax % 128 != 0 ||
+      (a->flags & ~CSA_TOPK_SEPARATE_SELECT) || a->select_wait_ns < 0)
+    return CSA_ERR_INVALID_ARG;
   if (a->H_I != 16 && a->H_I != 32 && a->H_I != 64) return CSA_ERR_UNSUPPORTED;
   if (a->k > 2048 || a->B > 1024 || a->Nmax > ((int64_t)1 << 30)) return CSA_ERR_UNSUPPORTED;
   if (a->B == 0) return CSA_OK;
@@ -322,14 +354,15 @@ static int indexer_common(const csa_topk_args* a, void* ws, size_t ws_bytes,
   if (a->Nmax == 0) {
     // no entry can be eligible: the select pass alone writes the -1 padding
   }
+  // the keys as [B][Nmax/128 tiles][128 entries][64 bytes], read four tiles per copy
   CUtensorMap kmap;
   std::memset(&kmap, 0, sizeof(kmap));
   if (a->Nmax > 0) {
-    const cuuint64_t dims[3] = {64, (cuuint64_t)a->Nmax, (cuuint64_t)a->B};
-    const cuuint64_t strides[2] = {64, (cuuint64_t)a->Nmax * 64};
-    const cuuint32_t box[3] = {64, 128, 1};
-    const cuuint32_t estr[3] = {1, 1, 1};
-    if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<uint8_t*>(a->k_fp4), dims,
+    const cuuint64_t dims[4] = {64, 128, (cuuint64_t)(a->Nmax / 128), (cuuint64_t)a->B};
+    const cuuint64_t strides[3] = {64, 128 * 64, (cuuint64_t)a->Nmax * 64};
+    const cuuint32_t box[4] = {64, 128, 4, 1};
+    const cuuint32_t estr[4] = {1, 1, 1, 1};
+    if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(a->k_fp4), dims,
             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return CSA_ERR_CUDA;

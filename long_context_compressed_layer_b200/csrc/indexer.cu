@@ -36,61 +36,46 @@ namespace csa {
 
 constexpr int kIxTile = 128;        // entries per tile = MMA M
 constexpr int kIxN = 64;            // MMA N: indexer heads padded to 64
-// One CTA per SM holding two independent pipelines (each: a TMA producer warp, a tcgen05
-// issuer warp and four epilogue warps, its own shared-memory ring and half of TMEM), so
-// that every SM streams with two producers and two issuers while the whole grid stays
-// resident for the cooperative launch that also runs the selection.
-constexpr int kIxPipes = 2;
-constexpr int kIxStages = 6;        // key tiles in flight per pipeline
-constexpr int kIxBatch = 1;         // tiles per accumulator hand-off
-constexpr int kIxNbuf = 3;          // accumulator buffers per pipeline
-constexpr int kIxAcc = kIxNbuf * kIxBatch;
-constexpr int kIxEpiWarps = 4;      // per pipeline, one per TMEM lane quadrant
-constexpr int kIxGroups = 1;
-constexpr int kIxPipeWarps = 2 + kIxEpiWarps;
-constexpr int kIxPipeCols = 256;    // TMEM columns per pipeline
-constexpr int kIxTmemCols = kIxPipes * kIxPipeCols;
-constexpr int kIxThreads = 32 * kIxPipeWarps * kIxPipes;
-static_assert(kIxAcc * 64 + 16 <= kIxPipeCols, "accumulators and scale factors fit TMEM");
+// The decode kernel: one CTA per SM (cooperative launch), one producer filling a ring of
+// key-tile quads, and three pipelines taking the tiles in turn, each an MMA issuer warp and
+// a group of four epilogue warps (see the file head).
+constexpr int kDxQuad = 4;          // key tiles per copy: one 32 KB tensor copy + 2 KB scales
+constexpr int kDxStages = 4;        // quads in flight per SM (136 KB)
+constexpr int kDxScTiles = 64;      // a CTA range of up to 64 tiles keeps its scores on chip
+constexpr int kDxGroups = 3;        // pipelines: issuer warp + epilogue warp group
+constexpr int kDxBufs = 2;          // accumulators per pipeline
+constexpr int kDxAcc = kDxGroups * kDxBufs;
+constexpr int kDxWarps = 1 + 5 * kDxGroups;
+constexpr int kDxThreads = 32 * kDxWarps;
+constexpr int kDxTmemCols = 512;
+constexpr int kDxMaxCtas = 256;     // grid limit (per-CTA counts in the workspace)
+constexpr int kDxCand = 2048;       // in-bin candidates staged in shared memory
+static_assert(kDxAcc * 64 + 16 * kDxGroups <= kDxTmemCols,
+              "accumulators and scale factors fit TMEM");
 constexpr int kIxKeyBytes = kIxTile * 64;
 constexpr int kIxSfBytes = 512;
 constexpr int kHistBits = 11;       // histogram of the top key bits (sign, exponent, 2 mantissa)
 constexpr int kLowBits = 32 - kHistBits;
 constexpr int kHist = 1 << kHistBits;
 constexpr int kIxMaxB = 1024;
-constexpr int kSelThreads = kIxThreads;     // the selection runs on the scoring CTAs
+constexpr int kSelThreads = 384;            // threads of the stand-alone selection kernels
 constexpr int kSelPer = 32;                 // consecutive entries per thread
 constexpr int kSelChunk = kSelThreads * kSelPer;  // entries per slice
 
-struct alignas(1024) PipeSmem {
-  uint8_t keys[kIxStages][kIxKeyBytes];  // 1024-byte aligned tiles
-  uint8_t q[2][kIxN * 64];               // queries, 64-byte swizzle, two sequence slots
-  uint32_t hist[kIxEpiWarps][kHist / 2]; // per-warp histograms, two 16-bit bins per word
-  uint8_t ksf[kIxStages][kIxSfBytes];
-  uint8_t qsf[2][512];
-  uint64_t full[kIxStages], empty[kIxStages];
-  uint64_t acc_full[kIxNbuf], acc_empty[kIxNbuf], q_free[2], done;
-  volatile int abort;
-};
-
-struct IxSmem {
-  PipeSmem pipe[kIxPipes];
-  int32_t prefix[kIxMaxB + 1];
-  uint32_t tmem_base;
-};
-
 // Workspace layout of csa_indexer_topk (all regions 256-byte aligned). Everything that must
 // be zero when a call starts sits at the front at offsets that do not depend on B: the
-// grid barrier, then one fixed-size block per sequence (counters, rule, histogram). A call
+// grid barriers, then one fixed-size block per sequence (counters, rule, histogram). A call
 // with fewer sequences therefore finds its blocks where a larger call left them zeroed.
 constexpr int kSeqWords = 8 + kHist;  // per-sequence block: counters[4], rule[4], hist
 
 struct IxWs {
-  uint32_t* grid_bar;   // [2]: arrival count, generation (grid-wide barrier)
+  uint32_t* grid_bar;   // two 64-bit arrival counters of the grid barriers
   uint32_t* seq;        // [B][kSeqWords]
   uint32_t* slice_cnt;  // [B][S]: above-bin count per slice, then the slice's output offset
   float* scores;        // [B][Nmax]
   uint64_t* cand;       // [B][Nmax]: (key << 32) | index of the in-bin candidates
+  uint4* cta_cnt;       // [B][kDxMaxCtas]: per CTA (above-bin count, in-bin count, bin)
+  uint64_t* cand_slots; // [B][kDxMaxCtas][32]: per CTA its first in-bin candidates
   int S;                // slices per sequence
   // counters: candidate count, ticket; rule: cut key, cut index, selected count, ready flag
   __device__ uint32_t* counters(int b) const { return seq + (size_t)b * kSeqWords; }
@@ -121,12 +106,16 @@ __host__ __device__ inline size_t ix_ws_layout(int B, int64_t Nmax, int k, char*
   char* p2 = take((size_t)B * S * 4);
   char* p3 = take((size_t)B * Nmax * 4);
   char* p4 = take((size_t)B * Nmax * 8);
+  char* p5 = take((size_t)B * kDxMaxCtas * sizeof(uint4));
+  char* p6 = take((size_t)B * kDxMaxCtas * 32 * sizeof(uint64_t));
   if (ws) {
     ws->grid_bar = (uint32_t*)p0;
     ws->seq = (uint32_t*)p1;
     ws->slice_cnt = (uint32_t*)p2;
     ws->scores = (float*)p3;
     ws->cand = (uint64_t*)p4;
+    ws->cta_cnt = (uint4*)p5;
+    ws->cand_slots = (uint64_t*)p6;
     ws->S = S;
   }
   return off;
@@ -140,6 +129,7 @@ struct IxParams {
   int B, H_I, k;
   int fused;  // 1: the selection follows in this (cooperative) launch
   int bf16;   // 1: scores are rounded to BF16 before they are stored and selected
+  uint64_t wait_ns;  // limit of the selection's grid-barrier waits
   int64_t Nmax;
   const int32_t* n_entries;
   const uint8_t* q_fp4;
@@ -160,144 +150,202 @@ __device__ __forceinline__ int clamp_n(int n, int64_t Nmax, int32_t* st) {
   return n;
 }
 
-__device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
-                                            const CUtensorMap& kmap, const IxParams& p,
-                                            const int g0, const int g1, const uint32_t tmem,
-                                            const uint32_t t_sfa, const uint32_t t_sfb,
-                                            const int wp);
-__device__ void select_fused(const IxParams& p, uint8_t* scratch);
+struct alignas(1024) DxSmem {
+  uint8_t keys[kDxStages][kDxQuad][kIxKeyBytes];  // quads of key tiles (64-byte swizzle)
+  uint8_t q[kDxGroups][2][kIxN * 64];     // queries (B operand) per pipeline, two slots
+  float sc[kDxScTiles * kIxTile];         // the CTA's scores (fused path, small ranges)
+  uint8_t ksf[kDxStages][kDxQuad][kIxSfBytes];  // key scale groups
+  uint8_t qsf[kDxGroups][2][512];         // query scale atoms
+  uint32_t hist[kDxGroups][kHist / 2];    // per-group histograms, two 16-bit bins per word
+  alignas(16) float w[kDxGroups][2][kIxN];  // head weights of each group's sequence (read
+                                            // as float4)
+  int32_t qprefix[kIxMaxB + 1];           // quads of sequences 0 .. b-1
+  int32_t tiles[kIxMaxB];                 // tiles of sequence b: ceil(n_b / 128)
+  uint64_t full[kDxStages], empty[kDxStages];
+  uint64_t acc_full[kDxAcc], acc_empty[kDxAcc], q_free[kDxGroups][2], done[kDxGroups];
+  uint64_t grp_bar[kDxGroups];            // the four warps of a group meet around a flush
+  int32_t grp_seq[kDxGroups];             // sequence whose counts a group histogram holds
+  uint32_t tmem_base;
+  volatile int abort;
+};
+// dynamic shared memory (+1 KB for alignment) and the static kilobyte of the helpers fit
+// the 227 KB a CTA may hold
+static_assert(sizeof(DxSmem) + 2048 <= 232448, "decode kernel shared memory");
+static_assert(offsetof(DxSmem, w) % 16 == 0 && offsetof(DxSmem, q) % 1024 == 0 &&
+                  offsetof(DxSmem, keys) % 1024 == 0 && offsetof(DxSmem, ksf) % 16 == 0 &&
+                  offsetof(DxSmem, qsf) % 16 == 0 && offsetof(DxSmem, hist) % 16 == 0 &&
+                  offsetof(DxSmem, sc) % 16 == 0,
+              "vector and bulk-copy fields of the decode kernel's shared memory are aligned");
 
-__global__ void __launch_bounds__(kIxThreads, 1)
-    indexer_score_kernel(const __grid_constant__ CUtensorMap kmap, IxParams p) {
+__device__ void select_decode(const IxParams& p, uint8_t* scratch, const DxSmem& s, int q0,
+                              int q1, bool on_chip, bool ok);
+
+// Adds a histogram of two 16-bit bins per word to sequence bb's global histogram: lanes
+// [from, from + stride) of the calling threads take every stride-th word.
+__device__ __forceinline__ void hist_flush(uint32_t* h, uint32_t* gh, int from, int stride) {
+  for (int i = from; i < kHist / 2; i += stride) {
+    const uint32_t v = h[i];
+    if (v) {
+      if (v & 0xFFFFu) atomicAdd(gh + 2 * i, v & 0xFFFFu);
+      if (v >> 16) atomicAdd(gh + 2 * i + 1, v >> 16);
+      h[i] = 0;
+    }
+  }
+}
+
+// The four warps of an epilogue group meet on an mbarrier (bounded wait): lane 0 of each
+// warp arrives, then waits for the phase to complete. The warp synchronises first, so the
+// shared-memory writes of all its lanes are ordered before lane 0's arrival (a release)
+// and visible to the warps that return from the wait (an acquire).
+__device__ __forceinline__ bool group_meet(uint64_t* bar, uint32_t& phase, int32_t* st) {
+  bool ok = true;
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) {
+    mbar_arrive(bar);
+    ok = mbar_wait(bar, phase, st);
+  }
+  phase ^= 1;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// The CTA's tiles in order: quads q0 .. q1-1 (quad q of sequence b = the tiles 4(q - qprefix[b])
+// .. +3 that exist), numbered it = 0, 1, ... over the CTA. Calls f(b, t, it, qq, sub, nt):
+// sequence, tile within the sequence, CTA tile index, CTA quad index, slot in the quad,
+// tiles in the quad. Stops early when f returns false.
+template <typename F>
+__device__ __forceinline__ void for_each_tile(const DxSmem& s, int q0, int q1, int b0, F&& f) {
+  int b = b0, it = 0;
+  for (int q = q0, qq = 0; q < q1; ++q, ++qq) {
+    while (s.qprefix[b + 1] <= q) ++b;
+    const int t0 = kDxQuad * (q - s.qprefix[b]);
+    const int nt = min(kDxQuad, s.tiles[b] - t0);
+    for (int sub = 0; sub < nt; ++sub, ++it)
+      if (!f(b, t0 + sub, it, qq, sub, nt)) return;
+  }
+}
+
+__global__ void __launch_bounds__(kDxThreads, 1)
+    indexer_decode_kernel(const __grid_constant__ CUtensorMap kmap, IxParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
-  IxSmem& s = *reinterpret_cast<IxSmem*>(
+  DxSmem& s = *reinterpret_cast<DxSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int pi = warp / kIxPipeWarps, wp = warp % kIxPipeWarps;  // pipeline, warp in it
-  PipeSmem& ps = s.pipe[pi];
   // set-up that touches no global memory overlaps the previous kernel's tail
-  if (wp == 1 && lane == 0) {
-    for (int i = 0; i < kIxStages; ++i) {
-      mbar_init(&ps.full[i], 1);
-      mbar_init(&ps.empty[i], 1);
+  if (warp == 1 && lane == 0) {
+    for (int i = 0; i < kDxStages; ++i) {
+      mbar_init(&s.full[i], 1);
+      mbar_init(&s.empty[i], kDxQuad);  // one MMA commit per tile of the quad
     }
-    for (int i = 0; i < kIxNbuf; ++i) {
-      mbar_init(&ps.acc_full[i], 1);
-      mbar_init(&ps.acc_empty[i], kIxEpiWarps);
+    for (int i = 0; i < kDxAcc; ++i) {
+      mbar_init(&s.acc_full[i], 1);
+      mbar_init(&s.acc_empty[i], 4);
     }
-    for (int i = 0; i < 2; ++i) mbar_init(&ps.q_free[i], 1);
-    mbar_init(&ps.done, 1);
-    ps.abort = 0;
+    for (int i = 0; i < kDxGroups; ++i) {
+      mbar_init(&s.q_free[i][0], 1);
+      mbar_init(&s.q_free[i][1], 1);
+      mbar_init(&s.grp_bar[i], 4);
+      mbar_init(&s.done[i], 1);
+    }
+    s.abort = 0;
     mbar_fence_init();
   }
   if (threadIdx.x == 0) prefetch_tensormap(&kmap);
-  {
-    uint32_t* hz = &ps.hist[0][0];
-    for (int i = threadIdx.x % (32 * kIxPipeWarps); i < kIxEpiWarps * kHist / 2; i += 32 * kIxPipeWarps)
-      hz[i] = 0;
-  }
-  if (warp == 1) tmem_alloc(&s.tmem_base, kIxTmemCols);
+  for (int i = threadIdx.x; i < kDxGroups * kHist / 2; i += kDxThreads) (&s.hist[0][0])[i] = 0;
+  if (threadIdx.x < kDxGroups) s.grp_seq[threadIdx.x] = -1;
+  if (warp == 1) tmem_alloc(&s.tmem_base, kDxTmemCols);
   pdl_wait();
   pdl_trigger();
 
-  // Tile schedule: sequence b owns ceil(n_b / 128) tiles; CTA c takes a contiguous range.
+  // Schedule: sequence b owns ceil(n_b / 128) tiles in ceil(tiles / 4) quads; CTA c takes a
+  // contiguous range of quads.
   if (warp == 0) {
     int carry = 0;
-    if (lane == 0) s.prefix[0] = 0;
+    if (lane == 0) s.qprefix[0] = 0;
     for (int base = 0; base < p.B; base += 32) {
       const int bb = base + lane;
       int v = 0;
-      if (bb < p.B) v = (clamp_n(p.n_entries[bb], p.Nmax, p.dev_status) + kIxTile - 1) / kIxTile;
+      if (bb < p.B) {
+        const int t = (clamp_n(p.n_entries[bb], p.Nmax, p.dev_status) + kIxTile - 1) / kIxTile;
+        s.tiles[bb] = t;
+        v = (t + kDxQuad - 1) / kDxQuad;
+      }
       int incl = v;
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, incl, o);
         if (lane >= o) incl += y;
       }
-      if (bb < p.B) s.prefix[bb + 1] = carry + incl;
+      if (bb < p.B) s.qprefix[bb + 1] = carry + incl;
       carry += __shfl_sync(0xffffffffu, incl, 31);
     }
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  const int total = s.prefix[p.B];
-  const int g0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
-  const int g1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
+  const int total = s.qprefix[p.B];
+  const int q0 = (int)((int64_t)total * blockIdx.x / gridDim.x);
+  const int q1 = (int)((int64_t)total * (blockIdx.x + 1) / gridDim.x);
   const uint32_t tmem = s.tmem_base;
-  {  // the pipelines split the CTA's tiles into two contiguous halves
-    const int gm = g0 + (g1 - g0 + 1) / 2;
-    const int pg0 = pi == 0 ? g0 : gm, pg1 = pi == 0 ? gm : g1;
-    const uint32_t tp = tmem + pi * kIxPipeCols;
-    const uint32_t t_sfa = tp + kIxAcc * kIxN, t_sfb = t_sfa + 8;
-    if (pg0 < pg1) score_roles(ps, s.prefix, kmap, p, pg0, pg1, tp, t_sfa, t_sfb, wp);
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc(tmem, kIxTmemCols);
-  }
-  if (p.fused) select_fused(p, reinterpret_cast<uint8_t*>(&s.pipe[0].keys[0][0]));
-}
+  // fused path with a short range: scores stay in shared memory
+  const bool on_chip = p.fused && (q1 - q0) * kDxQuad <= kDxScTiles;
+  int b0 = 0;  // first sequence of this CTA
+  while (b0 < p.B && s.qprefix[b0 + 1] <= q0) ++b0;
 
-// The three warp roles of one pipeline over its tiles [g0, g1); wp is the warp's index in
-// the pipeline (0 producer, 1 tcgen05 issuer, 2.. epilogue).
-__device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
-                                            const CUtensorMap& kmap, const IxParams& p,
-                                            const int g0, const int g1, const uint32_t tmem,
-                                            const uint32_t t_sfa, const uint32_t t_sfb,
-                                            const int wp) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-  // first sequence of this CTA
-  int b0 = 0;
-  while (prefix[b0 + 1] <= g0) ++b0;
-
-  if (wp == 0) {
+  if (q0 < q1 && warp == 0) {
     // ---------------------------------------------------------------- producer
     if (lane == 0) {
-      int b = b0, it = 0;
-      for (int g = g0; g < g1; ++g, ++it) {
-        while (prefix[b + 1] <= g) ++b;
-        const int t = g - prefix[b];
-        const int st = it % kIxStages;
-        if (s.abort || !mbar_wait(&s.empty[st], ((it / kIxStages) & 1) ^ 1, p.dev_status)) {
+      int b = b0, qq = 0;
+      const int groups = (int)(p.Nmax / kIxTile);
+      for (int q = q0; q < q1; ++q, ++qq) {
+        while (s.qprefix[b + 1] <= q) ++b;
+        const int t0 = kDxQuad * (q - s.qprefix[b]);
+        const int st = qq % kDxStages;
+        if (s.abort || !mbar_wait(&s.empty[st], ((qq / kDxStages) & 1) ^ 1, p.dev_status)) {
           s.abort = 1;
           break;
         }
-        mbar_arrive_expect_tx(&s.full[st], kIxKeyBytes + kIxSfBytes);
-        tma_load_3d(s.keys[st], &kmap, &s.full[st], 0, t * kIxTile, b);
-        bulk_load(s.ksf[st], p.k_sf + ((size_t)b * (p.Nmax / kIxTile) + t) * kIxSfBytes,
-                  kIxSfBytes, &s.full[st]);
+        // the quad's four key tiles in one tensor copy (tiles past Nmax read as zeros;
+        // tiles past n_b are read but not scored) and the scale groups that exist
+        const uint32_t sf_bytes = (uint32_t)min(kDxQuad, groups - t0) * kIxSfBytes;
+        mbar_arrive_expect_tx(&s.full[st], kDxQuad * kIxKeyBytes + sf_bytes);
+        tma_load_4d(&s.keys[st][0][0], &kmap, &s.full[st], 0, 0, t0, b);
+        bulk_load(&s.ksf[st][0][0], p.k_sf + ((size_t)b * groups + t0) * kIxSfBytes, sf_bytes,
+                  &s.full[st]);
       }
       // drain: every copy this warp issued has landed before the CTA winds down
-      const int issued = it;
-      for (int i = issued - kIxStages < 0 ? 0 : issued - kIxStages; i < issued; ++i)
-        mbar_wait(&s.full[i % kIxStages], (i / kIxStages) & 1, p.dev_status);
+      const int issued = qq;
+      for (int i = issued - kDxStages < 0 ? 0 : issued - kDxStages; i < issued; ++i)
+        mbar_wait(&s.full[i % kDxStages], (i / kDxStages) & 1, p.dev_status);
     }
-  } else if (wp == 1) {
-    // ---------------------------------------------------------------- MMA issuer
-    int b = -1, nseq = -1, it = 0;
+    __syncwarp();  // the warp reaches the CTA barrier below converged
+  } else if (q0 < q1 && warp <= kDxGroups) {
+    // ---------------------------------------------------------------- MMA issuers
+    // issuer pi takes the tiles it = pi, pi + 3, ... into its pipeline's two accumulators;
+    // its key and query scale factors have TMEM columns of their own
+    const int pi = warp - 1;
+    const uint32_t t_sfa = tmem + kDxAcc * kIxN + 16 * pi, t_sfb = t_sfa + 8;
+    int cur = -1, nseq = -1;
     uint32_t qslot = 0;
-    for (int g = g0; g < g1; ++g, ++it) {
-      int nb = b < 0 ? b0 : b;
-      while (prefix[nb + 1] <= g) ++nb;
-      if (nb != b) {  // stage this sequence's queries (B operand) and their scales
-        if (b >= 0 && lane == 0) mma_commit(&s.q_free[qslot]);
-        b = nb;
+    for_each_tile(s, q0, q1, b0, [&](int b, int t, int it, int qq, int sub, int nt) -> bool {
+      (void)t;
+      if (it % kDxGroups != pi) return true;
+      const int u = it / kDxGroups;
+      if (b != cur) {  // stage this sequence's queries (B operand) and their scales
+        if (cur >= 0 && lane == 0) mma_commit(&s.q_free[pi][qslot]);
+        cur = b;
         ++nseq;
         qslot = nseq & 1;
         bool ok = true;
-        if (lane == 0) ok = !s.abort && mbar_wait(&s.q_free[qslot], ((nseq >> 1) & 1) ^ 1,
+        if (lane == 0) ok = !s.abort && mbar_wait(&s.q_free[pi][qslot], ((nseq >> 1) & 1) ^ 1,
                                                   p.dev_status);
         ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) { s.abort = 1; break; }
+        if (!ok) { s.abort = 1; return false; }
         const uint8_t* qsrc = p.q_fp4 + (size_t)b * p.H_I * 64;
+        uint8_t* qdst = s.q[pi][qslot];
         for (int c = lane; c < kIxN * 4; c += 32) {  // 16-byte chunks, 64-byte swizzle
           const int r = c >> 2, ch = c & 3;
           uint4 v = make_uint4(0, 0, 0, 0);
           if (r < p.H_I) v = *reinterpret_cast<const uint4*>(qsrc + r * 64 + ch * 16);
-          *reinterpret_cast<uint4*>(&s.q[qslot][r * 64 + ((ch ^ ((r >> 1) & 3)) << 4)]) = v;
+          *reinterpret_cast<uint4*>(&qdst[r * 64 + ((ch ^ ((r >> 1) & 3)) << 4)]) = v;
         }
         {  // scale atom: lane r0 holds the 4 scales of heads r0, r0+32, r0+64, r0+96
           uint32_t wv[4];
@@ -308,135 +356,161 @@ __device__ __forceinline__ void score_roles(PipeSmem& s, const int32_t* prefix,
                         ? *reinterpret_cast<const uint32_t*>(p.q_sf + ((size_t)b * p.H_I + n) * 4)
                         : 0x7F7F7F7Fu;
           }
-          *reinterpret_cast<uint4*>(&s.qsf[qslot][lane * 16]) = make_uint4(wv[0], wv[1], wv[2], wv[3]);
+          *reinterpret_cast<uint4*>(&s.qsf[pi][qslot][lane * 16]) =
+              make_uint4(wv[0], wv[1], wv[2], wv[3]);
         }
         fence_async_smem();
         __syncwarp();
         if (lane == 0) {
           tc_fence_after();
-          tmem_cp_32x128b_x4(t_sfb, smem_desc(smem_u32(s.qsf[qslot]), 0, 128, kSwizzleNone));
+          tmem_cp_32x128b_x4(t_sfb, smem_desc(smem_u32(s.qsf[pi][qslot]), 0, 128, kSwizzleNone));
         }
       }
       if (lane == 0) {
-        // tile it goes to accumulator a of batch bt = it / kIxBatch, buffer bb
-        const int st = it % kIxStages, bt = it / kIxBatch, bb = bt % kIxNbuf;
-        const int a = bb * kIxBatch + it % kIxBatch;
+        const int st = qq % kDxStages, buf = pi * kDxBufs + (u & 1);
         bool ok = !s.abort;
-        if (ok && it % kIxBatch == 0) {  // first tile of a batch: its buffer must be free
-          ok = mbar_wait(&s.acc_empty[bb], ((bt / kIxNbuf) & 1) ^ 1, p.dev_status);
+        if (ok) {
+          ok = mbar_wait(&s.acc_empty[buf], ((u >> 1) & 1) ^ 1, p.dev_status);
           // the epilogue's TMEM reads of this buffer happen before our MMAs overwrite it
           tc_fence_after();
         }
         // (the key tile arrives through the async proxy: the barrier alone orders it)
-        ok = ok && mbar_wait(&s.full[st], (it / kIxStages) & 1, p.dev_status);
+        ok = ok && mbar_wait(&s.full[st], (qq / kDxStages) & 1, p.dev_status);
         if (!ok) {
           s.abort = 1;
         } else {
-          tmem_cp_32x128b_x4(t_sfa, smem_desc(smem_u32(s.ksf[st]), 0, 128, kSwizzleNone));
-          const uint32_t ka = smem_u32(s.keys[st]), qa = smem_u32(s.q[qslot]);
+          tmem_cp_32x128b_x4(t_sfa, smem_desc(smem_u32(s.ksf[st][sub]), 0, 128, kSwizzleNone));
+          const uint32_t ka = smem_u32(s.keys[st][sub]), qa = smem_u32(s.q[pi][qslot]);
 #pragma unroll
           for (int kh = 0; kh < 2; ++kh) {
-            mma_mxf4(tmem + a * kIxN, smem_desc(ka + 32 * kh, 16, 512, kSwizzle64B),
+            mma_mxf4(tmem + buf * kIxN, smem_desc(ka + 32 * kh, 16, 512, kSwizzle64B),
                      smem_desc(qa + 32 * kh, 16, 512, kSwizzle64B),
                      idesc_mxf4(kIxTile, kIxN, 2 * kh), t_sfa, t_sfb, kh);
           }
-          mma_commit(&s.empty[st]);
-          // last tile of the batch (or of this CTA): hand the batch to the epilogue
-          if (it % kIxBatch == kIxBatch - 1 || g + 1 == g1) mma_commit(&s.acc_full[bb]);
+          // the stage is free once the MMAs of all its tiles have read it: one arrival per
+          // tile, and the last tile of a short quad also stands in for the missing ones
+          const int arrivals = sub == nt - 1 ? 1 + kDxQuad - nt : 1;
+          for (int a = 0; a < arrivals; ++a) mma_commit(&s.empty[st]);
+          mma_commit(&s.acc_full[buf]);
         }
       }
-      if (__shfl_sync(0xffffffffu, s.abort, 0)) break;
-    }
-    if (lane == 0) {  // every tcgen05 operation of this CTA has completed
-      mma_commit(&s.done);
-      mbar_wait(&s.done, 0, p.dev_status);
+      return __shfl_sync(0xffffffffu, s.abort, 0) == 0;
+    });
+    if (lane == 0) {  // every tcgen05 operation of this issuer has completed
+      mma_commit(&s.done[pi]);
+      mbar_wait(&s.done[pi], 0, p.dev_status);
     }
     __syncwarp();
-  } else {
+  } else if (q0 < q1) {
     // ---------------------------------------------------------------- epilogue
-    const int ew = wp - 2;              // epilogue warp of this pipeline
-    const int grp = ew >> 2;            // takes the batches bt with bt % kIxGroups == grp
-    const int quad = warp & 3;          // TMEM lane quadrant
-    const int row = quad * 32 + lane;   // entry within the tile
-    uint32_t* hist = s.hist[ew];
-    int b = -1, n_b = 0, since_flush = 0;
-    float w[kIxN];
-    auto flush = [&](int bb) {  // warp-local: add the warp's counts to the global histogram
-      __syncwarp();
-      uint32_t* gh = p.ws.hist(bb);
-      for (int i = lane; i < kHist / 2; i += 32) {
-        const uint32_t v = hist[i];
-        if (v) {
-          if (v & 0xFFFFu) atomicAdd(gh + 2 * i, v & 0xFFFFu);
-          if (v >> 16) atomicAdd(gh + 2 * i + 1, v >> 16);
-          hist[i] = 0;
-        }
-      }
-      __syncwarp();
-    };
-    // batch bt holds tiles kIxBatch*bt .. of this CTA; group grp takes bt % kIxGroups == grp
-    const int ntiles = g1 - g0;
-    int bseq = b0;
+    const int ew = warp - 1 - kDxGroups, gi = ew >> 2;  // epilogue warp, its pipeline
+    const int quad = warp & 3;              // TMEM lane quadrant
+    const int row = quad * 32 + lane;       // entry within the tile
+    uint32_t* hist = s.hist[gi];
+    uint32_t meet_phase = 0;
+    int cur = -1, n_b = 0, since_flush = 0, wsl = 1;
     const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-    for (int bt = grp; bt * kIxBatch < ntiles; bt += kIxGroups) {
-      const int bb = bt % kIxNbuf;
+    for_each_tile(s, q0, q1, b0, [&](int b, int t, int it, int qq, int sub, int nt) -> bool {
+      (void)qq; (void)sub; (void)nt;
+      if (it % kDxGroups != gi) return true;
+      const int u = it / kDxGroups;
+      const int buf = gi * kDxBufs + (u & 1);
       bool ok = true;
-      if (lane == 0) ok = !s.abort && mbar_wait(&s.acc_full[bb], (bt / kIxNbuf) & 1, p.dev_status);
+      if (lane == 0) ok = !s.abort && mbar_wait(&s.acc_full[buf], (u >> 1) & 1, p.dev_status);
       if (!__shfl_sync(0xffffffffu, ok, 0)) {
         s.abort = 1;
-        break;
+        return false;
       }
       tc_fence_after();
-      const int it0 = bt * kIxBatch, it_end = min(ntiles, it0 + kIxBatch);
-      for (int it = it0; it < it_end; ++it) {
-        const int g = g0 + it;
-        while (prefix[bseq + 1] <= g) ++bseq;
-        // 16-bit counters: a warp adds at most 32 counts per tile, so flush every 2000
-        // tiles (< 65536 counts) as well as whenever the sequence changes
-        if (bseq != b || since_flush == 2000) {
-          if (b >= 0) flush(b);
-          since_flush = 0;
-          b = bseq;
-          n_b = clamp_n(p.n_entries[b], p.Nmax, nullptr);
-#pragma unroll
-          for (int h = 0; h < kIxN; ++h) w[h] = h < p.H_I ? __ldg(p.w + (size_t)b * p.H_I + h) : 0.f;
+      // 16-bit counters: a group adds 128 counts per tile, so flush every 400 tiles
+      // (< 65536 counts) as well as whenever the sequence changes; the group's four warps
+      // meet before the flush (all counts added) and after it (bins cleared). The head
+      // weights of a new sequence go to the other weight slot, which no warp of the group
+      // still reads once the first meeting has passed.
+      if (b != cur || since_flush == 400) {
+        if (cur >= 0) {
+          if (!group_meet(&s.grp_bar[gi], meet_phase, p.dev_status)) { s.abort = 1; return false; }
+          hist_flush(hist, p.ws.hist(cur), (ew & 3) * 32 + lane, 128);
         }
-        ++since_flush;
-        uint32_t r[2][32];
-        const uint32_t ta = lane_base + (bb * kIxBatch + (it - it0)) * kIxN;
-        tmem_ld32(ta, r[0]);
-        tmem_ld32(ta + 32, r[1]);
-        tmem_ld_wait();
-        // s = sum_h w_h * max(0, acc_h): eight independent partial sums (heads h = k mod 8)
-        // combined in a fixed tree, so the FMA latency chain is 8 deep instead of 64
-        float part[8];
-#pragma unroll
-        for (int k8 = 0; k8 < 8; ++k8) part[k8] = 0.f;
-#pragma unroll
-        for (int h = 0; h < kIxN; h += 2)  // heads h, h+1 -> partial sums h & 7, (h+1) & 7
-          fma2(part[h & 7], part[(h + 1) & 7], w[h], w[h + 1],
-               fmaxf(__uint_as_float(r[h >> 5][h & 31]), 0.f),
-               fmaxf(__uint_as_float(r[(h + 1) >> 5][(h + 1) & 31]), 0.f));
-        float sc = ((part[0] + part[1]) + (part[2] + part[3])) +
-                   ((part[4] + part[5]) + (part[6] + part[7]));
-        if (p.bf16) sc = bf16_bits_to_f32(f32_to_bf16_bits(sc));
-        const int j = (g - prefix[b]) * kIxTile + row;
-        if (j < n_b) {
-          p.ws.scores[(size_t)b * p.Nmax + j] = sc;
-          const uint32_t bin = float_key(sc) >> (32 - kHistBits);
-          atomicAdd(&hist[bin >> 1], 1u << (16 * (bin & 1)));
+        if (b != cur) {
+          wsl ^= 1;
+          if ((ew & 3) == 0)
+            for (int h = lane; h < kIxN; h += 32)
+              s.w[gi][wsl][h] = h < p.H_I ? __ldg(p.w + (size_t)b * p.H_I + h) : 0.f;
         }
+        if (!group_meet(&s.grp_bar[gi], meet_phase, p.dev_status)) { s.abort = 1; return false; }
+        since_flush = 0;
+        cur = b;
+        n_b = clamp_n(p.n_entries[cur], p.Nmax, nullptr);
       }
+      ++since_flush;
+      // s = sum_h w_h * max(0, acc_h): eight independent partial sums (heads h = k mod 8)
+      // combined in a fixed tree; all 64 columns are read before one wait
+      uint32_t r[2][32];
+      const uint32_t ta = lane_base + buf * kIxN;
+      tmem_ld32(ta, r[0]);
+      tmem_ld32(ta + 32, r[1]);
+      tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&s.acc_empty[bb]);
-    }
-    if (b >= 0) flush(b);
+      if (lane == 0) mbar_arrive(&s.acc_empty[buf]);  // TMEM reads done: buffer free
+      const float4* w4 = reinterpret_cast<const float4*>(s.w[gi][wsl]);
+      float part[8];
+#pragma unroll
+      for (int k8 = 0; k8 < 8; ++k8) part[k8] = 0.f;
+#pragma unroll
+      for (int h4 = 0; h4 < kIxN / 4; ++h4) {
+        const float4 wv = w4[h4];
+        const int h = 4 * h4;
+        fma2(part[h & 7], part[(h + 1) & 7], wv.x, wv.y,
+             fmaxf(__uint_as_float(r[h >> 5][h & 31]), 0.f),
+             fmaxf(__uint_as_float(r[(h + 1) >> 5][(h + 1) & 31]), 0.f));
+        fma2(part[(h + 2) & 7], part[(h + 3) & 7], wv.z, wv.w,
+             fmaxf(__uint_as_float(r[(h + 2) >> 5][(h + 2) & 31]), 0.f),
+             fmaxf(__uint_as_float(r[(h + 3) >> 5][(h + 3) & 31]), 0.f));
+      }
+      float sc = ((part[0] + part[1]) + (part[2] + part[3])) +
+                 ((part[4] + part[5]) + (part[6] + part[7]));
+      if (p.bf16) sc = bf16_bits_to_f32(f32_to_bf16_bits(sc));
+      const int j = t * kIxTile + row;
+      if (j < n_b) {
+        if (on_chip) s.sc[it * kIxTile + row] = sc;
+        else p.ws.scores[(size_t)cur * p.Nmax + j] = sc;
+        const uint32_t bin = float_key(sc) >> (32 - kHistBits);
+        atomicAdd(&hist[bin >> 1], 1u << (16 * (bin & 1)));
+      }
+      return true;
+    });
+    if ((ew & 3) == 0 && lane == 0) s.grp_seq[gi] = cur;
   }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kDxTmemCols);
+  }
+  // the groups' last histograms: counts of groups holding the same sequence are summed
+  // here, so each bin costs one global atomic per CTA
+  for (int gi = 0; gi < kDxGroups; ++gi) {
+    const int b = s.grp_seq[gi];
+    bool first = b >= 0;
+    for (int gj = 0; gj < gi; ++gj) first = first && s.grp_seq[gj] != b;
+    if (!first) continue;
+    uint32_t* gh = p.ws.hist(b);
+    for (int bin = threadIdx.x; bin < kHist; bin += kDxThreads) {
+      uint32_t c = 0;
+      for (int gj = gi; gj < kDxGroups; ++gj)
+        if (s.grp_seq[gj] == b) c += (s.hist[gj][bin >> 1] >> (16 * (bin & 1))) & 0xFFFFu;
+      if (c) atomicAdd(gh + bin, c);
+    }
+  }
+  const bool ok = !__syncthreads_or(s.abort);
+  if (p.fused)
+    select_decode(p, reinterpret_cast<uint8_t*>(&s.keys[0][0][0]), s, q0, q1, on_chip, ok);
 }
 
 // ------------------------------------------------------------------- select
-// Shared-memory scratch of the selection, carved from the (then idle) key ring.
+// Static shared-memory scratch of the stand-alone selection kernels.
 struct SelScratch {
   uint32_t h[kHist];
   uint64_t cand[2048];
@@ -444,12 +518,12 @@ struct SelScratch {
   int tbin, last;
   uint32_t above, prefix, rem, sum, pop;
 };
-static_assert(sizeof(SelScratch) <= sizeof(uint8_t[kIxStages][kIxKeyBytes]), "scratch fits the ring");
 constexpr uint32_t kCandStage = 2048;
 
-// Inclusive scan over the CTA (kSelThreads threads); tmp holds one word per warp.
+// Inclusive scan over the CTA (NT threads); tmp holds one word per warp.
+template <int NT = kSelThreads>
 __device__ __forceinline__ uint32_t block_incl_scan(uint32_t v, uint32_t* tmp, uint32_t* total) {
-  constexpr int nw = kSelThreads / 32;
+  constexpr int nw = NT / 32;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t y = __shfl_up_sync(0xffffffffu, v, o);
@@ -505,17 +579,19 @@ __device__ __forceinline__ uint64_t cand_at(const uint64_t* cand, uint32_t i, bo
 // `mask`, histogram the digit (field >> shift) & (2^bits - 1) and find the digit where the
 // running count (from the top when `descending`, else from the bottom) reaches *remaining.
 // Updates *prefix / *remaining (shared). Field: key = cand >> 32 (hi) or index (lo).
-__device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, bool hi,
-                           uint32_t key_eq, bool need_key_eq, uint32_t mask, int shift,
-                           int bits, bool descending, uint32_t* prefix, uint32_t* remaining,
-                           uint32_t* h, uint32_t* digit_pop = nullptr) {
+// Candidates are read through `get(i)` (the staged or global list).
+template <int NT, typename Get>
+__device__ void radix_step_g(const Get& get, uint32_t n_cand, bool hi, uint32_t key_eq,
+                             bool need_key_eq, uint32_t mask, int shift, int bits,
+                             bool descending, uint32_t* prefix, uint32_t* remaining, uint32_t* h,
+                             uint32_t* digit_pop = nullptr) {
   const int tid = threadIdx.x;
   const uint32_t nd = 1u << bits;
-  for (uint32_t i = tid; i < 256; i += kSelThreads) h[i] = 0;
+  for (uint32_t i = tid; i < nd; i += NT) h[i] = 0;
   __syncthreads();
   const uint32_t pre = *prefix;
-  for (uint32_t i = tid; i < n_cand; i += kSelThreads) {
-    const uint64_t c = cand_at(cand, i, staged);
+  for (uint32_t i = tid; i < n_cand; i += NT) {
+    const uint64_t c = get(i);
     const uint32_t key = (uint32_t)(c >> 32), ix = (uint32_t)c;
     if (need_key_eq && key != key_eq) continue;
     const uint32_t f = hi ? key : ix;
@@ -554,6 +630,15 @@ __device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, b
   __syncthreads();
 }
 
+__device__ void radix_step(const uint64_t* cand, bool staged, uint32_t n_cand, bool hi,
+                           uint32_t key_eq, bool need_key_eq, uint32_t mask, int shift,
+                           int bits, bool descending, uint32_t* prefix, uint32_t* remaining,
+                           uint32_t* h, uint32_t* digit_pop = nullptr) {
+  radix_step_g<kSelThreads>([&](uint32_t i) { return cand_at(cand, i, staged); }, n_cand, hi,
+                            key_eq, need_key_eq, mask, shift, bits, descending, prefix,
+                            remaining, h, digit_pop);
+}
+
 __device__ __forceinline__ int slices_of(int n) {
   return n == 0 ? 1 : (n + kSelChunk - 1) / kSelChunk;
 }
@@ -561,8 +646,7 @@ __device__ __forceinline__ int slices_of(int n) {
 // Phase 1 of the selection for slice sb of sequence b: the threshold bin (highest bin whose
 // suffix count reaches k), the slice's count above it and its in-bin candidates. The last
 // slice of the sequence to finish resolves the exact cut (finalize).
-__device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb,
-                                 uint32_t ready_gen) {
+__device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb) {
   const int tid = threadIdx.x;
   const int n = clamp_n(p.n_entries[b], p.Nmax, p.dev_status);
   const int k_eff = n < p.k ? n : p.k;
@@ -749,11 +833,6 @@ __device__ void select_threshold(const IxParams& p, SelScratch& x, int b, int sb
   uint32_t* gh = p.ws.hist(b);
   for (int i = tid; i < kHist; i += kSelThreads) gh[i] = 0;
   __syncthreads();
-  if (tid == 0 && p.fused) {  // publish the rule and offsets of this sequence
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(p.ws.rule(b) + 3),
-                 "r"(ready_gen)
-                 : "memory");
-  }
   __threadfence();
   __syncthreads();
 }
@@ -804,41 +883,426 @@ __device__ void select_write(const IxParams& p, SelScratch& x, int b, int sb) {
   __syncthreads();
 }
 
-// The selection inside the cooperative scoring launch: every CTA takes the slices
-// i = blockIdx.x, + gridDim.x, ... of the (sequence, slice) grid.
-__device__ void select_fused(const IxParams& p, uint8_t* scratch) {
-  SelScratch& x = *reinterpret_cast<SelScratch*>(scratch);
-  uint32_t gen;
-  if (!grid_barrier(p.ws.grid_bar, gridDim.x, p.dev_status, &gen)) return;
-  // the barrier generation is new in every call, so a flag left by an earlier call (or the
-  // zero-filled workspace) never matches it
-  const uint32_t ready_gen = gen;
-  const int items = p.B * p.ws.S;
-  for (int i = blockIdx.x; i < items; i += gridDim.x) {
-    const int b = i / p.ws.S, sb = i % p.ws.S;
-    int n = p.n_entries[b];
-    n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
-    if (sb < slices_of(n)) select_threshold(p, x, b, sb, ready_gen);
-  }
-  // phase 2 needs only its own sequence's rule: wait for its publication, not for the grid
-  for (int i = blockIdx.x; i < items; i += gridDim.x) {
-    const int b = i / p.ws.S, sb = i % p.ws.S;
-    int n = p.n_entries[b];
-    n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
-    if (sb >= slices_of(n)) continue;
-    bool ok = true;
-    if (threadIdx.x == 0) {
+// ------------------------------------------------------- decode selection (fused)
+// Grid-wide barrier of the cooperative decode launch on a 64-bit arrival counter that only
+// grows: a CTA's arrival returns the count before it, which fixes the barrier instance it
+// belongs to (all CTAs of a launch arrive once per instance), and it waits until the count
+// reaches the end of that instance. Every CTA arrives, also one that has already given
+// up, so later instances stay aligned; a CTA with ok == false does not wait. The wait is
+// bounded by limit_ns. Returns ok && the wait completed.
+__device__ bool grid_sync(unsigned long long* ctr, bool ok, uint64_t limit_ns,
+                          int32_t* dev_status) {
+  __shared__ int sh_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned long long old;
+    asm volatile("atom.add.release.gpu.global.u64 %0, [%1], 1;" : "=l"(old) : "l"(ctr) : "memory");
+    const unsigned long long G = gridDim.x;
+    const unsigned long long target = (old / G + 1) * G;
+    if (ok) {
       const uint64_t t0 = globaltimer();
-      while (ld_acquire(p.ws.rule(b) + 3) != ready_gen) {
-        if (globaltimer() - t0 > kWaitLimitNs) {
-          report(p.dev_status, CSA_ERR_TIMEOUT);
+      while (true) {
+        unsigned long long v;
+        asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(ctr) : "memory");
+        if (v >= target) break;
+        if (globaltimer() - t0 > limit_ns) {
+          report(dev_status, CSA_ERR_TIMEOUT);
           ok = false;
           break;
         }
       }
     }
-    if (!__syncthreads_and(ok)) return;
-    select_write(p, x, b, sb);
+    sh_ok = ok;
+  }
+  __syncthreads();
+  return sh_ok != 0;
+}
+
+constexpr int kDxSlot = 32;  // in-bin candidates a CTA publishes in its slot
+
+struct DxSel {
+  uint64_t cand[kDxCand];             // the sequence's in-bin candidates (key << 32 | index)
+  uint64_t dc[1024];                  // the candidates of the digit holding the cut
+  uint16_t seg[kDxCand];              // the covering CTA each candidate came from
+  uint32_t h[256];                    // digit histogram of the cut search
+  uint32_t seg_off[kDxMaxCtas + 1];   // candidate offsets of the covering CTAs
+  uint32_t nin[kDxMaxCtas];           // their in-bin counts
+  uint32_t above[kDxMaxCtas];         // their above-bin counts
+  uint32_t pass[kDxMaxCtas];          // their in-bin candidates that pass the cut
+  uint32_t tmp[32];
+  int32_t n[kIxMaxB];                 // eligible entries of the covered sequences
+  int tbin;
+  uint32_t cnt, above_total, off, prefix, rem, pop, spill;
+  uint64_t v_cut;
+};
+static_assert(sizeof(DxSel) <= sizeof(uint8_t[kDxStages][kDxQuad][kIxKeyBytes]),
+              "selection scratch fits the key ring");
+
+// c_lo: the first CTA whose range ends after quad P; c_hi: the last CTA whose range starts
+// before quad Q (CTA c covers quads [total*c/G, total*(c+1)/G)).
+__device__ __forceinline__ int cta_ending_after(int64_t total, int G, int64_t P) {
+  return (int)(((int64_t)G * (P + 1) + total - 1) / total) - 1;
+}
+__device__ __forceinline__ int cta_starting_before(int64_t total, int G, int64_t Q) {
+  return (int)(((int64_t)G * Q + total - 1) / total) - 1;
+}
+__device__ __forceinline__ int64_t cta_q0(int64_t total, int c, int G) { return total * c / G; }
+
+__device__ __forceinline__ uint64_t cand_value(uint32_t key, int j) {
+  // larger value = earlier in the (score descending, index ascending) order
+  return ((uint64_t)key << 32) | (uint32_t)(0xFFFFFFFFu - (uint32_t)j);
+}
+
+// The entries [ja, jb) of sequence b that a CTA with quads [q0, q1) owns (ja == jb: none).
+struct SeqPart {
+  int ja, jb, tiles;  // entry range, tiles it spans
+  int t_lo;           // its first tile within the sequence
+};
+__device__ __forceinline__ SeqPart seq_part(const DxSmem& s, int b, int n, int q0, int q1) {
+  SeqPart r;
+  const int qa = max(q0, s.qprefix[b]) - s.qprefix[b];
+  const int qb = min(q1, s.qprefix[b + 1]) - s.qprefix[b];
+  r.t_lo = kDxQuad * qa;
+  const int t_hi = min(kDxQuad * qb, s.tiles[b]);
+  r.tiles = qa < qb ? t_hi - r.t_lo : 0;
+  r.ja = r.t_lo * kIxTile;
+  r.jb = r.tiles > 0 ? min(t_hi * kIxTile, n) : r.ja;
+  return r;
+}
+
+// The selection inside the cooperative decode launch, after every CTA has added its
+// histogram counts and holds its scores (in shared memory, or for long ranges in the
+// workspace):
+//  barrier 1;
+//  B: for each sequence it covers (n > k), the CTA finds the threshold bin from the
+//     sequence's histogram (the highest bin whose count from the top reaches k), counts
+//     its own entries above that bin and publishes (above, in-bin count, bin) and its
+//     in-bin entries in index order (the first kDxSlot in its slot, the rest in its own part
+//     of the sequence's candidate array);
+//  barrier 2;
+//  C: every CTA of the sequence gathers all counts and candidates in one round trip and
+//     resolves the same exact cut: a 256-bin histogram of the next 8 key bits finds the
+//     digit holding it, and the candidates of that digit are ranked by (key, index) in
+//     full. The CTA counts the earlier CTAs' passing candidates, so it knows its output
+//     offset, and writes its selected entries in index order there. The first CTA of a
+//     sequence clears the sequence's histogram for the next call.
+// Each thread owns a contiguous run of the CTA's entries, so one block scan orders a pass.
+// ok == false (a wait of this CTA gave up) skips the work but still arrives at both
+// barriers. Sequences with n <= k select every entry in place.
+__device__ void select_decode(const IxParams& p, uint8_t* scratch, const DxSmem& s, int q0,
+                              int q1, bool on_chip, bool ok) {
+  DxSel& x = *reinterpret_cast<DxSel*>(scratch);
+  constexpr int NT = kDxThreads;
+  const int tid = threadIdx.x, c = blockIdx.x, G = gridDim.x;
+  const int64_t total = s.qprefix[p.B];
+  int bf = 0;  // covered sequences: bf .. bl (some may own no tile of this CTA)
+  while (bf < p.B && s.qprefix[bf + 1] <= q0) ++bf;
+  int bl = bf - 1;
+  if (q0 < q1) {
+    bl = bf;
+    while (bl + 1 < p.B && s.qprefix[bl + 1] < q1) ++bl;
+  }
+  for (int b = bf + tid; b <= bl; b += NT) x.n[b - bf] = clamp_n(p.n_entries[b], p.Nmax, nullptr);
+  ok = grid_sync(reinterpret_cast<unsigned long long*>(p.ws.grid_bar), ok, p.wait_ns,
+                 p.dev_status);
+  // scores of sequence b by entry index (the CTA's own entries only)
+  auto seq_scores = [&](int b, const SeqPart& r, int it_b0) -> const float* {
+    return on_chip ? s.sc + (int64_t)(it_b0 - r.t_lo) * kIxTile
+                   : p.ws.scores + (size_t)b * p.Nmax;
+  };
+
+  // ---- B: threshold bin, above-bin count and in-bin candidates per covered sequence
+  for (int b = bf, it_b0 = 0; ok && b <= bl; ++b) {
+    const int n = x.n[b - bf];
+    const SeqPart r = seq_part(s, b, n, q0, q1);
+    const int itb = it_b0;
+    it_b0 += r.tiles;
+    if (n <= p.k || r.tiles == 0) continue;
+    {  // the threshold bin from the complete histogram: thread t holds the bins
+       // 2047 - 4 kQ t down to 2048 - 4 kQ (t + 1), kQ = quads per thread
+      constexpr int kQ = (kHist / 4 + NT - 1) / NT;
+      uint32_t hb[4 * kQ];
+#pragma unroll
+      for (int q = 0; q < kQ; ++q) {
+        const int hq = kHist / 4 - 1 - (tid * kQ + q);
+        const uint4 hv = hq >= 0 ? __ldcg(reinterpret_cast<const uint4*>(p.ws.hist(b)) + hq)
+                                 : make_uint4(0u, 0u, 0u, 0u);
+        hb[4 * q] = hv.w; hb[4 * q + 1] = hv.z; hb[4 * q + 2] = hv.y; hb[4 * q + 3] = hv.x;
+      }
+      if (tid == 0) x.tbin = -1;
+      uint32_t mine = 0;
+#pragma unroll
+      for (int i = 0; i < 4 * kQ; ++i) mine += hb[i];
+      const uint32_t incl = block_incl_scan<NT>(mine, x.tmp, nullptr);
+      if (incl >= (uint32_t)p.k && incl - mine < (uint32_t)p.k) {
+        uint32_t cum = incl - mine;
+        for (int i = 0; i < 4 * kQ; ++i) {
+          if (cum + hb[i] >= (uint32_t)p.k) { x.tbin = kHist - 1 - 4 * kQ * tid - i; break; }
+          cum += hb[i];
+        }
+      }
+      __syncthreads();
+    }
+    const int tbin = x.tbin;
+    const float* sc = seq_scores(b, r, itb);
+    const int per = (r.jb - r.ja + NT - 1) / NT;
+    const int j0 = min(r.jb, r.ja + tid * per), j1 = min(r.jb, j0 + per);
+    uint32_t above = 0, in = 0;
+    for (int j = j0; j < j1; ++j) {
+      const int bin = (int)(float_key(sc[j]) >> kLowBits);
+      above += bin > tbin ? 1u : 0u;
+      in += bin == tbin ? 1u : 0u;
+    }
+    uint32_t nin_tot, above_tot;
+    const uint32_t pos0 = block_incl_scan<NT>(in, x.tmp, &nin_tot) - in;
+    block_incl_scan<NT>(above, x.tmp, &above_tot);
+    if (in) {  // this thread's in-bin entries, in index order
+      uint64_t* slot = p.ws.cand_slots + ((size_t)b * kDxMaxCtas + c) * kDxSlot;
+      uint64_t* spill = p.ws.cand + (size_t)b * p.Nmax + r.ja;
+      uint32_t pos = pos0;
+      for (int j = j0; j < j1; ++j) {
+        const uint32_t key = float_key(sc[j]);
+        if ((int)(key >> kLowBits) != tbin) continue;
+        const uint64_t cv = ((uint64_t)key << 32) | (uint32_t)j;
+        if (pos < (uint32_t)kDxSlot) slot[pos] = cv; else spill[pos] = cv;
+        ++pos;
+      }
+    }
+    if (tid == 0)
+      p.ws.cta_cnt[(size_t)b * kDxMaxCtas + c] = make_uint4(above_tot, nin_tot, (uint32_t)tbin, 0u);
+  }
+  ok = grid_sync(reinterpret_cast<unsigned long long*>(p.ws.grid_bar) + 1, ok, p.wait_ns,
+                 p.dev_status);
+  if (!ok) return;
+
+  // ---- C: the exact cut, this CTA's output offset, the ordered write
+  for (int b = c; b < p.B; b += G)  // sequences with no entry at all: padding only
+    if (s.qprefix[b + 1] == s.qprefix[b])
+      for (int i = tid; i < p.k; i += NT) {
+        p.idx[(size_t)b * p.k + i] = -1;
+        if (p.scores_out) p.scores_out[(size_t)b * p.k + i] = __int_as_float(0x7fc00000);
+      }
+  for (int b = bf, it_b0 = 0; b <= bl; ++b) {
+    const int n = x.n[b - bf];
+    const SeqPart r = seq_part(s, b, n, q0, q1);
+    const int itb = it_b0;
+    it_b0 += r.tiles;
+    if (r.tiles == 0) continue;
+    const int k_eff = n < p.k ? n : p.k;
+    const int c_lo = cta_ending_after(total, G, s.qprefix[b]);
+    const int c_hi = cta_starting_before(total, G, s.qprefix[b + 1]);
+    const float* sc = seq_scores(b, r, itb);
+    int32_t* out = p.idx + (size_t)b * p.k;
+    float* sout = p.scores_out ? p.scores_out + (size_t)b * p.k : nullptr;
+    uint64_t v_cut = 0;  // n <= k: every entry (every value is >= 0), at its own index
+    uint32_t base = (uint32_t)r.ja;
+    if (n > p.k) {
+      const int nseg = c_hi - c_lo + 1;
+      // one round trip: every covering CTA's counts and slot
+      for (int i = tid; i < nseg; i += NT) {
+        const int cc = c_lo + i;
+        const bool has = cta_q0(total, cc, G) < cta_q0(total, cc + 1, G);
+        const uint4 v = has ? __ldcg(p.ws.cta_cnt + (size_t)b * kDxMaxCtas + cc)
+                            : make_uint4(0u, 0u, 0u, 0u);
+        x.above[i] = v.x;
+        x.nin[i] = v.y;
+        x.pass[i] = 0;
+        if (cc == c) x.tbin = (int)v.z;
+      }
+      constexpr int kSlotLoads = (kDxMaxCtas * kDxSlot + NT - 1) / NT;
+      uint64_t sv[kSlotLoads];
+#pragma unroll
+      for (int u = 0; u < kSlotLoads; ++u) {
+        const int e = tid + u * NT;
+        sv[u] = e < nseg * kDxSlot
+                    ? __ldcg(p.ws.cand_slots + ((size_t)b * kDxMaxCtas + c_lo) * kDxSlot + e)
+                    : 0ull;
+      }
+      if (tid == 0) x.spill = 0;
+      __syncthreads();
+      {  // offsets of the candidates by covering CTA (nseg <= kDxMaxCtas < NT), totals
+        const uint32_t vv = tid < nseg ? x.nin[tid] : 0u;
+        const uint32_t av = tid < nseg ? x.above[tid] : 0u;
+        if (vv > (uint32_t)kDxSlot) x.spill = 1;
+        uint32_t tot, atot;
+        const uint32_t incl = block_incl_scan<NT>(vv, x.tmp, &tot);
+        if (tid < nseg) x.seg_off[tid + 1] = incl;
+        if (tid == 0) x.seg_off[0] = 0;
+        block_incl_scan<NT>(av, x.tmp, &atot);
+        if (tid == 0) x.above_total = atot;
+        __syncthreads();
+      }
+      const uint32_t ntot = x.seg_off[nseg], above_total = x.above_total;
+      const int tbin = x.tbin;
+      const int64_t need = (int64_t)k_eff - above_total;
+      const bool staged = ntot <= (uint32_t)kDxCand;
+      auto spill_src = [&](int sgi) {  // spill part of covering CTA c_lo + sgi
+        const int64_t sq0 = cta_q0(total, c_lo + sgi, G);
+        const int64_t ja_s = (sq0 > s.qprefix[b] ? sq0 - s.qprefix[b] : 0) * kDxQuad * kIxTile;
+        return p.ws.cand + (size_t)b * p.Nmax + ja_s;
+      };
+      if (staged) {  // the candidate list: the slots (already in registers), then any spill
+#pragma unroll
+        for (int u = 0; u < kSlotLoads; ++u) {
+          const int e = tid + u * NT;
+          if (e < nseg * kDxSlot) {
+            const int sgi = e / kDxSlot, i = e % kDxSlot;
+            if ((uint32_t)i < x.nin[sgi]) {
+              x.cand[x.seg_off[sgi] + i] = sv[u];
+              x.seg[x.seg_off[sgi] + i] = (uint16_t)sgi;
+            }
+          }
+        }
+        if (x.spill) {
+          for (int sgi = 0; sgi < nseg; ++sgi) {
+            if (x.nin[sgi] <= (uint32_t)kDxSlot) continue;
+            const uint64_t* src = spill_src(sgi);
+            for (uint32_t i = kDxSlot + tid; i < x.nin[sgi]; i += NT) {
+              x.cand[x.seg_off[sgi] + i] = __ldcg(src + i);
+              x.seg[x.seg_off[sgi] + i] = (uint16_t)sgi;
+            }
+          }
+        }
+        __syncthreads();
+      }
+      // candidate i of the concatenation (from shared memory, or for a very large bin from
+      // the slots and spill parts in global memory)
+      auto seg_of = [&](uint32_t i) {
+        int lo = 0, hi = nseg - 1;
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if (x.seg_off[mid] <= i) lo = mid; else hi = mid - 1;
+        }
+        return lo;
+      };
+      auto get = [&](uint32_t i) -> uint64_t {
+        if (staged) return x.cand[i];
+        const int sgi = seg_of(i);
+        const uint32_t ri = i - x.seg_off[sgi];
+        return ri < (uint32_t)kDxSlot
+                   ? __ldcg(p.ws.cand_slots + ((size_t)b * kDxMaxCtas + c_lo + sgi) * kDxSlot + ri)
+                   : __ldcg(spill_src(sgi) + ri);
+      };
+      auto value_of = [&](uint64_t cv) { return cand_value((uint32_t)(cv >> 32), (int)(uint32_t)cv); };
+      if (need <= 0) {  // the bin contributes nothing: the cut sits just above it (tbin is
+                        // below the top bin here, as the top bin has nothing above it)
+        if (need < 0) report(p.dev_status, CSA_ERR_DEVICE);
+        v_cut = cand_value((uint32_t)(tbin + 1) << kLowBits, -1);
+      } else if (need >= (int64_t)ntot) {  // the whole bin
+        if (need > (int64_t)ntot) report(p.dev_status, CSA_ERR_DEVICE);
+        v_cut = cand_value((uint32_t)tbin << kLowBits, 0x7FFFFFFF);
+      } else {
+        // the digit of key bits 13..20 that holds the need-th largest candidate
+        for (int i = tid; i < 256; i += NT) x.h[i] = 0;
+        if (tid == 0) x.cnt = 0;
+        __syncthreads();
+        for (uint32_t i = tid; i < ntot; i += NT)
+          atomicAdd(&x.h[(uint32_t)(get(i) >> 32 >> (kLowBits - 8)) & 255u], 1u);
+        __syncthreads();
+        const uint32_t hd = tid < 256 ? x.h[255 - tid] : 0u;  // descending digits
+        const uint32_t incl = block_incl_scan<NT>(hd, x.tmp, nullptr);
+        if (tid < 256 && incl >= (uint32_t)need && incl - hd < (uint32_t)need) {
+          x.tbin = 255 - tid;  // (reused) the digit
+          x.off = (uint32_t)need - (incl - hd);  // rank wanted inside the digit, from 1
+        }
+        __syncthreads();
+        const uint32_t digit = (uint32_t)x.tbin, want = x.off, m = x.h[digit];
+        auto digit_of = [&](uint64_t cv) { return ((uint32_t)(cv >> 32) >> (kLowBits - 8)) & 255u; };
+        if (staged && m <= 1024u) {
+          // the digit's candidates, each ranked by one warp: the one with want - 1 larger
+          // values in the digit is the cut (larger digits are all above it)
+          for (uint32_t i = tid; i < ntot; i += NT) {
+            const uint64_t cv = x.cand[i];
+            if (digit_of(cv) == digit) x.dc[atomicAdd(&x.cnt, 1u)] = value_of(cv);
+          }
+          __syncthreads();
+          const int warp = tid >> 5, lane = tid & 31;
+          for (uint32_t i = warp; i < m; i += NT / 32) {
+            const uint64_t v = x.dc[i];
+            uint32_t rank = 0;
+            for (uint32_t j2 = lane; j2 < m; j2 += 32) rank += x.dc[j2] > v ? 1u : 0u;
+            for (int o = 16; o > 0; o >>= 1) rank += __shfl_xor_sync(0xffffffffu, rank, o);
+            if (lane == 0 && rank == want - 1) x.v_cut = v;
+          }
+          __syncthreads();
+          v_cut = x.v_cut;
+        } else {
+          // many candidates in one digit (heavy ties): radix select on the remaining 13
+          // key bits, then the smallest indices among equal keys
+          if (tid == 0) {
+            x.prefix = ((uint32_t)tbin << kLowBits) | (digit << (kLowBits - 8));
+            x.rem = want;
+          }
+          __syncthreads();
+          radix_step_g<NT>(get, ntot, true, 0, false, ~0u << (kLowBits - 8), 5, 8, true,
+                           &x.prefix, &x.rem, x.h);
+          radix_step_g<NT>(get, ntot, true, 0, false, ~0u << 5, 0, 5, true, &x.prefix, &x.rem,
+                           x.h, &x.pop);
+          const uint32_t cut_key = x.prefix;
+          int32_t cut_idx = 0x7FFFFFFF;
+          if (x.pop != x.rem) {
+            __syncthreads();
+            if (tid == 0) x.prefix = 0;
+            __syncthreads();
+            radix_step_g<NT>(get, ntot, false, cut_key, true, 0u, 24, 8, false, &x.prefix,
+                             &x.rem, x.h);
+            radix_step_g<NT>(get, ntot, false, cut_key, true, 0xFF000000u, 16, 8, false,
+                             &x.prefix, &x.rem, x.h);
+            radix_step_g<NT>(get, ntot, false, cut_key, true, 0xFFFF0000u, 8, 8, false,
+                             &x.prefix, &x.rem, x.h);
+            radix_step_g<NT>(get, ntot, false, cut_key, true, 0xFFFFFF00u, 0, 8, false,
+                             &x.prefix, &x.rem, x.h);
+            cut_idx = (int32_t)x.prefix;
+          }
+          v_cut = cand_value(cut_key, cut_idx);
+        }
+      }
+      // output offset: above-bin entries and passing candidates of the earlier CTAs
+      const int myseg = c - c_lo;
+      for (uint32_t i = tid; i < x.seg_off[myseg]; i += NT)
+        if (value_of(get(i)) >= v_cut) atomicAdd(&x.pass[staged ? x.seg[i] : seg_of(i)], 1u);
+      __syncthreads();
+      if (tid < 32) {
+        uint32_t off = 0;
+        for (int i = tid; i < myseg; i += 32) off += x.above[i] + x.pass[i];
+        for (int o = 16; o > 0; o >>= 1) off += __shfl_xor_sync(0xffffffffu, off, o);
+        if (tid == 0) x.off = off;
+      }
+      __syncthreads();
+      base = x.off;
+    }
+    {  // ordered write of this CTA's selected entries: each thread its contiguous run
+      const int per = (r.jb - r.ja + NT - 1) / NT;
+      const int j0 = min(r.jb, r.ja + tid * per), j1 = min(r.jb, j0 + per);
+      uint32_t mine = 0;
+      for (int j = j0; j < j1; ++j) mine += cand_value(float_key(sc[j]), j) >= v_cut ? 1u : 0u;
+      uint32_t tot;
+      uint32_t pos = base + block_incl_scan<NT>(mine, x.tmp, &tot) - mine;
+      if (mine) {
+        for (int j = j0; j < j1; ++j) {
+          const float v = sc[j];
+          if (cand_value(float_key(v), j) < v_cut) continue;
+          if (pos < (uint32_t)p.k) {
+            out[pos] = j;
+            if (sout) sout[pos] = v;
+          } else {
+            report(p.dev_status, CSA_ERR_DEVICE);
+          }
+          ++pos;
+        }
+      }
+      base += tot;
+    }
+    if (c == c_hi) {  // the last CTA of the sequence: its end is the selection's end
+      if (base != (uint32_t)k_eff && tid == 0) report(p.dev_status, CSA_ERR_DEVICE);
+      for (int i = k_eff + tid; i < p.k; i += NT) {
+        out[i] = -1;
+        if (sout) sout[i] = __int_as_float(0x7fc00000);
+      }
+    }
+    if (c == c_lo)  // every CTA read this histogram before barrier 2
+      for (int i = tid; i < kHist; i += NT) p.ws.hist(b)[i] = 0;
+    __syncthreads();
   }
 }
 
@@ -851,7 +1315,7 @@ __global__ void __launch_bounds__(kSelThreads) topk_threshold_kernel(IxParams p)
   const int b = blockIdx.y, sb = blockIdx.x;
   int n = p.n_entries[b];
   n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
-  if (sb < slices_of(n)) select_threshold(p, *reinterpret_cast<SelScratch*>(raw), b, sb, 0u);
+  if (sb < slices_of(n)) select_threshold(p, *reinterpret_cast<SelScratch*>(raw), b, sb);
 }
 
 __global__ void __launch_bounds__(kSelThreads) topk_write_kernel(IxParams p) {
@@ -1330,37 +1794,41 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
                                 const CUtensorMap& kmap, cudaStream_t stream, int bf16) {
   IxWs ws;
   ix_ws_layout(a.B, a.Nmax, a.k, (char*)workspace, &ws);
-  IxParams p{a.B, a.H_I, a.k, 1, bf16, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
-             a.idx, a.scores, a.dev_status};
-  const size_t smem = sizeof(IxSmem) + 1024;
-  // the whole carveout as shared memory, so two CTAs fit on an SM
+  const uint64_t wait_ns = a.select_wait_ns > 0 ? (uint64_t)a.select_wait_ns : kWaitLimitNs;
+  IxParams p{a.B, a.H_I, a.k, 1, bf16, wait_ns, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w,
+             a.k_sf, ws, a.idx, a.scores, a.dev_status};
+  const size_t smem = sizeof(DxSmem) + 1024;
   static std::atomic<uint64_t> configured{0};
-  if (cudaError_t e = configure_smem_once(indexer_score_kernel, smem, configured, 100);
+  if (cudaError_t e = configure_smem_once(indexer_decode_kernel, smem, configured, 100);
       e != cudaSuccess)
     return e;
-  // Scoring and selection in one cooperative launch (every CTA resident, so the grid
-  // barrier between the phases always completes); the runtime refuses a grid that cannot
-  // be resident, and the selection then runs as two further kernels.
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kIxThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  cfg.gridDim = dim3(num_sms);
-  cudaError_t e = cudaLaunchKernelEx(&cfg, indexer_score_kernel, kmap, p);
-  if (e == cudaSuccess) return cudaSuccess;
-  (void)cudaGetLastError();
+  const int grid_max = num_sms < kDxMaxCtas ? num_sms : kDxMaxCtas;
+  cudaError_t e = cudaSuccess;
+  if (!(a.flags & CSA_TOPK_SEPARATE_SELECT)) {
+    // Scoring and selection in one cooperative launch (every CTA resident, so the grid
+    // barriers between the phases always complete); the runtime refuses a grid that
+    // cannot be resident, and the selection then runs as two further kernels.
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kDxThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    cfg.gridDim = dim3(grid_max);
+    e = cudaLaunchKernelEx(&cfg, indexer_decode_kernel, kmap, p);
+    if (e == cudaSuccess) return cudaSuccess;
+    (void)cudaGetLastError();
+  }
   p.fused = 0;
   const int64_t tiles_max = (int64_t)a.B * (a.Nmax / kIxTile);
-  int grid = num_sms;
+  int grid = grid_max;
   if (tiles_max < grid) grid = (int)(tiles_max > 0 ? tiles_max : 1);
-  e = launch_pdl(indexer_score_kernel, dim3(grid), dim3(kIxThreads), smem, stream, kmap, p);
+  e = launch_pdl(indexer_decode_kernel, dim3(grid), dim3(kDxThreads), smem, stream, kmap, p);
   if (e != cudaSuccess) return e;
   dim3 g2((unsigned)ws.S, a.B);
   e = launch_pdl(topk_threshold_kernel, g2, dim3(kSelThreads), 0, stream, p);
@@ -1374,8 +1842,8 @@ cudaError_t launch_prefill_indexer_topk(const csa_topk_args& a, void* workspace,
                                         const CUtensorMap& kmap, cudaStream_t stream) {
   IxWs ws;
   ix_ws_layout(a.B, a.Nmax, a.k, (char*)workspace, &ws);
-  IxParams p{a.B, a.H_I, a.k, 0, 0, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w, a.k_sf, ws,
-             a.idx, a.scores, a.dev_status};
+  IxParams p{a.B, a.H_I, a.k, 0, 0, kWaitLimitNs, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w,
+             a.k_sf, ws, a.idx, a.scores, a.dev_status};
   const size_t smem = sizeof(PxSmem) + 1024;
   static std::atomic<uint64_t> configured{0};
   if (cudaError_t e = configure_smem_once(prefill_score_kernel, smem, configured);

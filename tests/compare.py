@@ -5,11 +5,13 @@
   delta = 1e-5 (relative) of a rounding midpoint. There the GPU's code must be the
   round-to-nearest-even code of some value in [v - delta, v + delta]: normally the other
   code of that midpoint, the neighbour of the oracle's code. Such flips are counted and
-  returned. For the rotated BF16 dims delta is relative to the norm of the value's RoPE
-  pair: x0*cos - x1*sin is formed in fp32 from a pair of that size, so its error scales
-  with the pair, not with the (possibly cancelled) value; where the value is tiny next to
-  its pair the interval can span more than two codes, and the rule then admits exactly
-  the codes that rounding of a value within that error can give.
+  returned. "Relative" is to the scale the fp32 value was computed at, which is not always
+  the value itself: an E4M3 dim is a gated average of O(1) inputs that can cancel, then
+  normalised by the row's RMS, so its fp32 error scales with the row's RMS (delta = 1e-5 x
+  max(|v|, RMS of the row's v)); a rotated BF16 dim x0*cos - x1*sin is formed from a pair,
+  so its error scales with the pair's norm (delta = 1e-5 x max(|v|, pair norm)). Where the
+  value is tiny next to that scale the interval can span more than two codes, and the
+  rule then admits exactly the codes that rounding of a value within that error can give.
 - top-k sets: bit-exact, unless the oracle's k-th and (k+1)-th scores are within 1e-6
   (relative) of each other; mismatches are then counted and returned.
 """
@@ -61,11 +63,18 @@ def check_codes(kv_gpu, kv_ora, y, scale, what=""):
     its values y before quantisation -> number of codes that differ from the oracle's."""
     y = np.asarray(y, dtype=np.float64)
     v = y[..., :448] / np.asarray(scale, dtype=np.float64)[..., None]
+    rms = np.sqrt(np.mean(v * v, axis=-1, keepdims=True)) * np.ones_like(v)
     g8, o8 = kv_gpu[..., :448], kv_ora[..., :448]
     d8 = g8 != o8
-    ok8 = _codes_in_window(g8[d8], v[d8], MID_REL * np.abs(v[d8]), _e4m3_ordinal, 0x80)
-    assert ok8.all(), (f"{what}: {int((~ok8).sum())} E4M3 codes are not a rounding of a value "
-                       "within the midpoint tolerance of the oracle's")
+    delta8 = MID_REL * np.maximum(np.abs(v[d8]), rms[d8])
+    ok8 = _codes_in_window(g8[d8], v[d8], delta8, _e4m3_ordinal, 0x80)
+    if not ok8.all():
+        i = int(np.flatnonzero(~ok8)[0])
+        raise AssertionError(
+            f"{what}: {int((~ok8).sum())} E4M3 codes are not a rounding of a value within the "
+            f"midpoint tolerance of the oracle's (first: v = {v[d8][i]!r}, row RMS "
+            f"{rms[d8][i]:.4g}, oracle code {int(o8[d8][i]):#04x}, GPU code "
+            f"{int(g8[d8][i]):#04x})")
     rg = np.ascontiguousarray(kv_gpu[..., 448:]).view(np.uint16)
     ro = np.ascontiguousarray(kv_ora[..., 448:]).view(np.uint16)
     d2 = rg != ro
@@ -73,8 +82,13 @@ def check_codes(kv_gpu, kv_ora, y, scale, what=""):
     pair = np.hypot(y[..., 448::2], y[..., 449::2]).repeat(2, axis=-1)
     delta = MID_REL * np.maximum(np.abs(yr[d2]), pair[d2])
     ok2 = _codes_in_window(rg[d2], yr[d2], delta, _bf16_ordinal, 0x8000)
-    assert ok2.all(), (f"{what}: {int((~ok2).sum())} BF16 codes are not a rounding of a value "
-                       "within the midpoint tolerance of the oracle's")
+    if not ok2.all():
+        i = int(np.flatnonzero(~ok2)[0])
+        raise AssertionError(
+            f"{what}: {int((~ok2).sum())} BF16 codes are not a rounding of a value within the "
+            f"midpoint tolerance of the oracle's (first: v = {yr[d2][i]!r}, pair norm "
+            f"{pair[d2][i]:.4g}, oracle code {int(ro[d2][i]):#06x}, GPU code "
+            f"{int(rg[d2][i]):#06x})")
     return int(d8.sum()) + int(d2.sum())
 
 

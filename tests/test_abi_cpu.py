@@ -95,6 +95,8 @@ def test_indexer_rejects_on_host(L):
     assert L.csa_indexer_topk(None, FAKE, ws_ok, None) == csa.CSA_ERR_INVALID_ARG
     assert call(_topk_args(Nmax=1000)) == csa.CSA_ERR_INVALID_ARG  # not a multiple of 128
     assert call(_topk_args(k=0)) == csa.CSA_ERR_INVALID_ARG
+    assert call(_topk_args(flags=2)) == csa.CSA_ERR_INVALID_ARG  # an unknown flag bit
+    assert call(_topk_args(select_wait_ns=-1)) == csa.CSA_ERR_INVALID_ARG
     assert call(_topk_args(H_I=8)) == csa.CSA_ERR_UNSUPPORTED
     assert call(_topk_args(k=4096)) == csa.CSA_ERR_UNSUPPORTED
     assert call(_topk_args(q_fp4=FAKE + 8)) == csa.CSA_ERR_INVALID_ARG  # misaligned

@@ -71,6 +71,15 @@ def test_default_decode_line():
     assert d["roofline"]["algorithmic_bytes_per_launch"] == 71338000
 
 
+@pytest.mark.parametrize("mode,workload", [("flash", "csa_decode_flash_128k"),
+                                           ("tiny", "csa_decode_8k_tiny")])
+def test_other_decode_lines(mode, workload):
+    d = _line(["--workload", mode, "--steps", "16", "--warmup", "3"])
+    _contract(d)
+    assert d["config"]["workload"] == workload and d["steps"] == 16
+    assert d["roofline"]["bound"] == "hbm"
+
+
 def test_hca_line():
     d = _line(["--workload", "hca", "--steps", "20", "--warmup", "3"])
     _contract(d)

@@ -163,13 +163,16 @@ def test_grouped_out_proj_matches_oracle(T, H, G, d_g, d_model):
 
 
 # ------------------------------------------------------------- indexer top-k
-def _topk_case(B, H_I, Nmax, n, k, planted=0, seed=0):
+def _topk_case(B, H_I, Nmax, n, k, planted=0, seed=0, separate=False):
     rng = np.random.default_rng(seed)
     n = np.asarray(n, dtype=np.int32)
     ix = synth.indexer_inputs(rng, B, H_I, Nmax, n, planted)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
     idx, sc = csa.indexer_topk(dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]),
-                               dev(ix["k_fp4"]), dev(ix["k_sf"]), k, scores=True)
+                               dev(ix["k_fp4"]), dev(ix["k_sf"]), k, scores=True,
+                               separate_select=separate, dev_status=st)
     torch.cuda.synchronize()
+    assert int(st.item()) == 0
     ora = oracle.indexer_scores(n, ix["q_fp4"], ix["q_sf"], ix["w"], ix["k_fp4"], ix["k_sf"])
     return host(idx), host(sc), ora, n
 
@@ -179,10 +182,16 @@ def _topk_case(B, H_I, Nmax, n, k, planted=0, seed=0):
     (3, 64, 4096, [4096, 2999, 130], 512, 0),   # ragged lengths, n < k in one sequence
     (2, 32, 1024, [1000, 0], 64, 2),            # an empty sequence
     (2, 64, 16384, [16384, 12345], 1024, 8),    # planted runs, several CTAs per sequence
-    (1, 64, 256, [1], 1, 0),                    # one entry
+    (1, 64, 256, [1], 1, 0),                    # one entry: most CTAs own no tile
+    # many short sequences: CTAs spanning several sequences, some empty, some n <= k
+    (200, 32, 3072, list(np.random.default_rng(5).integers(0, 3072, 200)), 1000, 0),
 ])
-def test_indexer_topk_matches_oracle(B, H_I, Nmax, n, k, planted):
-    idx, sc, ora, n = _topk_case(B, H_I, Nmax, n, k, planted, seed=B * 7 + k)
+@pytest.mark.parametrize("separate", [False, True])
+def test_indexer_topk_matches_oracle(B, H_I, Nmax, n, k, planted, separate):
+    # separate: the selection as stand-alone kernels, the path the library takes when the
+    # runtime refuses the cooperative launch
+    idx, sc, ora, n = _topk_case(B, H_I, Nmax, n, k, planted, seed=B * 7 + k,
+                                 separate=separate)
     total = 0
     for b in range(B):
         total += compare.compare_topk(idx[b], ora[b], int(n[b]), k, what=f"seq {b}")
@@ -234,8 +243,9 @@ def test_indexer_scores_exact_on_integer_case():
     np.testing.assert_array_equal(sc[:1000], ora[0, :1000])
 
 
+@pytest.mark.parametrize("separate", [False, True])
 @pytest.mark.parametrize("k", [1, 100, 777, 2048])
-def test_indexer_exact_ties_keep_smaller_indices(k):
+def test_indexer_exact_ties_keep_smaller_indices(k, separate):
     # unit scales, w = 1, every query element 1.0 and key elements 0 or 1: each score is
     # 16 x (an integer dot <= 128), so the cut falls inside a group of exactly equal scores
     # and must keep the smaller indices (no tolerance here)
@@ -253,8 +263,37 @@ def test_indexer_exact_ties_keep_smaller_indices(k):
     assert len(np.unique(s)) <= 129  # the case really is tie-heavy
     want = oracle.topk(ora[0], 5000, k)
     idx = csa.indexer_topk(dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]),
-                           dev(ix["k_fp4"]), dev(ix["k_sf"]), k)
+                           dev(ix["k_fp4"]), dev(ix["k_sf"]), k, separate_select=separate)
     np.testing.assert_array_equal(host(idx)[0], want)
+
+
+def test_indexer_selection_wait_that_runs_out_reports_a_timeout():
+    # a 1 ns limit on the grid-barrier waits of the fused selection: every CTA that is not
+    # the last to arrive gives up at once. The waits bounded here start after scoring has
+    # drained its copies and MMAs. The call must return with CSA_ERR_TIMEOUT; after the
+    # workspace is zero-filled again (as the interface asks after any error) the next
+    # normal call on it matches the oracle.
+    B, H_I, Nmax, k = 4, 64, 32768, 1024
+    rng = np.random.default_rng(31)
+    n = np.array([32768, 30000, 20000, 1000], np.int32)
+    ix = synth.indexer_inputs(rng, B, H_I, Nmax, n, 4)
+    args = [dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]), dev(ix["k_fp4"]),
+            dev(ix["k_sf"]), k]
+    ws = csa.indexer_topk_workspace(B, Nmax, k)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    csa.indexer_topk(*args, workspace=ws, dev_status=st, select_wait_ns=1)
+    torch.cuda.synchronize()
+    assert int(st.item()) == csa.CSA_ERR_TIMEOUT
+    ws.zero_()
+    st.zero_()
+    idx = csa.indexer_topk(*args, workspace=ws, dev_status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ora = oracle.indexer_scores(n, ix["q_fp4"], ix["q_sf"], ix["w"], ix["k_fp4"], ix["k_sf"])
+    idx = host(idx)
+    flips = sum(compare.compare_topk(idx[b], ora[b], int(n[b]), k, what=f"seq {b}")
+                for b in range(B))
+    assert flips <= 2
 
 
 def test_indexer_workspace_stays_clean_across_calls():
