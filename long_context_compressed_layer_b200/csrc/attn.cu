@@ -31,10 +31,12 @@ constexpr int kAtThreads = 256;
 struct AtSmem {
   uint8_t q[8][128 * 128];      // 8 K-blocks of [128 heads x 64 dims] fp16, 128-B swizzle
   uint8_t v[8][kAtRows * 128];  // 8 dim-blocks of [64 rows x 64 dims] fp16, 128-B swizzle
-  uint8_t pm[128 * 128];        // P [128 heads x 64 rows] fp16, 128-B swizzle
+  uint8_t pm[128 * 128];        // P' [128 heads x 64 rows] fp16, 128-B swizzle
   const uint8_t* row[kAtRows];  // row source
   const float* scl[kAtRows];    // entry rows: address of the entry scale
   int kind[kAtRows];            // 0 invalid, 1 entry, 2 window row
+  float scale[kAtRows];         // the row's factor (entry scale; 1 for window rows)
+  float mx[2][128], sm[2][128]; // the two column halves' max and sum per head
   float inv_l[128];             // 1 / (chunk sum) per head
   uint64_t q_full, s_done, o_done;
   uint32_t tmem_base;
@@ -67,7 +69,32 @@ __device__ __forceinline__ uint4 bf16x8_to_f16x8(uint4 v) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// 16 E4M3 codes x scale -> two 16-byte chunks of FP16
+// 8 BF16 values times f -> 8 FP16 values (one rounding of the fp32 product)
+__device__ __forceinline__ uint4 bf16x8_scaled_to_f16x8(uint4 v, float f) {
+  uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    w[e] = pack_half2(bf16_bits_to_f32(w[e] & 0xFFFF) * f, bf16_bits_to_f32(w[e] >> 16) * f);
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// 16 E4M3 codes -> 16 FP16 values, exactly (every E4M3 value is an FP16 value): two packed
+// conversions per 32-bit word, the lower code of each pair in the lower half
+__device__ __forceinline__ void e4m3x16_codes_to_f16(uint4 raw, uint4* lo, uint4* hi) {
+  const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
+  uint32_t o[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __half2_raw a = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(in[e] & 0xFFFF), __NV_E4M3);
+    const __half2_raw b = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(in[e] >> 16), __NV_E4M3);
+    o[2 * e] = (uint32_t)a.x | ((uint32_t)a.y << 16);
+    o[2 * e + 1] = (uint32_t)b.x | ((uint32_t)b.y << 16);
+  }
+  *lo = make_uint4(o[0], o[1], o[2], o[3]);
+  *hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+// 16 E4M3 codes x scale -> two 16-byte chunks of FP16 (one rounding of the fp32 product)
 __device__ __forceinline__ void e4m3x16_to_f16(uint4 raw, float scl, uint4* lo, uint4* hi) {
   const uint32_t in[4] = {raw.x, raw.y, raw.z, raw.w};
   uint32_t o[8];
@@ -91,6 +118,12 @@ __device__ __forceinline__ int at_rows_total(const AtParams& p, int n) {
   return (p.sparse ? p.k : n) + kWin;
 }
 
+// The staged row of entry r is v'_r = [codes (448 dims, exact in FP16) | rope dims / scale_r]
+// with scale_r its entry scale, and a window row is itself with scale 1. Then
+//   q . v_r = scale_r (q . v'_r)   and   sum_r p_r v_r = sum_r (p_r scale_r) v'_r,
+// so the S product takes v' and the logits are multiplied by scale_r, and the P V product
+// takes P' = p * scale_r. The 448 E4M3 dims enter the products exactly; only the 64 rope
+// dims of entries are rounded (once, to FP16), where staging v_r itself would round all 448.
 __global__ void __launch_bounds__(kAtThreads, 1)
     attn_chunk_kernel(const __grid_constant__ CUtensorMap qmap, AtParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -160,13 +193,13 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s.tmem_base;
   // gather: four threads per row; every thread issues all of its 16-byte pieces (and the
-  // row's scale) before converting any, so ~40-64 KB are in flight per CTA
+  // row's scale) before converting any
   {
     const int r = tid >> 2, qd = tid & 3;
-    const int kind = s.kind[r];
+    int kind = s.kind[r];
     const uint8_t* src = s.row[r];
     const int units = kind == 1 ? 36 : (kind == 2 ? 64 : 0);  // 16-byte pieces of the row
-    const float scl = kind == 1 ? __ldg(s.scl[r]) : 0.f;
+    float scl = kind == 1 ? __ldg(s.scl[r]) : 1.f;
     uint4 buf[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -174,17 +207,27 @@ __global__ void __launch_bounds__(kAtThreads, 1)
       buf[i] = u < units ? __ldg(reinterpret_cast<const uint4*>(src + 16 * u))
                          : make_uint4(0, 0, 0, 0);
     }
+    if (kind == 1 && !(scl > 0.f && scl < INFINITY)) {  // the staging divides by the scale
+      if (qd == 0) report(p.dev_status, CSA_ERR_DEVICE);
+      kind = 0;
+      scl = 1.f;
+    }
+    if (qd == 0) {
+      s.scale[r] = scl;
+      s.kind[r] = kind;
+    }
     if (kind == 1) {
+      const float inv = 1.f / scl;
 #pragma unroll
       for (int i = 0; i < 9; ++i) {
         const int u = qd + 4 * i;
-        if (u < 28) {  // 16 E4M3 dims -> output chunks 2u, 2u+1
+        if (u < 28) {  // 16 E4M3 codes -> output chunks 2u, 2u+1
           uint4 lo, hi;
-          e4m3x16_to_f16(buf[i], scl, &lo, &hi);
+          e4m3x16_codes_to_f16(buf[i], &lo, &hi);
           store_v_chunk(s, r, 2 * u, lo);
           store_v_chunk(s, r, 2 * u + 1, hi);
-        } else {  // 8 BF16 RoPE dims -> chunk 56 + (u - 28)
-          store_v_chunk(s, r, 28 + u, bf16x8_to_f16x8(buf[i]));
+        } else {  // 8 BF16 RoPE dims / scale -> chunk 56 + (u - 28)
+          store_v_chunk(s, r, 28 + u, bf16x8_scaled_to_f16x8(buf[i], inv));
         }
       }
     } else if (kind == 2) {
@@ -204,16 +247,18 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   fence_async_smem();
   ok = __syncthreads_and(ok) != 0;
 
-  // S = Q V^T : M = 128 heads, N = 64 rows, K = 512 (32 steps of 16)
+  // S' = Q V'^T : M = 128 heads, N = 64 rows, K = 512 (32 steps of 16)
   const uint32_t t_o = tmem, t_s = tmem + 256;
   if (tid == 0) {
     if (ok) {
       tc_fence_after();
       const uint32_t id = idesc_f16(128, kAtRows, false);
-      for (int kk = 0; kk < 32; ++kk) {
-        const uint32_t off = (kk & 3) * 32;
-        mma_f16(t_s, smem_desc(smem_u32(s.q[kk >> 2]) + off, 16, 1024, kSwizzle128B),
-                smem_desc(smem_u32(s.v[kk >> 2]) + off, 16, 1024, kSwizzle128B), id, kk > 0);
+      const uint64_t qd0 = smem_desc(smem_u32(s.q[0]), 16, 1024, kSwizzle128B);
+      const uint64_t vd0 = smem_desc(smem_u32(s.v[0]), 16, 1024, kSwizzle128B);
+      for (int kk = 0; kk < 32; ++kk) {  // descriptor start addresses advance in 16-byte units
+        const uint64_t qoff = (uint64_t)(((kk >> 2) * 128 * 128 + (kk & 3) * 32) >> 4);
+        const uint64_t voff = (uint64_t)(((kk >> 2) * kAtRows * 128 + (kk & 3) * 32) >> 4);
+        mma_f16(t_s, qd0 + qoff, vd0 + voff, id, kk > 0);
       }
     }
     mma_commit(&s.s_done);
@@ -224,49 +269,61 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   }
   tc_fence_after();
 
-  // softmax rows: thread h < 128 owns head h (TMEM lane h)
-  const int h = tid;
-  float m_c = -INFINITY, l_c = 0.f;
-  if (tid < 128) {
-    uint32_t r0[32], r1[32];
-    const uint32_t ta = t_s + ((uint32_t)(warp * 32) << 16);
-    tmem_ld32(ta, r0);
-    tmem_ld32(ta + 32, r1);
+  // softmax over the chunk's 64 rows, all eight warps: warp w reads TMEM lane quadrant w % 4
+  // (heads), columns 32 (w / 4) .. +31 (rows); the two halves exchange max and sum
+  const int quad = warp & 3, ch = warp >> 2;
+  const int h = quad * 32 + (tid & 31);
+  float lg[32];
+  float m_c;
+  {
+    uint32_t r0[32];
+    tmem_ld32(t_s + ((uint32_t)(quad * 32) << 16) + 32 * ch, r0);
     tmem_ld_wait();
-    float lg[64];
+    float mloc = -INFINITY;
 #pragma unroll
     for (int r = 0; r < 32; ++r) {
-      lg[r] = s.kind[r] ? __uint_as_float(r0[r]) * p.tau : -INFINITY;
-      lg[32 + r] = s.kind[32 + r] ? __uint_as_float(r1[r]) * p.tau : -INFINITY;
+      const int rr = 32 * ch + r;
+      lg[r] = s.kind[rr] ? __uint_as_float(r0[r]) * (p.tau * s.scale[rr]) : -INFINITY;
+      mloc = fmaxf(mloc, lg[r]);
     }
-#pragma unroll
-    for (int r = 0; r < 64; ++r) m_c = fmaxf(m_c, lg[r]);
+    s.mx[ch][h] = mloc;
+  }
+  __syncthreads();
+  m_c = fmaxf(s.mx[0][h], s.mx[1][h]);
+  {
+    float l_loc = 0.f;
     uint8_t* prow = s.pm + h * 128;
 #pragma unroll
-    for (int ch = 0; ch < 8; ++ch) {
+    for (int c4 = 0; c4 < 4; ++c4) {  // 16-byte chunks 4 ch + c4 of the P' row
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int r = ch * 8 + 2 * e;
+        const int r = c4 * 8 + 2 * e, rr = 32 * ch + r;
         const float p0 = m_c == -INFINITY ? 0.f : expf(lg[r] - m_c);
         const float p1 = m_c == -INFINITY ? 0.f : expf(lg[r + 1] - m_c);
-        l_c += p0;
-        l_c += p1;
-        w[e] = pack_half2(p0, p1);
+        l_loc += p0;
+        l_loc += p1;
+        w[e] = pack_half2(p0 * s.scale[rr], p1 * s.scale[rr + 1]);
       }
-      *reinterpret_cast<uint4*>(prow + ((ch ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      const int chunk = 4 * ch + c4;
+      *reinterpret_cast<uint4*>(prow + ((chunk ^ (h & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
     }
-    s.inv_l[h] = l_c > 0.f ? 1.f / l_c : 0.f;
-    if (h < p.H) {
-      const size_t slot = ((size_t)b * p.C + c) * p.H + h;
-      p.part_ml[slot] = ok ? make_float2(m_c, l_c) : make_float2(-INFINITY, 0.f);
-    }
+    s.sm[ch][h] = l_loc;
   }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
+  if (tid < 128) {  // head tid: the chunk's max and sum (the halves summed in a fixed order)
+    const float l_c = s.sm[0][tid] + s.sm[1][tid];
+    s.inv_l[tid] = l_c > 0.f ? 1.f / l_c : 0.f;
+    if (tid < p.H) {
+      const size_t slot = ((size_t)b * p.C + c) * p.H + tid;
+      p.part_ml[slot] = ok ? make_float2(fmaxf(s.mx[0][tid], s.mx[1][tid]), l_c)
+                           : make_float2(-INFINITY, 0.f);
+    }
+  }
 
-  // O = P V : M = 128, N = 256 per half, K = 64 rows (4 steps of 16); V read MN-major
+  // O = P' V' : M = 128, N = 256 per half, K = 64 rows (4 steps of 16); V' read MN-major
   if (tid == 0) {
     if (ok) {
       tc_fence_after();
@@ -282,27 +339,34 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     mma_commit(&s.o_done);
   }
   mbar_wait(&s.o_done, 0, p.dev_status);
+  __syncthreads();  // inv_l written by threads 0-127 above
   tc_fence_after();
   {
-    // warp w reads lanes of quadrant w % 4, columns [256 * (w / 4), +256): 8 loads of 32
-    const int quad = warp & 3, colh = warp >> 2;
+    // warp w reads lanes of quadrant w % 4, columns [256 * (w / 4), +256): 8 blocks of 32,
+    // two TMEM loads per wait
+    const int colh = warp >> 2;
     const int hh = quad * 32 + (tid & 31);
     const float inv = s.inv_l[hh];
-    for (int i = 0; i < 8; ++i) {
-      const int cc = colh * 8 + i;  // 32-dim block
-      uint32_t r[32];
-      tmem_ld32(t_o + ((uint32_t)(quad * 32) << 16) + cc * 32, r);
+    for (int i = 0; i < 8; i += 2) {
+      uint32_t r[2][32];
+      const uint32_t ta = t_o + ((uint32_t)(quad * 32) << 16) + (colh * 8 + i) * 32;
+      tmem_ld32(ta, r[0]);
+      tmem_ld32(ta + 32, r[1]);
       tmem_ld_wait();
       if (hh < p.H) {
-        __half* dst = p.part_o + ((((size_t)b * p.C + c) * 16 + cc) * p.H + hh) * 32;
 #pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 v;
-          v.x = pack_half2(__uint_as_float(r[e]) * inv, __uint_as_float(r[e + 1]) * inv);
-          v.y = pack_half2(__uint_as_float(r[e + 2]) * inv, __uint_as_float(r[e + 3]) * inv);
-          v.z = pack_half2(__uint_as_float(r[e + 4]) * inv, __uint_as_float(r[e + 5]) * inv);
-          v.w = pack_half2(__uint_as_float(r[e + 6]) * inv, __uint_as_float(r[e + 7]) * inv);
-          *reinterpret_cast<uint4*>(dst + e) = v;
+        for (int i2 = 0; i2 < 2; ++i2) {
+          const int cc = colh * 8 + i + i2;  // 32-dim block
+          __half* dst = p.part_o + ((((size_t)b * p.C + c) * 16 + cc) * p.H + hh) * 32;
+#pragma unroll
+          for (int e = 0; e < 32; e += 8) {
+            uint4 v;
+            v.x = pack_half2(__uint_as_float(r[i2][e]) * inv, __uint_as_float(r[i2][e + 1]) * inv);
+            v.y = pack_half2(__uint_as_float(r[i2][e + 2]) * inv, __uint_as_float(r[i2][e + 3]) * inv);
+            v.z = pack_half2(__uint_as_float(r[i2][e + 4]) * inv, __uint_as_float(r[i2][e + 5]) * inv);
+            v.w = pack_half2(__uint_as_float(r[i2][e + 6]) * inv, __uint_as_float(r[i2][e + 7]) * inv);
+            *reinterpret_cast<uint4*>(dst + e) = v;
+          }
         }
       }
     }
@@ -317,6 +381,10 @@ __global__ void __launch_bounds__(kAtThreads, 1)
 
 // One CTA per (sequence, head): 128 threads x 4 dims. The chunks are merged in their fixed
 // order: o = sum_c exp(m_c - M) l_c o_c / Z,  Z = exp(sink - M) + sum_c exp(m_c - M) l_c.
+// Each thread issues its chunk loads in batches of 16, so a sequence of up to 16 chunks
+// costs one round trip.
+constexpr int kCbBatch = 16;
+
 __global__ void __launch_bounds__(128) attn_combine_kernel(AtParams p) {
   const int h = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
   __shared__ float rot[32][2];
@@ -368,14 +436,23 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AtParams p) {
   const __half* base = p.part_o + ((size_t)b * p.C * 16 + cc) * p.H * 32 + (size_t)h * 32 + e0;
   const size_t cstride = (size_t)16 * p.H * 32;
   float o[4] = {0.f, 0.f, 0.f, 0.f};
-  int c = 0;
-  for (; c + 4 <= C_b && c + 4 <= 64; c += 4) {  // four loads in flight
-    uint2 v[4];
+  for (int c0 = 0; c0 < C_b; c0 += kCbBatch) {
+    uint2 v[kCbBatch];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) v[u] = *reinterpret_cast<const uint2*>(base + (c + u) * cstride);
+    for (int u = 0; u < kCbBatch; ++u)
+      v[u] = c0 + u < C_b ? *reinterpret_cast<const uint2*>(base + (c0 + u) * cstride)
+                          : make_uint2(0u, 0u);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const float w = wgt[c + u];
+    for (int u = 0; u < kCbBatch; ++u) {
+      const int c = c0 + u;
+      if (c >= C_b) break;
+      float w;
+      if (c < 64) {
+        w = wgt[c];
+      } else {
+        const float2 ml = p.part_ml[((size_t)b * p.C + c) * p.H + h];
+        w = (M == INFINITY || ml.x == -INFINITY) ? 0.f : expf(ml.x - M) * ml.y / Z;
+      }
       const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&v[u].x));
       const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&v[u].y));
       o[0] = fmaf(w, a.x, o[0]);
@@ -383,22 +460,6 @@ __global__ void __launch_bounds__(128) attn_combine_kernel(AtParams p) {
       o[2] = fmaf(w, bb.x, o[2]);
       o[3] = fmaf(w, bb.y, o[3]);
     }
-  }
-  for (; c < C_b; ++c) {
-    float w;
-    if (c < 64) {
-      w = wgt[c];
-    } else {
-      const float2 ml = p.part_ml[((size_t)b * p.C + c) * p.H + h];
-      w = (M == INFINITY || ml.x == -INFINITY) ? 0.f : expf(ml.x - M) * ml.y / Z;
-    }
-    const uint2 v = *reinterpret_cast<const uint2*>(base + c * cstride);
-    const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&v.x));
-    const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&v.y));
-    o[0] = fmaf(w, a.x, o[0]);
-    o[1] = fmaf(w, a.y, o[1]);
-    o[2] = fmaf(w, bb.x, o[2]);
-    o[3] = fmaf(w, bb.y, o[3]);
   }
   if (p.derotate && d0 >= kNope) {
 #pragma unroll

@@ -164,6 +164,7 @@ struct alignas(1024) DxSmem {
   uint64_t full[kDxStages], empty[kDxStages];
   uint64_t acc_full[kDxAcc], acc_empty[kDxAcc], q_free[kDxGroups][2], done[kDxGroups];
   uint64_t grp_bar[kDxGroups];            // the four warps of a group meet around a flush
+  uint64_t roles_bar;                     // every warp has finished its role
   int32_t grp_seq[kDxGroups];             // sequence whose counts a group histogram holds
   uint32_t tmem_base;
   volatile int abort;
@@ -246,6 +247,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
       mbar_init(&s.grp_bar[i], 4);
       mbar_init(&s.done[i], 1);
     }
+    mbar_init(&s.roles_bar, kDxWarps);
     s.abort = 0;
     mbar_fence_init();
   }
@@ -483,7 +485,15 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     });
     if ((ew & 3) == 0 && lane == 0) s.grp_seq[gi] = cur;
   }
+  // Every warp has finished its role: a bounded meeting on an mbarrier first. (The CTA
+  // barrier alone, right after the roles, was seen to let thread 0 through while epilogue
+  // warps were still scoring their last tiles, and the histogram sum below must see all of
+  // their counts.)
   tc_fence_before();
+  {
+    uint32_t roles_phase = 0;
+    if (!group_meet(&s.roles_bar, roles_phase, p.dev_status)) s.abort = 1;
+  }
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
