@@ -337,3 +337,50 @@ def prefill(inp: dict, k: int, q_rows, tau: float | None = None, rope_base: floa
     if rc:
         raise ValueError("oracle prefill rejected its arguments")
     return {"out": out, "lse": lse, "idx": idx, "kv": kv, "kv_scale": sc}
+
+
+# ------------------------------------------------------------------ paged cache
+# The classical cache of compressed entries (walkthrough §3.5) kept in pages: pools of
+# pages that hold page_entries entries each, and a block table per sequence naming the
+# page of each logical page of the sequence. Entry j of sequence b lives in slot
+# j % page_entries of page block_table[b][j // page_entries]. Arrays grouped by 128 entries
+# (the indexer key scales, 512 bytes per group) page by whole groups: group g of sequence
+# b is group (g * 128 % page_entries) / 128 of page block_table[b][g * 128 // page_entries].
+# These two functions are the definition the paged kernels are checked against: the
+# oracle's own computations take the contiguous view.
+
+def paged_view(pool, block_table, page_entries: int, group: int = 1) -> np.ndarray:
+    """Contiguous per-sequence view [B][pages_max * page_entries / group][...] of a pool
+    [num_pages][page_entries / group][...]; units on table entries outside the pool
+    (e.g. -1 for pages not yet given) read as zeros."""
+    pool = np.asarray(pool)
+    table = np.asarray(block_table, dtype=np.int64)
+    B, pages_max = table.shape
+    per_page = page_entries // group
+    out = np.zeros((B, pages_max * per_page) + pool.shape[2:], dtype=pool.dtype)
+    for b in range(B):
+        for lp in range(pages_max):
+            page = int(table[b, lp])
+            if 0 <= page < pool.shape[0]:
+                out[b, lp * per_page:(lp + 1) * per_page] = pool[page]
+    return out
+
+
+def paged_scatter(view, block_table, page_entries: int, num_pages: int,
+                  group: int = 1) -> np.ndarray:
+    """The pool [num_pages][page_entries / group][...] that holds each sequence's units of
+    a contiguous view [B][units][...] at the places the block table names (pages the
+    table does not name are zero)."""
+    view = np.asarray(view)
+    table = np.asarray(block_table, dtype=np.int64)
+    B, pages_max = table.shape
+    per_page = page_entries // group
+    pool = np.zeros((num_pages, per_page) + view.shape[2:], dtype=view.dtype)
+    for b in range(B):
+        for lp in range(pages_max):
+            page = int(table[b, lp])
+            lo = lp * per_page
+            if 0 <= page < num_pages and lo < view.shape[1]:
+                hi = min(lo + per_page, view.shape[1])
+                pool[page, :hi - lo] = view[b, lo:hi]
+    return pool
