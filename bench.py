@@ -5,8 +5,10 @@ One step = one decode query for each of the B = 4 sequences of the workload
 head_dim 512, indexer 64 heads x 128 FP4 dims, top-k 1024, 128-token window, sink):
   csa_indexer_topk  (FP4 indexer scores over every entry + top-k selection)
   csa_sparse_attn_decode  (shared-KV MQA over the selected entries + window + sink)
-Metric: decode queries/s (whole job). Inputs are synthetic and seeded; four device copies
-of the streamed inputs are rotated so that consecutive steps never hit in L2.
+Metric: decode queries/s (whole job). Inputs are synthetic and seeded; device copies of the
+streamed inputs are rotated step by step (inside each replayed graph too) so that
+consecutive steps never hit in L2. The compressed cache sits in pages of 512 entries
+(2,048 tokens) behind a shuffled block table (--page-entries 0: contiguous per sequence).
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
                        [--workload decode|prefill|hca]
@@ -28,6 +30,7 @@ from __future__ import annotations
 
 import argparse
 import json
+import math
 import os
 import statistics
 import subprocess
@@ -151,6 +154,107 @@ def prefill_flops(P: int, T: int, m: int, H: int, H_I: int, k: int) -> tuple[int
     n = (t + 1) // m
     rows = np.minimum(k, n) + np.minimum(128, t + 1)
     return int(2 * H_I * 128 * n.sum()), int(4 * H * 512 * rows.sum())
+
+
+def capture_graph(torch, warm, body):
+    """A CUDA graph of `body`, captured on a side stream after one uncaptured `warm` call
+    (which fills the library's tensor-map and attribute caches)."""
+    g = torch.cuda.CUDAGraph()
+    s_cap = torch.cuda.Stream()
+    s_cap.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s_cap):
+        warm()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s_cap):
+            body()
+    torch.cuda.current_stream().wait_stream(s_cap)
+    torch.cuda.synchronize()
+    return g
+
+
+def rotation_graphs(torch, step, copies, reps):
+    """CUDA graphs of `reps` steps each in which the global step s runs on device copy
+    copies[s % len(copies)], so that no two consecutive steps read the same copy; replaying
+    the returned graphs round robin continues that sequence."""
+    n = len(copies)
+    graphs = []
+    for gi in range(n // math.gcd(n, reps)):
+        seq = [copies[(gi * reps + j) % n] for j in range(reps)]
+        graphs.append(capture_graph(torch, lambda seq=seq: step(seq[0]),
+                                    lambda seq=seq: [step(c) for c in seq]))
+    return graphs
+
+
+def packed(torch, specs: dict, host: bool):
+    """One byte buffer (pinned host memory, or device memory) holding a tensor per entry of
+    `specs` (name -> (shape, dtype)) at 256-byte aligned offsets: (buffer, {name: view})."""
+    offs, off = {}, 0
+    for key, (shape, dtype) in specs.items():
+        nbytes = math.prod(shape) * torch.empty((), dtype=dtype).element_size()
+        offs[key] = (off, nbytes)
+        off += -(-nbytes // 256) * 256
+    if host:
+        buf = torch.empty(off, dtype=torch.uint8, pin_memory=True)
+    else:
+        buf = torch.empty(off, dtype=torch.uint8, device="cuda")
+    return buf, {key: buf[o:o + nb].view(specs[key][1]).view(specs[key][0])
+                 for key, (o, nb) in offs.items()}
+
+
+def e2e_graphs(torch, launch, copies, inputs: dict, out_specs: dict, reps):
+    """CUDA graphs of `reps` end-to-end steps each, pipelined across steps. Step j uploads
+    its query-side inputs (`inputs`, host tensors, packed into one pinned buffer) in one copy
+    into device slot j % 2 on an upload stream, runs its kernels on the capture stream once
+    that copy is done (launch(copy, device input views, device output views)), and
+    downloads its packed outputs to pinned host memory in one copy on a download stream.
+    Slot reuse waits on events: an upload waits for the kernels two steps back, and kernels
+    wait for the download two steps back. Device copies rotate as in rotation_graphs.
+    Returns (graphs, h2d bytes per step, d2h bytes per step, host output views)."""
+    in_specs = {key: (tuple(v.shape), v.dtype) for key, v in inputs.items()}
+    h_in, h_in_v = packed(torch, in_specs, True)
+    for key, v in inputs.items():
+        h_in_v[key].copy_(v)
+    d_in = [packed(torch, in_specs, False) for _ in range(2)]
+    d_out = [packed(torch, out_specs, False) for _ in range(2)]
+    h_out, h_out_v = packed(torch, out_specs, True)
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    n = len(copies)
+
+    def body(seq):
+        comp = torch.cuda.current_stream()
+        up.wait_stream(comp)
+        down.wait_stream(comp)
+        done, fetched = [], []
+        for j, c in enumerate(seq):
+            s = j % 2
+            with torch.cuda.stream(up):
+                if j >= 2:
+                    up.wait_event(done[j - 2])
+                d_in[s][0].copy_(h_in, non_blocking=True)
+                e_up = torch.cuda.Event()
+                e_up.record(up)
+            comp.wait_event(e_up)
+            if j >= 2:
+                comp.wait_event(fetched[j - 2])
+            launch(c, d_in[s][1], d_out[s][1])
+            e_done = torch.cuda.Event()
+            e_done.record(comp)
+            done.append(e_done)
+            with torch.cuda.stream(down):
+                down.wait_event(e_done)
+                h_out.copy_(d_out[s][0], non_blocking=True)
+                e_f = torch.cuda.Event()
+                e_f.record(down)
+                fetched.append(e_f)
+        comp.wait_stream(up)
+        comp.wait_stream(down)
+
+    graphs = []
+    for gi in range(n // math.gcd(n, reps)):
+        seq = [copies[(gi * reps + j) % n] for j in range(reps)]
+        graphs.append(capture_graph(torch, lambda seq=seq: launch(seq[0], d_in[0][1], d_out[0][1]),
+                                    lambda seq=seq: body(seq)))
+    return graphs, h_in.numel(), h_out.numel(), h_out_v
 
 
 def max_over_ranks(vals: list[float], world: int, device) -> list[float]:
@@ -455,22 +559,8 @@ def bench_hca(args, rank: int, world: int, local: int) -> None:
 
     graph_steps = next(g for g in (8, 4, 2, 1) if args.steps % g == 0)  # exactly --steps
 
-    def capture(fn):
-        g = torch.cuda.CUDAGraph()
-        s_cap = torch.cuda.Stream()
-        s_cap.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s_cap):
-            fn()  # warm the tensor-map / attribute caches outside the capture
-            torch.cuda.synchronize()
-            with torch.cuda.graph(g, stream=s_cap):
-                for _ in range(graph_steps):
-                    fn()
-        torch.cuda.current_stream().wait_stream(s_cap)
-        torch.cuda.synchronize()
-        return g
-
-    def timed(graphs, n):
-        for i in range(max(3, len(graphs))):  # warm-up replays
+    def timed(graphs, n, per_graph=graph_steps):
+        for i in range(max(3, 2 * len(graphs))):  # warm-up replays
             graphs[i % len(graphs)].replay()
         torch.cuda.synchronize()
         if world > 1:
@@ -483,9 +573,10 @@ def bench_hca(args, rank: int, world: int, local: int) -> None:
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        return e0.elapsed_time(e1) / (n * graph_steps)
+        return e0.elapsed_time(e1) / (n * per_graph)
 
-    graphs = [capture(lambda c=c: step(c)) for c in copies]
+    # every step of a graph moves to the next device copy of the inputs
+    graphs = rotation_graphs(torch, step, copies, graph_steps)
     replays = max(1, (args.steps + graph_steps - 1) // graph_steps)
     sampler = ClockSampler(local)
     sampler.start()
@@ -494,23 +585,25 @@ def bench_hca(args, rank: int, world: int, local: int) -> None:
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during the benchmark")
 
-    # end to end: the step's queries, positions and lengths go up from pinned host memory
-    # and the output comes back, inside the replayed graphs
+    # end to end: every step uploads its queries, positions and lengths from pinned host
+    # memory (one packed copy) and downloads its output (one copy), on copy streams that
+    # overlap the neighbouring steps' kernels
     q_inputs = ("q", "pos", "n_entries")
-    pinned = {key: base[key].cpu().pin_memory() for key in q_inputs}
-    dev_in = {key: torch.empty_like(base[key]) for key in q_inputs}
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
-    d2h = out_h.numel() * out_h.element_size()
 
-    def e2e_step(c):
-        for key in q_inputs:
-            dev_in[key].copy_(pinned[key], non_blocking=True)
-        step({**c, **dev_in})
-        out_h.copy_(out, non_blocking=True)
+    def e2e_launch(c, din, dout):
+        csa.hca_attn_decode(din["q"], din["pos"], din["n_entries"], c["kv"], c["kv_scale"],
+                            c["swa"], c["sink"], workspace=ws, out=dout["out"],
+                            dev_status=status)
 
-    e2e_ms = timed([capture(lambda c=c: e2e_step(c)) for c in copies],
-                   max(4, min(replays, 256)))
+    e2e_steps = 24
+    e2e_g, h2d, d2h, h_out = e2e_graphs(torch, e2e_launch, copies,
+                                         {key: base[key].cpu() for key in q_inputs},
+                                         {"out": (tuple(out.shape), out.dtype)}, e2e_steps)
+    e2e_ms = timed(e2e_g, max(len(e2e_g), min(replays, 64)), e2e_steps)
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} in the end-to-end run")
+    if not torch.equal(h_out["out"], out.cpu()):
+        raise RuntimeError("end-to-end output differs from the device-resident call's")
     ms, e2e_ms = max_over_ranks([ms, e2e_ms], world, "cuda")
     if world > 1:
         dist.destroy_process_group()
@@ -522,14 +615,17 @@ def bench_hca(args, rank: int, world: int, local: int) -> None:
     achieved = step_bytes / (ms * 1e-3) / 1e9
     line = {
         "metric": HCA_METRIC, "value": whole_job_rate(B, world, ms), "unit": UNIT,
-        "n_gpus": world, "steps": replays * graph_steps, "warmup": max(3, HCA_COPIES) * graph_steps,
+        "n_gpus": world, "steps": replays * graph_steps, "warmup": max(3, 2 * len(graphs)) * graph_steps,
         "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "fp16", "data": "synthetic",
         "config": {"workload": w.name, "queries_per_step_per_gpu": B, "context": w.L,
                    "entries_per_seq": int(d["n_entries"][0]), "heads": w.H, "window": 128,
                    "l2": f"inputs rotated over {HCA_COPIES} device copies "
                          f"({HCA_COPIES * streamed_bytes / 1e6:.0f} MB of streamed inputs)",
-                   "launch": f"CUDA graphs of {graph_steps} steps, programmatic dependent launch"},
+                   "launch": f"CUDA graphs of {graph_steps} steps, programmatic dependent launch",
+                   "e2e_launch": f"CUDA graphs of {e2e_steps} steps; one packed upload and one "
+                                 "download per step on two copy streams, device inputs and "
+                                 "outputs double-buffered"},
         "roofline": {"bound": "hbm", "kernel": "hca_attn_decode (chunk + combine kernels)",
                      "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                      "frac": achieved / pk["hbm_gbs"], "peak_src": pk["src"],
@@ -628,8 +724,10 @@ L2_BYTES = 126 << 20
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=500)
+    ap.add_argument("--steps", type=int, default=None,
+                    help="timed steps (default 20000 for decode modes, 5 for prefill)")
+    ap.add_argument("--warmup", type=int, default=None,
+                    help="untimed steps first (default 500 for decode modes, 3 for prefill)")
     ap.add_argument("--impl", default="csa", choices=["csa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--copies", type=int, default=0,
@@ -637,7 +735,14 @@ def main():
                          "(0: enough that one rotation exceeds twice the L2)")
     ap.add_argument("--workload", default="decode",
                     choices=sorted(DECODE_MODES) + ["prefill", "hca"])
+    ap.add_argument("--page-entries", type=int, default=512,
+                    help="decode modes: compressed cache in pages of this many entries "
+                         "behind a shuffled block table (0: contiguous per sequence)")
     args = ap.parse_args()
+    if args.steps is None:
+        args.steps = 5 if args.workload == "prefill" else 20000
+    if args.warmup is None:
+        args.warmup = 3 if args.workload == "prefill" else 500
 
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -672,8 +777,24 @@ def main():
         x = np.ascontiguousarray(x)
         return torch.from_numpy(x.view(np.int16) if x.dtype == np.uint16 else x).cuda()
 
+    # the compressed cache (entries and indexer keys) in pages of P entries behind a
+    # shuffled block table, as a serving cache holds it; the oracle keeps the contiguous d
+    P = args.page_entries
+    dd, paging, cache_cfg = d, None, {"layout": "contiguous per sequence"}
+    if P:
+        table, num_pages = synth.page_table(np.random.default_rng(w.seed + 77), B, -(-Nmax // P))
+        dd = dict(d)
+        dd["k_fp4"] = synth.place_in_pages(d["k_fp4"], table, P, num_pages)
+        dd["k_sf"] = synth.place_in_pages(d["k_sf"].reshape(B, Nmax // 128, 512), table, P,
+                                          num_pages, group=128)
+        dd["kv"] = synth.place_in_pages(d["kv"], table, P, num_pages)
+        dd["kv_scale"] = synth.place_in_pages(d["kv_scale"], table, P, num_pages)
+        paging = csa.Paging(dev(table), P, Nmax)
+        cache_cfg = {"layout": "paged", "page_entries": P, "page_tokens": P * w.m,
+                     "block_table": "shuffled", "pool_pages": num_pages}
+
     streamed = ("k_fp4", "k_sf", "kv", "kv_scale", "q_fp4", "q_sf", "w", "q", "swa")
-    base = {key: dev(d[key]) for key in streamed + ("n_entries", "pos", "sink")}
+    base = {key: dev(dd[key]) for key in streamed + ("n_entries", "pos", "sink")}
     copy_bytes = sum(base[key].numel() * base[key].element_size() for key in streamed)
     ncopy = args.copies if args.copies > 0 else min(512, max(COPIES, -(-2 * L2_BYTES // copy_bytes)))
     copies = [base] + [{key: (base[key].clone() if key in streamed else base[key])
@@ -687,40 +808,26 @@ def main():
 
     def step_idx(c):
         csa.indexer_topk(c["n_entries"], c["q_fp4"], c["q_sf"], c["w"], c["k_fp4"], c["k_sf"],
-                         k, workspace=ws_idx, idx=idx, dev_status=status)
+                         k, workspace=ws_idx, idx=idx, dev_status=status, paging=paging)
 
     def step_att(c):
         csa.sparse_attn_decode(c["q"], c["pos"], c["n_entries"], c["kv"], c["kv_scale"],
                                c["swa"], c["sink"], idx, workspace=ws_att, out=out,
-                               dev_status=status)
+                               dev_status=status, paging=paging)
 
     def step(c):
         step_idx(c)
         step_att(c)
 
-    # The decode step is replayed from CUDA graphs (as a serving loop would): one graph per
-    # device copy of the inputs, each holding GRAPH_STEPS steps. Kernels launched with
-    # programmatic stream serialisation keep their programmatic edges inside the graph.
-    def capture(fn, reps):
-        g = torch.cuda.CUDAGraph()
-        s_cap = torch.cuda.Stream()
-        s_cap.wait_stream(torch.cuda.current_stream())
-        with torch.cuda.stream(s_cap):
-            fn()  # warm the tensor-map / attribute caches outside the capture
-            torch.cuda.synchronize()
-            with torch.cuda.graph(g, stream=s_cap):
-                for _ in range(reps):
-                    fn()
-        torch.cuda.current_stream().wait_stream(s_cap)
-        torch.cuda.synchronize()
-        return g
-
-    # graphs of 8 steps when --steps allows it, else of the largest power of two dividing
-    # it, so that the timed region runs exactly --steps steps
+    # The decode step is replayed from CUDA graphs (as a serving loop would), each holding
+    # GRAPH_STEPS steps that move to the next device copy of the inputs at every step.
+    # Kernels launched with programmatic stream serialisation keep their programmatic edges
+    # inside the graph. Graphs of 8 steps when --steps allows it, else of the largest power
+    # of two dividing it, so that the timed region runs exactly --steps steps.
     GRAPH_STEPS = next(g for g in (8, 4, 2, 1) if args.steps % g == 0)
-    step_graphs = [capture(lambda c=c: step(c), GRAPH_STEPS) for c in copies]
-    idx_graphs = [capture(lambda c=c: step_idx(c), GRAPH_STEPS) for c in copies]
-    att_graphs = [capture(lambda c=c: step_att(c), GRAPH_STEPS) for c in copies]
+    step_graphs = rotation_graphs(torch, step, copies, GRAPH_STEPS)
+    idx_graphs = rotation_graphs(torch, step_idx, copies, GRAPH_STEPS)
+    att_graphs = rotation_graphs(torch, step_att, copies, GRAPH_STEPS)
     replays = max(1, (args.steps + GRAPH_STEPS - 1) // GRAPH_STEPS)
     steps_run = replays * GRAPH_STEPS
 
@@ -746,14 +853,14 @@ def main():
     ms_total = t0.elapsed_time(t1)
 
     # live per-call timing of each ABI call (graphs of that call alone, same rotation)
-    def time_graphs(graphs, n):
+    def time_graphs(graphs, n, per_graph=GRAPH_STEPS):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        run_graphs(graphs, 2)
+        run_graphs(graphs, 2 * len(graphs))
         e0.record(stream)
         run_graphs(graphs, n)
         e1.record(stream)
         torch.cuda.synchronize()
-        return e0.elapsed_time(e1) / (n * GRAPH_STEPS)
+        return e0.elapsed_time(e1) / (n * per_graph)
 
     nprobe = max(4, min(replays, 256))
     t_idx = time_graphs(idx_graphs, nprobe)
@@ -765,9 +872,10 @@ def main():
 
     def step_idx_bf(c):
         csa.indexer_topk(c["n_entries"], c["q_fp4"], c["q_sf"], c["w"], c["k_fp4"], c["k_sf"],
-                         k, workspace=ws_idx, idx=idx_bf, dev_status=status, bf16_scores=True)
+                         k, workspace=ws_idx, idx=idx_bf, dev_status=status, bf16_scores=True,
+                         paging=paging)
 
-    bf_graphs = [capture(lambda c=c: step_idx_bf(c), GRAPH_STEPS) for c in copies]
+    bf_graphs = rotation_graphs(torch, step_idx_bf, copies, GRAPH_STEPS)
     t_idx_bf = time_graphs(bf_graphs, nprobe)
     step_idx(copies[0])
     step_idx_bf(copies[0])
@@ -779,27 +887,27 @@ def main():
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item())} during the benchmark")
 
-    # end to end through host buffers: the step's query-side inputs go up from pinned host
-    # memory, the outputs come back; copies and kernels replayed from one graph
+    # end to end through host buffers: every step uploads its query-side inputs from pinned
+    # host memory (one packed copy) and downloads its outputs and selected indices (one
+    # packed copy), on copy streams that overlap the neighbouring steps' kernels
     q_inputs = ("q", "q_fp4", "q_sf", "w", "pos", "n_entries")
-    pinned = {key: base[key].cpu().pin_memory() for key in q_inputs}
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    idx_h = torch.empty(idx.shape, dtype=idx.dtype).pin_memory()
-    dev_in = {key: torch.empty_like(base[key]) for key in q_inputs}
-    h2d = sum(pinned[key].numel() * pinned[key].element_size() for key in q_inputs)
-    d2h = out_h.numel() * 2 + idx_h.numel() * 4
+    out_specs = {"out": (tuple(out.shape), out.dtype), "idx": (tuple(idx.shape), idx.dtype)}
 
-    def e2e_step(c):
-        for key in q_inputs:
-            dev_in[key].copy_(pinned[key], non_blocking=True)
-        cc = dict(c)
-        cc.update(dev_in)
-        step(cc)
-        out_h.copy_(out, non_blocking=True)
-        idx_h.copy_(idx, non_blocking=True)
+    def e2e_launch(c, din, dout):
+        csa.indexer_topk(din["n_entries"], din["q_fp4"], din["q_sf"], din["w"], c["k_fp4"],
+                         c["k_sf"], k, workspace=ws_idx, idx=dout["idx"], dev_status=status,
+                         paging=paging)
+        csa.sparse_attn_decode(din["q"], din["pos"], din["n_entries"], c["kv"], c["kv_scale"],
+                               c["swa"], c["sink"], dout["idx"], workspace=ws_att,
+                               out=dout["out"], dev_status=status, paging=paging)
 
-    e2e_graphs = [capture(lambda c=c: e2e_step(c), GRAPH_STEPS) for c in copies]
-    e2e_ms = time_graphs(e2e_graphs, nprobe)
+    E2E_STEPS = 32
+    e2e_g, h2d, d2h, h_out = e2e_graphs(torch, e2e_launch, copies,
+                                         {key: base[key].cpu() for key in q_inputs},
+                                         out_specs, E2E_STEPS)
+    e2e_ms = time_graphs(e2e_g, max(len(e2e_g), min(replays, 64)), E2E_STEPS)
+    if not torch.equal(h_out["idx"], idx.cpu()):
+        raise RuntimeError("end-to-end indices differ from the device-resident call's")
 
     ms_step, e2e_ms = max_over_ranks([ms_total / steps_run, e2e_ms], world, "cuda")
     value = whole_job_rate(B, world, ms_step)
@@ -818,6 +926,7 @@ def main():
             "config": {"workload": w.name, "queries_per_step_per_gpu": B, "context": w.L,
                        "entries_per_seq": int(d["n_entries"][0]), "heads": w.H,
                        "indexer_heads": w.H_I, "top_k": w.k, "window": 128,
+                       "cache": cache_cfg,
                        "l2": f"inputs rotated over {ncopy} device copies "
                              f"({ncopy * copy_bytes / 1e6:.0f} MB of streamed inputs)",
                        "step_algorithmic_bytes": step_bytes,
@@ -826,7 +935,10 @@ def main():
                        "indexer_topk_ms": t_idx, "sparse_attn_ms": t_att,
                        "bf16_index_scores": {"indexer_topk_ms": t_idx_bf,
                                              "recall_of_fp32_topk": recall},
-                       "launch": f"CUDA graphs of {GRAPH_STEPS} steps, programmatic dependent launch"},
+                       "launch": f"CUDA graphs of {GRAPH_STEPS} steps, programmatic dependent launch",
+                       "e2e_launch": f"CUDA graphs of {E2E_STEPS} steps; one packed upload and "
+                                     "one packed download per step on two copy streams, "
+                                     "device inputs and outputs double-buffered"},
             "roofline": {"bound": "hbm", "kernel": "csa_indexer_topk (score + select)",
                          "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "peak_src": pk["src"],

@@ -65,6 +65,32 @@ enum {
 const char* csa_status_string(int status);
 
 /* ------------------------------------------------------------------------------------
+ * Paged compressed cache (walkthrough §3.5: the classical cache holds the compressed
+ * entries, in blocks aligned to 128 tokens, the least common multiple of the CSA and HCA
+ * block sizes). With block_table == NULL the cache arrays of a call are contiguous per
+ * sequence: kv [B][Nmax][576], kv_scale [B][Nmax], k_fp4 [B][Nmax][64],
+ * k_sf [B][Nmax/128][512]. Otherwise they are pools of num_pages pages of page_entries
+ * entries each: kv [num_pages][page_entries][576], kv_scale [num_pages][page_entries],
+ * k_fp4 [num_pages][page_entries][64], k_sf [num_pages][page_entries/128][512], and entry
+ * j of sequence b is slot j % page_entries of page block_table[b * pages_max +
+ * j / page_entries] (the key scales follow their entries: group g of sequence b is group
+ * (128 g % page_entries) / 128 of the page of entry 128 g).
+ *   page_entries: a power of two, 128 .. 1048576 (512 or more CSA tokens per page);
+ *   pages_max * page_entries >= Nmax; num_pages >= 1; block_table 16-byte aligned,
+ *   [B][pages_max] int32, read only.
+ * Only the pages that hold entries below n_entries[b] (or, for csa_decode_append, the
+ * entry being written) are read from the table; such an entry outside 0 .. num_pages-1 is
+ * reported as CSA_ERR_DEVICE (the call's results are then unspecified). Pages are never
+ * allocated or freed by the library.
+ */
+typedef struct {
+  const int32_t* block_table; /* [B][pages_max] physical page of each logical page, or NULL */
+  int32_t pages_max;          /* table row length */
+  int32_t page_entries;       /* entries per page */
+  int32_t num_pages;          /* pages in each pool */
+} csa_pages;
+
+/* ------------------------------------------------------------------------------------
  * csa_compress: gated-softmax block compression of the KV stream into stored entries.
  * (walkthrough §2.2: two independent KV sequences merged with softmax-normalised gate
  * weights, adjacent blocks overlap; chooseai §一: positional bias; walkthrough §2.3:
@@ -160,6 +186,7 @@ typedef struct {
   uint8_t* k_fp4;          /* [B][Nmax][64] */
   uint8_t* k_sf;           /* [B][Nmax/128][512] */
   int32_t* dev_status;     /* optional device word */
+  csa_pages pages;         /* kv, kv_scale, k_fp4, k_sf paged (block_table != NULL) */
 } csa_append_args;
 
 int csa_decode_append(const csa_append_args* args, csa_stream_t stream);
@@ -273,6 +300,7 @@ typedef struct {
   int32_t* dev_status;        /* optional device word, see conventions */
   uint32_t flags;             /* 0 or CSA_TOPK_SEPARATE_SELECT */
   int64_t select_wait_ns;     /* limit of a grid-barrier wait in ns; 0 = the default */
+  csa_pages pages;            /* k_fp4, k_sf paged (block_table != NULL) */
 } csa_topk_args;
 
 size_t csa_indexer_topk_workspace_size(int32_t B, int64_t Nmax, int32_t k);
@@ -301,9 +329,20 @@ int csa_indexer_topk_bf16(const csa_topk_args* args, void* workspace, size_t wor
  *   out[b][h] = sum_j exp(l_j) / Z * v_j,  lse[b][h] = log Z,
  * with v_j the dequantised entry (E4M3 code * entry scale, then the BF16 dims) or the
  * BF16 window row; when derotate = 1, output pairs (448+2j, 449+2j) are turned by
- * -t * rope_base^(-j/32). Products run on tcgen05 BF16 tensor cores (entries are
- * dequantised to BF16 in shared memory), accumulation and softmax in fp32.
- * H in {64, 128}. k <= 2048 (CSA); n_entries <= Nmax (HCA, any size).
+ * -t * rope_base^(-j/32). Products run on tcgen05 FP16 tensor cores: an entry row is
+ * staged as its E4M3 codes (exact in FP16) and its BF16 dims divided by the entry scale,
+ * the scale enters the logit and the probability instead; accumulation and softmax in
+ * fp32. H in {64, 128}. k <= 2048 (CSA); n_entries <= Nmax (HCA, any size).
+ *
+ * Workspace: csa_attn_workspace_size(B, H, rows_max) bytes with rows_max = k + 128 (CSA)
+ * or Nmax + 128 (HCA), 256-byte aligned. It holds the per-chunk partial outputs (rows are
+ * taken 64 at a time) and, per sequence, the two words of the chunk meeting: it must be
+ * zero-filled once before its first use, and again after a call that ended with a
+ * non-zero dev_status. When every chunk of the call can be resident on the GPU at once
+ * (B * ceil(rows_max / 64) CTAs, one per SM), the call is one cooperative launch whose
+ * chunks merge their partials themselves after meeting (a wait of at most 2 s, else
+ * CSA_ERR_TIMEOUT); otherwise a second kernel merges them. Both merges sum the chunks in
+ * index order, so results do not depend on the batch.
  */
 typedef struct {
   int32_t B;              /* queries (one per sequence) */
@@ -324,7 +363,14 @@ typedef struct {
   uint16_t* out;              /* out bf16 [B][H][512] */
   float* lse;                 /* optional out [B][H] */
   int32_t* dev_status;        /* optional device word */
+  uint32_t flags;             /* 0, or CSA_ATTN_SEPARATE_MERGE */
+  int64_t merge_wait_ns;      /* time limit of the chunk meeting; 0 selects 2 s */
+  csa_pages pages;            /* kv, kv_scale paged (block_table != NULL) */
 } csa_attn_args;
+
+/* Merge the chunk partials in a second kernel even when the cooperative launch would be
+ * possible (the path that grids too large to be resident take). */
+#define CSA_ATTN_SEPARATE_MERGE 1u
 
 size_t csa_attn_workspace_size(int32_t B, int32_t H, int32_t rows_max);
 int csa_sparse_attn_decode(const csa_attn_args* args, void* workspace, size_t workspace_bytes,

@@ -52,6 +52,42 @@ class OprojArgs(C.Structure):
                 ("dev_status", _vp)]
 
 
+class Pages(C.Structure):
+    """csa_pages: the block table of a paged compressed cache (all zero: contiguous)."""
+    _fields_ = [("block_table", _vp), ("pages_max", C.c_int32), ("page_entries", C.c_int32),
+                ("num_pages", C.c_int32)]
+
+
+class Paging:
+    """A paged compressed cache: block_table int32 [B][pages_max] (device) names the pool
+    page of each logical page of page_entries entries; Nmax is the entry capacity per
+    sequence (default pages_max * page_entries). Pools are kv uint8
+    [num_pages][page_entries][576], kv_scale float32 [num_pages][page_entries], k_fp4 uint8
+    [num_pages][page_entries][64] and k_sf uint8 [num_pages][page_entries // 128][512]."""
+
+    def __init__(self, block_table: torch.Tensor, page_entries: int, Nmax: int | None = None):
+        if block_table.dtype != torch.int32 or block_table.dim() != 2:
+            raise ValueError("block_table: int32 [B][pages_max]")
+        self.block_table = block_table.contiguous()
+        self.page_entries = int(page_entries)
+        self.pages_max = block_table.shape[1]
+        self.Nmax = int(Nmax) if Nmax is not None else self.pages_max * self.page_entries
+
+    def struct(self, pool_entries: int) -> Pages:
+        return Pages(_ptr(self.block_table, elem=4, name="block_table"), self.pages_max,
+                     self.page_entries, pool_entries // self.page_entries)
+
+
+def _pages(paging: "Paging | None", pool_entries: int, B: int) -> Pages:
+    if paging is None:
+        return Pages()
+    if paging.block_table.shape[0] != B:
+        raise ValueError(f"block_table: {paging.block_table.shape[0]} rows for {B} sequences")
+    if pool_entries % paging.page_entries:
+        raise ValueError("pool size is not a whole number of pages")
+    return paging.struct(pool_entries)
+
+
 class AppendArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("m", C.c_int32), ("overlap", C.c_int32),
                 ("rope_base", C.c_float), ("eps", C.c_float), ("pos", _vp), ("a", _vp),
@@ -60,14 +96,16 @@ class AppendArgs(C.Structure):
                 ("swa", _vp), ("kv", _vp), ("kv_scale", _vp), ("Nmax", C.c_int64),
                 ("n_entries", _vp), ("ia", _vp), ("ib", _vp), ("iza", _vp), ("izb", _vp),
                 ("ibias", _vp), ("itail_a", _vp), ("itail_za", _vp), ("itail_b", _vp),
-                ("itail_zb", _vp), ("k_fp4", _vp), ("k_sf", _vp), ("dev_status", _vp)]
+                ("itail_zb", _vp), ("k_fp4", _vp), ("k_sf", _vp), ("dev_status", _vp),
+                ("pages", Pages)]
 
 
 class TopkArgs(C.Structure):
     _fields_ = [("B", C.c_int32), ("H_I", C.c_int32), ("k", C.c_int32), ("Nmax", C.c_int64),
                 ("n_entries", _vp), ("q_fp4", _vp), ("q_sf", _vp), ("w", _vp),
                 ("k_fp4", _vp), ("k_sf", _vp), ("idx", _vp), ("scores", _vp),
-                ("dev_status", _vp), ("flags", C.c_uint32), ("select_wait_ns", C.c_int64)]
+                ("dev_status", _vp), ("flags", C.c_uint32), ("select_wait_ns", C.c_int64),
+                ("pages", Pages)]
 
 
 class AttnArgs(C.Structure):
@@ -75,7 +113,11 @@ class AttnArgs(C.Structure):
                 ("q", _vp), ("pos", _vp), ("idx", _vp), ("n_entries", _vp), ("kv", _vp),
                 ("kv_scale", _vp), ("swa", _vp), ("sink", _vp), ("tau", C.c_float),
                 ("rope_base", C.c_float), ("derotate", C.c_int32), ("out", _vp), ("lse", _vp),
-                ("dev_status", _vp)]
+                ("dev_status", _vp), ("flags", C.c_uint32), ("merge_wait_ns", C.c_int64),
+                ("pages", Pages)]
+
+
+ATTN_SEPARATE_MERGE = 1
 
 
 class PrefillArgs(C.Structure):
@@ -245,12 +287,18 @@ def new_decode_state(B: int, Nmax: int, m: int = 4, index_keys: bool = True, dev
 
 def decode_append(pos, a, za, bias, state, *, b=None, zb=None, m: int = 4, overlap: bool = True,
                   norm_w=None, rope_base: float = 10000.0, eps: float = 1e-6, ia=None, ib=None,
-                  iza=None, izb=None, ibias=None, dev_status=None, stream=None):
+                  iza=None, izb=None, ibias=None, dev_status=None,
+                  paging: Paging | None = None, stream=None):
     """Append one token per sequence (a, b bf16 [B][512]; za, zb [B][512]; ia.. [B][128]) at
-    positions pos [B] to a state from new_decode_state."""
+    positions pos [B] to a state from new_decode_state. With paging, the state's kv,
+    kv_scale, k_fp4 and k_sf are page pools (Paging) and a closed block's entry goes to
+    the slot its block table names."""
     B = a.shape[0]
     _dim(a, -1, HEAD_DIM, "a")
-    Nmax = state["kv"].shape[1]
+    if paging is None:
+        Nmax, pool = state["kv"].shape[1], B * state["kv"].shape[1]
+    else:
+        Nmax, pool = paging.Nmax, state["kv"].numel() // ROW_BYTES
     row, irow = B * HEAD_DIM, B * INDEX_DIM
     _sizes(pos=(pos, B), za=(za, row), b=(b, row), zb=(zb, row),
            bias=(bias, 2 * m if overlap else m), norm_w=(norm_w, HEAD_DIM), ia=(ia, irow),
@@ -258,21 +306,21 @@ def decode_append(pos, a, za, bias, state, *, b=None, zb=None, m: int = 4, overl
            tail_a=(state["tail_a"], B * m * HEAD_DIM), tail_za=(state["tail_za"], B * m * HEAD_DIM),
            tail_b=(state.get("tail_b"), 2 * B * m * HEAD_DIM),
            tail_zb=(state.get("tail_zb"), 2 * B * m * HEAD_DIM),
-           swa=(state["swa"], B * WINDOW * HEAD_DIM), kv=(state["kv"], B * Nmax * ROW_BYTES),
-           kv_scale=(state["kv_scale"], B * Nmax), n_entries=(state["n_entries"], B))
+           swa=(state["swa"], B * WINDOW * HEAD_DIM), kv=(state["kv"], pool * ROW_BYTES),
+           kv_scale=(state["kv_scale"], pool), n_entries=(state["n_entries"], B))
     if ia is not None:
         _sizes(itail_a=(state["itail_a"], B * m * INDEX_DIM),
                itail_za=(state["itail_za"], B * m * INDEX_DIM),
                itail_b=(state["itail_b"], 2 * B * m * INDEX_DIM),
                itail_zb=(state["itail_zb"], 2 * B * m * INDEX_DIM),
-               k_fp4=(state["k_fp4"], B * Nmax * 64), k_sf=(state["k_sf"], B * Nmax // 128 * 512))
+               k_fp4=(state["k_fp4"], pool * 64), k_sf=(state["k_sf"], pool // 128 * 512))
     g = lambda k_, el: _ptr(state.get(k_), elem=el, name=k_)
     args = AppendArgs(B, m, int(overlap), rope_base, eps, _ptr(pos, elem=4, name="pos"),
                       _ptr(a, elem=2, name="a"), _ptr(b, elem=2, name="b"),
                       _ptr(za, elem=4, name="za"), _ptr(zb, elem=4, name="zb"),
                       _ptr(bias, elem=4, name="bias"), _ptr(norm_w, elem=4, name="norm_w"),
                       g("tail_a", 2), g("tail_za", 4), g("tail_b", 2), g("tail_zb", 4),
-                      g("swa", 2), g("kv", 1), g("kv_scale", 4), state["kv"].shape[1],
+                      g("swa", 2), g("kv", 1), g("kv_scale", 4), Nmax,
                       g("n_entries", 4), _ptr(ia, elem=2, name="ia"), _ptr(ib, elem=2, name="ib"),
                       _ptr(iza, elem=4, name="iza"), _ptr(izb, elem=4, name="izb"),
                       _ptr(ibias, elem=4, name="ibias"),
@@ -282,7 +330,7 @@ def decode_append(pos, a, za, bias, state, *, b=None, zb=None, m: int = 4, overl
                       g("itail_zb", 4) if ia is not None else None,
                       g("k_fp4", 1) if ia is not None else None,
                       g("k_sf", 1) if ia is not None else None,
-                      _ptr(dev_status, elem=4, name="dev_status"))
+                      _ptr(dev_status, elem=4, name="dev_status"), _pages(paging, pool, B))
     _check(lib().csa_decode_append(C.byref(args), _stream(stream)), "csa_decode_append")
 
 
@@ -369,18 +417,23 @@ def indexer_topk_workspace(B: int, Nmax: int, k: int, device="cuda") -> torch.Te
 
 def indexer_topk(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, k: int, *, workspace=None, idx=None,
                  scores: bool = False, bf16_scores: bool = False, dev_status=None,
-                 separate_select: bool = False, select_wait_ns: int = 0, stream=None):
+                 separate_select: bool = False, select_wait_ns: int = 0,
+                 paging: Paging | None = None, stream=None):
     """Top-k entry indices [B][k] (ascending, -1 padded) and optionally their scores.
     bf16_scores selects on scores rounded to BF16 (csa_indexer_topk_bf16).
     separate_select runs the selection as separate kernels instead of inside the
     cooperative scoring launch; select_wait_ns bounds that launch's grid-barrier waits
     (0 = the library default). After a call whose dev_status reports an error, zero-fill
-    the workspace before reusing it."""
+    the workspace before reusing it. With paging, k_fp4 / k_sf are page pools (Paging)."""
     B, H_I, _ = q_fp4.shape
     _dim(q_fp4, 2, 64, "q_fp4")
-    Nmax = k_fp4.shape[1]
+    if paging is None:
+        Nmax, pool = k_fp4.shape[1], B * k_fp4.shape[1]
+    else:
+        Nmax, pool = paging.Nmax, k_fp4.numel() // 64
     _sizes(n_entries=(n_entries, B), q_sf=(q_sf, B * H_I * 4), w=(w, B * H_I),
-           k_fp4=(k_fp4, B * Nmax * 64), k_sf=(k_sf, B * Nmax // 128 * 512), idx=(idx, B * k))
+           k_fp4=(k_fp4, pool * 64), k_sf=(k_sf, pool // 128 * 512), idx=(idx, B * k))
+    pg = _pages(paging, pool, B)
     dev = q_fp4.device
     if workspace is None:
         workspace = indexer_topk_workspace(B, Nmax, k, dev)
@@ -392,7 +445,7 @@ def indexer_topk(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, k: int, *, workspace=No
                     _ptr(w, elem=4, name="w"), _ptr(k_fp4, elem=1, name="k_fp4"),
                     _ptr(k_sf, elem=1, name="k_sf"), _ptr(idx, elem=4, name="idx"),
                     _ptr(sc, elem=4, name="scores"), _ptr(dev_status, elem=4, name="dev_status"),
-                    TOPK_SEPARATE_SELECT if separate_select else 0, int(select_wait_ns))
+                    TOPK_SEPARATE_SELECT if separate_select else 0, int(select_wait_ns), pg)
     fn = "csa_indexer_topk_bf16" if bf16_scores else "csa_indexer_topk"
     _check(getattr(lib(), fn)(C.byref(args), workspace.data_ptr(), workspace.numel(),
                               _stream(stream)), fn)
@@ -401,20 +454,28 @@ def indexer_topk(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, k: int, *, workspace=No
 
 # ------------------------------------------------------------------ attention
 def attn_workspace(B: int, H: int, rows_max: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace (the library keeps its meeting words consistent between
+    calls; re-zero it after a call that reported a non-zero device status)."""
     n = lib().csa_attn_workspace_size(B, H, rows_max)
-    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
+    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
 
 
 def _attn(fn: str, sparse: bool, q, pos, n_entries, kv, kv_scale, swa, sink, idx, *,
           tau: float = 0.0, rope_base: float = 10000.0, derotate: bool = True,
-          workspace=None, out=None, lse: bool = False, dev_status=None, stream=None):
+          workspace=None, out=None, lse: bool = False, dev_status=None,
+          separate_merge: bool = False, merge_wait_ns: int = 0,
+          paging: Paging | None = None, stream=None):
     B, H, _ = q.shape
     _dim(q, 2, HEAD_DIM, "q")
-    Nmax = kv.shape[1]
+    if paging is None:
+        Nmax, pool = kv.shape[1], B * kv.shape[1]
+    else:
+        Nmax, pool = paging.Nmax, kv.numel() // ROW_BYTES
     k = idx.shape[1] if sparse else 0
-    _sizes(pos=(pos, B), n_entries=(n_entries, B), kv=(kv, B * Nmax * ROW_BYTES),
-           kv_scale=(kv_scale, B * Nmax), swa=(swa, B * WINDOW * HEAD_DIM), sink=(sink, H),
+    _sizes(pos=(pos, B), n_entries=(n_entries, B), kv=(kv, pool * ROW_BYTES),
+           kv_scale=(kv_scale, pool), swa=(swa, B * WINDOW * HEAD_DIM), sink=(sink, H),
            idx=(idx if sparse else None, B * k), out=(out, B * H * HEAD_DIM))
+    pg = _pages(paging, pool, B)
     dev = q.device
     noalloc = fn.endswith("_noalloc")
     if workspace is None and not noalloc:
@@ -428,7 +489,8 @@ def _attn(fn: str, sparse: bool, q, pos, n_entries, kv, kv_scale, swa, sink, idx
                     _ptr(kv_scale, elem=4, name="kv_scale"), _ptr(swa, elem=2, name="swa"),
                     _ptr(sink, elem=4, name="sink"), tau, rope_base, int(derotate),
                     _ptr(out, elem=2, name="out"), _ptr(l, elem=4, name="lse"),
-                    _ptr(dev_status, elem=4, name="dev_status"))
+                    _ptr(dev_status, elem=4, name="dev_status"),
+                    ATTN_SEPARATE_MERGE if separate_merge else 0, int(merge_wait_ns), pg)
     if noalloc:
         _check(getattr(lib(), fn)(C.byref(args), _stream(stream)), fn)
     else:

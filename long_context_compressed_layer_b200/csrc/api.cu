@@ -63,6 +63,14 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 
 bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
 
+// a paged-cache descriptor: unused (no table), or a consistent one covering Nmax entries
+bool ok_pages(const csa_pages& pg, int64_t Nmax) {
+  if (!pg.block_table) return true;
+  const int64_t pe = pg.page_entries;
+  return aligned16(pg.block_table) && pe >= 128 && pe <= (1 << 20) && (pe & (pe - 1)) == 0 &&
+         pg.pages_max >= 1 && pg.num_pages >= 1 && (int64_t)pg.pages_max * pe >= Nmax;
+}
+
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? CSA_OK : CSA_ERR_CUDA; }
 
 // Scratch of csa_sparse_attn_decode_noalloc: one array per device, zero-initialised when
@@ -234,7 +242,8 @@ int csa_decode_append(const csa_append_args* a, csa_stream_t stream) {
   if (!ok_ptr(a->pos) || !ok_ptr(a->a) || !ok_ptr(a->za) || !ok_ptr(a->bias) ||
       !ok_opt(a->norm_w) || !ok_ptr(a->tail_a) || !ok_ptr(a->tail_za) || !ok_ptr(a->swa) ||
       !ok_ptr(a->kv) || !ok_ptr(a->kv_scale) || !ok_ptr(a->n_entries) ||
-      (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)))
+      (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)) ||
+      !ok_pages(a->pages, a->Nmax))
     return CSA_ERR_INVALID_ARG;
   if (a->overlap && (!ok_ptr(a->b) || !ok_ptr(a->zb) || !ok_ptr(a->tail_b) || !ok_ptr(a->tail_zb)))
     return CSA_ERR_INVALID_ARG;
@@ -343,7 +352,8 @@ static int indexer_common(const csa_topk_args* a, void* ws, size_t ws_bytes,
   if (a->B == 0) return CSA_OK;
   if (!ok_ptr(a->n_entries) || !ok_ptr(a->q_fp4) || !ok_ptr(a->q_sf) || !ok_ptr(a->w) ||
       !ok_ptr(a->k_fp4) || !ok_ptr(a->k_sf) || !ok_ptr(a->idx) || !ok_opt(a->scores) ||
-      (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)))
+      (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)) ||
+      !ok_pages(a->pages, a->Nmax))
     return CSA_ERR_INVALID_ARG;
   if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255) ||
       ws_bytes < ix_workspace_size(a->B, a->Nmax, a->k))
@@ -354,13 +364,20 @@ static int indexer_common(const csa_topk_args* a, void* ws, size_t ws_bytes,
   if (a->Nmax == 0) {
     // no entry can be eligible: the select pass alone writes the -1 padding
   }
-  // the keys as [B][Nmax/128 tiles][128 entries][64 bytes], read four tiles per copy
+  // the keys as [B][Nmax/128 tiles][128 entries][64 bytes], read four tiles per copy; a
+  // paged pool as [num_pages][page_entries/128 tiles][128][64], read min(4, tiles per
+  // page) tiles per copy
   CUtensorMap kmap;
   std::memset(&kmap, 0, sizeof(kmap));
   if (a->Nmax > 0) {
-    const cuuint64_t dims[4] = {64, 128, (cuuint64_t)(a->Nmax / 128), (cuuint64_t)a->B};
-    const cuuint64_t strides[3] = {64, 128 * 64, (cuuint64_t)a->Nmax * 64};
-    const cuuint32_t box[4] = {64, 128, 4, 1};
+    const bool paged = a->pages.block_table != nullptr;
+    const int64_t tiles = paged ? a->pages.page_entries / 128 : a->Nmax / 128;
+    const cuuint64_t dims[4] = {64, 128, (cuuint64_t)tiles,
+                                (cuuint64_t)(paged ? a->pages.num_pages : a->B)};
+    const cuuint64_t strides[3] = {64, 128 * 64, (cuuint64_t)tiles * 128 * 64};
+    // contiguous: always four tiles (those past Nmax read as zeros, and the barrier expects
+    // the whole box); paged: the tiles of one copy never leave their page
+    const cuuint32_t box[4] = {64, 128, (cuuint32_t)(paged && tiles < 4 ? tiles : 4), 1};
     const cuuint32_t estr[4] = {1, 1, 1, 1};
     if (enc(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<uint8_t*>(a->k_fp4), dims,
             strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
@@ -389,7 +406,8 @@ static int attn_common(const csa_attn_args* a, int sparse, void* ws, size_t ws_b
                        csa_stream_t stream) {
   if (!a) return CSA_ERR_INVALID_ARG;
   if (a->B < 0 || a->Nmax < 0 || (sparse && a->k < 1) || !(a->tau >= 0.f) ||
-      !(a->rope_base > 0.f) || (a->derotate != 0 && a->derotate != 1))
+      !(a->rope_base > 0.f) || (a->derotate != 0 && a->derotate != 1) ||
+      (a->flags & ~CSA_ATTN_SEPARATE_MERGE) || a->merge_wait_ns < 0)
     return CSA_ERR_INVALID_ARG;
   if (a->H != 64 && a->H != 128) return CSA_ERR_UNSUPPORTED;
   if ((sparse && a->k > 2048) || a->B > 65535 || a->Nmax > ((int64_t)1 << 30))
@@ -398,7 +416,8 @@ static int attn_common(const csa_attn_args* a, int sparse, void* ws, size_t ws_b
   if (!ok_ptr(a->q) || !ok_ptr(a->pos) || !ok_ptr(a->n_entries) || !ok_ptr(a->kv) ||
       !ok_ptr(a->kv_scale) || !ok_ptr(a->swa) || !ok_ptr(a->sink) || !ok_ptr(a->out) ||
       !ok_opt(a->lse) || (sparse && !ok_ptr(a->idx)) ||
-      (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)))
+      (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)) ||
+      !ok_pages(a->pages, a->Nmax))
     return CSA_ERR_INVALID_ARG;
   const int64_t rows_max64 = (sparse ? (int64_t)a->k : a->Nmax) + CSA_WINDOW;
   const int rows_max = (int)rows_max64;

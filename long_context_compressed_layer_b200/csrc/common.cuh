@@ -26,6 +26,33 @@ constexpr int kWin = CSA_WINDOW;
 // Time limit of a bounded wait (ns of %globaltimer).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// Where the entries of the compressed cache live (csa_pages): contiguous per sequence
+// ([B][Nmax]) or in pages named by a block table. The physical entry index e of entry j
+// of sequence b addresses every cache array alike: kv row e, kv_scale[e], k_fp4 row e,
+// and the key scales of group e / 128 (pages hold whole 128-entry groups).
+struct PageMap {
+  const int32_t* table;  // null: contiguous
+  int32_t pages_max;
+  int32_t shift;         // log2(page_entries)
+  int32_t num_pages;
+  int64_t Nmax;
+};
+
+__host__ __device__ inline PageMap page_map(const csa_pages& pg, int64_t Nmax) {
+  PageMap m{pg.block_table, pg.pages_max, 0, pg.num_pages, Nmax};
+  if (m.table)
+    while (((int64_t)1 << m.shift) < pg.page_entries) ++m.shift;
+  return m;
+}
+
+// physical entry index of entry j of sequence b; -1 when its page is outside the pool
+__device__ __forceinline__ int64_t page_entry(const PageMap& m, int b, int64_t j) {
+  if (!m.table) return (int64_t)b * m.Nmax + j;
+  const int32_t page = __ldg(m.table + (size_t)b * m.pages_max + (j >> m.shift));
+  if (page < 0 || page >= m.num_pages) return -1;
+  return ((int64_t)page << m.shift) + (j & (((int64_t)1 << m.shift) - 1));
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -307,19 +307,23 @@ __global__ void __launch_bounds__(128) append_kernel(csa_append_args a) {
     *reinterpret_cast<uint2*>(a.swa + ((size_t)b * kWin + t % kWin) * kD + d0) = v;
   }
   if (r != m - 1) return;  // uniform: the block is still open
+  // the entry's place in the cache (contiguous, or the slot of its page)
+  const int64_t e = page_entry(page_map(a.pages, a.Nmax), b, blk);
+  if (e < 0) {
+    if (tid == 0) report(a.dev_status, CSA_ERR_DEVICE);
+    return;
+  }
   __syncthreads();  // every thread's tail rows are written before any is read
   const bool prev = a.overlap && blk > 0;
   const size_t pring = ((size_t)b * 2 + ((blk + 1) & 1)) * m * kD;
   compress_block(a.tail_a + tail, a.tail_za + tail, prev ? a.tail_b + pring : nullptr,
                  prev ? a.tail_zb + pring : nullptr, m, a.bias, a.norm_w, a.eps, blk * m,
-                 a.rope_base, a.kv + ((size_t)b * a.Nmax + blk) * kRow,
-                 a.kv_scale + (size_t)b * a.Nmax + blk, nullptr, red, rot);
+                 a.rope_base, a.kv + (size_t)e * kRow, a.kv_scale + e, nullptr, red, rot);
   if (a.ia) {
     const size_t itail = (size_t)b * m * kDI, ipring = ((size_t)b * 2 + ((blk + 1) & 1)) * m * kDI;
     ikey_block(a.itail_a + itail, a.itail_za + itail, prev ? a.itail_b + ipring : nullptr,
                prev ? a.itail_zb + ipring : nullptr, m, a.ibias,
-               a.k_fp4 + ((size_t)b * a.Nmax + blk) * (kDI / 2),
-               a.k_sf + (size_t)b * (a.Nmax / 128) * 512, blk, nullptr);
+               a.k_fp4 + (size_t)e * (kDI / 2), a.k_sf, e, nullptr);
   }
   if (tid == 0) a.n_entries[b] = (int32_t)(blk + 1);
 }

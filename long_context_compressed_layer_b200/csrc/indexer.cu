@@ -140,6 +140,8 @@ struct IxParams {
   int32_t* idx;
   float* scores_out;
   int32_t* dev_status;
+  PageMap pm;  // where the keys live (contiguous, or paged)
+  int tpl;     // paged keys: key tiles per copy (min(4, tiles per page))
 };
 
 __device__ __forceinline__ int clamp_n(int n, int64_t Nmax, int32_t* st) {
@@ -305,13 +307,37 @@ __global__ void __launch_bounds__(kDxThreads, 1)
           s.abort = 1;
           break;
         }
-        // the quad's four key tiles in one tensor copy (tiles past Nmax read as zeros;
-        // tiles past n_b are read but not scored) and the scale groups that exist
-        const uint32_t sf_bytes = (uint32_t)min(kDxQuad, groups - t0) * kIxSfBytes;
-        mbar_arrive_expect_tx(&s.full[st], kDxQuad * kIxKeyBytes + sf_bytes);
-        tma_load_4d(&s.keys[st][0][0], &kmap, &s.full[st], 0, 0, t0, b);
-        bulk_load(&s.ksf[st][0][0], p.k_sf + ((size_t)b * groups + t0) * kIxSfBytes, sf_bytes,
-                  &s.full[st]);
+        if (!p.pm.table) {
+          // the quad's four key tiles in one tensor copy (tiles past Nmax read as zeros;
+          // tiles past n_b are read but not scored) and the scale groups that exist
+          const uint32_t sf_bytes = (uint32_t)min(kDxQuad, groups - t0) * kIxSfBytes;
+          mbar_arrive_expect_tx(&s.full[st], kDxQuad * kIxKeyBytes + sf_bytes);
+          tma_load_4d(&s.keys[st][0][0], &kmap, &s.full[st], 0, 0, t0, b);
+          bulk_load(&s.ksf[st][0][0], p.k_sf + ((size_t)b * groups + t0) * kIxSfBytes,
+                    sf_bytes, &s.full[st]);
+        } else {
+          // paged keys: copies of tpl tiles from the page of each (a page holds whole
+          // copies); tiles past n_b that lie in another page are not read (their slots
+          // keep stale keys, which are not scored)
+          int64_t e[kDxQuad];
+          int nl = 0;
+          for (int t = t0; t < t0 + kDxQuad && t < s.tiles[b]; t += p.tpl)
+            e[nl++] = page_entry(p.pm, b, (int64_t)t * kIxTile);
+          mbar_arrive_expect_tx(&s.full[st], (uint32_t)(nl * p.tpl) * (kIxKeyBytes + kIxSfBytes));
+          const int64_t tiles_pp = ((int64_t)1 << p.pm.shift) / kIxTile;
+          for (int l = 0; l < nl; ++l) {
+            int64_t el = e[l];
+            if (el < 0) {  // a page outside the pool: reported; the first page is read instead
+              report(p.dev_status, CSA_ERR_DEVICE);
+              el = 0;
+            }
+            const int64_t g = el / kIxTile;  // the copy's first key group in the pool
+            tma_load_4d(&s.keys[st][l * p.tpl][0], &kmap, &s.full[st], 0, 0,
+                        (int)(g % tiles_pp), (int)(g / tiles_pp));
+            bulk_load(&s.ksf[st][l * p.tpl][0], p.k_sf + (size_t)g * kIxSfBytes,
+                      (uint32_t)p.tpl * kIxSfBytes, &s.full[st]);
+          }
+        }
       }
       // drain: every copy this warp issued has landed before the CTA winds down
       const int issued = qq;
@@ -1807,6 +1833,10 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
   const uint64_t wait_ns = a.select_wait_ns > 0 ? (uint64_t)a.select_wait_ns : kWaitLimitNs;
   IxParams p{a.B, a.H_I, a.k, 1, bf16, wait_ns, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w,
              a.k_sf, ws, a.idx, a.scores, a.dev_status};
+  p.pm = page_map(a.pages, a.Nmax);
+  p.tpl = a.pages.block_table ? (a.pages.page_entries / kIxTile < kDxQuad
+                                     ? a.pages.page_entries / kIxTile : kDxQuad)
+                              : kDxQuad;
   const size_t smem = sizeof(DxSmem) + 1024;
   static std::atomic<uint64_t> configured{0};
   if (cudaError_t e = configure_smem_once(indexer_decode_kernel, smem, configured, 100);

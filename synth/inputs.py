@@ -337,3 +337,31 @@ def prefill_inputs_device(P: int, T: int, m: int, H: int, H_I: int, seed: int,
         out["iprev_b"] = bf16n((m, D_I))
         out["iprev_zb"] = torch.randn((m, D_I), generator=g, device=device)
     return out
+
+
+def page_table(rng: np.random.Generator, B: int, pages_max: int, spare: int = 3
+               ) -> tuple[np.ndarray, int]:
+    """A shuffled block table int32 [B][pages_max] over a pool of B * pages_max + spare
+    pages (the spare pages are never named): (table, num_pages)."""
+    num_pages = B * pages_max + spare
+    table = rng.permutation(num_pages)[:B * pages_max].reshape(B, pages_max)
+    return table.astype(np.int32), num_pages
+
+
+def place_in_pages(per_seq: np.ndarray, table: np.ndarray, page_entries: int,
+                   num_pages: int, group: int = 1, fill: int = 0x5A) -> np.ndarray:
+    """Lay per-sequence rows [B][units][...] (a unit = `group` entries) out in a page pool
+    [num_pages][page_entries // group][...]: logical page lp of sequence b goes to pool
+    page table[b][lp]. Pool bytes no sequence owns hold `fill` (never read when the
+    table is honoured)."""
+    per_page = page_entries // group
+    B, units = per_seq.shape[:2]
+    flat = np.ascontiguousarray(per_seq)
+    pool = np.empty((num_pages, per_page) + flat.shape[2:], dtype=flat.dtype)
+    pool.view(np.uint8)[...] = fill
+    for b in range(B):
+        for lp in range(table.shape[1]):
+            lo, hi = lp * per_page, min((lp + 1) * per_page, units)
+            if lo < hi:
+                pool[table[b, lp], :hi - lo] = flat[b, lo:hi]
+    return pool

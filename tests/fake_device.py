@@ -36,6 +36,9 @@ class _Stream:
     def wait_stream(self, *a, **k):
         pass
 
+    def wait_event(self, *a, **k):
+        pass
+
 
 class _FakeLib:
     def __init__(self, real):
@@ -52,6 +55,7 @@ def _to_meta_device(fn):
         if str(k.get("device", "")).startswith("cuda"):
             k["device"] = "meta"
             k.pop("generator", None)
+        k.pop("pin_memory", None)
         return fn(*a, **k)
     return g
 
@@ -73,8 +77,10 @@ def install() -> None:
     T.cpu = lambda self, *a, **k: (torch.zeros(self.shape, dtype=self.dtype) if self.is_meta
                                    else real_cpu(self, *a, **k))
     T.item = lambda self: 0 if self.is_meta else real_item(self)
+    # a copy from the device leaves zeros in a host tensor (the fake device reads as zeros)
     T.copy_ = lambda self, src, non_blocking=False: (
-        self if (self.is_meta or src.is_meta) else real_copy(self, src, non_blocking))
+        self if self.is_meta else self.zero_() if src.is_meta
+        else real_copy(self, src, non_blocking))
     T.pin_memory = lambda self, *a, **k: self
     c = torch.cuda
     c.is_available = lambda: True

@@ -121,6 +121,15 @@ def test_attention_rejects_on_host(L):
     assert f(_attn_args(H=96)) == csa.CSA_ERR_UNSUPPORTED
     assert f(_attn_args(k=0)) == csa.CSA_ERR_INVALID_ARG
     assert f(_attn_args(derotate=2)) == csa.CSA_ERR_INVALID_ARG
+    assert f(_attn_args(flags=2)) == csa.CSA_ERR_INVALID_ARG  # an unknown flag bit
+    assert f(_attn_args(merge_wait_ns=-1)) == csa.CSA_ERR_INVALID_ARG
+    # paged-cache descriptors: page size a power of two >= 128, pages covering Nmax,
+    # an aligned table, a pool of at least one page
+    for pages in (csa.Pages(FAKE, 32, 100, 8), csa.Pages(FAKE, 64, 64, 8),
+                  csa.Pages(FAKE, 3, 1024, 8), csa.Pages(FAKE + 4, 32, 128, 8),
+                  csa.Pages(FAKE, 32, 128, 0), csa.Pages(FAKE, 0, 4096, 8)):
+        assert f(_attn_args(pages=pages)) == csa.CSA_ERR_INVALID_ARG
+    assert f(_attn_args(pages=csa.Pages(None, 0, 0, 0))) != csa.CSA_ERR_INVALID_ARG
     assert f(_attn_args(idx=None)) == csa.CSA_ERR_INVALID_ARG
     assert f(_attn_args(out=FAKE + 4)) == csa.CSA_ERR_INVALID_ARG
     assert f(_attn_args(), n=ws_ok - 1) == csa.CSA_ERR_WORKSPACE

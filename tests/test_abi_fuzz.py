@@ -65,6 +65,10 @@ def mutate(a, count):
         name, ty = fields[i]
         if ty is C.c_void_p:
             setattr(a, name, [None, F, MISALIGNED][rng.integers(3)])
+        elif ty is csa.Pages:  # a paged-cache descriptor: table and sizes perturbed together
+            setattr(a, name, csa.Pages([None, F, MISALIGNED][rng.integers(3)],
+                                       int(rng.choice(INTS)), int(rng.choice(INTS)),
+                                       int(rng.choice(INTS))))
         elif ty is C.c_float:
             setattr(a, name, float(rng.choice([-1.0, 0.0, 1e-6, 0.0442, 1.0, 1e4, np.nan])))
         elif ty is C.c_int64:

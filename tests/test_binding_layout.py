@@ -25,6 +25,7 @@ BINDING = {
     "csa_topk_args": csa.TopkArgs,
     "csa_attn_args": csa.AttnArgs,
     "csa_prefill_args": csa.PrefillArgs,
+    "csa_pages": csa.Pages,
 }
 
 
