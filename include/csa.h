@@ -335,14 +335,9 @@ int csa_indexer_topk_bf16(const csa_topk_args* args, void* workspace, size_t wor
  * fp32. H in {64, 128}. k <= 2048 (CSA); n_entries <= Nmax (HCA, any size).
  *
  * Workspace: csa_attn_workspace_size(B, H, rows_max) bytes with rows_max = k + 128 (CSA)
- * or Nmax + 128 (HCA), 256-byte aligned. It holds the per-chunk partial outputs (rows are
- * taken 64 at a time) and, per sequence, the two words of the chunk meeting: it must be
- * zero-filled once before its first use, and again after a call that ended with a
- * non-zero dev_status. When every chunk of the call can be resident on the GPU at once
- * (B * ceil(rows_max / 64) CTAs, one per SM), the call is one cooperative launch whose
- * chunks merge their partials themselves after meeting (a wait of at most 2 s, else
- * CSA_ERR_TIMEOUT); otherwise a second kernel merges them. Both merges sum the chunks in
- * index order, so results do not depend on the batch.
+ * or Nmax + 128 (HCA), 256-byte aligned, for the per-chunk partial outputs (rows are
+ * taken 64 at a time; a second kernel merges the chunks in index order, so results do not
+ * depend on the batch). It needs no initialisation.
  */
 typedef struct {
   int32_t B;              /* queries (one per sequence) */
@@ -363,14 +358,8 @@ typedef struct {
   uint16_t* out;              /* out bf16 [B][H][512] */
   float* lse;                 /* optional out [B][H] */
   int32_t* dev_status;        /* optional device word */
-  uint32_t flags;             /* 0, or CSA_ATTN_SEPARATE_MERGE */
-  int64_t merge_wait_ns;      /* time limit of the chunk meeting; 0 selects 2 s */
   csa_pages pages;            /* kv, kv_scale paged (block_table != NULL) */
 } csa_attn_args;
-
-/* Merge the chunk partials in a second kernel even when the cooperative launch would be
- * possible (the path that grids too large to be resident take). */
-#define CSA_ATTN_SEPARATE_MERGE 1u
 
 size_t csa_attn_workspace_size(int32_t B, int32_t H, int32_t rows_max);
 int csa_sparse_attn_decode(const csa_attn_args* args, void* workspace, size_t workspace_bytes,

@@ -113,11 +113,7 @@ class AttnArgs(C.Structure):
                 ("q", _vp), ("pos", _vp), ("idx", _vp), ("n_entries", _vp), ("kv", _vp),
                 ("kv_scale", _vp), ("swa", _vp), ("sink", _vp), ("tau", C.c_float),
                 ("rope_base", C.c_float), ("derotate", C.c_int32), ("out", _vp), ("lse", _vp),
-                ("dev_status", _vp), ("flags", C.c_uint32), ("merge_wait_ns", C.c_int64),
-                ("pages", Pages)]
-
-
-ATTN_SEPARATE_MERGE = 1
+                ("dev_status", _vp), ("pages", Pages)]
 
 
 class PrefillArgs(C.Structure):
@@ -454,16 +450,13 @@ def indexer_topk(n_entries, q_fp4, q_sf, w, k_fp4, k_sf, k: int, *, workspace=No
 
 # ------------------------------------------------------------------ attention
 def attn_workspace(B: int, H: int, rows_max: int, device="cuda") -> torch.Tensor:
-    """A zero-filled workspace (the library keeps its meeting words consistent between
-    calls; re-zero it after a call that reported a non-zero device status)."""
     n = lib().csa_attn_workspace_size(B, H, rows_max)
-    return torch.zeros(max(n, 256), dtype=torch.uint8, device=device)
+    return torch.empty(max(n, 256), dtype=torch.uint8, device=device)
 
 
 def _attn(fn: str, sparse: bool, q, pos, n_entries, kv, kv_scale, swa, sink, idx, *,
           tau: float = 0.0, rope_base: float = 10000.0, derotate: bool = True,
           workspace=None, out=None, lse: bool = False, dev_status=None,
-          separate_merge: bool = False, merge_wait_ns: int = 0,
           paging: Paging | None = None, stream=None):
     B, H, _ = q.shape
     _dim(q, 2, HEAD_DIM, "q")
@@ -489,8 +482,7 @@ def _attn(fn: str, sparse: bool, q, pos, n_entries, kv, kv_scale, swa, sink, idx
                     _ptr(kv_scale, elem=4, name="kv_scale"), _ptr(swa, elem=2, name="swa"),
                     _ptr(sink, elem=4, name="sink"), tau, rope_base, int(derotate),
                     _ptr(out, elem=2, name="out"), _ptr(l, elem=4, name="lse"),
-                    _ptr(dev_status, elem=4, name="dev_status"),
-                    ATTN_SEPARATE_MERGE if separate_merge else 0, int(merge_wait_ns), pg)
+                    _ptr(dev_status, elem=4, name="dev_status"), pg)
     if noalloc:
         _check(getattr(lib(), fn)(C.byref(args), _stream(stream)), fn)
     else:

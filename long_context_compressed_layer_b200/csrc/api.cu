@@ -406,8 +406,7 @@ static int attn_common(const csa_attn_args* a, int sparse, void* ws, size_t ws_b
                        csa_stream_t stream) {
   if (!a) return CSA_ERR_INVALID_ARG;
   if (a->B < 0 || a->Nmax < 0 || (sparse && a->k < 1) || !(a->tau >= 0.f) ||
-      !(a->rope_base > 0.f) || (a->derotate != 0 && a->derotate != 1) ||
-      (a->flags & ~CSA_ATTN_SEPARATE_MERGE) || a->merge_wait_ns < 0)
+      !(a->rope_base > 0.f) || (a->derotate != 0 && a->derotate != 1))
     return CSA_ERR_INVALID_ARG;
   if (a->H != 64 && a->H != 128) return CSA_ERR_UNSUPPORTED;
   if ((sparse && a->k > 2048) || a->B > 65535 || a->Nmax > ((int64_t)1 << 30))

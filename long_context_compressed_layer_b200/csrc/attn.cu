@@ -18,27 +18,15 @@
 //   - two tcgen05.mma N = 256 halves compute O[128 x 512] in TMEM (S's columns are reused);
 //   - O / l (FP16, [8-dim group][head][8] so every warp store covers 512 contiguous bytes),
 //     m and l go to the workspace.
-// The chunks of a sequence are then merged in fixed order with the sink, normalised, the
-// last 64 dims de-rotated, and stored as BF16 (and lse). When every chunk CTA of the grid
-// can be resident, the kernel is a cooperative launch and its chunk CTAs do this
-// themselves: the C chunks of a sequence meet on a barrier in the workspace, then chunk
-// c merges 1/C of the (32-dim block, head) units from the partials in L2. Otherwise
-// attn_combine_kernel does it as a second launch. The chunk count depends only on k (CSA)
-// or n (HCA), never on the batch, and both merges sum the chunks in index order, so
-// results are batch-invariant.
+// attn_combine_kernel then merges the chunks of a sequence in fixed order with the sink,
+// normalises, de-rotates the last 64 dims and stores BF16 (and lse). The chunk count
+// depends only on k (CSA) or n (HCA), never on the batch, so results are batch-invariant.
 #include "common.cuh"
 
 namespace csa {
 
 constexpr int kAtRows = 64;  // rows per chunk = N of the S MMA
 constexpr int kAtThreads = 256;
-// The chunk meeting of the cooperative launch: per sequence a generation word and one flag
-// per chunk, at fixed places at the start of the workspace (any call shape finds them
-// there). A cooperative launch holds at most one CTA per SM, so it covers at most
-// kMeetMaxB sequences and kMeetMaxC chunks of one sequence.
-constexpr int kMeetMaxB = 256;
-constexpr int kMeetMaxC = 256;
-
 struct AtSmem {
   uint8_t q[8][128 * 128];      // 8 K-blocks of [128 heads x 64 dims] fp16, 128-B swizzle
   uint8_t v[8][kAtRows * 128];  // 8 dim-blocks of [64 rows x 64 dims] fp16, 128-B swizzle
@@ -49,10 +37,6 @@ struct AtSmem {
   float scale[kAtRows];         // the row's factor (entry scale; 1 for window rows)
   float mx[2][128], sm[2][128]; // the two column halves' max and sum per head
   float inv_l[128];             // 1 / (chunk sum) per head
-  float rot[64];                // merge: de-rotation cos, sin per RoPE pair
-  float sink[128];              // merge: the sink logits
-  float mg_M[128], mg_iz[128];  // merge: per head M and 1 / Z
-  uint32_t gen;                 // merge: the sequence's meeting generation at the start
   uint64_t q_full, s_done, o_done;
   uint32_t tmem_base;
 };
@@ -73,10 +57,8 @@ struct AtParams {
   float* lse;
   __half* part_o;  // [B][C][64][H][8]: chunk output / chunk sum, fp16, 8-dim groups
   float2* part_ml; // [B][C][H]: (chunk max logit, chunk sum)
+  float* rot;      // [B][64]: cos, sin of -t theta_j per RoPE pair (chunk 0 writes them)
   PageMap pm;         // where the entries live (contiguous or paged)
-  uint32_t* meet;     // generations [kMeetMaxB], then flags [kMeetMaxB][2][kMeetMaxC]
-  int fused;          // 1: cooperative launch, the chunk CTAs merge (no combine kernel)
-  uint64_t wait_ns;   // time limit of the chunk meeting
   int32_t* dev_status;
 };
 
@@ -138,201 +120,6 @@ __device__ __forceinline__ int at_rows_total(const AtParams& p, int n) {
 }
 
 
-// The merge of the C_b chunk partials of sequence b, shared by the cooperative kernel and
-// attn_combine_kernel so that both give the same bits. Per head h: M = max(sink, chunk
-// maxima m_c); e_c = exp(m_c - M) l_c; Z = e_0 + e_1 + ... + e_{C_b-1} + exp(sink - M),
-// summed in that order; out = (sum_c e_c o_c) / Z with o_c the chunk's normalised output,
-// chunks taken in index order; lse = M + log Z. Rounding steps are explicit (no
-// contraction), so the result does not depend on how the work is spread.
-__device__ __forceinline__ float chunk_weight(float2 ml, float M) {
-  return (M == INFINITY || ml.x == -INFINITY) ? 0.f : __fmul_rn(expf(ml.x - M), ml.y);
-}
-
-// The sequence's chunk statistics [C_b][H] (max, sum) into shared memory, all threads.
-__device__ __forceinline__ void merge_load_stats(const AtParams& p, int b, int C_b, int nthreads,
-                                                 float2* ml_s) {
-  const float2* src = p.part_ml + (size_t)b * p.C * p.H;
-  const int n = C_b * p.H;
-#pragma unroll 8
-  for (int i = threadIdx.x; i < n; i += nthreads) ml_s[i] = __ldcg(src + i);
-}
-
-// thread of head h, statistics in shared memory (ml_s, from merge_load_stats) or, when
-// ml_s is null, in global memory: M, 1/Z (0 when Z is 0 or infinite), e_c in place of the
-// chunk maxima (ml_s[c * H + h].x), and lse when asked
-__device__ void merge_head_stats(const AtParams& p, int b, int h, int C_b, float2* ml_s,
-                                 float sink, float* M_out, float* inv_z, bool write_lse) {
-  const float2* g = p.part_ml + (size_t)b * p.C * p.H + h;
-  auto ml = [&](int c0) { return ml_s ? ml_s[c0 * p.H + h] : __ldcg(g + (size_t)c0 * p.H); };
-  float M = sink;
-  for (int c0 = 0; c0 < C_b; ++c0) M = fmaxf(M, ml(c0).x);
-  float Z = 0.f;
-  for (int c0 = 0; c0 < C_b; ++c0) {
-    const float e = chunk_weight(ml(c0), M);
-    if (ml_s) ml_s[c0 * p.H + h].x = e;
-    Z = __fadd_rn(Z, e);
-  }
-  if (M == INFINITY)
-    Z = INFINITY;
-  else
-    Z = __fadd_rn(Z, sink == -INFINITY ? 0.f : expf(sink - M));
-  M_out[h] = M;
-  inv_z[h] = (Z > 0.f && Z < INFINITY) ? 1.f / Z : 0.f;
-  if (write_lse && p.lse) p.lse[(size_t)b * p.H + h] = M == INFINITY ? INFINITY : M + logf(Z);
-}
-
-// units [u0, u1) of the 16 H units (32-dim block cc, head h), u = cc H + h, four threads
-// (of nthreads) per unit, eight dims each, two units per thread per pass with all of their
-// loads in flight together; e_c from shared memory (the .x of ml_s after
-// merge_head_stats), or recomputed from the chunk statistics when ml_s is null (the same
-// expression). kMgBatch: chunk partials loaded together per unit; the sums run in chunk
-// order whatever it is.
-__device__ __forceinline__ void merge_finish(const AtParams& p, int b, int u, float* o,
-                                             const float* inv_z, const float* rot) {
-  const int cc = u / p.H, h = u - cc * p.H, d0 = cc * 32 + (threadIdx.x & 3) * 8;
-  const float iz = inv_z[h];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) o[e] = __fmul_rn(o[e], iz);
-  if (p.derotate && d0 >= kNope) {
-#pragma unroll
-    for (int e = 0; e < 8; e += 2) {
-      const int j = (d0 + e - kNope) >> 1;
-      const float cs = rot[2 * j], sn = rot[2 * j + 1];
-      const float x0 = o[e], x1 = o[e + 1];
-      o[e] = fmaf(x0, cs, __fmul_rn(x1, sn));
-      o[e + 1] = fmaf(-x0, sn, __fmul_rn(x1, cs));
-    }
-  }
-  uint4 pk;
-  pk.x = (uint32_t)f32_to_bf16_bits(o[0]) | ((uint32_t)f32_to_bf16_bits(o[1]) << 16);
-  pk.y = (uint32_t)f32_to_bf16_bits(o[2]) | ((uint32_t)f32_to_bf16_bits(o[3]) << 16);
-  pk.z = (uint32_t)f32_to_bf16_bits(o[4]) | ((uint32_t)f32_to_bf16_bits(o[5]) << 16);
-  pk.w = (uint32_t)f32_to_bf16_bits(o[6]) | ((uint32_t)f32_to_bf16_bits(o[7]) << 16);
-  *reinterpret_cast<uint4*>(p.out + ((size_t)b * p.H + h) * kD + d0) = pk;
-}
-
-template <int kMgBatch>
-__device__ void merge_units(const AtParams& p, int b, int C_b, int u0, int u1, int nthreads,
-                            const float2* ml_s, const float* Ms, const float* inv_z,
-                            const float* rot) {
-  const int tid = threadIdx.x, per = nthreads / 4;
-  const size_t cstride = (size_t)64 * p.H * 8;  // halves from one chunk's partial to the next
-  for (int ua = u0 + (tid >> 2); ua < u1; ua += 2 * per) {
-    const int ub = ua + per;
-    const bool has_b = ub < u1;
-    const __half* src[2];
-    int hu[2];
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int u = k ? (has_b ? ub : ua) : ua;
-      const int cc = u / p.H, h = u - cc * p.H, g = cc * 4 + (tid & 3);
-      src[k] = p.part_o + (((size_t)b * p.C * 64 + g) * p.H + h) * 8;
-      hu[k] = h;
-    }
-    float o[2][8];
-#pragma unroll
-    for (int k = 0; k < 2; ++k)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) o[k][e] = 0.f;
-    for (int c0 = 0; c0 < C_b; c0 += kMgBatch) {
-      uint4 v[2][kMgBatch];
-#pragma unroll
-      for (int k = 0; k < 2; ++k)
-#pragma unroll
-        for (int i = 0; i < kMgBatch; ++i)
-          v[k][i] = (c0 + i < C_b && (k == 0 || has_b))
-                        ? __ldcg(reinterpret_cast<const uint4*>(src[k] + (size_t)(c0 + i) * cstride))
-                        : make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        const float2* ml = p.part_ml + (size_t)b * p.C * p.H + hu[k];
-#pragma unroll
-        for (int i = 0; i < kMgBatch; ++i) {
-          if (c0 + i >= C_b) break;
-          const float w = ml_s ? ml_s[(c0 + i) * p.H + hu[k]].x
-                               : chunk_weight(__ldcg(ml + (size_t)(c0 + i) * p.H), Ms[hu[k]]);
-          const uint32_t x[4] = {v[k][i].x, v[k][i].y, v[k][i].z, v[k][i].w};
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&x[q]));
-            o[k][2 * q] = fmaf(w, f.x, o[k][2 * q]);
-            o[k][2 * q + 1] = fmaf(w, f.y, o[k][2 * q + 1]);
-          }
-        }
-      }
-    }
-    merge_finish(p, b, ua, o[0], inv_z, rot);
-    if (has_b) merge_finish(p, b, ub, o[1], inv_z, rot);
-  }
-}
-
-// the de-rotation table by the 32 threads from `first`
-__device__ __forceinline__ void merge_rot_table(const AtParams& p, int b, int first, float* rot) {
-  const int j = (int)threadIdx.x - first;
-  if (j >= 0 && j < 32 && p.derotate) {
-    float cs, sn;
-    rope_cos_sin((double)p.pos[b], j, (double)p.rope_base, &cs, &sn);
-    rot[2 * j] = cs;
-    rot[2 * j + 1] = sn;
-  }
-}
-
-// The chunk meetings of the cooperative launch. With g the sequence's generation read at
-// the start of the kernel, a chunk publishes flag[b][k][c] = g + 1 (a release store after
-// every store it makes part of) and waits (at most wait_ns, then CSA_ERR_TIMEOUT) until the
-// flags k of all C_b chunks of its sequence have reached g + 1. Flags only grow by one per
-// call, so a flag left by an earlier call is below g + 1; chunk 0 advances the generation
-// once the last meeting has passed. Meeting 0 follows the chunk statistics (max, sum),
-// meeting 1 the partial outputs.
-__device__ bool chunk_meet(const AtParams& p, AtSmem& s, int b, int c, int C_b, int k) {
-  const int tid = threadIdx.x;
-  uint32_t* flags = p.meet + kMeetMaxB + ((size_t)b * 2 + k) * kMeetMaxC;
-  const uint32_t target = s.gen + 1;
-  __syncthreads();  // the CTA's stores before the meeting are issued
-  if (tid == 0) {
-    __threadfence();
-    asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flags + c), "r"(target) : "memory");
-  }
-  bool ok = true;
-  if (tid < C_b) {
-    const uint64_t t0 = globaltimer();
-    while (true) {
-      uint32_t v;
-      asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flags + tid) : "memory");
-      if ((int32_t)(v - target) >= 0) break;
-      if (globaltimer() - t0 > p.wait_ns) {
-        report(p.dev_status, CSA_ERR_TIMEOUT);
-        ok = false;
-        break;
-      }
-    }
-  }
-  return __syncthreads_and(ok) != 0;
-}
-
-// After meeting 0 (while this chunk's O product runs): the merge weights of the sequence,
-// e_c in place of the chunk maxima in s.q (the S product has finished with Q), M and 1/Z
-// per head, lse (chunk 0), and the de-rotation table.
-__device__ bool attn_merge_stats(const AtParams& p, AtSmem& s, int b, int c, int C_b) {
-  merge_rot_table(p, b, 32, s.rot);
-  if (!chunk_meet(p, s, b, c, C_b, 0)) return false;
-  float2* ml_s = reinterpret_cast<float2*>(s.q[0]);  // [C_b][H] <= 128 KB
-  merge_load_stats(p, b, C_b, kAtThreads, ml_s);
-  __syncthreads();
-  if ((int)threadIdx.x < p.H)
-    merge_head_stats(p, b, threadIdx.x, C_b, ml_s, s.sink[threadIdx.x], s.mg_M, s.mg_iz, c == 0);
-  return true;  // (the CTA barrier before the partial store orders these writes)
-}
-
-// After meeting 1: the merge of units [c U / C_b, (c + 1) U / C_b).
-__device__ void attn_merge_out(const AtParams& p, AtSmem& s, int b, int c, int C_b) {
-  if (!chunk_meet(p, s, b, c, C_b, 1)) return;
-  if (threadIdx.x == 0 && c == 0) p.meet[b] = s.gen + 1;  // every chunk read it long ago
-  const int U = 16 * p.H;
-  merge_units<18>(p, b, C_b, (int)((int64_t)c * U / C_b), (int)((int64_t)(c + 1) * U / C_b),
-                  kAtThreads, reinterpret_cast<const float2*>(s.q[0]), s.mg_M, s.mg_iz, s.rot);
-}
-
 // The staged row of entry r is v'_r = [codes (448 dims, exact in FP16) | rope dims / scale_r]
 // with scale_r its entry scale, and a window row is itself with scale 1. Then
 //   q . v_r = scale_r (q . v'_r)   and   sum_r p_r v_r = sum_r (p_r scale_r) v'_r,
@@ -364,9 +151,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   const int nwin_first = p.sparse ? p.k : n;  // list index of the first window row
 
   if (tid == 0) {
-    // the sequence's meeting generation, read before this chunk can publish its flag
-    if (p.fused)
-      asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(s.gen) : "l"(p.meet + b) : "memory");
     mbar_init(&s.q_full, 1);
     mbar_init(&s.s_done, 1);
     mbar_init(&s.o_done, 1);
@@ -376,7 +160,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     for (int blk = 0; blk < 8; ++blk) tma_load_2d(s.q[blk], &qmap, &s.q_full, blk * 64, b * p.H);
   }
   if (warp == 0) tmem_alloc(&s.tmem_base, 512);
-  if (tid < p.H) s.sink[tid] = p.sink[tid];
   // Q rows H..127 are zero padding (generic-proxy writes, fenced below)
   if (p.H < 128) {
     for (int i = tid; i < 8 * (128 - p.H) * 8; i += kAtThreads) {
@@ -487,6 +270,12 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
     mma_commit(&s.s_done);
   }
+  // chunk 0's warp 1: the de-rotation table of the sequence, while S is computed
+  if (c == 0 && warp == 1 && p.derotate) {
+    float cs, sn;
+    rope_cos_sin((double)t, tid & 31, (double)p.rope_base, &cs, &sn);
+    *reinterpret_cast<float2*>(p.rot + (size_t)b * 64 + 2 * (tid & 31)) = make_float2(cs, sn);
+  }
   {
     const bool waited = mbar_wait(&s.s_done, 0, p.dev_status);
     ok = __syncthreads_and(ok && waited) != 0;
@@ -562,8 +351,6 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     }
     mma_commit(&s.o_done);
   }
-  const int C_b = (rows_total + kAtRows - 1) / kAtRows;
-  bool merge_ok = p.fused && attn_merge_stats(p, s, b, c, C_b);
   mbar_wait(&s.o_done, 0, p.dev_status);
   __syncthreads();  // inv_l written by threads 0-127 above
   tc_fence_after();
@@ -605,36 +392,108 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-  if (merge_ok) attn_merge_out(p, s, b, c, C_b);
 }
 
-// The merge as a second launch, for grids that cannot be resident at once (or on
-// request): CTA (c, b) does what chunk c of sequence b does after the meeting in the
-// cooperative launch, with the same arithmetic. e_c stays in shared memory when the
-// sequence's chunks fit, else each unit recomputes it from the chunk statistics.
-constexpr int kCbThreads = 256;
-constexpr int kCbSmemStats = 5120;  // 40 KB of (max, sum) pairs
+// The merge of the chunk partials: one thread per (8-dim group g, head h) of a sequence,
+// CTA (g, b). Every load a thread needs (the C_b chunk statistics of its head and its
+// C_b partial groups) is issued before any is used, in batches of kCbBatch chunks. Per
+// head: M = max(sink, m_c), e_c = exp(m_c - M) l_c, Z = e_0 + ... + e_{C_b-1} +
+// exp(sink - M) in chunk order, out = (sum_c e_c o_c) / Z in chunk order (o_c the chunk's
+// normalised output), lse = M + log Z; the RoPE dims are de-rotated by -t theta_j.
+constexpr int kCbBatch = 18;
 
-__global__ void __launch_bounds__(kCbThreads) attn_combine_kernel(AtParams p) {
-  const int c = blockIdx.x, b = blockIdx.y;
-  __shared__ float2 ml_s[kCbSmemStats];
-  __shared__ float Ms[128], inv_z[128], rot[64];
+__global__ void __launch_bounds__(128) attn_combine_kernel(AtParams p) {
+  const int g = blockIdx.x, b = blockIdx.y, h = threadIdx.x;
   pdl_wait();
   pdl_trigger();
+  if (h >= p.H) return;
   int n = p.n_entries[b];
   n = n < 0 ? 0 : (n > p.Nmax ? (int)p.Nmax : n);
   const int C_b = (at_rows_total(p, n) + kAtRows - 1) / kAtRows;
-  if (c >= C_b) return;
-  float2* stats = C_b * p.H <= kCbSmemStats ? ml_s : nullptr;
-  merge_rot_table(p, b, 32, rot);
-  if (stats) merge_load_stats(p, b, C_b, kCbThreads, stats);
-  __syncthreads();
-  if ((int)threadIdx.x < p.H)
-    merge_head_stats(p, b, threadIdx.x, C_b, stats, p.sink[threadIdx.x], Ms, inv_z, c == 0);
-  __syncthreads();
-  const int U = 16 * p.H;
-  merge_units<9>(p, b, C_b, (int)((int64_t)c * U / C_b), (int)((int64_t)(c + 1) * U / C_b),
-                 kCbThreads, stats, Ms, inv_z, rot);
+  const float2* ml = p.part_ml + (size_t)b * p.C * p.H + h;
+  const __half* src = p.part_o + (((size_t)b * p.C * 64 + g) * p.H + h) * 8;
+  const size_t cstride = (size_t)64 * p.H * 8;  // halves from one chunk's partial to the next
+  const float sink = p.sink[h];
+  float M = sink, Z = 0.f;
+  float o[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (C_b <= kCbBatch) {  // the usual case: one round trip
+    float2 st[kCbBatch];
+    uint4 v[kCbBatch];
+#pragma unroll
+    for (int c = 0; c < kCbBatch; ++c) {
+      st[c] = c < C_b ? __ldcg(ml + (size_t)c * p.H) : make_float2(-INFINITY, 0.f);
+      v[c] = c < C_b ? __ldcg(reinterpret_cast<const uint4*>(src + (size_t)c * cstride))
+                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int c = 0; c < kCbBatch; ++c) M = fmaxf(M, st[c].x);
+#pragma unroll
+    for (int c = 0; c < kCbBatch; ++c) {
+      if (c >= C_b) break;
+      const float e = (M == INFINITY || st[c].x == -INFINITY) ? 0.f
+                                                              : __fmul_rn(expf(st[c].x - M), st[c].y);
+      Z = __fadd_rn(Z, e);
+      const uint32_t x[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&x[q]));
+        o[2 * q] = fmaf(e, f.x, o[2 * q]);
+        o[2 * q + 1] = fmaf(e, f.y, o[2 * q + 1]);
+      }
+    }
+  } else {  // long HCA rows: the maximum first, then batches of chunks
+    for (int c = 0; c < C_b; ++c) M = fmaxf(M, __ldcg(ml + (size_t)c * p.H).x);
+    for (int c0 = 0; c0 < C_b; c0 += kCbBatch) {
+      float2 st[kCbBatch];
+      uint4 v[kCbBatch];
+#pragma unroll
+      for (int i = 0; i < kCbBatch; ++i) {
+        st[i] = c0 + i < C_b ? __ldcg(ml + (size_t)(c0 + i) * p.H) : make_float2(-INFINITY, 0.f);
+        v[i] = c0 + i < C_b ? __ldcg(reinterpret_cast<const uint4*>(src + (size_t)(c0 + i) * cstride))
+                            : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll
+      for (int i = 0; i < kCbBatch; ++i) {
+        if (c0 + i >= C_b) break;
+        const float e = (M == INFINITY || st[i].x == -INFINITY) ? 0.f
+                                                                : __fmul_rn(expf(st[i].x - M), st[i].y);
+        Z = __fadd_rn(Z, e);
+        const uint32_t x[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&x[q]));
+          o[2 * q] = fmaf(e, f.x, o[2 * q]);
+          o[2 * q + 1] = fmaf(e, f.y, o[2 * q + 1]);
+        }
+      }
+    }
+  }
+  if (M == INFINITY)
+    Z = INFINITY;
+  else
+    Z = __fadd_rn(Z, sink == -INFINITY ? 0.f : expf(sink - M));
+  const float iz = (Z > 0.f && Z < INFINITY) ? 1.f / Z : 0.f;
+  if (g == 0 && p.lse) p.lse[(size_t)b * p.H + h] = M == INFINITY ? INFINITY : M + logf(Z);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) o[e] = __fmul_rn(o[e], iz);
+  const int d0 = g * 8;
+  if (p.derotate && d0 >= kNope) {  // pairs 4(g - 56) .. +3 from chunk 0's table
+    const float4* rt = reinterpret_cast<const float4*>(p.rot + (size_t)b * 64 + 2 * (d0 - kNope) / 2);
+    const float4 r0 = __ldcg(rt), r1 = __ldcg(rt + 1);
+    const float cs[4] = {r0.x, r0.z, r1.x, r1.z}, sn[4] = {r0.y, r0.w, r1.y, r1.w};
+#pragma unroll
+    for (int e = 0; e < 8; e += 2) {
+      const float x0 = o[e], x1 = o[e + 1];
+      o[e] = fmaf(x0, cs[e / 2], __fmul_rn(x1, sn[e / 2]));
+      o[e + 1] = fmaf(-x0, sn[e / 2], __fmul_rn(x1, cs[e / 2]));
+    }
+  }
+  uint4 pk;
+  pk.x = (uint32_t)f32_to_bf16_bits(o[0]) | ((uint32_t)f32_to_bf16_bits(o[1]) << 16);
+  pk.y = (uint32_t)f32_to_bf16_bits(o[2]) | ((uint32_t)f32_to_bf16_bits(o[3]) << 16);
+  pk.z = (uint32_t)f32_to_bf16_bits(o[4]) | ((uint32_t)f32_to_bf16_bits(o[5]) << 16);
+  pk.w = (uint32_t)f32_to_bf16_bits(o[6]) | ((uint32_t)f32_to_bf16_bits(o[7]) << 16);
+  *reinterpret_cast<uint4*>(p.out + ((size_t)b * p.H + h) * kD + d0) = pk;
 }
 
 // ------------------------------------------------------------- prefill attention
@@ -1027,16 +886,14 @@ cudaError_t launch_prefill_attn(const csa_attn_args& a, const __half* rows16, in
 
 size_t at_smem_bytes() { return sizeof(AtSmem) + 1024; }
 
-// workspace: the chunk meeting words (generations [kMeetMaxB], flags [kMeetMaxB][2][kMeetMaxC])
-// first, at the same place for every call shape, then partial outputs [B][C][64][H][8]
-// fp16 and (max, sum) [B][C][H], each part 256-byte aligned
+// workspace: partial outputs [B][C][64][H][8] fp16, then (max, sum) [B][C][H], then the
+// de-rotation tables [B][64], each 256-byte aligned
 static size_t at_align(size_t x) { return (x + 255) & ~(size_t)255; }
-constexpr size_t kMeetBytes = (size_t)kMeetMaxB * (1 + 2 * kMeetMaxC) * sizeof(uint32_t);
 
 size_t at_workspace_size(int B, int H, int rows_max) {
   const size_t C = (size_t)(rows_max + kAtRows - 1) / kAtRows;
-  return kMeetBytes + at_align((size_t)B * C * H * kD * sizeof(__half)) +
-         at_align((size_t)B * C * H * sizeof(float2));
+  return at_align((size_t)B * C * H * kD * sizeof(__half)) +
+         at_align((size_t)B * C * H * sizeof(float2)) + at_align((size_t)B * 64 * sizeof(float));
 }
 
 cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* workspace,
@@ -1061,11 +918,10 @@ cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* 
   p.out = a.out;
   p.lse = a.lse;
   char* ws = reinterpret_cast<char*>(workspace);
-  p.meet = reinterpret_cast<uint32_t*>(ws);
-  p.part_o = reinterpret_cast<__half*>(ws + kMeetBytes);
-  p.part_ml = reinterpret_cast<float2*>(
-      ws + kMeetBytes + at_align((size_t)a.B * p.C * a.H * kD * sizeof(__half)));
-  p.wait_ns = a.merge_wait_ns > 0 ? (uint64_t)a.merge_wait_ns : kWaitLimitNs;
+  p.part_o = reinterpret_cast<__half*>(ws);
+  const size_t o_bytes = at_align((size_t)a.B * p.C * a.H * kD * sizeof(__half));
+  p.part_ml = reinterpret_cast<float2*>(ws + o_bytes);
+  p.rot = reinterpret_cast<float*>(ws + o_bytes + at_align((size_t)a.B * p.C * a.H * sizeof(float2)));
   p.pm = page_map(a.pages, a.Nmax);
   p.dev_status = a.dev_status;
   const size_t smem = at_smem_bytes();
@@ -1073,33 +929,10 @@ cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* 
   if (cudaError_t e = configure_smem_once(attn_chunk_kernel, smem, configured);
       e != cudaSuccess)
     return e;
-  // one cooperative launch whose chunk CTAs merge the partials themselves; the runtime
-  // refuses it when the grid cannot be resident all at once, and the combine kernel then
-  // merges in a second launch
-  // (the merge keeps the sequence's chunk statistics in the 128 KB of the Q buffer)
-  if (!(a.flags & CSA_ATTN_SEPARATE_MERGE) && a.B <= kMeetMaxB && p.C <= kMeetMaxC &&
-      (size_t)p.C * a.H * sizeof(float2) <= sizeof(AtSmem::q)) {
-    p.fused = 1;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.C, a.B);
-    cfg.blockDim = dim3(kAtThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[2];
-    attr[0].id = cudaLaunchAttributeCooperative;
-    attr[0].val.cooperative = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 2;
-    if (cudaLaunchKernelEx(&cfg, attn_chunk_kernel, qmap, p) == cudaSuccess) return cudaSuccess;
-    (void)cudaGetLastError();
-  }
-  p.fused = 0;
   cudaError_t e = launch_pdl(attn_chunk_kernel, dim3(p.C, a.B), dim3(kAtThreads), smem, stream,
                              qmap, p);
   if (e != cudaSuccess) return e;
-  return launch_pdl(attn_combine_kernel, dim3(p.C, a.B), dim3(kCbThreads), 0, stream, p);
+  return launch_pdl(attn_combine_kernel, dim3(64, a.B), dim3(128), 0, stream, p);
 }
 
 }  // namespace csa

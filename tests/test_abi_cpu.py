@@ -121,8 +121,6 @@ def test_attention_rejects_on_host(L):
     assert f(_attn_args(H=96)) == csa.CSA_ERR_UNSUPPORTED
     assert f(_attn_args(k=0)) == csa.CSA_ERR_INVALID_ARG
     assert f(_attn_args(derotate=2)) == csa.CSA_ERR_INVALID_ARG
-    assert f(_attn_args(flags=2)) == csa.CSA_ERR_INVALID_ARG  # an unknown flag bit
-    assert f(_attn_args(merge_wait_ns=-1)) == csa.CSA_ERR_INVALID_ARG
     # paged-cache descriptors: page size a power of two >= 128, pages covering Nmax,
     # an aligned table, a pool of at least one page
     for pages in (csa.Pages(FAKE, 32, 100, 8), csa.Pages(FAKE, 64, 64, 8),

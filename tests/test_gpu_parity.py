@@ -352,11 +352,11 @@ def _attn_case(B, H, Nmax, n, pos, k=None, seed=0, sink_override=None):
     return dict(q=q, pos=pos, n=n, kv=kv, sc=sc, swa=swa, sink=sink, idx=idx)
 
 
-def _gpu_attn(d, derotate=True, separate=False, raw=False):
+def _gpu_attn(d, derotate=True, raw=False):
     args = (dev(d["q"]), dev(d["pos"]), dev(d["n"]), dev(d["kv"]), dev(d["sc"]), dev(d["swa"]),
             dev(d["sink"]))
     st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    kw = dict(lse=True, derotate=derotate, separate_merge=separate, dev_status=st)
+    kw = dict(lse=True, derotate=derotate, dev_status=st)
     if d["idx"] is not None:
         out, lse = csa.sparse_attn_decode(*args, dev(d["idx"]), **kw)
     else:
@@ -381,56 +381,17 @@ def _ora_attn(d, derotate=True):
     (1, 128, 4096, [4096], [16383], 2048),                # CSA at the largest k
     (1, 64, 8192, [8192], [1048575], None),               # HCA over a 1M-token context
 ])
-@pytest.mark.parametrize("separate", [False, True])
-def test_attention_matches_oracle(B, H, Nmax, n, pos, k, separate):
-    # separate: the chunk partials merged by a second kernel, the path of grids that cannot
-    # be resident at once; otherwise one cooperative launch merges them itself
+def test_attention_matches_oracle(B, H, Nmax, n, pos, k):
     d = _attn_case(B, H, Nmax, n, pos, k, seed=H + B)
-    out, lse = _gpu_attn(d, separate=separate)
+    out, lse = _gpu_attn(d)
     want, wlse = _ora_attn(d)
     compare.close(out, want, what="attention out")
     np.testing.assert_allclose(lse, wlse, rtol=1e-4, atol=1e-4)
 
 
-@pytest.mark.parametrize("B,H,Nmax,n,pos,k", [
-    (4, 128, 4096, [4096, 3000, 2000, 1500], [16383, 12001, 8003, 6000], 1024),
-    (3, 64, 1024, [1024, 7, 0], [131071, 900, 50], None),
-])
-def test_attention_merge_paths_agree_bitwise(B, H, Nmax, n, pos, k):
-    # which merge runs depends on whether the grid can be resident, i.e. on the batch; both
-    # must give the same bits so that a sequence's output does not depend on its batch
-    d = _attn_case(B, H, Nmax, n, pos, k, seed=77)
-    out_f, lse_f = _gpu_attn(d, raw=True)
-    out_s, lse_s = _gpu_attn(d, separate=True, raw=True)
-    np.testing.assert_array_equal(out_f, out_s)
-    np.testing.assert_array_equal(lse_f.view(np.int32), lse_s.view(np.int32))
-
-
-def test_attention_merge_wait_that_runs_out_reports_a_timeout():
-    # a 1 ns limit on the chunk meeting of the cooperative launch: every chunk but the
-    # last to arrive gives up at once. The call returns CSA_ERR_TIMEOUT; after the
-    # workspace is zero-filled again, as the interface asks after any error, the next call
-    # matches the oracle.
-    d = _attn_case(2, 128, 4096, [4096, 3000], [16383, 12001], 1024, seed=9)
-    args = (dev(d["q"]), dev(d["pos"]), dev(d["n"]), dev(d["kv"]), dev(d["sc"]), dev(d["swa"]),
-            dev(d["sink"]), dev(d["idx"]))
-    ws = csa.attn_workspace(2, 128, 1024 + 128)
-    st = torch.zeros(1, dtype=torch.int32, device="cuda")
-    csa.sparse_attn_decode(*args, workspace=ws, dev_status=st, merge_wait_ns=1)
-    torch.cuda.synchronize()
-    assert int(st.item()) == csa.CSA_ERR_TIMEOUT
-    ws.zero_()
-    st.zero_()
-    out = csa.sparse_attn_decode(*args, workspace=ws, dev_status=st)
-    torch.cuda.synchronize()
-    assert int(st.item()) == 0
-    want, _ = _ora_attn(d)
-    compare.close(out.float().cpu().numpy(), want, what="after the timeout")
-
-
 def test_attention_workspace_reused_across_calls_and_batches():
-    # the meeting words are left ready for the next call, also when the next call has
-    # other chunk counts per sequence (HCA lengths change between steps)
+    # one workspace for calls whose chunk counts per sequence change (HCA lengths grow
+    # between steps)
     ws = csa.attn_workspace(3, 64, 2048 + 128)
     for trial, n in enumerate(([2048, 100, 900], [700, 2048, 5], [64, 1, 2000])):
         d = _attn_case(3, 64, 2048, n, [9000, 8000, 7000], None, seed=trial)
