@@ -965,6 +965,7 @@ struct DxSel {
   uint32_t nin[kDxMaxCtas];           // their in-bin counts
   uint32_t above[kDxMaxCtas];         // their above-bin counts
   uint32_t pass[kDxMaxCtas];          // their in-bin candidates that pass the cut
+  uint32_t sub[kDxMaxCtas * 32];      // BF16 keys: their in-bin counts by the next 5 key bits
   uint32_t tmp[32];
   int32_t n[kIxMaxB];                 // eligible entries of the covered sequences
   int tbin;
@@ -1090,6 +1091,25 @@ __device__ void select_decode(const IxParams& p, uint8_t* scratch, const DxSmem&
       in += bin == tbin ? 1u : 0u;
     }
     uint32_t nin_tot, above_tot;
+    if (p.bf16) {
+      // 16-bit keys: the bin's 11 bits and the next 5 are the whole key, so the counts of
+      // the in-bin entries by those 5 bits (the CTA's slot, as 32 words) fix the cut
+      for (int i = tid; i < 32; i += NT) x.h[i] = 0;
+      __syncthreads();
+      for (int j = j0; j < j1; ++j) {
+        const uint32_t key = float_key(sc[j]);
+        if ((int)(key >> kLowBits) == tbin) atomicAdd(&x.h[(key >> 16) & 31u], 1u);
+      }
+      block_incl_scan<NT>(in, x.tmp, &nin_tot);
+      block_incl_scan<NT>(above, x.tmp, &above_tot);
+      if (tid < 32)
+        reinterpret_cast<uint32_t*>(p.ws.cand_slots + ((size_t)b * kDxMaxCtas + c) * kDxSlot)[tid] =
+            x.h[tid];
+      if (tid == 0)
+        p.ws.cta_cnt[(size_t)b * kDxMaxCtas + c] =
+            make_uint4(above_tot, nin_tot, (uint32_t)tbin, 0u);
+      continue;
+    }
     const uint32_t pos0 = block_incl_scan<NT>(in, x.tmp, &nin_tot) - in;
     block_incl_scan<NT>(above, x.tmp, &above_tot);
     if (in) {  // this thread's in-bin entries, in index order
@@ -1132,7 +1152,112 @@ __device__ void select_decode(const IxParams& p, uint8_t* scratch, const DxSmem&
     float* sout = p.scores_out ? p.scores_out + (size_t)b * p.k : nullptr;
     uint64_t v_cut = 0;  // n <= k: every entry (every value is >= 0), at its own index
     uint32_t base = (uint32_t)r.ja;
-    if (n > p.k) {
+    // BF16 keys: entries above the cut value cut16 (the key's top 16 bits) and entries at
+    // it with index <= cut_idx are selected (cut16 = -1: use v_cut)
+    int cut16 = -1;
+    int32_t cut_idx = -1;
+    if (n > p.k && p.bf16) {
+      const int nseg = c_hi - c_lo + 1;
+      const int myseg = c - c_lo;
+      uint32_t* sub = x.sub;  // [nseg][32]
+      // one round trip: every covering CTA's counts and its 32 sub-bin counts
+      for (int i = tid; i < nseg; i += NT) {
+        const int cc = c_lo + i;
+        const bool has = cta_q0(total, cc, G) < cta_q0(total, cc + 1, G);
+        const uint4 v = has ? __ldcg(p.ws.cta_cnt + (size_t)b * kDxMaxCtas + cc)
+                            : make_uint4(0u, 0u, 0u, 0u);
+        x.above[i] = v.x;
+        x.nin[i] = v.y;
+        if (cc == c) x.tbin = (int)v.z;
+      }
+      for (int e = tid; e < nseg * 32; e += NT) {
+        const int cc = c_lo + e / 32;
+        const bool has = cta_q0(total, cc, G) < cta_q0(total, cc + 1, G);
+        sub[e] = has ? __ldcg(reinterpret_cast<const uint32_t*>(
+                                  p.ws.cand_slots + ((size_t)b * kDxMaxCtas + cc) * kDxSlot) +
+                              (e & 31))
+                     : 0u;
+      }
+      if (tid < 32) x.h[tid] = 0;
+      __syncthreads();
+      uint32_t above_total, nin_total;
+      {
+        const uint32_t av = tid < nseg ? x.above[tid] : 0u;
+        const uint32_t nv = tid < nseg ? x.nin[tid] : 0u;
+        block_incl_scan<NT>(av, x.tmp, &above_total);
+        block_incl_scan<NT>(nv, x.tmp, &nin_total);
+      }
+      for (int e = tid; e < nseg * 32; e += NT)
+        if (sub[e]) atomicAdd(&x.h[e & 31], sub[e]);
+      __syncthreads();
+      const int tbin = x.tbin;
+      const int64_t need = (int64_t)k_eff - above_total;
+      if (need <= 0) {  // nothing from the bin (as in the fp32 path)
+        if (need < 0) report(p.dev_status, CSA_ERR_DEVICE);
+        v_cut = cand_value((uint32_t)(tbin + 1) << kLowBits, -1);
+      } else if (need >= (int64_t)nin_total) {  // the whole bin
+        if (need > (int64_t)nin_total) report(p.dev_status, CSA_ERR_DEVICE);
+        v_cut = cand_value((uint32_t)tbin << kLowBits, 0x7FFFFFFF);
+      } else {
+        if (tid == 0) {  // the sub-bin holding the need-th largest key, from the top
+          uint32_t cum = 0;
+          int sb = 31;
+          for (; sb > 0 && cum + x.h[sb] < (uint32_t)need; --sb) cum += x.h[sb];
+          x.off = (uint32_t)sb;
+          x.rem = (uint32_t)need - cum;  // entries wanted at the cut value, from 1
+        }
+        __syncthreads();
+        const uint32_t sb = x.off, need_in = x.rem;
+        cut16 = (tbin << 5) | (int)sb;
+        // per covering CTA: entries above the cut value, entries at it; the ties go to the
+        // smallest indices, i.e. to the CTAs in order
+        if (tid < 32) {
+          uint32_t before_gt = 0, before_tie = 0, my_tie = 0;
+          for (int i = tid; i < nseg; i += 32) {
+            uint32_t gt = 0;
+            for (int q = (int)sb + 1; q < 32; ++q) gt += sub[i * 32 + q];
+            const uint32_t tie = sub[i * 32 + sb];
+            if (i < myseg) { before_gt += x.above[i] + gt; before_tie += tie; }
+            if (i == myseg) my_tie = tie;
+          }
+          for (int o = 16; o > 0; o >>= 1) {
+            before_gt += __shfl_xor_sync(0xffffffffu, before_gt, o);
+            before_tie += __shfl_xor_sync(0xffffffffu, before_tie, o);
+            my_tie += __shfl_xor_sync(0xffffffffu, my_tie, o);
+          }
+          if (tid == 0) {
+            const uint32_t take_before = before_tie < need_in ? before_tie : need_in;
+            const uint32_t left = need_in - take_before;
+            const uint32_t take = my_tie < left ? my_tie : left;
+            x.off = before_gt + take_before;  // this CTA's output offset
+            x.pop = take;
+            x.cnt = my_tie;
+          }
+        }
+        __syncthreads();
+        base = x.off;
+        const uint32_t take = x.pop, my_tie = x.cnt;
+        if (take == 0) {
+          cut_idx = -1;
+        } else if (take == my_tie) {
+          cut_idx = 0x7FFFFFFF;
+        } else {  // the CTA where the cut falls: the index of its take-th entry at the cut
+          const float* scb = seq_scores(b, r, itb);
+          const int per = (r.jb - r.ja + NT - 1) / NT;
+          const int j0 = min(r.jb, r.ja + tid * per), j1 = min(r.jb, j0 + per);
+          uint32_t mt = 0;
+          for (int j = j0; j < j1; ++j) mt += (int)(float_key(scb[j]) >> 16) == cut16 ? 1u : 0u;
+          const uint32_t incl = block_incl_scan<NT>(mt, x.tmp, nullptr);
+          if (incl >= take && incl - mt < take) {
+            uint32_t cum = incl - mt;
+            for (int j = j0; j < j1; ++j)
+              if ((int)(float_key(scb[j]) >> 16) == cut16 && ++cum == take) { x.prefix = (uint32_t)j; break; }
+          }
+          __syncthreads();
+          cut_idx = (int32_t)x.prefix;
+        }
+      }
+    } else if (n > p.k) {
       const int nseg = c_hi - c_lo + 1;
       // one round trip: every covering CTA's counts and slot
       for (int i = tid; i < nseg; i += NT) {
@@ -1308,16 +1433,21 @@ __device__ void select_decode(const IxParams& p, uint8_t* scratch, const DxSmem&
       base = x.off;
     }
     {  // ordered write of this CTA's selected entries: each thread its contiguous run
+      auto selected = [&](float v, int j) {
+        if (cut16 < 0) return cand_value(float_key(v), j) >= v_cut;
+        const int k16 = (int)(float_key(v) >> 16);
+        return k16 > cut16 || (k16 == cut16 && j <= cut_idx);
+      };
       const int per = (r.jb - r.ja + NT - 1) / NT;
       const int j0 = min(r.jb, r.ja + tid * per), j1 = min(r.jb, j0 + per);
       uint32_t mine = 0;
-      for (int j = j0; j < j1; ++j) mine += cand_value(float_key(sc[j]), j) >= v_cut ? 1u : 0u;
+      for (int j = j0; j < j1; ++j) mine += selected(sc[j], j) ? 1u : 0u;
       uint32_t tot;
       uint32_t pos = base + block_incl_scan<NT>(mine, x.tmp, &tot) - mine;
       if (mine) {
         for (int j = j0; j < j1; ++j) {
           const float v = sc[j];
-          if (cand_value(float_key(v), j) < v_cut) continue;
+          if (!selected(v, j)) continue;
           if (pos < (uint32_t)p.k) {
             out[pos] = j;
             if (sout) sout[pos] = v;

@@ -226,6 +226,54 @@ def test_indexer_topk_bf16_scores_match_oracle(B, H_I, Nmax, n, k, planted):
     assert total <= 2 * B
 
 
+@pytest.mark.parametrize("B,H_I,Nmax,n,k,planted", [
+    (1, 16, 2048, [2048], 512, 0),
+    (3, 64, 4096, [4096, 2999, 130], 512, 0),
+    (2, 64, 16384, [16384, 12345], 1024, 8),
+    (4, 64, 65536, [65536, 60000, 30000, 900], 1024, 16),
+])
+def test_indexer_bf16_fused_selection_equals_separate_kernels(B, H_I, Nmax, n, k, planted):
+    # the cooperative launch's BF16 path (counts by the 5 key bits below the bin, ties
+    # split by index across CTAs) and the stand-alone selection kernels select on the same
+    # scores: the same indices
+    rng = np.random.default_rng(B * 13 + k)
+    n = np.asarray(n, dtype=np.int32)
+    ix = synth.indexer_inputs(rng, B, H_I, Nmax, n, planted)
+    args = (dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]), dev(ix["k_fp4"]),
+            dev(ix["k_sf"]), k)
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    fused = host(csa.indexer_topk(*args, bf16_scores=True, dev_status=st))
+    sep = host(csa.indexer_topk(*args, bf16_scores=True, separate_select=True, dev_status=st))
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(fused, sep)
+
+
+@pytest.mark.parametrize("separate", [False, True])
+def test_indexer_bf16_heavy_ties_exact(separate):
+    # unit scales and w = 1: scores are multiples of 1/4, exact in fp32 and, at these sizes,
+    # spread over few BF16 values, so thousands of entries tie at the cut; the selection
+    # must take the smallest indices among them, exactly as the oracle's BF16 selection
+    B, H_I, Nmax, k = 2, 16, 32768, 1024
+    rng = np.random.default_rng(17)
+    n = np.array([32768, 20000], np.int32)
+    ix = synth.indexer_inputs(rng, B, H_I, Nmax, n)
+    ix["q_sf"][:] = 127
+    ix["k_sf"][:] = 127
+    ix["w"][:] = 1.0
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx = host(csa.indexer_topk(dev(n), dev(ix["q_fp4"]), dev(ix["q_sf"]), dev(ix["w"]),
+                                dev(ix["k_fp4"]), dev(ix["k_sf"]), k, bf16_scores=True,
+                                separate_select=separate, dev_status=st))
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    ora = oracle.indexer_scores(n, ix["q_fp4"], ix["q_sf"], ix["w"], ix["k_fp4"], ix["k_sf"])
+    for b in range(B):
+        r = compare._bf16_round(ora[b][: n[b]])
+        assert (r == np.sort(r)[::-1][k - 1]).sum() > 50  # the case really has heavy ties
+        np.testing.assert_array_equal(idx[b], oracle.topk_bf16(ora[b][: n[b]], int(n[b]), k))
+
+
 def test_indexer_scores_exact_on_integer_case():
     # unit scales, w = 1: every score is a multiple of 1/4 below 2^24, exact in fp32
     B, H_I, Nmax, k = 1, 64, 1024, 1024
