@@ -257,6 +257,23 @@ def e2e_graphs(torch, launch, copies, inputs: dict, out_specs: dict, reps):
     return graphs, h_in.numel(), h_out.numel(), h_out_v
 
 
+def fp4_bf16_mma_rates(torch, csa, stream, iters: int = 20000) -> dict:
+    """Rates (TFLOP/s) of csa_mma_peak's back-to-back MMA loops, BF16 at N = 64 and 256 and
+    MXFP4 at N = 64, each timed with CUDA events after a warm-up launch, and the FP4 / BF16
+    ratio at the common shape N = 64."""
+    out = {}
+    for name, kind, N in (("bf16_n64", 1, 64), ("bf16_n256", 1, 256), ("mxf4_n64", 0, 64)):
+        csa.mma_peak(kind, N, iters)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        flops = sum(csa.mma_peak(kind, N, iters) for _ in range(5))
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name] = flops / (e0.elapsed_time(e1) * 1e-3) / 1e12
+    out["fp4_over_bf16"] = out["mxf4_n64"] / out["bf16_n64"]
+    return out
+
+
 def max_over_ranks(vals: list[float], world: int, device) -> list[float]:
     """Per-rank timings -> their maxima over all ranks (one all-reduce of a few floats,
     outside the data path)."""
@@ -392,6 +409,11 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
     op_flop = 2 * T * (G * d_g * K1 + d_model * G * d_g)
     del Wg, Wo, op_out, op_ws
 
+    # the tensor pipes' FP4 / BF16 rate ratio at one MMA shape (csa_mma_peak: back-to-back
+    # MMAs on shared-memory operands, M = 128, N = 64), which scales the measured BF16 GEMM
+    # peak into the FP4 peak of the roofline below
+    mma_rates = fp4_bf16_mma_rates(torch, csa, stream)
+
     # end to end: the new tokens' inputs go up from pinned host memory and the output
     # comes back, around the same call
     up = ("a", "b", "za", "zb", "q", "q_fp4", "q_sf", "w")
@@ -419,8 +441,9 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
     pk = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json"))) if os.path.exists(
         os.path.join(ROOT, "MEASURED_PEAKS.json")) else {}
     bf16_peak = pk.get("bf16_tflops_sustained", 1400.0)  # a long step: the sustained figure
-    # FP4 counts at the nominal 4x of dense BF16 (no FP4 peak is measured on this machine)
-    eq_tflops = (f4 / 4 + f16) / (ms * 1e-3) / 1e12
+    # FP4 FLOPs weighted by the measured BF16 / FP4 tensor-rate ratio (1/4 nominally)
+    fp4_ratio = mma_rates["fp4_over_bf16"]
+    eq_tflops = (f4 / fp4_ratio + f16) / (ms * 1e-3) / 1e12
     line = {
         "metric": PREFILL_METRIC, "value": whole_job_rate(T, world, ms), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": max(args.warmup, 3),
@@ -448,8 +471,11 @@ def bench_prefill(args, rank: int, world: int, local: int) -> None:
                      "frac": eq_tflops / bf16_peak,
                      "nominal_peak": NOMINAL_BF16_TFLOPS,
                      "frac_of_nominal": eq_tflops / NOMINAL_BF16_TFLOPS,
-                     "peak_src": ("measured sustained bf16; FP4 FLOPs weighted 1/4 (nominal ratio)"
+                     "peak_src": (f"measured sustained bf16; FP4 FLOPs weighted 1/{fp4_ratio:.2f} "
+                                  "(FP4 / BF16 tensor-rate ratio measured by csa_mma_peak)"
                                   if "bf16_tflops_sustained" in pk else "fallback"),
+                     "fp4_peak_tflops": bf16_peak * fp4_ratio,
+                     "mma_peak": mma_rates,
                      "traffic": None},
         "clocks": clocks,
         "e2e": {"value": whole_job_rate(T, world, e2e_ms), "unit": "tokens/s",

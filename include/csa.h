@@ -500,6 +500,20 @@ int csa_grouped_out_proj(const csa_oproj_args* args, void* workspace, size_t wor
 #define CSA_NOALLOC_SCRATCH_BYTES (12u << 20)
 int csa_sparse_attn_decode_noalloc(const csa_attn_args* args, csa_stream_t stream);
 
+/* ------------------------------------------------------------------------------------
+ * csa_mma_peak: a measurement helper, not part of the layer. One CTA per SM issues `iters`
+ * back-to-back tcgen05 MMAs (M = 128) on operands resident in shared memory, with no DRAM
+ * traffic: kind = 0 is kind::mxf4 (E2M1 inputs, E8M0 block scales, K = 64 per MMA, N = 64),
+ * kind = 1 is kind::f16 with BF16 inputs (K = 16 per MMA, N = 64 or 256). The caller times
+ * the launch on `stream`; csa_mma_peak_flops gives the FLOPs of one launch on the current
+ * device (0 for an unsupported kind or N). The ratio of the two kinds' rates at one shape
+ * scales a measured BF16 GEMM peak into an FP4 one. iters in 1 .. 1e6; a wait that runs
+ * out writes CSA_ERR_TIMEOUT to dev_status (optional).
+ */
+int csa_mma_peak(int32_t kind, int32_t N, int32_t iters, int32_t* dev_status,
+                 csa_stream_t stream);
+double csa_mma_peak_flops(int32_t kind, int32_t N, int32_t iters);
+
 #ifdef __cplusplus
 }
 #endif

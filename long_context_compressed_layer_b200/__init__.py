@@ -133,7 +133,7 @@ EXPORTS = ["csa_status_string", "csa_compress", "csa_compress_index_keys", "csa_
            "csa_indexer_topk_workspace_size",
            "csa_indexer_topk", "csa_indexer_topk_bf16", "csa_attn_workspace_size", "csa_sparse_attn_decode",
            "hca_attn_decode", "csa_sparse_attn_decode_noalloc", "csa_prefill_workspace_size",
-           "csa_prefill"]
+           "csa_prefill", "csa_mma_peak", "csa_mma_peak_flops"]
 
 NOALLOC_SCRATCH_BYTES = 12 << 20
 
@@ -178,6 +178,10 @@ def lib() -> C.CDLL:
         L.csa_prefill.argtypes = [C.POINTER(PrefillArgs), _vp, C.c_size_t, _vp]
         L.csa_sparse_attn_decode_noalloc.restype = C.c_int
         L.csa_sparse_attn_decode_noalloc.argtypes = [C.POINTER(AttnArgs), _vp]
+        L.csa_mma_peak.restype = C.c_int
+        L.csa_mma_peak.argtypes = [C.c_int32, C.c_int32, C.c_int32, _vp, _vp]
+        L.csa_mma_peak_flops.restype = C.c_double
+        L.csa_mma_peak_flops.argtypes = [C.c_int32, C.c_int32, C.c_int32]
         _lib = L
     return _lib
 
@@ -405,6 +409,15 @@ def grouped_out_proj(attn, Wg, Wo, *, workspace=None, out=None, dev_status=None,
 
 
 # ------------------------------------------------------------- indexer top-k
+def mma_peak(kind: int, N: int, iters: int, *, dev_status=None, stream=None) -> float:
+    """Launch csa_mma_peak (a tensor-pipe throughput measurement: kind 0 = MXFP4 N = 64,
+    kind 1 = BF16 N = 64 or 256) on the stream; returns the FLOPs of the launch, which the
+    caller divides by the time it measures."""
+    _check(lib().csa_mma_peak(kind, N, iters, _ptr(dev_status, elem=4, name="dev_status"),
+                              _stream(stream)), "csa_mma_peak")
+    return float(lib().csa_mma_peak_flops(kind, N, iters))
+
+
 def indexer_topk_workspace(B: int, Nmax: int, k: int, device="cuda") -> torch.Tensor:
     """A zero-filled workspace (the library keeps it zeroed between calls)."""
     n = lib().csa_indexer_topk_workspace_size(B, Nmax, k)

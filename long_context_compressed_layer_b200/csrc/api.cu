@@ -29,6 +29,9 @@ cudaError_t launch_prefill_prep(const csa_prefill_args& a, __half* lin, int32_t*
                                 int32_t* pos_all, cudaStream_t stream);
 cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* workspace,
                         const CUtensorMap& qmap, cudaStream_t stream);
+double mma_peak_flops_per_cta(int kind, int N, int iters);
+cudaError_t launch_mma_peak(int kind, int N, int iters, int num_sms, int32_t* dev_status,
+                            cudaStream_t stream);
 
 namespace {
 
@@ -559,6 +562,28 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
   return CSA_OK;
+}
+
+static bool mma_peak_shape(int32_t kind, int32_t N, int32_t iters) {
+  return ((kind == 0 && N == 64) || (kind == 1 && (N == 64 || N == 256))) && iters >= 1 &&
+         iters <= 1000000;
+}
+
+int csa_mma_peak(int32_t kind, int32_t N, int32_t iters, int32_t* dev_status,
+                 csa_stream_t stream) {
+  if (!mma_peak_shape(kind, N, iters) ||
+      (dev_status && (reinterpret_cast<uintptr_t>(dev_status) & 3)))
+    return CSA_ERR_INVALID_ARG;
+  const int sms = num_sms();
+  if (sms <= 0) return CSA_ERR_CUDA;
+  return cuda_status(
+      launch_mma_peak(kind, N, iters, sms, dev_status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+double csa_mma_peak_flops(int32_t kind, int32_t N, int32_t iters) {
+  if (!mma_peak_shape(kind, N, iters)) return 0.0;
+  const int sms = num_sms();
+  return sms > 0 ? sms * mma_peak_flops_per_cta(kind, N, iters) : 0.0;
 }
 
 int csa_sparse_attn_decode_noalloc(const csa_attn_args* a, csa_stream_t stream) {

@@ -69,7 +69,7 @@ constexpr int kSelChunk = kSelThreads * kSelPer;  // entries per slice
 constexpr int kSeqWords = 8 + kHist;  // per-sequence block: counters[4], rule[4], hist
 
 struct IxWs {
-  uint32_t* grid_bar;   // two 64-bit arrival counters of the grid barriers
+  uint32_t* grid_bar;   // the two grid barriers' 64-bit counters, at words 0 and 32
   uint32_t* seq;        // [B][kSeqWords]
   uint32_t* slice_cnt;  // [B][S]: above-bin count per slice, then the slice's output offset
   float* scores;        // [B][Nmax]
@@ -101,7 +101,7 @@ __host__ __device__ inline size_t ix_ws_layout(int B, int64_t Nmax, int k, char*
     off += align256(bytes);
     return p;
   };
-  char* p0 = take(8);
+  char* p0 = take(512);
   char* p1 = take((size_t)B * kSeqWords * 4);
   char* p2 = take((size_t)B * S * 4);
   char* p3 = take((size_t)B * Nmax * 4);
@@ -926,15 +926,22 @@ __device__ void select_write(const IxParams& p, SelScratch& x, int b, int sb) {
 // reaches the end of that instance. Every CTA arrives, also one that has already given
 // up, so later instances stay aligned; a CTA with ok == false does not wait. The wait is
 // bounded by limit_ns. Returns ok && the wait completed.
+// Grid barrier of the cooperative launch on a monotone 64-bit counter of the workspace.
+// Every barrier adds exactly 2^20 to it whatever the grid size G: CTA c adds
+// floor(2^20 (c+1) / G) - floor(2^20 c / G), so the counter is a multiple of 2^20 whenever no
+// barrier is in progress, and a CTA waits (at most limit_ns, then CSA_ERR_TIMEOUT) for the
+// next multiple above the value it found. Calls of any grid size can share the workspace.
 __device__ bool grid_sync(unsigned long long* ctr, bool ok, uint64_t limit_ns,
                           int32_t* dev_status) {
   __shared__ int sh_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
+    constexpr unsigned long long kRound = 1ull << 20;
+    const unsigned long long G = gridDim.x, c = blockIdx.x;
+    const unsigned long long w = (kRound * (c + 1)) / G - (kRound * c) / G;
     unsigned long long old;
-    asm volatile("atom.add.release.gpu.global.u64 %0, [%1], 1;" : "=l"(old) : "l"(ctr) : "memory");
-    const unsigned long long G = gridDim.x;
-    const unsigned long long target = (old / G + 1) * G;
+    asm volatile("atom.add.release.gpu.global.u64 %0, [%1], %2;" : "=l"(old) : "l"(ctr), "l"(w) : "memory");
+    const unsigned long long target = ((old >> 20) + 1) << 20;
     if (ok) {
       const uint64_t t0 = globaltimer();
       while (true) {
@@ -1127,7 +1134,7 @@ __device__ void select_decode(const IxParams& p, uint8_t* scratch, const DxSmem&
     if (tid == 0)
       p.ws.cta_cnt[(size_t)b * kDxMaxCtas + c] = make_uint4(above_tot, nin_tot, (uint32_t)tbin, 0u);
   }
-  ok = grid_sync(reinterpret_cast<unsigned long long*>(p.ws.grid_bar) + 1, ok, p.wait_ns,
+  ok = grid_sync(reinterpret_cast<unsigned long long*>(p.ws.grid_bar + 32), ok, p.wait_ns,
                  p.dev_status);
   if (!ok) return;
 
@@ -1972,7 +1979,11 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
   if (cudaError_t e = configure_smem_once(indexer_decode_kernel, smem, configured, 100);
       e != cudaSuccess)
     return e;
-  const int grid_max = num_sms < kDxMaxCtas ? num_sms : kDxMaxCtas;
+  // no more CTAs than the largest number of key quads the call can have (a short context
+  // then pays its grid barriers across a few CTAs, not across every SM)
+  const int64_t quads_max = (int64_t)a.B * ((a.Nmax + kDxQuad * kIxTile - 1) / (kDxQuad * kIxTile));
+  int grid_max = num_sms < kDxMaxCtas ? num_sms : kDxMaxCtas;
+  if (quads_max < grid_max) grid_max = quads_max > 0 ? (int)quads_max : 1;
   cudaError_t e = cudaSuccess;
   if (!(a.flags & CSA_TOPK_SEPARATE_SELECT)) {
     // Scoring and selection in one cooperative launch (every CTA resident, so the grid

@@ -1,0 +1,88 @@
+// Tensor-pipe throughput of back-to-back tcgen05 MMAs on operands resident in shared memory
+// (no DRAM traffic): kind::mxf4 (E2M1 with E8M0 block scales) and kind::f16 with BF16
+// inputs, M = 128. It gives the measured ratio of the FP4 and BF16 tensor rates at one MMA
+// shape, which scales the pool's measured BF16 GEMM peak into the FP4 peak that the prefill
+// roofline divides its FP4 FLOPs by. Shapes: mxf4 with N = 64 (the indexer's MMA), BF16 with
+// N = 64 or 256 (the attention's MMAs).
+#include "common.cuh"
+
+namespace csa {
+
+struct alignas(1024) PkSmem {
+  uint8_t a[128 * 64];  // A: 128 rows x 64 bytes, 64-byte swizzle
+  uint8_t b[256 * 64];  // B: up to 256 rows x 64 bytes
+  uint8_t sf[2][512];   // scale atoms for A and B (E8M0 code 127 = 1.0)
+  uint64_t done;
+  uint32_t tmem_base;
+};
+
+// one CTA per SM: thread 0 issues `iters` dependent MMAs into one accumulator
+template <int KIND, int N>  // KIND 0: mxf4, 1: BF16
+__global__ void __launch_bounds__(128, 1) mma_peak_kernel(int iters, int32_t* dev_status) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  PkSmem& s = *reinterpret_cast<PkSmem*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const int tid = threadIdx.x;
+  // finite operands: E2M1 1.0 in every nibble (0x22), or BF16 1.0 (0x3F80)
+  const uint32_t fill = KIND == 0 ? 0x22222222u : 0x3F803F80u;
+  for (int i = tid; i < (int)(sizeof(s.a) / 4); i += 128) reinterpret_cast<uint32_t*>(s.a)[i] = fill;
+  for (int i = tid; i < (int)(sizeof(s.b) / 4); i += 128) reinterpret_cast<uint32_t*>(s.b)[i] = fill;
+  for (int i = tid; i < (int)(sizeof(s.sf) / 4); i += 128)
+    reinterpret_cast<uint32_t*>(&s.sf[0][0])[i] = 0x7F7F7F7Fu;
+  if (tid == 0) {
+    mbar_init(&s.done, 1);
+    mbar_fence_init();
+  }
+  if (tid < 32) tmem_alloc(&s.tmem_base, 512);
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  if (tid == 0) {
+    const uint64_t ad = smem_desc(smem_u32(s.a), 16, 512, kSwizzle64B);
+    const uint64_t bd = smem_desc(smem_u32(s.b), 16, 512, kSwizzle64B);
+    if (KIND == 0) {
+      // the indexer's scale placement: A's atoms at column 384, B's 8 columns on
+      const uint32_t t_sfa = tmem + 384, t_sfb = t_sfa + 8;
+      tmem_cp_32x128b_x4(t_sfa, smem_desc(smem_u32(s.sf[0]), 0, 128, kSwizzleNone));
+      tmem_cp_32x128b_x4(t_sfb, smem_desc(smem_u32(s.sf[1]), 0, 128, kSwizzleNone));
+      const uint32_t id = idesc_mxf4(128, N, 0);
+      for (int i = 0; i < iters; ++i) mma_mxf4(tmem, ad, bd, id, t_sfa, t_sfb, i > 0);
+    } else {
+      const uint32_t id = idesc_bf16(128, N, false);
+      for (int i = 0; i < iters; ++i) mma_f16(tmem, ad, bd, id, i > 0);
+    }
+    mma_commit(&s.done);
+    mbar_wait(&s.done, 0, dev_status);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (tid < 32) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// K per MMA: 64 E2M1 elements or 16 BF16 elements
+double mma_peak_flops_per_cta(int kind, int N, int iters) {
+  return 2.0 * 128.0 * N * (kind == 0 ? 64.0 : 16.0) * iters;
+}
+
+cudaError_t launch_mma_peak(int kind, int N, int iters, int num_sms, int32_t* dev_status,
+                            cudaStream_t stream) {
+  // more shared memory than half an SM holds, so that every CTA has an SM of its own
+  const size_t smem = 120 * 1024;
+  auto run = [&](auto kernel) -> cudaError_t {
+    static std::atomic<uint64_t> configured{0};
+    if (cudaError_t e = configure_smem_once(kernel, smem, configured); e != cudaSuccess) return e;
+    kernel<<<num_sms, 128, smem, stream>>>(iters, dev_status);
+    return cudaGetLastError();
+  };
+  if (kind == 0 && N == 64) return run(mma_peak_kernel<0, 64>);
+  if (kind == 1 && N == 64) return run(mma_peak_kernel<1, 64>);
+  if (kind == 1 && N == 256) return run(mma_peak_kernel<1, 256>);
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace csa

@@ -91,7 +91,8 @@ def test_every_entry_point_has_a_signature_of_the_declared_arity():
     if not os.path.exists(csa.LIB_PATH):
         pytest.skip("library not built")
     L = csa.lib()
-    results = {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "const char*": ctypes.c_char_p}
+    results = {"int": ctypes.c_int, "size_t": ctypes.c_size_t, "const char*": ctypes.c_char_p,
+               "double": ctypes.c_double}
     assert decls
     for ret, name, params in decls:
         ret = re.sub(r"\s*\*", "*", " ".join(ret.split()))
