@@ -69,19 +69,26 @@ double mma_peak_flops_per_cta(int kind, int N, int iters) {
   return 2.0 * 128.0 * N * (kind == 0 ? 64.0 : 16.0) * iters;
 }
 
+// more shared memory than half an SM holds, so that every CTA has an SM of its own
+constexpr size_t kPkSmem = 120 * 1024;
+
+template <int KIND, int N>
+cudaError_t launch_mma_peak_one(int iters, int num_sms, int32_t* dev_status,
+                                cudaStream_t stream) {
+  static std::atomic<uint64_t> configured{0};  // one flag per instantiation
+  if (cudaError_t e = configure_smem_once(mma_peak_kernel<KIND, N>, kPkSmem, configured);
+      e != cudaSuccess)
+    return e;
+  mma_peak_kernel<KIND, N><<<num_sms, 128, kPkSmem, stream>>>(iters, dev_status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mma_peak(int kind, int N, int iters, int num_sms, int32_t* dev_status,
                             cudaStream_t stream) {
-  // more shared memory than half an SM holds, so that every CTA has an SM of its own
-  const size_t smem = 120 * 1024;
-  auto run = [&](auto kernel) -> cudaError_t {
-    static std::atomic<uint64_t> configured{0};
-    if (cudaError_t e = configure_smem_once(kernel, smem, configured); e != cudaSuccess) return e;
-    kernel<<<num_sms, 128, smem, stream>>>(iters, dev_status);
-    return cudaGetLastError();
-  };
-  if (kind == 0 && N == 64) return run(mma_peak_kernel<0, 64>);
-  if (kind == 1 && N == 64) return run(mma_peak_kernel<1, 64>);
-  if (kind == 1 && N == 256) return run(mma_peak_kernel<1, 256>);
+  if (kind == 0 && N == 64) return launch_mma_peak_one<0, 64>(iters, num_sms, dev_status, stream);
+  if (kind == 1 && N == 64) return launch_mma_peak_one<1, 64>(iters, num_sms, dev_status, stream);
+  if (kind == 1 && N == 256)
+    return launch_mma_peak_one<1, 256>(iters, num_sms, dev_status, stream);
   return cudaErrorInvalidValue;
 }
 
