@@ -299,6 +299,7 @@ __global__ void __launch_bounds__(kDxThreads, 1)
     if (lane == 0) {
       int b = b0, qq = 0;
       const int groups = (int)(p.Nmax / kIxTile);
+      const uint64_t stream_policy = l2_evict_first_policy();  // keys are read once
       for (int q = q0; q < q1; ++q, ++qq) {
         while (s.qprefix[b + 1] <= q) ++b;
         const int t0 = kDxQuad * (q - s.qprefix[b]);
@@ -312,9 +313,9 @@ __global__ void __launch_bounds__(kDxThreads, 1)
           // tiles past n_b are read but not scored) and the scale groups that exist
           const uint32_t sf_bytes = (uint32_t)min(kDxQuad, groups - t0) * kIxSfBytes;
           mbar_arrive_expect_tx(&s.full[st], kDxQuad * kIxKeyBytes + sf_bytes);
-          tma_load_4d(&s.keys[st][0][0], &kmap, &s.full[st], 0, 0, t0, b);
-          bulk_load(&s.ksf[st][0][0], p.k_sf + ((size_t)b * groups + t0) * kIxSfBytes,
-                    sf_bytes, &s.full[st]);
+          tma_load_4d_hint(&s.keys[st][0][0], &kmap, &s.full[st], 0, 0, t0, b, stream_policy);
+          bulk_load_hint(&s.ksf[st][0][0], p.k_sf + ((size_t)b * groups + t0) * kIxSfBytes,
+                         sf_bytes, &s.full[st], stream_policy);
         } else {
           // paged keys: copies of tpl tiles from the page of each (a page holds whole
           // copies); tiles past n_b that lie in another page are not read (their slots
@@ -332,10 +333,10 @@ __global__ void __launch_bounds__(kDxThreads, 1)
               el = 0;
             }
             const int64_t g = el / kIxTile;  // the copy's first key group in the pool
-            tma_load_4d(&s.keys[st][l * p.tpl][0], &kmap, &s.full[st], 0, 0,
-                        (int)(g % tiles_pp), (int)(g / tiles_pp));
-            bulk_load(&s.ksf[st][l * p.tpl][0], p.k_sf + (size_t)g * kIxSfBytes,
-                      (uint32_t)p.tpl * kIxSfBytes, &s.full[st]);
+            tma_load_4d_hint(&s.keys[st][l * p.tpl][0], &kmap, &s.full[st], 0, 0,
+                             (int)(g % tiles_pp), (int)(g / tiles_pp), stream_policy);
+            bulk_load_hint(&s.ksf[st][l * p.tpl][0], p.k_sf + (size_t)g * kIxSfBytes,
+                           (uint32_t)p.tpl * kIxSfBytes, &s.full[st], stream_policy);
           }
         }
       }
