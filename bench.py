@@ -943,7 +943,8 @@ def main():
         idx_bytes, step_bytes = algorithmic_bytes(d)
         pk = peaks()
         achieved = idx_bytes / (t_idx * 1e-3) / 1e9
-        traffic = ncu_traffic()
+        # the committed capture is of the 1M workload's indexer call; other workloads have none
+        traffic = ncu_traffic() if w.name == "csa_decode_pro_1m" else None
         line = {
             "metric": metric, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": steps_run, "warmup": args.warmup, "ms_per_step": ms_step,
