@@ -275,10 +275,11 @@ int csa_indexer_query(const csa_iquery_args* args, csa_stream_t stream);
  * for (the parts kept at zero sit at offsets that do not depend on B). Calls that share a
  * workspace must not overlap on the device.
  *
- * Scoring and selection normally run in one cooperative launch with one CTA per SM and
- * two grid-wide barriers; if the runtime refuses that launch (for instance when other
- * work holds SMs), scoring runs as an ordinary launch followed by two selection kernels,
- * with the same results. `flags` = CSA_TOPK_SEPARATE_SELECT takes that second path on
+ * Scoring and selection normally run in one cooperative launch with at most one CTA per
+ * SM (and no more CTAs than the call has 512-entry key quads) and two grid-wide barriers;
+ * if the runtime refuses that launch (for instance when other work holds SMs), scoring
+ * runs as an ordinary launch followed by two selection kernels, with the same results.
+ * The key stream is loaded with an L2 evict-first policy: it is read once per call. `flags` = CSA_TOPK_SEPARATE_SELECT takes that second path on
  * purpose (for testing it). `select_wait_ns` bounds each wait at the grid barriers of the
  * cooperative path (0 = 2 s); a wait that runs out writes CSA_ERR_TIMEOUT to dev_status
  * and the call returns with its outputs undefined.
