@@ -1970,7 +1970,7 @@ cudaError_t launch_indexer_topk(const csa_topk_args& a, void* workspace, int num
   ix_ws_layout(a.B, a.Nmax, a.k, (char*)workspace, &ws);
   const uint64_t wait_ns = a.select_wait_ns > 0 ? (uint64_t)a.select_wait_ns : kWaitLimitNs;
   IxParams p{a.B, a.H_I, a.k, 1, bf16, wait_ns, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w,
-             a.k_sf, ws, a.idx, a.scores, a.dev_status};
+             a.k_sf, ws, a.idx, a.scores, a.dev_status, PageMap{}, kDxQuad};
   p.pm = page_map(a.pages, a.Nmax);
   p.tpl = a.pages.block_table ? (a.pages.page_entries / kIxTile < kDxQuad
                                      ? a.pages.page_entries / kIxTile : kDxQuad)
@@ -2025,7 +2025,7 @@ cudaError_t launch_prefill_indexer_topk(const csa_topk_args& a, void* workspace,
   IxWs ws;
   ix_ws_layout(a.B, a.Nmax, a.k, (char*)workspace, &ws);
   IxParams p{a.B, a.H_I, a.k, 0, 0, kWaitLimitNs, a.Nmax, a.n_entries, a.q_fp4, a.q_sf, a.w,
-             a.k_sf, ws, a.idx, a.scores, a.dev_status};
+             a.k_sf, ws, a.idx, a.scores, a.dev_status, PageMap{}, kDxQuad};  // keys contiguous
   const size_t smem = sizeof(PxSmem) + 1024;
   static std::atomic<uint64_t> configured{0};
   if (cudaError_t e = configure_smem_once(prefill_score_kernel, smem, configured);
