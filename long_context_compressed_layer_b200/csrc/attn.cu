@@ -6,7 +6,9 @@
 //
 // The rows a query attends to form one list: the selected entries (CSA) or all eligible
 // entries (HCA), then the 128 window tokens t-127 .. t. The list is cut into chunks of
-// 64 rows. attn_chunk_kernel handles one (sequence, chunk):
+// 64 rows. attn_chunk_kernel handles one (sequence, chunk), or one (sequence, chunk, half
+// of the output dims) when twice the chunks still fit one wave of CTAs on the SMs (then a
+// chunk's two CTAs compute the same S and softmax):
 //   - Q [H heads x 512] arrives by TMA (128-byte swizzle, K-major), padded to 128 rows,
 //     and is widened in place from BF16 to FP16 (exact for |q| >= 2^-14);
 //   - the 64 rows are gathered and dequantised to FP16 in shared memory (E4M3 code x entry
@@ -15,7 +17,8 @@
 //     than BF16 (8) keeps the staging error well inside the output tolerance;
 //   - tcgen05.mma kind::f16 computes S[128 x 64] in TMEM; one thread per head turns its row
 //     into exp(tau*S - m) (fp32), keeps m and l = sum, and writes P as FP16 (K-major A);
-//   - two tcgen05.mma N = 256 halves compute O[128 x 512] in TMEM (S's columns are reused);
+//   - tcgen05.mma N = 256 products compute this CTA's halves of O[128 x 512] in TMEM (S's
+//     columns are reused);
 //   - O / l (FP16, [8-dim group][head][8] so every warp store covers 512 contiguous bytes),
 //     m and l go to the workspace.
 // attn_combine_kernel then merges the chunks of a sequence in fixed order with the sink,
@@ -58,6 +61,7 @@ struct AtParams {
   __half* part_o;  // [B][C][64][H][8]: chunk output / chunk sum, fp16, 8-dim groups
   float2* part_ml; // [B][C][H]: (chunk max logit, chunk sum)
   float* rot;      // [B][64]: cos, sin of -t theta_j per RoPE pair (chunk 0 writes them)
+  int split;       // CTAs per chunk: 2 (each half of the output dims) or 1
   PageMap pm;         // where the entries live (contiguous or paged)
   int32_t* dev_status;
 };
@@ -120,6 +124,41 @@ __device__ __forceinline__ int at_rows_total(const AtParams& p, int n) {
 }
 
 
+// O / l of this CTA's NBLK column blocks of 32 (per warp: lane quadrant quad, blocks
+// colh * NBLK ..), FP16, heads innermost; the next block loads from TMEM while the current
+// one is stored
+template <int NBLK>
+__device__ __forceinline__ void store_partial(const AtParams& p, const AtSmem& s, uint32_t t_o,
+                                              int b, int c, int dh, int quad, int colh,
+                                              int tid) {
+  const int hh = quad * 32 + (tid & 31);
+  const float inv = s.inv_l[hh];
+  const uint32_t ta0 = t_o + ((uint32_t)(quad * 32) << 16) + colh * NBLK * 32;
+  uint32_t r[2][32];
+  tmem_ld32(ta0, r[0]);
+  tmem_ld_wait();
+#pragma unroll
+  for (int i = 0; i < NBLK; ++i) {
+    if (i + 1 < NBLK) tmem_ld32(ta0 + (i + 1) * 32, r[(i + 1) & 1]);
+    if (hh < p.H) {
+      const uint32_t* x = r[i & 1];
+      const int g0 = (dh * 8 + colh * NBLK + i) * 4;  // first 8-dim group of this block
+#pragma unroll
+      for (int e = 0; e < 32; e += 8) {
+        uint4 v;
+        v.x = pack_half2(__uint_as_float(x[e]) * inv, __uint_as_float(x[e + 1]) * inv);
+        v.y = pack_half2(__uint_as_float(x[e + 2]) * inv, __uint_as_float(x[e + 3]) * inv);
+        v.z = pack_half2(__uint_as_float(x[e + 4]) * inv, __uint_as_float(x[e + 5]) * inv);
+        v.w = pack_half2(__uint_as_float(x[e + 6]) * inv, __uint_as_float(x[e + 7]) * inv);
+        // heads innermost: the warp's 32 heads store 512 contiguous bytes
+        *reinterpret_cast<uint4*>(
+            p.part_o + ((((size_t)b * p.C + c) * 64 + g0 + e / 8) * p.H + hh) * 8) = v;
+      }
+    }
+    tmem_ld_wait();
+  }
+}
+
 // The staged row of entry r is v'_r = [codes (448 dims, exact in FP16) | rope dims / scale_r]
 // with scale_r its entry scale, and a window row is itself with scale 1. Then
 //   q . v_r = scale_r (q . v'_r)   and   sum_r p_r v_r = sum_r (p_r scale_r) v'_r,
@@ -131,7 +170,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   AtSmem& s = *reinterpret_cast<AtSmem*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  const int c = blockIdx.x, b = blockIdx.y, tid = threadIdx.x;
+  // split = 2: CTA (2c + dh, b) is chunk c of sequence b for output dims [256 dh, +256) (S
+  // and the softmax are computed by both CTAs of a chunk, with the same bits); split = 1:
+  // CTA (c, b) computes all 512
+  const int c = blockIdx.x / p.split, dh = p.split == 2 ? (int)(blockIdx.x & 1) : 0;
+  const int b = blockIdx.y, tid = threadIdx.x;
   const int warp = tid >> 5;
   const int row0 = c * kAtRows;
   pdl_wait();
@@ -271,7 +314,7 @@ __global__ void __launch_bounds__(kAtThreads, 1)
     mma_commit(&s.s_done);
   }
   // chunk 0's warp 1: the de-rotation table of the sequence, while S is computed
-  if (c == 0 && warp == 1 && p.derotate) {
+  if (c == 0 && dh == 0 && warp == 1 && p.derotate) {
     float cs, sn;
     rope_cos_sin((double)t, tid & 31, (double)p.rope_base, &cs, &sn);
     *reinterpret_cast<float2*>(p.rot + (size_t)b * 64 + 2 * (tid & 31)) = make_float2(cs, sn);
@@ -329,22 +372,25 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   if (tid < 128) {  // head tid: the chunk's max and sum (the halves summed in a fixed order)
     const float l_c = s.sm[0][tid] + s.sm[1][tid];
     s.inv_l[tid] = l_c > 0.f ? 1.f / l_c : 0.f;
-    if (tid < p.H) {
+    if (tid < p.H && dh == 0) {
       const size_t slot = ((size_t)b * p.C + c) * p.H + tid;
       p.part_ml[slot] = ok ? make_float2(fmaxf(s.mx[0][tid], s.mx[1][tid]), l_c)
                            : make_float2(-INFINITY, 0.f);
     }
   }
 
-  // O = P' V' : M = 128, N = 256 per half, K = 64 rows (4 steps of 16); V' read MN-major
+  // O[:, 256 half .. +256] = P' V'[:, 256 half ..] for this CTA's halves: M = 128, N = 256,
+  // K = 64 rows (4 steps of 16); V' read MN-major
+  const int nh = 3 - p.split;  // halves of the output this CTA computes
   if (tid == 0) {
     if (ok) {
       tc_fence_after();
       const uint32_t id = idesc_f16(128, 256, true);
-      for (int half = 0; half < 2; ++half) {
+      for (int hf = 0; hf < nh; ++hf) {
         for (int kk = 0; kk < 4; ++kk) {
-          mma_f16(t_o + half * 256, smem_desc(smem_u32(s.pm) + kk * 32, 16, 1024, kSwizzle128B),
-                  smem_desc(smem_u32(s.v[half * 4]) + kk * 2048, kAtRows * 128, 1024, kSwizzle128B),
+          mma_f16(t_o + hf * 256, smem_desc(smem_u32(s.pm) + kk * 32, 16, 1024, kSwizzle128B),
+                  smem_desc(smem_u32(s.v[(dh + hf) * 4]) + kk * 2048, kAtRows * 128, 1024,
+                            kSwizzle128B),
                   id, kk > 0);
         }
       }
@@ -355,36 +401,11 @@ __global__ void __launch_bounds__(kAtThreads, 1)
   __syncthreads();  // inv_l written by threads 0-127 above
   tc_fence_after();
   {
-    // warp w reads lanes of quadrant w % 4, columns [256 * (w / 4), +256): 8 blocks of 32,
-    // two TMEM loads per wait
-    // the next 32 columns load from TMEM while the current ones are stored
-    const int colh = warp >> 2;
-    const int hh = quad * 32 + (tid & 31);
-    const float inv = s.inv_l[hh];
-    const uint32_t ta0 = t_o + ((uint32_t)(quad * 32) << 16) + colh * 8 * 32;
-    uint32_t r[2][32];
-    tmem_ld32(ta0, r[0]);
-    tmem_ld_wait();
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (i + 1 < 8) tmem_ld32(ta0 + (i + 1) * 32, r[(i + 1) & 1]);
-      if (hh < p.H) {
-        const uint32_t* x = r[i & 1];
-        const int g0 = (colh * 8 + i) * 4;  // first 8-dim group of this 32-dim block
-#pragma unroll
-        for (int e = 0; e < 32; e += 8) {
-          uint4 v;
-          v.x = pack_half2(__uint_as_float(x[e]) * inv, __uint_as_float(x[e + 1]) * inv);
-          v.y = pack_half2(__uint_as_float(x[e + 2]) * inv, __uint_as_float(x[e + 3]) * inv);
-          v.z = pack_half2(__uint_as_float(x[e + 4]) * inv, __uint_as_float(x[e + 5]) * inv);
-          v.w = pack_half2(__uint_as_float(x[e + 6]) * inv, __uint_as_float(x[e + 7]) * inv);
-          // heads innermost: the warp's 32 heads store 512 contiguous bytes
-          *reinterpret_cast<uint4*>(
-              p.part_o + ((((size_t)b * p.C + c) * 64 + g0 + e / 8) * p.H + hh) * 8) = v;
-        }
-      }
-      tmem_ld_wait();
-    }
+    // warp w reads lanes of quadrant w % 4 and the second or first half of this CTA's columns
+    if (nh == 2)
+      store_partial<8>(p, s, t_o, b, c, dh, quad, warp >> 2, tid);
+    else
+      store_partial<4>(p, s, t_o, b, c, dh, quad, warp >> 2, tid);
   }
   tc_fence_before();
   __syncthreads();
@@ -929,7 +950,13 @@ cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* 
   if (cudaError_t e = configure_smem_once(attn_chunk_kernel, smem, configured);
       e != cudaSuccess)
     return e;
-  cudaError_t e = launch_pdl(attn_chunk_kernel, dim3(p.C, a.B), dim3(kAtThreads), smem, stream,
+  // two CTAs per chunk (one per half of the output dims) when that still fits one wave
+  int sms = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    sms = 0;
+  p.split = (int64_t)2 * p.C * a.B <= sms ? 2 : 1;
+  cudaError_t e = launch_pdl(attn_chunk_kernel, dim3(p.split * p.C, a.B), dim3(kAtThreads), smem, stream,
                              qmap, p);
   if (e != cudaSuccess) return e;
   return launch_pdl(attn_combine_kernel, dim3(64, a.B), dim3(128), 0, stream, p);

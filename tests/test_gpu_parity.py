@@ -509,6 +509,23 @@ def test_batch_invariance_and_determinism():
         np.testing.assert_array_equal(out_b[0], out_all[b])
 
 
+def test_attention_bits_do_not_depend_on_the_output_split():
+    # a chunk's output is computed by one CTA (all 512 dims) when the batch's chunks fill
+    # the SMs, and by two (one per half) when twice the chunks still fit one wave; 8
+    # sequences of 18 chunks take the first path, each of them alone the second
+    d = _attn_case(8, 128, 2048, [2048, 1900, 1700, 1500, 1300, 1100, 900, 700],
+                   [9000, 8000, 7000, 6000, 5000, 4500, 3700, 2900], 1024, seed=23)
+    full = csa.sparse_attn_decode(dev(d["q"]), dev(d["pos"]), dev(d["n"]), dev(d["kv"]),
+                                  dev(d["sc"]), dev(d["swa"]), dev(d["sink"]), dev(d["idx"]))
+    full = full.view(torch.int16).cpu().numpy()
+    for b in range(8):
+        sl = slice(b, b + 1)
+        one = csa.sparse_attn_decode(dev(d["q"][sl]), dev(d["pos"][sl]), dev(d["n"][sl]),
+                                     dev(d["kv"][sl]), dev(d["sc"][sl]), dev(d["swa"][sl]),
+                                     dev(d["sink"]), dev(d["idx"][sl]))
+        np.testing.assert_array_equal(one.view(torch.int16).cpu().numpy()[0], full[b])
+
+
 # --------------------------------------------------- full decode, small workloads
 def test_workload0_decode_chain():
     """Compress the 8192-token stream, score/select, attend: each stage vs the oracle fed
