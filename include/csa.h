@@ -401,7 +401,9 @@ int hca_attn_decode(const csa_attn_args* args, void* workspace, size_t workspace
  * tile even when no block is complete), H in {64, 128}, H_I in {16, 32, 64},
  * 1 <= k <= 2048.
  * The workspace (csa_prefill_workspace_size) must be zero-filled once before its first
- * use; every call leaves the parts that must start at zero zeroed again.
+ * use; every call leaves the parts that must start at zero zeroed again. It includes a
+ * staging area of Nmax x 648 bytes that a call on a paged cache (csa_pages) fills with
+ * the prefix's rows and all keys before it runs, and copies the new rows back from.
  */
 typedef struct {
   int64_t P;                  /* prefix tokens, a multiple of m */
@@ -438,6 +440,7 @@ typedef struct {
   float* lse;                 /* optional */
   int32_t* idx;               /* optional: the selected sets */
   int32_t* dev_status;        /* optional device word */
+  csa_pages pages;            /* kv, kv_scale, k_fp4, k_sf paged (table [1][pages_max]) */
 } csa_prefill_args;
 
 size_t csa_prefill_workspace_size(int32_t T, int64_t Nmax, int32_t H, int32_t k);

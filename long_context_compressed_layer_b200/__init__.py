@@ -125,7 +125,7 @@ class PrefillArgs(C.Structure):
                 ("norm_w", _vp), ("prev_b", _vp), ("prev_zb", _vp), ("kv", _vp),
                 ("kv_scale", _vp), ("q_fp4", _vp), ("q_sf", _vp), ("w", _vp), ("k_fp4", _vp),
                 ("k_sf", _vp), ("q", _vp), ("sink", _vp), ("swa_prefix", _vp), ("out", _vp),
-                ("lse", _vp), ("idx", _vp), ("dev_status", _vp)]
+                ("lse", _vp), ("idx", _vp), ("dev_status", _vp), ("pages", Pages)]
 
 
 EXPORTS = ["csa_status_string", "csa_compress", "csa_compress_index_keys", "csa_decode_append",
@@ -536,20 +536,25 @@ def prefill(P: int, m: int, k: int, *, a, b, za, zb, bias, kv, kv_scale, q_fp4, 
             k_fp4, k_sf, q, sink, prev_b=None, prev_zb=None, swa_prefix=None, norm_w=None,
             tau: float = 0.0, rope_base: float = 10000.0, eps: float = 1e-6,
             derotate: bool = True, strict_eligibility: bool = False, workspace=None,
-            out=None, lse: bool = False, idx: bool = False, dev_status=None, stream=None):
+            out=None, lse: bool = False, idx: bool = False, dev_status=None,
+            paging: Paging | None = None, stream=None):
     """Causal CSA prefill of the T new tokens after a P-token prefix (one sequence).
     kv / kv_scale [Nmax] are updated in place with the new entries. Returns out
     [T][H][512] bf16 and, when asked, lse [T][H] and the selected sets idx [T][k].
     strict_eligibility: a query at t sees only blocks completed before t (floor(t/m)
-    entries) instead of also the block closing at t (floor((t+1)/m))."""
+    entries) instead of also the block closing at t (floor((t+1)/m)).
+    With paging (a one-row block table), kv, kv_scale, k_fp4 and k_sf are page pools."""
     T = a.shape[0]
     H, H_I = q.shape[1], q_fp4.shape[1]
-    Nmax = kv.shape[0]
+    if paging is None:
+        Nmax = pool = kv.shape[0]
+    else:
+        Nmax, pool = paging.Nmax, kv.numel() // ROW_BYTES
     tok = T * HEAD_DIM
     _sizes(a=(a, tok), b=(b, tok), za=(za, tok), zb=(zb, tok), bias=(bias, 2 * m),
-           kv=(kv, Nmax * ROW_BYTES), kv_scale=(kv_scale, Nmax), q_fp4=(q_fp4, T * H_I * 64),
-           q_sf=(q_sf, T * H_I * 4), w=(w, T * H_I), k_fp4=(k_fp4, Nmax * 64),
-           k_sf=(k_sf, Nmax // 128 * 512), q=(q, T * H * HEAD_DIM), sink=(sink, H),
+           kv=(kv, pool * ROW_BYTES), kv_scale=(kv_scale, pool), q_fp4=(q_fp4, T * H_I * 64),
+           q_sf=(q_sf, T * H_I * 4), w=(w, T * H_I), k_fp4=(k_fp4, pool * 64),
+           k_sf=(k_sf, pool // 128 * 512), q=(q, T * H * HEAD_DIM), sink=(sink, H),
            prev_b=(prev_b, m * HEAD_DIM), prev_zb=(prev_zb, m * HEAD_DIM),
            swa_prefix=(swa_prefix, WINDOW * HEAD_DIM), norm_w=(norm_w, HEAD_DIM),
            out=(out, T * H * HEAD_DIM))
@@ -575,7 +580,7 @@ def prefill(P: int, m: int, k: int, *, a, b, za, zb, bias, kv, kv_scale, q_fp4, 
                        _ptr(swa_prefix, elem=2, name="swa_prefix"),
                        _ptr(out, elem=2, name="out"), _ptr(l, elem=4, name="lse"),
                        _ptr(ix, elem=4, name="idx"),
-                       _ptr(dev_status, elem=4, name="dev_status"))
+                       _ptr(dev_status, elem=4, name="dev_status"), _pages(paging, pool, 1))
     _check(lib().csa_prefill(C.byref(args), workspace.data_ptr(), workspace.numel(),
                              _stream(stream)), "csa_prefill")
     res = [out]

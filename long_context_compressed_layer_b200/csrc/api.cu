@@ -29,6 +29,13 @@ cudaError_t launch_prefill_prep(const csa_prefill_args& a, __half* lin, int32_t*
                                 int32_t* pos_all, cudaStream_t stream);
 cudaError_t launch_attn(const csa_attn_args& a, int sparse, int rows_max, void* workspace,
                         const CUtensorMap& qmap, cudaStream_t stream);
+cudaError_t launch_page_gather(const PageMap& pm, const uint8_t* kv, const float* kv_scale,
+                               const uint8_t* k_fp4, const uint8_t* k_sf, uint8_t* kv_c,
+                               float* sc_c, uint8_t* kf_c, uint8_t* ksf_c, int64_t n_kv,
+                               int64_t n_keys, int32_t* dev_status, cudaStream_t stream);
+cudaError_t launch_page_scatter(const PageMap& pm, const uint8_t* kv_c, const float* sc_c,
+                                uint8_t* kv, float* kv_scale, int64_t j0, int64_t j1,
+                                int32_t* dev_status, cudaStream_t stream);
 double mma_peak_flops_per_cta(int kind, int N, int iters);
 cudaError_t launch_mma_peak(int kind, int N, int iters, int num_sms, int32_t* dev_status,
                             cudaStream_t stream);
@@ -133,6 +140,12 @@ struct PrefillWs {
   int32_t* pos_all;   // [T]
   __half* rows16;     // FP16 rows: [Nmax] entries, then [T + 127] window rows in position order
   int32_t* idx;       // [chunk][k] selected sets when the caller passes none
+  // contiguous staging of a paged cache: rows [Nmax][576], scales [Nmax], keys [Nmax][64],
+  // key scales [Nmax/128][512]
+  uint8_t* kv_c;
+  float* sc_c;
+  uint8_t* kf_c;
+  uint8_t* ksf_c;
 };
 
 size_t prefill_ws_layout(int T, int64_t Nmax, int H, int k, char* base, PrefillWs* w) {
@@ -148,8 +161,16 @@ size_t prefill_ws_layout(int T, int64_t Nmax, int H, int k, char* base, PrefillW
   char* pos_all = take((size_t)T * 4);
   char* rows16 = take(((size_t)Nmax + T + CSA_WINDOW - 1) * CSA_HEAD_DIM * 2);
   char* idx = take((size_t)qc * k * 4);
+  char* kv_c = take((size_t)Nmax * CSA_ROW_BYTES);
+  char* sc_c = take((size_t)Nmax * 4);
+  char* kf_c = take((size_t)Nmax * 64);
+  char* ksf_c = take((size_t)Nmax / 128 * 512);
   (void)H;
   if (w) {
+    w->kv_c = reinterpret_cast<uint8_t*>(kv_c);
+    w->sc_c = reinterpret_cast<float*>(sc_c);
+    w->kf_c = reinterpret_cast<uint8_t*>(kf_c);
+    w->ksf_c = reinterpret_cast<uint8_t*>(ksf_c);
     w->ix = ix;
     w->n_all = reinterpret_cast<int32_t*>(n_all);
     w->pos_all = reinterpret_cast<int32_t*>(pos_all);
@@ -470,7 +491,8 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
       !ok_ptr(a->kv) || !ok_ptr(a->kv_scale) || !ok_ptr(a->q_fp4) || !ok_ptr(a->q_sf) ||
       !ok_ptr(a->w) || !ok_ptr(a->k_fp4) || !ok_ptr(a->k_sf) || !ok_ptr(a->q) ||
       !ok_ptr(a->sink) || !ok_ptr(a->out) || !ok_opt(a->norm_w) || !ok_opt(a->lse) ||
-      !ok_opt(a->idx) || (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)))
+      !ok_opt(a->idx) || (a->dev_status && (reinterpret_cast<uintptr_t>(a->dev_status) & 3)) ||
+      !ok_pages(a->pages, a->Nmax))
     return CSA_ERR_INVALID_ARG;
   if (a->P > 0 && (!ok_ptr(a->prev_b) || !ok_ptr(a->prev_zb) || !ok_ptr(a->swa_prefix)))
     return CSA_ERR_INVALID_ARG;
@@ -483,8 +505,21 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
   cudaStream_t stream = reinterpret_cast<cudaStream_t>(stream_);
   PrefillWs w;
   prefill_ws_layout(a->T, a->Nmax, a->H, a->k, reinterpret_cast<char*>(ws), &w);
+  // a paged cache: the call runs on a contiguous staging copy (the prefix's rows, every
+  // key), and the new entries go back to their pages at the end
+  const bool paged = a->pages.block_table != nullptr;
+  const PageMap pm = page_map(a->pages, a->Nmax);
+  uint8_t* kv = paged ? w.kv_c : a->kv;
+  float* kv_scale = paged ? w.sc_c : a->kv_scale;
+  const uint8_t* k_fp4 = paged ? w.kf_c : a->k_fp4;
+  const uint8_t* k_sf = paged ? w.ksf_c : a->k_sf;
   CUtensorMap kmap;  // encoded before the first launch, so a refusal leaves no partial work
-  if (!encode_key_map(enc, &kmap, a->k_fp4, a->Nmax, 1)) return CSA_ERR_CUDA;
+  if (!encode_key_map(enc, &kmap, k_fp4, a->Nmax, 1)) return CSA_ERR_CUDA;
+  if (paged &&
+      launch_page_gather(pm, a->kv, a->kv_scale, a->k_fp4, a->k_sf, w.kv_c, w.sc_c, w.kf_c,
+                         w.ksf_c, a->P / a->m, (a->P + a->T) / a->m, a->dev_status,
+                         stream) != cudaSuccess)
+    return CSA_ERR_CUDA;
 
   // 1. the new blocks' entries
   csa_compress_args c;
@@ -504,8 +539,8 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
   c.norm_w = a->norm_w;
   c.prev_b = a->prev_b;
   c.prev_zb = a->prev_zb;
-  c.kv = a->kv;
-  c.kv_scale = a->kv_scale;
+  c.kv = kv;
+  c.kv_scale = kv_scale;
   c.Nmax = a->Nmax;
   cudaError_t e = launch_compress(c, stream);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
@@ -514,7 +549,7 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
   e = launch_prefill_prep(*a, w.rows16 + (size_t)a->Nmax * CSA_HEAD_DIM, w.n_all, w.pos_all,
                           stream);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
-  e = launch_prefill_rows16(a->kv, a->kv_scale, (a->P + a->T) / a->m, w.rows16, stream);
+  e = launch_prefill_rows16(kv, kv_scale, (a->P + a->T) / a->m, w.rows16, stream);
   if (e != cudaSuccess) return CSA_ERR_CUDA;
   // 3. per chunk of queries: indexer top-k over the shared keys, then attention
   for (int c0 = 0; c0 < a->T; c0 += kPrefillChunk) {
@@ -530,8 +565,8 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
     t.q_fp4 = a->q_fp4 + (size_t)c0 * a->H_I * 64;
     t.q_sf = a->q_sf + (size_t)c0 * a->H_I * 4;
     t.w = a->w + (size_t)c0 * a->H_I;
-    t.k_fp4 = a->k_fp4;
-    t.k_sf = a->k_sf;
+    t.k_fp4 = k_fp4;
+    t.k_sf = k_sf;
     t.idx = idx;
     t.dev_status = a->dev_status;
     e = launch_prefill_indexer_topk(t, w.ix, sms, kmap, stream);
@@ -546,8 +581,8 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
     at.pos = w.pos_all + c0;
     at.idx = idx;
     at.n_entries = w.n_all + c0;
-    at.kv = a->kv;
-    at.kv_scale = a->kv_scale;
+    at.kv = kv;
+    at.kv_scale = kv_scale;
     at.swa = nullptr;
     at.sink = a->sink;
     at.tau = a->tau;
@@ -561,6 +596,10 @@ int csa_prefill(const csa_prefill_args* a, void* ws, size_t ws_bytes, csa_stream
     e = launch_prefill_attn(at, w.rows16, a->P - (CSA_WINDOW - 1), qmap, stream);
     if (e != cudaSuccess) return CSA_ERR_CUDA;
   }
+  if (paged &&
+      launch_page_scatter(pm, w.kv_c, w.sc_c, a->kv, a->kv_scale, a->P / a->m,
+                          (a->P + a->T) / a->m, a->dev_status, stream) != cudaSuccess)
+    return CSA_ERR_CUDA;
   return CSA_OK;
 }
 

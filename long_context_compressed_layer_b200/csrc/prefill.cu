@@ -110,3 +110,84 @@ cudaError_t launch_prefill_prep(const csa_prefill_args& a, __half* lin, int32_t*
 }
 
 }  // namespace csa
+
+namespace csa {
+
+// Paged prefill (csa_pages in csa_prefill_args): the call runs on a contiguous staging copy
+// of the sequence's cache. page_gather_kernel copies entries 0 .. n_kv-1 (rows and scales)
+// and the keys of entries 0 .. n_keys-1 (rows, and the scale group of every 128 entries)
+// from their pages; page_scatter_kernel copies the rows and scales of entries
+// j0 .. j1-1 (the ones the call compressed) back to their pages. One warp per entry.
+__global__ void __launch_bounds__(256) page_gather_kernel(PageMap pm, const uint8_t* kv,
+                                                          const float* kv_scale,
+                                                          const uint8_t* k_fp4,
+                                                          const uint8_t* k_sf, uint8_t* kv_c,
+                                                          float* sc_c, uint8_t* kf_c,
+                                                          uint8_t* ksf_c, int64_t n_kv,
+                                                          int64_t n_keys, int32_t* dev_status) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t j = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (j >= n_kv && j >= n_keys) return;
+  const int64_t e = page_entry(pm, 0, j);
+  if (e < 0) {
+    if (lane == 0) report(dev_status, CSA_ERR_DEVICE);
+    return;
+  }
+  if (j < n_kv) {
+    const uint4* src = reinterpret_cast<const uint4*>(kv + (size_t)e * kRow);
+    uint4* dst = reinterpret_cast<uint4*>(kv_c + (size_t)j * kRow);
+    for (int u = lane; u < kRow / 16; u += 32) dst[u] = src[u];
+    if (lane == 0) sc_c[j] = kv_scale[e];
+  }
+  if (j < n_keys) {
+    if (lane < 4)
+      reinterpret_cast<uint4*>(kf_c + (size_t)j * 64)[lane] =
+          reinterpret_cast<const uint4*>(k_fp4 + (size_t)e * 64)[lane];
+    if ((j & 127) == 0)  // the group's 512 scale bytes (a page holds whole groups)
+      reinterpret_cast<uint4*>(ksf_c + (size_t)(j / 128) * 512)[lane] =
+          reinterpret_cast<const uint4*>(k_sf + (size_t)(e / 128) * 512)[lane];
+  }
+}
+
+__global__ void __launch_bounds__(256) page_scatter_kernel(PageMap pm, const uint8_t* kv_c,
+                                                           const float* sc_c, uint8_t* kv,
+                                                           float* kv_scale, int64_t j0,
+                                                           int64_t j1, int32_t* dev_status) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t j = j0 + (((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5);
+  const int lane = threadIdx.x & 31;
+  if (j >= j1) return;
+  const int64_t e = page_entry(pm, 0, j);
+  if (e < 0) {
+    if (lane == 0) report(dev_status, CSA_ERR_DEVICE);
+    return;
+  }
+  const uint4* src = reinterpret_cast<const uint4*>(kv_c + (size_t)j * kRow);
+  uint4* dst = reinterpret_cast<uint4*>(kv + (size_t)e * kRow);
+  for (int u = lane; u < kRow / 16; u += 32) dst[u] = src[u];
+  if (lane == 0) kv_scale[e] = sc_c[j];
+}
+
+cudaError_t launch_page_gather(const PageMap& pm, const uint8_t* kv, const float* kv_scale,
+                               const uint8_t* k_fp4, const uint8_t* k_sf, uint8_t* kv_c,
+                               float* sc_c, uint8_t* kf_c, uint8_t* ksf_c, int64_t n_kv,
+                               int64_t n_keys, int32_t* dev_status, cudaStream_t stream) {
+  const int64_t n = n_kv > n_keys ? n_kv : n_keys;
+  if (n <= 0) return cudaSuccess;
+  return launch_pdl(page_gather_kernel, dim3((unsigned)((n + 7) / 8)), dim3(256), 0, stream, pm,
+                    kv, kv_scale, k_fp4, k_sf, kv_c, sc_c, kf_c, ksf_c, n_kv, n_keys,
+                    dev_status);
+}
+
+cudaError_t launch_page_scatter(const PageMap& pm, const uint8_t* kv_c, const float* sc_c,
+                                uint8_t* kv, float* kv_scale, int64_t j0, int64_t j1,
+                                int32_t* dev_status, cudaStream_t stream) {
+  if (j1 <= j0) return cudaSuccess;
+  return launch_pdl(page_scatter_kernel, dim3((unsigned)((j1 - j0 + 7) / 8)), dim3(256), 0,
+                    stream, pm, kv_c, sc_c, kv, kv_scale, j0, j1, dev_status);
+}
+
+}  // namespace csa

@@ -204,3 +204,40 @@ def test_prefill_full_size_sampled_rows():
                kv_scale=host(d["kv_scale"]))
     check_cache(inp, got, ora)
     check_rows(inp, w.k, got, rows, ora)
+
+
+@pytest.mark.parametrize("P,T,page_entries", [(512, 300, 128), (2048, 700, 256)])
+def test_prefill_on_a_paged_cache_equals_contiguous(P, T, page_entries):
+    # the cache and keys behind a shuffled block table: the same outputs, selected sets and
+    # lse bits as the contiguous call, the prefix rows untouched in their pages and the new
+    # rows written to the pages the table names
+    inp = synth.prefill_inputs(P, T, 4, 64, 16, seed=P + T)
+    flat = run_prefill(inp, 64)
+    Nmax = inp["kv"].shape[0]
+    rng = np.random.default_rng(page_entries)
+    table, num_pages = synth.page_table(rng, 1, Nmax // page_entries)
+    kvp = synth.place_in_pages(inp["kv"][None], table, page_entries, num_pages)
+    scp = synth.place_in_pages(inp["kv_scale"][None], table, page_entries, num_pages)
+    kfp = synth.place_in_pages(inp["k_fp4"][None], table, page_entries, num_pages)
+    ksp = synth.place_in_pages(inp["k_sf"].reshape(1, Nmax // 128, 512), table, page_entries,
+                               num_pages, group=128)
+    kv_d, sc_d = dev(kvp), dev(scp)
+    opt = {x: dev(inp[x]) for x in ("prev_b", "prev_zb") if x in inp}
+    opt["swa_prefix"] = dev(inp["swa_prefix"])
+    st = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse, idx = csa.prefill(
+        P, 4, 64, a=dev(inp["a"]), b=dev(inp["b"]), za=dev(inp["za"]), zb=dev(inp["zb"]),
+        bias=dev(inp["bias"]), kv=kv_d, kv_scale=sc_d, q_fp4=dev(inp["q_fp4"]),
+        q_sf=dev(inp["q_sf"]), w=dev(inp["w"]), k_fp4=dev(kfp), k_sf=dev(ksp), q=dev(inp["q"]),
+        sink=dev(inp["sink"]), lse=True, idx=True, dev_status=st,
+        paging=csa.Paging(dev(table), page_entries, Nmax), **opt)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    np.testing.assert_array_equal(out.float().cpu().numpy(), flat["out"])
+    np.testing.assert_array_equal(host(lse), flat["lse"])
+    np.testing.assert_array_equal(host(idx), flat["idx"])
+    n1 = (P + T) // 4
+    view_kv = oracle.paged_view(host(kv_d), table, page_entries)[0]
+    view_sc = oracle.paged_view(host(sc_d), table, page_entries)[0]
+    np.testing.assert_array_equal(view_kv[:n1], flat["kv"][:n1])
+    np.testing.assert_array_equal(view_sc[:n1], flat["kv_scale"][:n1])
