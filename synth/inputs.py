@@ -74,13 +74,25 @@ _E4M3_EXP_P = np.array([1, 1, 1, 1, 1, 2, 2, 3, 4, 6, 9, 13, 17, 19, 14, 6], dty
 _E4M3_EXP_P /= _E4M3_EXP_P.sum()
 
 
+# Elementwise work on large draws runs over slices of this many elements, so that the
+# temporaries stay cache-sized; the random draws themselves are taken whole, in a fixed
+# order, so the values do not depend on the slicing.
+_CHUNK = 1 << 22
+
+
 def e4m3_codes(rng: np.random.Generator, shape) -> np.ndarray:
     n = int(np.prod(shape))
     e = _lut_sample(rng, n, _E4M3_EXP_P)
     low = rng.integers(0, 16, size=n, dtype=np.uint8)  # 3 mantissa bits + sign bit
-    mant, sign = low & 7, low >> 3
-    mant = np.where((e == 15) & (mant == 7), np.uint8(6), mant)
-    return ((sign << 7) | (e << 3) | mant).astype(np.uint8).reshape(shape)
+    out = np.empty(n, dtype=np.uint8)
+    for c in range(0, n, _CHUNK):
+        ec, lc, oc = e[c:c + _CHUNK], low[c:c + _CHUNK], out[c:c + _CHUNK]
+        mant = lc & 7
+        mant[(ec == 15) & (mant == 7)] = 6
+        np.left_shift(lc >> 3, 7, out=oc)
+        oc |= ec << 3
+        oc |= mant
+    return out.reshape(shape)
 
 
 # E2M1 magnitude codes 0..7 (values 0, .5, 1, 1.5, 2, 3, 4, 6) drawn with the
@@ -93,7 +105,11 @@ def _lut_sample(rng: np.random.Generator, n: int, p: np.ndarray) -> np.ndarray:
     edges = np.cumsum(p) / p.sum()
     u = (np.arange(65536, dtype=np.float64) + 0.5) / 65536.0
     lut = np.searchsorted(edges, u, side="right").clip(0, len(p) - 1).astype(np.uint8)
-    return lut[rng.integers(0, 65536, size=n, dtype=np.uint16)]
+    idx = rng.integers(0, 65536, size=n, dtype=np.uint16)
+    out = np.empty(n, dtype=np.uint8)
+    for c in range(0, n, _CHUNK):
+        np.take(lut, idx[c:c + _CHUNK], out=out[c:c + _CHUNK])
+    return out
 
 
 def e2m1_nibbles(rng: np.random.Generator, shape, sign_bias: np.ndarray | None = None,

@@ -8,6 +8,7 @@ Each mutant is (name, text in csa_oracle.cpp, replacement, which occurrence). Al
 change the oracle's arithmetic or layout; none of them touches the tests.
 """
 
+import json
 import os
 import shutil
 import subprocess
@@ -307,9 +308,9 @@ def _apply(src, old, new, which):
     return old.join(parts[:which + 1]) + new + old.join(parts[which + 1:])
 
 
-def _run(base, name, text):
-    """Copy the pins and the oracle under base/name with the given oracle source, build
-    it and run the pins; returns (name, build ok, pins passed, last line of output)."""
+def _prepare(base, name, text):
+    """Copy the pins and the oracle under base/name with the given oracle source and build
+    it; returns (name, directory, build ok, compiler message)."""
     d = os.path.join(base, name)
     shutil.copytree(os.path.join(ROOT, "synth"), os.path.join(d, "synth"),
                     ignore=shutil.ignore_patterns("__pycache__"))
@@ -324,14 +325,52 @@ def _run(base, name, text):
     so = os.path.join(d, "oracle", "liboracle.so")
     b = subprocess.run(["g++", "-O2", "-std=c++17", "-shared", "-fPIC", "-pthread", "-o", so,
                         cpp], capture_output=True, text=True)
-    if b.returncode:
-        return name, False, False, b.stderr[-300:]
-    tests = sorted(os.path.join("tests", f) for f in os.listdir(os.path.join(d, "tests"))
-                   if f.startswith("test_oracle_"))
-    r = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "not gpu", *tests],
-                       cwd=d, capture_output=True, text=True, timeout=600)
-    out = r.stdout.strip().splitlines()
-    return name, True, r.returncode == 0, out[-1] if out else r.stderr[-300:]
+    return name, d, b.returncode == 0, b.stderr[-300:]
+
+
+# A small fork server: it imports the heavy third-party modules once, then forks one child
+# per copy; the child moves into its copy (so that `oracle`, `synth` and `tests` resolve
+# there, none of them being imported before the fork), runs the pin files with pytest -x and
+# exits with pytest's status. It prints one JSON object {directory: status}.
+_SERVER = r"""
+import json, os, sys
+import numpy, torch, pytest
+dirs, workers = json.loads(sys.argv[1]), int(sys.argv[2])
+status, running, todo = {}, {}, list(dirs)
+while todo or running:
+    while todo and len(running) < workers:
+        d = todo.pop(0)
+        pid = os.fork()
+        if pid == 0:
+            try:
+                os.chdir(d)
+                fd = os.open(os.path.join(d, "pins.log"), os.O_WRONLY | os.O_CREAT, 0o644)
+                os.dup2(fd, 1)
+                os.dup2(fd, 2)
+                sys.path.insert(0, d)
+                tests = sorted(os.path.join("tests", f) for f in os.listdir("tests")
+                               if f.startswith("test_oracle_"))
+                rc = pytest.main(["-x", "-q", "-m", "not gpu", "-p", "no:cacheprovider",
+                                  *tests])
+                sys.stdout.flush()
+                sys.stderr.flush()
+                os._exit(int(rc))
+            except BaseException:
+                os._exit(99)
+        running[pid] = d
+    pid, st = os.wait()
+    status[running.pop(pid)] = os.waitstatus_to_exitcode(st)
+print(json.dumps(status))
+"""
+
+
+def _last_line(d):
+    try:
+        with open(os.path.join(d, "pins.log")) as f:
+            lines = f.read().strip().splitlines()
+        return lines[-1] if lines else ""
+    except OSError:
+        return "no log"
 
 
 @pytest.mark.slow
@@ -341,12 +380,23 @@ def test_every_planted_mistake_fails_a_pin(tmp_path):
     with open(os.path.join(ROOT, "oracle", "csa_oracle.cpp")) as f:
         src = f.read()
     jobs = [("unmutated", src)] + [(n, _apply(src, o, r, w)) for n, o, r, w in MUTANTS]
-    workers = max(1, min(8, (os.cpu_count() or 2) // 2))
-    with ThreadPoolExecutor(workers) as ex:
-        res = list(ex.map(lambda j: _run(str(tmp_path), *j), jobs))
+    cpus = os.cpu_count() or 2
+    with ThreadPoolExecutor(max(1, min(8, cpus))) as ex:
+        built = list(ex.map(lambda j: _prepare(str(tmp_path), *j), jobs))
+    unbuilt = [(n, msg) for n, _, ok, msg in built if not ok]
+    assert not unbuilt, f"copies that do not compile: {unbuilt}"
+    dirs = [d for _, d, _, _ in built]
+    r = subprocess.run([sys.executable, "-c", _SERVER, json.dumps(dirs),
+                        str(max(1, min(8, cpus)))],
+                       cwd=str(tmp_path), capture_output=True, text=True, timeout=1200)
+    assert r.returncode == 0, r.stderr[-600:]
+    status = json.loads(r.stdout.strip().splitlines()[-1])
+    res = [(n, status[d], _last_line(d)) for (n, d, _, _) in built]
     control = res[0]
-    assert control[1] and control[2], f"the unmutated oracle fails its pins: {control[3]}"
-    unbuilt = [(n, msg) for n, ok, _, msg in res[1:] if not ok]
-    assert not unbuilt, f"mutants that do not compile: {unbuilt}"
-    survivors = [(n, msg) for n, _, passed, msg in res[1:] if passed]
+    assert control[1] == 0, f"the unmutated oracle fails its pins: {control[2]}"
+    # 1: a pin failed; negative: the pins crashed the copy on a signal. Any other status
+    # (interrupted, internal or usage error, nothing collected) is a broken harness.
+    broken = [(n, rc, msg) for n, rc, msg in res[1:] if rc > 1]
+    assert not broken, f"pin runs that ended without a verdict: {broken}"
+    survivors = [(n, msg) for n, rc, msg in res[1:] if rc == 0]
     assert not survivors, f"planted mistakes no pin catches: {survivors}"

@@ -17,6 +17,21 @@ def test_e4m3_codes_never_nan_and_sit_near_the_top_of_the_range():
     assert np.mean(exp >= 10) > 0.7  # the exponent field is drawn near its top
 
 
+def test_sliced_generation_equals_one_pass_over_the_draws(monkeypatch):
+    """The E4M3 and table-sampled codes do not depend on the slice length: a length that
+    leaves a ragged last slice gives the same codes as one slice over the whole draw."""
+    shape = (3, 1000, 448)
+    monkeypatch.setattr(synth, "_CHUNK", 1 << 30)
+    whole = synth.e4m3_codes(np.random.default_rng(7), shape)
+    nib_whole = synth.e2m1_nibbles(np.random.default_rng(8), (5, 70001))
+    monkeypatch.setattr(synth, "_CHUNK", 100003)
+    np.testing.assert_array_equal(synth.e4m3_codes(np.random.default_rng(7), shape), whole)
+    np.testing.assert_array_equal(synth.e2m1_nibbles(np.random.default_rng(8), (5, 70001)),
+                                  nib_whole)
+    # the codes are the sign, exponent and mantissa fields of the draws, S.1111.111 excluded
+    assert whole.dtype == np.uint8 and not ((whole & 0x7F) == 0x7F).any()
+
+
 def test_e2m1_magnitudes_follow_the_table_and_signs_are_balanced():
     rng = np.random.default_rng(1)
     nib = synth.e2m1_nibbles(rng, (400000,))
