@@ -38,6 +38,29 @@ def sources_sha(files: list[str] | None = None) -> str:
     return h.hexdigest()[:16]
 
 
+def compile_objects(srcs: list[str], outdir: str, verbose: bool = False) -> tuple[list[str], str]:
+    """Compile each source to an object in outdir with the library's flags, all at once on
+    the host's cores (a faster check of every translation unit than build()); returns
+    the objects and the compilers' combined output (ptxas's resource report with verbose).
+    Raises CalledProcessError, carrying that output, if any source fails."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    def one(src):
+        obj = os.path.join(outdir, os.path.basename(src) + ".o")
+        cmd = [nvcc(), *ARCH, "-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC",
+               "-Xptxas", "-v" if verbose else "-O3", "-c", "-o", obj, src]
+        r = subprocess.run(cmd, capture_output=True, text=True)
+        return obj, r.returncode, cmd, r.stdout + r.stderr
+
+    with ThreadPoolExecutor(max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
+        res = list(ex.map(one, srcs))
+    log = "".join(r[3] for r in res)
+    for _, rc, cmd, out in res:
+        if rc:
+            raise subprocess.CalledProcessError(rc, cmd, output=log, stderr=out)
+    return [r[0] for r in res], log
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     srcs = sources()
     deps = srcs + glob.glob(os.path.join(HERE, "csrc", "*.cuh")) + [
