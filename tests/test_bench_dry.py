@@ -33,13 +33,49 @@ bench.main()
 """
 
 
-def _line(argv, small_prefill=False):
-    code = RUN.format(root=ROOT, argv=argv, small_prefill=small_prefill)
-    r = subprocess.run([sys.executable, "-c", code], cwd=ROOT, capture_output=True, text=True,
-                       timeout=600)
-    assert r.returncode == 0, r.stderr[-3000:]
-    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
-    assert len(lines) == 1, r.stdout[-2000:]
+# Every mode's run, by key: (bench.py arguments, whether the prefill workload is shrunk).
+RUNS = {
+    "default": (["--steps", "20", "--warmup", "3"], False),
+    "flash": (["--workload", "flash", "--steps", "16", "--warmup", "3"], False),
+    "tiny": (["--workload", "tiny", "--steps", "16", "--warmup", "3"], False),
+    "hca": (["--workload", "hca", "--steps", "20", "--warmup", "3"], False),
+    "prefill": (["--workload", "prefill", "--steps", "2", "--warmup", "3"], True),
+    "reference": (["--impl", "reference", "--steps", "1", "--warmup", "0"], False),
+}
+TEST_RUNS = {"test_default_decode_line": "default", "test_hca_line": "hca",
+             "test_prefill_line": "prefill", "test_reference_line": "reference"}
+
+
+def _key(item):
+    if item.originalname == "test_other_decode_lines":
+        return item.callspec.params["mode"]
+    return TEST_RUNS.get(item.originalname)
+
+
+@pytest.fixture(scope="module")
+def runs(request):
+    """Start the runs of every selected test of this module at once (each is a separate
+    process of about 2 GB); a test then waits for its own. Runs still going when the module
+    ends (a test failed first under -x) are ended by their process ids."""
+    keys = {_key(it) for it in request.session.items if it.module is request.module}
+    procs = {}
+    for k in sorted(x for x in keys if x):
+        argv, small = RUNS[k]
+        code = RUN.format(root=ROOT, argv=argv, small_prefill=small)
+        procs[k] = subprocess.Popen([sys.executable, "-c", code], cwd=ROOT, text=True,
+                                    stdout=subprocess.PIPE, stderr=subprocess.PIPE)
+    yield procs
+    for pr in procs.values():
+        if pr.poll() is None:
+            pr.kill()
+            pr.communicate()
+
+
+def _line(runs, key):
+    out, err = runs[key].communicate(timeout=600)
+    assert runs[key].returncode == 0, err[-3000:]
+    lines = [ln for ln in out.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, out[-2000:]
     return json.loads(lines[0])
 
 
@@ -63,8 +99,8 @@ def _contract(d, cpu_baseline=True):
 
 
 @pytest.mark.slow
-def test_default_decode_line():
-    d = _line(["--steps", "20", "--warmup", "3"])
+def test_default_decode_line(runs):
+    d = _line(runs, "default")
     _contract(d)
     assert d["steps"] == 20
     assert d["config"]["workload"] == "csa_decode_pro_1m" and d["roofline"]["bound"] == "hbm"
@@ -73,28 +109,28 @@ def test_default_decode_line():
 
 @pytest.mark.parametrize("mode,workload", [("flash", "csa_decode_flash_128k"),
                                            ("tiny", "csa_decode_8k_tiny")])
-def test_other_decode_lines(mode, workload):
-    d = _line(["--workload", mode, "--steps", "16", "--warmup", "3"])
+def test_other_decode_lines(runs, mode, workload):
+    d = _line(runs, mode)
     _contract(d)
     assert d["config"]["workload"] == workload and d["steps"] == 16
     assert d["roofline"]["bound"] == "hbm"
 
 
-def test_hca_line():
-    d = _line(["--workload", "hca", "--steps", "20", "--warmup", "3"])
+def test_hca_line(runs):
+    d = _line(runs, "hca")
     _contract(d)
     assert d["config"]["workload"] == "hca_decode_128k"
     assert d["steps"] == 20  # graphs of 4 steps: exactly the steps asked for
 
 
-def test_prefill_line():
-    d = _line(["--workload", "prefill", "--steps", "2", "--warmup", "3"], small_prefill=True)
+def test_prefill_line(runs):
+    d = _line(runs, "prefill")
     _contract(d)
     assert d["roofline"]["bound"] == "tensor"
 
 
-def test_reference_line():
-    d = _line(["--impl", "reference", "--steps", "1", "--warmup", "0"])
+def test_reference_line(runs):
+    d = _line(runs, "reference")
     assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
