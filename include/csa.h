@@ -131,6 +131,8 @@ typedef struct {
   float* dbg;            /* optional out [B][N][512]: fp32 y before quantisation */
 } csa_compress_args;
 
+/* Unlike the other compute calls, csa_compress takes no workspace: each block's merge,
+ * norm, rotation and quantisation stay on chip, so it needs no scratch memory. */
 int csa_compress(const csa_compress_args* args, csa_stream_t stream);
 
 /* ------------------------------------------------------------------------------------
@@ -265,8 +267,10 @@ int csa_indexer_query(const csa_iquery_args* args, csa_stream_t stream);
  * element 2i in the low nibble of byte i. q_sf [B][H_I][4] holds the 4 block scales of
  * each query head. k_sf is grouped by 128 entries: [B][Nmax/128][512] bytes, and the
  * scale of entry j (j = 128g + 32r1 + r0), block s, sits at byte 16*r0 + 4*r1 + s of
- * group g -- the tensor-core scale-factor atom, so a group is copied as is.
- * Nmax must be a multiple of 128. 1 <= k <= 2048, H_I in {16, 32, 64}.
+ * group g -- the tensor-core scale-factor atom, so a group is copied as is. This is not
+ * the plain per-entry order [B][Nmax][4]: the keys' writers (csa_compress_index_keys,
+ * csa_decode_append) store the atom order once, so no call has to repack the scales of
+ * every entry it reads. Nmax must be a multiple of 128. 1 <= k <= 2048, H_I in {16, 32, 64}.
  * The workspace must be zero-filled once before its first use; every call that ends with
  * dev_status still zero leaves it zeroed again. After a call that reported
  * CSA_ERR_TIMEOUT or CSA_ERR_DEVICE (or any call whose dev_status was not read), zero-fill
