@@ -4,8 +4,9 @@ wrong tie rule, a swapped nibble or slot order) and check that the CPU pin suite
 (tests/test_oracle_*.py) fails on every one of them. The unmutated copy must pass in the
 same harness, so a broken harness cannot pass the check by failing everything.
 
-Each mutant is (name, text in csa_oracle.cpp, replacement, which occurrence). All of them
-change the oracle's arithmetic or layout; none of them touches the tests.
+Each mutant is (name, text in the oracle's source, replacement, which occurrence): MUTANTS
+for csa_oracle.cpp, PY_MUTANTS for the Python layer. All of them change the oracle's
+arithmetic or layout; none of them touches the tests.
 """
 
 import json
@@ -302,22 +303,46 @@ MUTANTS = [
 ]
 
 
+# Mistakes planted in the oracle's Python layer (oracle/__init__.py): the paged-cache view
+# and scatter, whose arithmetic is written there rather than in the C++ file.
+PY_MUTANTS = [
+    ("pv_table_ignored",
+     "out[b, lp * per_page:(lp + 1) * per_page] = pool[page]",
+     "out[b, lp * per_page:(lp + 1) * per_page] = pool[lp % pool.shape[0]]", 0),
+    ("pv_negative_page_read",
+     "if 0 <= page < pool.shape[0]:",
+     "if page < pool.shape[0]:", 0),
+    ("pv_group_offset",
+     "out[b, lp * per_page:(lp + 1) * per_page] = pool[page]",
+     "out[b, lp * (page_entries // 128):(lp + 1) * (page_entries // 128)] = pool[page]", 0),
+    ("ps_wrong_sequence",
+     "pool[page, :hi - lo] = view[b, lo:hi]",
+     "pool[page, :hi - lo] = view[(b + 1) % B, lo:hi]", 0),
+    ("ps_table_transposed",
+     "page = int(table[b, lp])",
+     "page = int(table[lp % B, b % pages_max])", 1),
+    ("ps_slot_shift",
+     "pool[page, :hi - lo] = view[b, lo:hi]",
+     "pool[page, :hi - lo] = np.roll(view[b, lo:hi], 1, axis=0)", 0),
+]
+
 def _apply(src, old, new, which):
     parts = src.split(old)
     assert len(parts) >= which + 2, f"pattern not in the oracle: {old[:60]!r}"
     return old.join(parts[:which + 1]) + new + old.join(parts[which + 1:])
 
 
-def _prepare(base, name, text):
-    """Copy the pins and the oracle under base/name with the given oracle source and build
-    it; returns (name, directory, build ok, compiler message)."""
+def _prepare(base, name, text, py_text):
+    """Copy the pins and the oracle under base/name with the given oracle sources (C++ and
+    the Python layer) and build it; returns (name, directory, build ok, compiler message)."""
     d = os.path.join(base, name)
     shutil.copytree(os.path.join(ROOT, "synth"), os.path.join(d, "synth"),
                     ignore=shutil.ignore_patterns("__pycache__"))
     shutil.copytree(os.path.join(ROOT, "tests"), os.path.join(d, "tests"),
                     ignore=shutil.ignore_patterns("__pycache__", "c", "test_[!o]*"))
     os.makedirs(os.path.join(d, "oracle"))
-    shutil.copy(os.path.join(ROOT, "oracle", "__init__.py"), os.path.join(d, "oracle"))
+    with open(os.path.join(d, "oracle", "__init__.py"), "w") as f:
+        f.write(py_text)
     shutil.copy(os.path.join(ROOT, "pytest.ini"), d)
     cpp = os.path.join(d, "oracle", "csa_oracle.cpp")
     with open(cpp, "w") as f:
@@ -379,7 +404,11 @@ def test_every_planted_mistake_fails_a_pin(tmp_path):
         pytest.skip("no g++")
     with open(os.path.join(ROOT, "oracle", "csa_oracle.cpp")) as f:
         src = f.read()
-    jobs = [("unmutated", src)] + [(n, _apply(src, o, r, w)) for n, o, r, w in MUTANTS]
+    with open(os.path.join(ROOT, "oracle", "__init__.py")) as f:
+        py = f.read()
+    jobs = ([("unmutated", src, py)] +
+            [(n, _apply(src, o, r, w), py) for n, o, r, w in MUTANTS] +
+            [(n, src, _apply(py, o, r, w)) for n, o, r, w in PY_MUTANTS])
     cpus = os.cpu_count() or 2
     with ThreadPoolExecutor(max(1, min(8, cpus))) as ex:
         built = list(ex.map(lambda j: _prepare(str(tmp_path), *j), jobs))
