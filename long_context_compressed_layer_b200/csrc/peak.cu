@@ -1,7 +1,7 @@
 // Tensor-pipe throughput of back-to-back tcgen05 MMAs on operands resident in shared memory
 // (no DRAM traffic): kind::mxf4 (E2M1 with E8M0 block scales) and kind::f16 with BF16
 // inputs, M = 128. It gives the measured ratio of the FP4 and BF16 tensor rates at one MMA
-// shape, which scales the pool's measured BF16 GEMM peak into the FP4 peak that the prefill
+// shape, which scales a measured BF16 GEMM peak (cuBLAS) into the FP4 peak that the prefill
 // roofline divides its FP4 FLOPs by. Shapes: mxf4 with N = 64 (the indexer's MMA), BF16 with
 // N = 64 or 256 (the attention's MMAs).
 #include "common.cuh"
