@@ -72,6 +72,9 @@ double or_bf16_decode(uint16_t h) {
   return s ? -v : v;
 }
 
+// bfloat16 encoding [chooseai 一: the RoPE dims are stored in BF16]: round to 8
+// significand bits, nearest with ties to even (the IEEE-754 default), overflow to
+// infinity, NaN to the quiet NaN 0x7FC0 (the NaN payload is a reading).
 uint16_t or_bf16_encode(double x) {
   if (std::isnan(x)) return 0x7FC0;
   const uint16_t s = std::signbit(x) ? 0x8000 : 0;
@@ -99,8 +102,8 @@ double or_e4m3_decode(uint8_t c) {
   return s ? -v : v;
 }
 
-// Round-to-nearest-even, saturating to +-448 (a reading: the cache never stores NaN for
-// finite inputs).
+// E4M3 encoding [chooseai 一: the 448 non-RoPE dims are stored in FP8]: round to nearest
+// even, saturating to +-448 (a reading: the cache never stores NaN for finite inputs).
 uint8_t or_e4m3_encode(double x) {
   if (std::isnan(x)) return 0x7F;
   const uint8_t s = std::signbit(x) ? 0x80 : 0;
@@ -163,8 +166,10 @@ void or_mxfp4_block(const double* v, uint8_t* nib, uint8_t* sf) {
 }
 
 // Byte offset of the E8M0 scale of entry j, 32-element block s, in the indexer-key
-// scale array. Keys are grouped 128 to a 512-byte group; inside a group entry
-// j = r0 + 32*r1 (r0 < 32, r1 < 4) keeps its four block scales at 16*r0 + 4*r1 + s.
+// scale array [walkthrough §3.4: the indexer keys are MXFP4, one E8M0 scale per 32
+// elements; where the scales sit is a reading]. Keys are grouped 128 to a 512-byte group;
+// inside a group entry j = r0 + 32*r1 (r0 < 32, r1 < 4) keeps its four block scales at
+// 16*r0 + 4*r1 + s.
 size_t or_key_sf_offset(int64_t j, int s) {
   const int64_t g = j / 128, r = j % 128;
   return (size_t)(g * 512 + 16 * (r % 32) + 4 * (r / 32) + s);
@@ -408,7 +413,9 @@ int or_grouped_out_proj(int T, int H, int G, int d_g, int d_model, const uint16_
   return 0;
 }
 
-// Dequantise one stored entry (448 E4M3 codes times the entry scale, then 64 bf16).
+// Dequantise one stored entry [chooseai 一: 448 dims in FP8, the 64 RoPE dims in BF16;
+// one fp32 scale per entry is a reading]: 448 E4M3 codes times the entry scale, then the
+// 64 bf16 values.
 void or_dequant_row(const uint8_t* row, float scale, double* v) {
   for (int d = 0; d < kNope; ++d) v[d] = or_e4m3_decode(row[d]) * (double)scale;
   for (int d = kNope; d < kD; ++d) {
@@ -601,8 +608,9 @@ int or_attention(int B, int H, int k, int64_t Nmax, int sparse, const uint16_t* 
 }
 
 // ------------------------------------------------------------------ prefill
-// Sliding-window row of token t (a reading): the raw KV a[t] goes through the same RMSNorm
-// and the RoPE rotation at position t as an entry, and is stored as bf16.
+// Sliding-window row of token t [walkthrough §2.2: the last 128 tokens are attended to
+// uncompressed] (how the row is formed is a reading): the raw KV a[t] goes through the same
+// RMSNorm and the RoPE rotation at position t as an entry, and is stored as bf16.
 void or_swa_row(const uint16_t* a_row, int64_t t, double rope_base, double eps,
                 const float* norm_w, uint16_t* out_row) {
   std::vector<double> y(kD);
