@@ -165,3 +165,71 @@ def test_mxfp4_rule_accepts_the_oracle_and_catches_planted_deviations():
     three = codes.copy()
     three[:1, :1] = 3
     assert compare.check_mxfp4(three, two, sf.reshape(-1), sf.reshape(-1), mid) <= 1
+
+
+def test_a_boundary_gap_above_the_tie_tolerance_is_not_a_tie():
+    # the (k+1)-th score 1e-4 (relative) below the k-th: outside the 1e-6 tie window, so a
+    # set that takes it instead of the k-th is wrong
+    rng = np.random.default_rng(4)
+    n, k = 1000, 100
+    s = rng.standard_normal(n)
+    order = np.lexsort((np.arange(n), -s))
+    s[order[k]] = s[order[k - 1]] * (1 - 1e-4)
+    swapped = np.sort(np.r_[order[:k - 1], order[k]])
+    with pytest.raises(AssertionError, match="gap"):
+        compare.compare_topk(swapped, s, n, k)
+
+
+def test_inside_a_tie_every_chosen_entry_is_still_at_the_boundary():
+    # an exact tie between the k-th and (k+1)-th scores lets either be chosen, but not an
+    # entry far below them
+    rng = np.random.default_rng(5)
+    n, k = 1000, 100
+    s = rng.standard_normal(n)
+    order = np.lexsort((np.arange(n), -s))
+    s[order[k]] = s[order[k - 1]]
+    wrong = np.sort(np.r_[order[:k - 1], order[500]])
+    with pytest.raises(AssertionError, match="far below"):
+        compare.compare_topk(wrong, s, n, k)
+
+
+def test_a_flip_past_the_midpoint_window_is_rejected():
+    # the oracle's value 2e-3 of the row's RMS above a midpoint: well outside the 1e-5
+    # window, so the code below that midpoint is not a rounding of a nearby value
+    kv, sc, dbg, ora = _entries()
+    y = ora["y"].copy()
+    v = y[0, 1, :448] / float(sc[0, 1])
+    rms = float(np.sqrt(np.mean(v * v)))
+    lo = int(indep.f64_to_e4m3(np.array([rms]))[0]) & 0x7F
+    lo = lo - 1 if lo & 7 == 7 else lo
+    pair = indep.e4m3_to_f64(np.array([lo, lo + 1], dtype=np.uint8))
+    y[0, 1, 7] = ((pair[0] + pair[1]) / 2 + 2e-3 * rms) * float(sc[0, 1])
+    ref = kv.copy()
+    ref[0, 1, 7] = lo + 1  # the nearest code of the oracle's value
+    got = ref.copy()
+    got[0, 1, 7] = lo
+    with pytest.raises(AssertionError, match="E4M3"):
+        compare.check_codes(got, ref, y, sc)
+
+
+def test_bf16_topk_rejects_an_entry_several_steps_below_the_boundary():
+    # scores on the BF16 grid of [2, 4) (step 2^-6): the top 40 of 120 start at 3.25; an
+    # entry 3 grid steps below (0.047, above the rule's one step of 3.25 x 2^-7 = 0.025)
+    # may not replace the boundary entry
+    n, k = 120, 40
+    s = 2.0 + np.arange(n) * 2.0 ** -6
+    want = oracle.topk_bf16(s, n, k)
+    assert compare.compare_topk_bf16(want, s, n, k) == 0
+    wrong = np.sort(np.r_[np.setdiff1d(want, [80]), 77])
+    with pytest.raises(AssertionError, match="BF16 step"):
+        compare.compare_topk_bf16(wrong, s, n, k)
+
+
+def test_bf16_topk_checks_the_padding():
+    s = 1.0 + np.arange(10) * 0.25
+    want = oracle.topk_bf16(s, 10, 16)
+    assert compare.compare_topk_bf16(want, s, 10, 16) == 0
+    bad = want.copy()
+    bad[10:] = 0
+    with pytest.raises(AssertionError, match="padding"):
+        compare.compare_topk_bf16(bad, s, 10, 16)

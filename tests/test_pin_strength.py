@@ -9,14 +9,14 @@ for csa_oracle.cpp, PY_MUTANTS for the Python layer. All of them change the orac
 arithmetic or layout; none of them touches the tests.
 """
 
-import json
 import os
 import shutil
 import subprocess
-import sys
 from concurrent.futures import ThreadPoolExecutor
 
 import pytest
+
+from tests import mutation
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -326,11 +326,6 @@ PY_MUTANTS = [
      "pool[page, :hi - lo] = np.roll(view[b, lo:hi], 1, axis=0)", 0),
 ]
 
-def _apply(src, old, new, which):
-    parts = src.split(old)
-    assert len(parts) >= which + 2, f"pattern not in the oracle: {old[:60]!r}"
-    return old.join(parts[:which + 1]) + new + old.join(parts[which + 1:])
-
 
 def _prepare(base, name, text, py_text):
     """Copy the pins and the oracle under base/name with the given oracle sources (C++ and
@@ -353,51 +348,6 @@ def _prepare(base, name, text, py_text):
     return name, d, b.returncode == 0, b.stderr[-300:]
 
 
-# A small fork server: it imports the heavy third-party modules once, then forks one child
-# per copy; the child moves into its copy (so that `oracle`, `synth` and `tests` resolve
-# there, none of them being imported before the fork), runs the pin files with pytest -x and
-# exits with pytest's status. It prints one JSON object {directory: status}.
-_SERVER = r"""
-import json, os, sys
-import numpy, torch, pytest
-dirs, workers = json.loads(sys.argv[1]), int(sys.argv[2])
-status, running, todo = {}, {}, list(dirs)
-while todo or running:
-    while todo and len(running) < workers:
-        d = todo.pop(0)
-        pid = os.fork()
-        if pid == 0:
-            try:
-                os.chdir(d)
-                fd = os.open(os.path.join(d, "pins.log"), os.O_WRONLY | os.O_CREAT, 0o644)
-                os.dup2(fd, 1)
-                os.dup2(fd, 2)
-                sys.path.insert(0, d)
-                tests = sorted(os.path.join("tests", f) for f in os.listdir("tests")
-                               if f.startswith("test_oracle_"))
-                rc = pytest.main(["-x", "-q", "-m", "not gpu", "-p", "no:cacheprovider",
-                                  *tests])
-                sys.stdout.flush()
-                sys.stderr.flush()
-                os._exit(int(rc))
-            except BaseException:
-                os._exit(99)
-        running[pid] = d
-    pid, st = os.wait()
-    status[running.pop(pid)] = os.waitstatus_to_exitcode(st)
-print(json.dumps(status))
-"""
-
-
-def _last_line(d):
-    try:
-        with open(os.path.join(d, "pins.log")) as f:
-            lines = f.read().strip().splitlines()
-        return lines[-1] if lines else ""
-    except OSError:
-        return "no log"
-
-
 @pytest.mark.slow
 def test_every_planted_mistake_fails_a_pin(tmp_path):
     if not shutil.which("g++"):
@@ -407,25 +357,13 @@ def test_every_planted_mistake_fails_a_pin(tmp_path):
     with open(os.path.join(ROOT, "oracle", "__init__.py")) as f:
         py = f.read()
     jobs = ([("unmutated", src, py)] +
-            [(n, _apply(src, o, r, w), py) for n, o, r, w in MUTANTS] +
-            [(n, src, _apply(py, o, r, w)) for n, o, r, w in PY_MUTANTS])
-    cpus = os.cpu_count() or 2
-    with ThreadPoolExecutor(max(1, min(8, cpus))) as ex:
+            [(n, mutation.apply(src, o, r, w), py) for n, o, r, w in MUTANTS] +
+            [(n, src, mutation.apply(py, o, r, w)) for n, o, r, w in PY_MUTANTS])
+    workers = max(1, min(8, os.cpu_count() or 2))
+    with ThreadPoolExecutor(workers) as ex:
         built = list(ex.map(lambda j: _prepare(str(tmp_path), *j), jobs))
     unbuilt = [(n, msg) for n, _, ok, msg in built if not ok]
     assert not unbuilt, f"copies that do not compile: {unbuilt}"
-    dirs = [d for _, d, _, _ in built]
-    r = subprocess.run([sys.executable, "-c", _SERVER, json.dumps(dirs),
-                        str(max(1, min(8, cpus)))],
-                       cwd=str(tmp_path), capture_output=True, text=True, timeout=1200)
-    assert r.returncode == 0, r.stderr[-600:]
-    status = json.loads(r.stdout.strip().splitlines()[-1])
-    res = [(n, status[d], _last_line(d)) for (n, d, _, _) in built]
-    control = res[0]
-    assert control[1] == 0, f"the unmutated oracle fails its pins: {control[2]}"
-    # 1: a pin failed; negative: the pins crashed the copy on a signal. Any other status
-    # (interrupted, internal or usage error, nothing collected) is a broken harness.
-    broken = [(n, rc, msg) for n, rc, msg in res[1:] if rc > 1]
-    assert not broken, f"pin runs that ended without a verdict: {broken}"
-    survivors = [(n, msg) for n, rc, msg in res[1:] if rc == 0]
-    assert not survivors, f"planted mistakes no pin catches: {survivors}"
+    names, dirs = [b[0] for b in built], [b[1] for b in built]
+    status = mutation.run(dirs, ["test_oracle_"], str(tmp_path), workers)
+    mutation.verdict(names, dirs, status, "oracle")
