@@ -98,6 +98,22 @@ def _contract(d, cpu_baseline=True):
             assert key in d["cpu_baseline"], key
 
 
+def _arith(d, units_per_step, kernel_ms):
+    """The line's numbers agree with one another: the rate is the step's units over its
+    time, end to end too; the roofline's achieved rate is its work per launch over the
+    kernel's time, and its fractions are that rate over the stated peaks."""
+    approx = lambda x: pytest.approx(x, rel=1e-9)
+    assert d["value"] == approx(units_per_step * d["n_gpus"] / (d["ms_per_step"] * 1e-3))
+    assert d["e2e"]["value"] == approx(units_per_step * d["n_gpus"] /
+                                       (d["e2e"]["ms_per_step"] * 1e-3))
+    r = d["roofline"]
+    assert r["frac"] == approx(r["achieved"] / r["peak"])
+    assert r["frac_of_nominal"] == approx(r["achieved"] / r["nominal_peak"])
+    if r["bound"] == "hbm":
+        assert r["achieved"] == approx(r["algorithmic_bytes_per_launch"] / (kernel_ms * 1e-3)
+                                       / 1e9)
+
+
 @pytest.mark.slow
 def test_default_decode_line(runs):
     d = _line(runs, "default")
@@ -105,6 +121,10 @@ def test_default_decode_line(runs):
     assert d["steps"] == 20
     assert d["config"]["workload"] == "csa_decode_pro_1m" and d["roofline"]["bound"] == "hbm"
     assert d["roofline"]["algorithmic_bytes_per_launch"] == 71338000
+    c = d["config"]
+    _arith(d, c["queries_per_step_per_gpu"], c["indexer_topk_ms"])
+    assert c["step_achieved_gbs"] == pytest.approx(
+        c["step_algorithmic_bytes"] / (d["ms_per_step"] * 1e-3) / 1e9, rel=1e-9)
 
 
 @pytest.mark.parametrize("mode,workload", [("flash", "csa_decode_flash_128k"),
@@ -114,6 +134,7 @@ def test_other_decode_lines(runs, mode, workload):
     _contract(d)
     assert d["config"]["workload"] == workload and d["steps"] == 16
     assert d["roofline"]["bound"] == "hbm"
+    _arith(d, d["config"]["queries_per_step_per_gpu"], d["config"]["indexer_topk_ms"])
 
 
 def test_hca_line(runs):
@@ -121,12 +142,29 @@ def test_hca_line(runs):
     _contract(d)
     assert d["config"]["workload"] == "hca_decode_128k"
     assert d["steps"] == 20  # graphs of 4 steps: exactly the steps asked for
+    # the step is the attention call alone, so the kernel time is the step time
+    _arith(d, d["config"]["queries_per_step_per_gpu"], d["ms_per_step"])
 
 
 def test_prefill_line(runs):
     d = _line(runs, "prefill")
     _contract(d)
     assert d["roofline"]["bound"] == "tensor"
+    c, r = d["config"], d["roofline"]
+    _arith(d, c["new_tokens"], d["ms_per_step"])
+    # FLOPs of the shrunk workload by the layer's definition, restated here per query
+    P, T, m, H, H_I, k = c["prefix_tokens"], c["new_tokens"], 4, c["heads"], \
+        c["indexer_heads"], c["top_k"]
+    f4 = f16 = 0
+    for t in range(P, P + T):
+        n = (t + 1) // m
+        f4 += 2 * H_I * 128 * n
+        f16 += 4 * H * 512 * (min(k, n) + min(128, t + 1))
+    assert c["fp4_tflop"] == pytest.approx(f4 / 1e12, rel=1e-12)
+    assert c["bf16_tflop"] == pytest.approx(f16 / 1e12, rel=1e-12)
+    ratio = r["mma_peak"]["fp4_over_bf16"]
+    assert r["achieved"] == pytest.approx(
+        (f4 / ratio + f16) / (d["ms_per_step"] * 1e-3) / 1e12, rel=1e-9)
 
 
 def test_reference_line(runs):
@@ -134,3 +172,14 @@ def test_reference_line(runs):
     assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_full_prefill_flops_match_the_workload_figures():
+    # 65,536 new tokens after a 196,608-token prefix, m = 4, 128 heads, 64 indexer heads,
+    # top-1024: sum of n(t) = 3.758e9 eligible entries, so 61.57 TFLOP of FP4 indexer work;
+    # every query attends to 1,024 + 128 rows, so 128 x 1152 x 512 x 4 x 65,536 = 19.79 TFLOP
+    import bench
+
+    f4, f16 = bench.prefill_flops(196608, 65536, 4, 128, 64, 1024)
+    assert f4 == pytest.approx(61.57e12, rel=1e-3)
+    assert f16 == 128 * 1152 * 512 * 4 * 65536
