@@ -120,7 +120,14 @@ def test_default_decode_line(runs):
     _contract(d)
     assert d["steps"] == 20
     assert d["config"]["workload"] == "csa_decode_pro_1m" and d["roofline"]["bound"] == "hbm"
-    assert d["roofline"]["algorithmic_bytes_per_launch"] == 71338000
+    # per query: 262,144 keys of 64 B codes + 4 B scales, 64 indexer heads of 64 B codes +
+    # 4 B scales + a 4 B weight, 1,024 indices out, the length
+    assert d["roofline"]["algorithmic_bytes_per_launch"] == \
+        4 * (262144 * 68 + 64 * (64 + 4 + 4) + 1024 * 4 + 4) == 71338000
+    # and the attention: 1,024 rows of 576 B + a 4 B scale, 128 window rows of 1 KB, Q and O
+    # (128 heads x 1 KB each), the indices read back, position and length, 128 sink logits
+    assert d["config"]["step_algorithmic_bytes"] == 71338000 + \
+        4 * (1024 * 580 + 128 * 1024 + 2 * 128 * 1024 + 1024 * 4 + 8 + 128 * 4)
     c = d["config"]
     _arith(d, c["queries_per_step_per_gpu"], c["indexer_topk_ms"])
     assert c["step_achieved_gbs"] == pytest.approx(
