@@ -1,7 +1,8 @@
-"""bench.py's clock record (no GPU): the sampler reads nvidia-smi's CSV samples, reports
-the median SM clock under load, the largest maximum clock and every throttle reason seen
-active, skips lines it cannot read, and says so when nvidia-smi is missing. A fake
-nvidia-smi on PATH prints the samples; it changes no setting of any GPU."""
+"""bench.py's clock record and peaks (no GPU). The sampler reads nvidia-smi's CSV samples,
+reports the median SM clock under load, the largest maximum clock and every throttle reason
+seen active, skips lines it cannot read, and says so when nvidia-smi is missing; a fake
+nvidia-smi on PATH prints the samples and changes no setting of any GPU. The HBM peak comes
+from the measured peaks file when there is one, else from the stated fallback."""
 
 import os
 import time
@@ -54,3 +55,11 @@ def test_missing_nvidia_smi_is_stated(monkeypatch, tmp_path):
     s.start()
     got = s.stop()
     assert got["sm_mhz"] is None and got["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_peaks_come_from_the_measured_file_else_the_stated_fallback(monkeypatch, tmp_path):
+    # with no measured file the HBM denominator is the fallback 6.65 TB/s, labelled so
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.peaks() == {"hbm_gbs": 6650.0, "src": "fallback"}
+    (tmp_path / "MEASURED_PEAKS.json").write_text('{"hbm_gbs": 6541.8}')
+    assert bench.peaks() == {"hbm_gbs": 6541.8, "src": "measured"}
