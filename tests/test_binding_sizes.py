@@ -107,6 +107,36 @@ def test_indexer_topk():
     refused("idx", call, idx=t(B, k - 1, dtype=I32))
 
 
+def test_paged_indexer_and_attention_arguments():
+    # pools of 512-entry pages behind a [B][pages_max] table: a well-shaped call reaches the
+    # device-pointer check; a table of the wrong type or row count, a pool that is not a
+    # whole number of pages, and a pool one element short are refused on the host
+    B, H_I, H, P, pages_max, k = 4, 64, 128, 512, 8, 1024
+    pool = (B * pages_max + 3) * P
+    paging = csa.Paging(t(B, pages_max, dtype=I32), P)
+    assert paging.Nmax == pages_max * P
+    kw = dict(n_entries=t(B, dtype=I32), q_fp4=t(B, H_I, 64, dtype=U8),
+              q_sf=t(B, H_I, 4, dtype=U8), w=t(B, H_I), k_fp4=t(pool, 64, dtype=U8),
+              k_sf=t(pool // 128 * 512, dtype=U8), k=k, paging=paging)
+    call = lambda **o: csa.indexer_topk(**{**kw, **o})
+    passes_checks(call)
+    with pytest.raises(ValueError, match="block_table: int32"):
+        csa.Paging(t(B, pages_max, dtype=torch.int64), P)
+    with pytest.raises(ValueError, match="rows for 4 sequences"):
+        call(paging=csa.Paging(t(B - 1, pages_max, dtype=I32), P))
+    with pytest.raises(ValueError, match="whole number of pages"):
+        call(k_fp4=t(pool + 128, 64, dtype=U8), k_sf=t((pool + 128) // 128 * 512, dtype=U8))
+    refused("k_sf", call, k_sf=short(kw["k_sf"]))
+    akw = dict(q=t(B, H, 512, dtype=I16), pos=t(B, dtype=I32), n_entries=t(B, dtype=I32),
+               kv=t(pool, 576, dtype=U8), kv_scale=t(pool), swa=t(B, 128, 512, dtype=I16),
+               sink=t(H), idx=t(B, k, dtype=I32), paging=paging)
+    attn = lambda **o: csa.sparse_attn_decode(**{**akw, **o})
+    passes_checks(attn)
+    refused("kv_scale", attn, kv_scale=short(akw["kv_scale"]))
+    with pytest.raises(ValueError, match="whole number of pages"):
+        attn(kv=t(pool + 1, 576, dtype=U8), kv_scale=t(pool + 1))
+
+
 def test_attention():
     B, H, Nmax, k = 4, 128, 262144, 1024
     kw = dict(q=t(B, H, 512, dtype=I16), pos=t(B, dtype=I32), n_entries=t(B, dtype=I32),
