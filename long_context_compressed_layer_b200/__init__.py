@@ -314,6 +314,7 @@ def decode_append(pos, a, za, bias, state, *, b=None, zb=None, m: int = 4, overl
                itail_b=(state["itail_b"], 2 * B * m * INDEX_DIM),
                itail_zb=(state["itail_zb"], 2 * B * m * INDEX_DIM),
                k_fp4=(state["k_fp4"], pool * 64), k_sf=(state["k_sf"], pool // 128 * 512))
+    pg = _pages(paging, pool, B)
     g = lambda k_, el: _ptr(state.get(k_), elem=el, name=k_)
     args = AppendArgs(B, m, int(overlap), rope_base, eps, _ptr(pos, elem=4, name="pos"),
                       _ptr(a, elem=2, name="a"), _ptr(b, elem=2, name="b"),
@@ -330,7 +331,7 @@ def decode_append(pos, a, za, bias, state, *, b=None, zb=None, m: int = 4, overl
                       g("itail_zb", 4) if ia is not None else None,
                       g("k_fp4", 1) if ia is not None else None,
                       g("k_sf", 1) if ia is not None else None,
-                      _ptr(dev_status, elem=4, name="dev_status"), _pages(paging, pool, B))
+                      _ptr(dev_status, elem=4, name="dev_status"), pg)
     _check(lib().csa_decode_append(C.byref(args), _stream(stream)), "csa_decode_append")
 
 
@@ -558,6 +559,7 @@ def prefill(P: int, m: int, k: int, *, a, b, za, zb, bias, kv, kv_scale, q_fp4, 
            prev_b=(prev_b, m * HEAD_DIM), prev_zb=(prev_zb, m * HEAD_DIM),
            swa_prefix=(swa_prefix, WINDOW * HEAD_DIM), norm_w=(norm_w, HEAD_DIM),
            out=(out, T * H * HEAD_DIM))
+    pg = _pages(paging, pool, 1)
     dev = q.device
     if workspace is None:
         workspace = prefill_workspace(T, Nmax, H, k, dev)
@@ -580,7 +582,7 @@ def prefill(P: int, m: int, k: int, *, a, b, za, zb, bias, kv, kv_scale, q_fp4, 
                        _ptr(swa_prefix, elem=2, name="swa_prefix"),
                        _ptr(out, elem=2, name="out"), _ptr(l, elem=4, name="lse"),
                        _ptr(ix, elem=4, name="idx"),
-                       _ptr(dev_status, elem=4, name="dev_status"), _pages(paging, pool, 1))
+                       _ptr(dev_status, elem=4, name="dev_status"), pg)
     _check(lib().csa_prefill(C.byref(args), workspace.data_ptr(), workspace.numel(),
                              _stream(stream)), "csa_prefill")
     res = [out]

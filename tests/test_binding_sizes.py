@@ -170,3 +170,39 @@ def test_prefill():
         refused(name, call, **{name: short(kw[name])})
     refused("q", call, q=t(T - 1, H, 512, dtype=I16))
     refused("norm_w", call, norm_w=t(100))
+
+
+def test_paged_append_and_prefill_arguments():
+    # the append's state and the prefill's cache as page pools: well-shaped calls reach the
+    # device-pointer check; a table whose row count is not the batch's, or a pool that is
+    # not a whole number of pages, is refused on the host
+    B, m, P, pages_max = 2, 4, 256, 4
+    pool = (B * pages_max + 3) * P
+    st = csa.new_decode_state(B, 128, m, device="meta")
+    st.update(kv=t(pool, 576, dtype=U8), kv_scale=t(pool), k_fp4=t(pool, 64, dtype=U8),
+              k_sf=t(pool // 128 * 512, dtype=U8))
+    paging = csa.Paging(t(B, pages_max, dtype=I32), P)
+    kw = dict(pos=t(B, dtype=I32), a=t(B, 512, dtype=I16), za=t(B, 512), bias=t(2 * m),
+              state=st, b=t(B, 512, dtype=I16), zb=t(B, 512), m=m, ia=t(B, 128, dtype=I16),
+              ib=t(B, 128, dtype=I16), iza=t(B, 128), izb=t(B, 128), ibias=t(2 * m),
+              paging=paging)
+    call = lambda **o: csa.decode_append(**{**kw, **o})
+    passes_checks(call)
+    with pytest.raises(ValueError, match="rows for 2 sequences"):
+        call(paging=csa.Paging(t(B + 1, pages_max, dtype=I32), P))
+    refused("k_sf", call, state=dict(st, k_sf=short(st["k_sf"])))
+
+    Pp, T, H, H_I, k = 512, 301, 64, 16, 64
+    pk = dict(a=t(T, 512, dtype=I16), b=t(T, 512, dtype=I16), za=t(T, 512), zb=t(T, 512),
+              bias=t(2 * m), kv=t(pool, 576, dtype=U8), kv_scale=t(pool),
+              q_fp4=t(T, H_I, 64, dtype=U8), q_sf=t(T, H_I, 4, dtype=U8), w=t(T, H_I),
+              k_fp4=t(pool, 64, dtype=U8), k_sf=t(pool // 128 * 512, dtype=U8),
+              q=t(T, H, 512, dtype=I16), sink=t(H), prev_b=t(m, 512, dtype=I16),
+              prev_zb=t(m, 512), swa_prefix=t(128, 512, dtype=I16),
+              paging=csa.Paging(t(1, pages_max, dtype=I32), P))
+    pre = lambda **o: csa.prefill(Pp, m, k, **{**pk, **o})
+    passes_checks(pre)
+    with pytest.raises(ValueError, match="rows for 1 sequences"):
+        pre(paging=paging)  # a prefill is one sequence: its table has one row
+    with pytest.raises(ValueError, match="whole number of pages"):
+        pre(kv=t(pool + 7, 576, dtype=U8), kv_scale=t(pool + 7), k_fp4=t(pool + 7, 64, dtype=U8))
