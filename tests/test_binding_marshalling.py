@@ -1,8 +1,9 @@
-"""The binding hands each call's page table to the library as the C struct says (no GPU):
+"""The binding hands each call's arguments to the library as the C structs say (no GPU):
 with the library replaced by a recorder and device pointers by stand-in addresses, every
 paged call passes the table row length, the entries per page and the pool's page count
-(the pool's entries over the page size), and every contiguous call passes an empty
-struct. Host logic only: nothing here reaches a kernel."""
+(the pool's entries over the page size), every contiguous call passes an empty page
+struct, and the sizes, flags and scalars arrive as given. Host logic only: nothing here
+reaches a kernel."""
 
 import pytest
 import torch
@@ -19,12 +20,14 @@ def t(*shape, dtype=F32):
 
 
 class Recorder:
-    """Stands in for the library: records the csa_pages of each call and returns OK."""
+    """Stands in for the library: records each call's arguments and returns OK."""
 
     def __init__(self):
         self.pages = {}
+        self.args = {}
 
     def _rec(self, name, args):
+        self.args[name] = args._obj
         pg = args._obj.pages
         self.pages[name] = (bool(pg.block_table), pg.pages_max, pg.page_entries, pg.num_pages)
         return 0
@@ -97,3 +100,38 @@ def test_paged_calls_pass_the_table_and_the_pool_size(rec):
 def test_contiguous_calls_pass_an_empty_struct(rec):
     _calls(paged=False)
     assert set(rec.pages.values()) == {(False, 0, 0, 0)}
+
+
+def test_sizes_flags_and_scalars_arrive_as_given(rec):
+    ws = t(256, dtype=U8)
+    kf, ksf = t(B, 1024, 64, dtype=U8), t(B, 1024 // 128 * 512, dtype=U8)
+    common = (t(B, dtype=I32), t(B, 32, 64, dtype=U8), t(B, 32, 4, dtype=U8), t(B, 32), kf, ksf)
+    csa.indexer_topk(*common, 128, workspace=ws, idx=t(B, 128, dtype=I32))
+    a = rec.args["topk"]
+    assert (a.B, a.H_I, a.k, a.Nmax, a.flags, a.select_wait_ns) == (B, 32, 128, 1024, 0, 0)
+    csa.indexer_topk(*common, 128, workspace=ws, idx=t(B, 128, dtype=I32),
+                     separate_select=True, select_wait_ns=5000)
+    a = rec.args["topk"]
+    assert (a.flags & csa.TOPK_SEPARATE_SELECT, a.select_wait_ns) == (1, 5000)
+
+    csa.sparse_attn_decode(t(B, 128, 512, dtype=I16), t(B, dtype=I32), t(B, dtype=I32),
+                           t(B, 2048, 576, dtype=U8), t(B, 2048), t(B, 128, 512, dtype=I16),
+                           t(128), t(B, 512, dtype=I32), workspace=ws,
+                           out=t(B, 128, 512, dtype=I16), tau=0.125, rope_base=5e5,
+                           derotate=False)
+    a = rec.args["attn"]
+    assert (a.B, a.H, a.k, a.Nmax, a.derotate) == (B, 128, 512, 2048, 0)
+    assert (a.tau, a.rope_base) == (0.125, 5e5)
+
+    T = 301
+    csa.prefill(1024, M, 256, a=t(T, 512, dtype=I16), b=t(T, 512, dtype=I16), za=t(T, 512),
+                zb=t(T, 512), bias=t(2 * M), kv=t(1024, 576, dtype=U8), kv_scale=t(1024),
+                q_fp4=t(T, 16, 64, dtype=U8), q_sf=t(T, 16, 4, dtype=U8), w=t(T, 16),
+                k_fp4=t(1024, 64, dtype=U8), k_sf=t(1024 // 128 * 512, dtype=U8),
+                q=t(T, 64, 512, dtype=I16), sink=t(64), prev_b=t(M, 512, dtype=I16),
+                prev_zb=t(M, 512), swa_prefix=t(128, 512, dtype=I16), workspace=ws,
+                out=t(T, 64, 512, dtype=I16), strict_eligibility=True, eps=1e-5)
+    a = rec.args["prefill"]
+    assert (a.P, a.T, a.m, a.H, a.H_I, a.k, a.Nmax) == (1024, T, M, 64, 16, 256, 1024)
+    assert (a.strict_eligibility, a.derotate) == (1, 1)
+    assert a.eps == pytest.approx(1e-5, rel=1e-7)
